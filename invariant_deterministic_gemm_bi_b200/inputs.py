@@ -1,0 +1,176 @@
+"""Seeded synthetic inputs for the batch-invariant GEMM workloads.
+
+This module only draws random numbers and rounds them to the storage formats (bf16, e4m3,
+fp32 scales); it holds none of the GEMM's arithmetic.  Both the CUDA path (tests, benchmark)
+and the CPU oracle receive the arrays it returns, so the two sides always see the same bits.
+
+Recipes (all seeded; a generator is ``torch.Generator(device)`` seeded with the given seed):
+
+* bf16 Gaussian:   x ~ N(0, std^2) drawn in fp32, rounded to bf16 (RNE).
+* bf16 integer:    x uniform in {-4, ..., 4}, exact in bf16.
+* e4m3 Gaussian:   x ~ N(0, 1) in fp32, clamped to [-448, 448], rounded to e4m3 (RNE).
+* e4m3 integer:    x uniform in {-4, ..., 4}, exact in e4m3.
+* fp32 scales:     s = 2^u, u ~ U(-4, 4) (log-uniform in [2^-4, 2^4]); or s = 2^j with integer
+                   j uniform in [-4, 4] for the exactly representable variant.
+* MoE routing:     logits [T, E] ~ N(0, 1); each token takes the 8 largest logits (softmax is
+                   monotone, so this is top-8 by softmax); ties go to the lower expert index.
+                   The (token, slot) pairs are stably sorted by expert, so inside an expert's
+                   segment rows are in token order.
+
+Bits are returned as torch tensors (``torch.int16`` views for bf16, ``torch.uint8`` for e4m3)
+on the requested device; ``to_numpy_bits`` gives the host copies the oracle takes.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+
+def generator(seed: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def bf16_gaussian(shape, seed: int, std: float = 1.0, device="cpu") -> torch.Tensor:
+    """bf16 tensor with entries N(0, std^2), drawn in fp32 and rounded to nearest even."""
+    g = generator(seed, device)
+    x = torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(torch.bfloat16)
+
+
+def bf16_integers(shape, seed: int, lo: int = -4, hi: int = 4, device="cpu") -> torch.Tensor:
+    """bf16 tensor with integer entries uniform in [lo, hi] (exact in bf16)."""
+    g = generator(seed, device)
+    x = torch.randint(lo, hi + 1, tuple(shape), generator=g, device=device, dtype=torch.int32)
+    return x.to(torch.bfloat16)
+
+
+def e4m3_gaussian(shape, seed: int, device="cpu") -> torch.Tensor:
+    """e4m3 (fn) tensor: N(0,1) in fp32, clamped to +-448, rounded to nearest even."""
+    g = generator(seed, device)
+    x = torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+    x.clamp_(-448.0, 448.0)
+    return x.to(torch.float8_e4m3fn)
+
+
+def e4m3_integers(shape, seed: int, lo: int = -4, hi: int = 4, device="cpu") -> torch.Tensor:
+    g = generator(seed, device)
+    x = torch.randint(lo, hi + 1, tuple(shape), generator=g, device=device, dtype=torch.int32)
+    return x.to(torch.float32).to(torch.float8_e4m3fn)
+
+
+def scales_log_uniform(shape, seed: int, lo_exp: float = -4.0, hi_exp: float = 4.0,
+                       device="cpu") -> torch.Tensor:
+    """fp32 scales 2^u with u ~ U(lo_exp, hi_exp)."""
+    g = generator(seed, device)
+    u = torch.rand(*shape, generator=g, device=device, dtype=torch.float32)
+    u.mul_(hi_exp - lo_exp).add_(lo_exp)
+    return torch.exp2(u)
+
+
+def scales_pow2(shape, seed: int, lo: int = -4, hi: int = 4, device="cpu") -> torch.Tensor:
+    """fp32 scales 2^j with integer j uniform in [lo, hi] (exact products)."""
+    g = generator(seed, device)
+    j = torch.randint(lo, hi + 1, tuple(shape), generator=g, device=device, dtype=torch.int32)
+    return torch.exp2(j.to(torch.float32))
+
+
+def bits_of(t: torch.Tensor) -> torch.Tensor:
+    """Reinterpret a bf16 / e4m3 tensor as its raw integer bit pattern (no copy)."""
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8)
+    raise TypeError(f"no bit view for {t.dtype}")
+
+
+def to_numpy_bits(t: torch.Tensor) -> np.ndarray:
+    """Host numpy copy of the raw bits: uint16 for bf16, uint8 for e4m3, float32 as is."""
+    if t.dtype == torch.bfloat16:
+        return t.detach().view(torch.int16).cpu().numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.detach().view(torch.uint8).cpu().numpy()
+    if t.dtype == torch.float32:
+        return t.detach().cpu().numpy()
+    if t.dtype == torch.int32:
+        return t.detach().cpu().numpy()
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ---------------------------------------------------------------------------------------------
+# MoE routing (harness preparation for the grouped GEMM)
+# ---------------------------------------------------------------------------------------------
+
+@dataclass
+class Routing:
+    """Result of routing T tokens to experts, grouped by expert."""
+    num_experts: int
+    token_of_row: torch.Tensor     # int64 [R]: which token each grouped row comes from
+    expert_of_row: torch.Tensor    # int64 [R]
+    offsets: torch.Tensor          # int32 [E+1], offsets[0] = 0, offsets[E] = R
+
+    @property
+    def rows(self) -> int:
+        return int(self.token_of_row.numel())
+
+
+def route_topk(logits: torch.Tensor, top_k: int = 8) -> torch.Tensor:
+    """Top-k experts per token by logit, ties to the lower expert index.  Returns int64 [T,k]."""
+    order = torch.sort(-logits, dim=1, stable=True).indices
+    return order[:, :top_k].contiguous()
+
+
+def group_by_expert(experts: torch.Tensor, num_experts: int) -> Routing:
+    """Stable-sort the (token, slot) pairs of ``experts`` [T, k] by expert id."""
+    T, k = experts.shape
+    flat = experts.reshape(-1).to(torch.int64)
+    tokens = torch.arange(T, device=experts.device, dtype=torch.int64).repeat_interleave(k)
+    order = torch.sort(flat, stable=True).indices
+    expert_of_row = flat[order]
+    token_of_row = tokens[order]
+    counts = torch.bincount(expert_of_row, minlength=num_experts)
+    offsets = torch.zeros(num_experts + 1, dtype=torch.int64, device=experts.device)
+    offsets[1:] = torch.cumsum(counts, 0)
+    return Routing(num_experts, token_of_row, expert_of_row, offsets.to(torch.int32))
+
+
+def softmax_top8_routing(T: int, num_experts: int, seed: int, device="cpu") -> Routing:
+    """Router logits ~ N(0,1) [T, E]; top-8 per token; grouped by expert."""
+    g = generator(seed, device)
+    logits = torch.randn(T, num_experts, generator=g, device=device, dtype=torch.float32)
+    return group_by_expert(route_topk(logits, 8), num_experts)
+
+
+def routing_from_assignment(experts_per_row: np.ndarray, num_experts: int,
+                            token_of_row: np.ndarray | None = None) -> Routing:
+    """Build a routing from an explicit expert id per row (rows already grouped by expert)."""
+    e = np.asarray(experts_per_row, dtype=np.int64)
+    assert np.all(np.diff(e) >= 0), "rows must already be grouped by expert"
+    counts = np.bincount(e, minlength=num_experts)
+    offsets = np.zeros(num_experts + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    tok = np.arange(e.size) if token_of_row is None else np.asarray(token_of_row)
+    return Routing(num_experts, torch.from_numpy(tok.astype(np.int64)),
+                   torch.from_numpy(e), torch.from_numpy(offsets.astype(np.int32)))
+
+
+# ---------------------------------------------------------------------------------------------
+# seeds (one base seed per workload; derived seeds for batches, permutations and trials)
+# ---------------------------------------------------------------------------------------------
+
+WORKLOAD_BASE_SEED = {
+    "small": 1000,
+    "decode": 2000,
+    "prefill": 3000,
+    "fp8": 4000,
+    "moe": 5000,
+}
+
+
+def derived_seed(base: int, M: int, trial: int = 0, salt: int = 0) -> int:
+    return int(base + 17 * M + trial + 1_000_003 * salt)

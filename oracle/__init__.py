@@ -1,0 +1,15 @@
+"""CPU oracle for the batch-invariant GEMM -- test infrastructure only (see ``oracle.py``)."""
+from .oracle import (  # noqa: F401
+    bf16_to_f64,
+    OracleLib,
+    build,
+    compile_copy,
+    default_threads,
+    e4m3_to_f64,
+    f64_to_bf16,
+    gemm_bf16,
+    gemm_bf16_rows,
+    gemm_fp8_blockscaled,
+    gemm_fp8_rows,
+    grouped_gemm_bf16,
+)
