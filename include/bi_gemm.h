@@ -1,0 +1,199 @@
+/*
+ * bi_gemm.h -- C ABI of libbigemm, a batch-invariant GEMM for NVIDIA B200 (sm_100a).
+ *
+ *   C[M,N] = A[M,K] . B[N,K]^T          (alpha = 1, beta = 0, fp32 accumulation, bf16 output)
+ *
+ * Batch invariance: for a fixed plan, the bits of output row C[m,:] are a function of A[m,:],
+ * B (and, for FP8, the row's scales scale_a[:,m] and scale_b) only.  They do not depend on M,
+ * on m, on the other rows of A, on the expert offsets of a grouped call, on the stream, on the
+ * grid or on device occupancy.  This is the property defined in "DeepSeek不惜代价保住它！V4关键
+ * 特性被挖出来了" (QbitAI), section "什么是batch invariance": one token's output is bit-identical
+ * whatever its position in the batch, the batch size and its batch-mates.  The same article
+ * (section "牺牲了什么") attributes it to dropping split-K in a custom GEMM: a split K axis is
+ * summed in an order that changes with the split, and floating-point addition does not
+ * associate.  The library therefore never splits K: one CTA owns the whole K range of its output
+ * tile and walks it in ascending 128-byte blocks, and the tile shape, MMA instruction shape and
+ * K order are fixed by the plan, a pure function of (N, K, dtype, num_experts) that never sees M.
+ * There are no atomics on the data path.
+ *
+ * Memory and ownership.  The caller owns every buffer and the stream.  Device pointers must
+ * point to memory of the current CUDA device.  A plan is host state plus, created lazily at the
+ * first run on a device, one 4-byte device status word per device; nothing else allocates on
+ * the run path.  All run calls are asynchronous on `stream` (NULL = the legacy default stream)
+ * and do not synchronise.
+ *
+ * Errors.  Every entry point returns a bi_status_t; nothing throws across the ABI, calls exit or
+ * abort, or traps on the device.  Invalid arguments are rejected before any launch.  Launch
+ * failures map to BI_ERR_CUDA.  Device-side failures (a pipeline wait that exceeded its time
+ * limit, malformed grouped offsets) are written to the plan's status word and reported by
+ * bi_gemm_sync_status.
+ *
+ * Layouts (all row-major, strides in elements):
+ *   A        [M][lda]   K-contiguous, bf16 or e4m3; lda >= K
+ *   B        [N][ldb]   K-contiguous ("B^T" form, the weight layout); ldb >= K
+ *   C        [M][ldc]   bf16, N-contiguous; ldc >= N
+ *   scale_a  (FP8 only) fp32, K-block-major: the scale of row m and K block kb (columns
+ *            128*kb .. 128*kb+127) is scale_a[kb*ld_sa + m]; ld_sa >= M
+ *   scale_b  (FP8 only) fp32 [ceil(N/128)][ceil(K/128)] row-major: one scale per 128x128 block
+ * Alignment: A, B, C must be 16-byte aligned, and lda*elt, ldb*elt, ldc*2 must be multiples of
+ * 16 bytes (elt = 2 for bf16, 1 for e4m3).  scale_a and scale_b need 4-byte alignment.
+ */
+#ifndef BI_GEMM_H
+#define BI_GEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BI_GEMM_ABI_VERSION 1
+
+typedef enum {
+    BI_DTYPE_BF16 = 0,              /* A, B bf16; C bf16 */
+    BI_DTYPE_E4M3_BLOCKSCALED = 1   /* A, B e4m3 (fn) with fp32 block scales; C bf16 */
+} bi_dtype_t;
+
+typedef enum {
+    BI_OK = 0,
+    BI_ERR_INVALID_ARG = 1,         /* null pointer, negative size, stride below the extent */
+    BI_ERR_ALIGNMENT = 2,           /* pointer or stride not 16-byte aligned */
+    BI_ERR_UNSUPPORTED_SHAPE = 3,   /* a size outside what the plan supports */
+    BI_ERR_DTYPE_MISMATCH = 4,      /* scales given to a bf16 plan, missing for FP8, ... */
+    BI_ERR_CUDA = 5,                /* a CUDA runtime/driver call failed */
+    BI_ERR_DEVICE_TIMEOUT = 6,      /* a device pipeline wait exceeded its limit */
+    BI_ERR_BAD_OFFSETS = 7,         /* grouped offsets not 0 .. total_rows non-decreasing */
+    BI_ERR_NO_DEVICE = 8            /* no CUDA device, or the device is not sm_100 */
+} bi_status_t;
+
+/* Opaque, library-owned plan. */
+typedef struct bi_plan_s *bi_plan_t;
+
+/* What a plan fixed.  None of it depends on M. */
+typedef struct {
+    int64_t n, k;              /* the plan's N and K */
+    int dtype;                 /* bi_dtype_t */
+    int num_experts;           /* 1 = dense */
+    int block_m;               /* output rows per tile */
+    int block_n;               /* output columns per tile */
+    int block_k;               /* K elements per pipeline stage (128 bytes) */
+    int cta_group;             /* CTAs that share one MMA (1 or 2) */
+    int mma_m, mma_n, mma_k;   /* tcgen05.mma instruction shape */
+    int stages;                /* shared-memory pipeline depth */
+    int k_order_id;            /* 0 = ascending K blocks, whole K per CTA, no split-K */
+    int threads_per_cta;
+    int smem_bytes;            /* dynamic shared memory per CTA */
+    int tmem_columns;          /* tensor-memory columns allocated per CTA */
+} bi_plan_info_t;
+
+/* Library version check: returns BI_GEMM_ABI_VERSION. */
+int bi_gemm_abi_version(void);
+
+/* Human-readable name of a status code (static string; never NULL). */
+const char *bi_status_string(bi_status_t status);
+
+/*
+ * Create a plan for C = A . B^T with the given N, K and dtype.  num_experts = 1 makes a dense
+ * plan; num_experts > 1 makes a grouped (MoE) plan for bi_grouped_gemm_run (bf16 only).
+ * The plan is a pure function of its arguments: the same (N, K, dtype, num_experts) gives the
+ * same tile configuration in every process and on every device.  It touches no device and can
+ * be created on a machine without a GPU.
+ * Errors: BI_ERR_INVALID_ARG (out == NULL, N < 0, K < 0, num_experts < 1),
+ * BI_ERR_UNSUPPORTED_SHAPE (num_experts > 1024, or grouped with FP8).
+ */
+bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
+                         int num_experts);
+
+/* Destroy a plan and free its device status words.  NULL is accepted. */
+bi_status_t bi_gemm_plan_destroy(bi_plan_t plan);
+
+/* Copy the plan's fixed configuration into *info. */
+bi_status_t bi_gemm_plan_describe(bi_plan_t plan, bi_plan_info_t *info);
+
+/*
+ * Dense GEMM on device memory: C[0:M, 0:N] = A[0:M, 0:K] . B[0:N, 0:K]^T, rounded to bf16 (RNE).
+ * For BI_DTYPE_E4M3_BLOCKSCALED the operands are dequantised inside the kernel: the product of
+ * K block kb is scaled by scale_a[kb*ld_sa + m] * scale_b[(n/128)*ceil(K/128) + kb] and added to
+ * the fp32 accumulator in ascending kb (the fused dequantisation of "DeepSeek V4的batch
+ * invariance：大模型确定性推理的工程基石" (lshu.cn), section 3.2).  For bf16, pass
+ * scale_a = scale_b = NULL and ld_sa = 0.
+ * M = 0 (or N = 0) is a no-op returning BI_OK.  K = 0 writes zeros.
+ * Errors: BI_ERR_INVALID_ARG, BI_ERR_ALIGNMENT, BI_ERR_DTYPE_MISMATCH, BI_ERR_NO_DEVICE,
+ * BI_ERR_CUDA; a grouped plan returns BI_ERR_INVALID_ARG.
+ */
+bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M,
+                        const void *A, int64_t lda,
+                        const void *B, int64_t ldb,
+                        void *C, int64_t ldc,
+                        const float *scale_a, int64_t ld_sa,
+                        const float *scale_b,
+                        cudaStream_t stream);
+
+/*
+ * Grouped (MoE) GEMM, bf16: rows of A are grouped by expert; expert e owns the rows
+ * [offsets[e], offsets[e+1]) and multiplies them with its weight matrix
+ * B_e[n][k] = B[(e*N + n)*ldb + k]:   C[r, :] = A[r, :] . B_e^T.
+ * expert_offsets is a DEVICE array of E+1 int32 with offsets[0] = 0, non-decreasing,
+ * offsets[E] = total_rows; it is read only by the kernel (no host synchronisation).  Malformed
+ * offsets make the kernel compute nothing and set BI_ERR_BAD_OFFSETS in the status word.
+ * A grouped plan takes the tile configuration of the dense plan with the same N and K, so every
+ * row gets the bits a dense call with its expert's B_e would give it.
+ * Errors: as bi_gemm_run; a dense plan returns BI_ERR_INVALID_ARG.
+ */
+bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows,
+                                const void *A, int64_t lda,
+                                const void *B, int64_t ldb,
+                                void *C, int64_t ldc,
+                                const int32_t *expert_offsets,
+                                cudaStream_t stream);
+
+/*
+ * Dense GEMM from host memory: copies A (and scale_a) from the host buffers into the caller's
+ * device staging buffers, runs bi_gemm_run on them, and copies C back into C_host, all enqueued
+ * on `stream` (cudaMemcpyAsync; pinned host memory makes the copies asynchronous).  B and
+ * scale_b are device pointers (resident weights).  A_dev / C_dev / scale_a_dev must be large
+ * enough for M*lda, M*ldc and ceil(K/128)*ld_sa elements.  The call returns once everything is
+ * enqueued; synchronise `stream` before reading C_host.
+ * Errors: as bi_gemm_run, plus BI_ERR_INVALID_ARG for missing staging buffers.
+ */
+bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M,
+                             const void *A_host, int64_t lda,
+                             const void *B, int64_t ldb,
+                             void *C_host, int64_t ldc,
+                             const float *scale_a_host, int64_t ld_sa,
+                             const float *scale_b,
+                             void *A_dev, void *C_dev, float *scale_a_dev,
+                             cudaStream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear the plan's device status word for the current
+ * device.  Returns BI_OK, BI_ERR_DEVICE_TIMEOUT, BI_ERR_BAD_OFFSETS or BI_ERR_CUDA.  All runs
+ * of one plan on one device share the status word.
+ */
+bi_status_t bi_gemm_sync_status(bi_plan_t plan, cudaStream_t stream);
+
+/*
+ * Set the time limit, in nanoseconds, of every device-side pipeline wait of this plan's
+ * kernels (default 2e9, i.e. 2 s; 0 restores the default).  A wait that runs out sets
+ * BI_ERR_DEVICE_TIMEOUT, lets the CTA drain its own copies in flight, frees its tensor memory
+ * and returns, so the context stays usable.
+ */
+bi_status_t bi_gemm_set_wait_timeout(bi_plan_t plan, uint64_t timeout_ns);
+
+/*
+ * Test-only fault injection on the host side of the launch.  BI_DEBUG_SKIP_FIRST_LOAD makes
+ * the producer of every CTA skip its very first operand load, so that the first MMA wait of
+ * the CTA can never complete and must end by its time limit.  0 clears all flags.  Never set in
+ * production.
+ */
+#define BI_DEBUG_SKIP_FIRST_LOAD 1u
+bi_status_t bi_gemm_debug_set_flags(bi_plan_t plan, uint32_t flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BI_GEMM_H */

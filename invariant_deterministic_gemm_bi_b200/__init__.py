@@ -1,0 +1,28 @@
+"""Batch-invariant GEMM for NVIDIA B200 (sm_100a).
+
+C[M,N] = A[M,K] . B[N,K]^T with fp32 accumulation and bf16 output, computed by hand-written
+tcgen05/TMA kernels behind the C ABI in ``include/bi_gemm.h``.  Every output row is
+bit-identical whatever the batch size, the row's position and the other rows in the batch.
+
+``binding`` holds the ctypes wrapper (same names as the C ABI); ``inputs`` the seeded synthetic
+input generators; ``build`` the nvcc build of ``libbigemm.so``.
+"""
+from .binding import (  # noqa: F401
+    BI_DEBUG_SKIP_FIRST_LOAD,
+    BI_DTYPE_BF16,
+    BI_DTYPE_E4M3_BLOCKSCALED,
+    BiGemmError,
+    Plan,
+    bi_gemm_abi_version,
+    bi_gemm_debug_set_flags,
+    bi_gemm_plan,
+    bi_gemm_plan_describe,
+    bi_gemm_plan_destroy,
+    bi_gemm_run,
+    bi_gemm_run_host,
+    bi_gemm_set_wait_timeout,
+    bi_gemm_sync_status,
+    bi_grouped_gemm_run,
+    bi_status_string,
+    load_library,
+)

@@ -1,0 +1,218 @@
+"""Thin ctypes binding of libbigemm (include/bi_gemm.h), same names as the C ABI.
+
+Argument marshalling only: every function takes torch tensors (device memory owned by torch)
+or raw integers, passes their pointers, strides and the current CUDA stream to the C entry
+point of the same name, and raises ``BiGemmError`` on a non-OK status.  All arithmetic happens
+in the CUDA kernels behind the ABI; there is no fallback of any kind.  If the shared library is
+missing, loading fails loudly with instructions to build it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libbigemm.so")
+
+BI_DTYPE_BF16 = 0
+BI_DTYPE_E4M3_BLOCKSCALED = 1
+BI_DEBUG_SKIP_FIRST_LOAD = 1
+
+STATUS_NAMES = {
+    0: "BI_OK", 1: "BI_ERR_INVALID_ARG", 2: "BI_ERR_ALIGNMENT", 3: "BI_ERR_UNSUPPORTED_SHAPE",
+    4: "BI_ERR_DTYPE_MISMATCH", 5: "BI_ERR_CUDA", 6: "BI_ERR_DEVICE_TIMEOUT",
+    7: "BI_ERR_BAD_OFFSETS", 8: "BI_ERR_NO_DEVICE",
+}
+STATUS = {v: k for k, v in STATUS_NAMES.items()}
+
+# every symbol include/bi_gemm.h declares
+EXPORTED = [
+    "bi_gemm_abi_version", "bi_status_string", "bi_gemm_plan", "bi_gemm_plan_destroy",
+    "bi_gemm_plan_describe", "bi_gemm_run", "bi_grouped_gemm_run", "bi_gemm_run_host",
+    "bi_gemm_sync_status", "bi_gemm_set_wait_timeout", "bi_gemm_debug_set_flags",
+]
+
+
+class BiGemmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        self.name = STATUS_NAMES.get(status, f"status {status}")
+        super().__init__(f"{where}: {self.name}")
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [
+        ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("dtype", ctypes.c_int),
+        ("num_experts", ctypes.c_int), ("block_m", ctypes.c_int), ("block_n", ctypes.c_int),
+        ("block_k", ctypes.c_int), ("cta_group", ctypes.c_int), ("mma_m", ctypes.c_int),
+        ("mma_n", ctypes.c_int), ("mma_k", ctypes.c_int), ("stages", ctypes.c_int),
+        ("k_order_id", ctypes.c_int), ("threads_per_cta", ctypes.c_int),
+        ("smem_bytes", ctypes.c_int), ("tmem_columns", ctypes.c_int),
+    ]
+
+    def as_dict(self):
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+_LIB = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libbigemm.so and declare its signatures.  Raises ImportError if it is missing."""
+    global _LIB
+    if _LIB is not None and path == LIB_PATH:
+        return _LIB
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is not built: run `python -m invariant_deterministic_gemm_bi_b200.build`"
+                          " (the CUDA library is required; there is no fallback)")
+    lib = ctypes.CDLL(path)
+    i64, i32, u32, u64, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_void_p
+    lib.bi_gemm_abi_version.restype = i32
+    lib.bi_gemm_abi_version.argtypes = []
+    lib.bi_status_string.restype = ctypes.c_char_p
+    lib.bi_status_string.argtypes = [i32]
+    lib.bi_gemm_plan.restype = i32
+    lib.bi_gemm_plan.argtypes = [ctypes.POINTER(vp), i64, i64, i32, i32]
+    lib.bi_gemm_plan_destroy.restype = i32
+    lib.bi_gemm_plan_destroy.argtypes = [vp]
+    lib.bi_gemm_plan_describe.restype = i32
+    lib.bi_gemm_plan_describe.argtypes = [vp, ctypes.POINTER(PlanInfo)]
+    lib.bi_gemm_run.restype = i32
+    lib.bi_gemm_run.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, i64, vp, vp]
+    lib.bi_grouped_gemm_run.restype = i32
+    lib.bi_grouped_gemm_run.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, vp]
+    lib.bi_gemm_run_host.restype = i32
+    lib.bi_gemm_run_host.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, i64, vp, vp, vp, vp, vp]
+    lib.bi_gemm_sync_status.restype = i32
+    lib.bi_gemm_sync_status.argtypes = [vp, vp]
+    lib.bi_gemm_set_wait_timeout.restype = i32
+    lib.bi_gemm_set_wait_timeout.argtypes = [vp, u64]
+    lib.bi_gemm_debug_set_flags.restype = i32
+    lib.bi_gemm_debug_set_flags.argtypes = [vp, u32]
+    if path == LIB_PATH:
+        _LIB = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise BiGemmError(status, where)
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+@dataclass
+class Plan:
+    """A plan handle; destroy() (or garbage collection) releases it."""
+    handle: int
+    n: int
+    k: int
+    dtype: int
+    num_experts: int
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+    def destroy(self):
+        if self.handle:
+            bi_gemm_plan_destroy(self)
+            self.handle = 0
+
+
+def bi_gemm_abi_version() -> int:
+    return load_library().bi_gemm_abi_version()
+
+
+def bi_status_string(status: int) -> str:
+    return load_library().bi_status_string(status).decode()
+
+
+def bi_gemm_plan(N: int, K: int, dtype: int = BI_DTYPE_BF16, num_experts: int = 1) -> Plan:
+    h = ctypes.c_void_p()
+    _check(load_library().bi_gemm_plan(ctypes.byref(h), N, K, dtype, num_experts), "bi_gemm_plan")
+    return Plan(h.value, N, K, dtype, num_experts)
+
+
+def bi_gemm_plan_destroy(plan: Plan):
+    if plan.handle:
+        _check(load_library().bi_gemm_plan_destroy(plan.handle), "bi_gemm_plan_destroy")
+        plan.handle = 0
+
+
+def bi_gemm_plan_describe(plan: Plan) -> dict:
+    info = PlanInfo()
+    _check(load_library().bi_gemm_plan_describe(plan.handle, ctypes.byref(info)),
+           "bi_gemm_plan_describe")
+    return info.as_dict()
+
+
+def bi_gemm_run(plan: Plan, A, B, C, scale_a=None, scale_b=None, stream=None, M: int | None = None):
+    """C[:M] = A[:M] . B^T.  A [M, lda], B [N, ldb], C [M, ldc] (row-major, unit inner stride).
+
+    FP8: scale_a is fp32 [ceil(K/128), ld_sa] (K-block-major, ld_sa >= M), scale_b fp32
+    [ceil(N/128), ceil(K/128)].
+    """
+    M = A.shape[0] if M is None else M
+    ld_sa = scale_a.stride(0) if scale_a is not None else 0
+    st = load_library().bi_gemm_run(plan.handle, M, _ptr(A), A.stride(0), _ptr(B), B.stride(0),
+                                    _ptr(C), C.stride(0), _ptr(scale_a), ld_sa, _ptr(scale_b),
+                                    _stream_handle(stream))
+    _check(st, "bi_gemm_run")
+    return C
+
+
+def bi_grouped_gemm_run(plan: Plan, A, B, C, expert_offsets, stream=None):
+    """Grouped: rows of A grouped by expert (device int32 offsets [E+1]); B [E, N, ldb]."""
+    ldb = B.stride(-2)
+    st = load_library().bi_grouped_gemm_run(plan.handle, A.shape[0], _ptr(A), A.stride(0),
+                                            _ptr(B), ldb, _ptr(C), C.stride(0),
+                                            _ptr(expert_offsets), _stream_handle(stream))
+    _check(st, "bi_grouped_gemm_run")
+    return C
+
+
+def bi_gemm_run_host(plan: Plan, A_host, B, C_host, A_dev, C_dev, scale_a_host=None, scale_b=None,
+                     scale_a_dev=None, stream=None):
+    """Host-memory variant: copies A (and scale_a) in, runs, copies C out, all on `stream`."""
+    M = A_host.shape[0]
+    ld_sa = scale_a_host.stride(0) if scale_a_host is not None else 0
+    st = load_library().bi_gemm_run_host(plan.handle, M, _ptr(A_host), A_host.stride(0), _ptr(B),
+                                         B.stride(0), _ptr(C_host), C_host.stride(0),
+                                         _ptr(scale_a_host), ld_sa, _ptr(scale_b), _ptr(A_dev),
+                                         _ptr(C_dev), _ptr(scale_a_dev), _stream_handle(stream))
+    _check(st, "bi_gemm_run_host")
+    return C_host
+
+
+def bi_gemm_sync_status(plan: Plan, stream=None, raise_on_error: bool = True) -> int:
+    st = load_library().bi_gemm_sync_status(plan.handle, _stream_handle(stream))
+    if raise_on_error:
+        _check(st, "bi_gemm_sync_status")
+    return st
+
+
+def bi_gemm_set_wait_timeout(plan: Plan, timeout_ns: int):
+    _check(load_library().bi_gemm_set_wait_timeout(plan.handle, timeout_ns), "bi_gemm_set_wait_timeout")
+
+
+def bi_gemm_debug_set_flags(plan: Plan, flags: int):
+    _check(load_library().bi_gemm_debug_set_flags(plan.handle, flags), "bi_gemm_debug_set_flags")

@@ -1,0 +1,576 @@
+// bi_gemm.cu -- host side of libbigemm: plans, argument checks, TMA tensor maps, launches and
+// the extern "C" ABI declared in include/bi_gemm.h.
+//
+// The plan is a pure function of (N, K, dtype, num_experts): it picks one tile configuration
+// (tile shape, MMA instruction shape, pipeline depth) and never looks at M, at the device's
+// occupancy or at anything measured at run time.  This is the "fixed kernel path instead of
+// run-time heuristics" of "DeepSeek V4的batch invariance：大模型确定性推理的工程基石" (lshu.cn),
+// sections 3.1-3.2, with the split-K of the heuristic libraries removed altogether.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "../../include/bi_gemm.h"
+#include "bi_kernels.cuh"
+
+namespace {
+
+using bi::GemmParams;
+
+// ---------------------------------------------------------------------------------------------
+// Kernel registry: every instantiated configuration
+// ---------------------------------------------------------------------------------------------
+
+typedef void (*KernelFn)(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
+                         const GemmParams);
+
+struct KernelEntry {
+    int bn;
+    int stages;
+    bool fp8;
+    bool grouped;
+    KernelFn fn;
+    int smem;
+};
+
+#define BI_ENTRY(BN, ST, F8, GR)                                                                   \
+    KernelEntry{BN, ST, F8, GR, &bi::bi_gemm_kernel<BN, ST, F8, GR>,                               \
+                bi::smem_bytes_for<BN, ST, F8, GR>()}
+
+// Pipeline depth: as many stages as fit in ~200 KB of shared memory.
+const KernelEntry kKernels[] = {
+    BI_ENTRY(32, 10, false, false),  BI_ENTRY(64, 8, false, false),
+    BI_ENTRY(128, 6, false, false),  BI_ENTRY(256, 4, false, false),
+    BI_ENTRY(32, 10, true, false),   BI_ENTRY(64, 8, true, false),
+    BI_ENTRY(128, 6, true, false),   BI_ENTRY(32, 10, false, true),
+    BI_ENTRY(64, 8, false, true),    BI_ENTRY(128, 6, false, true),
+    BI_ENTRY(256, 4, false, true),
+};
+constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
+
+const KernelEntry *find_kernel(int bn, bool fp8, bool grouped)
+{
+    for (int i = 0; i < kNumKernels; ++i)
+        if (kKernels[i].bn == bn && kKernels[i].fp8 == fp8 && kKernels[i].grouped == grouped)
+            return &kKernels[i];
+    return nullptr;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Plan table
+// ---------------------------------------------------------------------------------------------
+
+// The output-tile width BN for (N, K, dtype).  Known projection shapes get the width tuned for
+// them; any other shape takes the widest BN that still gives >= 100 tiles at M <= 128, since
+// without split-K the N tiles are the only parallelism a small batch has.  A grouped plan uses
+// the dense plan's width for the same (N, K), so a row of an expert's segment gets the bits a
+// dense call with that expert's weights would give it.
+int choose_block_n(int64_t N, int64_t K, bi_dtype_t dtype)
+{
+    struct Row {
+        int64_t n, k;
+        int dtype, bn;
+    };
+    static const Row table[] = {
+        {4096, 7168, BI_DTYPE_BF16, 32},               // decode-shaped projection
+        {7168, 2048, BI_DTYPE_BF16, 256},              // prefill-shaped, wide N
+        {2048, 7168, BI_DTYPE_BF16, 128},              // prefill-shaped, long K; MoE experts
+        {256, 512, BI_DTYPE_BF16, 32},                 // small correctness shape
+        {7168, 7168, BI_DTYPE_E4M3_BLOCKSCALED, 64},   // FP8 projection
+    };
+    for (const Row &r : table)
+        if (r.n == N && r.k == K && r.dtype == dtype)
+            return r.bn;
+    const int max_bn = dtype == BI_DTYPE_E4M3_BLOCKSCALED ? 128 : 256;
+    for (int bn = max_bn; bn > 32; bn /= 2)
+        if ((N + bn - 1) / bn >= 100)
+            return bn;
+    return 32;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Per-device state
+// ---------------------------------------------------------------------------------------------
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool probed = false;
+    bool ok = false;       // sm_100 family
+    int num_sms = 0;
+    bool attr_set[kNumKernels] = {};
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bi_status_t current_device(int *dev_out, DeviceInfo **info_out)
+{
+    int count = 0;
+    if (cudaGetDeviceCount(&count) != cudaSuccess || count <= 0) {
+        cudaGetLastError();
+        return BI_ERR_NO_DEVICE;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return BI_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.probed) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess)
+            return BI_ERR_CUDA;
+        d.ok = prop.major == 10;
+        d.num_sms = prop.multiProcessorCount;
+        d.probed = true;
+    }
+    if (!d.ok)
+        return BI_ERR_NO_DEVICE;
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    if (!g_encode)
+        return BI_ERR_CUDA;
+    *dev_out = dev;
+    *info_out = &d;
+    return BI_OK;
+}
+
+} // namespace
+
+// ---------------------------------------------------------------------------------------------
+// The plan object
+// ---------------------------------------------------------------------------------------------
+
+struct bi_plan_s {
+    int64_t n = 0, k = 0;
+    bi_dtype_t dtype = BI_DTYPE_BF16;
+    int experts = 1;
+    const KernelEntry *kernel = nullptr;
+    int kernel_index = 0;
+    uint64_t timeout_ns = 2000000000ull;
+    uint32_t debug_flags = 0;
+    std::mutex mu;
+    int *status[kMaxDevices] = {};
+};
+
+namespace {
+
+bi_status_t plan_status_word(bi_plan_s *plan, int dev, int **out)
+{
+    std::lock_guard<std::mutex> lock(plan->mu);
+    if (!plan->status[dev]) {
+        int *p = nullptr;
+        if (cudaMalloc(&p, sizeof(int)) != cudaSuccess)
+            return BI_ERR_CUDA;
+        if (cudaMemset(p, 0, sizeof(int)) != cudaSuccess) {
+            cudaFree(p);
+            return BI_ERR_CUDA;
+        }
+        plan->status[dev] = p;
+    }
+    *out = plan->status[dev];
+    return BI_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bi_status_t encode_2d(CUtensorMap *map, const void *base, bool fp8, int64_t inner, int64_t rows,
+                      int64_t ld_elems, int box_rows)
+{
+    const int elt = fp8 ? 1 : 2;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_elems * elt)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(bi::kRowBytes / elt),
+                         static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                          2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status_t ensure_kernel_attr(bi_plan_s *plan, DeviceInfo *d)
+{
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (!d->attr_set[plan->kernel_index]) {
+        if (cudaFuncSetAttribute(reinterpret_cast<const void *>(plan->kernel->fn),
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 plan->kernel->smem) != cudaSuccess)
+            return BI_ERR_CUDA;
+        d->attr_set[plan->kernel_index] = true;
+    }
+    return BI_OK;
+}
+
+bi_status_t launch_zero(void *C, int64_t ldc, int64_t rows, int64_t n, cudaStream_t stream)
+{
+    const int64_t total = rows * n;
+    int blocks = static_cast<int>((total + 255) / 256);
+    if (blocks > 4096)
+        blocks = 4096;
+    if (blocks < 1)
+        blocks = 1;
+    bi::bi_zero_kernel<<<blocks, 256, 0, stream>>>(static_cast<__nv_bfloat16 *>(C), ldc, rows, n);
+    return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+// Checks shared by the dense and grouped runs (pointers, strides, alignment, 32-bit limits).
+bi_status_t check_common(const bi_plan_s *plan, int64_t rows, const void *A, int64_t lda,
+                         const void *B, int64_t ldb, const void *C, int64_t ldc)
+{
+    if (rows < 0)
+        return BI_ERR_INVALID_ARG;
+    if (rows == 0 || plan->n == 0)
+        return BI_OK;
+    if (!C)
+        return BI_ERR_INVALID_ARG;
+    if (ldc < plan->n)
+        return BI_ERR_INVALID_ARG;
+    if (!aligned16(C) || (ldc * 2) % 16 != 0)
+        return BI_ERR_ALIGNMENT;
+    if (plan->k == 0)
+        return BI_OK;
+    if (!A || !B)
+        return BI_ERR_INVALID_ARG;
+    if (lda < plan->k || ldb < plan->k)
+        return BI_ERR_INVALID_ARG;
+    const int elt = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED ? 1 : 2;
+    if (!aligned16(A) || !aligned16(B) || (lda * elt) % 16 != 0 || (ldb * elt) % 16 != 0)
+        return BI_ERR_ALIGNMENT;
+    if (rows > INT32_MAX - 256 || plan->n * plan->experts > INT32_MAX - 512 ||
+        plan->k > INT32_MAX - 256)
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    return BI_OK;
+}
+
+GemmParams base_params(const bi_plan_s *plan, int64_t rows, void *C, int64_t ldc, int *status)
+{
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    const int elt = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED ? 1 : 2;
+    p.rows = static_cast<int32_t>(rows);
+    p.n = static_cast<int32_t>(plan->n);
+    p.k = static_cast<int32_t>(plan->k);
+    p.num_k_blocks = static_cast<int32_t>((plan->k * elt + bi::kRowBytes - 1) / bi::kRowBytes);
+    p.num_n_blocks = static_cast<int32_t>((plan->n + plan->kernel->bn - 1) / plan->kernel->bn);
+    p.num_m_blocks = static_cast<int32_t>((rows + bi::kBlockM - 1) / bi::kBlockM);
+    p.num_experts = plan->experts;
+    p.raster_m = 16;
+    p.c = static_cast<__nv_bfloat16 *>(C);
+    p.ldc = ldc;
+    p.kb_scale = static_cast<int32_t>((plan->k + 127) / 128);
+    p.status = status;
+    p.timeout_ns = plan->timeout_ns;
+    p.debug_flags = plan->debug_flags;
+    return p;
+}
+
+bi_status_t launch_main(const bi_plan_s *plan, const CUtensorMap &ta, const CUtensorMap &tb,
+                        const GemmParams &p, int grid, cudaStream_t stream)
+{
+    if (grid < 1)
+        grid = 1;
+    plan->kernel->fn<<<grid, bi::kThreads, plan->kernel->smem, stream>>>(ta, tb, p);
+    return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+} // namespace
+
+// ---------------------------------------------------------------------------------------------
+// extern "C" ABI
+// ---------------------------------------------------------------------------------------------
+
+extern "C" {
+
+int bi_gemm_abi_version(void) { return BI_GEMM_ABI_VERSION; }
+
+const char *bi_status_string(bi_status_t s)
+{
+    switch (s) {
+    case BI_OK: return "BI_OK";
+    case BI_ERR_INVALID_ARG: return "BI_ERR_INVALID_ARG: invalid argument";
+    case BI_ERR_ALIGNMENT: return "BI_ERR_ALIGNMENT: pointer or stride not 16-byte aligned";
+    case BI_ERR_UNSUPPORTED_SHAPE: return "BI_ERR_UNSUPPORTED_SHAPE: shape not supported";
+    case BI_ERR_DTYPE_MISMATCH: return "BI_ERR_DTYPE_MISMATCH: arguments do not match the plan's dtype";
+    case BI_ERR_CUDA: return "BI_ERR_CUDA: a CUDA call failed";
+    case BI_ERR_DEVICE_TIMEOUT: return "BI_ERR_DEVICE_TIMEOUT: a device pipeline wait ran out of time";
+    case BI_ERR_BAD_OFFSETS: return "BI_ERR_BAD_OFFSETS: malformed grouped expert offsets";
+    case BI_ERR_NO_DEVICE: return "BI_ERR_NO_DEVICE: no sm_100 CUDA device";
+    }
+    return "BI_ERR_UNKNOWN";
+}
+
+bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype, int num_experts)
+{
+    if (!out)
+        return BI_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (N < 0 || K < 0 || num_experts < 1)
+        return BI_ERR_INVALID_ARG;
+    if (dtype != BI_DTYPE_BF16 && dtype != BI_DTYPE_E4M3_BLOCKSCALED)
+        return BI_ERR_INVALID_ARG;
+    if (num_experts > bi::kMaxExperts)
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    if (num_experts > 1 && dtype != BI_DTYPE_BF16)
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    if (N > INT32_MAX / 2 || K > INT32_MAX / 2 || N * num_experts > INT32_MAX / 2)
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    const bool fp8 = dtype == BI_DTYPE_E4M3_BLOCKSCALED;
+    const int bn = choose_block_n(N, K, dtype);
+    const KernelEntry *k = find_kernel(bn, fp8, num_experts > 1);
+    if (!k)
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    bi_plan_s *p = new (std::nothrow) bi_plan_s();
+    if (!p)
+        return BI_ERR_INVALID_ARG;
+    p->n = N;
+    p->k = K;
+    p->dtype = dtype;
+    p->experts = num_experts;
+    p->kernel = k;
+    p->kernel_index = static_cast<int>(k - kKernels);
+    *out = p;
+    return BI_OK;
+}
+
+bi_status_t bi_gemm_plan_destroy(bi_plan_t plan)
+{
+    if (!plan)
+        return BI_OK;
+    int cur = -1;
+    const bool have_dev = cudaGetDevice(&cur) == cudaSuccess;
+    for (int d = 0; d < kMaxDevices; ++d) {
+        if (plan->status[d]) {
+            cudaSetDevice(d);
+            cudaFree(plan->status[d]);
+        }
+    }
+    if (have_dev)
+        cudaSetDevice(cur);
+    cudaGetLastError();
+    delete plan;
+    return BI_OK;
+}
+
+bi_status_t bi_gemm_plan_describe(bi_plan_t plan, bi_plan_info_t *info)
+{
+    if (!plan || !info)
+        return BI_ERR_INVALID_ARG;
+    const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
+    std::memset(info, 0, sizeof(*info));
+    info->n = plan->n;
+    info->k = plan->k;
+    info->dtype = plan->dtype;
+    info->num_experts = plan->experts;
+    info->block_m = bi::kBlockM;
+    info->block_n = plan->kernel->bn;
+    info->block_k = fp8 ? 128 : 64;
+    info->cta_group = 1;
+    info->mma_m = bi::kBlockM;
+    info->mma_n = plan->kernel->bn;
+    info->mma_k = fp8 ? 32 : 16;
+    info->stages = plan->kernel->stages;
+    info->k_order_id = 0;
+    info->threads_per_cta = bi::kThreads;
+    info->smem_bytes = plan->kernel->smem;
+    const int nacc = fp8 ? ((512 / plan->kernel->bn) < 4 ? (512 / plan->kernel->bn) : 4) : 2;
+    int cols = 32;
+    while (cols < nacc * plan->kernel->bn)
+        cols *= 2;
+    info->tmem_columns = cols;
+    return BI_OK;
+}
+
+bi_status_t bi_gemm_set_wait_timeout(bi_plan_t plan, uint64_t timeout_ns)
+{
+    if (!plan)
+        return BI_ERR_INVALID_ARG;
+    plan->timeout_ns = timeout_ns ? timeout_ns : 2000000000ull;
+    return BI_OK;
+}
+
+bi_status_t bi_gemm_debug_set_flags(bi_plan_t plan, uint32_t flags)
+{
+    if (!plan)
+        return BI_ERR_INVALID_ARG;
+    plan->debug_flags = flags;
+    return BI_OK;
+}
+
+bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, const void *B,
+                        int64_t ldb, void *C, int64_t ldc, const float *scale_a, int64_t ld_sa,
+                        const float *scale_b, cudaStream_t stream)
+{
+    if (!plan)
+        return BI_ERR_INVALID_ARG;
+    if (plan->experts != 1)
+        return BI_ERR_INVALID_ARG;
+    const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
+    if (fp8) {
+        if (M > 0 && plan->n > 0 && plan->k > 0) {
+            if (!scale_a || !scale_b)
+                return BI_ERR_DTYPE_MISMATCH;
+            if (ld_sa < M)
+                return BI_ERR_INVALID_ARG;
+            if ((reinterpret_cast<uintptr_t>(scale_a) & 3u) || (reinterpret_cast<uintptr_t>(scale_b) & 3u))
+                return BI_ERR_ALIGNMENT;
+        }
+    } else if (scale_a || scale_b) {
+        return BI_ERR_DTYPE_MISMATCH;
+    }
+    bi_status_t st = check_common(plan, M, A, lda, B, ldb, C, ldc);
+    if (st != BI_OK || M == 0 || plan->n == 0)
+        return st;
+    int dev = 0;
+    DeviceInfo *d = nullptr;
+    if ((st = current_device(&dev, &d)) != BI_OK)
+        return st;
+    if (plan->k == 0)
+        return launch_zero(C, ldc, M, plan->n, stream);
+    int *status = nullptr;
+    if ((st = plan_status_word(plan, dev, &status)) != BI_OK)
+        return st;
+    if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
+        return st;
+    CUtensorMap ta, tb;
+    if ((st = encode_2d(&ta, A, fp8, plan->k, M, lda, bi::kBlockM)) != BI_OK)
+        return st;
+    if ((st = encode_2d(&tb, B, fp8, plan->k, plan->n, ldb, plan->kernel->bn)) != BI_OK)
+        return st;
+    GemmParams p = base_params(plan, M, C, ldc, status);
+    p.scale_a = scale_a;
+    p.ld_sa = ld_sa;
+    p.scale_b = scale_b;
+    const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
+    const int grid = static_cast<int>(tiles < d->num_sms ? tiles : d->num_sms);
+    return launch_main(plan, ta, tb, p, grid, stream);
+}
+
+bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *A, int64_t lda,
+                                const void *B, int64_t ldb, void *C, int64_t ldc,
+                                const int32_t *expert_offsets, cudaStream_t stream)
+{
+    if (!plan)
+        return BI_ERR_INVALID_ARG;
+    if (plan->experts <= 1)
+        return BI_ERR_INVALID_ARG;
+    bi_status_t st = check_common(plan, total_rows, A, lda, B, ldb, C, ldc);
+    if (st != BI_OK || total_rows == 0 || plan->n == 0)
+        return st;
+    if (!expert_offsets)
+        return BI_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(expert_offsets) & 3u)
+        return BI_ERR_ALIGNMENT;
+    int dev = 0;
+    DeviceInfo *d = nullptr;
+    if ((st = current_device(&dev, &d)) != BI_OK)
+        return st;
+    if (plan->k == 0)
+        return launch_zero(C, ldc, total_rows, plan->n, stream);
+    int *status = nullptr;
+    if ((st = plan_status_word(plan, dev, &status)) != BI_OK)
+        return st;
+    if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
+        return st;
+    CUtensorMap ta, tb;
+    if ((st = encode_2d(&ta, A, false, plan->k, total_rows, lda, bi::kBlockM)) != BI_OK)
+        return st;
+    if ((st = encode_2d(&tb, B, false, plan->k, plan->n * plan->experts, ldb, plan->kernel->bn)) != BI_OK)
+        return st;
+    GemmParams p = base_params(plan, total_rows, C, ldc, status);
+    p.offsets = expert_offsets;
+    // Upper bound on the tile count without reading the offsets: sum_e ceil(len_e/128) is at
+    // most total_rows/128 + E.
+    const int64_t max_tiles = (total_rows / bi::kBlockM + plan->experts) * p.num_n_blocks;
+    const int grid = static_cast<int>(max_tiles < d->num_sms ? max_tiles : d->num_sms);
+    return launch_main(plan, ta, tb, p, grid, stream);
+}
+
+bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M, const void *A_host, int64_t lda,
+                             const void *B, int64_t ldb, void *C_host, int64_t ldc,
+                             const float *scale_a_host, int64_t ld_sa, const float *scale_b,
+                             void *A_dev, void *C_dev, float *scale_a_dev, cudaStream_t stream)
+{
+    if (!plan)
+        return BI_ERR_INVALID_ARG;
+    if (M < 0)
+        return BI_ERR_INVALID_ARG;
+    if (M == 0 || plan->n == 0)
+        return BI_OK;
+    const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
+    if (!C_host || !C_dev || (plan->k > 0 && (!A_host || !A_dev)))
+        return BI_ERR_INVALID_ARG;
+    if (fp8 && plan->k > 0 && (!scale_a_host || !scale_a_dev))
+        return BI_ERR_DTYPE_MISMATCH;
+    const int elt = fp8 ? 1 : 2;
+    // Validate before enqueueing any copy.
+    bi_status_t st = check_common(plan, M, A_dev, lda, B, ldb, C_dev, ldc);
+    if (st != BI_OK)
+        return st;
+    if (plan->k > 0) {
+        if (cudaMemcpyAsync(A_dev, A_host, static_cast<size_t>(M * lda * elt),
+                            cudaMemcpyHostToDevice, stream) != cudaSuccess)
+            return BI_ERR_CUDA;
+        if (fp8 && cudaMemcpyAsync(scale_a_dev, scale_a_host,
+                                   static_cast<size_t>(((plan->k + 127) / 128) * ld_sa * 4),
+                                   cudaMemcpyHostToDevice, stream) != cudaSuccess)
+            return BI_ERR_CUDA;
+    }
+    st = bi_gemm_run(plan, M, A_dev, lda, B, ldb, C_dev, ldc, fp8 ? scale_a_dev : nullptr, ld_sa,
+                     fp8 ? scale_b : nullptr, stream);
+    if (st != BI_OK)
+        return st;
+    if (cudaMemcpyAsync(C_host, C_dev, static_cast<size_t>(M * ldc * 2), cudaMemcpyDeviceToHost,
+                        stream) != cudaSuccess)
+        return BI_ERR_CUDA;
+    return BI_OK;
+}
+
+bi_status_t bi_gemm_sync_status(bi_plan_t plan, cudaStream_t stream)
+{
+    if (!plan)
+        return BI_ERR_INVALID_ARG;
+    int dev = 0;
+    DeviceInfo *d = nullptr;
+    bi_status_t st = current_device(&dev, &d);
+    if (st != BI_OK)
+        return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess)
+        return BI_ERR_CUDA;
+    int *word = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(plan->mu);
+        word = plan->status[dev];
+    }
+    if (!word)
+        return BI_OK;
+    int host = 0;
+    if (cudaMemcpy(&host, word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return BI_ERR_CUDA;
+    if (host != 0 && cudaMemset(word, 0, sizeof(int)) != cudaSuccess)
+        return BI_ERR_CUDA;
+    return host == 0 ? BI_OK : static_cast<bi_status_t>(host);
+}
+
+} // extern "C"

@@ -1,0 +1,118 @@
+"""Host-side tests of the C ABI that need no GPU: the library loads, exports every symbol the
+header declares, plans are pure functions of (N, K, dtype, num_experts), and argument errors come
+back as status codes without any device call."""
+import ctypes
+import json
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+import invariant_deterministic_gemm_bi_b200 as bg
+from invariant_deterministic_gemm_bi_b200 import binding
+
+REPO = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(REPO, "include", "bi_gemm.h")
+
+
+def declared_functions():
+    text = open(HEADER, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bi_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(binding.LIB_PATH)
+    names = declared_functions()
+    assert len(names) >= 10
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in bi_gemm.h but not exported"
+    assert sorted(binding.EXPORTED) == names
+
+
+def test_abi_version_and_status_strings():
+    assert bg.bi_gemm_abi_version() == 1
+    for code, name in binding.STATUS_NAMES.items():
+        assert bg.bi_status_string(code).startswith(name)
+
+
+def test_plan_describe_is_m_free_and_sane():
+    for (N, K, dt, E) in [(4096, 7168, 0, 1), (7168, 2048, 0, 1), (2048, 7168, 0, 1),
+                          (7168, 7168, 1, 1), (2048, 7168, 0, 64), (256, 512, 0, 1), (5, 3, 0, 1)]:
+        info = bg.bi_gemm_plan_describe(bg.bi_gemm_plan(N, K, dt, E))
+        assert info["n"] == N and info["k"] == K and info["num_experts"] == E
+        assert info["k_order_id"] == 0 and info["block_m"] == 128
+        assert info["block_k"] * (1 if dt == 1 else 2) == 128
+        assert info["mma_n"] == info["block_n"] and info["block_n"] % 32 == 0
+        assert info["smem_bytes"] <= 232448
+        assert info["tmem_columns"] <= 512
+    # grouped plans share the dense plan's tile configuration
+    d = bg.bi_gemm_plan_describe(bg.bi_gemm_plan(2048, 7168, 0, 1))
+    g = bg.bi_gemm_plan_describe(bg.bi_gemm_plan(2048, 7168, 0, 64))
+    assert d["block_n"] == g["block_n"] and d["mma_n"] == g["mma_n"]
+
+
+def test_plan_is_the_same_in_a_fresh_process():
+    shapes = [(4096, 7168, 0, 1), (7168, 7168, 1, 1), (2048, 7168, 0, 64), (1000, 100, 0, 1)]
+    here = [bg.bi_gemm_plan_describe(bg.bi_gemm_plan(*s)) for s in shapes]
+    code = ("import json, invariant_deterministic_gemm_bi_b200 as bg;"
+            f"print(json.dumps([bg.bi_gemm_plan_describe(bg.bi_gemm_plan(*s)) for s in {shapes!r}]))")
+    out = subprocess.run([sys.executable, "-c", code], cwd=REPO, capture_output=True, text=True,
+                         check=True).stdout
+    assert json.loads(out.strip().splitlines()[-1]) == here
+
+
+@pytest.mark.parametrize("args,status", [
+    ((-1, 8, 0, 1), "BI_ERR_INVALID_ARG"),
+    ((8, -1, 0, 1), "BI_ERR_INVALID_ARG"),
+    ((8, 8, 0, 0), "BI_ERR_INVALID_ARG"),
+    ((8, 8, 7, 1), "BI_ERR_INVALID_ARG"),
+    ((8, 8, 1, 4), "BI_ERR_UNSUPPORTED_SHAPE"),
+    ((8, 8, 0, 2048), "BI_ERR_UNSUPPORTED_SHAPE"),
+])
+def test_plan_rejects_bad_arguments(args, status):
+    with pytest.raises(bg.BiGemmError) as e:
+        bg.bi_gemm_plan(*args)
+    assert e.value.name == status
+
+
+def test_run_rejects_bad_arguments_without_touching_a_device():
+    lib = binding.load_library()
+    plan = bg.bi_gemm_plan(64, 64)
+    h = plan.handle
+    S = binding.STATUS
+    # null plan
+    assert lib.bi_gemm_run(None, 1, 16, 64, 16, 64, 16, 64, None, 0, None, None) == S["BI_ERR_INVALID_ARG"]
+    # negative M
+    assert lib.bi_gemm_run(h, -1, 16, 64, 16, 64, 16, 64, None, 0, None, None) == S["BI_ERR_INVALID_ARG"]
+    # M = 0 is a no-op
+    assert lib.bi_gemm_run(h, 0, None, 64, None, 64, None, 64, None, 0, None, None) == 0
+    # null A / C
+    assert lib.bi_gemm_run(h, 1, None, 64, 16, 64, 16, 64, None, 0, None, None) == S["BI_ERR_INVALID_ARG"]
+    assert lib.bi_gemm_run(h, 1, 16, 64, 16, 64, None, 64, None, 0, None, None) == S["BI_ERR_INVALID_ARG"]
+    # strides below the extent, misaligned pointers and strides
+    assert lib.bi_gemm_run(h, 1, 16, 32, 16, 64, 16, 64, None, 0, None, None) == S["BI_ERR_INVALID_ARG"]
+    assert lib.bi_gemm_run(h, 1, 18, 64, 16, 64, 16, 64, None, 0, None, None) == S["BI_ERR_ALIGNMENT"]
+    assert lib.bi_gemm_run(h, 1, 16, 68, 16, 64, 16, 64, None, 0, None, None) == S["BI_ERR_ALIGNMENT"]
+    assert lib.bi_gemm_run(h, 1, 16, 64, 16, 64, 16, 66, None, 0, None, None) == S["BI_ERR_ALIGNMENT"]
+    # scales on a bf16 plan
+    assert lib.bi_gemm_run(h, 1, 16, 64, 16, 64, 16, 64, 16, 1, 16, None) == S["BI_ERR_DTYPE_MISMATCH"]
+    # a grouped call on a dense plan and the reverse
+    assert lib.bi_grouped_gemm_run(h, 1, 16, 64, 16, 64, 16, 64, 16, None) == S["BI_ERR_INVALID_ARG"]
+    gplan = bg.bi_gemm_plan(64, 64, 0, 4)
+    assert lib.bi_gemm_run(gplan.handle, 1, 16, 64, 16, 64, 16, 64, None, 0, None, None) == S["BI_ERR_INVALID_ARG"]
+    assert lib.bi_grouped_gemm_run(gplan.handle, 1, 16, 64, 16, 64, 16, 64, None, None) == S["BI_ERR_INVALID_ARG"]
+    # FP8 without scales, or ld_sa below M
+    fplan = bg.bi_gemm_plan(64, 128, 1, 1)
+    assert lib.bi_gemm_run(fplan.handle, 4, 16, 128, 16, 128, 16, 64, None, 4, None, None) == S["BI_ERR_DTYPE_MISMATCH"]
+    assert lib.bi_gemm_run(fplan.handle, 4, 16, 128, 16, 128, 16, 64, 16, 3, 16, None) == S["BI_ERR_INVALID_ARG"]
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="a GPU is present")
+def test_valid_run_without_a_device_reports_no_device():
+    lib = binding.load_library()
+    plan = bg.bi_gemm_plan(64, 64)
+    st = lib.bi_gemm_run(plan.handle, 1, 16, 64, 16, 64, 16, 64, None, 0, None, None)
+    assert binding.STATUS_NAMES[st] == "BI_ERR_NO_DEVICE"

@@ -1,0 +1,224 @@
+"""GPU batch invariance, bitwise: a row computed alone (M = 1) must come out with exactly the same
+bits inside every larger batch, at any position, under row permutations and among fresh random
+co-batched rows ("DeepSeek不惜代价保住它！V4关键特性被挖出来了" (QbitAI), section
+"什么是batch invariance").  Needs no oracle: the M = 1 result is the single correct bit pattern.
+"""
+import numpy as np
+import pytest
+import torch
+
+import invariant_deterministic_gemm_bi_b200 as bg
+from invariant_deterministic_gemm_bi_b200 import inputs
+from tests.gpu_util import kblock_major_scales
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+class Dense:
+    def __init__(self, B, dtype=bg.BI_DTYPE_BF16, scale_b=None):
+        self.B = B
+        self.N, self.K = B.shape
+        self.plan = bg.bi_gemm_plan(self.N, self.K, dtype, 1)
+        self.scale_b = scale_b
+
+    def __call__(self, A, sa_mk=None):
+        C = torch.empty((A.shape[0], self.N), dtype=torch.bfloat16, device=DEV)
+        sa = kblock_major_scales(sa_mk) if sa_mk is not None else None
+        bg.bi_gemm_run(self.plan, A, self.B, C, scale_a=sa, scale_b=self.scale_b)
+        bg.bi_gemm_sync_status(self.plan)
+        return C
+
+
+def alone(f, rows, scales=None):
+    """Each row computed on its own (M = 1)."""
+    out = []
+    for i in range(rows.shape[0]):
+        out.append(f(rows[i:i + 1].contiguous(), None if scales is None else scales[i:i + 1]))
+    return torch.cat(out).view(torch.int16)
+
+
+def check_in_batch(f, test_rows, ref_bits, M, seed, fresh, scales=None, fresh_scales=None,
+                   positions=None):
+    """Put min(M, T) test rows at random (or given) positions among fresh rows; compare bits."""
+    rng = np.random.default_rng(seed)
+    T = test_rows.shape[0]
+    k = min(M, T) if positions is None else len(positions)
+    pick = rng.choice(T, size=k, replace=False)
+    pos = rng.choice(M, size=k, replace=False) if positions is None else np.asarray(positions)[:k]
+    batch = fresh(M).clone()
+    batch[torch.from_numpy(pos).to(DEV)] = test_rows[torch.from_numpy(pick).to(DEV)]
+    bscales = None
+    if scales is not None:
+        bscales = fresh_scales(M).clone()
+        bscales[torch.from_numpy(pos).to(DEV)] = scales[torch.from_numpy(pick).to(DEV)]
+    C = f(batch, bscales).view(torch.int16)
+    got = C[torch.from_numpy(pos).to(DEV)]
+    want = ref_bits[torch.from_numpy(pick).to(DEV)]
+    bad = (got != want).any(dim=1)
+    assert not bad.any(), f"M={M}: {int(bad.sum())} of {k} rows differ from their M=1 bits"
+
+
+# ---------------------------------------------------------------------------------------------
+# small shape: M in {1, 3, 8, 17, 64} under permutations (Gaussian and integer inputs)
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", ["gaussian", "integer"])
+def test_small_rows_invariant_under_batch_size_and_permutation(kind):
+    gen = inputs.bf16_gaussian if kind == "gaussian" else inputs.bf16_integers
+    B = gen((256, 512), seed=1001, device=DEV)
+    f = Dense(B)
+    test_rows = gen((16, 512), seed=1002, device=DEV)
+    ref = alone(f, test_rows)
+    for M in [1, 3, 8, 17, 64]:
+        for trial in range(8):
+            s = inputs.derived_seed(1000, M, trial)
+            check_in_batch(f, test_rows, ref, M, s,
+                           lambda m, s=s: gen((m, 512), seed=s, device=DEV))
+    # a full permutation of one batch permutes its output rows bit for bit
+    A = gen((64, 512), seed=1003, device=DEV)
+    C = f(A).view(torch.int16)
+    for trial in range(8):
+        perm = torch.from_numpy(np.random.default_rng(trial).permutation(64)).to(DEV)
+        assert torch.equal(f(A[perm].contiguous()).view(torch.int16), C[perm])
+
+
+# ---------------------------------------------------------------------------------------------
+# decode-shaped: N = 4096, K = 7168, M = 1 .. 256, fresh co-batched rows, first/last positions
+# ---------------------------------------------------------------------------------------------
+
+def test_decode_rows_invariant_across_m_sweep():
+    N, K = 4096, 7168
+    B = inputs.bf16_gaussian((N, K), seed=2001, std=K ** -0.5, device=DEV)
+    f = Dense(B)
+    test_rows = inputs.bf16_gaussian((32, K), seed=2002, device=DEV)
+    ref = alone(f, test_rows)
+    for M in [2, 4, 8, 16, 32, 64, 128, 256]:
+        for trial in range(4):
+            s = inputs.derived_seed(2000, M, trial)
+            fresh = lambda m, s=s: inputs.bf16_gaussian((m, K), seed=s, device=DEV)
+            check_in_batch(f, test_rows, ref, M, s, fresh)
+        check_in_batch(f, test_rows, ref, M, M, fresh, positions=[0, M - 1])
+
+
+# ---------------------------------------------------------------------------------------------
+# prefill-shaped: both shapes, M in {1024, 4096, 16384}, plus the 1024-row subset test
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K", [(7168, 2048), (2048, 7168)])
+def test_prefill_rows_invariant_and_subsets(N, K):
+    B = inputs.bf16_gaussian((N, K), seed=3001, std=K ** -0.5, device=DEV)
+    f = Dense(B)
+    test_rows = inputs.bf16_gaussian((256, K), seed=3002, device=DEV)
+    ref = alone(f, test_rows)
+    batches = {}
+    for M in [1024, 4096, 16384]:
+        s = inputs.derived_seed(3000, M)
+        fresh = lambda m, s=s: inputs.bf16_gaussian((m, K), seed=s, device=DEV)
+        check_in_batch(f, test_rows, ref, M, s, fresh)
+        batches[M] = fresh(M)
+    # a random 1024-row subset of the 16384-row batch, run as its own call
+    big = batches[16384]
+    Cbig = f(big).view(torch.int16)
+    idx = torch.from_numpy(np.random.default_rng(7).choice(16384, 1024, replace=False)).to(DEV)
+    Csub = f(big[idx].contiguous()).view(torch.int16)
+    assert torch.equal(Csub, Cbig[idx])
+
+
+# ---------------------------------------------------------------------------------------------
+# FP8 block-scaled: M = 1 .. 4096, co-batched rows with different scales
+# ---------------------------------------------------------------------------------------------
+
+def test_fp8_rows_invariant_across_m_sweep():
+    N = K = 7168
+    KB = K // 128
+    qb = inputs.e4m3_gaussian((N, K), seed=4001, device=DEV)
+    sb = inputs.scales_log_uniform((N // 128, KB), seed=4002, device=DEV)
+    f = Dense(qb, bg.BI_DTYPE_E4M3_BLOCKSCALED, scale_b=sb)
+    test_rows = inputs.e4m3_gaussian((32, K), seed=4003, device=DEV)
+    test_scales = inputs.scales_log_uniform((32, KB), seed=4004, device=DEV)
+    ref = alone(f, test_rows, test_scales)
+    for M in [2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096]:
+        for trial in range(2):
+            s = inputs.derived_seed(4000, M, trial)
+            check_in_batch(f, test_rows, ref, M, s,
+                           lambda m, s=s: inputs.e4m3_gaussian((m, K), seed=s, device=DEV),
+                           scales=test_scales,
+                           fresh_scales=lambda m, s=s: inputs.scales_log_uniform((m, KB), seed=s + 1,
+                                                                                 device=DEV))
+
+
+# ---------------------------------------------------------------------------------------------
+# grouped MoE: per (token, expert) rows invariant to T and to the other tokens of the expert
+# ---------------------------------------------------------------------------------------------
+
+def moe_outputs(plan, B, tokens, routing):
+    A = tokens[routing.token_of_row.to(DEV)].contiguous()
+    C = torch.empty((A.shape[0], B.shape[1]), dtype=torch.bfloat16, device=DEV)
+    bg.bi_grouped_gemm_run(plan, A, B, C, routing.offsets.to(DEV))
+    bg.bi_gemm_sync_status(plan)
+    return C.view(torch.int16)
+
+
+def pair_bits(C, routing):
+    """{(token, expert): output bits} for a grouped result."""
+    tok = routing.token_of_row.tolist()
+    exp = routing.expert_of_row.tolist()
+    return {(t, e): C[i] for i, (t, e) in enumerate(zip(tok, exp))}
+
+
+def test_moe_rows_invariant_to_t_and_routing():
+    E, N, K = 64, 2048, 7168
+    plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_BF16, E)
+    B = inputs.bf16_gaussian((E, N, K), seed=5001, std=K ** -0.5, device=DEV)
+    test_tokens = inputs.bf16_gaussian((16, K), seed=5002, device=DEV)
+    test_logits_seed = 5003
+    # each test token alone (T = 1): its 8 (token, expert) rows
+    g = inputs.generator(test_logits_seed, DEV)
+    test_logits = torch.randn(16, E, generator=g, device=DEV)
+    test_experts = inputs.route_topk(test_logits, 8)
+    ref = {}
+    for i in range(16):
+        r = inputs.group_by_expert(test_experts[i:i + 1].cpu(), E)
+        out = pair_bits(moe_outputs(plan, B, test_tokens[i:i + 1], r), r)
+        for (t, e), v in out.items():
+            ref[(i, e)] = v
+    for T in [64, 1024, 8192]:
+        s = inputs.derived_seed(5000, T)
+        tokens = inputs.bf16_gaussian((T, K), seed=s, device=DEV)
+        logits = torch.randn(T, E, generator=inputs.generator(s + 1, DEV), device=DEV)
+        pos = np.random.default_rng(T).choice(T, size=16, replace=False)
+        tokens[torch.from_numpy(pos).to(DEV)] = test_tokens
+        logits[torch.from_numpy(pos).to(DEV)] = test_logits
+        r = inputs.group_by_expert(inputs.route_topk(logits, 8).cpu(), E)
+        out = pair_bits(moe_outputs(plan, B, tokens, r), r)
+        for i, p in enumerate(pos):
+            for e in test_experts[i].tolist():
+                assert torch.equal(out[(int(p), e)], ref[(i, e)]), f"T={T} token {i} expert {e}"
+
+
+@pytest.mark.parametrize("pattern", ["all_one_expert", "segments_127_128_129", "singletons"])
+def test_moe_adversarial_routings(pattern):
+    E, N, K = 8, 256, 512
+    plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_BF16, E)
+    B = inputs.bf16_gaussian((E, N, K), seed=5101, device=DEV)
+    tokens = inputs.bf16_gaussian((400, K), seed=5102, device=DEV)
+    if pattern == "all_one_expert":
+        experts = np.full(400, 3)
+    elif pattern == "segments_127_128_129":
+        experts = np.repeat([0, 1, 2, 5], [127, 128, 129, 16])
+    else:
+        experts = np.concatenate([np.arange(8), np.full(392, 7)])
+    experts = np.sort(experts)
+    r = inputs.routing_from_assignment(experts, E)
+    C = moe_outputs(plan, B, tokens, r)
+    # every row equals the same token computed alone with its expert (a one-row call)
+    for i in np.random.default_rng(1).choice(400, 40, replace=False):
+        e = int(experts[i])
+        one = inputs.routing_from_assignment(np.array([e]), E)
+        C1 = moe_outputs(plan, B, tokens[i:i + 1], one)
+        assert torch.equal(C1[0], C[i]), f"{pattern}: row {i}"
+    # and the same as a dense call with that expert's weights
+    f = Dense(B[3].contiguous()) if pattern == "all_one_expert" else None
+    if f is not None:
+        assert torch.equal(f(tokens).view(torch.int16), C)
