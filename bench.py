@@ -1,0 +1,582 @@
+"""Benchmark of the batch-invariant GEMM on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}] [--no-extras]
+
+One step is one pass of the decode-shaped workload: the bf16 GEMM C = A . B^T with N = 4096,
+K = 7168, swept over M = 1, 2, 4, ..., 256 (nine GEMM calls, each through the C ABI).  The
+weights rotate over enough copies that every call reads them from HBM (the copies together
+are larger than twice the 126 MB L2).  A step is captured once per rotation phase as a CUDA
+graph and replayed, so the timed region measures the kernels, not Python.  The metric is the
+algorithmic HBM throughput: weight, activation and output bytes, each counted once, over the
+device time (CUDA events on the launching stream, max over ranks).
+
+Under torchrun (N > 1) every rank runs the same sweep on its own GPU with its own data: the
+units are independent problems (weak scaling), and the only collectives are the barriers and
+the max of the timings.  Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle instead (the only other place this file runs it), on a
+bounded sample of the same workload, scaled to the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+REPO = os.path.dirname(os.path.abspath(__file__))
+if REPO not in sys.path:
+    sys.path.insert(0, REPO)
+
+METRIC = "batch-invariant GEMM TFLOP/s & HBM GB/s vs M, % roofline; 0 bitwise row diffs"
+N_DEC, K_DEC = 4096, 7168
+M_SWEEP = [1, 2, 4, 8, 16, 32, 64, 128, 256]
+WORKLOAD = ("decode-shaped bf16 GEMM C=A.B^T, N=4096, K=7168, M swept 1,2,4,...,256 "
+            "(9 GEMMs per step); A~N(0,1), B~N(0,1/K) in bf16")
+
+
+def sweep_bytes(n=N_DEC, k=K_DEC, ms=M_SWEEP, elt=2):
+    """Algorithmic bytes of one step: each operand once plus the output."""
+    return sum(n * k * elt + m * k * elt + 2 * m * n for m in ms)
+
+
+def sweep_flops(n=N_DEC, k=K_DEC, ms=M_SWEEP):
+    return sum(2 * m * n * k for m in ms)
+
+
+def sweep_macs(n=N_DEC, k=K_DEC, ms=M_SWEEP):
+    return sum(m * n * k for m in ms)
+
+
+def load_peaks():
+    path = os.path.join(REPO, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p.get("hbm_gbs", 6650.0), "bf16_tflops": p.get("bf16_tflops", 1590.0),
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", 1400.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    """Polls NVML (SM clock and throttle reasons) from a thread while the timed region runs."""
+
+    REASONS = {
+        "hw_slowdown": 0x0000000000000008, "sw_thermal_slowdown": 0x0000000000000020,
+        "hw_thermal_slowdown": 0x0000000000000040, "sw_power_cap": 0x0000000000000004,
+        "hw_power_brake_slowdown": 0x0000000000000080,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+
+    def _handle(self, device_index):
+        """The NVML handle of this process's CUDA device (NVML numbers every GPU of the host)."""
+        import torch
+        nv = self.nvml
+        props = torch.cuda.get_device_properties(device_index)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            try:
+                return nv.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+            except Exception:
+                pass
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(props, "pci_domain_id", 0)
+            devid = getattr(props, "pci_device_id", 0)
+            try:
+                return nv.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{devid:02x}.0")
+            except Exception:
+                pass
+        return nv.nvmlDeviceGetHandleByIndex(device_index)
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle (the baseline leg and the reference arm)
+# ---------------------------------------------------------------------------------------------
+
+def oracle_sample(seconds_budget: float, rng_seed: int = 2000):
+    """Time the CPU oracle on a bounded sample of the decode sweep.
+
+    The sample keeps every row of the sweep (sum of M = 511 rows) and the first n_cols output
+    columns, with n_cols chosen from a calibration run so the sample takes about
+    ``seconds_budget``.  The oracle's cost is proportional to multiply-adds, so its throughput
+    is reported as the full workload's algorithmic bytes scaled by the fraction of
+    multiply-adds done, per second.
+    """
+    import numpy as np
+
+    import oracle
+    from invariant_deterministic_gemm_bi_b200 import inputs
+
+    threads = oracle.default_threads()
+    rows = sum(M_SWEEP)
+    A = inputs.to_numpy_bits(inputs.bf16_gaussian((rows, K_DEC), seed=rng_seed))
+    Bfull = inputs.to_numpy_bits(inputs.bf16_gaussian((N_DEC, K_DEC), seed=rng_seed + 1,
+                                                      std=K_DEC ** -0.5))
+    t0 = time.perf_counter()
+    oracle.gemm_bf16(A, Bfull[:8], threads=threads)
+    per_col = max((time.perf_counter() - t0) / 8, 1e-6)
+    n_cols = int(max(1, min(N_DEC, seconds_budget / per_col)))
+    t0 = time.perf_counter()
+    oracle.gemm_bf16(A, Bfull[:n_cols], threads=threads)
+    dt = time.perf_counter() - t0
+    frac = n_cols / N_DEC
+    value = sweep_bytes() * frac / dt / 1e9
+    return {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"all {rows} rows of the M sweep x first {n_cols} of {N_DEC} output columns "
+                      f"({frac:.4f} of the step's multiply-adds) in {dt:.2f} s; value = step bytes x "
+                      f"fraction / time",
+            "seconds": dt, "n_cols": n_cols}
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    steps, warmup = args.steps, args.warmup
+    budget = max(0.02, min(5.0, 90.0 / max(1, steps + warmup)))
+    cal = oracle_sample(budget)
+    n_cols = cal["n_cols"]
+
+    import oracle
+    from invariant_deterministic_gemm_bi_b200 import inputs
+    rows = sum(M_SWEEP)
+    A = inputs.to_numpy_bits(inputs.bf16_gaussian((rows, K_DEC), seed=2000))
+    B = inputs.to_numpy_bits(inputs.bf16_gaussian((N_DEC, K_DEC), seed=2001, std=K_DEC ** -0.5))[:n_cols]
+    threads = oracle.default_threads()
+    for _ in range(warmup):
+        oracle.gemm_bf16(A, B, threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.gemm_bf16(A, B, threads=threads)
+    dt = time.perf_counter() - t0
+    frac = n_cols / N_DEC
+    value = sweep_bytes() * frac * steps / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": warmup,
+        "ms_per_step": dt / steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": f"first {n_cols} of {N_DEC} output columns per step"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"all {rows} sweep rows x {n_cols} output columns per step, "
+                                   f"scaled by the fraction of multiply-adds ({frac:.4f})"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true", help="skip the other workloads' timings")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["decode", "prefill", "fp8", "moe"], default=None,
+                    help="launch one workload --profile-launches times, untimed (for ncu captures)")
+    ap.add_argument("--profile-m", type=int, default=64, help="M (MoE: tokens T) for --profile")
+    ap.add_argument("--profile-launches", type=int, default=4)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return reference_arm(args)
+    if args.profile:
+        return profile_case(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import invariant_deterministic_gemm_bi_b200 as bg
+    from invariant_deterministic_gemm_bi_b200 import inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024) or 126 * 1024 * 1024
+    wbytes = N_DEC * K_DEC * 2
+    n_copies = math.ceil(2 * l2 / wbytes) + 1
+
+    # inputs resident in HBM before the timed region (rank-specific seeds: independent problems)
+    seed = 2000 + 97 * rank
+    Bs = [inputs.bf16_gaussian((N_DEC, K_DEC), seed=seed + 1 + i, std=K_DEC ** -0.5, device=dev)
+          for i in range(n_copies)]
+    Amax = inputs.bf16_gaussian((max(M_SWEEP), K_DEC), seed=seed, device=dev)
+    As = {m: Amax[:m] for m in M_SWEEP}
+    Cs = {m: torch.empty((m, N_DEC), dtype=torch.bfloat16, device=dev) for m in M_SWEEP}
+    plan = bg.bi_gemm_plan(N_DEC, K_DEC, bg.BI_DTYPE_BF16, 1)
+    stream = torch.cuda.Stream(device=dev)
+
+    def run_step(phase):
+        for i, m in enumerate(M_SWEEP):
+            b = Bs[(phase * len(M_SWEEP) + i) % n_copies]
+            bg.bi_gemm_run(plan, As[m], b, Cs[m], stream=stream)
+
+    # one CUDA graph per rotation phase
+    with torch.cuda.stream(stream):
+        run_step(0)
+        torch.cuda.synchronize()
+        bg.bi_gemm_sync_status(plan, stream=stream)
+        graphs = []
+        for ph in range(n_copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                run_step(ph)
+            graphs.append(g)
+    torch.cuda.synchronize()
+
+    for s in range(args.warmup):
+        graphs[s % n_copies].replay()
+    torch.cuda.synchronize()
+    barrier()
+
+    sampler = ClockSampler(local)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    torch.cuda.synchronize()
+    barrier()
+    sampler.start()
+    with torch.cuda.stream(stream):
+        ev[0].record(stream)
+        for s in range(args.steps):
+            graphs[s % n_copies].replay()
+            ev[s + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    st = bg.bi_gemm_sync_status(plan, stream=stream, raise_on_error=False)
+    if st != 0:
+        raise RuntimeError(f"device status after the timed region: {bg.binding.STATUS_NAMES[st]}")
+    total_ms = ev[0].elapsed_time(ev[-1])
+    step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+
+    peaks = load_peaks()
+    step_bytes = sweep_bytes()
+    value = step_bytes * args.steps * world / (total_ms * 1e-3) / 1e9
+    tflops = sweep_flops() * args.steps * world / (total_ms * 1e-3) / 1e12
+    # roofline of the (only) kernel of the step: average launch duration from the per-step events
+    launches = len(M_SWEEP)
+    avg_launch_s = (sum(step_ms) / len(step_ms)) / launches * 1e-3
+    achieved = step_bytes / launches / avg_launch_s / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": peaks["source"], "kernel": "bi_gemm_kernel<32,10,bf16>",
+                "note": "per-launch time = step time / 9 (graph gaps included)"}
+    traffic = os.path.join(REPO, "profiles", "decode_bf16_traffic.json")
+    if os.path.exists(traffic):
+        with open(traffic) as f:
+            tr = json.load(f)
+        if tr.get("kernel_source_hash") == kernel_source_hash():
+            roofline["traffic"] = tr["bytes_per_launch"]
+
+    # row invariance on this workload: the M=256 rows against the same rows run at M=1
+    row_diffs = 0
+    with torch.cuda.stream(stream):
+        C256 = torch.empty((256, N_DEC), dtype=torch.bfloat16, device=dev)
+        bg.bi_gemm_run(plan, Amax, Bs[0], C256, stream=stream)
+        for r in [0, 1, 63, 127, 128, 200, 255]:
+            c1 = torch.empty((1, N_DEC), dtype=torch.bfloat16, device=dev)
+            bg.bi_gemm_run(plan, Amax[r:r + 1], Bs[0], c1, stream=stream)
+            stream.synchronize()
+            row_diffs += int(not torch.equal(c1.view(torch.int16)[0], C256.view(torch.int16)[r]))
+    torch.cuda.synchronize()
+
+    e2e = measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier)
+    per_m = measure_per_m(bg, plan, As, Bs, Cs, dev, stream, n_copies, peaks)
+    extras = None if args.no_extras else measure_extras(bg, inputs, dev, stream, peaks)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(10.0)
+        cpu = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "per_gpu": "independent sweep per rank",
+                       "l2": f"{n_copies} rotating weight copies ({n_copies * wbytes / 2**20:.0f} MiB"
+                             f" > 2 x {l2 / 2**20:.0f} MiB L2)",
+                       "timing": "CUDA graph replay per step, CUDA events, max over ranks",
+                       "parallelism": f"replicas x{world} (M-sharded independent problems)"},
+            "tflops": tflops,
+            "roofline": roofline, "clocks": clocks, "e2e": e2e,
+            "gpu_launches": launches * args.steps, "row_diffs": row_diffs,
+            "per_m": per_m, "cpu_baseline": cpu, "extras": extras,
+        }
+        print(json.dumps(line), flush=True)
+    del graphs
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def profile_case(args):
+    """Launch one workload a fixed number of times with rotating weights (no timing)."""
+    import torch
+
+    import invariant_deterministic_gemm_bi_b200 as bg
+    from invariant_deterministic_gemm_bi_b200 import inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    M, L = args.profile_m, args.profile_launches
+    calls = []
+    if args.profile in ("decode", "prefill"):
+        N, K = (N_DEC, K_DEC) if args.profile == "decode" else (7168, 2048)
+        plan = bg.bi_gemm_plan(N, K)
+        copies = 3 if args.profile == "decode" else 1
+        Bs = [inputs.bf16_gaussian((N, K), seed=11 + i, std=K ** -0.5, device=dev) for i in range(copies)]
+        A = inputs.bf16_gaussian((M, K), seed=10, device=dev)
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        calls = [lambda i=i: bg.bi_gemm_run(plan, A, Bs[i % copies], C) for i in range(L)]
+    elif args.profile == "fp8":
+        N = K = 7168
+        KB = K // 128
+        plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_E4M3_BLOCKSCALED)
+        qbs = [inputs.e4m3_gaussian((N, K), seed=21 + i, device=dev) for i in range(3)]
+        sb = inputs.scales_log_uniform((N // 128, KB), seed=22, device=dev)
+        qa = inputs.e4m3_gaussian((M, K), seed=23, device=dev)
+        sa = inputs.scales_log_uniform((KB, ((M + 3) // 4) * 4), seed=24, device=dev)[:, :M]
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        calls = [lambda i=i: bg.bi_gemm_run(plan, qa, qbs[i % 3], C, scale_a=sa, scale_b=sb)
+                 for i in range(L)]
+    else:
+        E, N, K = 64, 2048, 7168
+        plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_BF16, E)
+        B = inputs.bf16_gaussian((E, N, K), seed=31, std=K ** -0.5, device=dev)
+        r = inputs.softmax_top8_routing(M, E, seed=32)
+        tokens = inputs.bf16_gaussian((M, K), seed=33, device=dev)
+        A = tokens[r.token_of_row.to(dev)].contiguous()
+        C = torch.empty((A.shape[0], N), dtype=torch.bfloat16, device=dev)
+        off = r.offsets.to(dev)
+        calls = [lambda: bg.bi_grouped_gemm_run(plan, A, B, C, off) for _ in range(L)]
+    for f in calls:
+        f()
+    torch.cuda.synchronize()
+    st = bg.bi_gemm_sync_status(plan, raise_on_error=False)
+    print(json.dumps({"profile": args.profile, "M": M, "launches": L, "status": st}))
+    return 0 if st == 0 else 1
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("bi_kernels.cuh", "ptx_sm100.cuh", "bi_gemm.cu"):
+        with open(os.path.join(REPO, "invariant_deterministic_gemm_bi_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
+    """The same sweep through bi_gemm_run_host: pinned host A in, kernel, host C out, per call."""
+    import torch
+    from invariant_deterministic_gemm_bi_b200 import inputs
+    steps = max(1, min(args.steps, 200))
+    A_host = inputs.bf16_gaussian((max(M_SWEEP), K_DEC), seed=77).pin_memory()
+    C_host = {m: torch.empty((m, N_DEC), dtype=torch.bfloat16).pin_memory() for m in M_SWEEP}
+    A_dev = torch.empty((max(M_SWEEP), K_DEC), dtype=torch.bfloat16, device=dev)
+    C_dev = torch.empty((max(M_SWEEP), N_DEC), dtype=torch.bfloat16, device=dev)
+    n_copies = len(Bs)
+
+    def step(s):
+        for i, m in enumerate(M_SWEEP):
+            bg.bi_gemm_run_host(plan, A_host[:m], Bs[(s * len(M_SWEEP) + i) % n_copies],
+                                C_host[m], A_dev, C_dev, stream=stream)
+
+    for s in range(3):
+        step(s)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(steps):
+        step(s)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    h2d = sum(m * K_DEC * 2 for m in M_SWEEP)
+    d2h = sum(m * N_DEC * 2 for m in M_SWEEP)
+    return {"value": sweep_bytes() * steps * world / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": ms / steps,
+            "path": "bi_gemm_run_host per GEMM (pinned host A -> device, kernel, device C -> pinned host)"}
+
+
+def graph_time_per_launch(fn_list, stream, reps=20):
+    """Capture the launches in fn_list into one graph, replay it, return seconds per launch."""
+    import torch
+    with torch.cuda.stream(stream):
+        for f in fn_list:
+            f()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for f in fn_list:
+                f()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    del g
+    return ms * 1e-3 / (reps * len(fn_list))
+
+
+def measure_per_m(bg, plan, As, Bs, Cs, dev, stream, n_copies, peaks):
+    out = []
+    for m in M_SWEEP:
+        fns = [lambda i=i: bg.bi_gemm_run(plan, As[m], Bs[i % n_copies], Cs[m], stream=stream)
+               for i in range(2 * n_copies)]
+        t = graph_time_per_launch(fns, stream)
+        b = N_DEC * K_DEC * 2 + m * K_DEC * 2 + m * N_DEC * 2
+        gbs = b / t / 1e9
+        out.append({"M": m, "us": t * 1e6, "GB/s": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                    "TFLOP/s": 2 * m * N_DEC * K_DEC / t / 1e12})
+    return out
+
+
+def measure_extras(bg, inputs, dev, stream, peaks):
+    """Prefill, FP8 and MoE workloads: throughput and roofline fraction (not part of `value`)."""
+    import torch
+    res = {}
+    bf16_peak = peaks["bf16_tflops"]
+    fp8_peak = 2.0 * bf16_peak          # nominal dense fp8 : bf16 ratio
+    hbm = peaks["hbm_gbs"]
+    # prefill, M = 16384 and 4096
+    for (N, K) in [(7168, 2048), (2048, 7168)]:
+        plan = bg.bi_gemm_plan(N, K)
+        B = inputs.bf16_gaussian((N, K), seed=3001, std=K ** -0.5, device=dev)
+        for M in [1024, 4096, 16384]:
+            A = inputs.bf16_gaussian((M, K), seed=3002, device=dev)
+            C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            t = graph_time_per_launch([lambda: bg.bi_gemm_run(plan, A, B, C, stream=stream)] * 5,
+                                      stream, reps=4)
+            tf = 2 * M * N * K / t / 1e12
+            res[f"prefill_N{N}_K{K}_M{M}"] = {"us": t * 1e6, "TFLOP/s": tf,
+                                              "tensor_frac": tf / bf16_peak}
+            del A, C
+    # FP8 N = K = 7168
+    N = K = 7168
+    KB = K // 128
+    plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_E4M3_BLOCKSCALED)
+    qbs = [inputs.e4m3_gaussian((N, K), seed=4001 + i, device=dev) for i in range(4)]
+    sb = inputs.scales_log_uniform((N // 128, KB), seed=4002, device=dev)
+    for M in [1, 64, 4096]:
+        qa = inputs.e4m3_gaussian((M, K), seed=4003, device=dev)
+        sa = inputs.scales_log_uniform((KB, ((M + 3) // 4) * 4), seed=4004, device=dev)[:, :M]
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        fns = [lambda i=i: bg.bi_gemm_run(plan, qa, qbs[i % 4], C, scale_a=sa, scale_b=sb,
+                                          stream=stream) for i in range(8)]
+        t = graph_time_per_launch(fns, stream, reps=4)
+        b = N * K + M * K + 2 * M * N + 4 * M * KB + 4 * (N // 128) * KB
+        tf = 2 * M * N * K / t / 1e12
+        res[f"fp8_M{M}"] = {"us": t * 1e6, "TFLOP/s": tf, "tensor_frac": tf / fp8_peak,
+                            "GB/s": b / t / 1e9, "hbm_frac": b / t / 1e9 / hbm}
+    del qbs
+    # MoE: 64 experts, N = 2048, K = 7168, top-8
+    E, N, K = 64, 2048, 7168
+    plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_BF16, E)
+    B = inputs.bf16_gaussian((E, N, K), seed=5001, std=K ** -0.5, device=dev)
+    for T in [1, 64, 1024, 8192]:
+        r = inputs.softmax_top8_routing(T, E, seed=5000 + T)
+        tokens = inputs.bf16_gaussian((T, K), seed=5002, device=dev)
+        A = tokens[r.token_of_row.to(dev)].contiguous()
+        C = torch.empty((A.shape[0], N), dtype=torch.bfloat16, device=dev)
+        off = r.offsets.to(dev)
+        t = graph_time_per_launch([lambda: bg.bi_grouped_gemm_run(plan, A, B, C, off, stream=stream)] * 3,
+                                  stream, reps=4)
+        active = int((r.offsets[1:] > r.offsets[:-1]).sum())
+        rows = A.shape[0]
+        b = active * N * K * 2 + rows * K * 2 + rows * N * 2
+        tf = 2 * rows * N * K / t / 1e12
+        res[f"moe_T{T}"] = {"us": t * 1e6, "TFLOP/s": tf, "tensor_frac": tf / bf16_peak,
+                            "GB/s": b / t / 1e9, "hbm_frac": b / t / 1e9 / hbm,
+                            "active_experts": active}
+    return res
+
+
+if __name__ == "__main__":
+    sys.exit(main())
