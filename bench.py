@@ -246,6 +246,9 @@ def main():
     import invariant_deterministic_gemm_bi_b200 as bg
     from invariant_deterministic_gemm_bi_b200 import inputs
 
+    global max_over_ranks
+    from invariant_deterministic_gemm_bi_b200.sharding import max_over_ranks
+
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -316,10 +319,7 @@ def main():
         raise RuntimeError(f"device status after the timed region: {bg.binding.STATUS_NAMES[st]}")
     total_ms = ev[0].elapsed_time(ev[-1])
     step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, device=dev)
 
     peaks = load_peaks()
     step_bytes = sweep_bytes()
@@ -466,12 +466,7 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
         step(s)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
     h2d = sum(m * K_DEC * 2 for m in M_SWEEP)
     d2h = sum(m * N_DEC * 2 for m in M_SWEEP)
     return {"value": sweep_bytes() * steps * world / (ms * 1e-3) / 1e9, "unit": "GB/s",

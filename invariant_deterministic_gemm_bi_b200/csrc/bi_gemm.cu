@@ -17,7 +17,7 @@
 #include <new>
 #include <vector>
 
-#include "../../include/bi_gemm.h"
+#include "bi_gemm.h"
 #include "bi_kernels.cuh"
 
 namespace {
@@ -264,6 +264,14 @@ bi_status_t check_common(const bi_plan_s *plan, int64_t rows, const void *A, int
     return BI_OK;
 }
 
+// Rows of A one TMA load brings for a dense problem of M rows: the tile's 128 rows, or, when the
+// problem is smaller than one tile, only the rows that exist (rounded up to the 8-row swizzle
+// atom).  This changes which shared-memory rows are written, not the MMA or its K order.
+int dense_a_box_rows(int64_t M)
+{
+    return M >= bi::kBlockM ? bi::kBlockM : static_cast<int>((M + 7) / 8 * 8);
+}
+
 GemmParams base_params(const bi_plan_s *plan, int64_t rows, void *C, int64_t ldc, int *status)
 {
     GemmParams p;
@@ -277,6 +285,7 @@ GemmParams base_params(const bi_plan_s *plan, int64_t rows, void *C, int64_t ldc
     p.num_m_blocks = static_cast<int32_t>((rows + bi::kBlockM - 1) / bi::kBlockM);
     p.num_experts = plan->experts;
     p.raster_m = 16;
+    p.a_box_rows = bi::kBlockM;
     p.c = static_cast<__nv_bfloat16 *>(C);
     p.ldc = ldc;
     p.kb_scale = static_cast<int32_t>((plan->k + 127) / 128);
@@ -454,11 +463,13 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
     if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
         return st;
     CUtensorMap ta, tb;
-    if ((st = encode_2d(&ta, A, fp8, plan->k, M, lda, bi::kBlockM)) != BI_OK)
+    const int a_rows = dense_a_box_rows(M);
+    if ((st = encode_2d(&ta, A, fp8, plan->k, M, lda, a_rows)) != BI_OK)
         return st;
     if ((st = encode_2d(&tb, B, fp8, plan->k, plan->n, ldb, plan->kernel->bn)) != BI_OK)
         return st;
     GemmParams p = base_params(plan, M, C, ldc, status);
+    p.a_box_rows = a_rows;
     p.scale_a = scale_a;
     p.ld_sa = ld_sa;
     p.scale_b = scale_b;

@@ -9,7 +9,10 @@
 // K-slices of the tile in ascending order into one TMEM accumulator (no split-K, no atomics,
 // no cross-CTA reduction).  The tile shape, the MMA instruction shape and the K order are
 // template constants chosen by the host plan from (N, K, dtype) only.  Rows past the end of A
-// are zero-filled by TMA and never stored.  The CTA <-> tile mapping does depend on M, which is
+// are zero-filled by TMA and never stored.  When the whole problem has fewer than 128 rows,
+// TMA brings only the first roundup(M, 8) rows of the A tile; the MMA still runs on all 128
+// rows, and the rows never loaded feed only output rows that are never stored (every output
+// element depends on its own A row alone).  The CTA <-> tile mapping does depend on M, which is
 // harmless: it decides where a tile is computed, not how.
 //
 // Roles inside a CTA (6 warps = 192 threads):
@@ -58,6 +61,7 @@ struct GemmParams {
     int32_t num_m_blocks;    // dense: ceil(M / 128)
     int32_t num_experts;     // grouped: E
     int32_t raster_m;        // dense raster band height in m-blocks
+    int32_t a_box_rows;      // rows of A one TMA load brings (<= 128, a multiple of 8)
     __nv_bfloat16 *c;
     int64_t ldc;
     const float *scale_a;    // FP8: [kb][ld_sa]
@@ -309,7 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (skip_next) {
                         skip_next = false;   // fault injection: this stage is never filled
                     } else {
-                        ptx::mbar_arrive_expect_tx(&full_bar[stage], L::kStageBytes);
+                        ptx::mbar_arrive_expect_tx(&full_bar[stage],
+                                                   (p.a_box_rows + BN) * kRowBytes);
                         ptx::tma_load_2d(smem_a + stage * L::kABytes, &tmap_a, &full_bar[stage],
                                          kb * kElemsPerRow, tc.m0, pol_a);
                         ptx::tma_load_2d(smem_b + stage * L::kBBytes, &tmap_b, &full_bar[stage],

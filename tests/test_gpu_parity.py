@@ -255,3 +255,17 @@ def test_grouped_full_size_sampled_rows(T):
         rows = sorted({int(off[e]), int(off[e + 1] - 1)})
         cref, _ = oracle.gemm_bf16(inputs.to_numpy_bits(A[rows]), inputs.to_numpy_bits(B[e]))
         parity.assert_within_tolerance(Cb[rows], cref, K, rms_a, rms_b, f"moe T={T} e={e}")
+
+
+def test_run_host_matches_device_run():
+    M, N, K = 100, 256, 512
+    plan = bg.bi_gemm_plan(N, K)
+    A = inputs.bf16_integers((M, K), seed=6001).pin_memory()
+    B = inputs.bf16_integers((N, K), seed=6002, device=DEV)
+    C_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    A_dev = torch.empty((M, K), dtype=torch.bfloat16, device=DEV)
+    C_dev = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    bg.bi_gemm_run_host(plan, A, B, C_host, A_dev, C_dev)
+    bg.bi_gemm_sync_status(plan)
+    _, want = oracle.gemm_bf16(inputs.to_numpy_bits(A), inputs.to_numpy_bits(B))
+    parity.assert_bits_equal_values(parity.bits(C_host), want, "run_host")
