@@ -169,6 +169,41 @@ bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M,
                              cudaStream_t stream);
 
 /*
+ * Dense GEMM from host memory for callers that must not allocate device memory.
+ *
+ * Some callers cannot call cudaMalloc: their device memory is owned by another allocator (a
+ * framework's caching allocator or an inference server's arena that has reserved the GPU), so
+ * a stray allocation fails or breaks the owner's accounting, or they run where allocating after
+ * start-up is not allowed.  This entry point does what bi_gemm_run_host does, but it takes no
+ * device staging buffers and allocates nothing: the device copies of A, scale_a and C and the
+ * kernel's status word live in one file-scope device array of BI_NOALLOC_SCRATCH_BYTES (8 MiB),
+ * which every GPU that loads the library holds until the process exits.  The paper has no
+ * counterpart to this entry point.
+ *
+ * Sizes: the call needs 256 bytes for the status word plus M*lda*elt (A), M*ldc*2 (C) and, for
+ * FP8, ceil(K/128)*ld_sa*4 (scale_a) bytes, each rounded up to 256; a call that needs more than
+ * BI_NOALLOC_SCRATCH_BYTES returns BI_ERR_UNSUPPORTED_SHAPE before touching the device.  (The
+ * decode shape N = 4096, K = 7168 in bf16 fits up to M = 372 rows.)
+ * Behaviour: copies A (and scale_a) in, runs the GEMM, copies C out, then synchronises `stream`
+ * and returns the kernel's status (BI_OK or BI_ERR_DEVICE_TIMEOUT), so C_host is ready on
+ * return.  B and scale_b are device pointers (resident weights).  The status word is cleared
+ * before every launch.  All calls share the one array and it keeps the last call's contents:
+ * calls that overlap on the GPU (from several host threads or streams) race on it and must be
+ * serialised by the caller.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before any stream
+ * capture.  Dense plans only (a grouped plan returns BI_ERR_INVALID_ARG).
+ * Errors: as bi_gemm_run_host, plus BI_ERR_UNSUPPORTED_SHAPE when the scratch is too small.
+ */
+#define BI_NOALLOC_SCRATCH_BYTES (8u << 20)
+bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M,
+                                     const void *A_host, int64_t lda,
+                                     const void *B, int64_t ldb,
+                                     void *C_host, int64_t ldc,
+                                     const float *scale_a_host, int64_t ld_sa,
+                                     const float *scale_b,
+                                     cudaStream_t stream);
+
+/*
  * Synchronise `stream`, then read and clear the plan's device status word for the current
  * device.  Returns BI_OK, BI_ERR_DEVICE_TIMEOUT, BI_ERR_BAD_OFFSETS or BI_ERR_CUDA.  All runs
  * of one plan on one device share the status word.

@@ -20,6 +20,7 @@ from .binding import (  # noqa: F401
     bi_gemm_plan_destroy,
     bi_gemm_run,
     bi_gemm_run_host,
+    bi_gemm_run_host_noalloc,
     bi_gemm_set_wait_timeout,
     bi_gemm_sync_status,
     bi_grouped_gemm_run,

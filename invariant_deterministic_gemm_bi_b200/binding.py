@@ -31,6 +31,7 @@ EXPORTED = [
     "bi_gemm_abi_version", "bi_status_string", "bi_gemm_plan", "bi_gemm_plan_destroy",
     "bi_gemm_plan_describe", "bi_gemm_run", "bi_grouped_gemm_run", "bi_gemm_run_host",
     "bi_gemm_sync_status", "bi_gemm_set_wait_timeout", "bi_gemm_debug_set_flags",
+    "bi_gemm_run_host_noalloc",
 ]
 
 
@@ -84,6 +85,8 @@ def load_library(path: str = LIB_PATH):
     lib.bi_grouped_gemm_run.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, vp]
     lib.bi_gemm_run_host.restype = i32
     lib.bi_gemm_run_host.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, i64, vp, vp, vp, vp, vp]
+    lib.bi_gemm_run_host_noalloc.restype = i32
+    lib.bi_gemm_run_host_noalloc.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, i64, vp, vp]
     lib.bi_gemm_sync_status.restype = i32
     lib.bi_gemm_sync_status.argtypes = [vp, vp]
     lib.bi_gemm_set_wait_timeout.restype = i32
@@ -200,6 +203,20 @@ def bi_gemm_run_host(plan: Plan, A_host, B, C_host, A_dev, C_dev, scale_a_host=N
                                          _ptr(scale_a_host), ld_sa, _ptr(scale_b), _ptr(A_dev),
                                          _ptr(C_dev), _ptr(scale_a_dev), _stream_handle(stream))
     _check(st, "bi_gemm_run_host")
+    return C_host
+
+
+def bi_gemm_run_host_noalloc(plan: Plan, A_host, B, C_host, scale_a_host=None, scale_b=None,
+                             stream=None):
+    """Host-memory variant that allocates no device memory: staging copies live in the
+    library's static device scratch.  Synchronous: C_host holds the result on return."""
+    M = A_host.shape[0]
+    ld_sa = scale_a_host.stride(0) if scale_a_host is not None else 0
+    st = load_library().bi_gemm_run_host_noalloc(plan.handle, M, _ptr(A_host), A_host.stride(0),
+                                                 _ptr(B), B.stride(0), _ptr(C_host),
+                                                 C_host.stride(0), _ptr(scale_a_host), ld_sa,
+                                                 _ptr(scale_b), _stream_handle(stream))
+    _check(st, "bi_gemm_run_host_noalloc")
     return C_host
 
 

@@ -307,6 +307,38 @@ bi_status_t launch_main(const bi_plan_s *plan, const CUtensorMap &ta, const CUte
 } // namespace
 
 // ---------------------------------------------------------------------------------------------
+// Static device scratch for bi_gemm_run_host_noalloc: status word + staging copies of A,
+// scale_a and C.  Host code must not use the symbol as an address: it looks the device address
+// up once per device with cudaGetSymbolAddress (the device current) and passes that pointer.
+// ---------------------------------------------------------------------------------------------
+
+static __device__ __align__(256) unsigned char bi_noalloc_scratch[BI_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+unsigned char *g_noalloc_ptr[kMaxDevices] = {};
+
+bi_status_t noalloc_scratch_for(int dev, unsigned char **out)
+{
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, bi_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return BI_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = static_cast<unsigned char *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return BI_OK;
+}
+
+constexpr int64_t round256(int64_t x) { return (x + 255) / 256 * 256; }
+
+} // namespace
+
+// ---------------------------------------------------------------------------------------------
 // extern "C" ABI
 // ---------------------------------------------------------------------------------------------
 
@@ -556,6 +588,94 @@ bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M, const void *A_host, int6
                         stream) != cudaSuccess)
         return BI_ERR_CUDA;
     return BI_OK;
+}
+
+bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_host, int64_t lda,
+                                     const void *B, int64_t ldb, void *C_host, int64_t ldc,
+                                     const float *scale_a_host, int64_t ld_sa,
+                                     const float *scale_b, cudaStream_t stream)
+{
+    if (!plan)
+        return BI_ERR_INVALID_ARG;
+    if (plan->experts != 1 || M < 0)
+        return BI_ERR_INVALID_ARG;
+    if (M == 0 || plan->n == 0)
+        return BI_OK;
+    const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
+    const int elt = fp8 ? 1 : 2;
+    if (!C_host || (plan->k > 0 && !A_host))
+        return BI_ERR_INVALID_ARG;
+    if (fp8 && plan->k > 0) {
+        if (!scale_a_host || !scale_b)
+            return BI_ERR_DTYPE_MISMATCH;
+        if (ld_sa < M)
+            return BI_ERR_INVALID_ARG;
+    } else if (!fp8 && (scale_a_host || scale_b)) {
+        return BI_ERR_DTYPE_MISMATCH;
+    }
+    if (lda < plan->k || ldc < plan->n || (fp8 && ld_sa < 0))
+        return BI_ERR_INVALID_ARG;
+    // Scratch layout: [status word | A | C | scale_a], each part 256-byte aligned.
+    const int64_t kb = (plan->k + 127) / 128;
+    const int64_t a_off = 256;
+    const int64_t c_off = a_off + round256(M * lda * elt);
+    const int64_t s_off = c_off + round256(M * ldc * 2);
+    const int64_t need = s_off + (fp8 ? round256(kb * ld_sa * 4) : 0);
+    if (need > static_cast<int64_t>(BI_NOALLOC_SCRATCH_BYTES))
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    int dev = 0;
+    DeviceInfo *d = nullptr;
+    bi_status_t st = current_device(&dev, &d);
+    if (st != BI_OK)
+        return st;
+    unsigned char *base = nullptr;
+    if ((st = noalloc_scratch_for(dev, &base)) != BI_OK)
+        return st;
+    int *status = reinterpret_cast<int *>(base);
+    void *A_dev = base + a_off;
+    void *C_dev = base + c_off;
+    float *sa_dev = reinterpret_cast<float *>(base + s_off);
+    if ((st = check_common(plan, M, A_dev, lda, B, ldb, C_dev, ldc)) != BI_OK)
+        return st;
+    if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess)
+        return BI_ERR_CUDA;
+    if (plan->k == 0) {
+        if ((st = launch_zero(C_dev, ldc, M, plan->n, stream)) != BI_OK)
+            return st;
+    } else {
+        if (cudaMemcpyAsync(A_dev, A_host, static_cast<size_t>(M * lda * elt),
+                            cudaMemcpyHostToDevice, stream) != cudaSuccess)
+            return BI_ERR_CUDA;
+        if (fp8 && cudaMemcpyAsync(sa_dev, scale_a_host, static_cast<size_t>(kb * ld_sa * 4),
+                                   cudaMemcpyHostToDevice, stream) != cudaSuccess)
+            return BI_ERR_CUDA;
+        if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
+            return st;
+        CUtensorMap ta, tb;
+        const int a_rows = dense_a_box_rows(M);
+        if ((st = encode_2d(&ta, A_dev, fp8, plan->k, M, lda, a_rows)) != BI_OK)
+            return st;
+        if ((st = encode_2d(&tb, B, fp8, plan->k, plan->n, ldb, plan->kernel->bn)) != BI_OK)
+            return st;
+        GemmParams p = base_params(plan, M, C_dev, ldc, status);
+        p.a_box_rows = a_rows;
+        p.scale_a = fp8 ? sa_dev : nullptr;
+        p.ld_sa = fp8 ? ld_sa : 0;
+        p.scale_b = fp8 ? scale_b : nullptr;
+        const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
+        const int grid = static_cast<int>(tiles < d->num_sms ? tiles : d->num_sms);
+        if ((st = launch_main(plan, ta, tb, p, grid, stream)) != BI_OK)
+            return st;
+    }
+    if (cudaMemcpyAsync(C_host, C_dev, static_cast<size_t>(M * ldc * 2), cudaMemcpyDeviceToHost,
+                        stream) != cudaSuccess)
+        return BI_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess)
+        return BI_ERR_CUDA;
+    int host = 0;
+    if (cudaMemcpy(&host, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return BI_ERR_CUDA;
+    return host == 0 ? BI_OK : static_cast<bi_status_t>(host);
 }
 
 bi_status_t bi_gemm_sync_status(bi_plan_t plan, cudaStream_t stream)
