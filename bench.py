@@ -331,7 +331,7 @@ def main():
     achieved = step_bytes / launches / avg_launch_s / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                "peak_source": peaks["source"], "kernel": "bi_gemm_kernel<32,10,bf16>",
+                "peak_source": peaks["source"], "kernel": kernel_label(bg, plan),
                 "note": "per-launch time = step time / 9 (graph gaps included)"}
     traffic = os.path.join(REPO, "profiles", "decode_bf16_traffic.json")
     if os.path.exists(traffic):
@@ -429,6 +429,12 @@ def profile_case(args):
     st = bg.bi_gemm_sync_status(plan, raise_on_error=False)
     print(json.dumps({"profile": args.profile, "M": M, "launches": L, "status": st}))
     return 0 if st == 0 else 1
+
+
+def kernel_label(bg, plan) -> str:
+    i = bg.bi_gemm_plan_describe(plan)
+    return (f"bi_gemm_kernel<BM={i['block_m']},BN={i['block_n']},{'e4m3' if i['dtype'] else 'bf16'}>"
+            f" rings A{i['stages_a']}/B{i['stages']}")
 
 
 def kernel_source_hash() -> str:

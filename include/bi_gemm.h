@@ -72,21 +72,24 @@ typedef enum {
 /* Opaque, library-owned plan. */
 typedef struct bi_plan_s *bi_plan_t;
 
-/* What a plan fixed.  None of it depends on M. */
+/* What a plan fixed.  None of it depends on M, except the two ring depths, which are reported
+ * for a full-height tile: a launch whose whole problem has fewer rows than one tile sizes its A
+ * slots to those rows and deepens both rings (scheduling only; the MMA and K order are fixed). */
 typedef struct {
     int64_t n, k;              /* the plan's N and K */
     int dtype;                 /* bi_dtype_t */
     int num_experts;           /* 1 = dense */
     int block_m;               /* output rows per tile */
     int block_n;               /* output columns per tile */
-    int block_k;               /* K elements per pipeline stage (128 bytes) */
+    int block_k;               /* K elements per pipeline stage (1, 2 or 4 chunks of 128 bytes) */
     int cta_group;             /* CTAs that share one MMA (1 or 2) */
     int mma_m, mma_n, mma_k;   /* tcgen05.mma instruction shape */
-    int stages;                /* shared-memory pipeline depth */
+    int stages;                /* depth of the B (weight) shared-memory ring */
     int k_order_id;            /* 0 = ascending K blocks, whole K per CTA, no split-K */
     int threads_per_cta;
     int smem_bytes;            /* dynamic shared memory per CTA */
     int tmem_columns;          /* tensor-memory columns allocated per CTA */
+    int stages_a;              /* depth of the A shared-memory ring (<= stages) */
 } bi_plan_info_t;
 
 /* Library version check: returns BI_GEMM_ABI_VERSION. */
@@ -212,7 +215,9 @@ bi_status_t bi_gemm_sync_status(bi_plan_t plan, cudaStream_t stream);
 
 /*
  * Set the time limit, in nanoseconds, of every device-side pipeline wait of this plan's
- * kernels (default 2e9, i.e. 2 s; 0 restores the default).  A wait that runs out sets
+ * kernels (default 2e9, i.e. 2 s; 0 restores the default).  The device counts the limit in SM
+ * clock cycles at 2 cycles per ns, at or above the highest B200 SM clock, so a wait lasts at least
+ * timeout_ns (longer when the clock runs lower).  A wait that runs out sets
  * BI_ERR_DEVICE_TIMEOUT, lets the CTA drain its own copies in flight, frees its tensor memory
  * and returns, so the context stays usable.
  */

@@ -50,6 +50,7 @@ class PlanInfo(ctypes.Structure):
         ("mma_n", ctypes.c_int), ("mma_k", ctypes.c_int), ("stages", ctypes.c_int),
         ("k_order_id", ctypes.c_int), ("threads_per_cta", ctypes.c_int),
         ("smem_bytes", ctypes.c_int), ("tmem_columns", ctypes.c_int),
+        ("stages_a", ctypes.c_int),
     ]
 
     def as_dict(self):

@@ -32,67 +32,123 @@ typedef void (*KernelFn)(const __grid_constant__ CUtensorMap, const __grid_const
                          const GemmParams);
 
 struct KernelEntry {
+    int bm;
     int bn;
-    int stages;
+    int kc;
     bool fp8;
     bool grouped;
     KernelFn fn;
     int smem;
 };
 
-#define BI_ENTRY(BN, ST, F8, GR)                                                                   \
-    KernelEntry{BN, ST, F8, GR, &bi::bi_gemm_kernel<BN, ST, F8, GR>,                               \
-                bi::smem_bytes_for<BN, ST, F8, GR>()}
+#define BI_ENTRY(BM, BN, KC, F8, GR)                                                               \
+    KernelEntry{BM, BN, KC, F8, GR, &bi::bi_gemm_kernel<BM, BN, KC, F8, GR>,                        \
+                bi::smem_bytes_for<BM, BN, KC, F8, GR>()}
 
-// Pipeline depth: as many stages as fit in ~200 KB of shared memory.
+// Every (BM, BN) tile in two forms: the tile's preferred number of 128-byte K chunks per
+// pipeline stage (3-D TMA boxes; needs K to be a multiple of the chunk), and one chunk per stage
+// for any other K.  Narrow tiles take more chunks per stage so that one weight box is ~16 KB.
 const KernelEntry kKernels[] = {
-    BI_ENTRY(32, 10, false, false),  BI_ENTRY(64, 8, false, false),
-    BI_ENTRY(128, 6, false, false),  BI_ENTRY(256, 4, false, false),
-    BI_ENTRY(32, 10, true, false),   BI_ENTRY(64, 8, true, false),
-    BI_ENTRY(128, 6, true, false),   BI_ENTRY(32, 10, false, true),
-    BI_ENTRY(64, 8, false, true),    BI_ENTRY(128, 6, false, true),
-    BI_ENTRY(256, 4, false, true),
+    BI_ENTRY(64, 32, 1, false, false),   BI_ENTRY(64, 32, 4, false, false),
+    BI_ENTRY(128, 32, 1, false, false),  BI_ENTRY(128, 32, 4, false, false),
+    BI_ENTRY(128, 64, 1, false, false),  BI_ENTRY(128, 64, 2, false, false),
+    BI_ENTRY(128, 128, 1, false, false), BI_ENTRY(128, 128, 2, false, false),
+    BI_ENTRY(128, 256, 1, false, false),
+    BI_ENTRY(128, 32, 1, true, false),   BI_ENTRY(128, 32, 4, true, false),
+    BI_ENTRY(128, 64, 1, true, false),   BI_ENTRY(128, 64, 2, true, false),
+    BI_ENTRY(128, 128, 1, true, false),  BI_ENTRY(128, 128, 2, true, false),
+    BI_ENTRY(128, 32, 1, false, true),   BI_ENTRY(128, 32, 4, false, true),
+    BI_ENTRY(128, 64, 1, false, true),   BI_ENTRY(128, 64, 2, false, true),
+    BI_ENTRY(128, 128, 1, false, true),  BI_ENTRY(128, 128, 2, false, true),
+    BI_ENTRY(128, 256, 1, false, true),
 };
 constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
 
-const KernelEntry *find_kernel(int bn, bool fp8, bool grouped)
+int preferred_chunks(int bn) { return bn <= 32 ? 4 : bn >= 256 ? 1 : 2; }
+
+const KernelEntry *find_kernel(int bm, int bn, int kc, bool fp8, bool grouped)
 {
     for (int i = 0; i < kNumKernels; ++i)
-        if (kKernels[i].bn == bn && kKernels[i].fp8 == fp8 && kKernels[i].grouped == grouped)
+        if (kKernels[i].bm == bm && kKernels[i].bn == bn && kKernels[i].kc == kc &&
+            kKernels[i].fp8 == fp8 && kKernels[i].grouped == grouped)
             return &kKernels[i];
     return nullptr;
+}
+
+// Ring geometry of one launch (see bi::Rings): A slots hold the a_rows rows TMA brings; wide
+// tiles give A and B the same depth, narrow ones keep up to ~96 KB for A and the rest for B.
+struct RingGeom {
+    int sa, sb;
+    uint32_t a_stride, b_offset;
+};
+
+RingGeom ring_geometry(const KernelEntry *k, int a_rows)
+{
+    const int chunk = bi::kRowBytes;
+    const int a_stride = k->kc * a_rows * chunk;
+    const int over = (k->bm - a_rows) * chunk;     // the MMA reads BM rows from each A chunk
+    const int b_stride = k->kc * k->bn * chunk;
+    int sa, sb, a_region;
+    if (k->bn >= 128) {
+        sa = (bi::kRingBytes - over) / (a_stride + b_stride);
+        if (sa > bi::kMaxSA)
+            sa = bi::kMaxSA;
+        sb = sa;
+        a_region = (sa * a_stride + over + 1023) / 1024 * 1024;
+        if (a_region + sb * b_stride > bi::kRingBytes)
+            --sa, --sb, a_region = (sa * a_stride + over + 1023) / 1024 * 1024;
+    } else {
+        sa = (96 * 1024 - over) / a_stride;
+        sa = sa < 2 ? 2 : sa > bi::kMaxSA ? bi::kMaxSA : sa;
+        for (;; --sa) {   // deepest A ring that still leaves B at least as deep
+            a_region = (sa * a_stride + over + 1023) / 1024 * 1024;
+            sb = (bi::kRingBytes - a_region) / b_stride;
+            if (sb > bi::kMaxSB)
+                sb = bi::kMaxSB;
+            if (sb >= sa || sa == 2)
+                break;
+        }
+    }
+    // The kernel relies on 2 <= sa <= sb (the A-slot reuse test reads the consumed ring) and, for
+    // FP8, on sb groups outlasting the partial-product ring.  Every tile in kKernels satisfies
+    // this for every a_rows in [8, BM]; tests/test_abi.py checks the reported depths.
+    return RingGeom{sa, sb, static_cast<uint32_t>(a_stride), static_cast<uint32_t>(a_region)};
 }
 
 // ---------------------------------------------------------------------------------------------
 // Plan table
 // ---------------------------------------------------------------------------------------------
 
-// The output-tile width BN for (N, K, dtype).  Known projection shapes get the width tuned for
-// them; any other shape takes the widest BN that still gives >= 100 tiles at M <= 128, since
-// without split-K the N tiles are the only parallelism a small batch has.  A grouped plan uses
-// the dense plan's width for the same (N, K), so a row of an expert's segment gets the bits a
+// The tile (BM x BN) for (N, K, dtype).  Known projection shapes get the tile tuned for them;
+// any other shape takes BM = 128 and the widest BN that still gives >= 100 tiles at M <= 128,
+// since without split-K the N tiles are the only parallelism a small batch has.  A grouped plan
+// uses the dense plan's tile for the same (N, K), so a row of an expert's segment gets the bits a
 // dense call with that expert's weights would give it.
-int choose_block_n(int64_t N, int64_t K, bi_dtype_t dtype)
+struct TileChoice {
+    int bm, bn;
+};
+
+TileChoice choose_tile(int64_t N, int64_t K, bi_dtype_t dtype)
 {
     struct Row {
         int64_t n, k;
-        int dtype, bn;
+        int dtype, bm, bn;
     };
     static const Row table[] = {
-        {4096, 7168, BI_DTYPE_BF16, 32},               // decode-shaped projection
-        {7168, 2048, BI_DTYPE_BF16, 256},              // prefill-shaped, wide N
-        {2048, 7168, BI_DTYPE_BF16, 128},              // prefill-shaped, long K; MoE experts
-        {256, 512, BI_DTYPE_BF16, 32},                 // small correctness shape
-        {7168, 7168, BI_DTYPE_E4M3_BLOCKSCALED, 64},   // FP8 projection
+        {4096, 7168, BI_DTYPE_BF16, 128, 32},              // decode-shaped projection
+        {7168, 2048, BI_DTYPE_BF16, 128, 256},             // prefill-shaped, wide N
+        {2048, 7168, BI_DTYPE_BF16, 128, 128},             // prefill-shaped, long K; MoE experts
+        {256, 512, BI_DTYPE_BF16, 128, 32},                // small correctness shape
+        {7168, 7168, BI_DTYPE_E4M3_BLOCKSCALED, 128, 64},  // FP8 projection
     };
     for (const Row &r : table)
         if (r.n == N && r.k == K && r.dtype == dtype)
-            return r.bn;
+            return {r.bm, r.bn};
     const int max_bn = dtype == BI_DTYPE_E4M3_BLOCKSCALED ? 128 : 256;
     for (int bn = max_bn; bn > 32; bn /= 2)
         if ((N + bn - 1) / bn >= 100)
-            return bn;
-    return 32;
+            return {128, bn};
+    return {128, 32};
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -194,19 +250,37 @@ bi_status_t plan_status_word(bi_plan_s *plan, int dev, int **out)
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bi_status_t encode_2d(CUtensorMap *map, const void *base, bool fp8, int64_t inner, int64_t rows,
-                      int64_t ld_elems, int box_rows)
+// TMA map of a K-major operand [rows][ld] with 128-byte rows per box, 128-byte swizzle.
+// kc == 1: 2-D, box {128 B of K, box_rows}.  kc > 1: 3-D view [K/chunk][rows][chunk] (the chunk
+// index has a 128-byte stride), box {chunk, box_rows, kc}, which lands in shared memory as kc
+// consecutive [box_rows x 128 B] tiles; it needs K to be a multiple of the chunk.
+bi_status_t encode_operand(CUtensorMap *map, const void *base, bool fp8, int64_t K, int64_t rows,
+                           int64_t ld_elems, int box_rows, int kc)
 {
     const int elt = fp8 ? 1 : 2;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_elems * elt)};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(bi::kRowBytes / elt),
-                         static_cast<cuuint32_t>(box_rows)};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                          2, const_cast<void *>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const int chunk = bi::kRowBytes / elt;
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r;
+    if (kc == 1) {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_elems * elt)};
+        cuuint32_t box[2] = {static_cast<cuuint32_t>(chunk), static_cast<cuuint32_t>(box_rows)};
+        r = g_encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        cuuint64_t dims[3] = {static_cast<cuuint64_t>(chunk), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(K / chunk)};
+        cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld_elems * elt),
+                                 static_cast<cuuint64_t>(bi::kRowBytes)};
+        cuuint32_t box[3] = {static_cast<cuuint32_t>(chunk), static_cast<cuuint32_t>(box_rows),
+                             static_cast<cuuint32_t>(kc)};
+        r = g_encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                     const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
     return r == CUDA_SUCCESS ? BI_OK : BI_ERR_CUDA;
 }
 
@@ -267,9 +341,20 @@ bi_status_t check_common(const bi_plan_s *plan, int64_t rows, const void *A, int
 // Rows of A one TMA load brings for a dense problem of M rows: the tile's 128 rows, or, when the
 // problem is smaller than one tile, only the rows that exist (rounded up to the 8-row swizzle
 // atom).  This changes which shared-memory rows are written, not the MMA or its K order.
-int dense_a_box_rows(int64_t M)
+int dense_a_box_rows(int64_t M, int bm)
 {
-    return M >= bi::kBlockM ? bi::kBlockM : static_cast<int>((M + 7) / 8 * 8);
+    return M >= bm ? bm : static_cast<int>((M + 7) / 8 * 8);
+}
+
+bool set_rows(GemmParams *p, const bi_plan_s *plan, int a_rows)
+{
+    const RingGeom g = ring_geometry(plan->kernel, a_rows);
+    p->a_box_rows = a_rows;
+    p->sa = g.sa;
+    p->sb = g.sb;
+    p->a_stride = g.a_stride;
+    p->b_offset = g.b_offset;
+    return g.sa >= 2 && g.sa <= g.sb && g.sa <= bi::kMaxSA && g.sb <= bi::kMaxSB;
 }
 
 GemmParams base_params(const bi_plan_s *plan, int64_t rows, void *C, int64_t ldc, int *status)
@@ -282,15 +367,17 @@ GemmParams base_params(const bi_plan_s *plan, int64_t rows, void *C, int64_t ldc
     p.k = static_cast<int32_t>(plan->k);
     p.num_k_blocks = static_cast<int32_t>((plan->k * elt + bi::kRowBytes - 1) / bi::kRowBytes);
     p.num_n_blocks = static_cast<int32_t>((plan->n + plan->kernel->bn - 1) / plan->kernel->bn);
-    p.num_m_blocks = static_cast<int32_t>((rows + bi::kBlockM - 1) / bi::kBlockM);
+    p.num_m_blocks = static_cast<int32_t>((rows + plan->kernel->bm - 1) / plan->kernel->bm);
     p.num_experts = plan->experts;
     p.raster_m = 16;
-    p.a_box_rows = bi::kBlockM;
+    (void)set_rows(&p, plan, plan->kernel->bm);
     p.c = static_cast<__nv_bfloat16 *>(C);
     p.ldc = ldc;
     p.kb_scale = static_cast<int32_t>((plan->k + 127) / 128);
     p.status = status;
-    p.timeout_ns = plan->timeout_ns;
+    // the wait limit is counted in SM cycles; 2 cycles per ns is at or above the B200's highest
+    // SM clock (1965 MHz), so a wait lasts at least timeout_ns
+    p.timeout_cycles = plan->timeout_ns * 2;
     p.debug_flags = plan->debug_flags;
     return p;
 }
@@ -378,8 +465,10 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     if (N > INT32_MAX / 2 || K > INT32_MAX / 2 || N * num_experts > INT32_MAX / 2)
         return BI_ERR_UNSUPPORTED_SHAPE;
     const bool fp8 = dtype == BI_DTYPE_E4M3_BLOCKSCALED;
-    const int bn = choose_block_n(N, K, dtype);
-    const KernelEntry *k = find_kernel(bn, fp8, num_experts > 1);
+    const TileChoice tile = choose_tile(N, K, dtype);
+    const int chunk_elems = fp8 ? 128 : 64;
+    const int kc = (K > 0 && K % chunk_elems == 0) ? preferred_chunks(tile.bn) : 1;
+    const KernelEntry *k = find_kernel(tile.bm, tile.bn, kc, fp8, num_experts > 1);
     if (!k)
         return BI_ERR_UNSUPPORTED_SHAPE;
     bi_plan_s *p = new (std::nothrow) bi_plan_s();
@@ -424,18 +513,20 @@ bi_status_t bi_gemm_plan_describe(bi_plan_t plan, bi_plan_info_t *info)
     info->k = plan->k;
     info->dtype = plan->dtype;
     info->num_experts = plan->experts;
-    info->block_m = bi::kBlockM;
+    info->block_m = plan->kernel->bm;
     info->block_n = plan->kernel->bn;
-    info->block_k = fp8 ? 128 : 64;
+    info->block_k = (fp8 ? 128 : 64) * plan->kernel->kc;
     info->cta_group = 1;
-    info->mma_m = bi::kBlockM;
+    info->mma_m = plan->kernel->bm;
     info->mma_n = plan->kernel->bn;
     info->mma_k = fp8 ? 32 : 16;
-    info->stages = plan->kernel->stages;
+    const RingGeom g = ring_geometry(plan->kernel, plan->kernel->bm);
+    info->stages = g.sb;
+    info->stages_a = g.sa;
     info->k_order_id = 0;
     info->threads_per_cta = bi::kThreads;
     info->smem_bytes = plan->kernel->smem;
-    const int nacc = fp8 ? ((512 / plan->kernel->bn) < 4 ? (512 / plan->kernel->bn) : 4) : 2;
+    const int nacc = fp8 ? ((512 / plan->kernel->bn) < 8 ? (512 / plan->kernel->bn) : 8) : 2;
     int cols = 32;
     while (cols < nacc * plan->kernel->bn)
         cols *= 2;
@@ -495,13 +586,14 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
     if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
         return st;
     CUtensorMap ta, tb;
-    const int a_rows = dense_a_box_rows(M);
-    if ((st = encode_2d(&ta, A, fp8, plan->k, M, lda, a_rows)) != BI_OK)
+    const int a_rows = dense_a_box_rows(M, plan->kernel->bm);
+    if ((st = encode_operand(&ta, A, fp8, plan->k, M, lda, a_rows, plan->kernel->kc)) != BI_OK)
         return st;
-    if ((st = encode_2d(&tb, B, fp8, plan->k, plan->n, ldb, plan->kernel->bn)) != BI_OK)
+    if ((st = encode_operand(&tb, B, fp8, plan->k, plan->n, ldb, plan->kernel->bn, plan->kernel->kc)) != BI_OK)
         return st;
     GemmParams p = base_params(plan, M, C, ldc, status);
-    p.a_box_rows = a_rows;
+    if (!set_rows(&p, plan, a_rows))
+        return BI_ERR_UNSUPPORTED_SHAPE;
     p.scale_a = scale_a;
     p.ld_sa = ld_sa;
     p.scale_b = scale_b;
@@ -537,15 +629,15 @@ bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *
     if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
         return st;
     CUtensorMap ta, tb;
-    if ((st = encode_2d(&ta, A, false, plan->k, total_rows, lda, bi::kBlockM)) != BI_OK)
+    if ((st = encode_operand(&ta, A, false, plan->k, total_rows, lda, plan->kernel->bm, plan->kernel->kc)) != BI_OK)
         return st;
-    if ((st = encode_2d(&tb, B, false, plan->k, plan->n * plan->experts, ldb, plan->kernel->bn)) != BI_OK)
+    if ((st = encode_operand(&tb, B, false, plan->k, plan->n * plan->experts, ldb, plan->kernel->bn, plan->kernel->kc)) != BI_OK)
         return st;
     GemmParams p = base_params(plan, total_rows, C, ldc, status);
     p.offsets = expert_offsets;
-    // Upper bound on the tile count without reading the offsets: sum_e ceil(len_e/128) is at
-    // most total_rows/128 + E.
-    const int64_t max_tiles = (total_rows / bi::kBlockM + plan->experts) * p.num_n_blocks;
+    // Upper bound on the tile count without reading the offsets: sum_e ceil(len_e/BM) is at
+    // most total_rows/BM + E.
+    const int64_t max_tiles = (total_rows / plan->kernel->bm + plan->experts) * p.num_n_blocks;
     const int grid = static_cast<int>(max_tiles < d->num_sms ? max_tiles : d->num_sms);
     return launch_main(plan, ta, tb, p, grid, stream);
 }
@@ -652,13 +744,14 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
         if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
             return st;
         CUtensorMap ta, tb;
-        const int a_rows = dense_a_box_rows(M);
-        if ((st = encode_2d(&ta, A_dev, fp8, plan->k, M, lda, a_rows)) != BI_OK)
+        const int a_rows = dense_a_box_rows(M, plan->kernel->bm);
+        if ((st = encode_operand(&ta, A_dev, fp8, plan->k, M, lda, a_rows, plan->kernel->kc)) != BI_OK)
             return st;
-        if ((st = encode_2d(&tb, B, fp8, plan->k, plan->n, ldb, plan->kernel->bn)) != BI_OK)
+        if ((st = encode_operand(&tb, B, fp8, plan->k, plan->n, ldb, plan->kernel->bn, plan->kernel->kc)) != BI_OK)
             return st;
         GemmParams p = base_params(plan, M, C_dev, ldc, status);
-        p.a_box_rows = a_rows;
+        if (!set_rows(&p, plan, a_rows))
+            return BI_ERR_UNSUPPORTED_SHAPE;
         p.scale_a = fp8 ? sa_dev : nullptr;
         p.ld_sa = fp8 ? ld_sa : 0;
         p.scale_b = fp8 ? scale_b : nullptr;

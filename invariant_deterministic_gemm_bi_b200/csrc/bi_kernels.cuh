@@ -16,8 +16,11 @@
 // harmless: it decides where a tile is computed, not how.
 //
 // Roles inside a CTA (6 warps = 192 threads):
-//   warp 0, lane 0 : TMA producer -- A tile [128 x 128 B] and B tile [BN x 128 B] per stage
-//                    into a STAGES-deep shared-memory ring (128-byte swizzle)
+//   warp 0, lane 0 : TMA producer -- A tiles [BM x 128 B] and B tiles [BN x 128 B] into two
+//                    shared-memory rings (128-byte swizzle).  The B (weight) ring is deeper
+//                    than the A ring: B streams from HBM and needs many bytes in flight, A is
+//                    small and L2-resident when the batch is small, so B loads run SB - SA
+//                    K blocks ahead of the A loads of the same K block.
 //   warp 1         : allocates tensor memory; lane 0 issues tcgen05.mma and commits
 //   warps 2..5     : epilogue -- tcgen05.ld from TMEM, fp32 -> bf16 (RNE), masked stores
 // bf16: the accumulator is double-buffered in TMEM so the epilogue of tile i overlaps the
@@ -42,8 +45,9 @@
 
 namespace bi {
 
-constexpr int kBlockM = 128;        // output rows per tile = MMA M (cta_group::1)
+constexpr int kBlockM = 128;        // largest output-tile height = largest MMA M (cta_group::1)
 constexpr int kRowBytes = 128;      // K bytes per stage per row: one 128-byte swizzle row
+constexpr int kRingBytes = 200 * 1024;   // shared memory for the two operand rings
 constexpr int kEpilogueWarps = 4;
 constexpr int kThreads = (2 + kEpilogueWarps) * 32;
 constexpr int kMaxExperts = 1024;
@@ -58,10 +62,13 @@ struct GemmParams {
     int32_t k;               // K (elements)
     int32_t num_k_blocks;    // ceil(K * elt / 128)
     int32_t num_n_blocks;    // ceil(N / BN)
-    int32_t num_m_blocks;    // dense: ceil(M / 128)
+    int32_t num_m_blocks;    // dense: ceil(M / BM)
     int32_t num_experts;     // grouped: E
     int32_t raster_m;        // dense raster band height in m-blocks
-    int32_t a_box_rows;      // rows of A one TMA load brings (<= 128, a multiple of 8)
+    int32_t a_box_rows;      // rows of A one TMA load brings (<= BM, a multiple of 8)
+    int32_t sa, sb;          // ring depths in groups (2..kMaxSA, sa..kMaxSB)
+    uint32_t a_stride;       // bytes between A slots (KC * a_box_rows * 128)
+    uint32_t b_offset;       // byte offset of the B ring in the ring region
     __nv_bfloat16 *c;
     int64_t ldc;
     const float *scale_a;    // FP8: [kb][ld_sa]
@@ -70,7 +77,7 @@ struct GemmParams {
     int32_t kb_scale;        // ceil(K / 128)
     const int32_t *offsets;  // grouped: [E+1] (device)
     int *status;             // device status word
-    uint64_t timeout_ns;
+    uint64_t timeout_cycles; // limit of every pipeline wait, in SM clock cycles
     uint32_t debug_flags;    // bit 0: skip the first load (fault-injection tests)
 };
 
@@ -81,16 +88,26 @@ struct TileCoord {
     int32_t b_row0;   // row of the tile's first B row in the (grouped: stacked) B tensor
 };
 
-template <int BN>
-struct SmemLayout {
-    static constexpr int kABytes = kBlockM * kRowBytes;
-    static constexpr int kBBytes = BN * kRowBytes;
-    static constexpr int kStageBytes = kABytes + kBBytes;
+// Operand rings.  A pipeline stage ("group") carries KC 128-byte K chunks: KC chunks of A rows
+// and KC chunks of BN B rows.  The ring depths and the A slot size are chosen per launch by the
+// host (GemmParams::sa, sb, a_stride, b_offset) inside kRingBytes: when a dense problem has
+// fewer rows than the tile, an A slot only holds the roundup(M, 8) rows TMA brings, which leaves
+// more of shared memory to the B (weight) ring.  The ring geometry decides how far ahead loads
+// run, never what the MMA computes.
+constexpr int kMaxSA = 8;
+constexpr int kMaxSB = 32;
+
+template <int BM, int BN, int KC>
+struct Rings {
+    static constexpr int kAChunkBytes = BM * kRowBytes;   // one full-height A chunk
+    static constexpr int kBChunkBytes = BN * kRowBytes;
+    static constexpr int kABytesMax = KC * kAChunkBytes;  // one A group at full height
+    static constexpr int kBBytes = KC * kBChunkBytes;     // one B group
 };
 
 // Dense tile id -> coordinates.  Tiles are rastered in bands of `raster_m` m-blocks; inside a
 // band the m-block varies fastest, so the CTAs running at the same time share B tiles in L2.
-__device__ __forceinline__ TileCoord dense_tile(const GemmParams &p, int bn, int t)
+__device__ __forceinline__ TileCoord dense_tile(const GemmParams &p, int bm, int bn, int t)
 {
     const int band_tiles = p.raster_m * p.num_n_blocks;
     const int band = t / band_tiles;
@@ -102,7 +119,7 @@ __device__ __forceinline__ TileCoord dense_tile(const GemmParams &p, int bn, int
     const int m_blk = m_first + within % g;
     const int n_blk = within / g;
     TileCoord tc;
-    tc.m0 = m_blk * kBlockM;
+    tc.m0 = m_blk * bm;
     tc.row_end = p.rows;
     tc.n0 = n_blk * bn;
     tc.b_row0 = tc.n0;
@@ -111,7 +128,7 @@ __device__ __forceinline__ TileCoord dense_tile(const GemmParams &p, int bn, int
 
 // Grouped tile id -> coordinates.  prefix[e] = number of tiles of experts < e (E+1 entries,
 // shared memory).  Inside an expert the m-block varies fastest (the segment's CTAs share B_e).
-__device__ __forceinline__ TileCoord grouped_tile(const GemmParams &p, int bn, int t,
+__device__ __forceinline__ TileCoord grouped_tile(const GemmParams &p, int bm, int bn, int t,
                                                   const int32_t *prefix, const int32_t *offs)
 {
     int lo = 0, hi = p.num_experts;   // invariant: prefix[lo] <= t < prefix[hi]
@@ -126,11 +143,11 @@ __device__ __forceinline__ TileCoord grouped_tile(const GemmParams &p, int bn, i
     const int local = t - prefix[e];
     const int seg0 = offs[e];
     const int seg1 = offs[e + 1];
-    const int mb = (seg1 - seg0 + kBlockM - 1) / kBlockM;
+    const int mb = (seg1 - seg0 + bm - 1) / bm;
     const int m_blk = local % mb;
     const int n_blk = local / mb;
     TileCoord tc;
-    tc.m0 = seg0 + m_blk * kBlockM;
+    tc.m0 = seg0 + m_blk * bm;
     tc.row_end = seg1;
     tc.n0 = n_blk * bn;
     tc.b_row0 = e * p.n + tc.n0;
@@ -173,25 +190,35 @@ __device__ __forceinline__ void store_row_chunk32(__nv_bfloat16 *crow, int col0,
 // The kernel
 // ---------------------------------------------------------------------------------------------
 //
+// BM      : output rows per tile = MMA M (64 or 128).  With M = 64 the accumulator's row i sits
+//           in TMEM lane (i % 16) + 32 * (i / 16), so each epilogue warp owns 16 rows.
 // BN      : output columns per tile = MMA N (multiple of 32, <= 256; FP8 <= 128)
-// STAGES  : shared-memory ring depth
 // FP8     : e4m3 operands with fp32 block scales (else bf16)
 // GROUPED : MoE grouped layout (bf16 only)
-template <int BN, int STAGES, bool FP8, bool GROUPED>
+// KC      : 128-byte K chunks per pipeline stage (group).  KC > 1 loads a group with one 3-D TMA
+//           box per operand (chunk index as the third coordinate), so the producer and MMA
+//           threads pay their per-stage handshakes once per KC chunks.  The MMA still walks the
+//           chunks of a tile one by one in ascending K: KC changes no bit of the result.
+// The ring depths follow from (BM, BN, KC) (see Rings).
+template <int BM, int BN, int KC, bool FP8, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, 1)
     bi_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b, const GemmParams p)
 {
+    static_assert(BM == 64 || BM == 128, "MMA M is 64 or 128");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32,256]");
     static_assert(!FP8 || BN <= 128, "FP8 keeps BN fp32 accumulators per thread: BN <= 128");
     static_assert(!(FP8 && GROUPED), "grouped FP8 is not built");
-    using L = SmemLayout<BN>;
-    constexpr int kElemsPerRow = FP8 ? 128 : 64;        // K elements per 128-byte row
+    static_assert(KC >= 1 && KC <= 4, "1..4 chunks per group");
+    using R = Rings<BM, BN, KC>;
+    constexpr int kElemsPerRow = FP8 ? 128 : 64;         // K elements per 128-byte row
     constexpr int kMmaK = FP8 ? 32 : 16;                 // K per tcgen05.mma
     constexpr int kMmaPerStage = kElemsPerRow / kMmaK;   // 4
     constexpr int kBytesPerMmaK = kMmaK * (FP8 ? 1 : 2); // 32 bytes
-    // TMEM buffers: bf16 double-buffers the accumulator; FP8 rings NPART partial products.
-    constexpr int kNumAcc = FP8 ? ((512 / BN) < 4 ? (512 / BN) : 4) : 2;
+    constexpr int kRowsPerWarp = BM / 4;                 // output rows owned by one epilogue warp
+    // TMEM buffers: bf16 double-buffers the accumulator; FP8 rings kNumAcc partial products
+    // (one per K chunk, at least two groups' worth so the promotion overlaps the next group).
+    constexpr int kNumAcc = FP8 ? ((512 / BN) < 8 ? (512 / BN) : 8) : 2;
     constexpr int kTmemColsNeeded = kNumAcc * BN;
     constexpr uint32_t kTmemCols = kTmemColsNeeded <= 32    ? 32
                                    : kTmemColsNeeded <= 64  ? 64
@@ -199,20 +226,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    : kTmemColsNeeded <= 256 ? 256
                                                             : 512;
     static_assert(kTmemColsNeeded <= 512, "TMEM holds 512 columns");
-    constexpr uint32_t kIdesc = FP8 ? ptx::idesc_e4m3(kBlockM, BN) : ptx::idesc_bf16(kBlockM, BN);
+    static_assert(!FP8 || kNumAcc >= 2 * KC, "FP8 needs two groups of partial buffers");
+    // (the host keeps sb > kNumAcc / KC so the FP8 epilogue can track partials on the consumed ring)
+    constexpr uint32_t kIdesc = FP8 ? ptx::idesc_e4m3(BM, BN) : ptx::idesc_bf16(BM, BN);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *smem_a = smem;
-    uint8_t *smem_b = smem + STAGES * L::kABytes;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * L::kStageBytes);
-    uint64_t *full_bar = bars;
-    uint64_t *empty_bar = bars + STAGES;
-    uint64_t *accf_bar = bars + 2 * STAGES;            // accumulator (or partial) full
-    uint64_t *acce_bar = bars + 2 * STAGES + kNumAcc;  // accumulator (or partial) empty
-    uint64_t *drain_bar = bars + 2 * STAGES + 2 * kNumAcc;
+    uint8_t *smem_b = smem + p.b_offset;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kRingBytes);
+    // full[j % sb]: both TMA loads of group j landed (two arrivals: the B load and, issued
+    // later, the A load).  consumed[j % sb]: the MMAs of group j completed, which frees B slot
+    // j % sb and A slot j % sa (one commit per group).  A group's two arrivals always land in
+    // its own phase: slot j % sb is refilled only after group j was consumed.
+    uint64_t *full = bars;
+    uint64_t *consumed = full + kMaxSB;
+    uint64_t *accf_bar = consumed + kMaxSB;    // accumulator (or partial) full
+    uint64_t *acce_bar = accf_bar + kNumAcc;   // accumulator (or partial) empty
+    uint64_t *drain_bar = acce_bar + kNumAcc;
     uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(drain_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
     int32_t *grp_prefix = reinterpret_cast<int32_t *>(tmem_base_smem + 4);   // [E+1]
@@ -222,9 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane = ptx::lane_id();
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            ptx::mbar_init(&full_bar[s], 1);
-            ptx::mbar_init(&empty_bar[s], 1);
+        for (int s = 0; s < kMaxSB; ++s) {
+            ptx::mbar_init(&full[s], 2);
+            ptx::mbar_init(&consumed[s], 1);
         }
         for (int a = 0; a < kNumAcc; ++a) {
             ptx::mbar_init(&accf_bar[a], 1);
@@ -263,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!s_bad) {
                 for (int e = 0; e < E; ++e) {
                     grp_prefix[e] = acc;
-                    const int mb = (grp_offs[e + 1] - grp_offs[e] + kBlockM - 1) / kBlockM;
+                    const int mb = (grp_offs[e + 1] - grp_offs[e] + BM - 1) / BM;
                     acc += mb * p.num_n_blocks;
                 }
             } else if (blockIdx.x == 0) {
@@ -285,68 +318,129 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     auto tile_at = [&](int t) -> TileCoord {
         if constexpr (GROUPED)
-            return grouped_tile(p, BN, t, grp_prefix, grp_offs);
+            return grouped_tile(p, BM, BN, t, grp_prefix, grp_offs);
         else
-            return dense_tile(p, BN, t);
+            return dense_tile(p, BM, BN, t);
     };
 
-    const int nkb = p.num_k_blocks;
+    const int nkb = p.num_k_blocks;              // 128-byte K chunks per tile
+    const int nkg = (nkb + KC - 1) / KC;         // groups per tile
+    const uint32_t a_chunk_pitch = static_cast<uint32_t>(p.a_box_rows) * kRowBytes;
 
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint64_t pol_a = ptx::policy_evict_normal();
-            const uint64_t pol_b = ptx::policy_evict_normal();
-            uint32_t issued = 0, issued_phase = 0;            // per-stage: a load in flight / its parity
-            int stage = 0;
-            uint32_t phase = 0;
-            bool skip_next = (p.debug_flags & 1u) != 0;
+            const uint64_t pol = ptx::policy_evict_normal();
+            // Two cursors over this CTA's (tile, group) sequence: B runs `lag` groups ahead.
+            struct Cursor {
+                int t, kg;
+                bool valid;
+                TileCoord tc;
+            };
+            Cursor cb{static_cast<int>(blockIdx.x), 0, static_cast<int>(blockIdx.x) < num_tiles, {}};
+            if (cb.valid)
+                cb.tc = tile_at(cb.t);
+            Cursor ca = cb;
+            auto advance = [&](Cursor &c) {
+                if (++c.kg == nkg) {
+                    c.kg = 0;
+                    c.t += gridDim.x;
+                    c.valid = c.t < num_tiles;
+                    if (c.valid)
+                        c.tc = tile_at(c.t);
+                }
+            };
+            auto load = [&](void *dst, const CUtensorMap *map, uint64_t *bar, int kg, int row) {
+                if constexpr (KC == 1)
+                    ptx::tma_load_2d(dst, map, bar, kg * kElemsPerRow, row, pol);
+                else
+                    ptx::tma_load_3d(dst, map, bar, 0, row, kg * KC, pol);
+            };
+            const int SA = p.sa, SB = p.sb, lag = SB - SA;   // B groups lead A groups by lag
+            int jb = 0, ja = 0;                 // groups issued so far
+            int bs = 0, as = 0, cs = 0;         // B slot of jb, A slot of ja, consumed slot of ja - SA
+            int fs = 0;                         // full-ring slot of group ja
+            uint32_t bph = 0, cph = 0;
+            bool skipped_b0 = false;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                const TileCoord tc = tile_at(t);
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, p.timeout_ns, abort_flag)) {
+            while (ok && (cb.valid || ca.valid)) {
+                if (cb.valid) {
+                    // slot bs is free once group jb - SB was consumed
+                    if (!ptx::mbar_wait(&consumed[bs], bph ^ 1u, p.timeout_cycles, abort_flag)) {
                         record_failure(p, abort_flag, kStatusTimeout);
                         ok = false;
                         break;
                     }
-                    if (skip_next) {
-                        skip_next = false;   // fault injection: this stage is never filled
+                    if (jb == 0 && (p.debug_flags & 1u)) {
+                        skipped_b0 = true;      // fault injection: this B group is never filled
                     } else {
-                        ptx::mbar_arrive_expect_tx(&full_bar[stage],
-                                                   (p.a_box_rows + BN) * kRowBytes);
-                        ptx::tma_load_2d(smem_a + stage * L::kABytes, &tmap_a, &full_bar[stage],
-                                         kb * kElemsPerRow, tc.m0, pol_a);
-                        ptx::tma_load_2d(smem_b + stage * L::kBBytes, &tmap_b, &full_bar[stage],
-                                         kb * kElemsPerRow, tc.b_row0, pol_b);
-                        issued |= 1u << stage;
-                        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                        ptx::mbar_arrive_expect_tx(&full[bs], R::kBBytes);
+                        load(smem_b + bs * R::kBBytes, &tmap_b, &full[bs], cb.kg, cb.tc.b_row0);
                     }
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
+                    advance(cb);
+                    ++jb;
+                    if (++bs == SB) {
+                        bs = 0;
+                        bph ^= 1u;
                     }
                 }
+                if (ca.valid && (ja + lag < jb || !cb.valid)) {
+                    // slot `as` is free once group ja - SA was consumed.  That group's consumed
+                    // barrier cannot have moved on to group ja - SA + SB yet: that one needs A
+                    // group ja + lag, which is not issued.
+                    if (ja >= SA) {
+                        if (!ptx::mbar_wait(&consumed[cs], cph, p.timeout_cycles, abort_flag)) {
+                            record_failure(p, abort_flag, kStatusTimeout);
+                            ok = false;
+                            break;
+                        }
+                        if (++cs == SB) {
+                            cs = 0;
+                            cph ^= 1u;
+                        }
+                    }
+                    ptx::mbar_arrive_expect_tx(&full[fs], KC * a_chunk_pitch);
+                    load(smem_a + as * p.a_stride, &tmap_a, &full[fs], ca.kg, ca.tc.m0);
+                    advance(ca);
+                    ++ja;
+                    if (++as == SA)
+                        as = 0;
+                    if (++fs == SB)
+                        fs = 0;
+                }
             }
-            // Drain: every load this thread issued must have landed before the CTA exits.
-            // (On the normal path they all have: the MMA warp consumed them.)
-            for (int s = 0; s < STAGES; ++s)
-                if (issued & (1u << s))
-                    ptx::mbar_wait(&full_bar[s], (issued_phase >> s) & 1u, p.timeout_ns, nullptr);
+            // Drain: every load this thread issued must have landed before the CTA exits (on
+            // the normal path they all have: the MMA warp consumed them).  Only the last SB
+            // groups can still be in flight.  A group whose A load was never issued (the loop
+            // stopped early) cannot complete its phase: its B bytes are waited for alone by
+            // letting this thread stand in for the missing A arrival.
+            for (int i = jb > SB ? jb - SB : 0; i < jb; ++i) {
+                if (i == 0 && skipped_b0)
+                    continue;
+                if (i >= ja)
+                    ptx::mbar_arrive(&full[i % SB]);
+                ptx::mbar_wait(&full[i % SB], static_cast<uint32_t>(i / SB) & 1u, p.timeout_cycles,
+                               nullptr);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t acc_iter = 0;   // bf16: tiles done; FP8: K blocks done
+            const int SA = p.sa, SB = p.sb;
+            int sa = 0, sb = 0;      // ring slots of the next group
+            uint32_t pb = 0;         // phase of full[sb] / consumed[sb]
+            // Shared-memory descriptors are linear in the address (start address >> 4 in the low
+            // bits), so every slot / chunk / K-step descriptor is a base plus an offset.
+            const uint64_t a_desc0 = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_a));
+            const uint64_t b_desc0 = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_b));
+            uint32_t acc_iter = 0;   // bf16: tiles done; FP8: K chunks done
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 uint32_t d_tmem = 0;
                 if (!FP8) {
                     const uint32_t a = acc_iter % kNumAcc;
                     const uint32_t par = (acc_iter / kNumAcc) & 1u;
-                    if (!ptx::mbar_wait(&acce_bar[a], par ^ 1u, p.timeout_ns, abort_flag)) {
+                    if (!ptx::mbar_wait(&acce_bar[a], par ^ 1u, p.timeout_cycles, abort_flag)) {
                         record_failure(p, abort_flag, kStatusTimeout);
                         ok = false;
                         break;
@@ -354,45 +448,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tc_fence_after_sync();
                     d_tmem = tmem_base + a * BN;
                 }
-                for (int kb = 0; kb < nkb; ++kb) {
-                    uint32_t part = 0;
-                    if (FP8) {
-                        part = acc_iter % kNumAcc;
-                        const uint32_t par = (acc_iter / kNumAcc) & 1u;
-                        if (!ptx::mbar_wait(&acce_bar[part], par ^ 1u, p.timeout_ns, abort_flag)) {
-                            record_failure(p, abort_flag, kStatusTimeout);
-                            ok = false;
-                            break;
-                        }
-                        ptx::tc_fence_after_sync();
-                        d_tmem = tmem_base + part * BN;
-                    }
-                    if (!ptx::mbar_wait(&full_bar[stage], phase, p.timeout_ns, abort_flag)) {
+                for (int kg = 0; kg < nkg; ++kg) {
+                    if (!ptx::mbar_wait(&full[sb], pb, p.timeout_cycles, abort_flag)) {
                         record_failure(p, abort_flag, kStatusTimeout);
                         ok = false;
                         break;
                     }
                     ptx::tc_fence_after_sync();
-                    const uint64_t a_desc = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_a + stage * L::kABytes));
-                    const uint64_t b_desc = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_b + stage * L::kBBytes));
+                    const uint64_t a_slot = a_desc0 + ((sa * p.a_stride) >> 4);
+                    const uint64_t b_slot = b_desc0 + ((sb * R::kBBytes) >> 4);
 #pragma unroll
-                    for (int j = 0; j < kMmaPerStage; ++j) {
-                        const uint64_t step = static_cast<uint64_t>((j * kBytesPerMmaK) >> 4);
-                        // bf16: accumulate across the whole K of the tile; FP8: one K block
-                        const uint32_t accumulate = FP8 ? (j > 0) : ((kb > 0) || (j > 0));
-                        if (FP8)
-                            ptx::mma_e4m3_ss(d_tmem, a_desc + step, b_desc + step, kIdesc, accumulate);
-                        else
-                            ptx::mma_bf16_ss(d_tmem, a_desc + step, b_desc + step, kIdesc, accumulate);
+                    for (int c = 0; c < KC; ++c) {
+                        const int chunk = kg * KC + c;
+                        if (chunk >= nkb)
+                            break;
+                        if (FP8) {
+                            // each K chunk's partial product goes to its own TMEM buffer
+                            const uint32_t part = acc_iter % kNumAcc;
+                            const uint32_t par = (acc_iter / kNumAcc) & 1u;
+                            if (!ptx::mbar_wait(&acce_bar[part], par ^ 1u, p.timeout_cycles, abort_flag)) {
+                                record_failure(p, abort_flag, kStatusTimeout);
+                                ok = false;
+                                break;
+                            }
+                            ptx::tc_fence_after_sync();
+                            d_tmem = tmem_base + part * BN;
+                            ++acc_iter;
+                        }
+                        const uint64_t a_desc = a_slot + ((c * a_chunk_pitch) >> 4);
+                        const uint64_t b_desc = b_slot + ((c * R::kBChunkBytes) >> 4);
+#pragma unroll
+                        for (int q = 0; q < kMmaPerStage; ++q) {
+                            const uint64_t step = static_cast<uint64_t>((q * kBytesPerMmaK) >> 4);
+                            // bf16: accumulate across the whole K of the tile; FP8: one K chunk
+                            const uint32_t accumulate = FP8 ? (q > 0) : ((chunk > 0) || (q > 0));
+                            if (FP8)
+                                ptx::mma_e4m3_ss(d_tmem, a_desc + step, b_desc + step, kIdesc, accumulate);
+                            else
+                                ptx::mma_bf16_ss(d_tmem, a_desc + step, b_desc + step, kIdesc, accumulate);
+                        }
                     }
-                    ptx::mma_commit(&empty_bar[stage]);   // frees the smem stage when the MMAs are done
-                    if (FP8) {
-                        ptx::mma_commit(&accf_bar[part]); // partial product of this K block ready
-                        ++acc_iter;
-                    }
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
+                    if (!ok)
+                        break;
+                    // one commit per group frees both smem slots and, for FP8, marks the group's
+                    // partial products ready for the epilogue
+                    ptx::mma_commit(&consumed[sb]);
+                    if (++sa == SA)
+                        sa = 0;
+                    if (++sb == SB) {
+                        sb = 0;
+                        pb ^= 1u;
                     }
                 }
                 if (!ok)
@@ -404,24 +509,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // Drain: wait for every MMA this thread issued before tensor memory is freed.
             ptx::mma_commit(drain_bar);
-            ptx::mbar_wait(drain_bar, 0, p.timeout_ns, nullptr);
+            ptx::mbar_wait(drain_bar, 0, p.timeout_cycles, nullptr);
         }
     } else {
         // ------------------------------------------------------------------ epilogue warps
         const uint32_t q = warp & 3u;                 // TMEM lane quarter of this warp
-        const uint32_t row_in_tile = q * 32 + lane;
+        const bool lane_holds_row = BM == 128 || lane < 16;
+        const uint32_t row_in_tile = q * kRowsPerWarp + (BM == 128 ? lane : (lane & 15u));
         const uint32_t lane_addr = (q * 32u) << 16;
-        uint32_t acc_iter = 0;
+        uint32_t acc_iter = 0;   // bf16: tiles; FP8: K chunks
+        int gs = 0;              // FP8: consumed-ring slot of the next group, and its phase
+        uint32_t gph = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
             const TileCoord tc = tile_at(t);
             const int row = tc.m0 + static_cast<int>(row_in_tile);
-            const bool row_ok = row < tc.row_end;
+            const bool row_ok = lane_holds_row && row < tc.row_end;
             __nv_bfloat16 *crow = p.c + static_cast<int64_t>(row) * p.ldc;
             if constexpr (!FP8) {
                 const uint32_t a = acc_iter % kNumAcc;
                 const uint32_t par = (acc_iter / kNumAcc) & 1u;
-                if (!ptx::mbar_wait(&accf_bar[a], par, p.timeout_ns, abort_flag)) {
+                if (!ptx::mbar_wait(&accf_bar[a], par, p.timeout_cycles, abort_flag)) {
                     record_failure(p, abort_flag, kStatusTimeout);
                     ok = false;
                     break;
@@ -438,8 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     float v[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        v[j] = __uint_as_float(r[j]);
+                    for (int jj = 0; jj < 32; ++jj)
+                        v[jj] = __uint_as_float(r[jj]);
                     if (row_ok)
                         store_row_chunk32(crow, tc.n0 + c * 32, p.n, v);
                 }
@@ -447,38 +555,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 float acc[BN];
 #pragma unroll
-                for (int j = 0; j < BN; ++j)
-                    acc[j] = 0.0f;
+                for (int jj = 0; jj < BN; ++jj)
+                    acc[jj] = 0.0f;
                 const float *sa_col = p.scale_a + (row_ok ? row : 0);
-                for (int kb = 0; kb < nkb; ++kb) {
-                    const uint32_t part = acc_iter % kNumAcc;
-                    const uint32_t par = (acc_iter / kNumAcc) & 1u;
-                    const float sa = row_ok ? __ldg(sa_col + static_cast<int64_t>(kb) * p.ld_sa) : 0.0f;
-                    if (!ptx::mbar_wait(&accf_bar[part], par, p.timeout_ns, abort_flag)) {
+                for (int kg = 0; kg < nkg && ok; ++kg) {
+                    // the group's partials are ready when its consumed barrier completes; the MMA
+                    // warp runs at most kNumAcc chunks (< sb groups) ahead, so the barrier cannot
+                    // have moved on to the group sb later
+                    if (!ptx::mbar_wait(&consumed[gs], gph, p.timeout_cycles, abort_flag)) {
                         record_failure(p, abort_flag, kStatusTimeout);
                         ok = false;
                         break;
                     }
-                    ptx::tc_fence_after_sync();
-#pragma unroll
-                    for (int c = 0; c < BN / 32; ++c) {
-                        uint32_t r[32];
-                        ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + part * BN + c * 32, r);
-                        ptx::tmem_wait_ld(r);
-                        // 32 columns never straddle a 128-column scale block (n0 and c*32 are
-                        // multiples of 32)
-                        const int col = tc.n0 + c * 32;
-                        const float sb = col < p.n
-                                             ? __ldg(p.scale_b + static_cast<int64_t>(col >> 7) * p.kb_scale + kb)
-                                             : 0.0f;
-                        const float s = sa * sb;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            acc[c * 32 + j] = fmaf(__uint_as_float(r[j]), s, acc[c * 32 + j]);
+                    if (++gs == p.sb) {
+                        gs = 0;
+                        gph ^= 1u;
                     }
-                    ptx::tc_fence_before_sync();
-                    ptx::mbar_arrive(&acce_bar[part]);
-                    ++acc_iter;
+                    ptx::tc_fence_after_sync();
+                    for (int cc = 0; cc < KC; ++cc) {
+                        const int kb = kg * KC + cc;
+                        if (kb >= nkb)
+                            break;
+                        const uint32_t part = acc_iter % kNumAcc;
+                        const float sa = row_ok ? __ldg(sa_col + static_cast<int64_t>(kb) * p.ld_sa) : 0.0f;
+#pragma unroll
+                        for (int c = 0; c < BN / 32; ++c) {
+                            uint32_t r[32];
+                            ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + part * BN + c * 32, r);
+                            ptx::tmem_wait_ld(r);
+                            // 32 columns never straddle a 128-column scale block (n0 and c*32
+                            // are multiples of 32)
+                            const int col = tc.n0 + c * 32;
+                            const float sb = col < p.n
+                                                 ? __ldg(p.scale_b + static_cast<int64_t>(col >> 7) * p.kb_scale + kb)
+                                                 : 0.0f;
+                            const float s = sa * sb;
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj)
+                                acc[c * 32 + jj] = fmaf(__uint_as_float(r[jj]), s, acc[c * 32 + jj]);
+                        }
+                        ptx::tc_fence_before_sync();
+                        ptx::mbar_arrive(&acce_bar[part]);
+                        ++acc_iter;
+                    }
                 }
                 if (!ok)
                     break;
@@ -487,8 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < BN / 32; ++c) {
                         float v[32];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            v[j] = acc[c * 32 + j];
+                        for (int jj = 0; jj < 32; ++jj)
+                            v[jj] = acc[c * 32 + jj];
                         store_row_chunk32(crow, tc.n0 + c * 32, p.n, v);
                     }
                 }
@@ -516,11 +635,10 @@ __global__ void bi_zero_kernel(__nv_bfloat16 *c, int64_t ldc, int64_t m, int64_t
     }
 }
 
-template <int BN, int STAGES, bool FP8, bool GROUPED>
+template <int BM, int BN, int KC, bool FP8, bool GROUPED>
 constexpr int smem_bytes_for()
 {
-    return 1024 + STAGES * SmemLayout<BN>::kStageBytes + 512 +
-           (GROUPED ? 2 * (kMaxExperts + 1) * 4 : 0);
+    return 1024 + kRingBytes + 1024 + (GROUPED ? 2 * (kMaxExperts + 1) * 4 : 0);
 }
 
 } // namespace bi

@@ -15,13 +15,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p)
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 
@@ -54,35 +47,41 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
 
 // True once the phase with the given parity has completed.  A fresh barrier (phase 0 running)
 // reports parity 1 as completed, which is how producers pass their first wait on "empty".
+// While the phase is incomplete the thread is suspended (it does not spin and take issue slots
+// from the producer and MMA threads) until the phase completes or the suspend-time hint
+// (1 ms) runs out, whichever comes first.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity)
 {
+    constexpr uint32_t kSuspendHintNs = 1000000;
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar_addr), "r"(parity)
+        : "r"(bar_addr), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
 
 // Bounded wait: returns true when the phase completed, false when `abort_flag` became non-zero
-// or `timeout_ns` of wall-clock time passed first.  Every pipeline wait goes through here, so
-// no wait in these kernels can spin forever.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
+// or `timeout_cycles` SM clock cycles passed first.  Every pipeline wait goes through here, so no
+// wait in these kernels can spin forever.  The limit is counted with the SM-local cycle counter:
+// it is cheap to read, whereas a read of the global nanosecond timer can stall the waiting thread
+// long enough to delay every producer/consumer hand-off.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t timeout_cycles,
                                           volatile int *abort_flag)
 {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity))
         return true;
-    const uint64_t t0 = globaltimer_ns();
+    const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(a, parity))
             return true;
         if (abort_flag != nullptr && *abort_flag != 0)
             return false;
-        if (globaltimer_ns() - t0 > timeout_ns)
+        if (static_cast<uint64_t>(clock64() - t0) > timeout_cycles)
             return false;
     }
 }
@@ -105,6 +104,20 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
         " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(cache_hint)
+        : "memory");
+}
+
+// 3-D tiled load: the operand viewed as [chunks][rows][128 bytes] (coordinate 0 inside a
+// chunk, 1 the row, 2 the 128-byte K chunk); one box of KC chunks lands in shared memory as KC
+// consecutive [rows x 128 B] tiles.
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map, uint64_t *bar,
+                                            int32_t x, int32_t y, int32_t z, uint64_t cache_hint)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z),
+        "l"(cache_hint)
         : "memory");
 }
 

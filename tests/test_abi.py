@@ -43,8 +43,9 @@ def test_plan_describe_is_m_free_and_sane():
                           (7168, 7168, 1, 1), (2048, 7168, 0, 64), (256, 512, 0, 1), (5, 3, 0, 1)]:
         info = bg.bi_gemm_plan_describe(bg.bi_gemm_plan(N, K, dt, E))
         assert info["n"] == N and info["k"] == K and info["num_experts"] == E
-        assert info["k_order_id"] == 0 and info["block_m"] == 128
-        assert info["block_k"] * (1 if dt == 1 else 2) == 128
+        assert info["k_order_id"] == 0 and info["block_m"] in (64, 128)
+        assert info["mma_m"] == info["block_m"] and 2 <= info["stages_a"] <= info["stages"]
+        assert info["block_k"] * (1 if dt == 1 else 2) in (128, 256, 512)
         assert info["mma_n"] == info["block_n"] and info["block_n"] % 32 == 0
         assert info["smem_bytes"] <= 232448
         assert info["tmem_columns"] <= 512
