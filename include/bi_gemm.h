@@ -142,8 +142,10 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M,
  * expert_offsets is a DEVICE array of E+1 int32 with offsets[0] = 0, non-decreasing,
  * offsets[E] = total_rows; it is read only by the kernel (no host synchronisation).  Malformed
  * offsets make the kernel compute nothing and set BI_ERR_BAD_OFFSETS in the status word.
- * A grouped plan takes the tile configuration of the dense plan with the same N and K, so every
- * row gets the bits a dense call with its expert's B_e would give it.
+ * Every row's bits are fixed by the grouped plan alone: they do not depend on total_rows, on the
+ * offsets or on the other rows of its expert.  (A grouped plan may choose a different tile from
+ * the dense plan of the same N and K; when the two plans' bi_plan_info_t agree, a row also gets
+ * the bits a dense call with its expert's B_e would give it.)
  * Errors: as bi_gemm_run; a dense plan returns BI_ERR_INVALID_ARG.
  */
 bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows,

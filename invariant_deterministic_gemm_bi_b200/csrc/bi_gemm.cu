@@ -19,6 +19,7 @@
 
 #include "bi_gemm.h"
 #include "bi_kernels.cuh"
+#include "bi_kernels_pair.cuh"
 
 namespace {
 
@@ -32,39 +33,46 @@ typedef void (*KernelFn)(const __grid_constant__ CUtensorMap, const __grid_const
                          const GemmParams);
 
 struct KernelEntry {
-    int bm;
+    int threads;   // threads per CTA
+    int bm;        // tile height = MMA M (256 for a CTA pair)
     int bn;
     int kc;
     bool fp8;
     bool grouped;
+    bool pair;     // cta_group::2 on a cluster of two CTAs
     KernelFn fn;
     int smem;
 };
 
 #define BI_ENTRY(BM, BN, KC, F8, GR)                                                               \
-    KernelEntry{BM, BN, KC, F8, GR, &bi::bi_gemm_kernel<BM, BN, KC, F8, GR>,                        \
+    KernelEntry{bi::Epi<F8, BN>::kThreads, BM, BN, KC, F8, GR, false,                              \
+                &bi::bi_gemm_kernel<BM, BN, KC, F8, GR>,                                           \
                 bi::smem_bytes_for<BM, BN, KC, F8, GR>()}
+#define BI_PAIR(BN, KC, F8, GR)                                                                    \
+    KernelEntry{bi::kThreads, 256, BN, KC, F8, GR, true, &bi::bi_gemm_kernel_pair<BN, KC, F8, GR>,  \
+                bi::smem_bytes_for_pair<BN, KC, F8, GR>()}
 
-// Every (BM, BN) tile in two forms: the tile's preferred number of 128-byte K chunks per
-// pipeline stage (3-D TMA boxes; needs K to be a multiple of the chunk), and one chunk per stage
-// for any other K.  Narrow tiles take more chunks per stage so that one weight box is ~16 KB.
+// Narrow tiles (BN <= 64) run on one CTA; wide ones (BN >= 128) on a CTA pair.  Every tile comes
+// in two forms: its preferred number of 128-byte K chunks per pipeline stage (3-D TMA boxes;
+// needs K to be a multiple of the chunk), and one chunk per stage for any other K.
 const KernelEntry kKernels[] = {
-    BI_ENTRY(64, 32, 1, false, false),   BI_ENTRY(64, 32, 4, false, false),
-    BI_ENTRY(128, 32, 1, false, false),  BI_ENTRY(128, 32, 4, false, false),
-    BI_ENTRY(128, 64, 1, false, false),  BI_ENTRY(128, 64, 2, false, false),
-    BI_ENTRY(128, 128, 1, false, false), BI_ENTRY(128, 128, 2, false, false),
-    BI_ENTRY(128, 256, 1, false, false),
-    BI_ENTRY(128, 32, 1, true, false),   BI_ENTRY(128, 32, 4, true, false),
-    BI_ENTRY(128, 64, 1, true, false),   BI_ENTRY(128, 64, 2, true, false),
-    BI_ENTRY(128, 128, 1, true, false),  BI_ENTRY(128, 128, 2, true, false),
-    BI_ENTRY(128, 32, 1, false, true),   BI_ENTRY(128, 32, 4, false, true),
-    BI_ENTRY(128, 64, 1, false, true),   BI_ENTRY(128, 64, 2, false, true),
-    BI_ENTRY(128, 128, 1, false, true),  BI_ENTRY(128, 128, 2, false, true),
-    BI_ENTRY(128, 256, 1, false, true),
+    BI_ENTRY(64, 32, 1, false, false),  BI_ENTRY(64, 32, 4, false, false),
+    BI_ENTRY(128, 32, 1, false, false), BI_ENTRY(128, 32, 4, false, false),
+    BI_ENTRY(128, 64, 1, false, false), BI_ENTRY(128, 64, 2, false, false),
+    BI_ENTRY(128, 32, 1, true, false),  BI_ENTRY(128, 32, 4, true, false),
+    BI_ENTRY(128, 64, 1, true, false),  BI_ENTRY(128, 64, 2, true, false),
+    BI_ENTRY(128, 32, 1, false, true),  BI_ENTRY(128, 32, 4, false, true),
+    BI_ENTRY(128, 64, 1, false, true),  BI_ENTRY(128, 64, 2, false, true),
+    BI_ENTRY(128, 128, 1, false, true), BI_ENTRY(128, 128, 2, false, true),
+    BI_PAIR(128, 1, false, false),      BI_PAIR(128, 2, false, false),
+    BI_PAIR(256, 1, false, false),      BI_PAIR(256, 2, false, false),
+    BI_PAIR(128, 1, true, false),       BI_PAIR(128, 2, true, false),
+    BI_PAIR(128, 1, false, true),       BI_PAIR(128, 2, false, true),
+    BI_PAIR(256, 1, false, true),       BI_PAIR(256, 2, false, true),
 };
 constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
 
-int preferred_chunks(int bn) { return bn <= 32 ? 4 : bn >= 256 ? 1 : 2; }
+int preferred_chunks(int bn) { return bn <= 32 ? 4 : 2; }
 
 const KernelEntry *find_kernel(int bm, int bn, int kc, bool fp8, bool grouped)
 {
@@ -85,6 +93,14 @@ struct RingGeom {
 RingGeom ring_geometry(const KernelEntry *k, int a_rows)
 {
     const int chunk = bi::kRowBytes;
+    if (k->pair) {   // fixed at compile time (bi::PairRings): 128 A rows and BN/2 B rows per CTA
+        const int a_bytes = k->kc * 128 * chunk;
+        const int b_bytes = k->kc * (k->bn / 2) * chunk;
+        int st = bi::kRingBytes / (a_bytes + b_bytes);
+        if (st > bi::kMaxSB)
+            st = bi::kMaxSB;
+        return RingGeom{st, st, static_cast<uint32_t>(a_bytes), static_cast<uint32_t>(st * a_bytes)};
+    }
     const int a_stride = k->kc * a_rows * chunk;
     const int over = (k->bm - a_rows) * chunk;     // the MMA reads BM rows from each A chunk
     const int b_stride = k->kc * k->bn * chunk;
@@ -119,35 +135,46 @@ RingGeom ring_geometry(const KernelEntry *k, int a_rows)
 // Plan table
 // ---------------------------------------------------------------------------------------------
 
-// The tile (BM x BN) for (N, K, dtype).  Known projection shapes get the tile tuned for them;
-// any other shape takes BM = 128 and the widest BN that still gives >= 100 tiles at M <= 128,
-// since without split-K the N tiles are the only parallelism a small batch has.  A grouped plan
-// uses the dense plan's tile for the same (N, K), so a row of an expert's segment gets the bits a
-// dense call with that expert's weights would give it.
+// The tile (BM x BN) for (N, K, dtype, experts).  Known projection shapes get the tile tuned for
+// them; any other shape takes the widest tile that still gives enough tiles for a small batch,
+// since without split-K the N tiles are the only parallelism such a batch has.  Tiles 256 rows
+// high run on a CTA pair.  Grouped (MoE) plans use one-CTA tiles: an expert's segment is often
+// only a few rows long, and a taller tile would only load more rows that are never stored.
 struct TileChoice {
     int bm, bn;
 };
 
-TileChoice choose_tile(int64_t N, int64_t K, bi_dtype_t dtype)
+TileChoice choose_tile(int64_t N, int64_t K, bi_dtype_t dtype, int experts)
 {
     struct Row {
         int64_t n, k;
-        int dtype, bm, bn;
+        int dtype, experts, bm, bn;
     };
     static const Row table[] = {
-        {4096, 7168, BI_DTYPE_BF16, 128, 32},              // decode-shaped projection
-        {7168, 2048, BI_DTYPE_BF16, 128, 256},             // prefill-shaped, wide N
-        {2048, 7168, BI_DTYPE_BF16, 128, 128},             // prefill-shaped, long K; MoE experts
-        {256, 512, BI_DTYPE_BF16, 128, 32},                // small correctness shape
-        {7168, 7168, BI_DTYPE_E4M3_BLOCKSCALED, 128, 64},  // FP8 projection
+        {4096, 7168, BI_DTYPE_BF16, 1, 128, 32},              // decode-shaped projection
+        {7168, 2048, BI_DTYPE_BF16, 1, 256, 256},             // prefill-shaped, wide N (CTA pair)
+        {2048, 7168, BI_DTYPE_BF16, 1, 256, 256},             // prefill-shaped, long K (CTA pair)
+        {256, 512, BI_DTYPE_BF16, 1, 128, 32},                // small correctness shape
+        {7168, 7168, BI_DTYPE_E4M3_BLOCKSCALED, 1, 128, 64},  // FP8 projection
+        {2048, 7168, BI_DTYPE_BF16, 64, 128, 128},            // MoE experts
     };
     for (const Row &r : table)
-        if (r.n == N && r.k == K && r.dtype == dtype)
+        if (r.n == N && r.k == K && r.dtype == dtype && r.experts == (experts > 1 ? 64 : 1) &&
+            (experts == 1 || experts == 64))
             return {r.bm, r.bn};
+    if (experts > 1) {
+        for (int bn = 128; bn > 32; bn /= 2)
+            if ((N + bn - 1) / bn >= 100)
+                return {128, bn};
+        return {128, 32};
+    }
+    // wide dense fallback tiles run on a CTA pair (256 rows)
     const int max_bn = dtype == BI_DTYPE_E4M3_BLOCKSCALED ? 128 : 256;
-    for (int bn = max_bn; bn > 32; bn /= 2)
+    for (int bn = max_bn; bn >= 128; bn /= 2)
         if ((N + bn - 1) / bn >= 100)
-            return {128, bn};
+            return {256, bn};
+    if ((N + 63) / 64 >= 100)
+        return {128, 64};
     return {128, 32};
 }
 
@@ -162,6 +189,7 @@ struct DeviceInfo {
     bool ok = false;       // sm_100 family
     int num_sms = 0;
     bool attr_set[kNumKernels] = {};
+    int max_pairs[kNumKernels] = {};   // co-resident CTA pairs of a pair kernel
 };
 
 std::mutex g_dev_mu;
@@ -287,14 +315,41 @@ bi_status_t encode_operand(CUtensorMap *map, const void *base, bool fp8, int64_t
 bi_status_t ensure_kernel_attr(bi_plan_s *plan, DeviceInfo *d)
 {
     std::lock_guard<std::mutex> lock(g_dev_mu);
-    if (!d->attr_set[plan->kernel_index]) {
+    const int ki = plan->kernel_index;
+    if (!d->attr_set[ki]) {
         if (cudaFuncSetAttribute(reinterpret_cast<const void *>(plan->kernel->fn),
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  plan->kernel->smem) != cudaSuccess)
             return BI_ERR_CUDA;
-        d->attr_set[plan->kernel_index] = true;
+        if (plan->kernel->pair) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(2 * (d->num_sms / 2));
+            cfg.blockDim = dim3(bi::kThreads);
+            cfg.dynamicSmemBytes = plan->kernel->smem;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, reinterpret_cast<const void *>(plan->kernel->fn),
+                                               &cfg) != cudaSuccess ||
+                clusters < 1) {
+                cudaGetLastError();
+                clusters = d->num_sms / 2;
+            }
+            d->max_pairs[ki] = clusters;
+        }
+        d->attr_set[ki] = true;
     }
     return BI_OK;
+}
+
+int pair_grid_limit(const bi_plan_s *plan, const DeviceInfo *d)
+{
+    return d->max_pairs[plan->kernel_index] > 0 ? d->max_pairs[plan->kernel_index] : d->num_sms / 2;
 }
 
 bi_status_t launch_zero(void *C, int64_t ldc, int64_t rows, int64_t n, cudaStream_t stream)
@@ -382,13 +437,46 @@ GemmParams base_params(const bi_plan_s *plan, int64_t rows, void *C, int64_t ldc
     return p;
 }
 
-bi_status_t launch_main(const bi_plan_s *plan, const CUtensorMap &ta, const CUtensorMap &tb,
-                        const GemmParams &p, int grid, cudaStream_t stream)
+// Launch the plan's kernel.  `units` is the number of work tiles; a one-CTA kernel gets
+// min(units, #SMs) CTAs, a pair kernel min(units, co-resident pairs) clusters of two CTAs.
+bi_status_t launch_main(const bi_plan_s *plan, const DeviceInfo *d, const CUtensorMap &ta,
+                        const CUtensorMap &tb, const GemmParams &p, int64_t units,
+                        cudaStream_t stream)
 {
-    if (grid < 1)
-        grid = 1;
-    plan->kernel->fn<<<grid, bi::kThreads, plan->kernel->smem, stream>>>(ta, tb, p);
-    return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+    if (units < 1)
+        units = 1;
+    if (!plan->kernel->pair) {
+        const int grid = static_cast<int>(units < d->num_sms ? units : d->num_sms);
+        plan->kernel->fn<<<grid, plan->kernel->threads, plan->kernel->smem, stream>>>(ta, tb, p);
+        return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+    }
+    const int lim = pair_grid_limit(plan, d);
+    const int pairs = static_cast<int>(units < lim ? units : lim);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(bi::kThreads);
+    cfg.dynamicSmemBytes = plan->kernel->smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, plan->kernel->fn, ta, tb, p);
+    return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+// Rows of A one TMA box covers and rows of B one box covers, for this plan and M.
+int a_box_rows_for(const bi_plan_s *plan, int64_t M)
+{
+    return plan->kernel->pair ? 128 : dense_a_box_rows(M, plan->kernel->bm);
+}
+
+int b_box_rows_for(const bi_plan_s *plan)
+{
+    return plan->kernel->pair ? plan->kernel->bn / 2 : plan->kernel->bn;
 }
 
 } // namespace
@@ -465,7 +553,7 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     if (N > INT32_MAX / 2 || K > INT32_MAX / 2 || N * num_experts > INT32_MAX / 2)
         return BI_ERR_UNSUPPORTED_SHAPE;
     const bool fp8 = dtype == BI_DTYPE_E4M3_BLOCKSCALED;
-    const TileChoice tile = choose_tile(N, K, dtype);
+    const TileChoice tile = choose_tile(N, K, dtype, num_experts);
     const int chunk_elems = fp8 ? 128 : 64;
     const int kc = (K > 0 && K % chunk_elems == 0) ? preferred_chunks(tile.bn) : 1;
     const KernelEntry *k = find_kernel(tile.bm, tile.bn, kc, fp8, num_experts > 1);
@@ -516,7 +604,7 @@ bi_status_t bi_gemm_plan_describe(bi_plan_t plan, bi_plan_info_t *info)
     info->block_m = plan->kernel->bm;
     info->block_n = plan->kernel->bn;
     info->block_k = (fp8 ? 128 : 64) * plan->kernel->kc;
-    info->cta_group = 1;
+    info->cta_group = plan->kernel->pair ? 2 : 1;
     info->mma_m = plan->kernel->bm;
     info->mma_n = plan->kernel->bn;
     info->mma_k = fp8 ? 32 : 16;
@@ -524,7 +612,7 @@ bi_status_t bi_gemm_plan_describe(bi_plan_t plan, bi_plan_info_t *info)
     info->stages = g.sb;
     info->stages_a = g.sa;
     info->k_order_id = 0;
-    info->threads_per_cta = bi::kThreads;
+    info->threads_per_cta = plan->kernel->threads;
     info->smem_bytes = plan->kernel->smem;
     const int nacc = fp8 ? ((512 / plan->kernel->bn) < 8 ? (512 / plan->kernel->bn) : 8) : 2;
     int cols = 32;
@@ -586,10 +674,10 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
     if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
         return st;
     CUtensorMap ta, tb;
-    const int a_rows = dense_a_box_rows(M, plan->kernel->bm);
+    const int a_rows = a_box_rows_for(plan, M);
     if ((st = encode_operand(&ta, A, fp8, plan->k, M, lda, a_rows, plan->kernel->kc)) != BI_OK)
         return st;
-    if ((st = encode_operand(&tb, B, fp8, plan->k, plan->n, ldb, plan->kernel->bn, plan->kernel->kc)) != BI_OK)
+    if ((st = encode_operand(&tb, B, fp8, plan->k, plan->n, ldb, b_box_rows_for(plan), plan->kernel->kc)) != BI_OK)
         return st;
     GemmParams p = base_params(plan, M, C, ldc, status);
     if (!set_rows(&p, plan, a_rows))
@@ -598,8 +686,7 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
     p.ld_sa = ld_sa;
     p.scale_b = scale_b;
     const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-    const int grid = static_cast<int>(tiles < d->num_sms ? tiles : d->num_sms);
-    return launch_main(plan, ta, tb, p, grid, stream);
+    return launch_main(plan, d, ta, tb, p, tiles, stream);
 }
 
 bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *A, int64_t lda,
@@ -629,17 +716,19 @@ bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *
     if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
         return st;
     CUtensorMap ta, tb;
-    if ((st = encode_operand(&ta, A, false, plan->k, total_rows, lda, plan->kernel->bm, plan->kernel->kc)) != BI_OK)
+    const int a_rows = plan->kernel->pair ? 128 : plan->kernel->bm;
+    if ((st = encode_operand(&ta, A, false, plan->k, total_rows, lda, a_rows, plan->kernel->kc)) != BI_OK)
         return st;
-    if ((st = encode_operand(&tb, B, false, plan->k, plan->n * plan->experts, ldb, plan->kernel->bn, plan->kernel->kc)) != BI_OK)
+    if ((st = encode_operand(&tb, B, false, plan->k, plan->n * plan->experts, ldb, b_box_rows_for(plan),
+                             plan->kernel->kc)) != BI_OK)
         return st;
     GemmParams p = base_params(plan, total_rows, C, ldc, status);
+    (void)set_rows(&p, plan, a_rows);
     p.offsets = expert_offsets;
     // Upper bound on the tile count without reading the offsets: sum_e ceil(len_e/BM) is at
     // most total_rows/BM + E.
     const int64_t max_tiles = (total_rows / plan->kernel->bm + plan->experts) * p.num_n_blocks;
-    const int grid = static_cast<int>(max_tiles < d->num_sms ? max_tiles : d->num_sms);
-    return launch_main(plan, ta, tb, p, grid, stream);
+    return launch_main(plan, d, ta, tb, p, max_tiles, stream);
 }
 
 bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M, const void *A_host, int64_t lda,
@@ -744,10 +833,10 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
         if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
             return st;
         CUtensorMap ta, tb;
-        const int a_rows = dense_a_box_rows(M, plan->kernel->bm);
+        const int a_rows = a_box_rows_for(plan, M);
         if ((st = encode_operand(&ta, A_dev, fp8, plan->k, M, lda, a_rows, plan->kernel->kc)) != BI_OK)
             return st;
-        if ((st = encode_operand(&tb, B, fp8, plan->k, plan->n, ldb, plan->kernel->bn, plan->kernel->kc)) != BI_OK)
+        if ((st = encode_operand(&tb, B, fp8, plan->k, plan->n, ldb, b_box_rows_for(plan), plan->kernel->kc)) != BI_OK)
             return st;
         GemmParams p = base_params(plan, M, C_dev, ldc, status);
         if (!set_rows(&p, plan, a_rows))
@@ -756,8 +845,7 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
         p.ld_sa = fp8 ? ld_sa : 0;
         p.scale_b = fp8 ? scale_b : nullptr;
         const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-        const int grid = static_cast<int>(tiles < d->num_sms ? tiles : d->num_sms);
-        if ((st = launch_main(plan, ta, tb, p, grid, stream)) != BI_OK)
+        if ((st = launch_main(plan, d, ta, tb, p, tiles, stream)) != BI_OK)
             return st;
     }
     if (cudaMemcpyAsync(C_host, C_dev, static_cast<size_t>(M * ldc * 2), cudaMemcpyDeviceToHost,

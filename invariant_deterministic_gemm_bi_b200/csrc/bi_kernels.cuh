@@ -48,8 +48,18 @@ namespace bi {
 constexpr int kBlockM = 128;        // largest output-tile height = largest MMA M (cta_group::1)
 constexpr int kRowBytes = 128;      // K bytes per stage per row: one 128-byte swizzle row
 constexpr int kRingBytes = 200 * 1024;   // shared memory for the two operand rings
-constexpr int kEpilogueWarps = 4;
+constexpr int kEpilogueWarps = 4;                       // bf16 (and narrow FP8) epilogue warps
 constexpr int kThreads = (2 + kEpilogueWarps) * 32;
+
+// FP8 tiles at least 64 wide split each lane quarter's columns in two halves across 8 epilogue
+// warps, so the per-K-chunk promotion keeps up with the MMAs.
+template <bool FP8, int BN>
+struct Epi {
+    static constexpr int kHalves = (FP8 && BN >= 64) ? 2 : 1;
+    static constexpr int kWarps = 4 * kHalves;
+    static constexpr int kThreads = (2 + kWarps) * 32;
+    static constexpr int kCols = BN / kHalves;             // columns per epilogue thread
+};
 constexpr int kMaxExperts = 1024;
 
 // Device status codes (the same values as bi_status_t).
@@ -201,7 +211,7 @@ __device__ __forceinline__ void store_row_chunk32(__nv_bfloat16 *crow, int col0,
 //           chunks of a tile one by one in ascending K: KC changes no bit of the result.
 // The ring depths follow from (BM, BN, KC) (see Rings).
 template <int BM, int BN, int KC, bool FP8, bool GROUPED>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     bi_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b, const GemmParams p)
 {
@@ -261,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < kNumAcc; ++a) {
             ptx::mbar_init(&accf_bar[a], 1);
-            ptx::mbar_init(&acce_bar[a], kEpilogueWarps * 32);
+            ptx::mbar_init(&acce_bar[a], Epi<FP8, BN>::kWarps * 32);
         }
         ptx::mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -514,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------------ epilogue warps
         const uint32_t q = warp & 3u;                 // TMEM lane quarter of this warp
+        const uint32_t half = (warp - 2) / 4;         // FP8 column half (0 with 4 epilogue warps)
         const bool lane_holds_row = BM == 128 || lane < 16;
         const uint32_t row_in_tile = q * kRowsPerWarp + (BM == 128 ? lane : (lane & 15u));
         const uint32_t lane_addr = (q * 32u) << 16;
@@ -553,9 +564,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ++acc_iter;
             } else {
-                float acc[BN];
+                // this thread promotes columns [col0, col0 + kCols) of its row
+                constexpr int kCols = Epi<FP8, BN>::kCols;
+                constexpr int kLoads = kCols / 32;
+                const int col0 = static_cast<int>(half) * kCols;
+                float acc[kCols];
 #pragma unroll
-                for (int jj = 0; jj < BN; ++jj)
+                for (int jj = 0; jj < kCols; ++jj)
                     acc[jj] = 0.0f;
                 const float *sa_col = p.scale_a + (row_ok ? row : 0);
                 for (int kg = 0; kg < nkg && ok; ++kg) {
@@ -578,24 +593,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                             break;
                         const uint32_t part = acc_iter % kNumAcc;
                         const float sa = row_ok ? __ldg(sa_col + static_cast<int64_t>(kb) * p.ld_sa) : 0.0f;
+                        // issue every TMEM load of this chunk, then wait once
+                        uint32_t r[kLoads][32];
 #pragma unroll
-                        for (int c = 0; c < BN / 32; ++c) {
-                            uint32_t r[32];
-                            ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + part * BN + c * 32, r);
-                            ptx::tmem_wait_ld(r);
-                            // 32 columns never straddle a 128-column scale block (n0 and c*32
-                            // are multiples of 32)
-                            const int col = tc.n0 + c * 32;
+                        for (int c = 0; c < kLoads; ++c)
+                            ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + part * BN + col0 + c * 32, r[c]);
+#pragma unroll
+                        for (int c = 0; c < kLoads; ++c)
+                            ptx::tmem_wait_ld(r[c]);
+                        ptx::tc_fence_before_sync();
+                        ptx::mbar_arrive(&acce_bar[part]);   // the partial buffer is free again
+#pragma unroll
+                        for (int c = 0; c < kLoads; ++c) {
+                            // 32 columns never straddle a 128-column scale block (n0, col0 and
+                            // c*32 are multiples of 32)
+                            const int col = tc.n0 + col0 + c * 32;
                             const float sb = col < p.n
                                                  ? __ldg(p.scale_b + static_cast<int64_t>(col >> 7) * p.kb_scale + kb)
                                                  : 0.0f;
                             const float s = sa * sb;
 #pragma unroll
                             for (int jj = 0; jj < 32; ++jj)
-                                acc[c * 32 + jj] = fmaf(__uint_as_float(r[jj]), s, acc[c * 32 + jj]);
+                                acc[c * 32 + jj] = fmaf(__uint_as_float(r[c][jj]), s, acc[c * 32 + jj]);
                         }
-                        ptx::tc_fence_before_sync();
-                        ptx::mbar_arrive(&acce_bar[part]);
                         ++acc_iter;
                     }
                 }
@@ -603,12 +623,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 if (row_ok) {
 #pragma unroll
-                    for (int c = 0; c < BN / 32; ++c) {
+                    for (int c = 0; c < kLoads; ++c) {
                         float v[32];
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj)
                             v[jj] = acc[c * 32 + jj];
-                        store_row_chunk32(crow, tc.n0 + c * 32, p.n, v);
+                        store_row_chunk32(crow, tc.n0 + col0 + c * 32, p.n, v);
                     }
                 }
             }

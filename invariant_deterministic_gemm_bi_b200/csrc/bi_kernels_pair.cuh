@@ -1,0 +1,418 @@
+// bi_kernels_pair.cuh -- the GEMM on a CTA pair (tcgen05 cta_group::2) for wide tiles.
+//
+// A cluster of two CTAs computes a 256 x BN output tile with one MMA stream: CTA r of the pair
+// holds rows [128 r, 128 r + 128) of the tile's A rows and rows [r BN/2, (r+1) BN/2) of its B
+// rows in its own shared memory; one thread of the leader CTA (rank 0) issues
+// tcgen05.mma.cta_group::2 with M = 256, N = BN, and each CTA's tensor memory receives its own
+// 128 output rows.  Each SM therefore reads only half of B per MMA, which halves the
+// shared-memory traffic per FLOP of a one-CTA 128 x BN tile.
+//
+// The batch-invariance argument is the one of bi_kernels.cuh: the pair owns the whole K range of
+// its tile, the K chunks are walked in ascending order, and the MMA instruction shape, the tile
+// and the K order are fixed by the plan from (N, K, dtype).  Which CTA of the pair (and which
+// half of the 256 rows) a row lands in depends on M; the arithmetic per row does not.
+//
+// Barriers (every CTA has the same layout):
+//   full[s]      leader only: the four TMA loads of group s (A and B of both CTAs) landed.  The
+//                leader arms it with both CTAs' bytes; the peer's loads complete on it remotely.
+//   consumed[s]  per CTA: the MMAs of group s completed (the leader commits to both CTAs).
+//   accf[a]      per CTA: tile accumulator a is ready (bf16), committed to both CTAs.
+//   acce[a]      leader only: both CTAs' epilogues are done with accumulator / partial a
+//                (8 arrivals: one per epilogue warp of each CTA).
+// No TMA load uses cluster multicast: every CTA loads its own boxes.
+#pragma once
+
+#include "bi_kernels.cuh"
+
+namespace bi {
+
+template <int BN, int KC>
+struct PairRings {
+    static constexpr int kAChunkBytes = 128 * kRowBytes;        // one CTA's 128 A rows
+    static constexpr int kBChunkBytes = (BN / 2) * kRowBytes;   // one CTA's half of the B rows
+    static constexpr int kABytes = KC * kAChunkBytes;
+    static constexpr int kBBytes = KC * kBChunkBytes;
+    static constexpr int kStages0 = kRingBytes / (kABytes + kBBytes);
+    static constexpr int kStages = kStages0 > kMaxSB ? kMaxSB : kStages0;
+    static_assert(kStages >= 2, "pair ring depth");
+};
+
+// BN      : output columns per pair tile = MMA N (128 or 256; FP8 128)
+// KC      : 128-byte K chunks per pipeline stage (1 or 2)
+template <int BN, int KC, bool FP8, bool GROUPED>
+__global__ void __launch_bounds__(kThreads, 1)
+    bi_gemm_kernel_pair(const __grid_constant__ CUtensorMap tmap_a,
+                        const __grid_constant__ CUtensorMap tmap_b, const GemmParams p)
+{
+    static_assert(BN == 128 || BN == 256, "pair tiles are 128 or 256 wide");
+    static_assert(!FP8 || BN == 128, "FP8 keeps BN fp32 accumulators per thread");
+    static_assert(!(FP8 && GROUPED), "grouped FP8 is not built");
+    static_assert(KC == 1 || KC == 2, "1 or 2 chunks per stage");
+    using R = PairRings<BN, KC>;
+    constexpr int S = R::kStages;
+    constexpr int kPairRows = 256;                       // tile height = MMA M
+    constexpr int kElemsPerRow = FP8 ? 128 : 64;
+    constexpr int kMmaK = FP8 ? 32 : 16;
+    constexpr int kMmaPerChunk = kElemsPerRow / kMmaK;   // 4
+    constexpr int kBytesPerMmaK = kMmaK * (FP8 ? 1 : 2); // 32
+    constexpr int kNumAcc = FP8 ? ((512 / BN) < 8 ? (512 / BN) : 8) : 2;
+    constexpr uint32_t kTmemCols = kNumAcc * BN <= 128 ? 128 : kNumAcc * BN <= 256 ? 256 : 512;
+    static_assert(kNumAcc * BN <= 512, "TMEM holds 512 columns");
+    static_assert(!FP8 || kNumAcc >= 2 * KC, "FP8 needs two groups of partial buffers");
+    static_assert(!FP8 || kNumAcc / KC < S, "the FP8 epilogue tracks partials on the consumed ring");
+    constexpr uint32_t kIdesc = FP8 ? ptx::idesc_e4m3(kPairRows, BN) : ptx::idesc_bf16(kPairRows, BN);
+    constexpr uint32_t kGroupBytesBoth = 2u * (R::kABytes + R::kBBytes);
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *smem_a = smem;
+    uint8_t *smem_b = smem + S * R::kABytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kRingBytes);
+    uint64_t *full = bars;
+    uint64_t *consumed = full + kMaxSB;
+    uint64_t *accf_bar = consumed + kMaxSB;
+    uint64_t *acce_bar = accf_bar + 8;
+    uint64_t *drain_bar = acce_bar + 8;
+    uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(drain_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
+    int32_t *grp_prefix = reinterpret_cast<int32_t *>(tmem_base_smem + 4);
+    int32_t *grp_offs = grp_prefix + (GROUPED ? (kMaxExperts + 1) : 0);
+
+    const uint32_t warp = ptx::warp_id();
+    const uint32_t lane = ptx::lane_id();
+    const uint32_t rank = ptx::cluster_ctarank();        // 0 = leader, 1 = peer
+    const int pair = static_cast<int>(ptx::cluster_id_x());
+    const int npairs = static_cast<int>(ptx::num_clusters_x());
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kMaxSB; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&consumed[s], 1);
+        }
+        for (int a = 0; a < 8; ++a) {
+            ptx::mbar_init(&accf_bar[a], 1);
+            ptx::mbar_init(&acce_bar[a], 2 * kEpilogueWarps);
+        }
+        ptx::mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        ptx::fence_mbarrier_init();
+        ptx::prefetch_tmap(&tmap_a);
+        ptx::prefetch_tmap(&tmap_b);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_pair(tmem_base_smem, kTmemCols);
+        ptx::tmem_relinquish_alloc_permit_pair();
+    }
+
+    __shared__ int32_t s_num_tiles;
+    if constexpr (GROUPED) {
+        __shared__ int s_bad;
+        if (threadIdx.x == 0)
+            s_bad = 0;
+        __syncthreads();
+        const int E = p.num_experts;
+        for (int e = threadIdx.x; e <= E; e += blockDim.x)
+            grp_offs[e] = p.offsets[e];
+        __syncthreads();
+        for (int e = threadIdx.x; e < E; e += blockDim.x)
+            if (grp_offs[e + 1] < grp_offs[e])
+                s_bad = 1;
+        if (threadIdx.x == 0 && (grp_offs[0] != 0 || grp_offs[E] != p.rows))
+            s_bad = 1;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int32_t acc = 0;
+            if (!s_bad) {
+                for (int e = 0; e < E; ++e) {
+                    grp_prefix[e] = acc;
+                    const int mb = (grp_offs[e + 1] - grp_offs[e] + kPairRows - 1) / kPairRows;
+                    acc += mb * p.num_n_blocks;
+                }
+            } else if (blockIdx.x == 0) {
+                atomicCAS(p.status, 0, kStatusBadOffsets);
+            }
+            grp_prefix[E] = acc;
+            s_num_tiles = acc;
+        }
+    } else {
+        if (threadIdx.x == 0)
+            s_num_tiles = p.num_m_blocks * p.num_n_blocks;
+    }
+
+    // Both CTAs' barriers are initialised and the pair's tensor memory is allocated before any
+    // CTA touches the other's shared memory.
+    ptx::tc_fence_before_sync();
+    __syncwarp();
+    ptx::cluster_sync();
+    ptx::tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_base_smem;
+    const int num_tiles = s_num_tiles;
+
+    auto tile_at = [&](int t) -> TileCoord {
+        if constexpr (GROUPED)
+            return grouped_tile(p, kPairRows, BN, t, grp_prefix, grp_offs);
+        else
+            return dense_tile(p, kPairRows, BN, t);
+    };
+
+    const int nkb = p.num_k_blocks;
+    const int nkg = (nkb + KC - 1) / KC;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer (both)
+        if (lane == 0) {
+            const uint64_t pol = ptx::policy_evict_normal();
+            const uint32_t full0_leader = ptx::mapa_shared(ptx::smem_u32(&full[0]), 0);
+            int s = 0, j = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += npairs) {
+                const TileCoord tc = tile_at(t);
+                const int a_row = tc.m0 + 128 * static_cast<int>(rank);
+                const int b_row = tc.b_row0 + (BN / 2) * static_cast<int>(rank);
+                for (int kg = 0; kg < nkg; ++kg, ++j) {
+                    if (!ptx::mbar_wait(&consumed[s], ph ^ 1u, p.timeout_cycles, abort_flag)) {
+                        record_failure(p, abort_flag, kStatusTimeout);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar = full0_leader + s * 8;
+                    if (!(j == 0 && (p.debug_flags & 1u) && rank == 0)) {   // fault injection skips
+                        if (rank == 0)                                        // the leader's first group
+                            ptx::mbar_arrive_expect_tx(&full[s], kGroupBytesBoth);
+                        if constexpr (KC == 1) {
+                            ptx::tma_load_2d_pair(smem_a + s * R::kABytes, &tmap_a, bar,
+                                                  kg * kElemsPerRow, a_row, pol);
+                            ptx::tma_load_2d_pair(smem_b + s * R::kBBytes, &tmap_b, bar,
+                                                  kg * kElemsPerRow, b_row, pol);
+                        } else {
+                            ptx::tma_load_3d_pair(smem_a + s * R::kABytes, &tmap_a, bar, 0, a_row,
+                                                  kg * KC, pol);
+                            ptx::tma_load_3d_pair(smem_b + s * R::kBBytes, &tmap_b, bar, 0, b_row,
+                                                  kg * KC, pol);
+                        }
+                    }
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            // Drain (leader): the loads of the last S groups of both CTAs land on its barriers.
+            // On the normal path they were all consumed; after a timeout the wait is bounded.
+            if (rank == 0) {
+                const bool skipped = (p.debug_flags & 1u) != 0;
+                for (int i = j > S ? j - S : 0; i < j; ++i)
+                    if (!(i == 0 && skipped))
+                        ptx::mbar_wait(&full[i % S], static_cast<uint32_t>(i / S) & 1u,
+                                       p.timeout_cycles, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer (leader)
+        if (lane == 0 && rank == 0) {
+            const uint32_t consumed_peer0 = ptx::mapa_shared(ptx::smem_u32(&consumed[0]), 1);
+            const uint32_t accf_peer0 = ptx::mapa_shared(ptx::smem_u32(&accf_bar[0]), 1);
+            const uint64_t a_desc0 = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_a));
+            const uint64_t b_desc0 = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_b));
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t acc_iter = 0;   // bf16: tiles; FP8: K chunks
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += npairs) {
+                uint32_t d_tmem = 0;
+                if (!FP8) {
+                    const uint32_t a = acc_iter % kNumAcc;
+                    const uint32_t par = (acc_iter / kNumAcc) & 1u;
+                    if (!ptx::mbar_wait(&acce_bar[a], par ^ 1u, p.timeout_cycles, abort_flag)) {
+                        record_failure(p, abort_flag, kStatusTimeout);
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after_sync();
+                    d_tmem = tmem_base + a * BN;
+                }
+                for (int kg = 0; kg < nkg; ++kg) {
+                    if (!ptx::mbar_wait(&full[s], ph, p.timeout_cycles, abort_flag)) {
+                        record_failure(p, abort_flag, kStatusTimeout);
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after_sync();
+                    const uint64_t a_slot = a_desc0 + ((s * R::kABytes) >> 4);
+                    const uint64_t b_slot = b_desc0 + ((s * R::kBBytes) >> 4);
+#pragma unroll
+                    for (int c = 0; c < KC; ++c) {
+                        const int chunk = kg * KC + c;
+                        if (chunk >= nkb)
+                            break;
+                        if (FP8) {
+                            const uint32_t part = acc_iter % kNumAcc;
+                            const uint32_t par = (acc_iter / kNumAcc) & 1u;
+                            if (!ptx::mbar_wait(&acce_bar[part], par ^ 1u, p.timeout_cycles, abort_flag)) {
+                                record_failure(p, abort_flag, kStatusTimeout);
+                                ok = false;
+                                break;
+                            }
+                            ptx::tc_fence_after_sync();
+                            d_tmem = tmem_base + part * BN;
+                            ++acc_iter;
+                        }
+                        const uint64_t a_desc = a_slot + ((c * R::kAChunkBytes) >> 4);
+                        const uint64_t b_desc = b_slot + ((c * R::kBChunkBytes) >> 4);
+#pragma unroll
+                        for (int q = 0; q < kMmaPerChunk; ++q) {
+                            const uint64_t step = static_cast<uint64_t>((q * kBytesPerMmaK) >> 4);
+                            const uint32_t accumulate = FP8 ? (q > 0) : ((chunk > 0) || (q > 0));
+                            if (FP8)
+                                ptx::mma_e4m3_ss_pair(d_tmem, a_desc + step, b_desc + step, kIdesc, accumulate);
+                            else
+                                ptx::mma_bf16_ss_pair(d_tmem, a_desc + step, b_desc + step, kIdesc, accumulate);
+                        }
+                    }
+                    if (!ok)
+                        break;
+                    // frees slot s in both CTAs (and marks FP8 partials ready in both)
+                    ptx::mma_commit_pair(ptx::smem_u32(&consumed[s]));
+                    ptx::mma_commit_pair(consumed_peer0 + s * 8);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                if (!FP8) {
+                    const uint32_t a = acc_iter % kNumAcc;
+                    ptx::mma_commit_pair(ptx::smem_u32(&accf_bar[a]));
+                    ptx::mma_commit_pair(accf_peer0 + a * 8);
+                    ++acc_iter;
+                }
+            }
+            ptx::mma_commit_pair(ptx::smem_u32(drain_bar));
+            ptx::mbar_wait(drain_bar, 0, p.timeout_cycles, nullptr);
+        }
+    } else {
+        // ------------------------------------------------------------------ epilogue (both)
+        const uint32_t q = warp & 3u;
+        const uint32_t row_in_tile = 128 * rank + q * 32 + lane;
+        const uint32_t lane_addr = (q * 32u) << 16;
+        const uint32_t acce_leader0 = ptx::mapa_shared(ptx::smem_u32(&acce_bar[0]), 0);
+        auto release = [&](uint32_t idx) {   // this warp is done with TMEM buffer idx
+            ptx::tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0)
+                    ptx::mbar_arrive(&acce_bar[idx]);
+                else
+                    ptx::mbar_arrive_cluster(acce_leader0 + idx * 8);
+            }
+        };
+        uint32_t acc_iter = 0;
+        int gs = 0;
+        uint32_t gph = 0;
+        bool ok = true;
+        for (int t = pair; t < num_tiles && ok; t += npairs) {
+            const TileCoord tc = tile_at(t);
+            const int row = tc.m0 + static_cast<int>(row_in_tile);
+            const bool row_ok = row < tc.row_end;
+            __nv_bfloat16 *crow = p.c + static_cast<int64_t>(row) * p.ldc;
+            if constexpr (!FP8) {
+                const uint32_t a = acc_iter % kNumAcc;
+                const uint32_t par = (acc_iter / kNumAcc) & 1u;
+                if (!ptx::mbar_wait(&accf_bar[a], par, p.timeout_cycles, abort_flag)) {
+                    record_failure(p, abort_flag, kStatusTimeout);
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after_sync();
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + a * BN + c * 32, r);
+                    ptx::tmem_wait_ld(r);
+                    if (c == BN / 32 - 1)
+                        release(a);
+                    float v[32];
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        v[jj] = __uint_as_float(r[jj]);
+                    if (row_ok)
+                        store_row_chunk32(crow, tc.n0 + c * 32, p.n, v);
+                }
+                ++acc_iter;
+            } else {
+                float acc[BN];
+#pragma unroll
+                for (int jj = 0; jj < BN; ++jj)
+                    acc[jj] = 0.0f;
+                const float *sa_col = p.scale_a + (row_ok ? row : 0);
+                for (int kg = 0; kg < nkg && ok; ++kg) {
+                    if (!ptx::mbar_wait(&consumed[gs], gph, p.timeout_cycles, abort_flag)) {
+                        record_failure(p, abort_flag, kStatusTimeout);
+                        ok = false;
+                        break;
+                    }
+                    if (++gs == S) {
+                        gs = 0;
+                        gph ^= 1u;
+                    }
+                    ptx::tc_fence_after_sync();
+                    for (int cc = 0; cc < KC; ++cc) {
+                        const int kb = kg * KC + cc;
+                        if (kb >= nkb)
+                            break;
+                        const uint32_t part = acc_iter % kNumAcc;
+                        const float sa = row_ok ? __ldg(sa_col + static_cast<int64_t>(kb) * p.ld_sa) : 0.0f;
+#pragma unroll
+                        for (int c = 0; c < BN / 32; ++c) {
+                            uint32_t r[32];
+                            ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + part * BN + c * 32, r);
+                            ptx::tmem_wait_ld(r);
+                            const int col = tc.n0 + c * 32;
+                            const float sb = col < p.n
+                                                 ? __ldg(p.scale_b + static_cast<int64_t>(col >> 7) * p.kb_scale + kb)
+                                                 : 0.0f;
+                            const float sc = sa * sb;
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj)
+                                acc[c * 32 + jj] = fmaf(__uint_as_float(r[jj]), sc, acc[c * 32 + jj]);
+                        }
+                        release(part);
+                        ++acc_iter;
+                    }
+                }
+                if (!ok)
+                    break;
+                if (row_ok) {
+#pragma unroll
+                    for (int c = 0; c < BN / 32; ++c) {
+                        float v[32];
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            v[jj] = acc[c * 32 + jj];
+                        store_row_chunk32(crow, tc.n0 + c * 32, p.n, v);
+                    }
+                }
+            }
+        }
+    }
+
+    // Nobody leaves while its pair may still touch its shared or tensor memory.
+    ptx::tc_fence_before_sync();
+    __syncwarp();
+    ptx::cluster_sync();
+    if (warp == 1) {
+        ptx::tc_fence_after_sync();
+        ptx::tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
+}
+
+template <int BN, int KC, bool FP8, bool GROUPED>
+constexpr int smem_bytes_for_pair()
+{
+    return 1024 + kRingBytes + 1024 + (GROUPED ? 2 * (kMaxExperts + 1) * 4 : 0);
+}
+
+} // namespace bi

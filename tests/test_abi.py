@@ -43,16 +43,16 @@ def test_plan_describe_is_m_free_and_sane():
                           (7168, 7168, 1, 1), (2048, 7168, 0, 64), (256, 512, 0, 1), (5, 3, 0, 1)]:
         info = bg.bi_gemm_plan_describe(bg.bi_gemm_plan(N, K, dt, E))
         assert info["n"] == N and info["k"] == K and info["num_experts"] == E
-        assert info["k_order_id"] == 0 and info["block_m"] in (64, 128)
+        assert info["k_order_id"] == 0 and info["block_m"] in (64, 128, 256)
         assert info["mma_m"] == info["block_m"] and 2 <= info["stages_a"] <= info["stages"]
+        assert info["cta_group"] == (2 if info["block_m"] == 256 else 1)
         assert info["block_k"] * (1 if dt == 1 else 2) in (128, 256, 512)
         assert info["mma_n"] == info["block_n"] and info["block_n"] % 32 == 0
         assert info["smem_bytes"] <= 232448
         assert info["tmem_columns"] <= 512
-    # grouped plans share the dense plan's tile configuration
-    d = bg.bi_gemm_plan_describe(bg.bi_gemm_plan(2048, 7168, 0, 1))
+    # grouped plans run on one CTA (an expert's segment is often a few rows long)
     g = bg.bi_gemm_plan_describe(bg.bi_gemm_plan(2048, 7168, 0, 64))
-    assert d["block_n"] == g["block_n"] and d["mma_n"] == g["mma_n"]
+    assert g["cta_group"] == 1 and g["block_m"] == 128
 
 
 def test_plan_is_the_same_in_a_fresh_process():

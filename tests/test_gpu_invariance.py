@@ -218,7 +218,13 @@ def test_moe_adversarial_routings(pattern):
         one = inputs.routing_from_assignment(np.array([e]), E)
         C1 = moe_outputs(plan, B, tokens[i:i + 1], one)
         assert torch.equal(C1[0], C[i]), f"{pattern}: row {i}"
-    # and the same as a dense call with that expert's weights
-    f = Dense(B[3].contiguous()) if pattern == "all_one_expert" else None
-    if f is not None:
-        assert torch.equal(f(tokens).view(torch.int16), C)
+    # and the same as a dense call with that expert's weights, where the two plans share a tile
+    if pattern == "all_one_expert":
+        f = Dense(B[3].contiguous())
+        dense_info = bg.bi_gemm_plan_describe(f.plan)
+        grouped_info = bg.bi_gemm_plan_describe(plan)
+        same = {k: v for k, v in dense_info.items() if k != "num_experts"} == \
+            {k: v for k, v in grouped_info.items() if k not in ("num_experts", "smem_bytes")} | \
+            {"smem_bytes": dense_info["smem_bytes"]}
+        if same:
+            assert torch.equal(f(tokens).view(torch.int16), C)
