@@ -49,7 +49,8 @@ struct KernelEntry {
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, GR>,                                           \
                 bi::smem_bytes_for<BM, BN, KC, F8, GR>()}
 #define BI_PAIR(BN, KC, F8, GR)                                                                    \
-    KernelEntry{bi::kThreads, 256, BN, KC, F8, GR, true, &bi::bi_gemm_kernel_pair<BN, KC, F8, GR>,  \
+    KernelEntry{bi::Epi<F8, BN>::kThreads, 256, BN, KC, F8, GR, true,                              \
+                &bi::bi_gemm_kernel_pair<BN, KC, F8, GR>,                                          \
                 bi::smem_bytes_for_pair<BN, KC, F8, GR>()}
 
 // Narrow tiles (BN <= 64) run on one CTA; wide ones (BN >= 128) on a CTA pair.  Every tile comes
@@ -329,7 +330,7 @@ bi_status_t ensure_kernel_attr(bi_plan_s *plan, DeviceInfo *d)
             attr[0].val.clusterDim.y = 1;
             attr[0].val.clusterDim.z = 1;
             cfg.gridDim = dim3(2 * (d->num_sms / 2));
-            cfg.blockDim = dim3(bi::kThreads);
+            cfg.blockDim = dim3(plan->kernel->threads);
             cfg.dynamicSmemBytes = plan->kernel->smem;
             cfg.attrs = attr;
             cfg.numAttrs = 1;
@@ -405,6 +406,8 @@ bool set_rows(GemmParams *p, const bi_plan_s *plan, int a_rows)
 {
     const RingGeom g = ring_geometry(plan->kernel, a_rows);
     p->a_box_rows = a_rows;
+    // the peer CTA of a pair has A rows to load unless the whole problem fits in 128 rows
+    p->pair_a1 = (plan->kernel->grouped || p->rows > 128) ? 1 : 0;
     p->sa = g.sa;
     p->sb = g.sb;
     p->a_stride = g.a_stride;
@@ -459,7 +462,7 @@ bi_status_t launch_main(const bi_plan_s *plan, const DeviceInfo *d, const CUtens
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2 * pairs);
-    cfg.blockDim = dim3(bi::kThreads);
+    cfg.blockDim = dim3(plan->kernel->threads);
     cfg.dynamicSmemBytes = plan->kernel->smem;
     cfg.stream = stream;
     cfg.attrs = attr;
@@ -468,10 +471,11 @@ bi_status_t launch_main(const bi_plan_s *plan, const DeviceInfo *d, const CUtens
     return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
-// Rows of A one TMA box covers and rows of B one box covers, for this plan and M.
+// Rows of A one TMA box covers and rows of B one box covers, for this plan and M.  A pair CTA
+// owns 128 rows of a tile; a dense problem smaller than that boxes only its roundup(M, 8) rows.
 int a_box_rows_for(const bi_plan_s *plan, int64_t M)
 {
-    return plan->kernel->pair ? 128 : dense_a_box_rows(M, plan->kernel->bm);
+    return dense_a_box_rows(M, plan->kernel->pair ? 128 : plan->kernel->bm);
 }
 
 int b_box_rows_for(const bi_plan_s *plan)

@@ -79,6 +79,7 @@ struct GemmParams {
     int32_t sa, sb;          // ring depths in groups (2..kMaxSA, sa..kMaxSB)
     uint32_t a_stride;       // bytes between A slots (KC * a_box_rows * 128)
     uint32_t b_offset;       // byte offset of the B ring in the ring region
+    int32_t pair_a1;         // CTA pair: 1 if the peer CTA loads A rows (the problem has > 128)
     __nv_bfloat16 *c;
     int64_t ldc;
     const float *scale_a;    // FP8: [kb][ld_sa]
@@ -202,6 +203,30 @@ __device__ __forceinline__ void store_row_chunk32(__nv_bfloat16 *crow, int col0,
 //
 // BM      : output rows per tile = MMA M (64 or 128).  With M = 64 the accumulator's row i sits
 //           in TMEM lane (i % 16) + 32 * (i / 16), so each epilogue warp owns 16 rows.
+// FP8: the scales one epilogue thread needs for the KC chunks of group kg -- scale_a of its row
+// and scale_b of each of its 32-column blocks (32 columns never straddle a 128-column scale
+// block: the tile origin, the thread's first column and c * 32 are all multiples of 32).  Chunks
+// past the end of K and columns past N read nothing and get 0.
+template <int KC, int kLoads>
+__device__ __forceinline__ void load_group_scales(const GemmParams &p, const float *sa_col, bool row_ok,
+                                                  int col_first, int kg, int nkb, float (&sa)[KC],
+                                                  float (&sb)[KC][kLoads])
+{
+#pragma unroll
+    for (int cc = 0; cc < KC; ++cc) {
+        const int kb = kg * KC + cc;
+        const bool kb_ok = kb < nkb;
+        sa[cc] = (row_ok && kb_ok) ? __ldg(sa_col + static_cast<int64_t>(kb) * p.ld_sa) : 0.0f;
+#pragma unroll
+        for (int c = 0; c < kLoads; ++c) {
+            const int col = col_first + c * 32;
+            sb[cc][c] = (kb_ok && col < p.n)
+                            ? __ldg(p.scale_b + static_cast<int64_t>(col >> 7) * p.kb_scale + kb)
+                            : 0.0f;
+        }
+    }
+}
+
 // BN      : output columns per tile = MMA N (multiple of 32, <= 256; FP8 <= 128)
 // FP8     : e4m3 operands with fp32 block scales (else bf16)
 // GROUPED : MoE grouped layout (bf16 only)
@@ -467,22 +492,19 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                     ptx::tc_fence_after_sync();
                     const uint64_t a_slot = a_desc0 + ((sa * p.a_stride) >> 4);
                     const uint64_t b_slot = b_desc0 + ((sb * R::kBBytes) >> 4);
-#pragma unroll
-                    for (int c = 0; c < KC; ++c) {
-                        const int chunk = kg * KC + c;
-                        if (chunk >= nkb)
-                            break;
-                        if (FP8) {
+                    // the MMAs of chunk c of this group (K chunk number `chunk` of the tile)
+                    auto issue_chunk = [&](int c, int chunk) -> bool {
+                        uint32_t d = d_tmem;
+                        if constexpr (FP8) {
                             // each K chunk's partial product goes to its own TMEM buffer
                             const uint32_t part = acc_iter % kNumAcc;
                             const uint32_t par = (acc_iter / kNumAcc) & 1u;
                             if (!ptx::mbar_wait(&acce_bar[part], par ^ 1u, p.timeout_cycles, abort_flag)) {
                                 record_failure(p, abort_flag, kStatusTimeout);
-                                ok = false;
-                                break;
+                                return false;
                             }
                             ptx::tc_fence_after_sync();
-                            d_tmem = tmem_base + part * BN;
+                            d = tmem_base + part * BN;
                             ++acc_iter;
                         }
                         const uint64_t a_desc = a_slot + ((c * a_chunk_pitch) >> 4);
@@ -491,12 +513,32 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                         for (int q = 0; q < kMmaPerStage; ++q) {
                             const uint64_t step = static_cast<uint64_t>((q * kBytesPerMmaK) >> 4);
                             // bf16: accumulate across the whole K of the tile; FP8: one K chunk
-                            const uint32_t accumulate = FP8 ? (q > 0) : ((chunk > 0) || (q > 0));
-                            if (FP8)
-                                ptx::mma_e4m3_ss(d_tmem, a_desc + step, b_desc + step, kIdesc, accumulate);
+                            const uint32_t accumulate = (q > 0) ? 1u : (FP8 ? 0u : (chunk > 0 ? 1u : 0u));
+                            if constexpr (FP8)
+                                ptx::mma_e4m3_ss(d, a_desc + step, b_desc + step, kIdesc, accumulate);
                             else
-                                ptx::mma_bf16_ss(d_tmem, a_desc + step, b_desc + step, kIdesc, accumulate);
+                                ptx::mma_bf16_ss(d, a_desc + step, b_desc + step, kIdesc, accumulate);
                         }
+                        return true;
+                    };
+                    // A full group issues its KC chunks as straight-line code: control flow
+                    // between consecutive tcgen05.mma instructions slows their issue.  Only the
+                    // last group of a tile can hold fewer chunks.
+                    const int nc = nkb - kg * KC;
+                    if (nc >= KC) {
+#pragma unroll
+                        for (int c = 0; c < KC; ++c)
+                            if (!issue_chunk(c, kg * KC + c)) {
+                                ok = false;
+                                break;
+                            }
+                    } else {
+#pragma unroll 1
+                        for (int c = 0; c < nc; ++c)
+                            if (!issue_chunk(c, kg * KC + c)) {
+                                ok = false;
+                                break;
+                            }
                     }
                     if (!ok)
                         break;
@@ -573,7 +615,13 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                 for (int jj = 0; jj < kCols; ++jj)
                     acc[jj] = 0.0f;
                 const float *sa_col = p.scale_a + (row_ok ? row : 0);
+                // the scales of group kg + 1 are loaded while group kg is promoted, so their
+                // global-memory latency stays off the per-chunk chain
+                float sa_g[KC], sb_g[KC][kLoads];
+                load_group_scales<KC, kLoads>(p, sa_col, row_ok, tc.n0 + col0, 0, nkb, sa_g, sb_g);
                 for (int kg = 0; kg < nkg && ok; ++kg) {
+                    float sa_n[KC], sb_n[KC][kLoads];
+                    load_group_scales<KC, kLoads>(p, sa_col, row_ok, tc.n0 + col0, kg + 1, nkb, sa_n, sb_n);
                     // the group's partials are ready when its consumed barrier completes; the MMA
                     // warp runs at most kNumAcc chunks (< sb groups) ahead, so the barrier cannot
                     // have moved on to the group sb later
@@ -587,12 +635,12 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                         gph ^= 1u;
                     }
                     ptx::tc_fence_after_sync();
+#pragma unroll
                     for (int cc = 0; cc < KC; ++cc) {
                         const int kb = kg * KC + cc;
                         if (kb >= nkb)
                             break;
                         const uint32_t part = acc_iter % kNumAcc;
-                        const float sa = row_ok ? __ldg(sa_col + static_cast<int64_t>(kb) * p.ld_sa) : 0.0f;
                         // issue every TMEM load of this chunk, then wait once
                         uint32_t r[kLoads][32];
 #pragma unroll
@@ -605,18 +653,19 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                         ptx::mbar_arrive(&acce_bar[part]);   // the partial buffer is free again
 #pragma unroll
                         for (int c = 0; c < kLoads; ++c) {
-                            // 32 columns never straddle a 128-column scale block (n0, col0 and
-                            // c*32 are multiples of 32)
-                            const int col = tc.n0 + col0 + c * 32;
-                            const float sb = col < p.n
-                                                 ? __ldg(p.scale_b + static_cast<int64_t>(col >> 7) * p.kb_scale + kb)
-                                                 : 0.0f;
-                            const float s = sa * sb;
+                            const float s = sa_g[cc] * sb_g[cc][c];
 #pragma unroll
                             for (int jj = 0; jj < 32; ++jj)
                                 acc[c * 32 + jj] = fmaf(__uint_as_float(r[c][jj]), s, acc[c * 32 + jj]);
                         }
                         ++acc_iter;
+                    }
+#pragma unroll
+                    for (int cc = 0; cc < KC; ++cc) {
+                        sa_g[cc] = sa_n[cc];
+#pragma unroll
+                        for (int c = 0; c < kLoads; ++c)
+                            sb_g[cc][c] = sb_n[cc][c];
                     }
                 }
                 if (!ok)

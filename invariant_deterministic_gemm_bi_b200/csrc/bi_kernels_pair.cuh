@@ -40,7 +40,7 @@ struct PairRings {
 // BN      : output columns per pair tile = MMA N (128 or 256; FP8 128)
 // KC      : 128-byte K chunks per pipeline stage (1 or 2)
 template <int BN, int KC, bool FP8, bool GROUPED>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     bi_gemm_kernel_pair(const __grid_constant__ CUtensorMap tmap_a,
                         const __grid_constant__ CUtensorMap tmap_b, const GemmParams p)
 {
@@ -61,7 +61,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     static_assert(!FP8 || kNumAcc >= 2 * KC, "FP8 needs two groups of partial buffers");
     static_assert(!FP8 || kNumAcc / KC < S, "the FP8 epilogue tracks partials on the consumed ring");
     constexpr uint32_t kIdesc = FP8 ? ptx::idesc_e4m3(kPairRows, BN) : ptx::idesc_bf16(kPairRows, BN);
-    constexpr uint32_t kGroupBytesBoth = 2u * (R::kABytes + R::kBBytes);
+    constexpr int kEpiWarps = Epi<FP8, BN>::kWarps;
+    // Bytes of one group over both CTAs: B halves always, A rows as the launch boxes them (fewer
+    // than 128 rows when the whole problem is smaller than a CTA's share; the peer loads no A
+    // at all when the problem has at most 128 rows).
+    const uint32_t a_chunk_pitch = static_cast<uint32_t>(p.a_box_rows) * kRowBytes;
+    const uint32_t group_bytes = 2u * R::kBBytes + KC * a_chunk_pitch * (p.pair_a1 ? 2u : 1u);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -92,7 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < 8; ++a) {
             ptx::mbar_init(&accf_bar[a], 1);
-            ptx::mbar_init(&acce_bar[a], 2 * kEpilogueWarps);
+            ptx::mbar_init(&acce_bar[a], 2 * kEpiWarps);
         }
         ptx::mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -180,15 +185,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t bar = full0_leader + s * 8;
                     if (!(j == 0 && (p.debug_flags & 1u) && rank == 0)) {   // fault injection skips
                         if (rank == 0)                                        // the leader's first group
-                            ptx::mbar_arrive_expect_tx(&full[s], kGroupBytesBoth);
+                            ptx::mbar_arrive_expect_tx(&full[s], group_bytes);
+                        const bool load_a = rank == 0 || p.pair_a1 != 0;
                         if constexpr (KC == 1) {
-                            ptx::tma_load_2d_pair(smem_a + s * R::kABytes, &tmap_a, bar,
-                                                  kg * kElemsPerRow, a_row, pol);
+                            if (load_a)
+                                ptx::tma_load_2d_pair(smem_a + s * R::kABytes, &tmap_a, bar,
+                                                      kg * kElemsPerRow, a_row, pol);
                             ptx::tma_load_2d_pair(smem_b + s * R::kBBytes, &tmap_b, bar,
                                                   kg * kElemsPerRow, b_row, pol);
                         } else {
-                            ptx::tma_load_3d_pair(smem_a + s * R::kABytes, &tmap_a, bar, 0, a_row,
-                                                  kg * KC, pol);
+                            if (load_a)
+                                ptx::tma_load_3d_pair(smem_a + s * R::kABytes, &tmap_a, bar, 0, a_row,
+                                                      kg * KC, pol);
                             ptx::tma_load_3d_pair(smem_b + s * R::kBBytes, &tmap_b, bar, 0, b_row,
                                                   kg * KC, pol);
                         }
@@ -242,34 +250,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tc_fence_after_sync();
                     const uint64_t a_slot = a_desc0 + ((s * R::kABytes) >> 4);
                     const uint64_t b_slot = b_desc0 + ((s * R::kBBytes) >> 4);
-#pragma unroll
-                    for (int c = 0; c < KC; ++c) {
-                        const int chunk = kg * KC + c;
-                        if (chunk >= nkb)
-                            break;
-                        if (FP8) {
+                    auto issue_chunk = [&](int c, int chunk) -> bool {
+                        uint32_t d = d_tmem;
+                        if constexpr (FP8) {
                             const uint32_t part = acc_iter % kNumAcc;
                             const uint32_t par = (acc_iter / kNumAcc) & 1u;
                             if (!ptx::mbar_wait(&acce_bar[part], par ^ 1u, p.timeout_cycles, abort_flag)) {
                                 record_failure(p, abort_flag, kStatusTimeout);
-                                ok = false;
-                                break;
+                                return false;
                             }
                             ptx::tc_fence_after_sync();
-                            d_tmem = tmem_base + part * BN;
+                            d = tmem_base + part * BN;
                             ++acc_iter;
                         }
-                        const uint64_t a_desc = a_slot + ((c * R::kAChunkBytes) >> 4);
+                        const uint64_t a_desc = a_slot + ((c * a_chunk_pitch) >> 4);
                         const uint64_t b_desc = b_slot + ((c * R::kBChunkBytes) >> 4);
 #pragma unroll
                         for (int q = 0; q < kMmaPerChunk; ++q) {
                             const uint64_t step = static_cast<uint64_t>((q * kBytesPerMmaK) >> 4);
-                            const uint32_t accumulate = FP8 ? (q > 0) : ((chunk > 0) || (q > 0));
-                            if (FP8)
-                                ptx::mma_e4m3_ss_pair(d_tmem, a_desc + step, b_desc + step, kIdesc, accumulate);
+                            const uint32_t accumulate = (q > 0) ? 1u : (FP8 ? 0u : (chunk > 0 ? 1u : 0u));
+                            if constexpr (FP8)
+                                ptx::mma_e4m3_ss_pair(d, a_desc + step, b_desc + step, kIdesc, accumulate);
                             else
-                                ptx::mma_bf16_ss_pair(d_tmem, a_desc + step, b_desc + step, kIdesc, accumulate);
+                                ptx::mma_bf16_ss_pair(d, a_desc + step, b_desc + step, kIdesc, accumulate);
                         }
+                        return true;
+                    };
+                    // straight-line MMAs for a full group; only a tile's last group can be short
+                    const int nc = nkb - kg * KC;
+                    if (nc >= KC) {
+#pragma unroll
+                        for (int c = 0; c < KC; ++c)
+                            if (!issue_chunk(c, kg * KC + c)) {
+                                ok = false;
+                                break;
+                            }
+                    } else {
+#pragma unroll 1
+                        for (int c = 0; c < nc; ++c)
+                            if (!issue_chunk(c, kg * KC + c)) {
+                                ok = false;
+                                break;
+                            }
                     }
                     if (!ok)
                         break;
@@ -296,6 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------------ epilogue (both)
         const uint32_t q = warp & 3u;
+        const uint32_t half = (warp - 2) / 4;   // FP8 column half (0 with 4 epilogue warps)
         const uint32_t row_in_tile = 128 * rank + q * 32 + lane;
         const uint32_t lane_addr = (q * 32u) << 16;
         const uint32_t acce_leader0 = ptx::mapa_shared(ptx::smem_u32(&acce_bar[0]), 0);
@@ -343,12 +366,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ++acc_iter;
             } else {
-                float acc[BN];
+                constexpr int kCols = Epi<FP8, BN>::kCols;
+                constexpr int kLoads = kCols / 32;
+                const int col0 = static_cast<int>(half) * kCols;
+                float acc[kCols];
 #pragma unroll
-                for (int jj = 0; jj < BN; ++jj)
+                for (int jj = 0; jj < kCols; ++jj)
                     acc[jj] = 0.0f;
                 const float *sa_col = p.scale_a + (row_ok ? row : 0);
+                float sa_g[KC], sb_g[KC][kLoads];   // scales of group kg, loaded one group ahead
+                load_group_scales<KC, kLoads>(p, sa_col, row_ok, tc.n0 + col0, 0, nkb, sa_g, sb_g);
                 for (int kg = 0; kg < nkg && ok; ++kg) {
+                    float sa_n[KC], sb_n[KC][kLoads];
+                    load_group_scales<KC, kLoads>(p, sa_col, row_ok, tc.n0 + col0, kg + 1, nkb, sa_n, sb_n);
                     if (!ptx::mbar_wait(&consumed[gs], gph, p.timeout_cycles, abort_flag)) {
                         record_failure(p, abort_flag, kStatusTimeout);
                         ok = false;
@@ -359,40 +389,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                         gph ^= 1u;
                     }
                     ptx::tc_fence_after_sync();
+#pragma unroll
                     for (int cc = 0; cc < KC; ++cc) {
                         const int kb = kg * KC + cc;
                         if (kb >= nkb)
                             break;
                         const uint32_t part = acc_iter % kNumAcc;
-                        const float sa = row_ok ? __ldg(sa_col + static_cast<int64_t>(kb) * p.ld_sa) : 0.0f;
+                        uint32_t r[kLoads][32];
 #pragma unroll
-                        for (int c = 0; c < BN / 32; ++c) {
-                            uint32_t r[32];
-                            ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + part * BN + c * 32, r);
-                            ptx::tmem_wait_ld(r);
-                            const int col = tc.n0 + c * 32;
-                            const float sb = col < p.n
-                                                 ? __ldg(p.scale_b + static_cast<int64_t>(col >> 7) * p.kb_scale + kb)
-                                                 : 0.0f;
-                            const float sc = sa * sb;
+                        for (int c = 0; c < kLoads; ++c)
+                            ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + part * BN + col0 + c * 32, r[c]);
+#pragma unroll
+                        for (int c = 0; c < kLoads; ++c)
+                            ptx::tmem_wait_ld(r[c]);
+                        release(part);
+#pragma unroll
+                        for (int c = 0; c < kLoads; ++c) {
+                            const float sc = sa_g[cc] * sb_g[cc][c];
 #pragma unroll
                             for (int jj = 0; jj < 32; ++jj)
-                                acc[c * 32 + jj] = fmaf(__uint_as_float(r[jj]), sc, acc[c * 32 + jj]);
+                                acc[c * 32 + jj] = fmaf(__uint_as_float(r[c][jj]), sc, acc[c * 32 + jj]);
                         }
-                        release(part);
                         ++acc_iter;
+                    }
+#pragma unroll
+                    for (int cc = 0; cc < KC; ++cc) {
+                        sa_g[cc] = sa_n[cc];
+#pragma unroll
+                        for (int c = 0; c < kLoads; ++c)
+                            sb_g[cc][c] = sb_n[cc][c];
                     }
                 }
                 if (!ok)
                     break;
                 if (row_ok) {
 #pragma unroll
-                    for (int c = 0; c < BN / 32; ++c) {
+                    for (int c = 0; c < kLoads; ++c) {
                         float v[32];
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj)
                             v[jj] = acc[c * 32 + jj];
-                        store_row_chunk32(crow, tc.n0 + c * 32, p.n, v);
+                        store_row_chunk32(crow, tc.n0 + col0 + c * 32, p.n, v);
                     }
                 }
             }
