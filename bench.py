@@ -40,6 +40,16 @@ WORKLOAD = ("decode-shaped bf16 GEMM C=A.B^T, N=4096, K=7168, M swept 1,2,4,...,
             "(9 GEMMs per step); A~N(0,1), B~N(0,1/K) in bf16")
 
 
+
+def weight_plan(N, K, dtype=None, experts=1):
+    """A plan for the benchmark's weights: they are written once before the timed region and
+    only read inside it, so every plan declares them resident (BI_PLAN_RESIDENT_WEIGHTS)."""
+    import invariant_deterministic_gemm_bi_b200 as bg
+    plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_BF16 if dtype is None else dtype, experts)
+    bg.bi_gemm_plan_set_flags(plan, bg.BI_PLAN_RESIDENT_WEIGHTS)
+    return plan
+
+
 def sweep_bytes(n=N_DEC, k=K_DEC, ms=M_SWEEP, elt=2):
     """Algorithmic bytes of one step: each operand once plus the output."""
     return sum(n * k * elt + m * k * elt + 2 * m * n for m in ms)
@@ -275,7 +285,7 @@ def main():
     Amax = inputs.bf16_gaussian((max(M_SWEEP), K_DEC), seed=seed, device=dev)
     As = {m: Amax[:m] for m in M_SWEEP}
     Cs = {m: torch.empty((m, N_DEC), dtype=torch.bfloat16, device=dev) for m in M_SWEEP}
-    plan = bg.bi_gemm_plan(N_DEC, K_DEC, bg.BI_DTYPE_BF16, 1)
+    plan = weight_plan(N_DEC, K_DEC)
     stream = torch.cuda.Stream(device=dev)
 
     def run_step(phase):
@@ -371,6 +381,8 @@ def main():
                        "l2": f"{n_copies} rotating weight copies ({n_copies * wbytes / 2**20:.0f} MiB"
                              f" > 2 x {l2 / 2**20:.0f} MiB L2)",
                        "timing": "CUDA graph replay per step, CUDA events, max over ranks",
+                       "weights": "resident (BI_PLAN_RESIDENT_WEIGHTS: B requested before the "
+                                  "previous GEMM in the stream completes)",
                        "parallelism": f"replicas x{world} (M-sharded independent problems)"},
             "tflops": tflops,
             "roofline": roofline, "clocks": clocks, "e2e": e2e,
@@ -396,7 +408,7 @@ def profile_case(args):
     calls = []
     if args.profile in ("decode", "prefill"):
         N, K = (N_DEC, K_DEC) if args.profile == "decode" else (7168, 2048)
-        plan = bg.bi_gemm_plan(N, K)
+        plan = weight_plan(N, K)
         copies = 3 if args.profile == "decode" else 1
         Bs = [inputs.bf16_gaussian((N, K), seed=11 + i, std=K ** -0.5, device=dev) for i in range(copies)]
         A = inputs.bf16_gaussian((M, K), seed=10, device=dev)
@@ -405,7 +417,7 @@ def profile_case(args):
     elif args.profile == "fp8":
         N = K = 7168
         KB = K // 128
-        plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_E4M3_BLOCKSCALED)
+        plan = weight_plan(N, K, bg.BI_DTYPE_E4M3_BLOCKSCALED)
         qbs = [inputs.e4m3_gaussian((N, K), seed=21 + i, device=dev) for i in range(3)]
         sb = inputs.scales_log_uniform((N // 128, KB), seed=22, device=dev)
         qa = inputs.e4m3_gaussian((M, K), seed=23, device=dev)
@@ -415,7 +427,7 @@ def profile_case(args):
                  for i in range(L)]
     else:
         E, N, K = 64, 2048, 7168
-        plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_BF16, E)
+        plan = weight_plan(N, K, bg.BI_DTYPE_BF16, E)
         B = inputs.bf16_gaussian((E, N, K), seed=31, std=K ** -0.5, device=dev)
         r = inputs.softmax_top8_routing(M, E, seed=32)
         tokens = inputs.bf16_gaussian((M, K), seed=33, device=dev)
@@ -528,7 +540,7 @@ def measure_extras(bg, inputs, dev, stream, peaks):
     hbm = peaks["hbm_gbs"]
     # prefill, M = 16384 and 4096
     for (N, K) in [(7168, 2048), (2048, 7168)]:
-        plan = bg.bi_gemm_plan(N, K)
+        plan = weight_plan(N, K)
         B = inputs.bf16_gaussian((N, K), seed=3001, std=K ** -0.5, device=dev)
         for M in [1024, 4096, 16384]:
             A = inputs.bf16_gaussian((M, K), seed=3002, device=dev)
@@ -542,7 +554,7 @@ def measure_extras(bg, inputs, dev, stream, peaks):
     # FP8 N = K = 7168
     N = K = 7168
     KB = K // 128
-    plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_E4M3_BLOCKSCALED)
+    plan = weight_plan(N, K, bg.BI_DTYPE_E4M3_BLOCKSCALED)
     qbs = [inputs.e4m3_gaussian((N, K), seed=4001 + i, device=dev) for i in range(4)]
     sb = inputs.scales_log_uniform((N // 128, KB), seed=4002, device=dev)
     for M in [1, 64, 4096]:
@@ -559,7 +571,7 @@ def measure_extras(bg, inputs, dev, stream, peaks):
     del qbs
     # MoE: 64 experts, N = 2048, K = 7168, top-8
     E, N, K = 64, 2048, 7168
-    plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_BF16, E)
+    plan = weight_plan(N, K, bg.BI_DTYPE_BF16, E)
     B = inputs.bf16_gaussian((E, N, K), seed=5001, std=K ** -0.5, device=dev)
     for T in [1, 64, 1024, 8192]:
         r = inputs.softmax_top8_routing(T, E, seed=5000 + T)

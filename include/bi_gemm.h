@@ -72,16 +72,19 @@ typedef enum {
 /* Opaque, library-owned plan. */
 typedef struct bi_plan_s *bi_plan_t;
 
-/* What a plan fixed.  None of it depends on M, except the two ring depths, which are reported
+/* What a plan fixed.  None of it depends on M, except the pipeline grouping, which is reported
  * for a full-height tile: a launch whose whole problem has fewer rows than one tile sizes its A
- * slots to those rows and deepens both rings (scheduling only; the MMA and K order are fixed). */
+ * slots to those rows and deepens both rings, and a bf16 128 x 32 plan groups 8 K chunks per
+ * pipeline stage when A has at most 64 rows (scheduling only; the tile, the MMA instruction and
+ * the K order are fixed, so no row's result changes). */
 typedef struct {
     int64_t n, k;              /* the plan's N and K */
     int dtype;                 /* bi_dtype_t */
     int num_experts;           /* 1 = dense */
     int block_m;               /* output rows per tile */
     int block_n;               /* output columns per tile */
-    int block_k;               /* K elements per pipeline stage (1, 2 or 4 chunks of 128 bytes) */
+    int block_k;               /* K elements per pipeline stage (1, 2 or 4 chunks of 128 bytes) for
+                                  a full-height tile */
     int cta_group;             /* CTAs that share one MMA (1 or 2) */
     int mma_m, mma_n, mma_k;   /* tcgen05.mma instruction shape */
     int stages;                /* depth of the B (weight) shared-memory ring */
@@ -224,6 +227,19 @@ bi_status_t bi_gemm_sync_status(bi_plan_t plan, cudaStream_t stream);
  * and returns, so the context stays usable.
  */
 bi_status_t bi_gemm_set_wait_timeout(bi_plan_t plan, uint64_t timeout_ns);
+
+/*
+ * Plan flags; 0 clears them all.
+ * BI_PLAN_RESIDENT_WEIGHTS: the caller promises that no kernel enqueued on a launch's stream
+ * before that launch writes the launch's B or scale_b (weights loaded once and then only read,
+ * as in inference).  A dense launch may then request its first pipeline groups of B while the
+ * previous kernel in the stream is still running; it still waits for that kernel to complete
+ * before it reads A or scale_a or writes C or the status word.  The flag changes when B is
+ * read, never a result.  Off by default; grouped plans ignore it.
+ * Errors: BI_ERR_INVALID_ARG (plan == NULL or an unknown flag bit).
+ */
+#define BI_PLAN_RESIDENT_WEIGHTS 1u
+bi_status_t bi_gemm_plan_set_flags(bi_plan_t plan, uint32_t flags);
 
 /*
  * Test-only fault injection on the host side of the launch.  BI_DEBUG_SKIP_FIRST_LOAD makes

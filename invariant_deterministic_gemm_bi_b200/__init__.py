@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     BI_DEBUG_SKIP_FIRST_LOAD,
     BI_DTYPE_BF16,
     BI_DTYPE_E4M3_BLOCKSCALED,
+    BI_PLAN_RESIDENT_WEIGHTS,
     BiGemmError,
     Plan,
     bi_gemm_abi_version,
@@ -18,6 +19,7 @@ from .binding import (  # noqa: F401
     bi_gemm_plan,
     bi_gemm_plan_describe,
     bi_gemm_plan_destroy,
+    bi_gemm_plan_set_flags,
     bi_gemm_run,
     bi_gemm_run_host,
     bi_gemm_run_host_noalloc,

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(PKG, "libbigemm.so")
 BI_DTYPE_BF16 = 0
 BI_DTYPE_E4M3_BLOCKSCALED = 1
 BI_DEBUG_SKIP_FIRST_LOAD = 1
+BI_PLAN_RESIDENT_WEIGHTS = 1
 
 STATUS_NAMES = {
     0: "BI_OK", 1: "BI_ERR_INVALID_ARG", 2: "BI_ERR_ALIGNMENT", 3: "BI_ERR_UNSUPPORTED_SHAPE",
@@ -31,7 +32,7 @@ EXPORTED = [
     "bi_gemm_abi_version", "bi_status_string", "bi_gemm_plan", "bi_gemm_plan_destroy",
     "bi_gemm_plan_describe", "bi_gemm_run", "bi_grouped_gemm_run", "bi_gemm_run_host",
     "bi_gemm_sync_status", "bi_gemm_set_wait_timeout", "bi_gemm_debug_set_flags",
-    "bi_gemm_run_host_noalloc",
+    "bi_gemm_run_host_noalloc", "bi_gemm_plan_set_flags",
 ]
 
 
@@ -94,6 +95,8 @@ def load_library(path: str = LIB_PATH):
     lib.bi_gemm_set_wait_timeout.argtypes = [vp, u64]
     lib.bi_gemm_debug_set_flags.restype = i32
     lib.bi_gemm_debug_set_flags.argtypes = [vp, u32]
+    lib.bi_gemm_plan_set_flags.restype = i32
+    lib.bi_gemm_plan_set_flags.argtypes = [vp, u32]
     if path == LIB_PATH:
         _LIB = lib
     return lib
@@ -230,6 +233,11 @@ def bi_gemm_sync_status(plan: Plan, stream=None, raise_on_error: bool = True) ->
 
 def bi_gemm_set_wait_timeout(plan: Plan, timeout_ns: int):
     _check(load_library().bi_gemm_set_wait_timeout(plan.handle, timeout_ns), "bi_gemm_set_wait_timeout")
+
+
+def bi_gemm_plan_set_flags(plan: Plan, flags: int):
+    """BI_PLAN_RESIDENT_WEIGHTS: B is never written by an earlier kernel on the launch's stream."""
+    _check(load_library().bi_gemm_plan_set_flags(plan.handle, flags), "bi_gemm_plan_set_flags")
 
 
 def bi_gemm_debug_set_flags(plan: Plan, flags: int):

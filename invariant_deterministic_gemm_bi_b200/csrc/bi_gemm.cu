@@ -55,10 +55,12 @@ struct KernelEntry {
 
 // Narrow tiles (BN <= 64) run on one CTA; wide ones (BN >= 128) on a CTA pair.  Every tile comes
 // in two forms: its preferred number of 128-byte K chunks per pipeline stage (3-D TMA boxes;
-// needs K to be a multiple of the chunk), and one chunk per stage for any other K.
+// needs K to be a multiple of the chunk), and one chunk per stage for any other K.  The bf16
+// 128 x 32 tile has a third, small-batch form with 8 chunks per stage (see small_batch_kernel).
 const KernelEntry kKernels[] = {
     BI_ENTRY(64, 32, 1, false, false),  BI_ENTRY(64, 32, 4, false, false),
     BI_ENTRY(128, 32, 1, false, false), BI_ENTRY(128, 32, 4, false, false),
+    BI_ENTRY(128, 32, 8, false, false),
     BI_ENTRY(128, 64, 1, false, false), BI_ENTRY(128, 64, 2, false, false),
     BI_ENTRY(128, 32, 1, true, false),  BI_ENTRY(128, 32, 4, true, false),
     BI_ENTRY(128, 64, 1, true, false),  BI_ENTRY(128, 64, 2, true, false),
@@ -128,7 +130,9 @@ RingGeom ring_geometry(const KernelEntry *k, int a_rows)
     }
     // The kernel relies on 2 <= sa <= sb (the A-slot reuse test reads the consumed ring) and, for
     // FP8, on sb groups outlasting the partial-product ring.  Every tile in kKernels satisfies
-    // this for every a_rows in [8, BM]; tests/test_abi.py checks the reported depths.
+    // this for every a_rows in [8, BM], except the 8-chunk small-batch form, which is valid up to
+    // 64 rows and used up to kSmallBatchRows = 64; set_rows reports a violation and the launch is
+    // refused.  tests/test_abi.py checks the reported depths.
     return RingGeom{sa, sb, static_cast<uint32_t>(a_stride), static_cast<uint32_t>(a_region)};
 }
 
@@ -251,9 +255,13 @@ struct bi_plan_s {
     bi_dtype_t dtype = BI_DTYPE_BF16;
     int experts = 1;
     const KernelEntry *kernel = nullptr;
-    int kernel_index = 0;
+    // The same tile with more K chunks per pipeline group, for launches whose A rows are few
+    // (dense plans only; may be null).  It issues the same MMAs in the same K order, so a row's
+    // result does not depend on which of the two a launch takes.
+    const KernelEntry *kernel_small = nullptr;
     uint64_t timeout_ns = 2000000000ull;
     uint32_t debug_flags = 0;
+    uint32_t flags = 0;      // BI_PLAN_* flags
     std::mutex mu;
     int *status[kMaxDevices] = {};
 };
@@ -313,16 +321,15 @@ bi_status_t encode_operand(CUtensorMap *map, const void *base, bool fp8, int64_t
     return r == CUDA_SUCCESS ? BI_OK : BI_ERR_CUDA;
 }
 
-bi_status_t ensure_kernel_attr(bi_plan_s *plan, DeviceInfo *d)
+bi_status_t ensure_kernel_attr(const KernelEntry *k, DeviceInfo *d)
 {
     std::lock_guard<std::mutex> lock(g_dev_mu);
-    const int ki = plan->kernel_index;
+    const int ki = static_cast<int>(k - kKernels);
     if (!d->attr_set[ki]) {
-        if (cudaFuncSetAttribute(reinterpret_cast<const void *>(plan->kernel->fn),
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 plan->kernel->smem) != cudaSuccess)
+        if (cudaFuncSetAttribute(reinterpret_cast<const void *>(k->fn),
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, k->smem) != cudaSuccess)
             return BI_ERR_CUDA;
-        if (plan->kernel->pair) {
+        if (k->pair) {
             cudaLaunchConfig_t cfg = {};
             cudaLaunchAttribute attr[1];
             attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -330,12 +337,12 @@ bi_status_t ensure_kernel_attr(bi_plan_s *plan, DeviceInfo *d)
             attr[0].val.clusterDim.y = 1;
             attr[0].val.clusterDim.z = 1;
             cfg.gridDim = dim3(2 * (d->num_sms / 2));
-            cfg.blockDim = dim3(plan->kernel->threads);
-            cfg.dynamicSmemBytes = plan->kernel->smem;
+            cfg.blockDim = dim3(k->threads);
+            cfg.dynamicSmemBytes = k->smem;
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             int clusters = 0;
-            if (cudaOccupancyMaxActiveClusters(&clusters, reinterpret_cast<const void *>(plan->kernel->fn),
+            if (cudaOccupancyMaxActiveClusters(&clusters, reinterpret_cast<const void *>(k->fn),
                                                &cfg) != cudaSuccess ||
                 clusters < 1) {
                 cudaGetLastError();
@@ -348,9 +355,10 @@ bi_status_t ensure_kernel_attr(bi_plan_s *plan, DeviceInfo *d)
     return BI_OK;
 }
 
-int pair_grid_limit(const bi_plan_s *plan, const DeviceInfo *d)
+int pair_grid_limit(const KernelEntry *k, const DeviceInfo *d)
 {
-    return d->max_pairs[plan->kernel_index] > 0 ? d->max_pairs[plan->kernel_index] : d->num_sms / 2;
+    const int ki = static_cast<int>(k - kKernels);
+    return d->max_pairs[ki] > 0 ? d->max_pairs[ki] : d->num_sms / 2;
 }
 
 bi_status_t launch_zero(void *C, int64_t ldc, int64_t rows, int64_t n, cudaStream_t stream)
@@ -402,12 +410,12 @@ int dense_a_box_rows(int64_t M, int bm)
     return M >= bm ? bm : static_cast<int>((M + 7) / 8 * 8);
 }
 
-bool set_rows(GemmParams *p, const bi_plan_s *plan, int a_rows)
+bool set_rows(GemmParams *p, const KernelEntry *k, int a_rows)
 {
-    const RingGeom g = ring_geometry(plan->kernel, a_rows);
+    const RingGeom g = ring_geometry(k, a_rows);
     p->a_box_rows = a_rows;
     // the peer CTA of a pair has A rows to load unless the whole problem fits in 128 rows
-    p->pair_a1 = (plan->kernel->grouped || p->rows > 128) ? 1 : 0;
+    p->pair_a1 = (k->grouped || p->rows > 128) ? 1 : 0;
     p->sa = g.sa;
     p->sb = g.sb;
     p->a_stride = g.a_stride;
@@ -415,7 +423,8 @@ bool set_rows(GemmParams *p, const bi_plan_s *plan, int a_rows)
     return g.sa >= 2 && g.sa <= g.sb && g.sa <= bi::kMaxSA && g.sb <= bi::kMaxSB;
 }
 
-GemmParams base_params(const bi_plan_s *plan, int64_t rows, void *C, int64_t ldc, int *status)
+GemmParams base_params(const bi_plan_s *plan, const KernelEntry *k, int64_t rows, void *C, int64_t ldc,
+                       int *status)
 {
     GemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -424,11 +433,11 @@ GemmParams base_params(const bi_plan_s *plan, int64_t rows, void *C, int64_t ldc
     p.n = static_cast<int32_t>(plan->n);
     p.k = static_cast<int32_t>(plan->k);
     p.num_k_blocks = static_cast<int32_t>((plan->k * elt + bi::kRowBytes - 1) / bi::kRowBytes);
-    p.num_n_blocks = static_cast<int32_t>((plan->n + plan->kernel->bn - 1) / plan->kernel->bn);
-    p.num_m_blocks = static_cast<int32_t>((rows + plan->kernel->bm - 1) / plan->kernel->bm);
+    p.num_n_blocks = static_cast<int32_t>((plan->n + k->bn - 1) / k->bn);
+    p.num_m_blocks = static_cast<int32_t>((rows + k->bm - 1) / k->bm);
     p.num_experts = plan->experts;
     p.raster_m = 16;
-    (void)set_rows(&p, plan, plan->kernel->bm);
+    (void)set_rows(&p, k, k->bm);
     p.c = static_cast<__nv_bfloat16 *>(C);
     p.ldc = ldc;
     p.kb_scale = static_cast<int32_t>((plan->k + 127) / 128);
@@ -437,50 +446,71 @@ GemmParams base_params(const bi_plan_s *plan, int64_t rows, void *C, int64_t ldc
     // SM clock (1965 MHz), so a wait lasts at least timeout_ns
     p.timeout_cycles = plan->timeout_ns * 2;
     p.debug_flags = plan->debug_flags;
+    p.prefetch_b = (plan->flags & BI_PLAN_RESIDENT_WEIGHTS) && !k->grouped ? 1 : 0;
     return p;
 }
 
-// Launch the plan's kernel.  `units` is the number of work tiles; a one-CTA kernel gets
-// min(units, #SMs) CTAs, a pair kernel min(units, co-resident pairs) clusters of two CTAs.
-bi_status_t launch_main(const bi_plan_s *plan, const DeviceInfo *d, const CUtensorMap &ta,
+// Launch kernel entry k.  `units` is the number of work tiles; a one-CTA kernel gets
+// min(units, #SMs) CTAs, a pair kernel min(units, co-resident pairs) clusters of two CTAs.  Every
+// launch is a programmatic dependent of the previous kernel in the stream: it may start (and set
+// up its shared and tensor memory) while that kernel finishes, and waits for it to complete
+// before touching global memory (bi::ptx::grid_dependency_wait).
+bi_status_t launch_main(const KernelEntry *k, const DeviceInfo *d, const CUtensorMap &ta,
                         const CUtensorMap &tb, const GemmParams &p, int64_t units,
                         cudaStream_t stream)
 {
     if (units < 1)
         units = 1;
-    if (!plan->kernel->pair) {
-        const int grid = static_cast<int>(units < d->num_sms ? units : d->num_sms);
-        plan->kernel->fn<<<grid, plan->kernel->threads, plan->kernel->smem, stream>>>(ta, tb, p);
-        return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
-    }
-    const int lim = pair_grid_limit(plan, d);
-    const int pairs = static_cast<int>(units < lim ? units : lim);
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(2 * pairs);
-    cfg.blockDim = dim3(plan->kernel->threads);
-    cfg.dynamicSmemBytes = plan->kernel->smem;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (!k->pair) {
+        cfg.gridDim = dim3(static_cast<unsigned>(units < d->num_sms ? units : d->num_sms));
+    } else {
+        const int lim = pair_grid_limit(k, d);
+        const int pairs = static_cast<int>(units < lim ? units : lim);
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 2;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+        cfg.gridDim = dim3(2 * pairs);
+    }
+    cfg.blockDim = dim3(k->threads);
+    cfg.dynamicSmemBytes = k->smem;
     cfg.stream = stream;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, plan->kernel->fn, ta, tb, p);
+    cfg.numAttrs = na;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k->fn, ta, tb, p);
     return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
 // Rows of A one TMA box covers and rows of B one box covers, for this plan and M.  A pair CTA
 // owns 128 rows of a tile; a dense problem smaller than that boxes only its roundup(M, 8) rows.
-int a_box_rows_for(const bi_plan_s *plan, int64_t M)
+int a_box_rows_for(const KernelEntry *k, int64_t M)
 {
-    return dense_a_box_rows(M, plan->kernel->pair ? 128 : plan->kernel->bm);
+    return dense_a_box_rows(M, k->pair ? 128 : k->bm);
 }
 
-int b_box_rows_for(const bi_plan_s *plan)
+int b_box_rows_for(const KernelEntry *k)
 {
-    return plan->kernel->pair ? plan->kernel->bn / 2 : plan->kernel->bn;
+    return k->pair ? k->bn / 2 : k->bn;
+}
+
+// A dense launch of M rows whose A boxes hold at most this many rows takes the plan's
+// small-batch kernel form (when it has one): with few A rows, groups of 8 K chunks halve the
+// per-group wait and commit overhead of the MMA thread, and the ring still holds two groups of
+// A and of B.
+constexpr int kSmallBatchRows = 64;
+
+const KernelEntry *dense_kernel_for(const bi_plan_s *plan, int64_t M)
+{
+    if (plan->kernel_small && a_box_rows_for(plan->kernel_small, M) <= kSmallBatchRows)
+        return plan->kernel_small;
+    return plan->kernel;
 }
 
 } // namespace
@@ -571,7 +601,8 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     p->dtype = dtype;
     p->experts = num_experts;
     p->kernel = k;
-    p->kernel_index = static_cast<int>(k - kKernels);
+    if (!fp8 && num_experts == 1 && k->bm == 128 && k->bn == 32 && k->kc == preferred_chunks(32))
+        p->kernel_small = find_kernel(128, 32, 8, false, false);
     *out = p;
     return BI_OK;
 }
@@ -634,6 +665,14 @@ bi_status_t bi_gemm_set_wait_timeout(bi_plan_t plan, uint64_t timeout_ns)
     return BI_OK;
 }
 
+bi_status_t bi_gemm_plan_set_flags(bi_plan_t plan, uint32_t flags)
+{
+    if (!plan || (flags & ~BI_PLAN_RESIDENT_WEIGHTS))
+        return BI_ERR_INVALID_ARG;
+    plan->flags = flags;
+    return BI_OK;
+}
+
 bi_status_t bi_gemm_debug_set_flags(bi_plan_t plan, uint32_t flags)
 {
     if (!plan)
@@ -675,22 +714,23 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
     int *status = nullptr;
     if ((st = plan_status_word(plan, dev, &status)) != BI_OK)
         return st;
-    if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
+    const KernelEntry *k = dense_kernel_for(plan, M);
+    if ((st = ensure_kernel_attr(k, d)) != BI_OK)
         return st;
     CUtensorMap ta, tb;
-    const int a_rows = a_box_rows_for(plan, M);
-    if ((st = encode_operand(&ta, A, fp8, plan->k, M, lda, a_rows, plan->kernel->kc)) != BI_OK)
+    const int a_rows = a_box_rows_for(k, M);
+    if ((st = encode_operand(&ta, A, fp8, plan->k, M, lda, a_rows, k->kc)) != BI_OK)
         return st;
-    if ((st = encode_operand(&tb, B, fp8, plan->k, plan->n, ldb, b_box_rows_for(plan), plan->kernel->kc)) != BI_OK)
+    if ((st = encode_operand(&tb, B, fp8, plan->k, plan->n, ldb, b_box_rows_for(k), k->kc)) != BI_OK)
         return st;
-    GemmParams p = base_params(plan, M, C, ldc, status);
-    if (!set_rows(&p, plan, a_rows))
+    GemmParams p = base_params(plan, k, M, C, ldc, status);
+    if (!set_rows(&p, k, a_rows))
         return BI_ERR_UNSUPPORTED_SHAPE;
     p.scale_a = scale_a;
     p.ld_sa = ld_sa;
     p.scale_b = scale_b;
     const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-    return launch_main(plan, d, ta, tb, p, tiles, stream);
+    return launch_main(k, d, ta, tb, p, tiles, stream);
 }
 
 bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *A, int64_t lda,
@@ -717,22 +757,23 @@ bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *
     int *status = nullptr;
     if ((st = plan_status_word(plan, dev, &status)) != BI_OK)
         return st;
-    if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
+    const KernelEntry *k = plan->kernel;
+    if ((st = ensure_kernel_attr(k, d)) != BI_OK)
         return st;
     CUtensorMap ta, tb;
-    const int a_rows = plan->kernel->pair ? 128 : plan->kernel->bm;
-    if ((st = encode_operand(&ta, A, false, plan->k, total_rows, lda, a_rows, plan->kernel->kc)) != BI_OK)
+    const int a_rows = k->pair ? 128 : k->bm;
+    if ((st = encode_operand(&ta, A, false, plan->k, total_rows, lda, a_rows, k->kc)) != BI_OK)
         return st;
-    if ((st = encode_operand(&tb, B, false, plan->k, plan->n * plan->experts, ldb, b_box_rows_for(plan),
-                             plan->kernel->kc)) != BI_OK)
+    if ((st = encode_operand(&tb, B, false, plan->k, plan->n * plan->experts, ldb, b_box_rows_for(k),
+                             k->kc)) != BI_OK)
         return st;
-    GemmParams p = base_params(plan, total_rows, C, ldc, status);
-    (void)set_rows(&p, plan, a_rows);
+    GemmParams p = base_params(plan, k, total_rows, C, ldc, status);
+    (void)set_rows(&p, k, a_rows);
     p.offsets = expert_offsets;
     // Upper bound on the tile count without reading the offsets: sum_e ceil(len_e/BM) is at
     // most total_rows/BM + E.
-    const int64_t max_tiles = (total_rows / plan->kernel->bm + plan->experts) * p.num_n_blocks;
-    return launch_main(plan, d, ta, tb, p, max_tiles, stream);
+    const int64_t max_tiles = (total_rows / k->bm + plan->experts) * p.num_n_blocks;
+    return launch_main(k, d, ta, tb, p, max_tiles, stream);
 }
 
 bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M, const void *A_host, int64_t lda,
@@ -834,22 +875,23 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
         if (fp8 && cudaMemcpyAsync(sa_dev, scale_a_host, static_cast<size_t>(kb * ld_sa * 4),
                                    cudaMemcpyHostToDevice, stream) != cudaSuccess)
             return BI_ERR_CUDA;
-        if ((st = ensure_kernel_attr(plan, d)) != BI_OK)
+        const KernelEntry *k = dense_kernel_for(plan, M);
+        if ((st = ensure_kernel_attr(k, d)) != BI_OK)
             return st;
         CUtensorMap ta, tb;
-        const int a_rows = a_box_rows_for(plan, M);
-        if ((st = encode_operand(&ta, A_dev, fp8, plan->k, M, lda, a_rows, plan->kernel->kc)) != BI_OK)
+        const int a_rows = a_box_rows_for(k, M);
+        if ((st = encode_operand(&ta, A_dev, fp8, plan->k, M, lda, a_rows, k->kc)) != BI_OK)
             return st;
-        if ((st = encode_operand(&tb, B, fp8, plan->k, plan->n, ldb, b_box_rows_for(plan), plan->kernel->kc)) != BI_OK)
+        if ((st = encode_operand(&tb, B, fp8, plan->k, plan->n, ldb, b_box_rows_for(k), k->kc)) != BI_OK)
             return st;
-        GemmParams p = base_params(plan, M, C_dev, ldc, status);
-        if (!set_rows(&p, plan, a_rows))
+        GemmParams p = base_params(plan, k, M, C_dev, ldc, status);
+        if (!set_rows(&p, k, a_rows))
             return BI_ERR_UNSUPPORTED_SHAPE;
         p.scale_a = fp8 ? sa_dev : nullptr;
         p.ld_sa = fp8 ? ld_sa : 0;
         p.scale_b = fp8 ? scale_b : nullptr;
         const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-        if ((st = launch_main(plan, d, ta, tb, p, tiles, stream)) != BI_OK)
+        if ((st = launch_main(k, d, ta, tb, p, tiles, stream)) != BI_OK)
             return st;
     }
     if (cudaMemcpyAsync(C_host, C_dev, static_cast<size_t>(M * ldc * 2), cudaMemcpyDeviceToHost,

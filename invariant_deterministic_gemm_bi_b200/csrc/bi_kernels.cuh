@@ -80,6 +80,8 @@ struct GemmParams {
     uint32_t a_stride;       // bytes between A slots (KC * a_box_rows * 128)
     uint32_t b_offset;       // byte offset of the B ring in the ring region
     int32_t pair_a1;         // CTA pair: 1 if the peer CTA loads A rows (the problem has > 128)
+    int32_t prefetch_b;      // dense, resident weights: request the first B groups before the
+                             // previous kernel in the stream has completed
     __nv_bfloat16 *c;
     int64_t ldc;
     const float *scale_a;    // FP8: [kb][ld_sa]
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32,256]");
     static_assert(!FP8 || BN <= 128, "FP8 keeps BN fp32 accumulators per thread: BN <= 128");
     static_assert(!(FP8 && GROUPED), "grouped FP8 is not built");
-    static_assert(KC >= 1 && KC <= 4, "1..4 chunks per group");
+    static_assert(KC >= 1 && KC <= 8, "1..8 chunks per group");
     using R = Rings<BM, BN, KC>;
     constexpr int kElemsPerRow = FP8 ? 128 : 64;         // K elements per 128-byte row
     constexpr int kMmaK = FP8 ? 32 : 16;                 // K per tcgen05.mma
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     const uint32_t lane = ptx::lane_id();
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kMaxSB; ++s) {
+        for (int s = 0; s < p.sb; ++s) {   // only the ring slots this launch uses
             ptx::mbar_init(&full[s], 2);
             ptx::mbar_init(&consumed[s], 1);
         }
@@ -308,6 +310,90 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
         ptx::tmem_alloc(tmem_base_smem, kTmemCols);
         ptx::tmem_relinquish_alloc_permit();
     }
+
+    const int nkb = p.num_k_blocks;              // 128-byte K chunks per tile
+    const int nkg = (nkb + KC - 1) / KC;         // groups per tile
+    const uint32_t a_chunk_pitch = static_cast<uint32_t>(p.a_box_rows) * kRowBytes;
+    int num_tiles = 0;                           // set below (grouped: from the offsets)
+    auto tile_at = [&](int t) -> TileCoord {
+        if constexpr (GROUPED)
+            return grouped_tile(p, BM, BN, t, grp_prefix, grp_offs);
+        else
+            return dense_tile(p, BM, BN, t);
+    };
+
+    // TMA producer state (used by thread 0 only).  Two cursors walk this CTA's (tile, group)
+    // sequence: the B loads run `lag` = sb - sa groups ahead of the A loads.
+    struct Cursor {
+        int t, kg;
+        bool valid;
+        TileCoord tc;
+    };
+    Cursor cb{}, ca{};
+    int jb = 0, ja = 0;                 // groups issued so far
+    int bs = 0, as = 0, cs = 0;         // B slot of jb, A slot of ja, consumed slot of ja - sa
+    int fs = 0;                         // full-ring slot of group ja
+    uint32_t bph = 0, cph = 0;
+    bool skipped_b0 = false;
+    const uint64_t pol = ptx::policy_evict_normal();
+    auto advance = [&](Cursor &c) {
+        if (++c.kg == nkg) {
+            c.kg = 0;
+            c.t += gridDim.x;
+            c.valid = c.t < num_tiles;
+            if (c.valid)
+                c.tc = tile_at(c.t);
+        }
+    };
+    auto first_cursor = [&]() {
+        Cursor c{static_cast<int>(blockIdx.x), 0, static_cast<int>(blockIdx.x) < num_tiles, {}};
+        if (c.valid)
+            c.tc = tile_at(c.t);
+        return c;
+    };
+    auto load = [&](void *dst, const CUtensorMap *map, uint64_t *bar, int kg, int row) {
+        if constexpr (KC == 1)
+            ptx::tma_load_2d(dst, map, bar, kg * kElemsPerRow, row, pol);
+        else
+            ptx::tma_load_3d(dst, map, bar, 0, row, kg * KC, pol);
+    };
+    // B group jb into slot bs; its slot is free (the consumed wait, if any, is done)
+    auto issue_b = [&]() {
+        if (jb == 0 && (p.debug_flags & 1u)) {
+            skipped_b0 = true;      // fault injection: this B group is never filled
+        } else {
+            ptx::mbar_arrive_expect_tx(&full[bs], R::kBBytes);
+            load(smem_b + bs * R::kBBytes, &tmap_b, &full[bs], cb.kg, cb.tc.b_row0);
+        }
+        advance(cb);
+        ++jb;
+        if (++bs == p.sb) {
+            bs = 0;
+            bph ^= 1u;
+        }
+    };
+    bool b_started = false;
+    if constexpr (!GROUPED) {
+        // Resident weights: B is not written by the previous kernel in the stream, so the first
+        // sb groups of B (their slots are free in a fresh ring) are requested before that
+        // kernel has completed.
+        if (threadIdx.x == 0 && p.prefetch_b) {
+            num_tiles = p.num_m_blocks * p.num_n_blocks;
+            cb = first_cursor();
+            for (int i = 0; i < p.sb && cb.valid; ++i)
+                issue_b();
+            b_started = true;
+        }
+    }
+
+    // Everything above touches only this CTA's shared and tensor memory, the kernel parameters
+    // and (resident weights only) B, so it overlaps the tail of the previous kernel in the
+    // stream when this one was launched as its programmatic dependent.  No thread reads A, the
+    // scales or the offsets, or writes anything to global memory, before the previous grid has
+    // completed.
+    ptx::grid_dependency_wait();
+    if (threadIdx.x == 0)
+        ptx::launch_dependents();
 
     // Grouped: read and validate the expert offsets, build the tile prefix sum.
     __shared__ int32_t s_num_tiles;
@@ -349,76 +435,17 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_base_smem;
-    const int num_tiles = s_num_tiles;
-
-    auto tile_at = [&](int t) -> TileCoord {
-        if constexpr (GROUPED)
-            return grouped_tile(p, BM, BN, t, grp_prefix, grp_offs);
-        else
-            return dense_tile(p, BM, BN, t);
-    };
-
-    const int nkb = p.num_k_blocks;              // 128-byte K chunks per tile
-    const int nkg = (nkb + KC - 1) / KC;         // groups per tile
-    const uint32_t a_chunk_pitch = static_cast<uint32_t>(p.a_box_rows) * kRowBytes;
+    num_tiles = s_num_tiles;
 
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint64_t pol = ptx::policy_evict_normal();
-            // Two cursors over this CTA's (tile, group) sequence: B runs `lag` groups ahead.
-            struct Cursor {
-                int t, kg;
-                bool valid;
-                TileCoord tc;
-            };
-            Cursor cb{static_cast<int>(blockIdx.x), 0, static_cast<int>(blockIdx.x) < num_tiles, {}};
-            if (cb.valid)
-                cb.tc = tile_at(cb.t);
-            Cursor ca = cb;
-            auto advance = [&](Cursor &c) {
-                if (++c.kg == nkg) {
-                    c.kg = 0;
-                    c.t += gridDim.x;
-                    c.valid = c.t < num_tiles;
-                    if (c.valid)
-                        c.tc = tile_at(c.t);
-                }
-            };
-            auto load = [&](void *dst, const CUtensorMap *map, uint64_t *bar, int kg, int row) {
-                if constexpr (KC == 1)
-                    ptx::tma_load_2d(dst, map, bar, kg * kElemsPerRow, row, pol);
-                else
-                    ptx::tma_load_3d(dst, map, bar, 0, row, kg * KC, pol);
-            };
+            if (!b_started)
+                cb = first_cursor();
+            ca = first_cursor();
             const int SA = p.sa, SB = p.sb, lag = SB - SA;   // B groups lead A groups by lag
-            int jb = 0, ja = 0;                 // groups issued so far
-            int bs = 0, as = 0, cs = 0;         // B slot of jb, A slot of ja, consumed slot of ja - SA
-            int fs = 0;                         // full-ring slot of group ja
-            uint32_t bph = 0, cph = 0;
-            bool skipped_b0 = false;
             bool ok = true;
             while (ok && (cb.valid || ca.valid)) {
-                if (cb.valid) {
-                    // slot bs is free once group jb - SB was consumed
-                    if (!ptx::mbar_wait(&consumed[bs], bph ^ 1u, p.timeout_cycles, abort_flag)) {
-                        record_failure(p, abort_flag, kStatusTimeout);
-                        ok = false;
-                        break;
-                    }
-                    if (jb == 0 && (p.debug_flags & 1u)) {
-                        skipped_b0 = true;      // fault injection: this B group is never filled
-                    } else {
-                        ptx::mbar_arrive_expect_tx(&full[bs], R::kBBytes);
-                        load(smem_b + bs * R::kBBytes, &tmap_b, &full[bs], cb.kg, cb.tc.b_row0);
-                    }
-                    advance(cb);
-                    ++jb;
-                    if (++bs == SB) {
-                        bs = 0;
-                        bph ^= 1u;
-                    }
-                }
                 if (ca.valid && (ja + lag < jb || !cb.valid)) {
                     // slot `as` is free once group ja - SA was consumed.  That group's consumed
                     // barrier cannot have moved on to group ja - SA + SB yet: that one needs A
@@ -442,7 +469,16 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                         as = 0;
                     if (++fs == SB)
                         fs = 0;
+                    continue;
                 }
+                // A is `lag` groups behind B (or done): the next B group.  Slot bs is free once
+                // group jb - SB was consumed, whose A load was issued above.
+                if (!ptx::mbar_wait(&consumed[bs], bph ^ 1u, p.timeout_cycles, abort_flag)) {
+                    record_failure(p, abort_flag, kStatusTimeout);
+                    ok = false;
+                    break;
+                }
+                issue_b();
             }
             // Drain: every load this thread issued must have landed before the CTA exits (on
             // the normal path they all have: the MMA warp consumed them).  Only the last SB

@@ -109,6 +109,11 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
         ptx::tmem_alloc_pair(tmem_base_smem, kTmemCols);
         ptx::tmem_relinquish_alloc_permit_pair();
     }
+    // No global memory is touched before the previous grid in the stream has completed (see
+    // bi_gemm_kernel); the set-up above overlaps its tail.
+    ptx::grid_dependency_wait();
+    if (threadIdx.x == 0)
+        ptx::launch_dependents();
 
     __shared__ int32_t s_num_tiles;
     if constexpr (GROUPED) {

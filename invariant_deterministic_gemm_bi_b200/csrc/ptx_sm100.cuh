@@ -87,6 +87,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
 }
 
 // ---------------------------------------------------------------------------------------------
+// Programmatic dependent launch
+// ---------------------------------------------------------------------------------------------
+
+// Wait until every grid this one depends on (the previous kernel in the stream, when this one
+// was launched with programmatic stream serialization) has completed and its memory operations
+// are visible.  Returns at once for a kernel launched without that attribute.
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next kernel in the stream to launch (it still waits in grid_dependency_wait for this
+// grid to complete before it touches global memory).
+__device__ __forceinline__ void launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------------------------
 // TMA (tensor loads, no multicast)
 // ---------------------------------------------------------------------------------------------
 

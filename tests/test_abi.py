@@ -117,3 +117,18 @@ def test_valid_run_without_a_device_reports_no_device():
     plan = bg.bi_gemm_plan(64, 64)
     st = lib.bi_gemm_run(plan.handle, 1, 16, 64, 16, 64, 16, 64, None, 0, None, None)
     assert binding.STATUS_NAMES[st] == "BI_ERR_NO_DEVICE"
+
+
+def test_plan_flags_accept_known_bits_only():
+    lib = binding.load_library()
+    plan = bg.bi_gemm_plan(64, 64)
+    S = binding.STATUS
+    assert lib.bi_gemm_plan_set_flags(None, 0) == S["BI_ERR_INVALID_ARG"]
+    assert lib.bi_gemm_plan_set_flags(plan.handle, bg.BI_PLAN_RESIDENT_WEIGHTS) == 0
+    assert lib.bi_gemm_plan_set_flags(plan.handle, 0) == 0
+    assert lib.bi_gemm_plan_set_flags(plan.handle, 2) == S["BI_ERR_INVALID_ARG"]
+    assert lib.bi_gemm_plan_set_flags(plan.handle, 0x80000000) == S["BI_ERR_INVALID_ARG"]
+    # the flags change when B is read, never the plan
+    before = bg.bi_gemm_plan_describe(plan)
+    bg.bi_gemm_plan_set_flags(plan, bg.BI_PLAN_RESIDENT_WEIGHTS)
+    assert bg.bi_gemm_plan_describe(plan) == before
