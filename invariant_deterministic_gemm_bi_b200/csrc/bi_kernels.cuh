@@ -528,19 +528,26 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                     ptx::tc_fence_after_sync();
                     const uint64_t a_slot = a_desc0 + ((sa * p.a_stride) >> 4);
                     const uint64_t b_slot = b_desc0 + ((sb * R::kBBytes) >> 4);
+                    const int nc = nkb - kg * KC;   // chunks in this group: KC, except at a tile's end
+                    if constexpr (FP8) {
+                        // Each K chunk's partial product goes to its own TMEM buffer.  Every
+                        // epilogue thread hands the buffers back in chunk order, so the buffer of
+                        // the group's last chunk being free means the others are free as well:
+                        // one wait per group.
+                        const uint32_t last = acc_iter + static_cast<uint32_t>((nc < KC ? nc : KC) - 1);
+                        if (!ptx::mbar_wait(&acce_bar[last % kNumAcc], ((last / kNumAcc) & 1u) ^ 1u,
+                                            p.timeout_cycles, abort_flag)) {
+                            record_failure(p, abort_flag, kStatusTimeout);
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after_sync();
+                    }
                     // the MMAs of chunk c of this group (K chunk number `chunk` of the tile)
                     auto issue_chunk = [&](int c, int chunk) -> bool {
                         uint32_t d = d_tmem;
                         if constexpr (FP8) {
-                            // each K chunk's partial product goes to its own TMEM buffer
-                            const uint32_t part = acc_iter % kNumAcc;
-                            const uint32_t par = (acc_iter / kNumAcc) & 1u;
-                            if (!ptx::mbar_wait(&acce_bar[part], par ^ 1u, p.timeout_cycles, abort_flag)) {
-                                record_failure(p, abort_flag, kStatusTimeout);
-                                return false;
-                            }
-                            ptx::tc_fence_after_sync();
-                            d = tmem_base + part * BN;
+                            d = tmem_base + (acc_iter % kNumAcc) * BN;
                             ++acc_iter;
                         }
                         const uint64_t a_desc = a_slot + ((c * a_chunk_pitch) >> 4);
@@ -560,7 +567,6 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                     // A full group issues its KC chunks as straight-line code: control flow
                     // between consecutive tcgen05.mma instructions slows their issue.  Only the
                     // last group of a tile can hold fewer chunks.
-                    const int nc = nkb - kg * KC;
                     if (nc >= KC) {
 #pragma unroll
                         for (int c = 0; c < KC; ++c)

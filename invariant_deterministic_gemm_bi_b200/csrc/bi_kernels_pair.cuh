@@ -255,17 +255,23 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                     ptx::tc_fence_after_sync();
                     const uint64_t a_slot = a_desc0 + ((s * R::kABytes) >> 4);
                     const uint64_t b_slot = b_desc0 + ((s * R::kBBytes) >> 4);
+                    const int nc = nkb - kg * KC;   // chunks in this group: KC, except at a tile's end
+                    if constexpr (FP8) {
+                        // every epilogue warp of both CTAs releases the partial buffers in chunk
+                        // order: the group's last buffer being free frees them all
+                        const uint32_t last = acc_iter + static_cast<uint32_t>((nc < KC ? nc : KC) - 1);
+                        if (!ptx::mbar_wait(&acce_bar[last % kNumAcc], ((last / kNumAcc) & 1u) ^ 1u,
+                                            p.timeout_cycles, abort_flag)) {
+                            record_failure(p, abort_flag, kStatusTimeout);
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after_sync();
+                    }
                     auto issue_chunk = [&](int c, int chunk) -> bool {
                         uint32_t d = d_tmem;
                         if constexpr (FP8) {
-                            const uint32_t part = acc_iter % kNumAcc;
-                            const uint32_t par = (acc_iter / kNumAcc) & 1u;
-                            if (!ptx::mbar_wait(&acce_bar[part], par ^ 1u, p.timeout_cycles, abort_flag)) {
-                                record_failure(p, abort_flag, kStatusTimeout);
-                                return false;
-                            }
-                            ptx::tc_fence_after_sync();
-                            d = tmem_base + part * BN;
+                            d = tmem_base + (acc_iter % kNumAcc) * BN;
                             ++acc_iter;
                         }
                         const uint64_t a_desc = a_slot + ((c * a_chunk_pitch) >> 4);
@@ -282,7 +288,6 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                         return true;
                     };
                     // straight-line MMAs for a full group; only a tile's last group can be short
-                    const int nc = nkb - kg * KC;
                     if (nc >= KC) {
 #pragma unroll
                         for (int c = 0; c < KC; ++c)
