@@ -74,9 +74,9 @@ typedef struct bi_plan_s *bi_plan_t;
 
 /* What a plan fixed.  None of it depends on M, except the pipeline grouping, which is reported
  * for a full-height tile: a launch whose whole problem has fewer rows than one tile sizes its A
- * slots to those rows and deepens both rings, and a bf16 128 x 32 plan groups 8 K chunks per
- * pipeline stage when A has at most 64 rows (scheduling only; the tile, the MMA instruction and
- * the K order are fixed, so no row's result changes). */
+ * slots to those rows and deepens both rings, and a bf16 128 x 32 (FP8 128 x 64) plan groups 8
+ * (4) K chunks per pipeline stage when A has at most 64 rows (scheduling only; the tile, the MMA
+ * instruction and the K order are fixed, so no row's result changes). */
 typedef struct {
     int64_t n, k;              /* the plan's N and K */
     int dtype;                 /* bi_dtype_t */

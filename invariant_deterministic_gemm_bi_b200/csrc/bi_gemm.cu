@@ -56,7 +56,8 @@ struct KernelEntry {
 // Narrow tiles (BN <= 64) run on one CTA; wide ones (BN >= 128) on a CTA pair.  Every tile comes
 // in two forms: its preferred number of 128-byte K chunks per pipeline stage (3-D TMA boxes;
 // needs K to be a multiple of the chunk), and one chunk per stage for any other K.  The bf16
-// 128 x 32 tile has a third, small-batch form with 8 chunks per stage (see small_batch_kernel).
+// 128 x 32 and the FP8 128 x 64 tiles have a third, small-batch form with twice the preferred
+// chunks per stage (see dense_kernel_for).
 const KernelEntry kKernels[] = {
     BI_ENTRY(64, 32, 1, false, false),  BI_ENTRY(64, 32, 4, false, false),
     BI_ENTRY(128, 32, 1, false, false), BI_ENTRY(128, 32, 4, false, false),
@@ -64,6 +65,7 @@ const KernelEntry kKernels[] = {
     BI_ENTRY(128, 64, 1, false, false), BI_ENTRY(128, 64, 2, false, false),
     BI_ENTRY(128, 32, 1, true, false),  BI_ENTRY(128, 32, 4, true, false),
     BI_ENTRY(128, 64, 1, true, false),  BI_ENTRY(128, 64, 2, true, false),
+    BI_ENTRY(128, 64, 4, true, false),
     BI_ENTRY(128, 32, 1, false, true),  BI_ENTRY(128, 32, 4, false, true),
     BI_ENTRY(128, 64, 1, false, true),  BI_ENTRY(128, 64, 2, false, true),
     BI_ENTRY(128, 128, 1, false, true), BI_ENTRY(128, 128, 2, false, true),
@@ -130,8 +132,8 @@ RingGeom ring_geometry(const KernelEntry *k, int a_rows)
     }
     // The kernel relies on 2 <= sa <= sb (the A-slot reuse test reads the consumed ring) and, for
     // FP8, on sb groups outlasting the partial-product ring.  Every tile in kKernels satisfies
-    // this for every a_rows in [8, BM], except the 8-chunk small-batch form, which is valid up to
-    // 64 rows and used up to kSmallBatchRows = 64; set_rows reports a violation and the launch is
+    // this for every a_rows in [8, BM], except the small-batch forms, which are valid up to 64
+    // (bf16, 8 chunks) and 96 (FP8, 4 chunks) rows and used up to kSmallBatchRows = 64; set_rows reports a violation and the launch is
     // refused.  tests/test_abi.py checks the reported depths.
     return RingGeom{sa, sb, static_cast<uint32_t>(a_stride), static_cast<uint32_t>(a_region)};
 }
@@ -413,6 +415,8 @@ int dense_a_box_rows(int64_t M, int bm)
 bool set_rows(GemmParams *p, const KernelEntry *k, int a_rows)
 {
     const RingGeom g = ring_geometry(k, a_rows);
+    // FP8: the epilogue tracks partial products on the consumed ring, which must outlast them
+    const int nacc = k->fp8 ? ((512 / k->bn) < 8 ? (512 / k->bn) : 8) : 0;
     p->a_box_rows = a_rows;
     // the peer CTA of a pair has A rows to load unless the whole problem fits in 128 rows
     p->pair_a1 = (k->grouped || p->rows > 128) ? 1 : 0;
@@ -420,7 +424,8 @@ bool set_rows(GemmParams *p, const KernelEntry *k, int a_rows)
     p->sb = g.sb;
     p->a_stride = g.a_stride;
     p->b_offset = g.b_offset;
-    return g.sa >= 2 && g.sa <= g.sb && g.sa <= bi::kMaxSA && g.sb <= bi::kMaxSB;
+    return g.sa >= 2 && g.sa <= g.sb && g.sa <= bi::kMaxSA && g.sb <= bi::kMaxSB &&
+           (!k->fp8 || k->pair || g.sb > nacc / k->kc);
 }
 
 GemmParams base_params(const bi_plan_s *plan, const KernelEntry *k, int64_t rows, void *C, int64_t ldc,
@@ -501,9 +506,9 @@ int b_box_rows_for(const KernelEntry *k)
 }
 
 // A dense launch of M rows whose A boxes hold at most this many rows takes the plan's
-// small-batch kernel form (when it has one): with few A rows, groups of 8 K chunks halve the
-// per-group wait and commit overhead of the MMA thread, and the ring still holds two groups of
-// A and of B.
+// small-batch kernel form (when it has one): with few A rows, groups of twice the chunks halve
+// the per-group wait and commit overhead of the MMA thread, and the ring still holds two groups
+// of A and of B (and, for FP8, more groups than partial-product buffers).
 constexpr int kSmallBatchRows = 64;
 
 const KernelEntry *dense_kernel_for(const bi_plan_s *plan, int64_t M)
@@ -601,8 +606,9 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     p->dtype = dtype;
     p->experts = num_experts;
     p->kernel = k;
-    if (!fp8 && num_experts == 1 && k->bm == 128 && k->bn == 32 && k->kc == preferred_chunks(32))
-        p->kernel_small = find_kernel(128, 32, 8, false, false);
+    if (num_experts == 1 && !k->pair && k->bm == 128 && k->kc == preferred_chunks(k->bn) &&
+        k->bn == (fp8 ? 64 : 32))
+        p->kernel_small = find_kernel(128, k->bn, 2 * k->kc, fp8, false);
     *out = p;
     return BI_OK;
 }
