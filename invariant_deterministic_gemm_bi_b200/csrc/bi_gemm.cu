@@ -42,26 +42,32 @@ struct KernelEntry {
     bool pair;     // cta_group::2 on a cluster of two CTAs
     KernelFn fn;
     int smem;
+    int nsplit;    // MMAs per K step (MMA N = bn / nsplit)
 };
 
 #define BI_ENTRY(BM, BN, KC, F8, GR)                                                               \
     KernelEntry{bi::Epi<F8, BN>::kThreads, BM, BN, KC, F8, GR, false,                              \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, GR>,                                           \
-                bi::smem_bytes_for<BM, BN, KC, F8, GR>()}
+                bi::smem_bytes_for<BM, BN, KC, F8, GR>(), 1}
+#define BI_ENTRY_SPLIT2(BM, BN, KC)                                                                \
+    KernelEntry{bi::Epi<false, BN>::kThreads, BM, BN, KC, false, false, false,                     \
+                &bi::bi_gemm_kernel<BM, BN, KC, false, false, 2>,                                  \
+                bi::smem_bytes_for<BM, BN, KC, false, false, 2>(), 2}
 #define BI_PAIR(BN, KC, F8, GR)                                                                    \
     KernelEntry{bi::Epi<F8, BN>::kThreads, 256, BN, KC, F8, GR, true,                              \
                 &bi::bi_gemm_kernel_pair<BN, KC, F8, GR>,                                          \
-                bi::smem_bytes_for_pair<BN, KC, F8, GR>()}
+                bi::smem_bytes_for_pair<BN, KC, F8, GR>(), 1}
 
 // Narrow tiles (BN <= 64) run on one CTA; wide ones (BN >= 128) on a CTA pair.  Every tile comes
 // in two forms: its preferred number of 128-byte K chunks per pipeline stage (3-D TMA boxes;
 // needs K to be a multiple of the chunk), and one chunk per stage for any other K.  The bf16
 // 128 x 32 and the FP8 128 x 64 tiles have a third, small-batch form with twice the preferred
-// chunks per stage (see dense_kernel_for).
+// chunks per stage, and the bf16 128 x 32 tile a wide form that runs two adjacent tiles in
+// lockstep on one A operand (see dense_kernel_for).
 const KernelEntry kKernels[] = {
     BI_ENTRY(64, 32, 1, false, false),  BI_ENTRY(64, 32, 4, false, false),
     BI_ENTRY(128, 32, 1, false, false), BI_ENTRY(128, 32, 4, false, false),
-    BI_ENTRY(128, 32, 8, false, false),
+    BI_ENTRY(128, 32, 8, false, false), BI_ENTRY_SPLIT2(128, 64, 2),
     BI_ENTRY(128, 64, 1, false, false), BI_ENTRY(128, 64, 2, false, false),
     BI_ENTRY(128, 32, 1, true, false),  BI_ENTRY(128, 32, 4, true, false),
     BI_ENTRY(128, 64, 1, true, false),  BI_ENTRY(128, 64, 2, true, false),
@@ -83,7 +89,7 @@ const KernelEntry *find_kernel(int bm, int bn, int kc, bool fp8, bool grouped)
 {
     for (int i = 0; i < kNumKernels; ++i)
         if (kKernels[i].bm == bm && kKernels[i].bn == bn && kKernels[i].kc == kc &&
-            kKernels[i].fp8 == fp8 && kKernels[i].grouped == grouped)
+            kKernels[i].fp8 == fp8 && kKernels[i].grouped == grouped && kKernels[i].nsplit == 1)
             return &kKernels[i];
     return nullptr;
 }
@@ -261,6 +267,9 @@ struct bi_plan_s {
     // (dense plans only; may be null).  It issues the same MMAs in the same K order, so a row's
     // result does not depend on which of the two a launch takes.
     const KernelEntry *kernel_small = nullptr;
+    // Two adjacent tiles in lockstep on one A operand (the same MMA instructions in the same K
+    // order), for dense launches with more tiles than SMs.  May be null.
+    const KernelEntry *kernel_wide = nullptr;
     uint64_t timeout_ns = 2000000000ull;
     uint32_t debug_flags = 0;
     uint32_t flags = 0;      // BI_PLAN_* flags
@@ -511,10 +520,19 @@ int b_box_rows_for(const KernelEntry *k)
 // of A and of B (and, for FP8, more groups than partial-product buffers).
 constexpr int kSmallBatchRows = 64;
 
-const KernelEntry *dense_kernel_for(const bi_plan_s *plan, int64_t M)
+// A dense launch with more tiles than the device has SMs takes the plan's wide form (when it has
+// one): a CTA runs two adjacent column tiles in lockstep, so each A chunk is loaded once for both
+// and the launch needs half the CTAs, i.e. fewer waves.
+const KernelEntry *dense_kernel_for(const bi_plan_s *plan, const DeviceInfo *d, int64_t M)
 {
     if (plan->kernel_small && a_box_rows_for(plan->kernel_small, M) <= kSmallBatchRows)
         return plan->kernel_small;
+    if (plan->kernel_wide) {
+        const int64_t tiles = (M + plan->kernel->bm - 1) / plan->kernel->bm *
+                              ((plan->n + plan->kernel->bn - 1) / plan->kernel->bn);
+        if (tiles > d->num_sms)
+            return plan->kernel_wide;
+    }
     return plan->kernel;
 }
 
@@ -609,6 +627,11 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     if (num_experts == 1 && !k->pair && k->bm == 128 && k->kc == preferred_chunks(k->bn) &&
         k->bn == (fp8 ? 64 : 32))
         p->kernel_small = find_kernel(128, k->bn, 2 * k->kc, fp8, false);
+    if (num_experts == 1 && !fp8 && k->bm == 128 && k->bn == 32 && K % 64 == 0) {
+        for (int i = 0; i < kNumKernels; ++i)
+            if (kKernels[i].nsplit == 2 && kKernels[i].bm == 128 && kKernels[i].bn == 64)
+                p->kernel_wide = &kKernels[i];
+    }
     *out = p;
     return BI_OK;
 }
@@ -720,7 +743,7 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
     int *status = nullptr;
     if ((st = plan_status_word(plan, dev, &status)) != BI_OK)
         return st;
-    const KernelEntry *k = dense_kernel_for(plan, M);
+    const KernelEntry *k = dense_kernel_for(plan, d, M);
     if ((st = ensure_kernel_attr(k, d)) != BI_OK)
         return st;
     CUtensorMap ta, tb;
@@ -881,7 +904,7 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
         if (fp8 && cudaMemcpyAsync(sa_dev, scale_a_host, static_cast<size_t>(kb * ld_sa * 4),
                                    cudaMemcpyHostToDevice, stream) != cudaSuccess)
             return BI_ERR_CUDA;
-        const KernelEntry *k = dense_kernel_for(plan, M);
+        const KernelEntry *k = dense_kernel_for(plan, d, M);
         if ((st = ensure_kernel_attr(k, d)) != BI_OK)
             return st;
         CUtensorMap ta, tb;

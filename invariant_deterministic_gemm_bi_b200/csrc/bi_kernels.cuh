@@ -229,15 +229,20 @@ __device__ __forceinline__ void load_group_scales(const GemmParams &p, const flo
     }
 }
 
-// BN      : output columns per tile = MMA N (multiple of 32, <= 256; FP8 <= 128)
+// BN      : output columns per tile (multiple of 32, <= 256; FP8 <= 128)
 // FP8     : e4m3 operands with fp32 block scales (else bf16)
 // GROUPED : MoE grouped layout (bf16 only)
 // KC      : 128-byte K chunks per pipeline stage (group).  KC > 1 loads a group with one 3-D TMA
 //           box per operand (chunk index as the third coordinate), so the producer and MMA
 //           threads pay their per-stage handshakes once per KC chunks.  The MMA still walks the
 //           chunks of a tile one by one in ascending K: KC changes no bit of the result.
+// NSPLIT  : MMAs per K step.  The MMA instruction is BM x (BN / NSPLIT) x K; split s covers the
+//           tile's columns [s BN/NSPLIT, (s+1) BN/NSPLIT) and accumulates into the same columns
+//           of the TMEM accumulator.  NSPLIT = 2 runs two adjacent (BN/2)-wide tiles of a plan in
+//           lockstep on one A operand: every output element is still computed by a
+//           BM x (BN/2) x K instruction sequence in ascending K, as in a (BN/2)-wide launch.
 // The ring depths follow from (BM, BN, KC) (see Rings).
-template <int BM, int BN, int KC, bool FP8, bool GROUPED>
+template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1>
 __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     bi_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b, const GemmParams p)
@@ -247,6 +252,9 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     static_assert(!FP8 || BN <= 128, "FP8 keeps BN fp32 accumulators per thread: BN <= 128");
     static_assert(!(FP8 && GROUPED), "grouped FP8 is not built");
     static_assert(KC >= 1 && KC <= 8, "1..8 chunks per group");
+    static_assert(NSPLIT == 1 || (NSPLIT == 2 && !FP8 && !GROUPED && BN == 64),
+                  "split MMAs: bf16 dense 64-wide tiles as two 32-wide instructions");
+    constexpr int kMmaN = BN / NSPLIT;                   // MMA instruction N
     using R = Rings<BM, BN, KC>;
     constexpr int kElemsPerRow = FP8 ? 128 : 64;         // K elements per 128-byte row
     constexpr int kMmaK = FP8 ? 32 : 16;                 // K per tcgen05.mma
@@ -265,7 +273,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     static_assert(kTmemColsNeeded <= 512, "TMEM holds 512 columns");
     static_assert(!FP8 || kNumAcc >= 2 * KC, "FP8 needs two groups of partial buffers");
     // (the host keeps sb > kNumAcc / KC so the FP8 epilogue can track partials on the consumed ring)
-    constexpr uint32_t kIdesc = FP8 ? ptx::idesc_e4m3(BM, BN) : ptx::idesc_bf16(BM, BN);
+    constexpr uint32_t kIdesc = FP8 ? ptx::idesc_e4m3(BM, kMmaN) : ptx::idesc_bf16(BM, kMmaN);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
@@ -557,10 +565,16 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                             const uint64_t step = static_cast<uint64_t>((q * kBytesPerMmaK) >> 4);
                             // bf16: accumulate across the whole K of the tile; FP8: one K chunk
                             const uint32_t accumulate = (q > 0) ? 1u : (FP8 ? 0u : (chunk > 0 ? 1u : 0u));
-                            if constexpr (FP8)
-                                ptx::mma_e4m3_ss(d, a_desc + step, b_desc + step, kIdesc, accumulate);
-                            else
-                                ptx::mma_bf16_ss(d, a_desc + step, b_desc + step, kIdesc, accumulate);
+#pragma unroll
+                            for (int sp = 0; sp < NSPLIT; ++sp) {
+                                // split sp: B rows and accumulator columns [sp kMmaN, (sp+1) kMmaN)
+                                const uint64_t b_sp = static_cast<uint64_t>((sp * kMmaN * kRowBytes) >> 4);
+                                if constexpr (FP8)
+                                    ptx::mma_e4m3_ss(d, a_desc + step, b_desc + step, kIdesc, accumulate);
+                                else
+                                    ptx::mma_bf16_ss(d + sp * kMmaN, a_desc + step, b_desc + b_sp + step,
+                                                     kIdesc, accumulate);
+                            }
                         }
                         return true;
                     };
@@ -746,7 +760,7 @@ __global__ void bi_zero_kernel(__nv_bfloat16 *c, int64_t ldc, int64_t m, int64_t
     }
 }
 
-template <int BM, int BN, int KC, bool FP8, bool GROUPED>
+template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1>
 constexpr int smem_bytes_for()
 {
     return 1024 + kRingBytes + 1024 + (GROUPED ? 2 * (kMaxExperts + 1) * 4 : 0);
