@@ -49,10 +49,10 @@ struct KernelEntry {
     KernelEntry{bi::Epi<F8, BN>::kThreads, BM, BN, KC, F8, GR, false,                              \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, GR>,                                           \
                 bi::smem_bytes_for<BM, BN, KC, F8, GR>(), 1}
-#define BI_ENTRY_SPLIT2(BM, BN, KC)                                                                \
-    KernelEntry{bi::Epi<false, BN>::kThreads, BM, BN, KC, false, false, false,                     \
-                &bi::bi_gemm_kernel<BM, BN, KC, false, false, 2>,                                  \
-                bi::smem_bytes_for<BM, BN, KC, false, false, 2>(), 2}
+#define BI_ENTRY_SPLIT2(BM, BN, KC, F8)                                                            \
+    KernelEntry{bi::Epi<F8, BN>::kThreads, BM, BN, KC, F8, false, false,                           \
+                &bi::bi_gemm_kernel<BM, BN, KC, F8, false, 2>,                                     \
+                bi::smem_bytes_for<BM, BN, KC, F8, false, 2>(), 2}
 #define BI_PAIR(BN, KC, F8, GR)                                                                    \
     KernelEntry{bi::Epi<F8, BN>::kThreads, 256, BN, KC, F8, GR, true,                              \
                 &bi::bi_gemm_kernel_pair<BN, KC, F8, GR>,                                          \
@@ -62,16 +62,16 @@ struct KernelEntry {
 // in two forms: its preferred number of 128-byte K chunks per pipeline stage (3-D TMA boxes;
 // needs K to be a multiple of the chunk), and one chunk per stage for any other K.  The bf16
 // 128 x 32 and the FP8 128 x 64 tiles have a third, small-batch form with twice the preferred
-// chunks per stage, and the bf16 128 x 32 tile a wide form that runs two adjacent tiles in
-// lockstep on one A operand (see dense_kernel_for).
+// chunks per stage, and a wide form that runs two adjacent tiles in lockstep on one A operand
+// (see dense_kernel_for).
 const KernelEntry kKernels[] = {
     BI_ENTRY(64, 32, 1, false, false),  BI_ENTRY(64, 32, 4, false, false),
     BI_ENTRY(128, 32, 1, false, false), BI_ENTRY(128, 32, 4, false, false),
-    BI_ENTRY(128, 32, 8, false, false), BI_ENTRY_SPLIT2(128, 64, 2),
+    BI_ENTRY(128, 32, 8, false, false), BI_ENTRY_SPLIT2(128, 64, 2, false),
     BI_ENTRY(128, 64, 1, false, false), BI_ENTRY(128, 64, 2, false, false),
     BI_ENTRY(128, 32, 1, true, false),  BI_ENTRY(128, 32, 4, true, false),
     BI_ENTRY(128, 64, 1, true, false),  BI_ENTRY(128, 64, 2, true, false),
-    BI_ENTRY(128, 64, 4, true, false),
+    BI_ENTRY(128, 64, 4, true, false),  BI_ENTRY_SPLIT2(128, 128, 2, true),
     BI_ENTRY(128, 32, 1, false, true),  BI_ENTRY(128, 32, 4, false, true),
     BI_ENTRY(128, 64, 1, false, true),  BI_ENTRY(128, 64, 2, false, true),
     BI_ENTRY(128, 128, 1, false, true), BI_ENTRY(128, 128, 2, false, true),
@@ -627,9 +627,11 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     if (num_experts == 1 && !k->pair && k->bm == 128 && k->kc == preferred_chunks(k->bn) &&
         k->bn == (fp8 ? 64 : 32))
         p->kernel_small = find_kernel(128, k->bn, 2 * k->kc, fp8, false);
-    if (num_experts == 1 && !fp8 && k->bm == 128 && k->bn == 32 && K % 64 == 0) {
+    if (num_experts == 1 && !k->pair && k->bm == 128 && k->bn == (fp8 ? 64 : 32) &&
+        K % chunk_elems == 0) {
         for (int i = 0; i < kNumKernels; ++i)
-            if (kKernels[i].nsplit == 2 && kKernels[i].bm == 128 && kKernels[i].bn == 64)
+            if (kKernels[i].nsplit == 2 && kKernels[i].bm == 128 && kKernels[i].bn == 2 * k->bn &&
+                kKernels[i].fp8 == fp8)
                 p->kernel_wide = &kKernels[i];
     }
     *out = p;

@@ -238,9 +238,10 @@ __device__ __forceinline__ void load_group_scales(const GemmParams &p, const flo
 //           chunks of a tile one by one in ascending K: KC changes no bit of the result.
 // NSPLIT  : MMAs per K step.  The MMA instruction is BM x (BN / NSPLIT) x K; split s covers the
 //           tile's columns [s BN/NSPLIT, (s+1) BN/NSPLIT) and accumulates into the same columns
-//           of the TMEM accumulator.  NSPLIT = 2 runs two adjacent (BN/2)-wide tiles of a plan in
-//           lockstep on one A operand: every output element is still computed by a
-//           BM x (BN/2) x K instruction sequence in ascending K, as in a (BN/2)-wide launch.
+//           of the TMEM accumulator (FP8: of each partial-product buffer).  NSPLIT = 2 runs two
+//           adjacent (BN/2)-wide tiles of a plan in lockstep on one A operand: every output
+//           element is still computed by a BM x (BN/2) x K instruction sequence in ascending K
+//           (FP8: and promoted in ascending kb), as in a (BN/2)-wide launch.
 // The ring depths follow from (BM, BN, KC) (see Rings).
 template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1>
 __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
@@ -252,8 +253,8 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     static_assert(!FP8 || BN <= 128, "FP8 keeps BN fp32 accumulators per thread: BN <= 128");
     static_assert(!(FP8 && GROUPED), "grouped FP8 is not built");
     static_assert(KC >= 1 && KC <= 8, "1..8 chunks per group");
-    static_assert(NSPLIT == 1 || (NSPLIT == 2 && !FP8 && !GROUPED && BN == 64),
-                  "split MMAs: bf16 dense 64-wide tiles as two 32-wide instructions");
+    static_assert(NSPLIT == 1 || (NSPLIT == 2 && !GROUPED && BN == (FP8 ? 128 : 64)),
+                  "split MMAs: dense bf16 64-wide (FP8 128-wide) tiles as two half-width instructions");
     constexpr int kMmaN = BN / NSPLIT;                   // MMA instruction N
     using R = Rings<BM, BN, KC>;
     constexpr int kElemsPerRow = FP8 ? 128 : 64;         // K elements per 128-byte row
@@ -570,7 +571,8 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                                 // split sp: B rows and accumulator columns [sp kMmaN, (sp+1) kMmaN)
                                 const uint64_t b_sp = static_cast<uint64_t>((sp * kMmaN * kRowBytes) >> 4);
                                 if constexpr (FP8)
-                                    ptx::mma_e4m3_ss(d, a_desc + step, b_desc + step, kIdesc, accumulate);
+                                    ptx::mma_e4m3_ss(d + sp * kMmaN, a_desc + step, b_desc + b_sp + step,
+                                                     kIdesc, accumulate);
                                 else
                                     ptx::mma_bf16_ss(d + sp * kMmaN, a_desc + step, b_desc + b_sp + step,
                                                      kIdesc, accumulate);
