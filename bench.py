@@ -601,6 +601,26 @@ def measure_extras(bg, inputs, dev, stream, peaks):
         res[f"moe_T{T}"] = {"us": t * 1e6, "TFLOP/s": tf, "tensor_frac": tf / bf16_peak,
                             "GB/s": b / t / 1e9, "hbm_frac": b / t / 1e9 / hbm,
                             "active_experts": active}
+    del B
+    # Fixed-split-K research variant on the decode shape (not the product path): what dropping
+    # split-K costs at small M.  Bytes are the algorithmic ones (workspace traffic not counted).
+    N, K = N_DEC, K_DEC
+    Bs = [inputs.bf16_gaussian((N, K), seed=6001 + i, std=K ** -0.5, device=dev) for i in range(4)]
+    for S in (2, 4, 8):
+        plan = bg.bi_gemm_plan_splitk(N, K, S)
+        for M in (1, 16, 64, 256):
+            A = inputs.bf16_gaussian((M, K), seed=6002, device=dev)
+            C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(bg.bi_gemm_splitk_workspace_bytes(plan, M) // 4, dtype=torch.float32,
+                             device=dev)
+            fns = [lambda i=i: bg.bi_gemm_run_splitk(plan, A, Bs[i % 4], C, ws, stream=stream)
+                   for i in range(8)]
+            t = graph_time_per_launch(fns, stream, reps=4)
+            b = 2 * N * K + 2 * M * K + 2 * M * N
+            res[f"splitk_S{S}_M{M}"] = {"us": t * 1e6, "GB/s": b / t / 1e9,
+                                        "hbm_frac": b / t / 1e9 / hbm,
+                                        "tile": f"128x{bg.bi_gemm_plan_describe(plan)['block_n']}"}
+            del A, C, ws
     return res
 
 

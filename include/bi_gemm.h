@@ -88,11 +88,13 @@ typedef struct {
     int cta_group;             /* CTAs that share one MMA (1 or 2) */
     int mma_m, mma_n, mma_k;   /* tcgen05.mma instruction shape */
     int stages;                /* depth of the B (weight) shared-memory ring */
-    int k_order_id;            /* 0 = ascending K blocks, whole K per CTA, no split-K */
+    int k_order_id;            /* 0 = ascending K blocks, whole K per CTA, no split-K;
+                                  1 = fixed split-K research plan (see bi_gemm_plan_splitk) */
     int threads_per_cta;
     int smem_bytes;            /* dynamic shared memory per CTA */
     int tmem_columns;          /* tensor-memory columns allocated per CTA */
     int stages_a;              /* depth of the A shared-memory ring (<= stages) */
+    int k_splits;              /* 1, or the split count of a split-K research plan */
 } bi_plan_info_t;
 
 /* Library version check: returns BI_GEMM_ABI_VERSION. */
@@ -227,6 +229,37 @@ bi_status_t bi_gemm_sync_status(bi_plan_t plan, cudaStream_t stream);
  * and returns, so the context stays usable.
  */
 bi_status_t bi_gemm_set_wait_timeout(bi_plan_t plan, uint64_t timeout_ns);
+
+/*
+ * Fixed-split-K research variant.  NOT the batch-invariant product path: the pages drop split-K
+ * from the GEMM because a split count chosen by heuristics (per batch size, occupancy or memory
+ * pressure) changes the reduction order ("DeepSeek V4 的隐藏关键特性被挖出来了" (wmrh.cn), section
+ * 2.2).  This plan fixes the split instead: splits = 2, 4 or 8, chosen by the caller, and the tile
+ * (128 x BN, BN the widest of 128 / 64 / 32 that gives at least 100 work units) follow from
+ * (N, K, splits) alone.  Split s of a tile accumulates the K chunks (128 bytes each)
+ * [s*nkb/splits, (s+1)*nkb/splits) (integer division) in ascending K into an fp32 workspace, and a
+ * second kernel adds the splits in a fixed pairwise tree, ((p0 + p1) + (p2 + p3)) + ..., then
+ * rounds once to bf16.  The split points and the merge order depend on (N, K, splits) only, so a
+ * row's bits still do not depend on M, but they differ from the product plan's bits for the same
+ * (N, K).  bf16 only.  bi_gemm_run refuses such a plan; bi_gemm_run_splitk refuses any other.
+ * Errors: BI_ERR_INVALID_ARG (splits not 2, 4 or 8), BI_ERR_UNSUPPORTED_SHAPE (fewer K chunks
+ * than splits).
+ */
+bi_status_t bi_gemm_plan_splitk(bi_plan_t *out, int64_t N, int64_t K, int splits);
+
+/* Bytes of fp32 workspace bi_gemm_run_splitk needs for M rows: splits * M * roundup(N, 4) * 4
+ * (0 for a plan that is not a split-K plan, or M <= 0). */
+size_t bi_gemm_splitk_workspace_bytes(bi_plan_t plan, int64_t M);
+
+/* C = A . B^T with a split-K plan.  Arguments as bi_gemm_run (bf16, no scales), plus a caller-
+ * owned, 16-byte aligned device workspace of at least bi_gemm_splitk_workspace_bytes(plan, M)
+ * bytes, which the call overwrites.  Two kernels on `stream`: the split GEMM and the merge. */
+bi_status_t bi_gemm_run_splitk(bi_plan_t plan, int64_t M,
+                               const void *A, int64_t lda,
+                               const void *B, int64_t ldb,
+                               void *C, int64_t ldc,
+                               void *workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
 
 /*
  * Plan flags; 0 clears them all.

@@ -20,10 +20,13 @@ from .binding import (  # noqa: F401
     bi_gemm_plan_describe,
     bi_gemm_plan_destroy,
     bi_gemm_plan_set_flags,
+    bi_gemm_plan_splitk,
     bi_gemm_run,
     bi_gemm_run_host,
     bi_gemm_run_host_noalloc,
+    bi_gemm_run_splitk,
     bi_gemm_set_wait_timeout,
+    bi_gemm_splitk_workspace_bytes,
     bi_gemm_sync_status,
     bi_grouped_gemm_run,
     bi_status_string,

@@ -33,6 +33,7 @@ EXPORTED = [
     "bi_gemm_plan_describe", "bi_gemm_run", "bi_grouped_gemm_run", "bi_gemm_run_host",
     "bi_gemm_sync_status", "bi_gemm_set_wait_timeout", "bi_gemm_debug_set_flags",
     "bi_gemm_run_host_noalloc", "bi_gemm_plan_set_flags",
+    "bi_gemm_plan_splitk", "bi_gemm_splitk_workspace_bytes", "bi_gemm_run_splitk",
 ]
 
 
@@ -51,7 +52,7 @@ class PlanInfo(ctypes.Structure):
         ("mma_n", ctypes.c_int), ("mma_k", ctypes.c_int), ("stages", ctypes.c_int),
         ("k_order_id", ctypes.c_int), ("threads_per_cta", ctypes.c_int),
         ("smem_bytes", ctypes.c_int), ("tmem_columns", ctypes.c_int),
-        ("stages_a", ctypes.c_int),
+        ("stages_a", ctypes.c_int), ("k_splits", ctypes.c_int),
     ]
 
     def as_dict(self):
@@ -97,6 +98,12 @@ def load_library(path: str = LIB_PATH):
     lib.bi_gemm_debug_set_flags.argtypes = [vp, u32]
     lib.bi_gemm_plan_set_flags.restype = i32
     lib.bi_gemm_plan_set_flags.argtypes = [vp, u32]
+    lib.bi_gemm_plan_splitk.restype = i32
+    lib.bi_gemm_plan_splitk.argtypes = [ctypes.POINTER(vp), i64, i64, i32]
+    lib.bi_gemm_splitk_workspace_bytes.restype = ctypes.c_size_t
+    lib.bi_gemm_splitk_workspace_bytes.argtypes = [vp, i64]
+    lib.bi_gemm_run_splitk.restype = i32
+    lib.bi_gemm_run_splitk.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, ctypes.c_size_t, vp]
     if path == LIB_PATH:
         _LIB = lib
     return lib
@@ -233,6 +240,29 @@ def bi_gemm_sync_status(plan: Plan, stream=None, raise_on_error: bool = True) ->
 
 def bi_gemm_set_wait_timeout(plan: Plan, timeout_ns: int):
     _check(load_library().bi_gemm_set_wait_timeout(plan.handle, timeout_ns), "bi_gemm_set_wait_timeout")
+
+
+def bi_gemm_plan_splitk(N: int, K: int, splits: int) -> Plan:
+    """Fixed-split-K research plan (not the batch-invariant product path), bf16."""
+    h = ctypes.c_void_p()
+    _check(load_library().bi_gemm_plan_splitk(ctypes.byref(h), N, K, splits), "bi_gemm_plan_splitk")
+    return Plan(h.value, N, K, BI_DTYPE_BF16, 1)
+
+
+def bi_gemm_splitk_workspace_bytes(plan: Plan, M: int) -> int:
+    return int(load_library().bi_gemm_splitk_workspace_bytes(plan.handle, M))
+
+
+def bi_gemm_run_splitk(plan: Plan, A, B, C, workspace, stream=None, M: int | None = None):
+    """C[:M] = A[:M] . B^T with a split-K plan; workspace is a device tensor of at least
+    bi_gemm_splitk_workspace_bytes(plan, M) bytes."""
+    M = A.shape[0] if M is None else M
+    nbytes = workspace.numel() * workspace.element_size()
+    st = load_library().bi_gemm_run_splitk(plan.handle, M, _ptr(A), A.stride(0), _ptr(B), B.stride(0),
+                                           _ptr(C), C.stride(0), _ptr(workspace), nbytes,
+                                           _stream_handle(stream))
+    _check(st, "bi_gemm_run_splitk")
+    return C
 
 
 def bi_gemm_plan_set_flags(plan: Plan, flags: int):

@@ -43,20 +43,25 @@ struct KernelEntry {
     KernelFn fn;
     int smem;
     int nsplit;    // MMAs per K step (MMA N = bn / nsplit)
+    bool ksplit;   // fixed-split-K research variant (fp32 partials + merge)
 };
 
 #define BI_ENTRY(BM, BN, KC, F8, GR)                                                               \
     KernelEntry{bi::Epi<F8, BN>::kThreads, BM, BN, KC, F8, GR, false,                              \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, GR>,                                           \
-                bi::smem_bytes_for<BM, BN, KC, F8, GR>(), 1}
+                bi::smem_bytes_for<BM, BN, KC, F8, GR>(), 1, false}
+#define BI_ENTRY_KSPLIT(BM, BN, KC)                                                                \
+    KernelEntry{bi::Epi<false, BN>::kThreads, BM, BN, KC, false, false, false,                     \
+                &bi::bi_gemm_kernel<BM, BN, KC, false, false, 1, true>,                            \
+                bi::smem_bytes_for<BM, BN, KC, false, false, 1, true>(), 1, true}
 #define BI_ENTRY_SPLIT2(BM, BN, KC, F8)                                                            \
     KernelEntry{bi::Epi<F8, BN>::kThreads, BM, BN, KC, F8, false, false,                           \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, false, 2>,                                     \
-                bi::smem_bytes_for<BM, BN, KC, F8, false, 2>(), 2}
+                bi::smem_bytes_for<BM, BN, KC, F8, false, 2>(), 2, false}
 #define BI_PAIR(BN, KC, F8, GR)                                                                    \
     KernelEntry{bi::Epi<F8, BN>::kThreads, 256, BN, KC, F8, GR, true,                              \
                 &bi::bi_gemm_kernel_pair<BN, KC, F8, GR>,                                          \
-                bi::smem_bytes_for_pair<BN, KC, F8, GR>(), 1}
+                bi::smem_bytes_for_pair<BN, KC, F8, GR>(), 1, false}
 
 // Narrow tiles (BN <= 64) run on one CTA; wide ones (BN >= 128) on a CTA pair.  Every tile comes
 // in two forms: its preferred number of 128-byte K chunks per pipeline stage (3-D TMA boxes;
@@ -80,6 +85,10 @@ const KernelEntry kKernels[] = {
     BI_PAIR(128, 1, true, false),       BI_PAIR(128, 2, true, false),
     BI_PAIR(128, 1, false, true),       BI_PAIR(128, 2, false, true),
     BI_PAIR(256, 1, false, true),       BI_PAIR(256, 2, false, true),
+    // fixed-split-K research variant (bi_gemm_plan_splitk), not the product path
+    BI_ENTRY_KSPLIT(128, 32, 1),        BI_ENTRY_KSPLIT(128, 32, 4),
+    BI_ENTRY_KSPLIT(128, 64, 1),        BI_ENTRY_KSPLIT(128, 64, 2),
+    BI_ENTRY_KSPLIT(128, 128, 1),       BI_ENTRY_KSPLIT(128, 128, 2),
 };
 constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
 
@@ -89,7 +98,8 @@ const KernelEntry *find_kernel(int bm, int bn, int kc, bool fp8, bool grouped)
 {
     for (int i = 0; i < kNumKernels; ++i)
         if (kKernels[i].bm == bm && kKernels[i].bn == bn && kKernels[i].kc == kc &&
-            kKernels[i].fp8 == fp8 && kKernels[i].grouped == grouped && kKernels[i].nsplit == 1)
+            kKernels[i].fp8 == fp8 && kKernels[i].grouped == grouped && kKernels[i].nsplit == 1 &&
+            !kKernels[i].ksplit)
             return &kKernels[i];
     return nullptr;
 }
@@ -273,6 +283,7 @@ struct bi_plan_s {
     uint64_t timeout_ns = 2000000000ull;
     uint32_t debug_flags = 0;
     uint32_t flags = 0;      // BI_PLAN_* flags
+    int k_splits = 1;        // > 1: fixed-split-K research plan (bi_gemm_plan_splitk)
     std::mutex mu;
     int *status[kMaxDevices] = {};
 };
@@ -677,7 +688,8 @@ bi_status_t bi_gemm_plan_describe(bi_plan_t plan, bi_plan_info_t *info)
     const RingGeom g = ring_geometry(plan->kernel, plan->kernel->bm);
     info->stages = g.sb;
     info->stages_a = g.sa;
-    info->k_order_id = 0;
+    info->k_order_id = plan->k_splits > 1 ? 1 : 0;
+    info->k_splits = plan->k_splits;
     info->threads_per_cta = plan->kernel->threads;
     info->smem_bytes = plan->kernel->smem;
     const int nacc = fp8 ? ((512 / plan->kernel->bn) < 8 ? (512 / plan->kernel->bn) : 8) : 2;
@@ -718,7 +730,7 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
 {
     if (!plan)
         return BI_ERR_INVALID_ARG;
-    if (plan->experts != 1)
+    if (plan->experts != 1 || plan->k_splits > 1)
         return BI_ERR_INVALID_ARG;
     const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
     if (fp8) {
@@ -854,7 +866,7 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
 {
     if (!plan)
         return BI_ERR_INVALID_ARG;
-    if (plan->experts != 1 || M < 0)
+    if (plan->experts != 1 || plan->k_splits > 1 || M < 0)
         return BI_ERR_INVALID_ARG;
     if (M == 0 || plan->n == 0)
         return BI_OK;
@@ -934,6 +946,109 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
     if (cudaMemcpy(&host, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return BI_ERR_CUDA;
     return host == 0 ? BI_OK : static_cast<bi_status_t>(host);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Fixed-split-K research variant (not the batch-invariant product path)
+// ---------------------------------------------------------------------------------------------
+
+bi_status_t bi_gemm_plan_splitk(bi_plan_t *out, int64_t N, int64_t K, int splits)
+{
+    if (!out)
+        return BI_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (N < 0 || K < 0 || (splits != 2 && splits != 4 && splits != 8))
+        return BI_ERR_INVALID_ARG;
+    if (N > INT32_MAX / 2 || K > INT32_MAX / 2)
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    const int64_t nkb = (K * 2 + bi::kRowBytes - 1) / bi::kRowBytes;
+    if (nkb < splits)
+        return BI_ERR_UNSUPPORTED_SHAPE;   // every split must own at least one K chunk
+    // the widest tile that still gives >= 100 work units (tiles x splits) for one row tile
+    int bn = 32;
+    for (int cand = 128; cand >= 32; cand /= 2)
+        if ((N + cand - 1) / cand * splits >= 100) {
+            bn = cand;
+            break;
+        }
+    const int kc = (K > 0 && K % 64 == 0) ? preferred_chunks(bn) : 1;
+    const KernelEntry *k = nullptr;
+    for (int i = 0; i < kNumKernels; ++i)
+        if (kKernels[i].ksplit && kKernels[i].bn == bn && kKernels[i].kc == kc)
+            k = &kKernels[i];
+    if (!k)
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    bi_plan_s *p = new (std::nothrow) bi_plan_s();
+    if (!p)
+        return BI_ERR_INVALID_ARG;
+    p->n = N;
+    p->k = K;
+    p->dtype = BI_DTYPE_BF16;
+    p->experts = 1;
+    p->kernel = k;
+    p->k_splits = splits;
+    *out = p;
+    return BI_OK;
+}
+
+size_t bi_gemm_splitk_workspace_bytes(bi_plan_t plan, int64_t M)
+{
+    if (!plan || plan->k_splits <= 1 || M <= 0)
+        return 0;
+    const int64_t ld_ws = (plan->n + 3) / 4 * 4;
+    return static_cast<size_t>(plan->k_splits) * static_cast<size_t>(M) * static_cast<size_t>(ld_ws) * 4u;
+}
+
+bi_status_t bi_gemm_run_splitk(bi_plan_t plan, int64_t M, const void *A, int64_t lda, const void *B,
+                               int64_t ldb, void *C, int64_t ldc, void *workspace,
+                               size_t workspace_bytes, cudaStream_t stream)
+{
+    if (!plan || plan->k_splits <= 1)
+        return BI_ERR_INVALID_ARG;
+    bi_status_t st = check_common(plan, M, A, lda, B, ldb, C, ldc);
+    if (st != BI_OK || M == 0 || plan->n == 0)
+        return st;
+    if (!workspace || workspace_bytes < bi_gemm_splitk_workspace_bytes(plan, M))
+        return BI_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u)
+        return BI_ERR_ALIGNMENT;
+    int dev = 0;
+    DeviceInfo *d = nullptr;
+    if ((st = current_device(&dev, &d)) != BI_OK)
+        return st;
+    if (plan->k == 0)
+        return launch_zero(C, ldc, M, plan->n, stream);
+    int *status = nullptr;
+    if ((st = plan_status_word(plan, dev, &status)) != BI_OK)
+        return st;
+    const KernelEntry *k = plan->kernel;
+    if ((st = ensure_kernel_attr(k, d)) != BI_OK)
+        return st;
+    CUtensorMap ta, tb;
+    const int a_rows = a_box_rows_for(k, M);
+    if ((st = encode_operand(&ta, A, false, plan->k, M, lda, a_rows, k->kc)) != BI_OK)
+        return st;
+    if ((st = encode_operand(&tb, B, false, plan->k, plan->n, ldb, b_box_rows_for(k), k->kc)) != BI_OK)
+        return st;
+    GemmParams p = base_params(plan, k, M, C, ldc, status);
+    if (!set_rows(&p, k, a_rows))
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    p.prefetch_b = 0;
+    p.k_splits = plan->k_splits;
+    p.ws = static_cast<float *>(workspace);
+    p.ld_ws = (plan->n + 3) / 4 * 4;
+    p.ws_split_stride = M * p.ld_ws;
+    const int64_t units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks * plan->k_splits;
+    if ((st = launch_main(k, d, ta, tb, p, units, stream)) != BI_OK)
+        return st;
+    const int64_t total = M * plan->n;
+    const int64_t blocks = (total + 255) / 256;
+    const int grid = static_cast<int>(blocks < d->num_sms * 8 ? blocks : d->num_sms * 8);
+    bi::bi_splitk_merge_kernel<<<grid, 256, 0, stream>>>(p.ws, p.ld_ws, p.ws_split_stride,
+                                                          plan->k_splits,
+                                                          static_cast<__nv_bfloat16 *>(C), ldc, M,
+                                                          plan->n);
+    return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
 bi_status_t bi_gemm_sync_status(bi_plan_t plan, cudaStream_t stream)

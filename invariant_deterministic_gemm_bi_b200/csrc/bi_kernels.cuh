@@ -92,6 +92,13 @@ struct GemmParams {
     int *status;             // device status word
     uint64_t timeout_cycles; // limit of every pipeline wait, in SM clock cycles
     uint32_t debug_flags;    // bit 0: skip the first load (fault-injection tests)
+    // fixed-split-K research variant only (SPLIT kernels): K chunks [s nkb / S, (s+1) nkb / S)
+    // (integer division; S = k_splits <= nkb) of a tile form split s; its fp32 partial goes to
+    // ws[s*ws_split_stride + row*ld_ws + col]
+    int32_t k_splits;
+    float *ws;
+    int64_t ld_ws;
+    int64_t ws_split_stride;
 };
 
 struct TileCoord {
@@ -99,6 +106,9 @@ struct TileCoord {
     int32_t row_end;  // one past the last row that belongs to this tile's problem
     int32_t n0;       // first output column
     int32_t b_row0;   // row of the tile's first B row in the (grouped: stacked) B tensor
+    int32_t kb0;      // first K chunk of this work unit (0 except for the split-K variant)
+    int32_t nkb;      // K chunks of this work unit
+    int32_t split;    // split index (split-K variant)
 };
 
 // Operand rings.  A pipeline stage ("group") carries KC 128-byte K chunks: KC chunks of A rows
@@ -136,6 +146,21 @@ __device__ __forceinline__ TileCoord dense_tile(const GemmParams &p, int bm, int
     tc.row_end = p.rows;
     tc.n0 = n_blk * bn;
     tc.b_row0 = tc.n0;
+    tc.kb0 = 0;
+    tc.nkb = p.num_k_blocks;
+    tc.split = 0;
+    return tc;
+}
+
+// Split-K variant: work unit u is split u % S of dense tile u / S.  The split points are fixed
+// by (K, S): split s owns the K chunks [s nkb / S, (s+1) nkb / S), never empty for S <= nkb.
+__device__ __forceinline__ TileCoord split_unit(const GemmParams &p, int bm, int bn, int u)
+{
+    TileCoord tc = dense_tile(p, bm, bn, u / p.k_splits);
+    tc.split = u % p.k_splits;
+    const int64_t nkb = p.num_k_blocks;
+    tc.kb0 = static_cast<int32_t>(tc.split * nkb / p.k_splits);
+    tc.nkb = static_cast<int32_t>((tc.split + 1) * nkb / p.k_splits) - tc.kb0;
     return tc;
 }
 
@@ -164,6 +189,9 @@ __device__ __forceinline__ TileCoord grouped_tile(const GemmParams &p, int bm, i
     tc.row_end = seg1;
     tc.n0 = n_blk * bn;
     tc.b_row0 = e * p.n + tc.n0;
+    tc.kb0 = 0;
+    tc.nkb = p.num_k_blocks;
+    tc.split = 0;
     return tc;
 }
 
@@ -196,6 +224,22 @@ __device__ __forceinline__ void store_row_chunk32(__nv_bfloat16 *crow, int col0,
         for (int j = 0; j < 32; ++j)
             if (col0 + j < n)
                 crow[col0 + j] = __float2bfloat16_rn(v[j]);
+    }
+}
+
+// Split-K variant: 32 consecutive fp32 partial sums of one row (row pitch a multiple of 4).
+__device__ __forceinline__ void store_row_chunk32_f32(float *wrow, int col0, int n, const float (&v)[32])
+{
+    if (col0 + 32 <= n) {
+        float4 *dst = reinterpret_cast<float4 *>(wrow + col0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (col0 + j < n)
+                wrow[col0 + j] = v[j];
     }
 }
 
@@ -242,8 +286,11 @@ __device__ __forceinline__ void load_group_scales(const GemmParams &p, const flo
 //           adjacent (BN/2)-wide tiles of a plan in lockstep on one A operand: every output
 //           element is still computed by a BM x (BN/2) x K instruction sequence in ascending K
 //           (FP8: and promoted in ascending kb), as in a (BN/2)-wide launch.
+// SPLIT   : the fixed-split-K research variant (bf16 dense only, not the batch-invariant product
+//           path): a work unit is one K split of a tile and its epilogue writes fp32 partial
+//           sums; bi_splitk_merge_kernel adds the splits in a fixed order.
 // The ring depths follow from (BM, BN, KC) (see Rings).
-template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1>
+template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool SPLIT = false>
 __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     bi_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b, const GemmParams p)
@@ -255,6 +302,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     static_assert(KC >= 1 && KC <= 8, "1..8 chunks per group");
     static_assert(NSPLIT == 1 || (NSPLIT == 2 && !GROUPED && BN == (FP8 ? 128 : 64)),
                   "split MMAs: dense bf16 64-wide (FP8 128-wide) tiles as two half-width instructions");
+    static_assert(!SPLIT || (!FP8 && !GROUPED && NSPLIT == 1), "split-K variant: bf16 dense");
     constexpr int kMmaN = BN / NSPLIT;                   // MMA instruction N
     using R = Rings<BM, BN, KC>;
     constexpr int kElemsPerRow = FP8 ? 128 : 64;         // K elements per 128-byte row
@@ -327,9 +375,19 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     auto tile_at = [&](int t) -> TileCoord {
         if constexpr (GROUPED)
             return grouped_tile(p, BM, BN, t, grp_prefix, grp_offs);
+        else if constexpr (SPLIT)
+            return split_unit(p, BM, BN, t);
         else
             return dense_tile(p, BM, BN, t);
     };
+    // groups of a work unit (a tile, or one K split of a tile)
+    auto groups_of = [&](const TileCoord &tc) -> int {
+        if constexpr (SPLIT)
+            return (tc.nkb + KC - 1) / KC;
+        else
+            return nkg;
+    };
+    const int tile_units = SPLIT ? p.k_splits : 1;
 
     // TMA producer state (used by thread 0 only).  Two cursors walk this CTA's (tile, group)
     // sequence: the B loads run `lag` = sb - sa groups ahead of the A loads.
@@ -346,7 +404,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     bool skipped_b0 = false;
     const uint64_t pol = ptx::policy_evict_normal();
     auto advance = [&](Cursor &c) {
-        if (++c.kg == nkg) {
+        if (++c.kg == groups_of(c.tc)) {
             c.kg = 0;
             c.t += gridDim.x;
             c.valid = c.t < num_tiles;
@@ -360,11 +418,12 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
             c.tc = tile_at(c.t);
         return c;
     };
-    auto load = [&](void *dst, const CUtensorMap *map, uint64_t *bar, int kg, int row) {
+    // load group kg of a work unit whose first K chunk is kb0
+    auto load = [&](void *dst, const CUtensorMap *map, uint64_t *bar, int kb0, int kg, int row) {
         if constexpr (KC == 1)
-            ptx::tma_load_2d(dst, map, bar, kg * kElemsPerRow, row, pol);
+            ptx::tma_load_2d(dst, map, bar, (kb0 + kg) * kElemsPerRow, row, pol);
         else
-            ptx::tma_load_3d(dst, map, bar, 0, row, kg * KC, pol);
+            ptx::tma_load_3d(dst, map, bar, 0, row, kb0 + kg * KC, pol);
     };
     // B group jb into slot bs; its slot is free (the consumed wait, if any, is done)
     auto issue_b = [&]() {
@@ -372,7 +431,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
             skipped_b0 = true;      // fault injection: this B group is never filled
         } else {
             ptx::mbar_arrive_expect_tx(&full[bs], R::kBBytes);
-            load(smem_b + bs * R::kBBytes, &tmap_b, &full[bs], cb.kg, cb.tc.b_row0);
+            load(smem_b + bs * R::kBBytes, &tmap_b, &full[bs], cb.tc.kb0, cb.kg, cb.tc.b_row0);
         }
         advance(cb);
         ++jb;
@@ -387,7 +446,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
         // sb groups of B (their slots are free in a fresh ring) are requested before that
         // kernel has completed.
         if (threadIdx.x == 0 && p.prefetch_b) {
-            num_tiles = p.num_m_blocks * p.num_n_blocks;
+            num_tiles = p.num_m_blocks * p.num_n_blocks * tile_units;
             cb = first_cursor();
             for (int i = 0; i < p.sb && cb.valid; ++i)
                 issue_b();
@@ -437,7 +496,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
         }
     } else {
         if (threadIdx.x == 0)
-            s_num_tiles = p.num_m_blocks * p.num_n_blocks;
+            s_num_tiles = p.num_m_blocks * p.num_n_blocks * tile_units;
     }
 
     ptx::tc_fence_before_sync();
@@ -471,7 +530,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                         }
                     }
                     ptx::mbar_arrive_expect_tx(&full[fs], KC * a_chunk_pitch);
-                    load(smem_a + as * p.a_stride, &tmap_a, &full[fs], ca.kg, ca.tc.m0);
+                    load(smem_a + as * p.a_stride, &tmap_a, &full[fs], ca.tc.kb0, ca.kg, ca.tc.m0);
                     advance(ca);
                     ++ja;
                     if (++as == SA)
@@ -528,7 +587,14 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                     ptx::tc_fence_after_sync();
                     d_tmem = tmem_base + a * BN;
                 }
-                for (int kg = 0; kg < nkg; ++kg) {
+                // chunks and groups of this work unit (the whole K of a tile, or one K split)
+                int unit_nkb = nkb, unit_nkg = nkg;
+                if constexpr (SPLIT) {
+                    const TileCoord tu = tile_at(t);
+                    unit_nkb = tu.nkb;
+                    unit_nkg = groups_of(tu);
+                }
+                for (int kg = 0; kg < unit_nkg; ++kg) {
                     if (!ptx::mbar_wait(&full[sb], pb, p.timeout_cycles, abort_flag)) {
                         record_failure(p, abort_flag, kStatusTimeout);
                         ok = false;
@@ -537,7 +603,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                     ptx::tc_fence_after_sync();
                     const uint64_t a_slot = a_desc0 + ((sa * p.a_stride) >> 4);
                     const uint64_t b_slot = b_desc0 + ((sb * R::kBBytes) >> 4);
-                    const int nc = nkb - kg * KC;   // chunks in this group: KC, except at a tile's end
+                    const int nc = unit_nkb - kg * KC;   // chunks in this group: KC, except at a unit's end
                     if constexpr (FP8) {
                         // Each K chunk's partial product goes to its own TMEM buffer.  Every
                         // epilogue thread hands the buffers back in chunk order, so the buffer of
@@ -659,8 +725,14 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj)
                         v[jj] = __uint_as_float(r[jj]);
-                    if (row_ok)
-                        store_row_chunk32(crow, tc.n0 + c * 32, p.n, v);
+                    if (row_ok) {
+                        if constexpr (SPLIT)
+                            store_row_chunk32_f32(p.ws + tc.split * p.ws_split_stride +
+                                                      static_cast<int64_t>(row) * p.ld_ws,
+                                                  tc.n0 + c * 32, p.n, v);
+                        else
+                            store_row_chunk32(crow, tc.n0 + c * 32, p.n, v);
+                    }
                 }
                 ++acc_iter;
             } else {
@@ -762,7 +834,31 @@ __global__ void bi_zero_kernel(__nv_bfloat16 *c, int64_t ldc, int64_t m, int64_t
     }
 }
 
-template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1>
+// Split-K variant: C = bf16_rne(sum of the S fp32 partials), added in a fixed pairwise tree,
+// ((p0 + p1) + (p2 + p3)) + ..., the same for every M.  S is 2, 4 or 8.
+__global__ void bi_splitk_merge_kernel(const float *ws, int64_t ld_ws, int64_t split_stride, int S,
+                                       __nv_bfloat16 *c, int64_t ldc, int64_t m, int64_t n)
+{
+    const int64_t total = m * n;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / n;
+        const int64_t col = i - r * n;
+        float v[8];
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            v[s] = s < S ? ws[s * split_stride + r * ld_ws + col] : 0.0f;
+#pragma unroll
+        for (int w = 1; w < 8; w *= 2)
+#pragma unroll
+            for (int s = 0; s + w < 8; s += 2 * w)
+                if (s + w < S)
+                    v[s] = v[s] + v[s + w];
+        c[r * ldc + col] = __float2bfloat16_rn(v[0]);
+    }
+}
+
+template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool SPLIT = false>
 constexpr int smem_bytes_for()
 {
     return 1024 + kRingBytes + 1024 + (GROUPED ? 2 * (kMaxExperts + 1) * 4 : 0);

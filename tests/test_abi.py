@@ -132,3 +132,31 @@ def test_plan_flags_accept_known_bits_only():
     before = bg.bi_gemm_plan_describe(plan)
     bg.bi_gemm_plan_set_flags(plan, bg.BI_PLAN_RESIDENT_WEIGHTS)
     assert bg.bi_gemm_plan_describe(plan) == before
+
+
+def test_splitk_research_plan_arguments():
+    lib = binding.load_library()
+    S = binding.STATUS
+    import ctypes
+    h = ctypes.c_void_p()
+    assert lib.bi_gemm_plan_splitk(ctypes.byref(h), 4096, 7168, 3) == S["BI_ERR_INVALID_ARG"]
+    assert lib.bi_gemm_plan_splitk(ctypes.byref(h), 4096, 7168, 16) == S["BI_ERR_INVALID_ARG"]
+    assert lib.bi_gemm_plan_splitk(None, 4096, 7168, 4) == S["BI_ERR_INVALID_ARG"]
+    # K = 192 is 3 chunks of 128 bytes: fewer than 4 splits
+    assert lib.bi_gemm_plan_splitk(ctypes.byref(h), 256, 192, 4) == S["BI_ERR_UNSUPPORTED_SHAPE"]
+    plan = bg.bi_gemm_plan_splitk(4096, 7168, 4)
+    info = bg.bi_gemm_plan_describe(plan)
+    assert info["k_splits"] == 4 and info["k_order_id"] == 1
+    assert info["block_n"] == 128            # 32 column tiles x 4 splits = 128 work units
+    assert bg.bi_gemm_splitk_workspace_bytes(plan, 64) == 4 * 64 * 4096 * 4
+    assert bg.bi_gemm_splitk_workspace_bytes(plan, 0) == 0
+    # a split-K plan is refused by the product entry points, and a product plan by the split one
+    h2 = plan.handle
+    assert lib.bi_gemm_run(h2, 1, 16, 7168, 16, 7168, 16, 4096, None, 0, None, None) == S["BI_ERR_INVALID_ARG"]
+    prod = bg.bi_gemm_plan(4096, 7168)
+    assert bg.bi_gemm_plan_describe(prod)["k_splits"] == 1
+    assert lib.bi_gemm_run_splitk(prod.handle, 1, 16, 7168, 16, 7168, 16, 4096, 16, 1 << 20, None) == S["BI_ERR_INVALID_ARG"]
+    # missing or short workspace
+    assert lib.bi_gemm_run_splitk(h2, 2, 16, 7168, 16, 7168, 16, 4096, None, 0, None) == S["BI_ERR_INVALID_ARG"]
+    need = bg.bi_gemm_splitk_workspace_bytes(plan, 2)
+    assert lib.bi_gemm_run_splitk(h2, 2, 16, 7168, 16, 7168, 16, 4096, 16, need - 4, None) == S["BI_ERR_INVALID_ARG"]
