@@ -1,7 +1,8 @@
 """Batch-invariant GEMM for NVIDIA B200 (sm_100a).
 
 C[M,N] = A[M,K] . B[N,K]^T with fp32 accumulation and bf16 output, computed by hand-written
-tcgen05/TMA kernels behind the C ABI in ``include/bi_gemm.h``.  Every output row is
+tcgen05/TMA kernels behind the C ABI in ``include/bi_gemm.h``; the MoE routing, dispatch, gather
+and combine steps around the grouped GEMM are in ``include/bi_moe.h``.  Every output row is
 bit-identical whatever the batch size, the row's position and the other rows in the batch.
 
 ``binding`` holds the ctypes wrapper (same names as the C ABI); ``inputs`` the seeded synthetic
@@ -29,6 +30,10 @@ from .binding import (  # noqa: F401
     bi_gemm_splitk_workspace_bytes,
     bi_gemm_sync_status,
     bi_grouped_gemm_run,
+    bi_moe_combine,
+    bi_moe_dispatch,
+    bi_moe_gather_rows,
+    bi_moe_route_topk,
     bi_status_string,
     load_library,
 )

@@ -1,4 +1,4 @@
-"""Thin ctypes binding of libbigemm (include/bi_gemm.h), same names as the C ABI.
+"""Thin ctypes binding of libbigemm (include/bi_gemm.h, include/bi_moe.h), same names as the C ABI.
 
 Argument marshalling only: every function takes torch tensors (device memory owned by torch)
 or raw integers, passes their pointers, strides and the current CUDA stream to the C entry
@@ -34,6 +34,7 @@ EXPORTED = [
     "bi_gemm_sync_status", "bi_gemm_set_wait_timeout", "bi_gemm_debug_set_flags",
     "bi_gemm_run_host_noalloc", "bi_gemm_plan_set_flags",
     "bi_gemm_plan_splitk", "bi_gemm_splitk_workspace_bytes", "bi_gemm_run_splitk",
+    "bi_moe_route_topk", "bi_moe_dispatch", "bi_moe_gather_rows", "bi_moe_combine",
 ]
 
 
@@ -104,6 +105,14 @@ def load_library(path: str = LIB_PATH):
     lib.bi_gemm_splitk_workspace_bytes.argtypes = [vp, i64]
     lib.bi_gemm_run_splitk.restype = i32
     lib.bi_gemm_run_splitk.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, ctypes.c_size_t, vp]
+    lib.bi_moe_route_topk.restype = i32
+    lib.bi_moe_route_topk.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp]
+    lib.bi_moe_dispatch.restype = i32
+    lib.bi_moe_dispatch.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
+    lib.bi_moe_gather_rows.restype = i32
+    lib.bi_moe_gather_rows.argtypes = [vp, i64, i64, vp, i64, vp, i64, vp]
+    lib.bi_moe_combine.restype = i32
+    lib.bi_moe_combine.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, i64, vp]
     if path == LIB_PATH:
         _LIB = lib
     return lib
@@ -272,3 +281,44 @@ def bi_gemm_plan_set_flags(plan: Plan, flags: int):
 
 def bi_gemm_debug_set_flags(plan: Plan, flags: int):
     _check(load_library().bi_gemm_debug_set_flags(plan.handle, flags), "bi_gemm_debug_set_flags")
+
+
+# ---------------------------------------------------------------------------------------------
+# MoE steps either side of the grouped GEMM (include/bi_moe.h)
+# ---------------------------------------------------------------------------------------------
+
+def bi_moe_route_topk(logits, k: int, experts, weights, stream=None):
+    """logits fp32 [T, E] -> experts int32 [T, k], weights fp32 [T, k] (device tensors)."""
+    T, E = logits.shape
+    _check(load_library().bi_moe_route_topk(_ptr(logits), logits.stride(0), T, E, k, _ptr(experts),
+                                            _ptr(weights), _stream_handle(stream)), "bi_moe_route_topk")
+    return experts, weights
+
+
+def bi_moe_dispatch(experts, num_experts: int, offsets, token_of_row, row_of_slot, stream=None):
+    """experts int32 [T, k] -> offsets int32 [E+1], token_of_row int32 [T*k], row_of_slot int32 [T*k]."""
+    T, k = experts.shape
+    _check(load_library().bi_moe_dispatch(_ptr(experts), T, num_experts, k, _ptr(offsets),
+                                          _ptr(token_of_row), _ptr(row_of_slot), _stream_handle(stream)),
+           "bi_moe_dispatch")
+    return offsets, token_of_row, row_of_slot
+
+
+def bi_moe_gather_rows(X, token_of_row, A_perm, stream=None):
+    """A_perm[r] = X[token_of_row[r]] (bf16 rows)."""
+    R = token_of_row.numel()
+    K = X.shape[1]
+    _check(load_library().bi_moe_gather_rows(_ptr(X), X.stride(0), K, _ptr(token_of_row), R,
+                                             _ptr(A_perm), A_perm.stride(0), _stream_handle(stream)),
+           "bi_moe_gather_rows")
+    return A_perm
+
+
+def bi_moe_combine(C_perm, row_of_slot, weights, Y, stream=None):
+    """Y[t] = sum_j weights[t, j] * C_perm[row_of_slot[t*k + j]] in slot order (bf16 out)."""
+    T, k = weights.shape
+    N = C_perm.shape[1]
+    _check(load_library().bi_moe_combine(_ptr(C_perm), C_perm.stride(0), N, _ptr(row_of_slot),
+                                         _ptr(weights), T, k, _ptr(Y), Y.stride(0),
+                                         _stream_handle(stream)), "bi_moe_combine")
+    return Y

@@ -17,9 +17,10 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 REPO = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = [os.path.join(CSRC, "bi_gemm.cu")]
-HEADERS = [os.path.join(CSRC, "bi_kernels.cuh"), os.path.join(CSRC, "ptx_sm100.cuh"),
-           os.path.join(REPO, "include", "bi_gemm.h")]
+SOURCES = [os.path.join(CSRC, "bi_gemm.cu"), os.path.join(CSRC, "bi_moe.cu")]
+HEADERS = [os.path.join(CSRC, "bi_kernels.cuh"), os.path.join(CSRC, "bi_kernels_pair.cuh"),
+           os.path.join(CSRC, "ptx_sm100.cuh"), os.path.join(REPO, "include", "bi_gemm.h"),
+           os.path.join(REPO, "include", "bi_moe.h")]
 LIB = os.path.join(PKG, "libbigemm.so")
 
 NVCC_FLAGS = [

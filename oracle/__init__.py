@@ -1,4 +1,5 @@
-"""CPU oracle for the batch-invariant GEMM -- test infrastructure only (see ``oracle.py``)."""
+"""CPU oracle for the batch-invariant GEMM -- test infrastructure only (see ``oracle.py``; the MoE
+steps around the grouped GEMM are in ``moe.py``)."""
 from .oracle import (  # noqa: F401
     bf16_to_f64,
     OracleLib,
@@ -13,3 +14,4 @@ from .oracle import (  # noqa: F401
     gemm_fp8_rows,
     grouped_gemm_bf16,
 )
+from . import moe  # noqa: F401,E402

@@ -14,13 +14,17 @@ import invariant_deterministic_gemm_bi_b200 as bg
 from invariant_deterministic_gemm_bi_b200 import binding
 
 REPO = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(REPO, "include", "bi_gemm.h")
+HEADERS = [os.path.join(REPO, "include", h) for h in sorted(os.listdir(os.path.join(REPO, "include")))
+           if h.endswith(".h")]
 
 
 def declared_functions():
-    text = open(HEADER, encoding="utf-8").read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(bi_[a-z0-9_]+)\s*\(", text)))
+    names = set()
+    for header in HEADERS:
+        text = open(header, encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(bi_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_library_exports_every_declared_symbol():
@@ -28,7 +32,7 @@ def test_library_exports_every_declared_symbol():
     names = declared_functions()
     assert len(names) >= 10
     for name in names:
-        assert hasattr(lib, name), f"{name} declared in bi_gemm.h but not exported"
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
     assert sorted(binding.EXPORTED) == names
 
 
