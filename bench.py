@@ -602,6 +602,35 @@ def measure_extras(bg, inputs, dev, stream, peaks):
                             "GB/s": b / t / 1e9, "hbm_frac": b / t / 1e9 / hbm,
                             "active_experts": active}
     del B
+    # The MoE layer around the grouped GEMM at T = 8192 and 64: route, dispatch, gather, combine
+    # (each timed on its own; bytes are the algorithmic ones of each step)
+    E, N, K, k = 64, 2048, 7168, 8
+    for T in (64, 8192):
+        g = inputs.generator(7000 + T, "cpu")
+        logits = torch.randn(T, E, generator=g, dtype=torch.float32).to(dev)
+        toks = inputs.bf16_gaussian((T, K), seed=7001, device=dev)
+        R = T * k
+        ex = torch.empty((T, k), dtype=torch.int32, device=dev)
+        w = torch.empty((T, k), dtype=torch.float32, device=dev)
+        off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        tok = torch.empty(R, dtype=torch.int32, device=dev)
+        ros = torch.empty(R, dtype=torch.int32, device=dev)
+        A = torch.empty((R, K), dtype=torch.bfloat16, device=dev)
+        Cp = inputs.bf16_gaussian((R, N), seed=7002, device=dev)
+        Y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+        steps = {
+            "route": (lambda: bg.bi_moe_route_topk(logits, k, ex, w, stream=stream), T * E * 4 + T * k * 8),
+            "dispatch": (lambda: bg.bi_moe_dispatch(ex, E, off, tok, ros, stream=stream), R * 4 * 3 + (E + 1) * 4),
+            "gather": (lambda: bg.bi_moe_gather_rows(toks, tok, A, stream=stream), 2 * R * K * 2 + R * 4),
+            "combine": (lambda: bg.bi_moe_combine(Cp, ros, w, Y, stream=stream), R * N * 2 + T * N * 2 + R * 8),
+        }
+        bg.bi_moe_route_topk(logits, k, ex, w, stream=stream)
+        bg.bi_moe_dispatch(ex, E, off, tok, ros, stream=stream)
+        for name, (fn, b) in steps.items():
+            t = graph_time_per_launch([fn] * 8, stream, reps=4)
+            res[f"moe_layer_T{T}_{name}"] = {"us": t * 1e6, "GB/s": b / t / 1e9,
+                                             "hbm_frac": b / t / 1e9 / hbm}
+        del A, Cp, Y, toks
     # Fixed-split-K research variant on the decode shape (not the product path): what dropping
     # split-K costs at small M.  Bytes are the algorithmic ones (workspace traffic not counted).
     N, K = N_DEC, K_DEC

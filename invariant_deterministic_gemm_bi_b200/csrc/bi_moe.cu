@@ -16,11 +16,14 @@ namespace {
 constexpr int kMaxE = 1024;
 constexpr int kMaxK = 8;
 constexpr unsigned kFull = 0xffffffffu;
+constexpr int kPerThread = 8;   // dispatch: consecutive pairs per thread per pass
 
 // ---------------------------------------------------------------------------------------------
 // Router: one warp per token.  Lane l holds the logits of experts l, l + 32, l + 64, ...
 // ---------------------------------------------------------------------------------------------
 
+// PL = logit slots per lane (ceil(E / 32) rounded up to a power of two)
+template <int PL>
 __global__ void __launch_bounds__(256) moe_route_kernel(const float *logits, int64_t ld, int64_t T,
                                                         int E, int k, int32_t *experts,
                                                         float *weights)
@@ -30,17 +33,16 @@ __global__ void __launch_bounds__(256) moe_route_kernel(const float *logits, int
     if (t >= T)
         return;   // warp-uniform
     const float *row = logits + t * ld;
-    const int per_lane = (E + 31) >> 5;
-    float v[kMaxE / 32];
+    float v[PL];
 #pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i) {
+    for (int i = 0; i < PL; ++i) {
         const int e = i * 32 + lane;
-        v[i] = (i < per_lane && e < E) ? row[e] : -INFINITY;
+        v[i] = e < E ? row[e] : -INFINITY;
     }
     // max over all experts (exact whatever the order)
     float m = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i)
+    for (int i = 0; i < PL; ++i)
         m = fmaxf(m, v[i]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1)
@@ -49,8 +51,8 @@ __global__ void __launch_bounds__(256) moe_route_kernel(const float *logits, int
     // lane adds the same pairs, so all lanes end with the same bits)
     float s = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i)
-        if (i < per_lane && i * 32 + lane < E)
+    for (int i = 0; i < PL; ++i)
+        if (i * 32 + lane < E)
             s = s + expf(v[i] - m);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1)
@@ -61,9 +63,9 @@ __global__ void __launch_bounds__(256) moe_route_kernel(const float *logits, int
         float bv = -INFINITY;
         int be = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < kMaxE / 32; ++i) {
+        for (int i = 0; i < PL; ++i) {
             const int e = i * 32 + lane;
-            if (i < per_lane && e < E && !((used >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
+            if (e < E && !((used >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
                 bv = v[i];
                 be = e;
             }
@@ -95,8 +97,12 @@ __global__ void __launch_bounds__(256) moe_count_kernel(const int32_t *experts, 
 {
     const int e = blockIdx.x;
     int c = 0;
-    for (int64_t i = threadIdx.x; i < n; i += blockDim.x)
-        c += experts[i] == e ? 1 : 0;
+    for (int64_t base = static_cast<int64_t>(threadIdx.x) * kPerThread; base < n;
+         base += static_cast<int64_t>(blockDim.x) * kPerThread) {
+#pragma unroll
+        for (int q = 0; q < kPerThread; ++q)
+            c += (base + q < n && experts[base + q] == e) ? 1 : 0;
+    }
     __shared__ int part[256];
     part[threadIdx.x] = c;
     __syncthreads();
@@ -131,28 +137,46 @@ __global__ void __launch_bounds__(256) moe_fill_kernel(const int32_t *experts, i
                                                        const int32_t *offsets, int32_t *token_of_row,
                                                        int32_t *row_of_slot)
 {
+    // One block per expert.  A pass covers 256 * 8 consecutive pairs: thread t owns the 8 pairs
+    // [base + 8t, base + 8t + 8), so an exclusive scan of the per-thread hit counts in thread
+    // order places the expert's rows in ascending pair order.
     const int e = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __shared__ int32_t wcount[8];
+    __shared__ int32_t wsum[8];
     int32_t running = offsets[e];
-    for (int64_t base = 0; base < n; base += blockDim.x) {
-        const int64_t i = base + threadIdx.x;
-        const bool hit = i < n && experts[i] == e;
-        const unsigned mask = __ballot_sync(kFull, hit);
-        if (lane == 0)
-            wcount[warp] = __popc(mask);
+    const int64_t span = static_cast<int64_t>(blockDim.x) * kPerThread;
+    for (int64_t base = 0; base < n; base += span) {
+        const int64_t i0 = base + static_cast<int64_t>(threadIdx.x) * kPerThread;
+        uint32_t hits = 0;
+#pragma unroll
+        for (int q = 0; q < kPerThread; ++q)
+            if (i0 + q < n && experts[i0 + q] == e)
+                hits |= 1u << q;
+        const int cnt = __popc(hits);
+        int incl = cnt;   // inclusive scan inside the warp
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off)
+                incl += y;
+        }
+        if (lane == 31)
+            wsum[warp] = incl;
         __syncthreads();
         int32_t before = 0, total = 0;
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
-            before += w < warp ? wcount[w] : 0;
-            total += wcount[w];
+            before += w < warp ? wsum[w] : 0;
+            total += wsum[w];
         }
-        if (hit) {
-            const int32_t r = running + before + __popc(mask & ((1u << lane) - 1u));
-            token_of_row[r] = static_cast<int32_t>(i / k);
-            row_of_slot[i] = r;
-        }
+        int32_t r = running + before + incl - cnt;
+#pragma unroll
+        for (int q = 0; q < kPerThread; ++q)
+            if ((hits >> q) & 1u) {
+                token_of_row[r] = static_cast<int32_t>((i0 + q) / k);
+                row_of_slot[i0 + q] = r;
+                ++r;
+            }
         running += total;
         __syncthreads();
     }
@@ -266,9 +290,20 @@ bi_status_t bi_moe_route_topk(const float *logits, int64_t ld_logits, int64_t T,
     bi_status_t st = moe_device(&sms);
     if (st != BI_OK)
         return st;
-    const int64_t blocks = (T * 32 + 255) / 256;
-    moe_route_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(logits, ld_logits, T, E, k,
-                                                                        experts, weights);
+    const unsigned blocks = static_cast<unsigned>((T * 32 + 255) / 256);
+    const int pl = (E + 31) / 32;
+    if (pl <= 1)
+        moe_route_kernel<1><<<blocks, 256, 0, stream>>>(logits, ld_logits, T, E, k, experts, weights);
+    else if (pl <= 2)
+        moe_route_kernel<2><<<blocks, 256, 0, stream>>>(logits, ld_logits, T, E, k, experts, weights);
+    else if (pl <= 4)
+        moe_route_kernel<4><<<blocks, 256, 0, stream>>>(logits, ld_logits, T, E, k, experts, weights);
+    else if (pl <= 8)
+        moe_route_kernel<8><<<blocks, 256, 0, stream>>>(logits, ld_logits, T, E, k, experts, weights);
+    else if (pl <= 16)
+        moe_route_kernel<16><<<blocks, 256, 0, stream>>>(logits, ld_logits, T, E, k, experts, weights);
+    else
+        moe_route_kernel<32><<<blocks, 256, 0, stream>>>(logits, ld_logits, T, E, k, experts, weights);
     return last_launch();
 }
 
