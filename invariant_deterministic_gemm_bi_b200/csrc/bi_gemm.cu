@@ -29,8 +29,9 @@ using bi::GemmParams;
 // Kernel registry: every instantiated configuration
 // ---------------------------------------------------------------------------------------------
 
+// (A map, B map, 8-row A map for short grouped segments, parameters)
 typedef void (*KernelFn)(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
-                         const GemmParams);
+                         const __grid_constant__ CUtensorMap, const GemmParams);
 
 struct KernelEntry {
     int threads;   // threads per CTA
@@ -58,6 +59,10 @@ struct KernelEntry {
     KernelEntry{bi::Epi<F8, BN>::kThreads, BM, BN, KC, F8, false, false,                           \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, false, 2>,                                     \
                 bi::smem_bytes_for<BM, BN, KC, F8, false, 2>(), 2, false}
+#define BI_ENTRY_GROUPED_SPLIT2(BM, BN, KC)                                                        \
+    KernelEntry{bi::Epi<false, BN>::kThreads, BM, BN, KC, false, true, false,                      \
+                &bi::bi_gemm_kernel<BM, BN, KC, false, true, 2>,                                   \
+                bi::smem_bytes_for<BM, BN, KC, false, true, 2>(), 2, false}
 #define BI_PAIR(BN, KC, F8, GR)                                                                    \
     KernelEntry{bi::Epi<F8, BN>::kThreads, 256, BN, KC, F8, GR, true,                              \
                 &bi::bi_gemm_kernel_pair<BN, KC, F8, GR>,                                          \
@@ -80,6 +85,7 @@ const KernelEntry kKernels[] = {
     BI_ENTRY(128, 32, 1, false, true),  BI_ENTRY(128, 32, 4, false, true),
     BI_ENTRY(128, 64, 1, false, true),  BI_ENTRY(128, 64, 2, false, true),
     BI_ENTRY(128, 128, 1, false, true), BI_ENTRY(128, 128, 2, false, true),
+    BI_ENTRY_GROUPED_SPLIT2(128, 256, 1),
     BI_PAIR(128, 1, false, false),      BI_PAIR(128, 2, false, false),
     BI_PAIR(256, 1, false, false),      BI_PAIR(256, 2, false, false),
     BI_PAIR(128, 1, true, false),       BI_PAIR(128, 2, true, false),
@@ -278,7 +284,8 @@ struct bi_plan_s {
     // result does not depend on which of the two a launch takes.
     const KernelEntry *kernel_small = nullptr;
     // Two adjacent tiles in lockstep on one A operand (the same MMA instructions in the same K
-    // order), for dense launches with more tiles than SMs.  May be null.
+    // order), for dense launches with more tiles than SMs and grouped launches with at least a
+    // tile's worth of rows per expert on average.  May be null.
     const KernelEntry *kernel_wide = nullptr;
     uint64_t timeout_ns = 2000000000ull;
     uint32_t debug_flags = 0;
@@ -481,8 +488,8 @@ GemmParams base_params(const bi_plan_s *plan, const KernelEntry *k, int64_t rows
 // up its shared and tensor memory) while that kernel finishes, and waits for it to complete
 // before touching global memory (bi::ptx::grid_dependency_wait).
 bi_status_t launch_main(const KernelEntry *k, const DeviceInfo *d, const CUtensorMap &ta,
-                        const CUtensorMap &tb, const GemmParams &p, int64_t units,
-                        cudaStream_t stream)
+                        const CUtensorMap &tb, const CUtensorMap &ta8, const GemmParams &p,
+                        int64_t units, cudaStream_t stream)
 {
     if (units < 1)
         units = 1;
@@ -509,7 +516,7 @@ bi_status_t launch_main(const KernelEntry *k, const DeviceInfo *d, const CUtenso
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, k->fn, ta, tb, p);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k->fn, ta, tb, ta8, p);
     return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
@@ -638,6 +645,11 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     if (num_experts == 1 && !k->pair && k->bm == 128 && k->kc == preferred_chunks(k->bn) &&
         k->bn == (fp8 ? 64 : 32))
         p->kernel_small = find_kernel(128, k->bn, 2 * k->kc, fp8, false);
+    if (num_experts > 1 && !k->pair && k->bm == 128 && k->bn == 128) {
+        for (int i = 0; i < kNumKernels; ++i)
+            if (kKernels[i].nsplit == 2 && kKernels[i].grouped && kKernels[i].bn == 256)
+                p->kernel_wide = &kKernels[i];
+    }
     if (num_experts == 1 && !k->pair && k->bm == 128 && k->bn == (fp8 ? 64 : 32) &&
         K % chunk_elems == 0) {
         for (int i = 0; i < kNumKernels; ++i)
@@ -773,7 +785,7 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
     p.ld_sa = ld_sa;
     p.scale_b = scale_b;
     const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-    return launch_main(k, d, ta, tb, p, tiles, stream);
+    return launch_main(k, d, ta, tb, ta, p, tiles, stream);
 }
 
 bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *A, int64_t lda,
@@ -800,12 +812,19 @@ bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *
     int *status = nullptr;
     if ((st = plan_status_word(plan, dev, &status)) != BI_OK)
         return st;
+    // With at least a tile's worth of rows per expert on average, adjacent column tiles run in
+    // lockstep on one A operand (the wide form: same MMA instructions, same K order).
     const KernelEntry *k = plan->kernel;
+    if (plan->kernel_wide && total_rows >= static_cast<int64_t>(plan->kernel->bm) * plan->experts)
+        k = plan->kernel_wide;
     if ((st = ensure_kernel_attr(k, d)) != BI_OK)
         return st;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, ta8;
     const int a_rows = k->pair ? 128 : k->bm;
     if ((st = encode_operand(&ta, A, false, plan->k, total_rows, lda, a_rows, k->kc)) != BI_OK)
+        return st;
+    // short segments load their rows as 8-row boxes
+    if ((st = encode_operand(&ta8, A, false, plan->k, total_rows, lda, 8, k->kc)) != BI_OK)
         return st;
     if ((st = encode_operand(&tb, B, false, plan->k, plan->n * plan->experts, ldb, b_box_rows_for(k),
                              k->kc)) != BI_OK)
@@ -816,7 +835,7 @@ bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *
     // Upper bound on the tile count without reading the offsets: sum_e ceil(len_e/BM) is at
     // most total_rows/BM + E.
     const int64_t max_tiles = (total_rows / k->bm + plan->experts) * p.num_n_blocks;
-    return launch_main(k, d, ta, tb, p, max_tiles, stream);
+    return launch_main(k, d, ta, tb, ta8, p, max_tiles, stream);
 }
 
 bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M, const void *A_host, int64_t lda,
@@ -934,7 +953,7 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
         p.ld_sa = fp8 ? ld_sa : 0;
         p.scale_b = fp8 ? scale_b : nullptr;
         const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-        if ((st = launch_main(k, d, ta, tb, p, tiles, stream)) != BI_OK)
+        if ((st = launch_main(k, d, ta, tb, ta, p, tiles, stream)) != BI_OK)
             return st;
     }
     if (cudaMemcpyAsync(C_host, C_dev, static_cast<size_t>(M * ldc * 2), cudaMemcpyDeviceToHost,
@@ -1039,7 +1058,7 @@ bi_status_t bi_gemm_run_splitk(bi_plan_t plan, int64_t M, const void *A, int64_t
     p.ld_ws = (plan->n + 3) / 4 * 4;
     p.ws_split_stride = M * p.ld_ws;
     const int64_t units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks * plan->k_splits;
-    if ((st = launch_main(k, d, ta, tb, p, units, stream)) != BI_OK)
+    if ((st = launch_main(k, d, ta, tb, ta, p, units, stream)) != BI_OK)
         return st;
     const int64_t total = M * plan->n;
     const int64_t blocks = (total + 255) / 256;

@@ -152,6 +152,18 @@ __device__ __forceinline__ TileCoord dense_tile(const GemmParams &p, int bm, int
     return tc;
 }
 
+// Grouped tiles whose segment has at most kShortSegmentRows rows from the tile's first row load
+// their A rows as ceil(rows / 8) boxes of 8 rows x KC chunks instead of one full box; the
+// shared-memory layout is then [8-row group][chunk][8 rows], which the MMA reads with a stride byte
+// offset of KC * 1024.  (More small boxes per stage cost more than the rows they save: TMA issues
+// small boxes slowly.)  Returns the number of 8-row boxes, or 0 for a full box.
+constexpr int kShortSegmentRows = 16;
+__device__ __forceinline__ int short_segment_boxes(const TileCoord &tc, int limit_rows)
+{
+    const int rows = tc.row_end - tc.m0;
+    return rows <= limit_rows ? (rows + 7) >> 3 : 0;
+}
+
 // Split-K variant: work unit u is split u % S of dense tile u / S.  The split points are fixed
 // by (K, S): split s owns the K chunks [s nkb / S, (s+1) nkb / S), never empty for S <= nkb.
 __device__ __forceinline__ TileCoord split_unit(const GemmParams &p, int bm, int bn, int u)
@@ -293,15 +305,18 @@ __device__ __forceinline__ void load_group_scales(const GemmParams &p, const flo
 template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool SPLIT = false>
 __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     bi_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                   const __grid_constant__ CUtensorMap tmap_b, const GemmParams p)
+                   const __grid_constant__ CUtensorMap tmap_b,
+                   const __grid_constant__ CUtensorMap tmap_a8, const GemmParams p)
 {
     static_assert(BM == 64 || BM == 128, "MMA M is 64 or 128");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32,256]");
     static_assert(!FP8 || BN <= 128, "FP8 keeps BN fp32 accumulators per thread: BN <= 128");
     static_assert(!(FP8 && GROUPED), "grouped FP8 is not built");
     static_assert(KC >= 1 && KC <= 8, "1..8 chunks per group");
-    static_assert(NSPLIT == 1 || (NSPLIT == 2 && !GROUPED && BN == (FP8 ? 128 : 64)),
-                  "split MMAs: dense bf16 64-wide (FP8 128-wide) tiles as two half-width instructions");
+    static_assert(NSPLIT == 1 ||
+                      (NSPLIT == 2 && (GROUPED ? (!FP8 && BN == 256) : BN == (FP8 ? 128 : 64))),
+                  "split MMAs: dense bf16 64-wide, FP8 128-wide and grouped bf16 256-wide tiles as "
+                  "two half-width instructions");
     static_assert(!SPLIT || (!FP8 && !GROUPED && NSPLIT == 1), "split-K variant: bf16 dense");
     constexpr int kMmaN = BN / NSPLIT;                   // MMA instruction N
     using R = Rings<BM, BN, KC>;
@@ -362,6 +377,8 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
         ptx::fence_mbarrier_init();
         ptx::prefetch_tmap(&tmap_a);
         ptx::prefetch_tmap(&tmap_b);
+        if constexpr (GROUPED)
+            ptx::prefetch_tmap(&tmap_a8);
     }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_base_smem, kTmemCols);
@@ -529,8 +546,19 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                             cph ^= 1u;
                         }
                     }
-                    ptx::mbar_arrive_expect_tx(&full[fs], KC * a_chunk_pitch);
-                    load(smem_a + as * p.a_stride, &tmap_a, &full[fs], ca.tc.kb0, ca.kg, ca.tc.m0);
+                    int nsub = 0;
+                    if constexpr (GROUPED)
+                        nsub = short_segment_boxes(ca.tc, kShortSegmentRows);
+                    if (nsub == 0) {
+                        ptx::mbar_arrive_expect_tx(&full[fs], KC * a_chunk_pitch);
+                        load(smem_a + as * p.a_stride, &tmap_a, &full[fs], ca.tc.kb0, ca.kg, ca.tc.m0);
+                    } else {
+                        // a short segment: its rows as 8-row boxes of all KC chunks
+                        ptx::mbar_arrive_expect_tx(&full[fs], static_cast<uint32_t>(nsub) * KC * 1024u);
+                        for (int i = 0; i < nsub; ++i)
+                            load(smem_a + as * p.a_stride + i * KC * 1024, &tmap_a8, &full[fs],
+                                 ca.tc.kb0, ca.kg, ca.tc.m0 + 8 * i);
+                    }
                     advance(ca);
                     ++ja;
                     if (++as == SA)
@@ -572,9 +600,19 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
             // bits), so every slot / chunk / K-step descriptor is a base plus an offset.
             const uint64_t a_desc0 = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_a));
             const uint64_t b_desc0 = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_b));
+            // A of a short grouped segment: 8-row groups KC * 1024 bytes apart, chunks 1024 apart
+            const uint64_t a_desc0_short = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_a), KC * 1024u);
             uint32_t acc_iter = 0;   // bf16: tiles done; FP8: K chunks done
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                uint64_t a_base = a_desc0;
+                uint32_t a_cp = a_chunk_pitch;   // bytes between the K chunks of an A slot
+                if constexpr (GROUPED) {
+                    if (short_segment_boxes(tile_at(t), kShortSegmentRows) != 0) {
+                        a_base = a_desc0_short;
+                        a_cp = 1024u;
+                    }
+                }
                 uint32_t d_tmem = 0;
                 if (!FP8) {
                     const uint32_t a = acc_iter % kNumAcc;
@@ -601,7 +639,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                         break;
                     }
                     ptx::tc_fence_after_sync();
-                    const uint64_t a_slot = a_desc0 + ((sa * p.a_stride) >> 4);
+                    const uint64_t a_slot = a_base + ((sa * p.a_stride) >> 4);
                     const uint64_t b_slot = b_desc0 + ((sb * R::kBBytes) >> 4);
                     const int nc = unit_nkb - kg * KC;   // chunks in this group: KC, except at a unit's end
                     if constexpr (FP8) {
@@ -625,7 +663,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                             d = tmem_base + (acc_iter % kNumAcc) * BN;
                             ++acc_iter;
                         }
-                        const uint64_t a_desc = a_slot + ((c * a_chunk_pitch) >> 4);
+                        const uint64_t a_desc = a_slot + ((c * a_cp) >> 4);
                         const uint64_t b_desc = b_slot + ((c * R::kBChunkBytes) >> 4);
 #pragma unroll
                         for (int q = 0; q < kMmaPerStage; ++q) {

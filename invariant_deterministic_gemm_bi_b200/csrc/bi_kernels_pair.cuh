@@ -42,7 +42,8 @@ struct PairRings {
 template <int BN, int KC, bool FP8, bool GROUPED>
 __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     bi_gemm_kernel_pair(const __grid_constant__ CUtensorMap tmap_a,
-                        const __grid_constant__ CUtensorMap tmap_b, const GemmParams p)
+                        const __grid_constant__ CUtensorMap tmap_b,
+                        const __grid_constant__ CUtensorMap tmap_a8, const GemmParams p)
 {
     static_assert(BN == 128 || BN == 256, "pair tiles are 128 or 256 wide");
     static_assert(!FP8 || BN == 128, "FP8 keeps BN fp32 accumulators per thread");
@@ -66,7 +67,27 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     // than 128 rows when the whole problem is smaller than a CTA's share; the peer loads no A
     // at all when the problem has at most 128 rows).
     const uint32_t a_chunk_pitch = static_cast<uint32_t>(p.a_box_rows) * kRowBytes;
-    const uint32_t group_bytes = 2u * R::kBBytes + KC * a_chunk_pitch * (p.pair_a1 ? 2u : 1u);
+    // How a tile's A rows are loaded.  Dense: each CTA loads its 128 rows (boxed to the problem's
+    // rows when it has fewer), the peer nothing when the problem has at most 128 rows.  Grouped:
+    // the segment's rows from the tile's first row decide -- at most kShortSegmentRows come in as 8-row boxes
+    // (layout [8-row group][chunk][8 rows]) to the leader, at most 128 as the leader's full box,
+    // more as both CTAs' full boxes.
+    struct ALoad {
+        int nsub;          // 8-row boxes of the leader (0: one full box)
+        bool peer;         // the peer CTA loads its 128 rows
+        uint32_t bytes;    // A bytes of one group over both CTAs
+    };
+    auto a_load = [&](const TileCoord &tc) -> ALoad {
+        ALoad al{0, p.pair_a1 != 0, 0};
+        if constexpr (GROUPED) {
+            const int rows = tc.row_end - tc.m0;
+            al.nsub = rows <= kShortSegmentRows ? (rows + 7) >> 3 : 0;
+            al.peer = rows > 128;
+        }
+        al.bytes = (al.nsub ? static_cast<uint32_t>(al.nsub) * 1024u : a_chunk_pitch) * KC +
+                   (al.peer ? KC * a_chunk_pitch : 0u);
+        return al;
+    };
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -104,6 +125,8 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
         ptx::fence_mbarrier_init();
         ptx::prefetch_tmap(&tmap_a);
         ptx::prefetch_tmap(&tmap_b);
+        if constexpr (GROUPED)
+            ptx::prefetch_tmap(&tmap_a8);
     }
     if (warp == 1) {
         ptx::tmem_alloc_pair(tmem_base_smem, kTmemCols);
@@ -181,6 +204,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                 const TileCoord tc = tile_at(t);
                 const int a_row = tc.m0 + 128 * static_cast<int>(rank);
                 const int b_row = tc.b_row0 + (BN / 2) * static_cast<int>(rank);
+                const ALoad al = a_load(tc);
                 for (int kg = 0; kg < nkg; ++kg, ++j) {
                     if (!ptx::mbar_wait(&consumed[s], ph ^ 1u, p.timeout_cycles, abort_flag)) {
                         record_failure(p, abort_flag, kStatusTimeout);
@@ -190,21 +214,24 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                     const uint32_t bar = full0_leader + s * 8;
                     if (!(j == 0 && (p.debug_flags & 1u) && rank == 0)) {   // fault injection skips
                         if (rank == 0)                                        // the leader's first group
-                            ptx::mbar_arrive_expect_tx(&full[s], group_bytes);
-                        const bool load_a = rank == 0 || p.pair_a1 != 0;
-                        if constexpr (KC == 1) {
-                            if (load_a)
-                                ptx::tma_load_2d_pair(smem_a + s * R::kABytes, &tmap_a, bar,
-                                                      kg * kElemsPerRow, a_row, pol);
+                            ptx::mbar_arrive_expect_tx(&full[s], 2u * R::kBBytes + al.bytes);
+                        const bool load_a = rank == 0 || al.peer;
+                        const int nbox = (rank == 0 && al.nsub) ? al.nsub : (load_a ? 1 : 0);
+                        const CUtensorMap *amap = (rank == 0 && al.nsub) ? &tmap_a8 : &tmap_a;
+                        // 8-row boxes go KC * 1024 bytes apart (each holds all KC chunks)
+                        for (int i = 0; i < nbox; ++i) {
+                            uint8_t *dst = smem_a + s * R::kABytes + i * KC * 1024;
+                            if constexpr (KC == 1)
+                                ptx::tma_load_2d_pair(dst, amap, bar, kg * kElemsPerRow, a_row + 8 * i, pol);
+                            else
+                                ptx::tma_load_3d_pair(dst, amap, bar, 0, a_row + 8 * i, kg * KC, pol);
+                        }
+                        if constexpr (KC == 1)
                             ptx::tma_load_2d_pair(smem_b + s * R::kBBytes, &tmap_b, bar,
                                                   kg * kElemsPerRow, b_row, pol);
-                        } else {
-                            if (load_a)
-                                ptx::tma_load_3d_pair(smem_a + s * R::kABytes, &tmap_a, bar, 0, a_row,
-                                                      kg * KC, pol);
+                        else
                             ptx::tma_load_3d_pair(smem_b + s * R::kBBytes, &tmap_b, bar, 0, b_row,
                                                   kg * KC, pol);
-                        }
                     }
                     if (++s == S) {
                         s = 0;
@@ -233,7 +260,16 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
             uint32_t ph = 0;
             uint32_t acc_iter = 0;   // bf16: tiles; FP8: K chunks
             bool ok = true;
+            const uint64_t a_desc0_short = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_a), KC * 1024u);
             for (int t = pair; t < num_tiles && ok; t += npairs) {
+                uint64_t a_base = a_desc0;
+                uint32_t a_cp = a_chunk_pitch;   // bytes between the K chunks of an A slot
+                if constexpr (GROUPED) {
+                    if (a_load(tile_at(t)).nsub != 0) {
+                        a_base = a_desc0_short;
+                        a_cp = 1024u;
+                    }
+                }
                 uint32_t d_tmem = 0;
                 if (!FP8) {
                     const uint32_t a = acc_iter % kNumAcc;
@@ -253,7 +289,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                         break;
                     }
                     ptx::tc_fence_after_sync();
-                    const uint64_t a_slot = a_desc0 + ((s * R::kABytes) >> 4);
+                    const uint64_t a_slot = a_base + ((s * R::kABytes) >> 4);
                     const uint64_t b_slot = b_desc0 + ((s * R::kBBytes) >> 4);
                     const int nc = nkb - kg * KC;   // chunks in this group: KC, except at a tile's end
                     if constexpr (FP8) {
@@ -274,7 +310,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                             d = tmem_base + (acc_iter % kNumAcc) * BN;
                             ++acc_iter;
                         }
-                        const uint64_t a_desc = a_slot + ((c * a_chunk_pitch) >> 4);
+                        const uint64_t a_desc = a_slot + ((c * a_cp) >> 4);
                         const uint64_t b_desc = b_slot + ((c * R::kBChunkBytes) >> 4);
 #pragma unroll
                         for (int q = 0; q < kMmaPerChunk; ++q) {

@@ -197,18 +197,20 @@ __device__ __forceinline__ void tc_fence_after_sync()
 }
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA with the 128-byte
-// swizzle: rows of 128 bytes, 8-row core groups 1024 bytes apart.  Fields (sm_100 format):
+// swizzle: rows of 128 bytes, 8-row core groups sbo_bytes apart (1024 when the groups are
+// contiguous; KC * 1024 when each 8-row group holds all KC chunks of a stage, as the 8-row TMA
+// boxes of short grouped segments write them).  Fields (sm_100 format):
 // start address >> 4 in bits [0,14), leading byte offset >> 4 in [16,30) (unused by swizzled
 // K-major layouts, set to 1), stride byte offset >> 4 in [32,46), descriptor version 1 in
 // [46,48), base offset 0 in [49,52), layout type 2 (128-byte swizzle) in [61,64).
 // The tile base must be 1024-byte aligned; stepping K inside the 128-byte row is done by
 // adding (bytes >> 4) to the start address.
-__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr)
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr, uint32_t sbo_bytes = 1024u)
 {
     uint64_t d = 0;
     d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
     d |= static_cast<uint64_t>(1u) << 16;
-    d |= static_cast<uint64_t>(1024u >> 4) << 32;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
     d |= static_cast<uint64_t>(1u) << 46;
     d |= static_cast<uint64_t>(2u) << 61;
     return d;
