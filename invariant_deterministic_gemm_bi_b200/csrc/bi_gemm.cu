@@ -89,8 +89,6 @@ const KernelEntry kKernels[] = {
     BI_PAIR(128, 1, false, false),      BI_PAIR(128, 2, false, false),
     BI_PAIR(256, 1, false, false),      BI_PAIR(256, 2, false, false),
     BI_PAIR(128, 1, true, false),       BI_PAIR(128, 2, true, false),
-    BI_PAIR(128, 1, false, true),       BI_PAIR(128, 2, false, true),
-    BI_PAIR(256, 1, false, true),       BI_PAIR(256, 2, false, true),
     // fixed-split-K research variant (bi_gemm_plan_splitk), not the product path
     BI_ENTRY_KSPLIT(128, 32, 1),        BI_ENTRY_KSPLIT(128, 32, 4),
     BI_ENTRY_KSPLIT(128, 64, 1),        BI_ENTRY_KSPLIT(128, 64, 2),
