@@ -2,7 +2,8 @@
 
 C[M,N] = A[M,K] . B[N,K]^T with fp32 accumulation and bf16 output, computed by hand-written
 tcgen05/TMA kernels behind the C ABI in ``include/bi_gemm.h``; the MoE routing, dispatch, gather
-and combine steps around the grouped GEMM are in ``include/bi_moe.h``.  Every output row is
+and combine steps around the grouped GEMM are in ``include/bi_moe.h``, and the dual-kernel
+decode attention in ``include/bi_attention.h``.  Every output row is
 bit-identical whatever the batch size, the row's position and the other rows in the batch.
 
 ``binding`` holds the ctypes wrapper (same names as the C ABI); ``inputs`` the seeded synthetic
@@ -15,6 +16,8 @@ from .binding import (  # noqa: F401
     BI_PLAN_RESIDENT_WEIGHTS,
     BiGemmError,
     Plan,
+    bi_decode_attention,
+    bi_decode_attention_workspace_bytes,
     bi_gemm_abi_version,
     bi_gemm_debug_set_flags,
     bi_gemm_plan,

@@ -1,4 +1,5 @@
-"""Thin ctypes binding of libbigemm (include/bi_gemm.h, include/bi_moe.h), same names as the C ABI.
+"""Thin ctypes binding of libbigemm (include/bi_gemm.h, bi_moe.h, bi_attention.h), same names as
+the C ABI.
 
 Argument marshalling only: every function takes torch tensors (device memory owned by torch)
 or raw integers, passes their pointers, strides and the current CUDA stream to the C entry
@@ -35,6 +36,7 @@ EXPORTED = [
     "bi_gemm_run_host_noalloc", "bi_gemm_plan_set_flags",
     "bi_gemm_plan_splitk", "bi_gemm_splitk_workspace_bytes", "bi_gemm_run_splitk",
     "bi_moe_route_topk", "bi_moe_dispatch", "bi_moe_gather_rows", "bi_moe_combine",
+    "bi_decode_attention", "bi_decode_attention_workspace_bytes",
 ]
 
 
@@ -113,6 +115,11 @@ def load_library(path: str = LIB_PATH):
     lib.bi_moe_gather_rows.argtypes = [vp, i64, i64, vp, i64, vp, i64, vp]
     lib.bi_moe_combine.restype = i32
     lib.bi_moe_combine.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, i64, vp]
+    lib.bi_decode_attention_workspace_bytes.restype = ctypes.c_size_t
+    lib.bi_decode_attention_workspace_bytes.argtypes = [i64, i32, i32, i32]
+    lib.bi_decode_attention.restype = i32
+    lib.bi_decode_attention.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i64, ctypes.c_float, i32,
+                                        vp, ctypes.c_size_t, vp, vp]
     if path == LIB_PATH:
         _LIB = lib
     return lib
@@ -322,3 +329,24 @@ def bi_moe_combine(C_perm, row_of_slot, weights, Y, stream=None):
                                          _ptr(weights), T, k, _ptr(Y), Y.stride(0),
                                          _stream_handle(stream)), "bi_moe_combine")
     return Y
+
+
+# ---------------------------------------------------------------------------------------------
+# Dual-kernel decode attention (include/bi_attention.h)
+# ---------------------------------------------------------------------------------------------
+
+def bi_decode_attention_workspace_bytes(B: int, Hq: int, D: int, splits: int) -> int:
+    return int(load_library().bi_decode_attention_workspace_bytes(B, Hq, D, splits))
+
+
+def bi_decode_attention(Q, K, V, lengths, O, scale: float, splits: int = 1, workspace=None,
+                        stream=None):
+    """Q [B, Hq, D], K/V [B, Lmax, Hkv, D] bf16, lengths int32 [B] (device) -> O [B, Hq, D].
+    splits 1 (no split), 2 or 4 (split-KV), or 0 (automatic); every choice gives the same bits."""
+    B, Hq, D = Q.shape
+    _, Lmax, Hkv, _ = K.shape
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().bi_decode_attention(_ptr(Q), _ptr(K), _ptr(V), _ptr(lengths), B, Hq, Hkv, D,
+                                              Lmax, scale, splits, _ptr(workspace), nbytes, _ptr(O),
+                                              _stream_handle(stream)), "bi_decode_attention")
+    return O

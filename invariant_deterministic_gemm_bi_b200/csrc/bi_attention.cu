@@ -1,0 +1,372 @@
+// bi_attention.cu -- dual-kernel decode attention (include/bi_attention.h).
+//
+// One CTA serves one (sequence, key/value head) pair -- or, split-KV, a part of its chunks --
+// with one warp per query head of the group (grouped-query attention).  A sequence's keys are cut
+// into kChunks = 4 chunks by its own length, and every chunk is reduced by chunk_attention():
+// blocks of 32 keys in ascending order, lane j scoring key j (q . k_j summed over d ascending),
+// an online softmax whose block max and block sum are fixed butterflies, and the value sum
+// o = o * corr + sum_j p_j v_j with j ascending.  merge() combines two chunk results, always as
+// ((c0 + c1) + (c2 + c3)).  The no-split kernel and the split-KV kernels run exactly this
+// arithmetic, so their outputs are bitwise equal.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "bi_attention.h"
+
+namespace {
+
+constexpr int kD = 128;             // head dimension
+constexpr int kChunks = 4;          // chunks per sequence (fixed: the merge tree has 4 leaves)
+constexpr int kBlockKeys = 32;      // keys per block = lanes of a warp
+constexpr int kMaxGroup = 8;        // query heads per key/value head
+constexpr int kRowStride = kD * 2 + 16;   // bytes per key row in shared memory (bank spread)
+constexpr unsigned kFull = 0xffffffffu;
+
+// The running state of one query head: max, sum of exp, and this lane's 4 output dimensions
+// (unnormalised).
+struct Partial {
+    float m, l;
+    float o[4];
+};
+
+__device__ __forceinline__ Partial empty_partial()
+{
+    Partial p;
+    p.m = -INFINITY;
+    p.l = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        p.o[i] = 0.0f;
+    return p;
+}
+
+// a + b of two partials of the same query head (same lane's dimensions).
+__device__ __forceinline__ Partial merge(const Partial &a, const Partial &b)
+{
+    const float m = fmaxf(a.m, b.m);
+    if (m == -INFINITY)
+        return a;   // both empty
+    const float fa = expf(a.m - m);
+    const float fb = expf(b.m - m);
+    Partial r;
+    r.m = m;
+    r.l = fmaf(b.l, fb, a.l * fa);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        r.o[i] = fmaf(b.o[i], fb, a.o[i] * fa);
+    return r;
+}
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid)
+{
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    const int n = valid ? 16 : 0;   // 0: fill the 16 bytes with zeros
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+struct AttnArgs {
+    const __nv_bfloat16 *q, *k, *v;
+    const int32_t *lengths;
+    int64_t lmax;
+    int hq, hkv, group;
+    float scale;
+};
+
+// Keys [k0, k1) of sequence b, key/value head kvh, into this warp's partial.  Every thread of the
+// CTA calls it with the same arguments (it loads shared K/V blocks and synchronises).
+__device__ Partial chunk_attention(const AttnArgs &a, int64_t b, int kvh, int k0, int k1,
+                                   const float *q_s, uint8_t *kv_s)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nthreads = blockDim.x;
+    Partial st = empty_partial();
+    const int nblk = (k1 - k0 + kBlockKeys - 1) / kBlockKeys;
+    const int64_t row_pitch = static_cast<int64_t>(a.hkv) * kD;   // elements between keys
+    const __nv_bfloat16 *kbase = a.k + (b * a.lmax * a.hkv + kvh) * kD;
+    const __nv_bfloat16 *vbase = a.v + (b * a.lmax * a.hkv + kvh) * kD;
+    auto load_block = [&](int blk, int buf) {
+        uint8_t *ks = kv_s + buf * 2 * kBlockKeys * kRowStride;
+        uint8_t *vs = ks + kBlockKeys * kRowStride;
+        // 32 keys x 16 pieces of 16 bytes, for K and for V
+        for (int i = threadIdx.x; i < kBlockKeys * 16; i += nthreads) {
+            const int j = i >> 4, piece = i & 15;
+            const int key = k0 + blk * kBlockKeys + j;
+            const bool ok = key < k1;
+            const int64_t off = (ok ? key : k0) * row_pitch + piece * 8;
+            cp_async16(ks + j * kRowStride + piece * 16, kbase + off, ok);
+            cp_async16(vs + j * kRowStride + piece * 16, vbase + off, ok);
+        }
+    };
+    if (nblk > 0)
+        load_block(0, 0);
+    cp_async_commit();
+    for (int blk = 0; blk < nblk; ++blk) {
+        if (blk + 1 < nblk)
+            load_block(blk + 1, (blk + 1) & 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        const uint8_t *ks = kv_s + (blk & 1) * 2 * kBlockKeys * kRowStride;
+        const uint8_t *vs = ks + kBlockKeys * kRowStride;
+        if (warp < a.group) {
+            // lane j: the score of key j of the block, d ascending
+            const int key = k0 + blk * kBlockKeys + lane;
+            const float *qh = q_s + warp * kD;
+            const uint4 *krow = reinterpret_cast<const uint4 *>(ks + lane * kRowStride);
+            float s = 0.0f;
+#pragma unroll 4
+            for (int piece = 0; piece < 16; ++piece) {
+                const uint4 raw = krow[piece];
+                const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const float2 f = __bfloat1622float2(h2[t]);
+                    s = fmaf(qh[piece * 8 + 2 * t], f.x, s);
+                    s = fmaf(qh[piece * 8 + 2 * t + 1], f.y, s);
+                }
+            }
+            s = key < k1 ? s * a.scale : -INFINITY;
+            float mb = s;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                mb = fmaxf(mb, __shfl_xor_sync(kFull, mb, off));
+            const float m_new = fmaxf(st.m, mb);
+            const float corr = expf(st.m - m_new);   // 0 for the first block (st.m = -inf)
+            const float p = expf(s - m_new);         // 0 for masked keys
+            float ps = p;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+                ps = ps + __shfl_xor_sync(kFull, ps, off);
+            st.l = fmaf(st.l, corr, ps);
+            float acc[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                acc[i] = st.o[i] * corr;
+            for (int j = 0; j < kBlockKeys; ++j) {
+                const float pj = __shfl_sync(kFull, p, j);
+                const __nv_bfloat162 *vrow =
+                    reinterpret_cast<const __nv_bfloat162 *>(vs + j * kRowStride) + lane * 2;
+                const float2 v01 = __bfloat1622float2(vrow[0]);
+                const float2 v23 = __bfloat1622float2(vrow[1]);
+                acc[0] = fmaf(pj, v01.x, acc[0]);
+                acc[1] = fmaf(pj, v01.y, acc[1]);
+                acc[2] = fmaf(pj, v23.x, acc[2]);
+                acc[3] = fmaf(pj, v23.y, acc[3]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                st.o[i] = acc[i];
+            st.m = m_new;
+        }
+        __syncthreads();   // the buffer is refilled two blocks later
+    }
+    return st;
+}
+
+__device__ __forceinline__ int chunk_begin(int c, int L) { return static_cast<int>((static_cast<int64_t>(c) * L) / kChunks); }
+
+// Load the group's query heads into shared memory as fp32.
+__device__ void load_q(const AttnArgs &a, int64_t b, int kvh, float *q_s)
+{
+    for (int i = threadIdx.x; i < a.group * kD; i += blockDim.x) {
+        const int h = kvh * a.group + i / kD;
+        q_s[i] = __bfloat162float(a.q[(b * a.hq + h) * kD + (i % kD)]);
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ int valid_length(const AttnArgs &a, int64_t b)
+{
+    const int L = a.lengths[b];
+    return (L >= 1 && L <= a.lmax) ? L : -1;
+}
+
+__device__ __forceinline__ void store_output(const AttnArgs &a, int64_t b, int h, const Partial &p,
+                                             bool valid, __nv_bfloat16 *out)
+{
+    const int lane = threadIdx.x & 31;
+    __nv_bfloat16 *o = out + (b * a.hq + h) * kD + lane * 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        o[i] = __float2bfloat16_rn(valid ? p.o[i] / p.l : NAN);
+}
+
+// No split: one CTA per (sequence, key/value head) walks the 4 chunks and merges them.
+__global__ void __launch_bounds__(256) attn_nosplit_kernel(AttnArgs a, __nv_bfloat16 *out)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    float *q_s = reinterpret_cast<float *>(smem);
+    uint8_t *kv_s = smem + kMaxGroup * kD * 4;
+    const int64_t b = blockIdx.x / a.hkv;
+    const int kvh = blockIdx.x % a.hkv;
+    const int L = valid_length(a, b);
+    load_q(a, b, kvh, q_s);
+    Partial c[kChunks];
+#pragma unroll
+    for (int ci = 0; ci < kChunks; ++ci)
+        c[ci] = L > 0 ? chunk_attention(a, b, kvh, chunk_begin(ci, L), chunk_begin(ci + 1, L), q_s, kv_s)
+                      : empty_partial();
+    const int warp = threadIdx.x >> 5;
+    if (warp < a.group)
+        store_output(a, b, kvh * a.group + warp, merge(merge(c[0], c[1]), merge(c[2], c[3])), L > 0, out);
+}
+
+// Split-KV: CTA `part` of `splits` for (sequence, key/value head) reduces chunks
+// [part * 4 / splits, (part + 1) * 4 / splits) (merging them pairwise when it has two) and writes
+// its partial to ws[((b * hq + h) * 4 + part) * (kD + 2)].
+__global__ void __launch_bounds__(256) attn_split_kernel(AttnArgs a, int splits, float *ws)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    float *q_s = reinterpret_cast<float *>(smem);
+    uint8_t *kv_s = smem + kMaxGroup * kD * 4;
+    const int part = blockIdx.x % splits;
+    const int64_t pair = blockIdx.x / splits;
+    const int64_t b = pair / a.hkv;
+    const int kvh = static_cast<int>(pair % a.hkv);
+    const int L = valid_length(a, b);
+    load_q(a, b, kvh, q_s);
+    const int per = kChunks / splits;
+    Partial r = empty_partial();
+    if (L > 0) {
+        if (per == 1) {
+            r = chunk_attention(a, b, kvh, chunk_begin(part, L), chunk_begin(part + 1, L), q_s, kv_s);
+        } else {
+            const Partial c0 = chunk_attention(a, b, kvh, chunk_begin(2 * part, L), chunk_begin(2 * part + 1, L), q_s, kv_s);
+            const Partial c1 = chunk_attention(a, b, kvh, chunk_begin(2 * part + 1, L), chunk_begin(2 * part + 2, L), q_s, kv_s);
+            r = merge(c0, c1);
+        }
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp < a.group) {
+        const int h = kvh * a.group + warp;
+        float *w = ws + ((b * a.hq + h) * kChunks + part) * (kD + 2);
+        if (lane == 0) {
+            w[0] = r.m;
+            w[1] = r.l;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            w[2 + lane * 4 + i] = r.o[i];
+    }
+}
+
+// Merge of the split partials: one warp per (sequence, query head).
+__global__ void __launch_bounds__(256) attn_merge_kernel(AttnArgs a, int splits, const float *ws,
+                                                         __nv_bfloat16 *out, int64_t B)
+{
+    const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (wid >= B * a.hq)
+        return;
+    const int64_t b = wid / a.hq;
+    const int h = static_cast<int>(wid % a.hq);
+    Partial p[kChunks];
+    for (int part = 0; part < splits; ++part) {
+        const float *w = ws + (wid * kChunks + part) * (kD + 2);
+        p[part].m = w[0];
+        p[part].l = w[1];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            p[part].o[i] = w[2 + lane * 4 + i];
+    }
+    const Partial r = splits == 4 ? merge(merge(p[0], p[1]), merge(p[2], p[3])) : merge(p[0], p[1]);
+    store_output(a, b, h, r, valid_length(a, b) > 0, out);
+}
+
+bi_status_t attn_device(int *num_sms)
+{
+    int count = 0;
+    if (cudaGetDeviceCount(&count) != cudaSuccess || count <= 0) {
+        cudaGetLastError();
+        return BI_ERR_NO_DEVICE;
+    }
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return BI_ERR_CUDA;
+    return major == 10 ? BI_OK : BI_ERR_NO_DEVICE;
+}
+
+constexpr int kSmemBytes = kMaxGroup * kD * 4 + 2 * 2 * kBlockKeys * kRowStride;
+
+} // namespace
+
+extern "C" {
+
+size_t bi_decode_attention_workspace_bytes(int64_t B, int Hq, int D, int splits)
+{
+    if (B <= 0 || Hq <= 0 || D <= 0 || splits <= 1)
+        return 0;
+    return static_cast<size_t>(B) * static_cast<size_t>(Hq) * kChunks * static_cast<size_t>(D + 2) * 4u;
+}
+
+bi_status_t bi_decode_attention(const void *Q, const void *K, const void *V,
+                                const int32_t *lengths, int64_t B, int Hq, int Hkv, int D,
+                                int64_t Lmax, float scale, int splits, float *workspace,
+                                size_t workspace_bytes, void *O, cudaStream_t stream)
+{
+    if (B < 0 || Hq < 1 || Hkv < 1 || Lmax < 1 || (splits != 0 && splits != 1 && splits != 2 && splits != 4))
+        return BI_ERR_INVALID_ARG;
+    if (D != kD || Hq % Hkv != 0 || Hq / Hkv > kMaxGroup)
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0)
+        return BI_OK;
+    if (!Q || !K || !V || !lengths || !O)
+        return BI_ERR_INVALID_ARG;
+    auto al16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (!al16(Q) || !al16(K) || !al16(V) || !al16(O) || (reinterpret_cast<uintptr_t>(lengths) & 3u))
+        return BI_ERR_ALIGNMENT;
+    if (Lmax > INT32_MAX / 4 || B * Hkv > INT32_MAX / 4)
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    int sms = 0;
+    bi_status_t st = attn_device(&sms);
+    if (st != BI_OK)
+        return st;
+    if (splits == 0) {   // automatic: the fewest splits that give every SM a CTA (no bit changes)
+        splits = 4;
+        for (int s = 1; s <= 2; s *= 2)
+            if (B * Hkv * s >= sms) {
+                splits = s;
+                break;
+            }
+    }
+    if (splits > 1) {
+        if (!workspace || workspace_bytes < bi_decode_attention_workspace_bytes(B, Hq, D, splits))
+            return BI_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(workspace) & 15u)
+            return BI_ERR_ALIGNMENT;
+    }
+    AttnArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(Q);
+    a.k = static_cast<const __nv_bfloat16 *>(K);
+    a.v = static_cast<const __nv_bfloat16 *>(V);
+    a.lengths = lengths;
+    a.lmax = Lmax;
+    a.hq = Hq;
+    a.hkv = Hkv;
+    a.group = Hq / Hkv;
+    a.scale = scale;
+    const int threads = 32 * a.group;
+    const int64_t pairs = B * Hkv;
+    if (splits == 1) {
+        attn_nosplit_kernel<<<static_cast<unsigned>(pairs), threads, kSmemBytes, stream>>>(
+            a, static_cast<__nv_bfloat16 *>(O));
+        return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+    }
+    attn_split_kernel<<<static_cast<unsigned>(pairs * splits), threads, kSmemBytes, stream>>>(a, splits, workspace);
+    if (cudaGetLastError() != cudaSuccess)
+        return BI_ERR_CUDA;
+    const int64_t warps = B * Hq;
+    attn_merge_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, stream>>>(
+        a, splits, workspace, static_cast<__nv_bfloat16 *>(O), B);
+    return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+} // extern "C"

@@ -1,5 +1,5 @@
 """CPU oracle for the batch-invariant GEMM -- test infrastructure only (see ``oracle.py``; the MoE
-steps around the grouped GEMM are in ``moe.py``)."""
+steps around the grouped GEMM are in ``moe.py``, the decode attention in ``attention.py``)."""
 from .oracle import (  # noqa: F401
     bf16_to_f64,
     OracleLib,
@@ -14,4 +14,4 @@ from .oracle import (  # noqa: F401
     gemm_fp8_rows,
     grouped_gemm_bf16,
 )
-from . import moe  # noqa: F401,E402
+from . import attention, moe  # noqa: F401,E402
