@@ -631,6 +631,31 @@ def measure_extras(bg, inputs, dev, stream, peaks):
             res[f"moe_layer_T{T}_{name}"] = {"us": t * 1e6, "GB/s": b / t / 1e9,
                                              "hbm_frac": b / t / 1e9 / hbm}
         del A, Cp, Y, toks
+    # Dual-kernel decode attention: Hq = 32, Hkv = 8, D = 128, bf16 KV cache, every sequence at
+    # length L; no split vs split-KV (bitwise equal outputs).  Bytes: K and V once, Q and O.
+    import math
+    Hq, Hkv, D = 32, 8, 128
+    for (Bsz, L) in ((16, 4096), (64, 4096), (16, 32768)):
+        Q = inputs.bf16_gaussian((Bsz, Hq, D), seed=8001, device=dev)
+        Kc = inputs.bf16_gaussian((Bsz, L, Hkv, D), seed=8002, device=dev)
+        Vc = inputs.bf16_gaussian((Bsz, L, Hkv, D), seed=8003, device=dev)
+        lens = torch.full((Bsz,), L, dtype=torch.int32, device=dev)
+        O = torch.empty((Bsz, Hq, D), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(bg.bi_decode_attention_workspace_bytes(Bsz, Hq, D, 4) // 4,
+                         dtype=torch.float32, device=dev)
+        b = 2 * Bsz * L * Hkv * D * 2 + 2 * Bsz * Hq * D * 2
+        outs = {}
+        for splits in (1, 2, 4):
+            fn = lambda splits=splits: bg.bi_decode_attention(Q, Kc, Vc, lens, O, 1.0 / math.sqrt(D),
+                                                              splits=splits, workspace=ws, stream=stream)
+            t = graph_time_per_launch([fn] * 4, stream, reps=4)
+            torch.cuda.synchronize()
+            outs[splits] = O.clone()
+            res[f"attention_B{Bsz}_L{L}_splits{splits}"] = {"us": t * 1e6, "GB/s": b / t / 1e9,
+                                                            "hbm_frac": b / t / 1e9 / hbm}
+        res[f"attention_B{Bsz}_L{L}_splits{splits}"]["bitwise_equal_to_no_split"] = all(
+            torch.equal(outs[1].view(torch.int16), o.view(torch.int16)) for o in outs.values())
+        del Q, Kc, Vc, O, ws
     # Fixed-split-K research variant on the decode shape (not the product path): what dropping
     # split-K costs at small M.  Bytes are the algorithmic ones (workspace traffic not counted).
     N, K = N_DEC, K_DEC

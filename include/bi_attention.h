@@ -13,7 +13,8 @@
  *   O[b][h] = sum_j softmax(s)_j * v_j, rounded once to bf16.
  * The reduction order is fixed by L_b alone: the keys are cut into 4 chunks
  * [floor(c L_b / 4), floor((c+1) L_b / 4)), each chunk is reduced by the same code (blocks of 32
- * keys in ascending order, an online softmax with fixed-order warp reductions), and the 4 chunk
+ * keys in ascending order, scores in a fixed summation order, an online softmax with fixed-order
+ * warp reductions), and the 4 chunk
  * results are merged as ((c0 + c1) + (c2 + c3)).  `splits` only decides how many CTAs share a
  * sequence's chunks -- 1 (no split: one CTA walks all 4 chunks), 2 or 4 (split-KV: 2 or 4 CTAs,
  * then a merge kernel) -- so every value of `splits` gives the same bits, and a sequence's output
