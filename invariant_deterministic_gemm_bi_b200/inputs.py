@@ -12,6 +12,11 @@ Recipes (all seeded; a generator is ``torch.Generator(device)`` seeded with the 
 * e4m3 integer:    x uniform in {-4, ..., 4}, exact in e4m3.
 * fp32 scales:     s = 2^u, u ~ U(-4, 4) (log-uniform in [2^-4, 2^4]); or s = 2^j with integer
                    j uniform in [-4, 4] for the exactly representable variant.
+* e2m1 weights:    every 4-bit code uniform in 0..15 (the values +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}
+                   equally often), packed two per byte, the even K index in the low four bits.
+* e2m1 channel scales: 2^-j with integer j uniform in [1, 12]; zero points z = fp16(x * s),
+                   x ~ N(0, 1), rounded to fp16 (RNE) and held in fp32; or, for the exactly
+                   representable variant, z = i * 2^-6 with integer i uniform in [-64, 64].
 * MoE routing:     logits [T, E] ~ N(0, 1); each token takes the 8 largest logits (softmax is
                    monotone, so this is top-8 by softmax); ties go to the lower expert index.
                    The (token, slot) pairs are stably sorted by expert, so inside an expert's
@@ -78,6 +83,36 @@ def scales_pow2(shape, seed: int, lo: int = -4, hi: int = 4, device="cpu") -> to
     g = generator(seed, device)
     j = torch.randint(lo, hi + 1, tuple(shape), generator=g, device=device, dtype=torch.int32)
     return torch.exp2(j.to(torch.float32))
+
+
+def e2m1_packed_uniform(rows: int, K: int, seed: int, device="cpu") -> torch.Tensor:
+    """uint8 [rows, K/2]: uniformly drawn e2m1 codes, value k in the low four bits of byte k//2
+    when k is even and in the high four bits when k is odd."""
+    assert K % 2 == 0
+    g = generator(seed, device)
+    codes = torch.randint(0, 16, (rows, K), generator=g, device=device, dtype=torch.int32)
+    return (codes[:, 0::2] | (codes[:, 1::2] << 4)).to(torch.uint8)
+
+
+def channel_scales_pow2(n: int, seed: int, lo: int = 1, hi: int = 12, device="cpu") -> torch.Tensor:
+    """fp32 [n]: 2^-j with integer j uniform in [lo, hi]."""
+    g = generator(seed, device)
+    j = torch.randint(lo, hi + 1, (n,), generator=g, device=device, dtype=torch.int32)
+    return torch.exp2(-j.to(torch.float32))
+
+
+def channel_zeros_fp16(scales: torch.Tensor, seed: int) -> torch.Tensor:
+    """fp32 zero points z[n] = fp16(x[n] * scales[n]), x ~ N(0, 1) (values fp16 holds exactly)."""
+    g = generator(seed, scales.device)
+    x = torch.randn(scales.shape, generator=g, device=scales.device, dtype=torch.float32)
+    return (x * scales).to(torch.float16).to(torch.float32)
+
+
+def channel_zeros_grid(n: int, seed: int, device="cpu") -> torch.Tensor:
+    """fp32 zero points i * 2^-6 with integer i uniform in [-64, 64]."""
+    g = generator(seed, device)
+    i = torch.randint(-64, 65, (n,), generator=g, device=device, dtype=torch.int32)
+    return i.to(torch.float32) * 2.0 ** -6
 
 
 def bits_of(t: torch.Tensor) -> torch.Tensor:
@@ -169,6 +204,7 @@ WORKLOAD_BASE_SEED = {
     "prefill": 3000,
     "fp8": 4000,
     "moe": 5000,
+    "w4a8": 6000,
 }
 
 

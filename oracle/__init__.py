@@ -6,12 +6,15 @@ from .oracle import (  # noqa: F401
     build,
     compile_copy,
     default_threads,
+    e2m1_to_f64,
     e4m3_to_f64,
     f64_to_bf16,
     gemm_bf16,
     gemm_bf16_rows,
     gemm_fp8_blockscaled,
     gemm_fp8_rows,
+    gemm_w4a8,
+    gemm_w4a8_rows,
     grouped_gemm_bf16,
 )
 from . import attention, moe  # noqa: F401,E402

@@ -16,6 +16,12 @@
  *     scale of its block: A per 1x128 K-block, B per 128x128 block), then the dense GEMM above.
  *     The pages only say that the dequantisation is fused into the GEMM (lshu.cn article,
  *     section 3.2); the block shapes are those of the FP8 workload this library targets.
+ *   e2m1 weights x e4m3 activations (W4A8): the weights are dequantised as
+ *     W[n][k] = e2m1(Q[n][k]) * scale[n] + zero[n], the quantisation of the lshu.cn article,
+ *     section 4.3 (one scale 2^-j, j in [1, 12], and one fp16-exact zero point per output
+ *     channel), the activations as in the FP8 GEMM (per 1x128 K-block scales); then the dense
+ *     GEMM above.  Every dequantised weight is exact in fp64 (a 2-bit significand times a power
+ *     of two plus an 11-bit one, spanning at most 2^15 .. 2^-24).
  *   Grouped (MoE) GEMM: for expert e and every row r in [offsets[e], offsets[e+1]),
  *     C[r][n] = sum_k A[r][k] * B_e[n][k].  MoE is listed among the V4 components in
  *     "DeepSeek不惜代价保住它！V4关键特性被挖出来了" (QbitAI), section "什么是batch invariance".
@@ -29,6 +35,9 @@
  *   bf16  = 1 sign bit, 8 exponent bits (bias 127), 7 fraction bits (upper half of binary32).
  *   e4m3  = 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits; exponent field 0 is
  *           subnormal (value = fraction * 2^-9); S.1111.111 is NaN; no infinities; max 448.
+ *   e2m1  = 1 sign bit, 2 exponent bits (bias 1), 1 fraction bit; exponent field 0 is
+ *           subnormal (value = fraction * 2^-1); no infinities or NaN; max 6.  Packed two per
+ *           byte, value k of a row in byte k/2, the even k in the low four bits.
  *
  * Threads: output rows are split across POSIX threads; every output element is still one
  * sequential fp64 loop, so the oracle is itself deterministic and batch-invariant.
@@ -76,6 +85,20 @@ double oracle_e4m3_to_f64(uint8_t bits)
     } else {
         v = ldexp((double)(8 + frac), expo - 7 - 3);   /* 1.frac * 2^(e-7) */
     }
+    return sign ? -v : v;
+}
+
+/* e2m1 4-bit code (the low four bits of `code`) -> exact fp64 value. */
+double oracle_e2m1_to_f64(uint8_t code)
+{
+    int sign = (code >> 3) & 1;
+    int expo = (code >> 1) & 0x3;
+    int frac = code & 0x1;
+    double v;
+    if (expo == 0)
+        v = ldexp((double)frac, -1);                   /* 0.frac * 2^0 = frac * 2^-1 */
+    else
+        v = ldexp((double)(2 + frac), expo - 1 - 1);   /* 1.frac * 2^(e-1) */
     return sign ? -v : v;
 }
 
@@ -242,6 +265,41 @@ int oracle_gemm_fp8_blockscaled(int64_t M, int64_t N, int64_t K, const uint8_t *
     for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k)
             b[n * K + k] = oracle_e4m3_to_f64(QB[n * K + k]) * (double)SB[(n / 128) * kb + k / 128];
+    int rc = run_rows(a, b, NULL, M, N, K, cref, cbits, threads);
+    free(a);
+    free(b);
+    return rc;
+}
+
+/* e2m1 weights x e4m3 activations:
+ *   a_deq[m][k] = e4m3(QA[m][k]) * SA[m][k/128]           SA is [M][ceil(K/128)] row-major
+ *   w_deq[n][k] = e2m1(QW[n][k]) * WS[n] + WZ[n]          QW packed [N][K/2] bytes; WZ may be NULL
+ *   cref[m][n]  = sum_k a_deq[m][k] * w_deq[n][k]
+ * K must be even.  Returns 0, or -1 on allocation failure. */
+int oracle_gemm_w4a8(int64_t M, int64_t N, int64_t K, const uint8_t *QA, const float *SA,
+                     const uint8_t *QW, const float *WS, const float *WZ, double *cref,
+                     uint16_t *cbits, int threads)
+{
+    int64_t kb = (K + 127) / 128;
+    double *a = (double *)malloc(sizeof(double) * (size_t)(M * K > 0 ? M * K : 1));
+    double *b = (double *)malloc(sizeof(double) * (size_t)(N * K > 0 ? N * K : 1));
+    if (!a || !b) {
+        free(a);
+        free(b);
+        return -1;
+    }
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k)
+            a[m * K + k] = oracle_e4m3_to_f64(QA[m * K + k]) * (double)SA[m * kb + k / 128];
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t byte = QW[n * (K / 2) + k / 2];
+            uint8_t code = (k % 2 == 0) ? (uint8_t)(byte & 0xF) : (uint8_t)(byte >> 4);
+            double w = oracle_e2m1_to_f64(code) * (double)WS[n];
+            if (WZ)
+                w += (double)WZ[n];
+            b[n * K + k] = w;
+        }
     int rc = run_rows(a, b, NULL, M, N, K, cref, cbits, threads);
     free(a);
     free(b);

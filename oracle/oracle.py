@@ -49,6 +49,10 @@ class OracleLib:
         lib.oracle_gemm_bf16.argtypes = [i64, i64, i64, vp, vp, vp, vp, i32]
         lib.oracle_gemm_fp8_blockscaled.restype = i32
         lib.oracle_gemm_fp8_blockscaled.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, i32]
+        lib.oracle_e2m1_to_f64.restype = ctypes.c_double
+        lib.oracle_e2m1_to_f64.argtypes = [ctypes.c_uint8]
+        lib.oracle_gemm_w4a8.restype = i32
+        lib.oracle_gemm_w4a8.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, i32]
         lib.oracle_grouped_gemm_bf16.restype = i32
         lib.oracle_grouped_gemm_bf16.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp, vp, i32]
         self.c = lib
@@ -112,6 +116,17 @@ def e4m3_to_f64(bits, lib=None) -> np.ndarray:
     return out
 
 
+def e2m1_to_f64(codes, lib=None) -> np.ndarray:
+    """e2m1 4-bit codes (one per array element, values 0..15) -> exact fp64 values."""
+    lib = lib or _lib()
+    b = np.asarray(codes, dtype=np.uint8)
+    out = np.empty(b.shape, dtype=np.float64)
+    flat, oflat = b.reshape(-1), out.reshape(-1)
+    for i in range(flat.size):
+        oflat[i] = lib.oracle_e2m1_to_f64(int(flat[i]))
+    return out
+
+
 def f64_to_bf16(x, lib=None) -> np.ndarray:
     """fp64 values -> bf16 bit patterns, round to nearest even (oracle codec)."""
     lib = lib or _lib()
@@ -167,6 +182,39 @@ def gemm_fp8_blockscaled(QA_bits, QB_bits, SA, SB, threads: int | None = None, l
     if rc != 0:
         raise MemoryError("oracle_gemm_fp8_blockscaled failed")
     return cref, cbits
+
+
+def gemm_w4a8(QA_bits, SA, QW_packed, w_scale, w_zero=None, threads: int | None = None, lib=None):
+    """e2m1 weights x e4m3 activations, C = deq(A) . deq(W)^T.
+
+    QA [M,K] e4m3 bit patterns with SA fp32 [M, ceil(K/128)]; QW_packed uint8 [N, K/2] (value k
+    of a row in byte k//2, the even k in the low four bits); w_scale fp32 [N]; w_zero fp32 [N] or
+    None.  Returns (cref fp64 [M,N], c bf16 bits [M,N]).
+    """
+    QA = _c(QA_bits, np.uint8)
+    QW = _c(QW_packed, np.uint8)
+    M, K = QA.shape
+    N, K2 = QW.shape
+    assert K % 2 == 0 and K2 == K // 2, (QA.shape, QW.shape)
+    kb = (K + 127) // 128
+    SA = _c(SA, np.float32)
+    assert SA.shape == (M, kb), SA.shape
+    WS = _c(w_scale, np.float32).reshape(N)
+    WZ = None if w_zero is None else _c(w_zero, np.float32).reshape(N)
+    cref = np.empty((M, N), dtype=np.float64)
+    cbits = np.empty((M, N), dtype=np.uint16)
+    rc = (lib or _lib()).oracle_gemm_w4a8(M, N, K, _ptr(QA), _ptr(SA), _ptr(QW), _ptr(WS),
+                                          None if WZ is None else _ptr(WZ), _ptr(cref), _ptr(cbits),
+                                          threads or default_threads())
+    if rc != 0:
+        raise MemoryError("oracle_gemm_w4a8 failed")
+    return cref, cbits
+
+
+def gemm_w4a8_rows(QA_bits, SA, QW_packed, w_scale, w_zero, rows, threads: int | None = None):
+    rows = np.asarray(rows, dtype=np.int64)
+    return gemm_w4a8(_c(QA_bits, np.uint8)[rows], _c(SA, np.float32)[rows], QW_packed, w_scale,
+                     w_zero, threads)
 
 
 def grouped_gemm_bf16(A_bits, B_bits, offsets, threads: int | None = None, lib=None):

@@ -82,3 +82,50 @@ def fp8_cases():
                     out += [float(v)] * int(cnt)
                 case["c"] = np.array(out, dtype=np.float64).reshape(M, N)
         yield case
+
+
+def e2m1_cases():
+    """Yield (code, value as Fraction, negative_zero flag, reason) from e2m1_codes.txt."""
+    for line in _lines("e2m1_codes.txt"):
+        code, m, e, *reason = line.split()
+        yield int(code, 16), Fraction(int(m)) * Fraction(2) ** int(e), m == "-0", " ".join(reason)
+
+
+def pack_e2m1(codes: np.ndarray) -> np.ndarray:
+    """[rows, K] 4-bit codes -> [rows, K/2] bytes, value k in byte k//2, even k in the low bits."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    return (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+
+
+def w4a8_cases():
+    """Yield dicts with qa (uint8 [M,K]), sa (float32 [M,KB]), qw (packed uint8 [N,K/2]),
+    scale (float32 [N]), zero (float32 [N] or None) and c (float64 [M,N]) from w4a8_worked.txt."""
+    it = _lines("w4a8_worked.txt")
+    for line in it:
+        parts = line.split()
+        assert parts[0] == "case", line
+        name, M, N, K = parts[1], int(parts[2]), int(parts[3]), int(parts[4])
+        kb = math.ceil(K / 128)
+        qa = np.zeros((M, K), np.uint8)
+        codes = np.zeros((N, K), np.uint8)
+        case = {"name": name, "M": M, "N": N, "K": K, "zero": None}
+        for line in it:
+            if line == "end":
+                break
+            tag, *vals = line.split()
+            if tag == "a":
+                qa[int(vals[0]), int(vals[1])] = int(vals[2], 16)
+            elif tag == "w":
+                codes[int(vals[0]), int(vals[1])] = int(vals[2], 16)
+            elif tag == "sa":
+                case["sa"] = np.array([float(v) for v in vals], dtype=np.float32).reshape(M, kb)
+            elif tag == "scale":
+                case["scale"] = np.array([float(v) for v in vals], dtype=np.float32)
+            elif tag == "zero":
+                if vals != ["none"]:
+                    case["zero"] = np.array([float(v) for v in vals], dtype=np.float32)
+            elif tag == "c":
+                case["c"] = np.array([float(v) for v in vals], dtype=np.float64).reshape(M, N)
+        case["qa"] = qa
+        case["qw"] = pack_e2m1(codes)
+        yield case

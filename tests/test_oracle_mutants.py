@@ -40,6 +40,15 @@ MUTANTS = {
     "B scale indexed by row, not row block": ("(double)SB[(n / 128) * kb + k / 128]",
                                                "(double)SB[(n % 2) * kb + k / 128]"),
     "B scale ignored": ("* (double)SB[(n / 128) * kb + k / 128]", ""),
+    "e2m1 nibbles swapped": ("(k % 2 == 0) ? (uint8_t)(byte & 0xF) : (uint8_t)(byte >> 4)",
+                             "(k % 2 == 1) ? (uint8_t)(byte & 0xF) : (uint8_t)(byte >> 4)"),
+    "e2m1 bias 2": ("ldexp((double)(2 + frac), expo - 1 - 1)", "ldexp((double)(2 + frac), expo - 2 - 1)"),
+    "e2m1 sign ignored": ("    return sign ? -v : v;\n}\n\n/* fp64 -> bf16",
+                          "    return v;\n}\n\n/* fp64 -> bf16"),
+    "e2m1 zero point scaled": ("w += (double)WZ[n];", "w += (double)WZ[n] * (double)WS[n];"),
+    "e2m1 zero point ignored": ("w += (double)WZ[n];", "w += 0.0;"),
+    "e2m1 scale of channel 0": ("oracle_e2m1_to_f64(code) * (double)WS[n]",
+                                "oracle_e2m1_to_f64(code) * (double)WS[0]"),
     "grouped rows use expert 0": ("row_b[r] = e * N * K;", "row_b[r] = 0;"),
     "grouped rows use the next expert": ("row_b[r] = e * N * K;",
                                          "row_b[r] = ((e + 1) % E) * N * K;"),
@@ -133,6 +142,28 @@ def battery(lib):
                     * Fraction(float(sa[m, k])) * Fraction(float(sb[n // 128, k])) for k in range(2))
             ok &= cref[m, n] == float(q)
     check("fp8 pow2 closed form", ok)
+
+    # e2m1 table and the worked W4A8 cases
+    got = oracle.e2m1_to_f64(np.arange(16, dtype=np.uint8), lib=lib)
+    ok = all(got[c] == float(v) and (v != 0 or bool(np.signbit(got[c])) == nz)
+             for c, v, nz, _ in golden_io.e2m1_cases())
+    check("e2m1 table", ok)
+    ok = True
+    for case in golden_io.w4a8_cases():
+        cref, _ = oracle.gemm_w4a8(case["qa"], case["sa"], case["qw"], case["scale"], case["zero"],
+                                   lib=lib)
+        ok &= np.array_equal(cref, case["c"])
+    check("golden w4a8", ok)
+    # zero point: all-zero codes give C = zero[n] * rowsum(a)[m]; a second channel scale differs
+    r = np.random.default_rng(13)
+    qa = torch.from_numpy(r.integers(-4, 5, (2, 128)).astype(np.float32)) \
+        .to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    sa = np.exp2(r.integers(-2, 3, (2, 1))).astype(np.float32)
+    ws = np.array([0.5, 0.125, 0.25], np.float32)
+    wz = np.array([0.25, -0.75, 1.5], np.float32)
+    cref, _ = oracle.gemm_w4a8(qa, sa, np.zeros((3, 64), np.uint8), ws, wz, lib=lib)
+    rs = (e4m3_values(qa) * sa.astype(np.float64)).sum(axis=1)
+    check("w4a8 zero-point closed form", np.array_equal(cref, np.outer(rs, wz.astype(np.float64))))
 
     # grouped: integer data, distinct experts, one empty
     E, N, K = 3, 4, 8
