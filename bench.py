@@ -239,7 +239,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true", help="skip the other workloads' timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["decode", "prefill", "fp8", "moe"], default=None,
+    ap.add_argument("--profile", choices=["decode", "prefill", "fp8", "w4a8", "moe"], default=None,
                     help="launch one workload --profile-launches times, untimed (for ncu captures)")
     ap.add_argument("--profile-m", type=int, default=64, help="M (MoE: tokens T) for --profile")
     ap.add_argument("--profile-launches", type=int, default=4)
@@ -425,6 +425,19 @@ def profile_case(args):
         C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         calls = [lambda i=i: bg.bi_gemm_run(plan, qa, qbs[i % 3], C, scale_a=sa, scale_b=sb)
                  for i in range(L)]
+    elif args.profile == "w4a8":
+        N = K = 7168
+        KB = K // 128
+        plan = weight_plan(N, K, bg.BI_DTYPE_E2M1_W4A8)
+        qws = [inputs.e2m1_packed_uniform(N, K, seed=61 + i, device=dev) for i in range(6)]
+        ws = inputs.channel_scales_pow2(N, seed=62, device=dev)
+        wz = inputs.channel_zeros_fp16(ws, seed=63)
+        qa = inputs.e4m3_gaussian((M, K), seed=64, device=dev)
+        sa = inputs.scales_log_uniform((KB, ((M + 3) // 4) * 4), seed=65, device=dev)[:, :M]
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        work = torch.empty(bg.bi_gemm_w4a8_workspace_bytes(M) // 4, dtype=torch.float32, device=dev)
+        calls = [lambda i=i: bg.bi_gemm_run_w4a8(plan, qa, sa, qws[i % 6], ws, C, w_zero=wz,
+                                                 workspace=work) for i in range(L)]
     else:
         E, N, K = 64, 2048, 7168
         plan = weight_plan(N, K, bg.BI_DTYPE_BF16, E)
@@ -445,7 +458,8 @@ def profile_case(args):
 
 def kernel_label(bg, plan) -> str:
     i = bg.bi_gemm_plan_describe(plan)
-    return (f"bi_gemm_kernel<BM={i['block_m']},BN={i['block_n']},{'e4m3' if i['dtype'] else 'bf16'}>"
+    dt = {0: "bf16", 1: "e4m3", 2: "e2m1 x e4m3"}[i["dtype"]]
+    return (f"bi_gemm_kernel<BM={i['block_m']},BN={i['block_n']},{dt}>"
             f" rings A{i['stages_a']}/B{i['stages']}")
 
 
@@ -582,6 +596,32 @@ def measure_extras(bg, inputs, dev, stream, peaks):
         res[f"fp8_M{M}"] = {"us": t * 1e6, "TFLOP/s": tf, "tensor_frac": tf / fp8_peak,
                             "GB/s": b / t / 1e9, "hbm_frac": b / t / 1e9 / hbm}
     del qbs
+    # e2m1 weights (per-channel 2^-j scale and fp16 zero point) x e4m3 activations, N = K = 7168;
+    # 8 weight copies (205 MB) rotate so that every launch reads W from HBM
+    plan = weight_plan(N, K, bg.BI_DTYPE_E2M1_W4A8)
+    qws = [inputs.e2m1_packed_uniform(N, K, seed=6001 + i, device=dev) for i in range(8)]
+    ws = inputs.channel_scales_pow2(N, seed=6002, device=dev)
+    wz = inputs.channel_zeros_fp16(ws, seed=6003)
+    for M in [1, 64, 4096]:
+        qa = inputs.e4m3_gaussian((M, K), seed=6004, device=dev)
+        sa = inputs.scales_log_uniform((KB, ((M + 3) // 4) * 4), seed=6005, device=dev)[:, :M]
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        work = torch.empty(bg.bi_gemm_w4a8_workspace_bytes(M) // 4, dtype=torch.float32, device=dev)
+        fns = [lambda i=i: bg.bi_gemm_run_w4a8(plan, qa, sa, qws[i % 8], ws, C, w_zero=wz,
+                                               workspace=work, stream=stream) for i in range(8)]
+        t = graph_time_per_launch(fns, stream, reps=4)
+        b = N * K // 2 + M * K + 2 * M * N + 4 * M * KB + 8 * N + 8 * M
+        tf = 2 * M * N * K / t / 1e12
+        res[f"w4a8_M{M}"] = {"us": t * 1e6, "TFLOP/s": tf, "tensor_frac": tf / fp8_peak,
+                             "GB/s": b / t / 1e9, "hbm_frac": b / t / 1e9 / hbm}
+        if M in (1, 4096):   # without zero points: no row-sum kernel, C = scale * acc
+            fns = [lambda i=i: bg.bi_gemm_run_w4a8(plan, qa, sa, qws[i % 8], ws, C, stream=stream)
+                   for i in range(8)]
+            t = graph_time_per_launch(fns, stream, reps=4)
+            b = N * K // 2 + M * K + 2 * M * N + 4 * M * KB + 4 * N
+            res[f"w4a8_M{M}_no_zero"] = {"us": t * 1e6, "TFLOP/s": 2 * M * N * K / t / 1e12,
+                                         "GB/s": b / t / 1e9, "hbm_frac": b / t / 1e9 / hbm}
+    del qws
     # MoE: 64 experts, N = 2048, K = 7168, top-8
     E, N, K = 64, 2048, 7168
     plan = weight_plan(N, K, bg.BI_DTYPE_BF16, E)

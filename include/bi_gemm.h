@@ -54,7 +54,10 @@ extern "C" {
 
 typedef enum {
     BI_DTYPE_BF16 = 0,              /* A, B bf16; C bf16 */
-    BI_DTYPE_E4M3_BLOCKSCALED = 1   /* A, B e4m3 (fn) with fp32 block scales; C bf16 */
+    BI_DTYPE_E4M3_BLOCKSCALED = 1,  /* A, B e4m3 (fn) with fp32 block scales; C bf16 */
+    BI_DTYPE_E2M1_W4A8 = 2          /* A e4m3 with fp32 block scales, B packed e2m1 weights with a
+                                       power-of-two scale and a zero point per output column;
+                                       C bf16 (bi_gemm_run_w4a8) */
 } bi_dtype_t;
 
 typedef enum {
@@ -110,7 +113,8 @@ const char *bi_status_string(bi_status_t status);
  * same tile configuration in every process and on every device.  It touches no device and can
  * be created on a machine without a GPU.
  * Errors: BI_ERR_INVALID_ARG (out == NULL, N < 0, K < 0, num_experts < 1),
- * BI_ERR_UNSUPPORTED_SHAPE (num_experts > 1024, or grouped with FP8).
+ * BI_ERR_UNSUPPORTED_SHAPE (num_experts > 1024, grouped with FP8 or e2m1, or e2m1 with K not a
+ * multiple of 128).
  */
 bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
                          int num_experts);
@@ -130,7 +134,8 @@ bi_status_t bi_gemm_plan_describe(bi_plan_t plan, bi_plan_info_t *info);
  * scale_a = scale_b = NULL and ld_sa = 0.
  * M = 0 (or N = 0) is a no-op returning BI_OK.  K = 0 writes zeros.
  * Errors: BI_ERR_INVALID_ARG, BI_ERR_ALIGNMENT, BI_ERR_DTYPE_MISMATCH, BI_ERR_NO_DEVICE,
- * BI_ERR_CUDA; a grouped plan returns BI_ERR_INVALID_ARG.
+ * BI_ERR_CUDA; a grouped plan returns BI_ERR_INVALID_ARG, a BI_DTYPE_E2M1_W4A8 plan
+ * BI_ERR_DTYPE_MISMATCH (it runs through bi_gemm_run_w4a8).
  */
 bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M,
                         const void *A, int64_t lda,
@@ -159,6 +164,52 @@ bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows,
                                 void *C, int64_t ldc,
                                 const int32_t *expert_offsets,
                                 cudaStream_t stream);
+
+/*
+ * e2m1 (FP4) weights x e4m3 (FP8) activations, plan dtype BI_DTYPE_E2M1_W4A8.
+ *
+ * The weights follow the quantisation of "DeepSeek V4的batch invariance：大模型确定性推理的工程
+ * 基石" (lshu.cn), section 4.3: W[n][k] = q[n][k] * w_scale[n] + w_zero[n], where q is an e2m1
+ * value (1 sign, 2 exponent bits with bias 1, 1 fraction bit: 0, 0.5, 1, 1.5, 2, 3, 4, 6), the
+ * per-channel scale is 2^-j with j in [1, 12] and the zero point is a value fp16 represents
+ * exactly, so every dequantised weight is exact.  The activations are as for
+ * BI_DTYPE_E4M3_BLOCKSCALED: a[m][k] = e4m3(A[m][k]) * scale_a[(k/128)*ld_sa + m].
+ *
+ *   C[m][n] = bf16( sum_k a[m][k] * W[n][k] )
+ *
+ * computed as: the MMA takes the e2m1 codes directly (tcgen05 kind::f8f6f4), each 128-wide K
+ * block's partial product is promoted with scale_a alone in ascending kb (acc = fma(P_kb,
+ * scale_a[m,kb], acc)), and the column's constants are applied once at the end:
+ * C = fma(w_zero[n], rowsum[m], w_scale[n] * acc), with rowsum[m] = sum_k a[m][k] (fixed order:
+ * per 128-block, then ascending kb).  A power-of-two scale multiplies exactly, so it can leave the
+ * K sum.  The bits of C[m, :] depend on row m of A and scale_a, W and the column constants only.
+ *
+ * Device pointers:
+ *   A        e4m3 [M][lda] (lda >= K, 16-byte aligned rows)
+ *   scale_a  fp32, K-block-major [K/128][ld_sa], ld_sa >= M
+ *   W        packed e2m1 [N][ldw / 2 bytes]: value k of row n is in byte k/2 of the row, the even
+ *            k in the low four bits.  ldw (in values) >= K and a multiple of 64; W 32-byte aligned.
+ *   w_scale  fp32 [N], each 2^-j with j in [1, 12]
+ *   w_zero   fp32 [N] of fp16-exact values, or NULL for no zero points (then C = w_scale * acc)
+ *   workspace  fp32 scratch of at least bi_gemm_w4a8_workspace_bytes(M) bytes (16-byte aligned)
+ *              for the row sums; needed only with w_zero (may be NULL otherwise)
+ *   C        bf16 [M][ldc]
+ * K must be a multiple of 128 (the plan refuses others).  A scale outside {2^-1 .. 2^-12} or a
+ * zero point fp16 cannot represent is reported on the device: the launch completes and
+ * bi_gemm_sync_status returns BI_ERR_INVALID_ARG.
+ * Errors: BI_ERR_INVALID_ARG, BI_ERR_ALIGNMENT, BI_ERR_DTYPE_MISMATCH (not a W4A8 plan),
+ * BI_ERR_NO_DEVICE, BI_ERR_CUDA.
+ */
+size_t bi_gemm_w4a8_workspace_bytes(int64_t M);
+
+bi_status_t bi_gemm_run_w4a8(bi_plan_t plan, int64_t M,
+                             const void *A, int64_t lda,
+                             const float *scale_a, int64_t ld_sa,
+                             const void *W, int64_t ldw,
+                             const float *w_scale, const float *w_zero,
+                             float *workspace, size_t workspace_bytes,
+                             void *C, int64_t ldc,
+                             cudaStream_t stream);
 
 /*
  * Dense GEMM from host memory: copies A (and scale_a) from the host buffers into the caller's

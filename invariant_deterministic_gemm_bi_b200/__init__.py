@@ -1,7 +1,8 @@
 """Batch-invariant GEMM for NVIDIA B200 (sm_100a).
 
 C[M,N] = A[M,K] . B[N,K]^T with fp32 accumulation and bf16 output, computed by hand-written
-tcgen05/TMA kernels behind the C ABI in ``include/bi_gemm.h``; the MoE routing, dispatch, gather
+tcgen05/TMA kernels behind the C ABI in ``include/bi_gemm.h`` (bf16, FP8 e4m3 with block scales,
+and e2m1 weights with per-channel power-of-two scales and zero points x e4m3 activations); the MoE routing, dispatch, gather
 and combine steps around the grouped GEMM are in ``include/bi_moe.h``, and the dual-kernel
 decode attention in ``include/bi_attention.h``.  Every output row is
 bit-identical whatever the batch size, the row's position and the other rows in the batch.
@@ -12,6 +13,7 @@ input generators; ``build`` the nvcc build of ``libbigemm.so``.
 from .binding import (  # noqa: F401
     BI_DEBUG_SKIP_FIRST_LOAD,
     BI_DTYPE_BF16,
+    BI_DTYPE_E2M1_W4A8,
     BI_DTYPE_E4M3_BLOCKSCALED,
     BI_PLAN_RESIDENT_WEIGHTS,
     BiGemmError,
@@ -29,9 +31,11 @@ from .binding import (  # noqa: F401
     bi_gemm_run_host,
     bi_gemm_run_host_noalloc,
     bi_gemm_run_splitk,
+    bi_gemm_run_w4a8,
     bi_gemm_set_wait_timeout,
     bi_gemm_splitk_workspace_bytes,
     bi_gemm_sync_status,
+    bi_gemm_w4a8_workspace_bytes,
     bi_grouped_gemm_run,
     bi_moe_combine,
     bi_moe_dispatch,

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(PKG, "libbigemm.so")
 
 BI_DTYPE_BF16 = 0
 BI_DTYPE_E4M3_BLOCKSCALED = 1
+BI_DTYPE_E2M1_W4A8 = 2
 BI_DEBUG_SKIP_FIRST_LOAD = 1
 BI_PLAN_RESIDENT_WEIGHTS = 1
 
@@ -35,6 +36,7 @@ EXPORTED = [
     "bi_gemm_sync_status", "bi_gemm_set_wait_timeout", "bi_gemm_debug_set_flags",
     "bi_gemm_run_host_noalloc", "bi_gemm_plan_set_flags",
     "bi_gemm_plan_splitk", "bi_gemm_splitk_workspace_bytes", "bi_gemm_run_splitk",
+    "bi_gemm_w4a8_workspace_bytes", "bi_gemm_run_w4a8",
     "bi_moe_route_topk", "bi_moe_dispatch", "bi_moe_gather_rows", "bi_moe_combine",
     "bi_decode_attention", "bi_decode_attention_workspace_bytes",
 ]
@@ -107,6 +109,11 @@ def load_library(path: str = LIB_PATH):
     lib.bi_gemm_splitk_workspace_bytes.argtypes = [vp, i64]
     lib.bi_gemm_run_splitk.restype = i32
     lib.bi_gemm_run_splitk.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, ctypes.c_size_t, vp]
+    lib.bi_gemm_w4a8_workspace_bytes.restype = ctypes.c_size_t
+    lib.bi_gemm_w4a8_workspace_bytes.argtypes = [i64]
+    lib.bi_gemm_run_w4a8.restype = i32
+    lib.bi_gemm_run_w4a8.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, vp, vp, ctypes.c_size_t,
+                                     vp, i64, vp]
     lib.bi_moe_route_topk.restype = i32
     lib.bi_moe_route_topk.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp]
     lib.bi_moe_dispatch.restype = i32
@@ -278,6 +285,29 @@ def bi_gemm_run_splitk(plan: Plan, A, B, C, workspace, stream=None, M: int | Non
                                            _ptr(C), C.stride(0), _ptr(workspace), nbytes,
                                            _stream_handle(stream))
     _check(st, "bi_gemm_run_splitk")
+    return C
+
+
+def bi_gemm_w4a8_workspace_bytes(M: int) -> int:
+    return int(load_library().bi_gemm_w4a8_workspace_bytes(M))
+
+
+def bi_gemm_run_w4a8(plan: Plan, A, scale_a, W, w_scale, C, w_zero=None, workspace=None,
+                     stream=None, M: int | None = None):
+    """e2m1 weights x e4m3 activations: C[:M] = deq(A[:M]) . deq(W)^T.
+
+    A e4m3 (or uint8) [M, lda]; scale_a fp32 [K/128, ld_sa] (K-block-major); W uint8 [N, ldw/2]
+    packed e2m1 (two values per byte, the even K index in the low four bits); w_scale fp32 [N]
+    (each 2^-j, j in 1..12); w_zero fp32 [N] or None; workspace a device tensor of at least
+    bi_gemm_w4a8_workspace_bytes(M) bytes when w_zero is given.
+    """
+    M = A.shape[0] if M is None else M
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = load_library().bi_gemm_run_w4a8(plan.handle, M, _ptr(A), A.stride(0), _ptr(scale_a),
+                                         scale_a.stride(0), _ptr(W), W.stride(0) * 2, _ptr(w_scale),
+                                         _ptr(w_zero), _ptr(workspace), nbytes, _ptr(C), C.stride(0),
+                                         _stream_handle(stream))
+    _check(st, "bi_gemm_run_w4a8")
     return C
 
 

@@ -45,28 +45,37 @@ struct KernelEntry {
     int smem;
     int nsplit;    // MMAs per K step (MMA N = bn / nsplit)
     bool ksplit;   // fixed-split-K research variant (fp32 partials + merge)
+    bool w4;       // e2m1 weights with per-column scale and zero point (with fp8)
 };
 
 #define BI_ENTRY(BM, BN, KC, F8, GR)                                                               \
     KernelEntry{bi::Epi<F8, BN>::kThreads, BM, BN, KC, F8, GR, false,                              \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, GR>,                                           \
-                bi::smem_bytes_for<BM, BN, KC, F8, GR>(), 1, false}
+                bi::smem_bytes_for<BM, BN, KC, F8, GR>(), 1, false, false}
+#define BI_ENTRY_W4(BM, BN, KC)                                                                    \
+    KernelEntry{bi::Epi<true, BN>::kThreads, BM, BN, KC, true, false, false,                       \
+                &bi::bi_gemm_kernel<BM, BN, KC, true, false, 1, false, true>,                      \
+                bi::smem_bytes_for<BM, BN, KC, true, false, 1, false, true>(), 1, false, true}
+#define BI_ENTRY_W4_SPLIT2(BM, BN, KC)                                                             \
+    KernelEntry{bi::Epi<true, BN>::kThreads, BM, BN, KC, true, false, false,                       \
+                &bi::bi_gemm_kernel<BM, BN, KC, true, false, 2, false, true>,                      \
+                bi::smem_bytes_for<BM, BN, KC, true, false, 2, false, true>(), 2, false, true}
 #define BI_ENTRY_KSPLIT(BM, BN, KC)                                                                \
     KernelEntry{bi::Epi<false, BN>::kThreads, BM, BN, KC, false, false, false,                     \
                 &bi::bi_gemm_kernel<BM, BN, KC, false, false, 1, true>,                            \
-                bi::smem_bytes_for<BM, BN, KC, false, false, 1, true>(), 1, true}
+                bi::smem_bytes_for<BM, BN, KC, false, false, 1, true>(), 1, true, false}
 #define BI_ENTRY_SPLIT2(BM, BN, KC, F8)                                                            \
     KernelEntry{bi::Epi<F8, BN>::kThreads, BM, BN, KC, F8, false, false,                           \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, false, 2>,                                     \
-                bi::smem_bytes_for<BM, BN, KC, F8, false, 2>(), 2, false}
+                bi::smem_bytes_for<BM, BN, KC, F8, false, 2>(), 2, false, false}
 #define BI_ENTRY_GROUPED_SPLIT2(BM, BN, KC)                                                        \
     KernelEntry{bi::Epi<false, BN>::kThreads, BM, BN, KC, false, true, false,                      \
                 &bi::bi_gemm_kernel<BM, BN, KC, false, true, 2>,                                   \
-                bi::smem_bytes_for<BM, BN, KC, false, true, 2>(), 2, false}
+                bi::smem_bytes_for<BM, BN, KC, false, true, 2>(), 2, false, false}
 #define BI_PAIR(BN, KC, F8, GR)                                                                    \
     KernelEntry{bi::Epi<F8, BN>::kThreads, 256, BN, KC, F8, GR, true,                              \
                 &bi::bi_gemm_kernel_pair<BN, KC, F8, GR>,                                          \
-                bi::smem_bytes_for_pair<BN, KC, F8, GR>(), 1, false}
+                bi::smem_bytes_for_pair<BN, KC, F8, GR>(), 1, false, false}
 
 // Narrow tiles (BN <= 64) run on one CTA; wide ones (BN >= 128) on a CTA pair.  Every tile comes
 // in two forms: its preferred number of 128-byte K chunks per pipeline stage (3-D TMA boxes;
@@ -89,6 +98,9 @@ const KernelEntry kKernels[] = {
     BI_PAIR(128, 1, false, false),      BI_PAIR(128, 2, false, false),
     BI_PAIR(256, 1, false, false),      BI_PAIR(256, 2, false, false),
     BI_PAIR(128, 1, true, false),       BI_PAIR(128, 2, true, false),
+    // e2m1 weights x e4m3 activations (the FP8 tiles; K is a multiple of 128)
+    BI_ENTRY_W4(128, 32, 4),            BI_ENTRY_W4(128, 64, 2),
+    BI_ENTRY_W4(128, 64, 4),            BI_ENTRY_W4_SPLIT2(128, 128, 2),
     // fixed-split-K research variant (bi_gemm_plan_splitk), not the product path
     BI_ENTRY_KSPLIT(128, 32, 1),        BI_ENTRY_KSPLIT(128, 32, 4),
     BI_ENTRY_KSPLIT(128, 64, 1),        BI_ENTRY_KSPLIT(128, 64, 2),
@@ -98,12 +110,12 @@ constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
 
 int preferred_chunks(int bn) { return bn <= 32 ? 4 : 2; }
 
-const KernelEntry *find_kernel(int bm, int bn, int kc, bool fp8, bool grouped)
+const KernelEntry *find_kernel(int bm, int bn, int kc, bool fp8, bool grouped, bool w4 = false)
 {
     for (int i = 0; i < kNumKernels; ++i)
         if (kKernels[i].bm == bm && kKernels[i].bn == bn && kKernels[i].kc == kc &&
             kKernels[i].fp8 == fp8 && kKernels[i].grouped == grouped && kKernels[i].nsplit == 1 &&
-            !kKernels[i].ksplit)
+            !kKernels[i].ksplit && kKernels[i].w4 == w4)
             return &kKernels[i];
     return nullptr;
 }
@@ -183,6 +195,7 @@ TileChoice choose_tile(int64_t N, int64_t K, bi_dtype_t dtype, int experts)
         {2048, 7168, BI_DTYPE_BF16, 1, 256, 256},             // prefill-shaped, long K (CTA pair)
         {256, 512, BI_DTYPE_BF16, 1, 128, 32},                // small correctness shape
         {7168, 7168, BI_DTYPE_E4M3_BLOCKSCALED, 1, 128, 64},  // FP8 projection
+        {7168, 7168, BI_DTYPE_E2M1_W4A8, 1, 128, 64},         // the same projection, e2m1 weights
         {2048, 7168, BI_DTYPE_BF16, 64, 128, 128},            // MoE experts
     };
     for (const Row &r : table)
@@ -195,6 +208,8 @@ TileChoice choose_tile(int64_t N, int64_t K, bi_dtype_t dtype, int experts)
                 return {128, bn};
         return {128, 32};
     }
+    if (dtype == BI_DTYPE_E2M1_W4A8)   // one-CTA tiles only
+        return {128, (N + 63) / 64 >= 100 ? 64 : 32};
     // wide dense fallback tiles run on a CTA pair (256 rows)
     const int max_bn = dtype == BI_DTYPE_E4M3_BLOCKSCALED ? 128 : 256;
     for (int bn = max_bn; bn >= 128; bn /= 2)
@@ -348,6 +363,35 @@ bi_status_t encode_operand(CUtensorMap *map, const void *base, bool fp8, int64_t
     return r == CUDA_SUCCESS ? BI_OK : BI_ERR_CUDA;
 }
 
+// TMA map of packed e2m1 weights [rows][ld_elems / 2 bytes] (value k of a row in byte k / 2, the
+// even value in the low four bits).  The boxes are those of an 8-bit operand -- 128 values of K
+// per row, kc chunks per 3-D box -- and land in shared memory in the 16-byte-aligned form the
+// MMA reads (each 8 bytes of values followed by 8 unused bytes, so 128 bytes per box row).  The
+// format needs a 32-byte aligned base, row pitches of 32 bytes and K a multiple of 128.
+bi_status_t encode_e2m1(CUtensorMap *map, const void *base, int64_t K, int64_t rows, int64_t ld_elems,
+                        int box_rows, int kc)
+{
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r;
+    if (kc == 1) {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_elems / 2)};
+        cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+        r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        // [K / 128][rows][128 values]; a chunk of 128 values is 64 bytes of global memory
+        cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K / 128)};
+        cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld_elems / 2), 64u};
+        cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(kc)};
+        r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
+    return r == CUDA_SUCCESS ? BI_OK : BI_ERR_CUDA;
+}
+
 bi_status_t ensure_kernel_attr(const KernelEntry *k, DeviceInfo *d)
 {
     std::lock_guard<std::mutex> lock(g_dev_mu);
@@ -420,9 +464,16 @@ bi_status_t check_common(const bi_plan_s *plan, int64_t rows, const void *A, int
         return BI_ERR_INVALID_ARG;
     if (lda < plan->k || ldb < plan->k)
         return BI_ERR_INVALID_ARG;
-    const int elt = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED ? 1 : 2;
-    if (!aligned16(A) || !aligned16(B) || (lda * elt) % 16 != 0 || (ldb * elt) % 16 != 0)
+    const int elt = plan->dtype == BI_DTYPE_BF16 ? 2 : 1;   // bytes per A element
+    if (!aligned16(A) || (lda * elt) % 16 != 0)
         return BI_ERR_ALIGNMENT;
+    if (plan->dtype == BI_DTYPE_E2M1_W4A8) {
+        // packed e2m1 rows (two values per byte): 32-byte aligned base and row pitch
+        if ((reinterpret_cast<uintptr_t>(B) & 31u) != 0 || ldb % 64 != 0)
+            return BI_ERR_ALIGNMENT;
+    } else if (!aligned16(B) || (ldb * elt) % 16 != 0) {
+        return BI_ERR_ALIGNMENT;
+    }
     if (rows > INT32_MAX - 256 || plan->n * plan->experts > INT32_MAX - 512 ||
         plan->k > INT32_MAX - 256)
         return BI_ERR_UNSUPPORTED_SHAPE;
@@ -458,7 +509,7 @@ GemmParams base_params(const bi_plan_s *plan, const KernelEntry *k, int64_t rows
 {
     GemmParams p;
     std::memset(&p, 0, sizeof(p));
-    const int elt = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED ? 1 : 2;
+    const int elt = plan->dtype == BI_DTYPE_BF16 ? 2 : 1;   // bytes per A element
     p.rows = static_cast<int32_t>(rows);
     p.n = static_cast<int32_t>(plan->n);
     p.k = static_cast<int32_t>(plan->k);
@@ -617,7 +668,7 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     *out = nullptr;
     if (N < 0 || K < 0 || num_experts < 1)
         return BI_ERR_INVALID_ARG;
-    if (dtype != BI_DTYPE_BF16 && dtype != BI_DTYPE_E4M3_BLOCKSCALED)
+    if (dtype != BI_DTYPE_BF16 && dtype != BI_DTYPE_E4M3_BLOCKSCALED && dtype != BI_DTYPE_E2M1_W4A8)
         return BI_ERR_INVALID_ARG;
     if (num_experts > bi::kMaxExperts)
         return BI_ERR_UNSUPPORTED_SHAPE;
@@ -625,11 +676,14 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
         return BI_ERR_UNSUPPORTED_SHAPE;
     if (N > INT32_MAX / 2 || K > INT32_MAX / 2 || N * num_experts > INT32_MAX / 2)
         return BI_ERR_UNSUPPORTED_SHAPE;
-    const bool fp8 = dtype == BI_DTYPE_E4M3_BLOCKSCALED;
+    const bool w4 = dtype == BI_DTYPE_E2M1_W4A8;
+    if (w4 && K % 128 != 0)   // the packed e2m1 tensor format counts K in 128-value units
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    const bool fp8 = dtype != BI_DTYPE_BF16;
     const TileChoice tile = choose_tile(N, K, dtype, num_experts);
     const int chunk_elems = fp8 ? 128 : 64;
-    const int kc = (K > 0 && K % chunk_elems == 0) ? preferred_chunks(tile.bn) : 1;
-    const KernelEntry *k = find_kernel(tile.bm, tile.bn, kc, fp8, num_experts > 1);
+    const int kc = ((K > 0 && K % chunk_elems == 0) || w4) ? preferred_chunks(tile.bn) : 1;
+    const KernelEntry *k = find_kernel(tile.bm, tile.bn, kc, fp8, num_experts > 1, w4);
     if (!k)
         return BI_ERR_UNSUPPORTED_SHAPE;
     bi_plan_s *p = new (std::nothrow) bi_plan_s();
@@ -642,7 +696,7 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     p->kernel = k;
     if (num_experts == 1 && !k->pair && k->bm == 128 && k->kc == preferred_chunks(k->bn) &&
         k->bn == (fp8 ? 64 : 32))
-        p->kernel_small = find_kernel(128, k->bn, 2 * k->kc, fp8, false);
+        p->kernel_small = find_kernel(128, k->bn, 2 * k->kc, fp8, false, w4);
     if (num_experts > 1 && !k->pair && k->bm == 128 && k->bn == 128) {
         for (int i = 0; i < kNumKernels; ++i)
             if (kKernels[i].nsplit == 2 && kKernels[i].grouped && kKernels[i].bn == 256)
@@ -652,7 +706,7 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
         K % chunk_elems == 0) {
         for (int i = 0; i < kNumKernels; ++i)
             if (kKernels[i].nsplit == 2 && kKernels[i].bm == 128 && kKernels[i].bn == 2 * k->bn &&
-                kKernels[i].fp8 == fp8)
+                kKernels[i].fp8 == fp8 && kKernels[i].w4 == w4 && !kKernels[i].grouped)
                 p->kernel_wide = &kKernels[i];
     }
     *out = p;
@@ -682,7 +736,7 @@ bi_status_t bi_gemm_plan_describe(bi_plan_t plan, bi_plan_info_t *info)
 {
     if (!plan || !info)
         return BI_ERR_INVALID_ARG;
-    const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
+    const bool fp8 = plan->dtype != BI_DTYPE_BF16;
     std::memset(info, 0, sizeof(*info));
     info->n = plan->n;
     info->k = plan->k;
@@ -742,6 +796,8 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
         return BI_ERR_INVALID_ARG;
     if (plan->experts != 1 || plan->k_splits > 1)
         return BI_ERR_INVALID_ARG;
+    if (plan->dtype == BI_DTYPE_E2M1_W4A8)
+        return BI_ERR_DTYPE_MISMATCH;   // bi_gemm_run_w4a8
     const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
     if (fp8) {
         if (M > 0 && plan->n > 0 && plan->k > 0) {
@@ -845,6 +901,8 @@ bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M, const void *A_host, int6
         return BI_ERR_INVALID_ARG;
     if (M < 0)
         return BI_ERR_INVALID_ARG;
+    if (plan->dtype == BI_DTYPE_E2M1_W4A8)
+        return BI_ERR_DTYPE_MISMATCH;
     if (M == 0 || plan->n == 0)
         return BI_OK;
     const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
@@ -885,6 +943,8 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
         return BI_ERR_INVALID_ARG;
     if (plan->experts != 1 || plan->k_splits > 1 || M < 0)
         return BI_ERR_INVALID_ARG;
+    if (plan->dtype == BI_DTYPE_E2M1_W4A8)
+        return BI_ERR_DTYPE_MISMATCH;
     if (M == 0 || plan->n == 0)
         return BI_OK;
     const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
@@ -963,6 +1023,92 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
     if (cudaMemcpy(&host, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return BI_ERR_CUDA;
     return host == 0 ? BI_OK : static_cast<bi_status_t>(host);
+}
+
+// ---------------------------------------------------------------------------------------------
+// e2m1 weights x e4m3 activations
+// ---------------------------------------------------------------------------------------------
+
+size_t bi_gemm_w4a8_workspace_bytes(int64_t M)
+{
+    return M > 0 ? static_cast<size_t>(round256(M * 4)) : 0;
+}
+
+bi_status_t bi_gemm_run_w4a8(bi_plan_t plan, int64_t M, const void *A, int64_t lda,
+                             const float *scale_a, int64_t ld_sa, const void *W, int64_t ldw,
+                             const float *w_scale, const float *w_zero, float *workspace,
+                             size_t workspace_bytes, void *C, int64_t ldc, cudaStream_t stream)
+{
+    if (!plan)
+        return BI_ERR_INVALID_ARG;
+    if (plan->dtype != BI_DTYPE_E2M1_W4A8)
+        return BI_ERR_DTYPE_MISMATCH;
+    if (plan->experts != 1 || plan->k_splits > 1)
+        return BI_ERR_INVALID_ARG;
+    bi_status_t st = check_common(plan, M, A, lda, W, ldw, C, ldc);
+    if (st != BI_OK || M == 0 || plan->n == 0)
+        return st;
+    if (plan->k > 0) {
+        if (!scale_a || !w_scale)
+            return BI_ERR_INVALID_ARG;
+        if (ld_sa < M)
+            return BI_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(scale_a) & 3u) || (reinterpret_cast<uintptr_t>(w_scale) & 3u) ||
+            (reinterpret_cast<uintptr_t>(w_zero) & 3u))
+            return BI_ERR_ALIGNMENT;
+        if (w_zero) {
+            if (!workspace || workspace_bytes < bi_gemm_w4a8_workspace_bytes(M))
+                return BI_ERR_INVALID_ARG;
+            if (reinterpret_cast<uintptr_t>(workspace) & 15u)
+                return BI_ERR_ALIGNMENT;
+        }
+    }
+    int dev = 0;
+    DeviceInfo *d = nullptr;
+    if ((st = current_device(&dev, &d)) != BI_OK)
+        return st;
+    if (plan->k == 0)
+        return launch_zero(C, ldc, M, plan->n, stream);
+    int *status = nullptr;
+    if ((st = plan_status_word(plan, dev, &status)) != BI_OK)
+        return st;
+    const KernelEntry *k = dense_kernel_for(plan, d, M);
+    if ((st = ensure_kernel_attr(k, d)) != BI_OK)
+        return st;
+    CUtensorMap ta, tb;
+    const int a_rows = a_box_rows_for(k, M);
+    if ((st = encode_operand(&ta, A, true, plan->k, M, lda, a_rows, k->kc)) != BI_OK)
+        return st;
+    if ((st = encode_e2m1(&tb, W, plan->k, plan->n, ldw, b_box_rows_for(k), k->kc)) != BI_OK)
+        return st;
+    GemmParams p = base_params(plan, k, M, C, ldc, status);
+    if (!set_rows(&p, k, a_rows))
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    p.scale_a = scale_a;
+    p.ld_sa = ld_sa;
+    p.w_scale = w_scale;
+    p.w_zero = w_zero;
+    p.w_rowsum = w_zero ? workspace : nullptr;
+    if (w_zero) {
+        // the row sums of the dequantised A, for the zero-point term (one CTA per row); the
+        // GEMM reads them after this grid has completed (it is this kernel's programmatic
+        // dependent and waits for it before touching global memory)
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.gridDim = dim3(static_cast<unsigned>(M));
+        cfg.blockDim = dim3(256);
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, bi::bi_w4_rowsum_kernel, static_cast<const uint8_t *>(A), lda,
+                               scale_a, ld_sa, static_cast<int32_t>(M), static_cast<int32_t>(plan->k),
+                               workspace) != cudaSuccess)
+            return BI_ERR_CUDA;
+    }
+    const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
+    return launch_main(k, d, ta, tb, ta, p, tiles, stream);
 }
 
 // ---------------------------------------------------------------------------------------------

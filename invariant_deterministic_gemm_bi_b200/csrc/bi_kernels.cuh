@@ -40,6 +40,8 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "ptx_sm100.cuh"
 
@@ -63,6 +65,7 @@ struct Epi {
 constexpr int kMaxExperts = 1024;
 
 // Device status codes (the same values as bi_status_t).
+constexpr int kStatusInvalidArg = 1;
 constexpr int kStatusTimeout = 6;
 constexpr int kStatusBadOffsets = 7;
 
@@ -88,6 +91,12 @@ struct GemmParams {
     int64_t ld_sa;
     const float *scale_b;    // FP8: [ceil(N/128)][kb_scale]
     int32_t kb_scale;        // ceil(K / 128)
+    // e2m1 weights (W4 kernels) only, per output column n: the scale w_scale[n] = 2^-j with j in
+    // [1, 12] and the zero point w_zero[n] (a value fp16 represents exactly; null for none);
+    // w_rowsum[m] = the sum over k of row m of the dequantised A (read only with w_zero)
+    const float *w_scale;
+    const float *w_zero;
+    const float *w_rowsum;
     const int32_t *offsets;  // grouped: [E+1] (device)
     int *status;             // device status word
     uint64_t timeout_cycles; // limit of every pipeline wait, in SM clock cycles
@@ -262,10 +271,10 @@ __device__ __forceinline__ void store_row_chunk32_f32(float *wrow, int col0, int
 // BM      : output rows per tile = MMA M (64 or 128).  With M = 64 the accumulator's row i sits
 //           in TMEM lane (i % 16) + 32 * (i / 16), so each epilogue warp owns 16 rows.
 // FP8: the scales one epilogue thread needs for the KC chunks of group kg -- scale_a of its row
-// and scale_b of each of its 32-column blocks (32 columns never straddle a 128-column scale
-// block: the tile origin, the thread's first column and c * 32 are all multiples of 32).  Chunks
-// past the end of K and columns past N read nothing and get 0.
-template <int KC, int kLoads>
+// and (kBlockB) scale_b of each of its 32-column blocks (32 columns never straddle a 128-column
+// scale block: the tile origin, the thread's first column and c * 32 are all multiples of 32).
+// Chunks past the end of K and columns past N read nothing and get 0.
+template <int KC, int kLoads, bool kBlockB = true>
 __device__ __forceinline__ void load_group_scales(const GemmParams &p, const float *sa_col, bool row_ok,
                                                   int col_first, int kg, int nkb, float (&sa)[KC],
                                                   float (&sb)[KC][kLoads])
@@ -275,14 +284,137 @@ __device__ __forceinline__ void load_group_scales(const GemmParams &p, const flo
         const int kb = kg * KC + cc;
         const bool kb_ok = kb < nkb;
         sa[cc] = (row_ok && kb_ok) ? __ldg(sa_col + static_cast<int64_t>(kb) * p.ld_sa) : 0.0f;
+        if constexpr (kBlockB) {
 #pragma unroll
-        for (int c = 0; c < kLoads; ++c) {
-            const int col = col_first + c * 32;
-            sb[cc][c] = (kb_ok && col < p.n)
-                            ? __ldg(p.scale_b + static_cast<int64_t>(col >> 7) * p.kb_scale + kb)
-                            : 0.0f;
+            for (int c = 0; c < kLoads; ++c) {
+                const int col = col_first + c * 32;
+                sb[cc][c] = (kb_ok && col < p.n)
+                                ? __ldg(p.scale_b + static_cast<int64_t>(col >> 7) * p.kb_scale + kb)
+                                : 0.0f;
+            }
         }
     }
+}
+
+// e2m1 weights: the column constants of one epilogue thread's kLoads 32-column blocks, loaded
+// once per tile and spread over the warp (lane j holds column col_first + 32 c + j), and the
+// zero-point row sum of the thread's row.  A scale that is not 2^-j (j in [1, 12]) or a zero point
+// fp16 cannot represent sets BI_ERR_INVALID_ARG in the status word (the columns are computed all
+// the same).  Columns past N get scale 1 and zero 0 and are never stored.
+template <int kLoads>
+struct W4Consts {
+    float scale[kLoads];
+    float zero[kLoads];
+    float rowsum;
+};
+
+template <int kLoads>
+__device__ __forceinline__ W4Consts<kLoads> w4_load_consts(const GemmParams &p, int row, bool row_ok,
+                                                           int col_first, uint32_t lane)
+{
+    W4Consts<kLoads> w;
+    const bool zp = p.w_zero != nullptr;
+    bool bad = false;
+#pragma unroll
+    for (int c = 0; c < kLoads; ++c) {
+        const int col = col_first + c * 32 + static_cast<int>(lane);
+        const bool ok = col < p.n;
+        w.scale[c] = ok ? __ldg(p.w_scale + col) : 1.0f;
+        w.zero[c] = (ok && zp) ? __ldg(p.w_zero + col) : 0.0f;
+        const uint32_t sbits = __float_as_uint(w.scale[c]);
+        const uint32_t e = sbits >> 23;   // sign 0 and a biased exponent in [115, 126]
+        bad |= ok && ((sbits & 0x7FFFFFu) != 0u || e < 127u - 12u || e > 127u - 1u);
+        bad |= ok && zp && __half2float(__float2half_rn(w.zero[c])) != w.zero[c];
+    }
+    w.rowsum = (zp && row_ok) ? __ldg(p.w_rowsum + row) : 0.0f;
+    if (bad)
+        atomicCAS(p.status, 0, kStatusInvalidArg);
+    return w;
+}
+
+// C = fma(zero[n], rowsum[m], scale[n] * acc), or scale[n] * acc without zero points, for the
+// thread's 32 kLoads promoted sums.  Warp-collective (the constants come by shuffle).
+template <int kLoads>
+__device__ __forceinline__ void w4_finish(const GemmParams &p, const W4Consts<kLoads> &w,
+                                          float (&acc)[32 * kLoads])
+{
+    const bool zp = p.w_zero != nullptr;
+#pragma unroll
+    for (int c = 0; c < kLoads; ++c) {
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+            const float s = __shfl_sync(0xFFFFFFFFu, w.scale[c], jj);
+            const float z = __shfl_sync(0xFFFFFFFFu, w.zero[c], jj);
+            const float v = s * acc[c * 32 + jj];
+            acc[c * 32 + jj] = zp ? fmaf(z, w.rowsum, v) : v;
+        }
+    }
+}
+
+// e2m1 weights with zero points: rowsum[m] = the sum over the K chunks kb (ascending) of
+// scale_a[m,kb] * t[m,kb], in fp32, where t[m,kb] is the sum of row m's 128 e4m3 values of chunk
+// kb: lane l of a warp adds the values 4l .. 4l+3 in order and the warp adds the 32 lane sums in a
+// fixed butterfly.  One CTA per row: its warps take the chunks in turn and one thread then runs
+// the chain r = fma(t, scale_a, r).  The order is fixed by K alone, so rowsum[m] depends on row m
+// only.  K is a multiple of 128.
+__global__ void __launch_bounds__(256) bi_w4_rowsum_kernel(const uint8_t *a, int64_t lda,
+                                                           const float *scale_a, int64_t ld_sa,
+                                                           int32_t m_rows, int32_t k, float *rowsum)
+{
+    constexpr int kSeg = 256;   // chunks per pass through shared memory
+    constexpr int kWarps = 8;
+    __shared__ float s_t[kSeg], s_s[kSeg];
+    ptx::grid_dependency_wait();
+    if (threadIdx.x == 0)
+        ptx::launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t row = blockIdx.x;
+    if (row >= m_rows)
+        return;
+    const uint8_t *arow = a + row * lda;
+    const int nkb = k / 128;
+    float r = 0.0f;
+    for (int kb0 = 0; kb0 < nkb; kb0 += kSeg) {
+        const int nseg = nkb - kb0 < kSeg ? nkb - kb0 : kSeg;
+        for (int c0 = warp; c0 < nseg; c0 += 8 * kWarps) {
+            uint32_t wv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + i * kWarps;
+                wv[i] = c < nseg
+                            ? __ldg(reinterpret_cast<const uint32_t *>(arow + static_cast<int64_t>(kb0 + c) * 128) + lane)
+                            : 0u;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + i * kWarps;
+                if (c >= nseg)
+                    break;
+                float t = 0.0f;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    __nv_fp8_e4m3 q;
+                    q.__x = static_cast<__nv_fp8_storage_t>((wv[i] >> (8 * b)) & 0xFFu);
+                    t += static_cast<float>(q);
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1)
+                    t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+                if (lane == 0) {
+                    s_t[c] = t;
+                    s_s[c] = __ldg(scale_a + static_cast<int64_t>(kb0 + c) * ld_sa + row);
+                }
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x == 0)
+            for (int c = 0; c < nseg; ++c)
+                r = fmaf(s_t[c], s_s[c], r);
+        __syncthreads();
+    }
+    if (threadIdx.x == 0)
+        rowsum[row] = r;
 }
 
 // BN      : output columns per tile (multiple of 32, <= 256; FP8 <= 128)
@@ -301,8 +433,17 @@ __device__ __forceinline__ void load_group_scales(const GemmParams &p, const flo
 // SPLIT   : the fixed-split-K research variant (bf16 dense only, not the batch-invariant product
 //           path): a work unit is one K split of a tile and its epilogue writes fp32 partial
 //           sums; bi_splitk_merge_kernel adds the splits in a fixed order.
+// W4      : (with FP8, dense) B holds e2m1 weights with one power-of-two scale and one zero point
+//           per output column ("DeepSeek V4的batch invariance：大模型确定性推理的工程基石"
+//           (lshu.cn), section 4.3: W = W_fp4 * scale + zero, scale in {2^-j : j = 1..12}).  The
+//           MMA takes the e2m1 codes as they are (kind::f8f6f4, B format e2m1) and the epilogue
+//           promotes each K chunk with scale_a alone, acc = fma(partial, scale_a[m,kb], acc), kb
+//           ascending; then C = fma(zero[n], rowsum[m], scale[n] * acc), or scale[n] * acc
+//           without zero points.  A power-of-two scale multiplies exactly, so pulling it out of
+//           the K sum changes no rounding.
 // The ring depths follow from (BM, BN, KC) (see Rings).
-template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool SPLIT = false>
+template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool SPLIT = false,
+          bool W4 = false>
 __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     bi_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,
@@ -318,6 +459,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                   "split MMAs: dense bf16 64-wide, FP8 128-wide and grouped bf16 256-wide tiles as "
                   "two half-width instructions");
     static_assert(!SPLIT || (!FP8 && !GROUPED && NSPLIT == 1), "split-K variant: bf16 dense");
+    static_assert(!W4 || (FP8 && !GROUPED && !SPLIT), "e2m1 weights: the dense FP8 kernel");
     constexpr int kMmaN = BN / NSPLIT;                   // MMA instruction N
     using R = Rings<BM, BN, KC>;
     constexpr int kElemsPerRow = FP8 ? 128 : 64;         // K elements per 128-byte row
@@ -337,7 +479,12 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     static_assert(kTmemColsNeeded <= 512, "TMEM holds 512 columns");
     static_assert(!FP8 || kNumAcc >= 2 * KC, "FP8 needs two groups of partial buffers");
     // (the host keeps sb > kNumAcc / KC so the FP8 epilogue can track partials on the consumed ring)
-    constexpr uint32_t kIdesc = FP8 ? ptx::idesc_e4m3(BM, kMmaN) : ptx::idesc_bf16(BM, kMmaN);
+    constexpr uint32_t kIdesc = W4    ? ptx::idesc_e4m3_e2m1(BM, kMmaN)
+                                : FP8 ? ptx::idesc_e4m3(BM, kMmaN)
+                                      : ptx::idesc_bf16(BM, kMmaN);
+    // bytes a B group brings: e2m1 values travel packed (two per byte) and land in shared memory
+    // in the 16-byte-aligned form, one byte of the tile per value
+    constexpr uint32_t kBTxBytes = W4 ? R::kBBytes / 2 : R::kBBytes;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
@@ -447,7 +594,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
         if (jb == 0 && (p.debug_flags & 1u)) {
             skipped_b0 = true;      // fault injection: this B group is never filled
         } else {
-            ptx::mbar_arrive_expect_tx(&full[bs], R::kBBytes);
+            ptx::mbar_arrive_expect_tx(&full[bs], kBTxBytes);
             load(smem_b + bs * R::kBBytes, &tmap_b, &full[bs], cb.tc.kb0, cb.kg, cb.tc.b_row0);
         }
         advance(cb);
@@ -786,10 +933,14 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                 // the scales of group kg + 1 are loaded while group kg is promoted, so their
                 // global-memory latency stays off the per-chunk chain
                 float sa_g[KC], sb_g[KC][kLoads];
-                load_group_scales<KC, kLoads>(p, sa_col, row_ok, tc.n0 + col0, 0, nkb, sa_g, sb_g);
+                load_group_scales<KC, kLoads, !W4>(p, sa_col, row_ok, tc.n0 + col0, 0, nkb, sa_g, sb_g);
+                // e2m1 weights: this tile's column constants, loaded before the K loop
+                W4Consts<kLoads> w4c;
+                if constexpr (W4)
+                    w4c = w4_load_consts<kLoads>(p, row, row_ok, tc.n0 + col0, lane);
                 for (int kg = 0; kg < nkg && ok; ++kg) {
                     float sa_n[KC], sb_n[KC][kLoads];
-                    load_group_scales<KC, kLoads>(p, sa_col, row_ok, tc.n0 + col0, kg + 1, nkb, sa_n, sb_n);
+                    load_group_scales<KC, kLoads, !W4>(p, sa_col, row_ok, tc.n0 + col0, kg + 1, nkb, sa_n, sb_n);
                     // the group's partials are ready when its consumed barrier completes; the MMA
                     // warp runs at most kNumAcc chunks (< sb groups) ahead, so the barrier cannot
                     // have moved on to the group sb later
@@ -821,7 +972,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                         ptx::mbar_arrive(&acce_bar[part]);   // the partial buffer is free again
 #pragma unroll
                         for (int c = 0; c < kLoads; ++c) {
-                            const float s = sa_g[cc] * sb_g[cc][c];
+                            const float s = W4 ? sa_g[cc] : sa_g[cc] * sb_g[cc][c];
 #pragma unroll
                             for (int jj = 0; jj < 32; ++jj)
                                 acc[c * 32 + jj] = fmaf(__uint_as_float(r[c][jj]), s, acc[c * 32 + jj]);
@@ -838,6 +989,8 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                 }
                 if (!ok)
                     break;
+                if constexpr (W4)
+                    w4_finish<kLoads>(p, w4c, acc);
                 if (row_ok) {
 #pragma unroll
                     for (int c = 0; c < kLoads; ++c) {
@@ -896,7 +1049,8 @@ __global__ void bi_splitk_merge_kernel(const float *ws, int64_t ld_ws, int64_t s
     }
 }
 
-template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool SPLIT = false>
+template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool SPLIT = false,
+          bool W4 = false>
 constexpr int smem_bytes_for()
 {
     return 1024 + kRingBytes + 1024 + (GROUPED ? 2 * (kMaxExperts + 1) * 4 : 0);

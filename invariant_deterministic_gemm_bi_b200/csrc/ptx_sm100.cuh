@@ -231,6 +231,15 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int m, int n)
            (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// kind::f8f6f4 with A = e4m3 (format 0) and B = e2m1 (format 5).  The e2m1 operand sits in
+// shared memory in the 16-byte-aligned form (16 values in 8 bytes, then 8 unused bytes), so its
+// tiles have the byte layout of an 8-bit operand: 128 K values per 128-byte swizzle row.
+__host__ __device__ constexpr uint32_t idesc_e4m3_e2m1(int m, int n)
+{
+    return (1u << 4) | (0u << 7) | (5u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
+
 // D[tmem] (+)= A[smem] . B[smem]^T, one elected thread.  accumulate = 0 overwrites D.
 __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate)

@@ -44,13 +44,14 @@ def test_abi_version_and_status_strings():
 
 def test_plan_describe_is_m_free_and_sane():
     for (N, K, dt, E) in [(4096, 7168, 0, 1), (7168, 2048, 0, 1), (2048, 7168, 0, 1),
-                          (7168, 7168, 1, 1), (2048, 7168, 0, 64), (256, 512, 0, 1), (5, 3, 0, 1)]:
+                          (7168, 7168, 1, 1), (2048, 7168, 0, 64), (256, 512, 0, 1), (5, 3, 0, 1),
+                          (7168, 7168, 2, 1), (256, 512, 2, 1)]:
         info = bg.bi_gemm_plan_describe(bg.bi_gemm_plan(N, K, dt, E))
         assert info["n"] == N and info["k"] == K and info["num_experts"] == E
         assert info["k_order_id"] == 0 and info["block_m"] in (64, 128, 256)
         assert info["mma_m"] == info["block_m"] and 2 <= info["stages_a"] <= info["stages"]
         assert info["cta_group"] == (2 if info["block_m"] == 256 else 1)
-        assert info["block_k"] * (1 if dt == 1 else 2) in (128, 256, 512)
+        assert info["block_k"] * (1 if dt in (1, 2) else 2) in (128, 256, 512)
         assert info["mma_n"] == info["block_n"] and info["block_n"] % 32 == 0
         assert info["smem_bytes"] <= 232448
         assert info["tmem_columns"] <= 512
@@ -164,3 +165,63 @@ def test_splitk_research_plan_arguments():
     assert lib.bi_gemm_run_splitk(h2, 2, 16, 7168, 16, 7168, 16, 4096, None, 0, None) == S["BI_ERR_INVALID_ARG"]
     need = bg.bi_gemm_splitk_workspace_bytes(plan, 2)
     assert lib.bi_gemm_run_splitk(h2, 2, 16, 7168, 16, 7168, 16, 4096, 16, need - 4, None) == S["BI_ERR_INVALID_ARG"]
+
+
+def test_w4a8_plan_and_argument_checks():
+    lib = binding.load_library()
+    S = binding.STATUS
+    W4 = bg.BI_DTYPE_E2M1_W4A8
+    # K must be a multiple of 128; no grouped e2m1 plan
+    for args in [(64, 200, W4, 1), (64, 64, W4, 1), (64, 128, W4, 4)]:
+        with pytest.raises(bg.BiGemmError) as e:
+            bg.bi_gemm_plan(*args)
+        assert e.value.name == "BI_ERR_UNSUPPORTED_SHAPE", args
+    plan = bg.bi_gemm_plan(7168, 7168, W4)
+    info = bg.bi_gemm_plan_describe(plan)
+    fp8 = bg.bi_gemm_plan_describe(bg.bi_gemm_plan(7168, 7168, bg.BI_DTYPE_E4M3_BLOCKSCALED))
+    # the e2m1 plan uses the FP8 tile and MMA shape (kind::f8f6f4, K = 32 per instruction)
+    for key in ("block_m", "block_n", "block_k", "cta_group", "mma_m", "mma_n", "mma_k", "stages",
+                "stages_a", "k_order_id", "tmem_columns"):
+        assert info[key] == fp8[key], key
+    assert info["dtype"] == W4 and info["cta_group"] == 1
+    assert bg.bi_gemm_w4a8_workspace_bytes(0) == 0
+    assert bg.bi_gemm_w4a8_workspace_bytes(5) == 256
+    assert bg.bi_gemm_w4a8_workspace_bytes(100) == 512
+    h = plan.handle
+    K = N = 7168
+    ws = bg.bi_gemm_w4a8_workspace_bytes(4)
+    run = lib.bi_gemm_run_w4a8
+    # (plan, M, A, lda, scale_a, ld_sa, W, ldw, w_scale, w_zero, workspace, bytes, C, ldc, stream)
+    ok = (h, 4, 256, K, 256, 4, 256, K, 256, 256, 256, ws, 256, N, None)
+
+    def call(**kw):
+        a = list(ok)
+        names = ["plan", "M", "A", "lda", "sa", "ld_sa", "W", "ldw", "ws", "wz", "work", "nbytes", "C",
+                 "ldc", "stream"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return run(*a)
+
+    assert call(plan=None) == S["BI_ERR_INVALID_ARG"]
+    assert call(M=-1) == S["BI_ERR_INVALID_ARG"]
+    assert call(M=0) == 0
+    assert call(sa=None) == S["BI_ERR_INVALID_ARG"]
+    assert call(ws=None) == S["BI_ERR_INVALID_ARG"]
+    assert call(ld_sa=3) == S["BI_ERR_INVALID_ARG"]
+    assert call(W=272) == S["BI_ERR_ALIGNMENT"]           # not 32-byte aligned
+    assert call(ldw=K + 32) == S["BI_ERR_ALIGNMENT"]      # row pitch of 3600 bytes: not 32-byte
+    assert call(ldw=K - 64) == S["BI_ERR_INVALID_ARG"]    # below K
+    assert call(A=264) == S["BI_ERR_ALIGNMENT"]
+    assert call(ws=258) == S["BI_ERR_ALIGNMENT"]
+    assert call(work=None) == S["BI_ERR_INVALID_ARG"]     # zero points need the row-sum workspace
+    assert call(nbytes=ws - 4) == S["BI_ERR_INVALID_ARG"]
+    assert call(work=264) == S["BI_ERR_ALIGNMENT"]
+    # the dtypes do not cross: bi_gemm_run refuses an e2m1 plan, bi_gemm_run_w4a8 other plans
+    assert lib.bi_gemm_run(h, 4, 256, K, 256, K, 256, N, 256, 4, 256, None) == S["BI_ERR_DTYPE_MISMATCH"]
+    f8 = bg.bi_gemm_plan(7168, 7168, bg.BI_DTYPE_E4M3_BLOCKSCALED)
+    assert call(plan=f8.handle) == S["BI_ERR_DTYPE_MISMATCH"]
+    assert lib.bi_gemm_run_host(h, 4, 256, K, 256, K, 256, N, 256, 4, 256, 256, 256, 256, None) == \
+        S["BI_ERR_DTYPE_MISMATCH"]
+    if not __import__("torch").cuda.is_available():
+        assert call() == S["BI_ERR_NO_DEVICE"]
+        assert call(wz=None, work=None, nbytes=0) == S["BI_ERR_NO_DEVICE"]
