@@ -180,9 +180,9 @@ bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows,
  * computed as: the MMA takes the e2m1 codes directly (tcgen05 kind::f8f6f4), each 128-wide K
  * block's partial product is promoted with scale_a alone in ascending kb (acc = fma(P_kb,
  * scale_a[m,kb], acc)), and the column's constants are applied once at the end:
- * C = fma(w_zero[n], rowsum[m], w_scale[n] * acc), with rowsum[m] = sum_k a[m][k] (fixed order:
- * per 128-block, then ascending kb).  A power-of-two scale multiplies exactly, so it can leave the
- * K sum.  The bits of C[m, :] depend on row m of A and scale_a, W and the column constants only.
+ * C = fma(w_zero[n], rowsum[m], w_scale[n] * acc), with rowsum[m] = sum_k a[m][k] in fp32 in an
+ * order fixed by K (32 interleaved slices, each accumulated over kb ascending, then a fixed tree).
+ * A power-of-two scale multiplies exactly, so it can leave the K sum.  The bits of C[m, :] depend on row m of A and scale_a, W and the column constants only.
  *
  * Device pointers:
  *   A        e4m3 [M][lda] (lda >= K, 16-byte aligned rows)

@@ -1090,20 +1090,23 @@ bi_status_t bi_gemm_run_w4a8(bi_plan_t plan, int64_t M, const void *A, int64_t l
     p.w_zero = w_zero;
     p.w_rowsum = w_zero ? workspace : nullptr;
     if (w_zero) {
-        // the row sums of the dequantised A, for the zero-point term (one CTA per row); the
-        // GEMM reads them after this grid has completed (it is this kernel's programmatic
-        // dependent and waits for it before touching global memory)
+        // the row sums of the dequantised A, for the zero-point term: one CTA per row for a few
+        // rows, one warp per row once there are enough rows to fill the device (the two compute
+        // the same bits).  The GEMM reads them after this grid has completed: it is this
+        // kernel's programmatic dependent and waits for it before touching global memory.
+        const bool warp_per_row = M > 1024;
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.gridDim = dim3(static_cast<unsigned>(M));
+        cfg.gridDim = dim3(static_cast<unsigned>(warp_per_row ? (M + 7) / 8 : M));
         cfg.blockDim = dim3(256);
         cfg.stream = stream;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, bi::bi_w4_rowsum_kernel, static_cast<const uint8_t *>(A), lda,
-                               scale_a, ld_sa, static_cast<int32_t>(M), static_cast<int32_t>(plan->k),
+        if (cudaLaunchKernelEx(&cfg, warp_per_row ? bi::bi_w4_rowsum_warp_kernel : bi::bi_w4_rowsum_kernel,
+                               static_cast<const uint8_t *>(A), lda, scale_a, ld_sa,
+                               static_cast<int32_t>(M), static_cast<int32_t>(plan->k),
                                workspace) != cudaSuccess)
             return BI_ERR_CUDA;
     }

@@ -351,19 +351,78 @@ __device__ __forceinline__ void w4_finish(const GemmParams &p, const W4Consts<kL
     }
 }
 
-// e2m1 weights with zero points: rowsum[m] = the sum over the K chunks kb (ascending) of
-// scale_a[m,kb] * t[m,kb], in fp32, where t[m,kb] is the sum of row m's 128 e4m3 values of chunk
-// kb: lane l of a warp adds the values 4l .. 4l+3 in order and the warp adds the 32 lane sums in a
-// fixed butterfly.  One CTA per row: its warps take the chunks in turn and one thread then runs
-// the chain r = fma(t, scale_a, r).  The order is fixed by K alone, so rowsum[m] depends on row m
-// only.  K is a multiple of 128.
+// e2m1 weights with zero points: rowsum[m] = sum_k a[m][k] in fp32, in an order fixed by K alone
+// (so rowsum[m] depends on row m only).  Lane l of a 32-lane group owns the values 4l .. 4l+3 of
+// every 128-value K chunk kb: it adds the four e4m3 values of its slice of the chunk in order,
+// p = ((v0 + v1) + v2) + v3, and accumulates r_l = fma(p, scale_a[m,kb], r_l) over kb ascending;
+// the 32 lane sums are then added in a fixed butterfly.  The two kernels below split the work
+// differently and compute the same bits.  K is a multiple of 128.
+__device__ __forceinline__ float e4m3x4_sum(uint32_t w)
+{
+    float t = 0.0f;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        __nv_fp8_e4m3 q;
+        q.__x = static_cast<__nv_fp8_storage_t>((w >> (8 * b)) & 0xFFu);
+        t += static_cast<float>(q);
+    }
+    return t;
+}
+
+__device__ __forceinline__ float lane_butterfly_sum(float r)
+{
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1)
+        r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
+    return r;
+}
+
+// Many rows: one warp per row (8 rows per CTA), 16 chunks in flight per batch.
+__global__ void __launch_bounds__(256) bi_w4_rowsum_warp_kernel(const uint8_t *a, int64_t lda,
+                                                                const float *scale_a, int64_t ld_sa,
+                                                                int32_t m_rows, int32_t k, float *rowsum)
+{
+    constexpr int kBatch = 16;
+    ptx::grid_dependency_wait();
+    if (threadIdx.x == 0)
+        ptx::launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (row >= m_rows)
+        return;
+    const uint8_t *arow = a + row * lda;
+    const int nkb = k / 128;
+    float r = 0.0f;
+    for (int c0 = 0; c0 < nkb; c0 += kBatch) {
+        uint32_t wv[kBatch];
+        float sv[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            const bool ok = c0 + i < nkb;
+            wv[i] = ok ? __ldg(reinterpret_cast<const uint32_t *>(arow + static_cast<int64_t>(c0 + i) * 128) + lane)
+                       : 0u;
+            sv[i] = ok ? __ldg(scale_a + static_cast<int64_t>(c0 + i) * ld_sa + row) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i)
+            if (c0 + i < nkb)
+                r = fmaf(e4m3x4_sum(wv[i]), sv[i], r);
+    }
+    r = lane_butterfly_sum(r);
+    if (lane == 0)
+        rowsum[row] = r;
+}
+
+// Few rows: one CTA per row.  Its 8 warps take the chunks in turn and leave each lane's slice sum
+// in shared memory; warp 0 then runs the 32 per-lane chains in kb order.
 __global__ void __launch_bounds__(256) bi_w4_rowsum_kernel(const uint8_t *a, int64_t lda,
                                                            const float *scale_a, int64_t ld_sa,
                                                            int32_t m_rows, int32_t k, float *rowsum)
 {
-    constexpr int kSeg = 256;   // chunks per pass through shared memory
+    constexpr int kSeg = 128;   // chunks per pass through shared memory
     constexpr int kWarps = 8;
-    __shared__ float s_t[kSeg], s_s[kSeg];
+    __shared__ float s_p[kSeg][32];
+    __shared__ float s_s[kSeg];
     ptx::grid_dependency_wait();
     if (threadIdx.x == 0)
         ptx::launch_dependents();
@@ -386,35 +445,28 @@ __global__ void __launch_bounds__(256) bi_w4_rowsum_kernel(const uint8_t *a, int
                             ? __ldg(reinterpret_cast<const uint32_t *>(arow + static_cast<int64_t>(kb0 + c) * 128) + lane)
                             : 0u;
             }
+            // lane i < 8 loads the scale of this warp's i-th chunk
+            const int ci = c0 + lane * kWarps;
+            if (lane < 8 && ci < nseg)
+                s_s[ci] = __ldg(scale_a + static_cast<int64_t>(kb0 + ci) * ld_sa + row);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int c = c0 + i * kWarps;
-                if (c >= nseg)
-                    break;
-                float t = 0.0f;
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    __nv_fp8_e4m3 q;
-                    q.__x = static_cast<__nv_fp8_storage_t>((wv[i] >> (8 * b)) & 0xFFu);
-                    t += static_cast<float>(q);
-                }
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1)
-                    t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
-                if (lane == 0) {
-                    s_t[c] = t;
-                    s_s[c] = __ldg(scale_a + static_cast<int64_t>(kb0 + c) * ld_sa + row);
-                }
+                if (c < nseg)
+                    s_p[c][lane] = e4m3x4_sum(wv[i]);
             }
         }
         __syncthreads();
-        if (threadIdx.x == 0)
+        if (warp == 0)
             for (int c = 0; c < nseg; ++c)
-                r = fmaf(s_t[c], s_s[c], r);
+                r = fmaf(s_p[c][lane], s_s[c], r);
         __syncthreads();
     }
-    if (threadIdx.x == 0)
-        rowsum[row] = r;
+    if (warp == 0) {
+        r = lane_butterfly_sum(r);
+        if (lane == 0)
+            rowsum[row] = r;
+    }
 }
 
 // BN      : output columns per tile (multiple of 32, <= 256; FP8 <= 128)
