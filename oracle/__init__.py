@@ -9,6 +9,8 @@ from .oracle import (  # noqa: F401
     e2m1_to_f64,
     e4m3_to_f64,
     f64_to_bf16,
+    f64_to_e2m1,
+    fp16_to_f64,
     gemm_bf16,
     gemm_bf16_rows,
     gemm_fp8_blockscaled,
@@ -16,5 +18,6 @@ from .oracle import (  # noqa: F401
     gemm_w4a8,
     gemm_w4a8_rows,
     grouped_gemm_bf16,
+    quantize_e2m1,
 )
 from . import attention, moe  # noqa: F401,E402

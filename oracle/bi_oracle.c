@@ -22,6 +22,10 @@
  *     channel), the activations as in the FP8 GEMM (per 1x128 K-block scales); then the dense
  *     GEMM above.  Every dequantised weight is exact in fp64 (a 2-bit significand times a power
  *     of two plus an 11-bit one, spanning at most 2^15 .. 2^-24).
+ *   e2m1 weight quantisation, the same section's W_fp4 = round((W - zero) / scale): x is formed
+ *     in fp64 from the 16-bit weight (bf16 or fp16), the zero point and the scale, and rounded to
+ *     the nearest e2m1 value, ties to the even fraction bit (the IEEE default the pages fix for
+ *     their GEMM, wmrh.cn article section 3.1); values beyond +-6 saturate to +-6, NaN gives +0.
  *   Grouped (MoE) GEMM: for expert e and every row r in [offsets[e], offsets[e+1]),
  *     C[r][n] = sum_k A[r][k] * B_e[n][k].  MoE is listed among the V4 components in
  *     "DeepSeek不惜代价保住它！V4关键特性被挖出来了" (QbitAI), section "什么是batch invariance".
@@ -35,6 +39,8 @@
  *   bf16  = 1 sign bit, 8 exponent bits (bias 127), 7 fraction bits (upper half of binary32).
  *   e4m3  = 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits; exponent field 0 is
  *           subnormal (value = fraction * 2^-9); S.1111.111 is NaN; no infinities; max 448.
+ *   fp16  = 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits; exponent field 0 is
+ *           subnormal (value = fraction * 2^-24); exponent field 31 is infinity or NaN.
  *   e2m1  = 1 sign bit, 2 exponent bits (bias 1), 1 fraction bit; exponent field 0 is
  *           subnormal (value = fraction * 2^-1); no infinities or NaN; max 6.  Packed two per
  *           byte, value k of a row in byte k/2, the even k in the low four bits.
@@ -100,6 +106,44 @@ double oracle_e2m1_to_f64(uint8_t code)
     else
         v = ldexp((double)(2 + frac), expo - 1 - 1);   /* 1.frac * 2^(e-1) */
     return sign ? -v : v;
+}
+
+/* fp16 bit pattern -> exact fp64 value. */
+double oracle_fp16_to_f64(uint16_t bits)
+{
+    int sign = (bits >> 15) & 1;
+    int expo = (bits >> 10) & 0x1F;
+    int frac = bits & 0x3FF;
+    double v;
+    if (expo == 0x1F)
+        v = frac ? NAN : INFINITY;
+    else if (expo == 0)
+        v = ldexp((double)frac, -24);                  /* 0.frac * 2^-14 */
+    else
+        v = ldexp((double)(1024 + frac), expo - 15 - 10);   /* 1.frac * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/* fp64 -> e2m1 4-bit code: round to nearest, ties to the even fraction bit, saturating at +-6;
+ * NaN gives +0.  The e2m1 values in [0, 2) are 0.5 apart, in [2, 4) 1 apart and in [4, 8) 2
+ * apart (6 being the largest); the sign bit follows the sign of x, so a negative x that rounds to
+ * zero gives -0. */
+uint8_t oracle_f64_to_e2m1(double x)
+{
+    if (isnan(x))
+        return 0;
+    uint8_t sign = signbit(x) ? 8 : 0;
+    double a = fabs(x);
+    double q = a < 2.0 ? 0.5 : (a < 4.0 ? 1.0 : 2.0);   /* spacing in a's binade */
+    double v = nearbyint(a / q) * q;                      /* ties to an even multiple of q */
+    if (v > 6.0)
+        v = 6.0;
+    static const double values[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    uint8_t code = 0;
+    for (uint8_t c = 0; c < 8; ++c)
+        if (values[c] == v)
+            code = c;
+    return (uint8_t)(sign | code);
 }
 
 /* fp64 -> bf16 bit pattern, round to nearest, ties to even; overflow goes to +-inf,
@@ -304,6 +348,26 @@ int oracle_gemm_w4a8(int64_t M, int64_t N, int64_t K, const uint8_t *QA, const f
     free(a);
     free(b);
     return rc;
+}
+
+/* e2m1 quantisation of 16-bit weights W [N][K] (bf16 bits, or fp16 bits when is_fp16):
+ *   q[n][k] = e2m1_rne((W[n][k] - WZ[n]) / WS[n])   (WZ may be NULL: zero points 0)
+ * written packed, Q [N][K/2] bytes, value k in byte k/2, the even k in the low four bits.  K must
+ * be even. */
+void oracle_quantize_e2m1(int64_t N, int64_t K, const uint16_t *W, int is_fp16, const float *WS,
+                          const float *WZ, uint8_t *Q)
+{
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; k += 2) {
+            uint8_t code[2];
+            for (int h = 0; h < 2; ++h) {
+                uint16_t bits = W[n * K + k + h];
+                double w = is_fp16 ? oracle_fp16_to_f64(bits) : oracle_bf16_to_f64(bits);
+                double z = WZ ? (double)WZ[n] : 0.0;
+                code[h] = oracle_f64_to_e2m1((w - z) / (double)WS[n]);
+            }
+            Q[n * (K / 2) + k / 2] = (uint8_t)(code[0] | (code[1] << 4));
+        }
 }
 
 /* Grouped bf16 (MoE):  A [R][K] rows grouped by expert, B [E][N][K], offsets [E+1] with

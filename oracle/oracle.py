@@ -51,6 +51,12 @@ class OracleLib:
         lib.oracle_gemm_fp8_blockscaled.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, i32]
         lib.oracle_e2m1_to_f64.restype = ctypes.c_double
         lib.oracle_e2m1_to_f64.argtypes = [ctypes.c_uint8]
+        lib.oracle_fp16_to_f64.restype = ctypes.c_double
+        lib.oracle_fp16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.oracle_f64_to_e2m1.restype = ctypes.c_uint8
+        lib.oracle_f64_to_e2m1.argtypes = [ctypes.c_double]
+        lib.oracle_quantize_e2m1.restype = None
+        lib.oracle_quantize_e2m1.argtypes = [i64, i64, vp, i32, vp, vp, vp]
         lib.oracle_gemm_w4a8.restype = i32
         lib.oracle_gemm_w4a8.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, i32]
         lib.oracle_grouped_gemm_bf16.restype = i32
@@ -125,6 +131,42 @@ def e2m1_to_f64(codes, lib=None) -> np.ndarray:
     for i in range(flat.size):
         oflat[i] = lib.oracle_e2m1_to_f64(int(flat[i]))
     return out
+
+
+def fp16_to_f64(bits, lib=None) -> np.ndarray:
+    """fp16 bit patterns -> exact fp64 values (oracle codec)."""
+    lib = lib or _lib()
+    b = np.asarray(bits, dtype=np.uint16)
+    out = np.empty(b.shape, dtype=np.float64)
+    flat, oflat = b.reshape(-1), out.reshape(-1)
+    for i in range(flat.size):
+        oflat[i] = lib.oracle_fp16_to_f64(int(flat[i]))
+    return out
+
+
+def f64_to_e2m1(x, lib=None) -> np.ndarray:
+    """fp64 values -> e2m1 codes (round to nearest even, saturating at +-6, NaN -> +0)."""
+    lib = lib or _lib()
+    v = np.asarray(x, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint8)
+    flat, oflat = v.reshape(-1), out.reshape(-1)
+    for i in range(flat.size):
+        oflat[i] = lib.oracle_f64_to_e2m1(float(flat[i]))
+    return out
+
+
+def quantize_e2m1(W_bits, w_scale, w_zero=None, fp16: bool = False, lib=None) -> np.ndarray:
+    """Quantise 16-bit weights [N, K] (bf16 bits, or fp16 bits with fp16=True) to packed e2m1
+    codes [N, K/2]: q = round_to_nearest_even((W - zero) / scale), saturating at +-6."""
+    W = _c(W_bits, np.uint16)
+    N, K = W.shape
+    assert K % 2 == 0
+    WS = _c(w_scale, np.float32).reshape(N)
+    WZ = None if w_zero is None else _c(w_zero, np.float32).reshape(N)
+    Q = np.empty((N, K // 2), dtype=np.uint8)
+    (lib or _lib()).oracle_quantize_e2m1(N, K, _ptr(W), 1 if fp16 else 0, _ptr(WS),
+                                         None if WZ is None else _ptr(WZ), _ptr(Q))
+    return Q
 
 
 def f64_to_bf16(x, lib=None) -> np.ndarray:

@@ -129,3 +129,14 @@ def w4a8_cases():
         case["qa"] = qa
         case["qw"] = pack_e2m1(codes)
         yield case
+
+
+def e2m1_rounding_cases():
+    """Yield (x as float, expected code, reason) from e2m1_rounding.txt."""
+    for line in _lines("e2m1_rounding.txt"):
+        m, e, code, *reason = line.split()
+        if m in ("nan", "inf", "-inf"):
+            x = float(m)
+        else:
+            x = float(Fraction(int(m)) * Fraction(2) ** int(e))
+        yield x, int(code, 16), " ".join(reason)

@@ -43,12 +43,24 @@ MUTANTS = {
     "e2m1 nibbles swapped": ("(k % 2 == 0) ? (uint8_t)(byte & 0xF) : (uint8_t)(byte >> 4)",
                              "(k % 2 == 1) ? (uint8_t)(byte & 0xF) : (uint8_t)(byte >> 4)"),
     "e2m1 bias 2": ("ldexp((double)(2 + frac), expo - 1 - 1)", "ldexp((double)(2 + frac), expo - 2 - 1)"),
-    "e2m1 sign ignored": ("    return sign ? -v : v;\n}\n\n/* fp64 -> bf16",
-                          "    return v;\n}\n\n/* fp64 -> bf16"),
+    "e2m1 sign ignored": ("    return sign ? -v : v;\n}\n\n/* fp16 bit pattern",
+                          "    return v;\n}\n\n/* fp16 bit pattern"),
+    "fp16 sign ignored": ("    return sign ? -v : v;\n}\n\n/* fp64 -> e2m1",
+                          "    return v;\n}\n\n/* fp64 -> e2m1"),
     "e2m1 zero point scaled": ("w += (double)WZ[n];", "w += (double)WZ[n] * (double)WS[n];"),
     "e2m1 zero point ignored": ("w += (double)WZ[n];", "w += 0.0;"),
     "e2m1 scale of channel 0": ("oracle_e2m1_to_f64(code) * (double)WS[n]",
                                 "oracle_e2m1_to_f64(code) * (double)WS[0]"),
+    "e2m1 rounding ties away from zero": ("double v = nearbyint(a / q) * q;", "double v = round(a / q) * q;"),
+    "e2m1 rounding truncates": ("double v = nearbyint(a / q) * q;", "double v = floor(a / q) * q;"),
+    "e2m1 no saturation": ("    if (v > 6.0)\n        v = 6.0;\n", ""),
+    "e2m1 rounding drops the sign": ("uint8_t sign = signbit(x) ? 8 : 0;", "uint8_t sign = 0;"),
+    "quantise ignores the zero point": ("double z = WZ ? (double)WZ[n] : 0.0;", "double z = 0.0;"),
+    "quantise multiplies by the scale": ("code[h] = oracle_f64_to_e2m1((w - z) / (double)WS[n]);",
+                                         "code[h] = oracle_f64_to_e2m1((w - z) * (double)WS[n]);"),
+    "quantise packs high nibble first": ("(uint8_t)(code[0] | (code[1] << 4))",
+                                         "(uint8_t)(code[1] | (code[0] << 4))"),
+    "fp16 bias 16": ("ldexp((double)(1024 + frac), expo - 15 - 10)", "ldexp((double)(1024 + frac), expo - 16 - 10)"),
     "grouped rows use expert 0": ("row_b[r] = e * N * K;", "row_b[r] = 0;"),
     "grouped rows use the next expert": ("row_b[r] = e * N * K;",
                                          "row_b[r] = ((e + 1) % E) * N * K;"),
@@ -164,6 +176,21 @@ def battery(lib):
     cref, _ = oracle.gemm_w4a8(qa, sa, np.zeros((3, 64), np.uint8), ws, wz, lib=lib)
     rs = (e4m3_values(qa) * sa.astype(np.float64)).sum(axis=1)
     check("w4a8 zero-point closed form", np.array_equal(cref, np.outer(rs, wz.astype(np.float64))))
+
+    # e2m1 rounding golden cases, fp16 decode, and a quantisation worked by hand
+    ok = all(int(oracle.f64_to_e2m1([x], lib=lib)[0]) == c for x, c, _ in golden_io.e2m1_rounding_cases())
+    check("e2m1 rounding golden", ok)
+    hb = np.arange(0, 1 << 16, 61, dtype=np.uint32).astype(np.uint16)
+    hv = hb.view(np.float16).astype(np.float64)
+    hg = oracle.fp16_to_f64(hb, lib=lib)
+    fin = np.isfinite(hv)
+    check("fp16 decode vs numpy", np.array_equal(hg[fin], hv[fin]))
+    Wq = np.array([[2.0, -0.25, 0.5, 1.875], [0.25, 0.375, -1.0, 8.0]], np.float32)
+    bq = torch.from_numpy(Wq).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.quantize_e2m1(bq, np.array([0.25, 0.5], np.float32), np.array([0.5, 0.0], np.float32),
+                               lib=lib)
+    want = golden_io.pack_e2m1(np.array([[0x7, 0xD, 0x0, 0x7], [0x1, 0x2, 0xC, 0x7]], np.uint8))
+    check("quantise worked case", np.array_equal(got, want))
 
     # grouped: integer data, distinct experts, one empty
     E, N, K = 3, 4, 8

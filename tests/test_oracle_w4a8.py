@@ -130,3 +130,79 @@ def test_w4a8_brute_force_exact_rationals():
                 q += av * wv
             assert abs(Fraction(float(cref[m, n])) - q) <= abs(q) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 80)
             assert cbits[m, n] == exact.rne_bf16(q), (m, n)
+
+
+# ---------------------------------------------------------------------------------------------
+# e2m1 quantisation of 16-bit weights: W_fp4 = round((W - zero) / scale)
+# ---------------------------------------------------------------------------------------------
+
+def test_e2m1_rounding_golden_cases():
+    n = 0
+    for x, code, why in golden_io.e2m1_rounding_cases():
+        assert int(oracle.f64_to_e2m1([x])[0]) == code, (x, why)
+        n += 1
+    assert n >= 15
+
+
+def test_e2m1_rounding_round_trips_every_value():
+    vals = [float(v) if not neg else -0.0 for _, (v, neg) in sorted(E2M1_TABLE.items())]
+    codes = oracle.f64_to_e2m1(vals)
+    assert list(codes) == list(range(16))
+
+
+def test_e2m1_rounding_is_nearest_with_ties_to_even_brute_force():
+    rng = np.random.default_rng(641)
+    xs = list(rng.uniform(-9, 9, 400))
+    # every midpoint between neighbouring values, and both of its neighbours in binary64
+    mags = [float(E2M1_TABLE[c][0]) for c in range(8)]
+    for a, b in zip(mags, mags[1:]):
+        mid = (a + b) / 2
+        xs += [mid, np.nextafter(mid, 0), np.nextafter(mid, 9), -mid]
+    got = oracle.f64_to_e2m1(xs)
+    for x, c in zip(xs, got):
+        fx = Fraction(float(x))
+        cands = sorted(range(8), key=lambda cc: (abs(abs(fx) - E2M1_TABLE[cc][0]), cc & 1))
+        want = cands[0] if abs(fx) <= 6 else 7
+        if fx < 0 or (fx == 0 and np.signbit(x)):
+            want |= 8
+        assert int(c) == want, (x, int(c), want)
+
+
+def test_fp16_decode_exhaustive_vs_numpy_bit_view():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    want = bits.view(np.float16).astype(np.float64)
+    got = oracle.fp16_to_f64(bits)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(want[~nan]))
+
+
+def test_quantize_applies_zero_then_scale_and_packs_low_nibble_first():
+    # row 0: scale 2^-2, zero 0.5: (W - 0.5) * 4 for W = [2, -0.25, 0.5, 1.875] -> [6, -3, 0, 5.5]
+    #   -> codes [0x7, 0xD, 0x0, 0x7 (5.5 is nearer 6)]
+    # row 1: scale 2^-1, no zero point effect (zero 0): W = [0.25, 0.375, -1, 8] -> [0.5, 0.75, -2, 16]
+    #   -> codes [0x1, 0x2 (tie -> 1), 0xC, 0x7]
+    W = np.array([[2.0, -0.25, 0.5, 1.875], [0.25, 0.375, -1.0, 8.0]], np.float32)
+    ws = np.array([0.25, 0.5], np.float32)
+    wz = np.array([0.5, 0.0], np.float32)
+    want = golden_io.pack_e2m1(np.array([[0x7, 0xD, 0x0, 0x7], [0x1, 0x2, 0xC, 0x7]], np.uint8))
+    bf = torch.from_numpy(W).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.quantize_e2m1(bf, ws, wz), want)
+    hf = W.astype(np.float16).view(np.uint16)
+    assert np.array_equal(oracle.quantize_e2m1(hf, ws, wz, fp16=True), want)
+
+
+def test_quantize_then_gemm_reproduces_exactly_representable_weights():
+    # weights that are e2m1 values times the channel scale plus its zero point quantise to those
+    # values, so quantise -> W4A8 GEMM equals the W4A8 GEMM of the original codes
+    N, K = 20, 256
+    codes = np.random.default_rng(651).integers(0, 16, (N, K)).astype(np.uint8)
+    ws = np.exp2(-np.random.default_rng(652).integers(1, 5, N)).astype(np.float32)
+    wz = (np.random.default_rng(653).integers(-8, 9, N) * 2.0 ** -3).astype(np.float32)
+    w = table_values(codes) * ws[:, None].astype(np.float64) + wz[:, None].astype(np.float64)
+    bf = torch.from_numpy(w.astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(bf.to(torch.float64).numpy(), w)        # exact in bf16
+    q = oracle.quantize_e2m1(bf.view(torch.int16).numpy().view(np.uint16), ws, wz)
+    vals = table_values(unpack(q))
+    assert np.array_equal(vals, table_values(codes))              # -0 and +0 both decode to 0
