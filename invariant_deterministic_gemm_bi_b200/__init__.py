@@ -1,11 +1,12 @@
 """Batch-invariant GEMM for NVIDIA B200 (sm_100a).
 
 C[M,N] = A[M,K] . B[N,K]^T with fp32 accumulation and bf16 output, computed by hand-written
-tcgen05/TMA kernels behind the C ABI in ``include/bi_gemm.h`` (bf16, FP8 e4m3 with block scales,
-and e2m1 weights with per-channel power-of-two scales and zero points x e4m3 activations); the MoE routing, dispatch, gather
-and combine steps around the grouped GEMM are in ``include/bi_moe.h``, and the dual-kernel
-decode attention in ``include/bi_attention.h``.  Every output row is
-bit-identical whatever the batch size, the row's position and the other rows in the batch.
+tcgen05/TMA kernels behind the C ABI in ``include/bi_gemm.h``: bf16, FP8 e4m3 with block scales,
+and e2m1 weights (per-channel power-of-two scale and zero point) x e4m3 activations.  The MoE
+routing, dispatch, gather and combine steps around the grouped GEMM are in ``include/bi_moe.h``,
+the dual-kernel decode attention in ``include/bi_attention.h``, and the e2m1 weight quantisation
+in ``include/bi_quantize.h``.  Every output row is bit-identical whatever the batch size, the
+row's position and the other rows in the batch.
 
 ``binding`` holds the ctypes wrapper (same names as the C ABI); ``inputs`` the seeded synthetic
 input generators; ``build`` the nvcc build of ``libbigemm.so``.
@@ -41,6 +42,7 @@ from .binding import (  # noqa: F401
     bi_moe_dispatch,
     bi_moe_gather_rows,
     bi_moe_route_topk,
+    bi_quantize_e2m1,
     bi_status_string,
     load_library,
 )

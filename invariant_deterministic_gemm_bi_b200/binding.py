@@ -1,5 +1,5 @@
-"""Thin ctypes binding of libbigemm (include/bi_gemm.h, bi_moe.h, bi_attention.h), same names as
-the C ABI.
+"""Thin ctypes binding of libbigemm (include/bi_gemm.h, bi_moe.h, bi_attention.h, bi_quantize.h),
+same names as the C ABI.
 
 Argument marshalling only: every function takes torch tensors (device memory owned by torch)
 or raw integers, passes their pointers, strides and the current CUDA stream to the C entry
@@ -39,6 +39,7 @@ EXPORTED = [
     "bi_gemm_w4a8_workspace_bytes", "bi_gemm_run_w4a8",
     "bi_moe_route_topk", "bi_moe_dispatch", "bi_moe_gather_rows", "bi_moe_combine",
     "bi_decode_attention", "bi_decode_attention_workspace_bytes",
+    "bi_quantize_e2m1",
 ]
 
 
@@ -127,6 +128,8 @@ def load_library(path: str = LIB_PATH):
     lib.bi_decode_attention.restype = i32
     lib.bi_decode_attention.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i64, ctypes.c_float, i32,
                                         vp, ctypes.c_size_t, vp, vp]
+    lib.bi_quantize_e2m1.restype = i32
+    lib.bi_quantize_e2m1.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, i64, vp]
     if path == LIB_PATH:
         _LIB = lib
     return lib
@@ -380,3 +383,21 @@ def bi_decode_attention(Q, K, V, lengths, O, scale: float, splits: int = 1, work
                                               Lmax, scale, splits, _ptr(workspace), nbytes, _ptr(O),
                                               _stream_handle(stream)), "bi_decode_attention")
     return O
+
+
+# ---------------------------------------------------------------------------------------------
+# e2m1 weight quantisation (include/bi_quantize.h)
+# ---------------------------------------------------------------------------------------------
+
+def bi_quantize_e2m1(W, w_scale, Q, w_zero=None, stream=None):
+    """Packed e2m1 codes Q (uint8 [N, ldq/2]) of the bf16 or fp16 weights W [N, ldw]:
+    q = round_to_nearest_even((W - w_zero) / w_scale), saturating at +-6."""
+    import torch
+    if W.dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError("W must be bf16 or fp16")
+    N, K = W.shape
+    st = load_library().bi_quantize_e2m1(_ptr(W), 1 if W.dtype == torch.float16 else 0, W.stride(0), N, K,
+                                         _ptr(w_scale), _ptr(w_zero), _ptr(Q), Q.stride(0) * 2,
+                                         _stream_handle(stream))
+    _check(st, "bi_quantize_e2m1")
+    return Q

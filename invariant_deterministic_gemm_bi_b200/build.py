@@ -18,10 +18,11 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 REPO = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 SOURCES = [os.path.join(CSRC, "bi_gemm.cu"), os.path.join(CSRC, "bi_moe.cu"),
-           os.path.join(CSRC, "bi_attention.cu")]
+           os.path.join(CSRC, "bi_attention.cu"), os.path.join(CSRC, "bi_quantize.cu")]
 HEADERS = [os.path.join(CSRC, "bi_kernels.cuh"), os.path.join(CSRC, "bi_kernels_pair.cuh"),
            os.path.join(CSRC, "ptx_sm100.cuh"), os.path.join(REPO, "include", "bi_gemm.h"),
-           os.path.join(REPO, "include", "bi_moe.h"), os.path.join(REPO, "include", "bi_attention.h")]
+           os.path.join(REPO, "include", "bi_moe.h"), os.path.join(REPO, "include", "bi_attention.h"),
+           os.path.join(REPO, "include", "bi_quantize.h")]
 LIB = os.path.join(PKG, "libbigemm.so")
 
 NVCC_FLAGS = [

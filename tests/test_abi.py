@@ -225,3 +225,34 @@ def test_w4a8_plan_and_argument_checks():
     if not __import__("torch").cuda.is_available():
         assert call() == S["BI_ERR_NO_DEVICE"]
         assert call(wz=None, work=None, nbytes=0) == S["BI_ERR_NO_DEVICE"]
+
+
+def test_quantize_argument_checks():
+    lib = binding.load_library()
+    S = binding.STATUS
+    q = lib.bi_quantize_e2m1
+    # (W, is_fp16, ldw, N, K, w_scale, w_zero, Q, ldq, stream)
+    ok = [256, 0, 64, 4, 64, 256, 256, 256, 64, None]
+
+    def call(i=None, v=None):
+        a = list(ok)
+        if i is not None:
+            a[i] = v
+        return q(*a)
+
+    assert call(3, 0) == 0 and call(4, 0) == 0            # empty: no-op
+    assert call(3, -1) == S["BI_ERR_INVALID_ARG"]
+    assert call(4, 63) == S["BI_ERR_INVALID_ARG"]         # odd K
+    assert call(1, 2) == S["BI_ERR_INVALID_ARG"]          # neither bf16 nor fp16
+    assert call(0, None) == S["BI_ERR_INVALID_ARG"]
+    assert call(7, None) == S["BI_ERR_INVALID_ARG"]
+    assert call(5, None) == S["BI_ERR_INVALID_ARG"]
+    assert call(2, 32) == S["BI_ERR_INVALID_ARG"]         # ldw < K
+    assert call(8, 62) == S["BI_ERR_INVALID_ARG"]         # ldq < K
+    assert call(8, 65) == S["BI_ERR_INVALID_ARG"]         # odd ldq
+    assert call(0, 257) == S["BI_ERR_ALIGNMENT"]
+    assert call(5, 258) == S["BI_ERR_ALIGNMENT"]
+    assert call(6, 258) == S["BI_ERR_ALIGNMENT"]
+    if not __import__("torch").cuda.is_available():   # valid arguments: only without a GPU
+        assert call() == S["BI_ERR_NO_DEVICE"]
+        assert call(6, None) == S["BI_ERR_NO_DEVICE"]
