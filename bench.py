@@ -622,6 +622,14 @@ def measure_extras(bg, inputs, dev, stream, peaks):
             res[f"w4a8_M{M}_no_zero"] = {"us": t * 1e6, "TFLOP/s": 2 * M * N * K / t / 1e12,
                                          "GB/s": b / t / 1e9, "hbm_frac": b / t / 1e9 / hbm}
     del qws
+    # e2m1 quantisation of the bf16 weights of the same shape (a weight-preparation step)
+    Wb = inputs.bf16_gaussian((N, K), seed=6006, std=0.01, device=dev)
+    Qw = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    t = graph_time_per_launch([lambda: bg.bi_quantize_e2m1(Wb, ws, Qw, w_zero=wz, stream=stream)] * 4,
+                              stream, reps=4)
+    b = N * K * 2 + N * K // 2 + 8 * N
+    res["quantize_e2m1_7168x7168"] = {"us": t * 1e6, "GB/s": b / t / 1e9, "hbm_frac": b / t / 1e9 / hbm}
+    del Wb, Qw
     # MoE: 64 experts, N = 2048, K = 7168, top-8
     E, N, K = 64, 2048, 7168
     plan = weight_plan(N, K, bg.BI_DTYPE_BF16, E)

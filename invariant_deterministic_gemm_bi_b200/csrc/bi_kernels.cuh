@@ -23,6 +23,8 @@
 //                    K blocks ahead of the A loads of the same K block.
 //   warp 1         : allocates tensor memory; lane 0 issues tcgen05.mma and commits
 //   warps 2..5     : epilogue -- tcgen05.ld from TMEM, fp32 -> bf16 (RNE), masked stores
+//   (FP8 tiles at least 64 wide have 8 epilogue warps, 2..9; the dense wide lockstep form adds
+//   one more warp after the epilogue warps whose lane 0 issues the second column half's MMAs)
 // bf16: the accumulator is double-buffered in TMEM so the epilogue of tile i overlaps the
 // MMAs of tile i+1.  FP8 (e4m3, block scales): each 128-wide K block is accumulated by the MMA
 // into its own TMEM partial buffer (a ring of NPART), and the epilogue warps promote it into
@@ -61,6 +63,19 @@ struct Epi {
     static constexpr int kWarps = 4 * kHalves;
     static constexpr int kThreads = (2 + kWarps) * 32;
     static constexpr int kCols = BN / kHalves;             // columns per epilogue thread
+};
+
+// MMA-issuing threads of a kernel: one, or in the dense wide lockstep form (NSPLIT = 2) two --
+// each issues one column half's instruction chain.  A thread's next tcgen05.mma waits on the issue
+// of its previous one, which costs ~50 cycles beyond the instruction's math for these tile shapes;
+// two issuers overlap that cost.  The grouped wide form (two 128 x 128 instructions per K step) is
+// bound by shared-memory bandwidth instead and keeps one issuer.  The second issuer is the warp
+// after the epilogue warps.
+template <bool FP8, int BN, int NSPLIT, bool GROUPED = false>
+struct Issue {
+    static constexpr int kIssuers = GROUPED ? 1 : NSPLIT;
+    static constexpr int kSecondWarp = 2 + Epi<FP8, BN>::kWarps;
+    static constexpr int kThreads = Epi<FP8, BN>::kThreads + (kIssuers - 1) * 32;
 };
 constexpr int kMaxExperts = 1024;
 
@@ -377,8 +392,9 @@ __device__ __forceinline__ float lane_butterfly_sum(float r)
     return r;
 }
 
-// Many rows: one warp per row (8 rows per CTA), 16 chunks in flight per batch.
-__global__ void __launch_bounds__(256) bi_w4_rowsum_warp_kernel(const uint8_t *a, int64_t lda,
+// Many rows: one warp per row (8 rows per CTA), 16 chunks in flight per batch; 4 CTAs per SM
+// (at most 64 registers a thread) keep the rows of a 4096-row batch in one wave.
+__global__ void __launch_bounds__(256, 4) bi_w4_rowsum_warp_kernel(const uint8_t *a, int64_t lda,
                                                                 const float *scale_a, int64_t ld_sa,
                                                                 int32_t m_rows, int32_t k, float *rowsum)
 {
@@ -496,7 +512,7 @@ __global__ void __launch_bounds__(256) bi_w4_rowsum_kernel(const uint8_t *a, int
 // The ring depths follow from (BM, BN, KC) (see Rings).
 template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool SPLIT = false,
           bool W4 = false>
-__global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
+__global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED>::kThreads, 1)
     bi_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_a8, const GemmParams p)
@@ -513,6 +529,7 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     static_assert(!SPLIT || (!FP8 && !GROUPED && NSPLIT == 1), "split-K variant: bf16 dense");
     static_assert(!W4 || (FP8 && !GROUPED && !SPLIT), "e2m1 weights: the dense FP8 kernel");
     constexpr int kMmaN = BN / NSPLIT;                   // MMA instruction N
+    constexpr int kIssuers = Issue<FP8, BN, NSPLIT, GROUPED>::kIssuers;   // threads issuing MMAs
     using R = Rings<BM, BN, KC>;
     constexpr int kElemsPerRow = FP8 ? 128 : 64;         // K elements per 128-byte row
     constexpr int kMmaK = FP8 ? 32 : 16;                 // K per tcgen05.mma
@@ -553,8 +570,8 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     uint64_t *consumed = full + kMaxSB;
     uint64_t *accf_bar = consumed + kMaxSB;    // accumulator (or partial) full
     uint64_t *acce_bar = accf_bar + kNumAcc;   // accumulator (or partial) empty
-    uint64_t *drain_bar = acce_bar + kNumAcc;
-    uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(drain_bar + 1);
+    uint64_t *drain_bar = acce_bar + kNumAcc;  // one per MMA issuer
+    uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(drain_bar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
     int32_t *grp_prefix = reinterpret_cast<int32_t *>(tmem_base_smem + 4);   // [E+1]
     int32_t *grp_offs = grp_prefix + (GROUPED ? (kMaxExperts + 1) : 0);       // [E+1]
@@ -565,13 +582,14 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.sb; ++s) {   // only the ring slots this launch uses
             ptx::mbar_init(&full[s], 2);
-            ptx::mbar_init(&consumed[s], 1);
+            ptx::mbar_init(&consumed[s], kIssuers);   // one commit per issuer
         }
         for (int a = 0; a < kNumAcc; ++a) {
-            ptx::mbar_init(&accf_bar[a], 1);
+            ptx::mbar_init(&accf_bar[a], kIssuers);
             ptx::mbar_init(&acce_bar[a], Epi<FP8, BN>::kWarps * 32);
         }
-        ptx::mbar_init(drain_bar, 1);
+        for (int i = 0; i < kIssuers; ++i)
+            ptx::mbar_init(&drain_bar[i], 1);
         *abort_flag = 0;
         ptx::fence_mbarrier_init();
         ptx::prefetch_tmap(&tmap_a);
@@ -789,8 +807,13 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                                nullptr);
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || (kIssuers > 1 && warp == Issue<FP8, BN, NSPLIT, GROUPED>::kSecondWarp)) {
+        // ------------------------------------------------------------------ MMA issuers
+        // Issuer `iss` issues the MMAs of split iss (all splits with one issuer), for every K step
+        // of every tile in ascending order.  Both issuers wait on the same barriers, and each
+        // commits every group (the consumed and accumulator-full barriers count one commit per
+        // issuer), so a slot or an accumulator is handed on when both halves are done with it.
+        const int iss = warp == 1 ? 0 : 1;
         if (lane == 0) {
             const int SA = p.sa, SB = p.sb;
             int sa = 0, sb = 0;      // ring slots of the next group
@@ -870,8 +893,9 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                             // bf16: accumulate across the whole K of the tile; FP8: one K chunk
                             const uint32_t accumulate = (q > 0) ? 1u : (FP8 ? 0u : (chunk > 0 ? 1u : 0u));
 #pragma unroll
-                            for (int sp = 0; sp < NSPLIT; ++sp) {
+                            for (int j = 0; j < NSPLIT / kIssuers; ++j) {
                                 // split sp: B rows and accumulator columns [sp kMmaN, (sp+1) kMmaN)
+                                const int sp = j + iss;
                                 const uint64_t b_sp = static_cast<uint64_t>((sp * kMmaN * kRowBytes) >> 4);
                                 if constexpr (FP8)
                                     ptx::mma_e4m3_ss(d + sp * kMmaN, a_desc + step, b_desc + b_sp + step,
@@ -921,8 +945,8 @@ __global__ void __launch_bounds__(Epi<FP8, BN>::kThreads, 1)
                 }
             }
             // Drain: wait for every MMA this thread issued before tensor memory is freed.
-            ptx::mma_commit(drain_bar);
-            ptx::mbar_wait(drain_bar, 0, p.timeout_cycles, nullptr);
+            ptx::mma_commit(&drain_bar[iss]);
+            ptx::mbar_wait(&drain_bar[iss], 0, p.timeout_cycles, nullptr);
         }
     } else {
         // ------------------------------------------------------------------ epilogue warps

@@ -98,3 +98,31 @@ def test_quantised_weights_feed_the_w4a8_gemm():
     got = C.view(torch.int16).cpu().numpy().view(np.uint16)
     zero = ((got & 0x7FFF) == 0) & ((want & 0x7FFF) == 0)
     assert np.all((got == want) | zero)
+
+
+@pytest.mark.parametrize("fp16", [False, True])
+def test_vector_rows_with_a_ragged_tail(fp16):
+    # 16-byte-aligned rows (pitch 144 values) whose K = 138 leaves one code byte past the last
+    # whole 8-value group
+    N, K = 33, 138
+    dtype = torch.float16 if fp16 else torch.bfloat16
+    w, ws, wz = weights(N, K, seed=7300, dtype=dtype)
+    want = oracle_codes(w, ws, wz)
+    Wd = strided_rows(w.to(DEV), 144)
+    Q = torch.full((N, 72), 0xEE, dtype=torch.uint8, device=DEV)
+    bg.bi_quantize_e2m1(Wd, ws.to(DEV), Q[:, : K // 2], w_zero=wz.to(DEV))
+    got = Q.cpu().numpy()
+    assert np.array_equal(got[:, : K // 2], want), np.argwhere(got[:, : K // 2] != want)[:5]
+    assert np.all(got[:, K // 2:] == 0xEE)
+
+
+@pytest.mark.parametrize("N,K", [(64, 512), (21, 130)])
+def test_scales_that_are_not_powers_of_two(N, K):
+    # any non-zero fp32 scale is accepted: these divide in fp64 instead of multiplying by an exact
+    # reciprocal (512: the vector kernel; 130: the scalar one)
+    w, _, wz = weights(N, K, seed=7400 + K, dtype=torch.bfloat16)
+    ws = inputs.scales_log_uniform((N,), seed=7401) * 0.1
+    ws[0] = -0.3                                 # a negative scale flips the codes' signs
+    want = oracle_codes(w, ws, wz)
+    got = run(w, ws, wz)
+    assert np.array_equal(got[:, : K // 2], want), np.argwhere(got[:, : K // 2] != want)[:5]
