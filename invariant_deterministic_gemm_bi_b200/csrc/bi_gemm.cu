@@ -49,27 +49,27 @@ struct KernelEntry {
 };
 
 #define BI_ENTRY(BM, BN, KC, F8, GR)                                                               \
-    KernelEntry{bi::Epi<F8, BN>::kThreads, BM, BN, KC, F8, GR, false,                              \
+    KernelEntry{bi::Issue<F8, BN, 1, GR, KC>::kThreads, BM, BN, KC, F8, GR, false,                              \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, GR>,                                           \
                 bi::smem_bytes_for<BM, BN, KC, F8, GR>(), 1, false, false}
 #define BI_ENTRY_W4(BM, BN, KC)                                                                    \
-    KernelEntry{bi::Epi<true, BN>::kThreads, BM, BN, KC, true, false, false,                       \
+    KernelEntry{bi::Issue<true, BN, 1, false, KC>::kThreads, BM, BN, KC, true, false, false,                       \
                 &bi::bi_gemm_kernel<BM, BN, KC, true, false, 1, false, true>,                      \
                 bi::smem_bytes_for<BM, BN, KC, true, false, 1, false, true>(), 1, false, true}
 #define BI_ENTRY_W4_SPLIT2(BM, BN, KC)                                                             \
-    KernelEntry{bi::Issue<true, BN, 2>::kThreads, BM, BN, KC, true, false, false,                       \
+    KernelEntry{bi::Issue<true, BN, 2, false, KC>::kThreads, BM, BN, KC, true, false, false,                       \
                 &bi::bi_gemm_kernel<BM, BN, KC, true, false, 2, false, true>,                      \
                 bi::smem_bytes_for<BM, BN, KC, true, false, 2, false, true>(), 2, false, true}
 #define BI_ENTRY_KSPLIT(BM, BN, KC)                                                                \
-    KernelEntry{bi::Epi<false, BN>::kThreads, BM, BN, KC, false, false, false,                     \
+    KernelEntry{bi::Issue<false, BN, 1, false, KC>::kThreads, BM, BN, KC, false, false, false,                     \
                 &bi::bi_gemm_kernel<BM, BN, KC, false, false, 1, true>,                            \
                 bi::smem_bytes_for<BM, BN, KC, false, false, 1, true>(), 1, true, false}
 #define BI_ENTRY_SPLIT2(BM, BN, KC, F8)                                                            \
-    KernelEntry{bi::Issue<F8, BN, 2>::kThreads, BM, BN, KC, F8, false, false,                           \
+    KernelEntry{bi::Issue<F8, BN, 2, false, KC>::kThreads, BM, BN, KC, F8, false, false,                           \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, false, 2>,                                     \
                 bi::smem_bytes_for<BM, BN, KC, F8, false, 2>(), 2, false, false}
 #define BI_ENTRY_GROUPED_SPLIT2(BM, BN, KC)                                                        \
-    KernelEntry{bi::Issue<false, BN, 2, true>::kThreads, BM, BN, KC, false, true, false,                      \
+    KernelEntry{bi::Issue<false, BN, 2, true, KC>::kThreads, BM, BN, KC, false, true, false,                      \
                 &bi::bi_gemm_kernel<BM, BN, KC, false, true, 2>,                                   \
                 bi::smem_bytes_for<BM, BN, KC, false, true, 2>(), 2, false, false}
 #define BI_PAIR(BN, KC, F8, GR)                                                                    \

@@ -65,15 +65,21 @@ struct Epi {
     static constexpr int kCols = BN / kHalves;             // columns per epilogue thread
 };
 
-// MMA-issuing threads of a kernel: one, or in the dense wide lockstep form (NSPLIT = 2) two --
-// each issues one column half's instruction chain.  A thread's next tcgen05.mma waits on the issue
-// of its previous one, which costs ~50 cycles beyond the instruction's math for these tile shapes;
-// two issuers overlap that cost.  The grouped wide form (two 128 x 128 instructions per K step) is
-// bound by shared-memory bandwidth instead and keeps one issuer.  The second issuer is the warp
-// after the epilogue warps.
-template <bool FP8, int BN, int NSPLIT, bool GROUPED = false>
+// MMA-issuing threads of a kernel.  A thread's next tcgen05.mma waits on the issue of its previous
+// one, which costs ~50 cycles beyond the instruction's math for these tile shapes; two issuing
+// threads overlap that cost.  Two issuers split the work so that every accumulator still receives
+// its instructions from one thread in ascending K:
+//   - by column half, in the dense wide lockstep form (NSPLIT = 2);
+//   - by K-chunk parity, in the other dense FP8 forms with an even number of chunks per group: each
+//     128-wide K chunk has its own partial-product buffer, and the epilogue promotes the buffers in
+//     ascending kb whoever issued them.
+// The grouped wide form (two 128 x 128 instructions per K step) is bound by shared-memory bandwidth
+// instead and keeps one issuer.  The second issuer is the warp after the epilogue warps.
+template <bool FP8, int BN, int NSPLIT, bool GROUPED = false, int KC = 1>
 struct Issue {
-    static constexpr int kIssuers = GROUPED ? 1 : NSPLIT;
+    static constexpr bool kBySplit = !GROUPED && NSPLIT == 2;
+    static constexpr bool kByChunk = FP8 && !GROUPED && NSPLIT == 1 && KC % 2 == 0;
+    static constexpr int kIssuers = (kBySplit || kByChunk) ? 2 : 1;
     static constexpr int kSecondWarp = 2 + Epi<FP8, BN>::kWarps;
     static constexpr int kThreads = Epi<FP8, BN>::kThreads + (kIssuers - 1) * 32;
 };
@@ -512,7 +518,7 @@ __global__ void __launch_bounds__(256) bi_w4_rowsum_kernel(const uint8_t *a, int
 // The ring depths follow from (BM, BN, KC) (see Rings).
 template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool SPLIT = false,
           bool W4 = false>
-__global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED>::kThreads, 1)
+__global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC>::kThreads, 1)
     bi_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_a8, const GemmParams p)
@@ -529,7 +535,8 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED>::kThreads, 1)
     static_assert(!SPLIT || (!FP8 && !GROUPED && NSPLIT == 1), "split-K variant: bf16 dense");
     static_assert(!W4 || (FP8 && !GROUPED && !SPLIT), "e2m1 weights: the dense FP8 kernel");
     constexpr int kMmaN = BN / NSPLIT;                   // MMA instruction N
-    constexpr int kIssuers = Issue<FP8, BN, NSPLIT, GROUPED>::kIssuers;   // threads issuing MMAs
+    using Iss = Issue<FP8, BN, NSPLIT, GROUPED, KC>;
+    constexpr int kIssuers = Iss::kIssuers;              // threads issuing MMAs
     using R = Rings<BM, BN, KC>;
     constexpr int kElemsPerRow = FP8 ? 128 : 64;         // K elements per 128-byte row
     constexpr int kMmaK = FP8 ? 32 : 16;                 // K per tcgen05.mma
@@ -807,13 +814,16 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED>::kThreads, 1)
                                nullptr);
             }
         }
-    } else if (warp == 1 || (kIssuers > 1 && warp == Issue<FP8, BN, NSPLIT, GROUPED>::kSecondWarp)) {
+    } else if (warp == 1 || (kIssuers > 1 && warp == Iss::kSecondWarp)) {
         // ------------------------------------------------------------------ MMA issuers
-        // Issuer `iss` issues the MMAs of split iss (all splits with one issuer), for every K step
-        // of every tile in ascending order.  Both issuers wait on the same barriers, and each
-        // commits every group (the consumed and accumulator-full barriers count one commit per
-        // issuer), so a slot or an accumulator is handed on when both halves are done with it.
+        // Issuer `iss` issues the MMAs of split iss (wide form) or of the K chunks of parity iss
+        // (FP8), each accumulator's instructions in ascending K.  Both issuers wait on the same
+        // barriers, and each commits every group (the consumed and accumulator-full barriers count
+        // one commit per issuer), so a slot or an accumulator is handed on when both are done.
         const int iss = warp == 1 ? 0 : 1;
+        const int split_iss = Iss::kBySplit ? iss : 0;
+        const int chunk_iss = Iss::kByChunk ? iss : 0;
+        constexpr int kSplitsPerIssuer = Iss::kBySplit ? NSPLIT / 2 : NSPLIT;
         if (lane == 0) {
             const int SA = p.sa, SB = p.sb;
             int sa = 0, sb = 0;      // ring slots of the next group
@@ -881,10 +891,8 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED>::kThreads, 1)
                     // the MMAs of chunk c of this group (K chunk number `chunk` of the tile)
                     auto issue_chunk = [&](int c, int chunk) -> bool {
                         uint32_t d = d_tmem;
-                        if constexpr (FP8) {
-                            d = tmem_base + (acc_iter % kNumAcc) * BN;
-                            ++acc_iter;
-                        }
+                        if constexpr (FP8)   // chunk c of the group has partial buffer acc_iter + c
+                            d = tmem_base + ((acc_iter + static_cast<uint32_t>(c)) % kNumAcc) * BN;
                         const uint64_t a_desc = a_slot + ((c * a_cp) >> 4);
                         const uint64_t b_desc = b_slot + ((c * R::kBChunkBytes) >> 4);
 #pragma unroll
@@ -893,9 +901,9 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED>::kThreads, 1)
                             // bf16: accumulate across the whole K of the tile; FP8: one K chunk
                             const uint32_t accumulate = (q > 0) ? 1u : (FP8 ? 0u : (chunk > 0 ? 1u : 0u));
 #pragma unroll
-                            for (int j = 0; j < NSPLIT / kIssuers; ++j) {
+                            for (int j = 0; j < kSplitsPerIssuer; ++j) {
                                 // split sp: B rows and accumulator columns [sp kMmaN, (sp+1) kMmaN)
-                                const int sp = j + iss;
+                                const int sp = j + split_iss;
                                 const uint64_t b_sp = static_cast<uint64_t>((sp * kMmaN * kRowBytes) >> 4);
                                 if constexpr (FP8)
                                     ptx::mma_e4m3_ss(d + sp * kMmaN, a_desc + step, b_desc + b_sp + step,
@@ -911,22 +919,22 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED>::kThreads, 1)
                     // between consecutive tcgen05.mma instructions slows their issue.  Only the
                     // last group of a tile can hold fewer chunks.
                     if (nc >= KC) {
+                        if constexpr (Iss::kByChunk) {
 #pragma unroll
-                        for (int c = 0; c < KC; ++c)
-                            if (!issue_chunk(c, kg * KC + c)) {
-                                ok = false;
-                                break;
-                            }
+                            for (int j = 0; j < KC / 2; ++j)
+                                issue_chunk(2 * j + chunk_iss, kg * KC + 2 * j + chunk_iss);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < KC; ++c)
+                                issue_chunk(c, kg * KC + c);
+                        }
                     } else {
 #pragma unroll 1
-                        for (int c = 0; c < nc; ++c)
-                            if (!issue_chunk(c, kg * KC + c)) {
-                                ok = false;
-                                break;
-                            }
+                        for (int c = chunk_iss; c < nc; c += (Iss::kByChunk ? 2 : 1))
+                            issue_chunk(c, kg * KC + c);
                     }
-                    if (!ok)
-                        break;
+                    if constexpr (FP8)
+                        acc_iter += static_cast<uint32_t>(nc < KC ? nc : KC);
                     // one commit per group frees both smem slots and, for FP8, marks the group's
                     // partial products ready for the epilogue
                     ptx::mma_commit(&consumed[sb]);
