@@ -13,6 +13,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "bi_attention.h"
 
@@ -79,10 +80,14 @@ struct AttnArgs {
 };
 
 // Keys [k0, k1) of sequence b, key/value head kvh, into this warp's partial.  Every thread of the
-// CTA calls it with the same arguments (it loads shared K/V blocks and synchronises).
+// CTA calls it with the same arguments (it loads shared K/V blocks and synchronises).  The K/V
+// blocks stream through S shared-memory stages, S - 1 blocks ahead of the one being reduced; the
+// depth changes when a block arrives, never the arithmetic.
+template <int S>
 __device__ Partial chunk_attention(const AttnArgs &a, int64_t b, int kvh, int k0, int k1,
                                    const float *q_s, uint8_t *kv_s)
 {
+    static_assert(S >= 2, "at least double buffering");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nthreads = blockDim.x;
     Partial st = empty_partial();
@@ -103,16 +108,22 @@ __device__ Partial chunk_attention(const AttnArgs &a, int64_t b, int kvh, int k0
             cp_async16(vs + j * kRowStride + piece * 16, vbase + off, ok);
         }
     };
-    if (nblk > 0)
-        load_block(0, 0);
-    cp_async_commit();
-    for (int blk = 0; blk < nblk; ++blk) {
-        if (blk + 1 < nblk)
-            load_block(blk + 1, (blk + 1) & 1);
+    // blocks 0 .. S-2 first, one commit group each (empty groups past the end keep the count)
+#pragma unroll
+    for (int i = 0; i < S - 1; ++i) {
+        if (i < nblk)
+            load_block(i, i);
         cp_async_commit();
-        cp_async_wait<1>();
+    }
+    for (int blk = 0; blk < nblk; ++blk) {
+        // block blk + S - 1 into the stage block blk - 1 used (freed by the barrier that ended
+        // the previous iteration)
+        if (blk + S - 1 < nblk)
+            load_block(blk + S - 1, (blk + S - 1) % S);
+        cp_async_commit();
+        cp_async_wait<S - 1>();   // block blk's group (number blk) has landed
         __syncthreads();
-        const uint8_t *ks = kv_s + (blk & 1) * 2 * kBlockKeys * kRowStride;
+        const uint8_t *ks = kv_s + (blk % S) * 2 * kBlockKeys * kRowStride;
         const uint8_t *vs = ks + kBlockKeys * kRowStride;
         if (warp < a.group) {
             // lane j: the score of key j of the block, d ascending
@@ -164,7 +175,7 @@ __device__ Partial chunk_attention(const AttnArgs &a, int64_t b, int kvh, int k0
                 st.o[i] = acc[i];
             st.m = m_new;
         }
-        __syncthreads();   // the buffer is refilled two blocks later
+        __syncthreads();   // the stage is refilled in the next iteration
     }
     return st;
 }
@@ -198,7 +209,8 @@ __device__ __forceinline__ void store_output(const AttnArgs &a, int64_t b, int h
 }
 
 // No split: one CTA per (sequence, key/value head) walks the 4 chunks and merges them.
-__global__ void __launch_bounds__(256) attn_nosplit_kernel(AttnArgs a, __nv_bfloat16 *out)
+template <int S>
+__global__ void __launch_bounds__(256, 2) attn_nosplit_kernel(AttnArgs a, __nv_bfloat16 *out)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     float *q_s = reinterpret_cast<float *>(smem);
@@ -210,7 +222,7 @@ __global__ void __launch_bounds__(256) attn_nosplit_kernel(AttnArgs a, __nv_bflo
     Partial c[kChunks];
 #pragma unroll
     for (int ci = 0; ci < kChunks; ++ci)
-        c[ci] = L > 0 ? chunk_attention(a, b, kvh, chunk_begin(ci, L), chunk_begin(ci + 1, L), q_s, kv_s)
+        c[ci] = L > 0 ? chunk_attention<S>(a, b, kvh, chunk_begin(ci, L), chunk_begin(ci + 1, L), q_s, kv_s)
                       : empty_partial();
     const int warp = threadIdx.x >> 5;
     if (warp < a.group)
@@ -220,7 +232,8 @@ __global__ void __launch_bounds__(256) attn_nosplit_kernel(AttnArgs a, __nv_bflo
 // Split-KV: CTA `part` of `splits` for (sequence, key/value head) reduces chunks
 // [part * 4 / splits, (part + 1) * 4 / splits) (merging them pairwise when it has two) and writes
 // its partial to ws[((b * hq + h) * 4 + part) * (kD + 2)].
-__global__ void __launch_bounds__(256) attn_split_kernel(AttnArgs a, int splits, float *ws)
+template <int S>
+__global__ void __launch_bounds__(256, 2) attn_split_kernel(AttnArgs a, int splits, float *ws)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     float *q_s = reinterpret_cast<float *>(smem);
@@ -235,10 +248,10 @@ __global__ void __launch_bounds__(256) attn_split_kernel(AttnArgs a, int splits,
     Partial r = empty_partial();
     if (L > 0) {
         if (per == 1) {
-            r = chunk_attention(a, b, kvh, chunk_begin(part, L), chunk_begin(part + 1, L), q_s, kv_s);
+            r = chunk_attention<S>(a, b, kvh, chunk_begin(part, L), chunk_begin(part + 1, L), q_s, kv_s);
         } else {
-            const Partial c0 = chunk_attention(a, b, kvh, chunk_begin(2 * part, L), chunk_begin(2 * part + 1, L), q_s, kv_s);
-            const Partial c1 = chunk_attention(a, b, kvh, chunk_begin(2 * part + 1, L), chunk_begin(2 * part + 2, L), q_s, kv_s);
+            const Partial c0 = chunk_attention<S>(a, b, kvh, chunk_begin(2 * part, L), chunk_begin(2 * part + 1, L), q_s, kv_s);
+            const Partial c1 = chunk_attention<S>(a, b, kvh, chunk_begin(2 * part + 1, L), chunk_begin(2 * part + 2, L), q_s, kv_s);
             r = merge(c0, c1);
         }
     }
@@ -294,7 +307,35 @@ bi_status_t attn_device(int *num_sms)
     return major == 10 ? BI_OK : BI_ERR_NO_DEVICE;
 }
 
-constexpr int kSmemBytes = kMaxGroup * kD * 4 + 2 * 2 * kBlockKeys * kRowStride;
+template <int S>
+constexpr int smem_bytes() { return kMaxGroup * kD * 4 + S * 2 * kBlockKeys * kRowStride; }
+
+// Stage depths: a launch with at most two CTAs per SM takes the deep pipeline (6 stages, 108 KB,
+// two CTAs per SM), any other the shallow one (2 stages, 39 KB, five CTAs per SM): with few CTAs a
+// CTA needs many blocks in flight, with many CTAs occupancy matters more.
+constexpr int kDeep = 6, kShallow = 2;
+
+// Both kernels at both depths need more than the default 48 KB of dynamic shared memory; the
+// opt-in is set once per device.
+std::mutex g_attr_mu;
+bool g_attr_set[64] = {};
+
+bi_status_t ensure_attributes(int dev)
+{
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    if (dev < 0 || dev >= 64)
+        return BI_ERR_CUDA;
+    if (g_attr_set[dev])
+        return BI_OK;
+    const cudaFuncAttribute attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    if (cudaFuncSetAttribute(attn_nosplit_kernel<kDeep>, attr, smem_bytes<kDeep>()) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_nosplit_kernel<kShallow>, attr, smem_bytes<kShallow>()) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_split_kernel<kDeep>, attr, smem_bytes<kDeep>()) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_split_kernel<kShallow>, attr, smem_bytes<kShallow>()) != cudaSuccess)
+        return BI_ERR_CUDA;
+    g_attr_set[dev] = true;
+    return BI_OK;
+}
 
 } // namespace
 
@@ -355,12 +396,25 @@ bi_status_t bi_decode_attention(const void *Q, const void *K, const void *V,
     a.scale = scale;
     const int threads = 32 * a.group;
     const int64_t pairs = B * Hkv;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || (st = ensure_attributes(dev)) != BI_OK)
+        return st == BI_OK ? BI_ERR_CUDA : st;
+    const bool deep = pairs * splits <= 2LL * sms;
     if (splits == 1) {
-        attn_nosplit_kernel<<<static_cast<unsigned>(pairs), threads, kSmemBytes, stream>>>(
-            a, static_cast<__nv_bfloat16 *>(O));
+        if (deep)
+            attn_nosplit_kernel<kDeep><<<static_cast<unsigned>(pairs), threads, smem_bytes<kDeep>(), stream>>>(
+                a, static_cast<__nv_bfloat16 *>(O));
+        else
+            attn_nosplit_kernel<kShallow><<<static_cast<unsigned>(pairs), threads, smem_bytes<kShallow>(), stream>>>(
+                a, static_cast<__nv_bfloat16 *>(O));
         return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
     }
-    attn_split_kernel<<<static_cast<unsigned>(pairs * splits), threads, kSmemBytes, stream>>>(a, splits, workspace);
+    if (deep)
+        attn_split_kernel<kDeep><<<static_cast<unsigned>(pairs * splits), threads, smem_bytes<kDeep>(), stream>>>(
+            a, splits, workspace);
+    else
+        attn_split_kernel<kShallow><<<static_cast<unsigned>(pairs * splits), threads, smem_bytes<kShallow>(), stream>>>(
+            a, splits, workspace);
     if (cudaGetLastError() != cudaSuccess)
         return BI_ERR_CUDA;
     const int64_t warps = B * Hq;

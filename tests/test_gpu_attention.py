@@ -43,7 +43,11 @@ def lengths_for(B, Lmax, seed):
     return L
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,Lmax", [(4, 8, 2, 300), (16, 32, 8, 1024), (3, 16, 2, 5)])
+# The K/V pipeline depth follows the CTA count (6 stages up to two CTAs per SM, else 2), so these
+# cases compare kernels of both depths: (16, 32, 8) runs the no-split kernel deep and split-4
+# shallow, (48, 32, 8) every kernel shallow.
+@pytest.mark.parametrize("B,Hq,Hkv,Lmax", [(4, 8, 2, 300), (16, 32, 8, 1024), (3, 16, 2, 5),
+                                           (48, 32, 8, 200)])
 def test_split_kernels_match_the_no_split_kernel_bitwise(B, Hq, Hkv, Lmax):
     Q, K, V = make(B, Hq, Hkv, Lmax, 9900 + B)
     L = lengths_for(B, Lmax, 9910 + B).to(DEV)

@@ -18,10 +18,12 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.mark.parametrize("N,K,dtype", [(256, 512, bg.BI_DTYPE_BF16),
-                                       (256, 512, bg.BI_DTYPE_E4M3_BLOCKSCALED)])
-def test_wait_timeout_is_reported_and_context_survives(N, K, dtype):
-    M = 64
+# (256, 512, FP8): two warps issue alternate K chunks; (4096, 512, bf16) at M = 256: 256 tiles run
+# in the wide lockstep form, two warps issuing one column half each
+@pytest.mark.parametrize("M,N,K,dtype", [(64, 256, 512, bg.BI_DTYPE_BF16),
+                                         (64, 256, 512, bg.BI_DTYPE_E4M3_BLOCKSCALED),
+                                         (256, 4096, 512, bg.BI_DTYPE_BF16)])
+def test_wait_timeout_is_reported_and_context_survives(M, N, K, dtype):
     plan = bg.bi_gemm_plan(N, K, dtype, 1)
     if dtype == bg.BI_DTYPE_BF16:
         A = inputs.bf16_integers((M, K), seed=1, device=DEV)
