@@ -239,9 +239,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true", help="skip the other workloads' timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["decode", "prefill", "fp8", "w4a8", "moe"], default=None,
+    ap.add_argument("--profile", choices=["decode", "prefill", "fp8", "w4a8", "moe", "attention"],
+                    default=None,
                     help="launch one workload --profile-launches times, untimed (for ncu captures)")
-    ap.add_argument("--profile-m", type=int, default=64, help="M (MoE: tokens T) for --profile")
+    ap.add_argument("--profile-m", type=int, default=64,
+                    help="M for --profile (MoE: tokens T; attention: batch, sequences of length 4096)")
+    ap.add_argument("--profile-splits", type=int, default=4, help="attention: KV splits (1, 2, 4)")
     ap.add_argument("--profile-launches", type=int, default=4)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -438,6 +441,25 @@ def profile_case(args):
         work = torch.empty(bg.bi_gemm_w4a8_workspace_bytes(M) // 4, dtype=torch.float32, device=dev)
         calls = [lambda i=i: bg.bi_gemm_run_w4a8(plan, qa, sa, qws[i % 6], ws, C, w_zero=wz,
                                                  workspace=work) for i in range(L)]
+    elif args.profile == "attention":
+        # the attention_B{M}_L4096 workload of the extras: Hq = 32, Hkv = 8, D = 128
+        import math
+        Hq, Hkv, D, L4 = 32, 8, 128, 4096
+        Q = inputs.bf16_gaussian((M, Hq, D), seed=8001, device=dev)
+        Kc = inputs.bf16_gaussian((M, L4, Hkv, D), seed=8002, device=dev)
+        Vc = inputs.bf16_gaussian((M, L4, Hkv, D), seed=8003, device=dev)
+        lens = torch.full((M,), L4, dtype=torch.int32, device=dev)
+        O = torch.empty((M, Hq, D), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(bg.bi_decode_attention_workspace_bytes(M, Hq, D, 4) // 4, dtype=torch.float32,
+                         device=dev)
+        for _ in range(L):
+            bg.bi_decode_attention(Q, Kc, Vc, lens, O, 1.0 / math.sqrt(D), splits=args.profile_splits,
+                                   workspace=ws)
+        torch.cuda.synchronize()
+        ok = not bool(torch.isnan(O.float()).any())
+        print(json.dumps({"profile": "attention", "B": M, "splits": args.profile_splits, "launches": L,
+                          "finite": ok}))
+        return 0 if ok else 1
     else:
         E, N, K = 64, 2048, 7168
         plan = weight_plan(N, K, bg.BI_DTYPE_BF16, E)
@@ -477,10 +499,14 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
 
     Consecutive GEMMs of the sweep alternate between two streams, each with its own device
     staging buffers, so one GEMM's copies overlap the previous GEMM's kernel (within a stream
-    the copy-in, kernel and copy-out of a call stay in order)."""
+    the copy-in, kernel and copy-out of a call stay in order).  The reported value replays the
+    calls of two steps (the two weight-rotation phases) captured in one CUDA graph, as a serving
+    loop would: every replay copies that step's A in from pinned host memory and its C back out.
+    The same calls issued one by one from Python are reported as `eager`."""
     import torch
     from invariant_deterministic_gemm_bi_b200 import inputs
-    steps = max(1, min(args.steps, 200))
+    steps = max(2, min(args.steps, 200))
+    steps -= steps % 2
     A_host = inputs.bf16_gaussian((max(M_SWEEP), K_DEC), seed=77).pin_memory()
     C_host = {m: torch.empty((m, N_DEC), dtype=torch.bfloat16).pin_memory() for m in M_SWEEP}
     streams = [torch.cuda.Stream(device=dev) for _ in range(2)]
@@ -494,30 +520,69 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
             bg.bi_gemm_run_host(plan, A_host[:m], Bs[(s * len(M_SWEEP) + i) % n_copies],
                                 C_host[m], A_dev[j], C_dev[j], stream=streams[j])
 
+    def timed(run_steps):
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for st in streams:
+            st.wait_event(e0)
+        run_steps()
+        for st in streams:
+            ev = torch.cuda.Event()
+            ev.record(st)
+            stream.wait_event(ev)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), device=dev)
+
     for s in range(3):
         step(s)
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for st in streams:
-        st.wait_event(e0)
-    for s in range(steps):
-        step(s)
-    for st in streams:
-        ev = torch.cuda.Event()
-        ev.record(st)
-        stream.wait_event(ev)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
+    eager_ms = timed(lambda: [step(s) for s in range(steps)])
+
+    # two steps (weight phases 0 and 1 of the rotation) in one graph, replayed steps / 2 times
+    graph_ms, graph_err = None, None
+    try:
+        cap = torch.cuda.Stream(device=dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            for st in streams:
+                st.wait_stream(cap)
+            step(0)
+            step(1)
+            for st in streams:
+                cap.wait_stream(st)
+
+        def replays():   # on the timed stream, after its start event
+            with torch.cuda.stream(stream):
+                for _ in range(steps // 2):
+                    g.replay()
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+        graph_ms = timed(replays)
+        del g
+    except RuntimeError as e:   # capture refused: report the eager number alone
+        graph_err = str(e).splitlines()[0][:200]
+        torch.cuda.synchronize()
+        timed(lambda: None)      # every rank takes the same collective steps
+        graph_ms = None
+
     h2d = sum(m * K_DEC * 2 for m in M_SWEEP)
     d2h = sum(m * N_DEC * 2 for m in M_SWEEP)
-    return {"value": sweep_bytes() * steps * world / (ms * 1e-3) / 1e9, "unit": "GB/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": ms / steps,
-            "path": "bi_gemm_run_host per GEMM (pinned host A -> device, kernel, device C -> "
-                    "pinned host), consecutive GEMMs on two alternating streams"}
+    per = lambda ms: sweep_bytes() * steps * world / (ms * 1e-3) / 1e9
+    out = {"value": per(graph_ms if graph_ms is not None else eager_ms), "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+           "ms_per_step": (graph_ms if graph_ms is not None else eager_ms) / steps,
+           "path": "bi_gemm_run_host per GEMM (pinned host A -> device, kernel, device C -> "
+                   "pinned host), consecutive GEMMs on two alternating streams, "
+                   + ("two steps captured in one CUDA graph and replayed" if graph_ms is not None
+                      else "issued call by call"),
+           "eager": {"value": per(eager_ms), "ms_per_step": eager_ms / steps,
+                     "path": "the same calls issued one by one from Python"}}
+    if graph_err:
+        out["graph_capture_error"] = graph_err
+    return out
 
 
 def graph_time_per_launch(fn_list, stream, reps=20):
