@@ -495,14 +495,14 @@ def kernel_source_hash() -> str:
 
 
 def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
-    """The same sweep through bi_gemm_run_host: pinned host A in, kernel, host C out, per call.
+    """The same sweep end to end: every step copies its A slices in from pinned host memory and
+    its C results back out.
 
-    Consecutive GEMMs of the sweep alternate between two streams, each with its own device
-    staging buffers, so one GEMM's copies overlap the previous GEMM's kernel (within a stream
-    the copy-in, kernel and copy-out of a call stay in order).  The reported value replays the
-    calls of two steps (the two weight-rotation phases) captured in one CUDA graph, as a serving
-    loop would: every replay copies that step's A in from pinned host memory and its C back out.
-    The same calls issued one by one from Python are reported as `eager`."""
+    The reported value pipelines a step's copies against the neighbouring steps' GEMMs, as a
+    serving loop would (see below), captured in CUDA graphs.  `eager` is the host-buffer entry
+    point bi_gemm_run_host called GEMM by GEMM from Python: consecutive GEMMs alternate between
+    two streams, each with its own device staging buffers (within a stream the copy-in, kernel and
+    copy-out of a call stay in order)."""
     import torch
     from invariant_deterministic_gemm_bi_b200 import inputs
     steps = max(2, min(args.steps, 200))
@@ -540,29 +540,63 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
         step(s)
     eager_ms = timed(lambda: [step(s) for s in range(steps)])
 
-    # two steps (weight phases 0 and 1 of the rotation) in one graph, replayed steps / 2 times
+    # Software-pipelined, as a serving loop would run it: while step s's nine GEMMs run back to
+    # back on the compute stream (bi_gemm_run, so consecutive launches overlap set-up and tail),
+    # a copy-in stream brings step s+1's A slices from pinned host memory and a copy-out stream
+    # returns step s-1's C results to pinned host memory.  Device staging alternates between two
+    # buffers by step parity; graph p (one per parity, which is also the weight-rotation phase)
+    # holds one such step, and replays run one after another on the timed stream.  The timed
+    # region also holds the first step's copy-in and the last step's copy-out, so it moves every
+    # step's input and result (and one more of each at the two ends of the pipeline).
     graph_ms, graph_err = None, None
     try:
-        cap = torch.cuda.Stream(device=dev)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap):
-            for st in streams:
-                st.wait_stream(cap)
-            step(0)
-            step(1)
-            for st in streams:
-                cap.wait_stream(st)
+        A_buf = [{m: torch.empty((m, K_DEC), dtype=torch.bfloat16, device=dev) for m in M_SWEEP}
+                 for _ in range(2)]
+        C_buf = [{m: torch.empty((m, N_DEC), dtype=torch.bfloat16, device=dev) for m in M_SWEEP}
+                 for _ in range(2)]
+        cap, cin, cout = (torch.cuda.Stream(device=dev) for _ in range(3))
+
+        def copy_in(par):
+            for m in M_SWEEP:
+                A_buf[par][m].copy_(A_host[:m], non_blocking=True)
+
+        def copy_out(par):
+            for m in M_SWEEP:
+                C_host[m].copy_(C_buf[par][m], non_blocking=True)
+
+        def pipelined_step(par):
+            cin.wait_stream(cap)    # fork
+            cout.wait_stream(cap)
+            with torch.cuda.stream(cin):
+                copy_in(1 - par)                      # the next step's input
+            with torch.cuda.stream(cout):
+                copy_out(1 - par)                     # the previous step's result
+            for i, m in enumerate(M_SWEEP):
+                bg.bi_gemm_run(plan, A_buf[par][m], Bs[(par * len(M_SWEEP) + i) % n_copies],
+                               C_buf[par][m], stream=cap)
+            cap.wait_stream(cin)    # join
+            cap.wait_stream(cout)
+
+        graphs = []
+        for par in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                pipelined_step(par)
+            graphs.append(g)
 
         def replays():   # on the timed stream, after its start event
             with torch.cuda.stream(stream):
-                for _ in range(steps // 2):
-                    g.replay()
+                copy_in(0)                            # the first step's input
+                for s in range(steps):
+                    graphs[s % 2].replay()
+                copy_out((steps - 1) % 2)             # the last step's result
         with torch.cuda.stream(stream):
-            for _ in range(3):
-                g.replay()
+            copy_in(0)
+            for s in range(4):
+                graphs[s % 2].replay()
         graph_ms = timed(replays)
-        del g
-    except RuntimeError as e:   # capture refused: report the eager number alone
+        del graphs
+    except RuntimeError as e:   # capture refused: report the call-by-call number alone
         graph_err = str(e).splitlines()[0][:200]
         torch.cuda.synchronize()
         timed(lambda: None)      # every rank takes the same collective steps
@@ -574,12 +608,16 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
     out = {"value": per(graph_ms if graph_ms is not None else eager_ms), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
            "ms_per_step": (graph_ms if graph_ms is not None else eager_ms) / steps,
-           "path": "bi_gemm_run_host per GEMM (pinned host A -> device, kernel, device C -> "
-                   "pinned host), consecutive GEMMs on two alternating streams, "
-                   + ("two steps captured in one CUDA graph and replayed" if graph_ms is not None
-                      else "issued call by call"),
+           "path": ("software-pipelined steps: step s's nine GEMMs (bi_gemm_run) back to back on "
+                    "the compute stream while step s+1's nine A slices come in from pinned host "
+                    "memory and step s-1's nine C results go out to pinned host memory on two "
+                    "copy streams; double-buffered device staging; one CUDA graph per buffer "
+                    "parity, replayed step by step") if graph_ms is not None else
+                   "bi_gemm_run_host per GEMM, issued call by call (graph capture refused)",
            "eager": {"value": per(eager_ms), "ms_per_step": eager_ms / steps,
-                     "path": "the same calls issued one by one from Python"}}
+                     "path": "bi_gemm_run_host per GEMM (pinned host A -> device, kernel, device C -> "
+                             "pinned host) issued call by call from Python, consecutive GEMMs on two "
+                             "alternating streams"}}
     if graph_err:
         out["graph_capture_error"] = graph_err
     return out
