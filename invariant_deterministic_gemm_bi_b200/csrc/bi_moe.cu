@@ -16,7 +16,6 @@ namespace {
 constexpr int kMaxE = 1024;
 constexpr int kMaxK = 8;
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kPerThread = 8;   // dispatch: consecutive pairs per thread per pass
 
 // ---------------------------------------------------------------------------------------------
 // Router: one warp per token.  Lane l holds the logits of experts l, l + 32, l + 64, ...
@@ -90,29 +89,98 @@ __global__ void __launch_bounds__(256) moe_route_kernel(const float *logits, int
 
 // ---------------------------------------------------------------------------------------------
 // Dispatch: counts per expert, their exclusive scan, then each expert's rows in pair order.
+// One block per expert, 32 warps; warp w owns the contiguous pairs [w * seg, (w + 1) * seg) (seg a
+// multiple of 128) and walks them 128 at a time, lane l holding pairs 4l .. 4l+3 of each step (one
+// coalesced 16-byte load per lane when the id array is 16-byte aligned).  Ranks follow pair order:
+// warps in order, steps in order, lanes in order, a lane's four pairs in order.
 // ---------------------------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(256) moe_count_kernel(const int32_t *experts, int64_t n,
-                                                        int32_t *offsets)
+constexpr int kDispatchThreads = 1024;   // 32 warps: enough loads in flight per SM
+constexpr int kDispatchSteps = 8;        // 128-pair steps loaded per batch
+constexpr int kDispatchWarps = kDispatchThreads / 32;
+
+__device__ __forceinline__ int64_t dispatch_segment(int64_t n)
+{
+    const int64_t per = (n + kDispatchWarps - 1) / kDispatchWarps;
+    return (per + 127) & ~static_cast<int64_t>(127);
+}
+
+// The four ids of pairs i .. i+3 (-1 past n, which matches no expert).  VEC: experts is 16-byte
+// aligned and i is a multiple of 4.
+template <bool VEC>
+__device__ __forceinline__ int4 load_ids(const int32_t *__restrict__ experts, int64_t i, int64_t n)
+{
+    if (VEC && i + 4 <= n)
+        return __ldg(reinterpret_cast<const int4 *>(experts + i));
+    int4 v;
+    v.x = i < n ? __ldg(experts + i) : -1;
+    v.y = i + 1 < n ? __ldg(experts + i + 1) : -1;
+    v.z = i + 2 < n ? __ldg(experts + i + 2) : -1;
+    v.w = i + 3 < n ? __ldg(experts + i + 3) : -1;
+    return v;
+}
+
+__device__ __forceinline__ uint32_t hit_mask(const int4 &v, int e)
+{
+    return (v.x == e ? 1u : 0u) | (v.y == e ? 2u : 0u) | (v.z == e ? 4u : 0u) | (v.w == e ? 8u : 0u);
+}
+
+// Hits of expert e in this warp's segment (every lane gets the total).
+template <bool VEC>
+__device__ __forceinline__ int warp_count(const int32_t *__restrict__ experts, int64_t lo, int64_t hi,
+                                          int64_t n, int e)
+{
+    const int lane = threadIdx.x & 31;
+    int c = 0;
+    for (int64_t base = lo; base < hi; base += kDispatchSteps * 128) {
+        int4 v[kDispatchSteps];
+#pragma unroll
+        for (int u = 0; u < kDispatchSteps; ++u) {
+            const int64_t i = base + 128 * u + 4 * lane;
+            v[u] = (base + 128 * u < hi) ? load_ids<VEC>(experts, i, n) : make_int4(-1, -1, -1, -1);
+        }
+#pragma unroll
+        for (int u = 0; u < kDispatchSteps; ++u)
+            c += __popc(hit_mask(v[u], e));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        c += __shfl_xor_sync(kFull, c, off);
+    return c;
+}
+
+// Exclusive prefix of one count per warp, in warp order, and the block total.
+__device__ __forceinline__ int warp_prefix(int warp_total, int *total)
+{
+    __shared__ int sums[kDispatchWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0)
+        sums[warp] = warp_total;
+    __syncthreads();
+    int before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < kDispatchWarps; ++w) {
+        before += w < warp ? sums[w] : 0;
+        all += sums[w];
+    }
+    *total = all;
+    return before;
+}
+
+template <bool VEC>
+__global__ void __launch_bounds__(kDispatchThreads) moe_count_kernel(const int32_t *__restrict__ experts,
+                                                                     int64_t n, int32_t *offsets)
 {
     const int e = blockIdx.x;
-    int c = 0;
-    for (int64_t base = static_cast<int64_t>(threadIdx.x) * kPerThread; base < n;
-         base += static_cast<int64_t>(blockDim.x) * kPerThread) {
-#pragma unroll
-        for (int q = 0; q < kPerThread; ++q)
-            c += (base + q < n && experts[base + q] == e) ? 1 : 0;
-    }
-    __shared__ int part[256];
-    part[threadIdx.x] = c;
-    __syncthreads();
-    for (int w = 128; w > 0; w >>= 1) {
-        if (threadIdx.x < w)
-            part[threadIdx.x] += part[threadIdx.x + w];
-        __syncthreads();
-    }
+    const int warp = threadIdx.x >> 5;
+    const int64_t seg = dispatch_segment(n);
+    const int64_t lo = warp * seg;
+    const int64_t hi = lo + seg < n ? lo + seg : n;
+    const int c = warp_count<VEC>(experts, lo, hi, n, e);
+    int total = 0;
+    (void)warp_prefix(c, &total);
     if (threadIdx.x == 0)
-        offsets[e + 1] = part[0];
+        offsets[e + 1] = total;
 }
 
 __global__ void __launch_bounds__(kMaxE) moe_scan_kernel(int32_t *offsets, int E)
@@ -133,52 +201,52 @@ __global__ void __launch_bounds__(kMaxE) moe_scan_kernel(int32_t *offsets, int E
         offsets[0] = 0;
 }
 
-__global__ void __launch_bounds__(256) moe_fill_kernel(const int32_t *experts, int64_t n, int k,
-                                                       const int32_t *offsets, int32_t *token_of_row,
-                                                       int32_t *row_of_slot)
+template <bool VEC>
+__global__ void __launch_bounds__(kDispatchThreads) moe_fill_kernel(const int32_t *__restrict__ experts,
+                                                                    int64_t n, int k,
+                                                                    const int32_t *__restrict__ offsets,
+                                                                    int32_t *__restrict__ token_of_row,
+                                                                    int32_t *__restrict__ row_of_slot)
 {
-    // One block per expert.  A pass covers 256 * 8 consecutive pairs: thread t owns the 8 pairs
-    // [base + 8t, base + 8t + 8), so an exclusive scan of the per-thread hit counts in thread
-    // order places the expert's rows in ascending pair order.
     const int e = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __shared__ int32_t wsum[8];
-    int32_t running = offsets[e];
-    const int64_t span = static_cast<int64_t>(blockDim.x) * kPerThread;
-    for (int64_t base = 0; base < n; base += span) {
-        const int64_t i0 = base + static_cast<int64_t>(threadIdx.x) * kPerThread;
-        uint32_t hits = 0;
+    const int64_t seg = dispatch_segment(n);
+    const int64_t lo = warp * seg;
+    const int64_t hi = lo + seg < n ? lo + seg : n;
+    const int c = warp_count<VEC>(experts, lo, hi, n, e);
+    int total = 0;
+    int32_t r = offsets[e] + warp_prefix(c, &total);   // this warp's first row
+    if (c == 0)
+        return;
+    for (int64_t base = lo; base < hi; base += kDispatchSteps * 128) {
+        int4 v[kDispatchSteps];
 #pragma unroll
-        for (int q = 0; q < kPerThread; ++q)
-            if (i0 + q < n && experts[i0 + q] == e)
-                hits |= 1u << q;
-        const int cnt = __popc(hits);
-        int incl = cnt;   // inclusive scan inside the warp
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(kFull, incl, off);
-            if (lane >= off)
-                incl += y;
+        for (int u = 0; u < kDispatchSteps; ++u) {
+            const int64_t i = base + 128 * u + 4 * lane;
+            v[u] = (base + 128 * u < hi) ? load_ids<VEC>(experts, i, n) : make_int4(-1, -1, -1, -1);
         }
-        if (lane == 31)
-            wsum[warp] = incl;
-        __syncthreads();
-        int32_t before = 0, total = 0;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            before += w < warp ? wsum[w] : 0;
-            total += wsum[w];
-        }
-        int32_t r = running + before + incl - cnt;
+        for (int u = 0; u < kDispatchSteps; ++u) {
+            const uint32_t m = hit_mask(v[u], e);
+            const int h = __popc(m);
+            int incl = h;   // rows of the lanes before this one in the step, then this lane's
 #pragma unroll
-        for (int q = 0; q < kPerThread; ++q)
-            if ((hits >> q) & 1u) {
-                token_of_row[r] = static_cast<int32_t>((i0 + q) / k);
-                row_of_slot[i0 + q] = r;
-                ++r;
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(kFull, incl, off);
+                if (lane >= off)
+                    incl += y;
             }
-        running += total;
-        __syncthreads();
+            int32_t row = r + incl - h;
+            const int64_t i0 = base + 128 * u + 4 * lane;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if ((m >> j) & 1u) {
+                    token_of_row[row] = static_cast<int32_t>((i0 + j) / k);
+                    row_of_slot[i0 + j] = row;
+                    ++row;
+                }
+            r += __shfl_sync(kFull, incl, 31);   // the step's hits
+        }
     }
 }
 
@@ -326,7 +394,11 @@ bi_status_t bi_moe_dispatch(const int32_t *experts, int64_t T, int E, int k, int
     if (st != BI_OK)
         return st;
     const int64_t n = T * k;
-    moe_count_kernel<<<E, 256, 0, stream>>>(experts, n, offsets);
+    const bool vec = aligned(experts, 16);
+    if (vec)
+        moe_count_kernel<true><<<E, kDispatchThreads, 0, stream>>>(experts, n, offsets);
+    else
+        moe_count_kernel<false><<<E, kDispatchThreads, 0, stream>>>(experts, n, offsets);
     if ((st = last_launch()) != BI_OK)
         return st;
     moe_scan_kernel<<<1, kMaxE, 0, stream>>>(offsets, E);
@@ -334,7 +406,12 @@ bi_status_t bi_moe_dispatch(const int32_t *experts, int64_t T, int E, int k, int
         return st;
     if (n == 0)
         return BI_OK;
-    moe_fill_kernel<<<E, 256, 0, stream>>>(experts, n, k, offsets, token_of_row, row_of_slot);
+    if (vec)
+        moe_fill_kernel<true><<<E, kDispatchThreads, 0, stream>>>(experts, n, k, offsets, token_of_row,
+                                                                  row_of_slot);
+    else
+        moe_fill_kernel<false><<<E, kDispatchThreads, 0, stream>>>(experts, n, k, offsets, token_of_row,
+                                                                   row_of_slot);
     return last_launch();
 }
 

@@ -46,11 +46,27 @@ def test_route_matches_oracle(T, kind):
     assert np.all(np.abs(wg - ow) <= 8e-6 * ow + 1e-12), float(np.max(np.abs(wg - ow) / ow))
 
 
-@pytest.mark.parametrize("T", [1, 7, 4096])
+@pytest.mark.parametrize("T", [1, 7, 4096, 8192])
 def test_dispatch_matches_oracle(T):
     g = inputs.generator(9500 + T, "cpu")
     experts = torch.randint(0, E, (T, TOPK), generator=g, dtype=torch.int32)
     off, tok, ros = gpu_dispatch(experts.to(DEV))
+    ooff, otok, oros = omoe.dispatch(experts.numpy(), E)
+    assert (off.cpu().numpy() == ooff).all()
+    assert (tok.cpu().numpy() == otok).all()
+    assert (ros.cpu().numpy() == oros).all()
+
+
+def test_dispatch_with_ids_not_16_byte_aligned():
+    # ids 4 bytes past a 16-byte boundary take the scalar loads; the grouping is the same
+    T = 1001
+    g = inputs.generator(9550, "cpu")
+    experts = torch.randint(0, E, (T, TOPK), generator=g, dtype=torch.int32)
+    buf = torch.empty(T * TOPK + 4, dtype=torch.int32, device=DEV)
+    view = buf[1:1 + T * TOPK].view(T, TOPK)
+    view.copy_(experts.to(DEV))
+    assert view.data_ptr() % 16 == 4
+    off, tok, ros = gpu_dispatch(view)
     ooff, otok, oros = omoe.dispatch(experts.numpy(), E)
     assert (off.cpu().numpy() == ooff).all()
     assert (tok.cpu().numpy() == otok).all()
