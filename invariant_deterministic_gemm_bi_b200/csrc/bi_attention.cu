@@ -79,17 +79,31 @@ struct AttnArgs {
     float scale;
 };
 
+// A group of `nthreads` threads of the CTA (thread `tid` of the group; one warp per query head)
+// that synchronises on named barrier `bar` (0: the whole CTA).
+struct Group {
+    int tid, nthreads, bar;
+};
+
+__device__ __forceinline__ void group_sync(const Group &g)
+{
+    if (g.bar == 0)
+        __syncthreads();
+    else
+        asm volatile("bar.sync %0, %1;" ::"r"(g.bar), "r"(g.nthreads) : "memory");
+}
+
 // Keys [k0, k1) of sequence b, key/value head kvh, into this warp's partial.  Every thread of the
-// CTA calls it with the same arguments (it loads shared K/V blocks and synchronises).  The K/V
-// blocks stream through S shared-memory stages, S - 1 blocks ahead of the one being reduced; the
-// depth changes when a block arrives, never the arithmetic.
+// group calls it with the same arguments (it loads shared K/V blocks into kv_s and synchronises
+// the group).  The K/V blocks stream through S shared-memory stages, S - 1 blocks ahead of the one
+// being reduced; the depth changes when a block arrives, never the arithmetic.
 template <int S>
 __device__ Partial chunk_attention(const AttnArgs &a, int64_t b, int kvh, int k0, int k1,
-                                   const float *q_s, uint8_t *kv_s)
+                                   const float *q_s, uint8_t *kv_s, const Group &grp)
 {
     static_assert(S >= 2, "at least double buffering");
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nthreads = blockDim.x;
+    const int warp = grp.tid >> 5, lane = grp.tid & 31;
+    const int nthreads = grp.nthreads;
     Partial st = empty_partial();
     const int nblk = (k1 - k0 + kBlockKeys - 1) / kBlockKeys;
     const int64_t row_pitch = static_cast<int64_t>(a.hkv) * kD;   // elements between keys
@@ -99,7 +113,7 @@ __device__ Partial chunk_attention(const AttnArgs &a, int64_t b, int kvh, int k0
         uint8_t *ks = kv_s + buf * 2 * kBlockKeys * kRowStride;
         uint8_t *vs = ks + kBlockKeys * kRowStride;
         // 32 keys x 16 pieces of 16 bytes, for K and for V
-        for (int i = threadIdx.x; i < kBlockKeys * 16; i += nthreads) {
+        for (int i = grp.tid; i < kBlockKeys * 16; i += nthreads) {
             const int j = i >> 4, piece = i & 15;
             const int key = k0 + blk * kBlockKeys + j;
             const bool ok = key < k1;
@@ -122,7 +136,7 @@ __device__ Partial chunk_attention(const AttnArgs &a, int64_t b, int kvh, int k0
             load_block(blk + S - 1, (blk + S - 1) % S);
         cp_async_commit();
         cp_async_wait<S - 1>();   // block blk's group (number blk) has landed
-        __syncthreads();
+        group_sync(grp);
         const uint8_t *ks = kv_s + (blk % S) * 2 * kBlockKeys * kRowStride;
         const uint8_t *vs = ks + kBlockKeys * kRowStride;
         if (warp < a.group) {
@@ -175,7 +189,7 @@ __device__ Partial chunk_attention(const AttnArgs &a, int64_t b, int kvh, int k0
                 st.o[i] = acc[i];
             st.m = m_new;
         }
-        __syncthreads();   // the stage is refilled in the next iteration
+        group_sync(grp);   // the stage is refilled in the next iteration
     }
     return st;
 }
@@ -222,11 +236,62 @@ __global__ void __launch_bounds__(256, 2) attn_nosplit_kernel(AttnArgs a, __nv_b
     Partial c[kChunks];
 #pragma unroll
     for (int ci = 0; ci < kChunks; ++ci)
-        c[ci] = L > 0 ? chunk_attention<S>(a, b, kvh, chunk_begin(ci, L), chunk_begin(ci + 1, L), q_s, kv_s)
+        c[ci] = L > 0 ? chunk_attention<S>(a, b, kvh, chunk_begin(ci, L), chunk_begin(ci + 1, L), q_s, kv_s,
+                                           Group{static_cast<int>(threadIdx.x), static_cast<int>(blockDim.x), 0})
                       : empty_partial();
     const int warp = threadIdx.x >> 5;
     if (warp < a.group)
         store_output(a, b, kvh * a.group + warp, merge(merge(c[0], c[1]), merge(c[2], c[3])), L > 0, out);
+}
+
+// No split, the four chunks at once (query groups of up to 4 heads): warp group c -- one warp per
+// query head -- reduces chunk c with its own K/V stages and named barrier 1 + c; the four partials
+// meet in shared memory and group 0 merges them as ((c0 + c1) + (c2 + c3)).  Each chunk is the
+// same chunk_attention() call as in the kernels above, so the outputs are bitwise equal to theirs.
+constexpr int kParStages = 3;
+constexpr int kStageBytes = 2 * kBlockKeys * kRowStride;   // one K block and one V block
+
+__global__ void __launch_bounds__(kChunks * 4 * 32, 1) attn_nosplit_par_kernel(AttnArgs a,
+                                                                              __nv_bfloat16 *out)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    float *q_s = reinterpret_cast<float *>(smem);
+    uint8_t *kv_base = smem + kMaxGroup * kD * 4;
+    const int64_t b = blockIdx.x / a.hkv;
+    const int kvh = blockIdx.x % a.hkv;
+    const int L = valid_length(a, b);
+    load_q(a, b, kvh, q_s);
+    const int gthreads = 32 * a.group;
+    const int c = static_cast<int>(threadIdx.x) / gthreads;
+    const Group grp{static_cast<int>(threadIdx.x) - c * gthreads, gthreads, 1 + c};
+    const Partial r = L > 0 ? chunk_attention<kParStages>(a, b, kvh, chunk_begin(c, L), chunk_begin(c + 1, L), q_s,
+                                                          kv_base + c * kParStages * kStageBytes, grp)
+                            : empty_partial();
+    __syncthreads();   // every group is done with its stages: they now hold the partials
+    float *part = reinterpret_cast<float *>(kv_base);   // [chunk][head][m, l, o[kD]]
+    const int warp = grp.tid >> 5, lane = threadIdx.x & 31;
+    float *w = part + (c * kMaxGroup + warp) * (kD + 2);
+    if (lane == 0) {
+        w[0] = r.m;
+        w[1] = r.l;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        w[2 + lane * 4 + i] = r.o[i];
+    __syncthreads();
+    if (c == 0) {
+        Partial p[kChunks];
+#pragma unroll
+        for (int ci = 0; ci < kChunks; ++ci) {
+            const float *q = part + (ci * kMaxGroup + warp) * (kD + 2);
+            p[ci].m = q[0];
+            p[ci].l = q[1];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                p[ci].o[i] = q[2 + lane * 4 + i];
+        }
+        store_output(a, b, kvh * a.group + warp, merge(merge(p[0], p[1]), merge(p[2], p[3])), L > 0, out);
+    }
 }
 
 // Split-KV: CTA `part` of `splits` for (sequence, key/value head) reduces chunks
@@ -245,13 +310,14 @@ __global__ void __launch_bounds__(256, 2) attn_split_kernel(AttnArgs a, int spli
     const int L = valid_length(a, b);
     load_q(a, b, kvh, q_s);
     const int per = kChunks / splits;
+    const Group all{static_cast<int>(threadIdx.x), static_cast<int>(blockDim.x), 0};
     Partial r = empty_partial();
     if (L > 0) {
         if (per == 1) {
-            r = chunk_attention<S>(a, b, kvh, chunk_begin(part, L), chunk_begin(part + 1, L), q_s, kv_s);
+            r = chunk_attention<S>(a, b, kvh, chunk_begin(part, L), chunk_begin(part + 1, L), q_s, kv_s, all);
         } else {
-            const Partial c0 = chunk_attention<S>(a, b, kvh, chunk_begin(2 * part, L), chunk_begin(2 * part + 1, L), q_s, kv_s);
-            const Partial c1 = chunk_attention<S>(a, b, kvh, chunk_begin(2 * part + 1, L), chunk_begin(2 * part + 2, L), q_s, kv_s);
+            const Partial c0 = chunk_attention<S>(a, b, kvh, chunk_begin(2 * part, L), chunk_begin(2 * part + 1, L), q_s, kv_s, all);
+            const Partial c1 = chunk_attention<S>(a, b, kvh, chunk_begin(2 * part + 1, L), chunk_begin(2 * part + 2, L), q_s, kv_s, all);
             r = merge(c0, c1);
         }
     }
@@ -314,6 +380,9 @@ constexpr int smem_bytes() { return kMaxGroup * kD * 4 + S * 2 * kBlockKeys * kR
 // two CTAs per SM), any other the shallow one (2 stages, 39 KB, five CTAs per SM): with few CTAs a
 // CTA needs many blocks in flight, with many CTAs occupancy matters more.
 constexpr int kDeep = 6, kShallow = 2;
+constexpr int kParSmemBytes = kMaxGroup * kD * 4 + kChunks * kParStages * kStageBytes;
+static_assert(kChunks * kMaxGroup * (kD + 2) * 4 <= kChunks * kParStages * kStageBytes,
+              "the partials fit in the stages");
 
 // Both kernels at both depths need more than the default 48 KB of dynamic shared memory; the
 // opt-in is set once per device.
@@ -328,7 +397,8 @@ bi_status_t ensure_attributes(int dev)
     if (g_attr_set[dev])
         return BI_OK;
     const cudaFuncAttribute attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
-    if (cudaFuncSetAttribute(attn_nosplit_kernel<kDeep>, attr, smem_bytes<kDeep>()) != cudaSuccess ||
+    if (cudaFuncSetAttribute(attn_nosplit_par_kernel, attr, kParSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_nosplit_kernel<kDeep>, attr, smem_bytes<kDeep>()) != cudaSuccess ||
         cudaFuncSetAttribute(attn_nosplit_kernel<kShallow>, attr, smem_bytes<kShallow>()) != cudaSuccess ||
         cudaFuncSetAttribute(attn_split_kernel<kDeep>, attr, smem_bytes<kDeep>()) != cudaSuccess ||
         cudaFuncSetAttribute(attn_split_kernel<kShallow>, attr, smem_bytes<kShallow>()) != cudaSuccess)
@@ -400,6 +470,13 @@ bi_status_t bi_decode_attention(const void *Q, const void *K, const void *V,
     if (cudaGetDevice(&dev) != cudaSuccess || (st = ensure_attributes(dev)) != BI_OK)
         return st == BI_OK ? BI_ERR_CUDA : st;
     const bool deep = pairs * splits <= 2LL * sms;
+    // No split with at most one CTA per SM: the four chunks at once (with more CTAs the shallow
+    // sequential kernel keeps five CTAs per SM instead)
+    if (splits == 1 && a.group <= 4 && pairs <= sms) {
+        attn_nosplit_par_kernel<<<static_cast<unsigned>(pairs), kChunks * threads, kParSmemBytes, stream>>>(
+            a, static_cast<__nv_bfloat16 *>(O));
+        return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+    }
     if (splits == 1) {
         if (deep)
             attn_nosplit_kernel<kDeep><<<static_cast<unsigned>(pairs), threads, smem_bytes<kDeep>(), stream>>>(

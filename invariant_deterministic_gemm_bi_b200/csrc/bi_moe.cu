@@ -8,6 +8,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 
 #include "bi_moe.h"
 
@@ -89,19 +90,20 @@ __global__ void __launch_bounds__(256) moe_route_kernel(const float *logits, int
 
 // ---------------------------------------------------------------------------------------------
 // Dispatch: counts per expert, their exclusive scan, then each expert's rows in pair order.
-// One block per expert, 32 warps; warp w owns the contiguous pairs [w * seg, (w + 1) * seg) (seg a
+// One block per expert, of 8 or 32 warps; warp w owns the contiguous pairs [w * seg, (w + 1) * seg) (seg a
 // multiple of 128) and walks them 128 at a time, lane l holding pairs 4l .. 4l+3 of each step (one
 // coalesced 16-byte load per lane when the id array is 16-byte aligned).  Ranks follow pair order:
 // warps in order, steps in order, lanes in order, a lane's four pairs in order.
 // ---------------------------------------------------------------------------------------------
 
-constexpr int kDispatchThreads = 1024;   // 32 warps: enough loads in flight per SM
-constexpr int kDispatchSteps = 8;        // 128-pair steps loaded per batch
-constexpr int kDispatchWarps = kDispatchThreads / 32;
+constexpr int kDispatchSteps = 8;   // 128-pair steps loaded per batch
+// Warps per expert block: 8 for up to kFewPairs pairs, else 32 (enough loads in flight per SM).
+constexpr int kFewPairs = 16384;
 
+template <int WARPS>
 __device__ __forceinline__ int64_t dispatch_segment(int64_t n)
 {
-    const int64_t per = (n + kDispatchWarps - 1) / kDispatchWarps;
+    const int64_t per = (n + WARPS - 1) / WARPS;
     return (per + 127) & ~static_cast<int64_t>(127);
 }
 
@@ -150,16 +152,17 @@ __device__ __forceinline__ int warp_count(const int32_t *__restrict__ experts, i
 }
 
 // Exclusive prefix of one count per warp, in warp order, and the block total.
+template <int WARPS>
 __device__ __forceinline__ int warp_prefix(int warp_total, int *total)
 {
-    __shared__ int sums[kDispatchWarps];
+    __shared__ int sums[WARPS];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (lane == 0)
         sums[warp] = warp_total;
     __syncthreads();
     int before = 0, all = 0;
 #pragma unroll
-    for (int w = 0; w < kDispatchWarps; ++w) {
+    for (int w = 0; w < WARPS; ++w) {
         before += w < warp ? sums[w] : 0;
         all += sums[w];
     }
@@ -167,18 +170,18 @@ __device__ __forceinline__ int warp_prefix(int warp_total, int *total)
     return before;
 }
 
-template <bool VEC>
-__global__ void __launch_bounds__(kDispatchThreads) moe_count_kernel(const int32_t *__restrict__ experts,
-                                                                     int64_t n, int32_t *offsets)
+template <bool VEC, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32) moe_count_kernel(const int32_t *__restrict__ experts,
+                                                               int64_t n, int32_t *offsets)
 {
     const int e = blockIdx.x;
     const int warp = threadIdx.x >> 5;
-    const int64_t seg = dispatch_segment(n);
+    const int64_t seg = dispatch_segment<WARPS>(n);
     const int64_t lo = warp * seg;
     const int64_t hi = lo + seg < n ? lo + seg : n;
     const int c = warp_count<VEC>(experts, lo, hi, n, e);
     int total = 0;
-    (void)warp_prefix(c, &total);
+    (void)warp_prefix<WARPS>(c, &total);
     if (threadIdx.x == 0)
         offsets[e + 1] = total;
 }
@@ -201,21 +204,21 @@ __global__ void __launch_bounds__(kMaxE) moe_scan_kernel(int32_t *offsets, int E
         offsets[0] = 0;
 }
 
-template <bool VEC>
-__global__ void __launch_bounds__(kDispatchThreads) moe_fill_kernel(const int32_t *__restrict__ experts,
-                                                                    int64_t n, int k,
-                                                                    const int32_t *__restrict__ offsets,
-                                                                    int32_t *__restrict__ token_of_row,
-                                                                    int32_t *__restrict__ row_of_slot)
+template <bool VEC, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32) moe_fill_kernel(const int32_t *__restrict__ experts,
+                                                              int64_t n, int k,
+                                                              const int32_t *__restrict__ offsets,
+                                                              int32_t *__restrict__ token_of_row,
+                                                              int32_t *__restrict__ row_of_slot)
 {
     const int e = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t seg = dispatch_segment(n);
+    const int64_t seg = dispatch_segment<WARPS>(n);
     const int64_t lo = warp * seg;
     const int64_t hi = lo + seg < n ? lo + seg : n;
     const int c = warp_count<VEC>(experts, lo, hi, n, e);
     int total = 0;
-    int32_t r = offsets[e] + warp_prefix(c, &total);   // this warp's first row
+    int32_t r = offsets[e] + warp_prefix<WARPS>(c, &total);   // this warp's first row
     if (c == 0)
         return;
     for (int64_t base = lo; base < hi; base += kDispatchSteps * 128) {
@@ -395,10 +398,25 @@ bi_status_t bi_moe_dispatch(const int32_t *experts, int64_t T, int E, int k, int
         return st;
     const int64_t n = T * k;
     const bool vec = aligned(experts, 16);
+    const bool few = n <= kFewPairs;
+    auto count = [&](auto vec_tag, auto warps_tag) {
+        constexpr bool V = decltype(vec_tag)::value;
+        constexpr int W = decltype(warps_tag)::value;
+        moe_count_kernel<V, W><<<E, W * 32, 0, stream>>>(experts, n, offsets);
+    };
+    auto fill = [&](auto vec_tag, auto warps_tag) {
+        constexpr bool V = decltype(vec_tag)::value;
+        constexpr int W = decltype(warps_tag)::value;
+        moe_fill_kernel<V, W><<<E, W * 32, 0, stream>>>(experts, n, k, offsets, token_of_row, row_of_slot);
+    };
+    using T8 = std::integral_constant<int, 8>;
+    using T32 = std::integral_constant<int, 32>;
+    using VT = std::true_type;
+    using VF = std::false_type;
     if (vec)
-        moe_count_kernel<true><<<E, kDispatchThreads, 0, stream>>>(experts, n, offsets);
+        few ? count(VT{}, T8{}) : count(VT{}, T32{});
     else
-        moe_count_kernel<false><<<E, kDispatchThreads, 0, stream>>>(experts, n, offsets);
+        few ? count(VF{}, T8{}) : count(VF{}, T32{});
     if ((st = last_launch()) != BI_OK)
         return st;
     moe_scan_kernel<<<1, kMaxE, 0, stream>>>(offsets, E);
@@ -407,11 +425,9 @@ bi_status_t bi_moe_dispatch(const int32_t *experts, int64_t T, int E, int k, int
     if (n == 0)
         return BI_OK;
     if (vec)
-        moe_fill_kernel<true><<<E, kDispatchThreads, 0, stream>>>(experts, n, k, offsets, token_of_row,
-                                                                  row_of_slot);
+        few ? fill(VT{}, T8{}) : fill(VT{}, T32{});
     else
-        moe_fill_kernel<false><<<E, kDispatchThreads, 0, stream>>>(experts, n, k, offsets, token_of_row,
-                                                                   row_of_slot);
+        few ? fill(VF{}, T8{}) : fill(VF{}, T32{});
     return last_launch();
 }
 

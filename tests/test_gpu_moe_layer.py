@@ -57,10 +57,11 @@ def test_dispatch_matches_oracle(T):
     assert (ros.cpu().numpy() == oros).all()
 
 
-def test_dispatch_with_ids_not_16_byte_aligned():
-    # ids 4 bytes past a 16-byte boundary take the scalar loads; the grouping is the same
-    T = 1001
-    g = inputs.generator(9550, "cpu")
+@pytest.mark.parametrize("T", [1001, 3001])
+def test_dispatch_with_ids_not_16_byte_aligned(T):
+    # ids 4 bytes past a 16-byte boundary take the scalar loads, with 8 warps per expert block
+    # (8008 pairs) and with 32 (24008 pairs); the grouping is the same
+    g = inputs.generator(9550 + T, "cpu")
     experts = torch.randint(0, E, (T, TOPK), generator=g, dtype=torch.int32)
     buf = torch.empty(T * TOPK + 4, dtype=torch.int32, device=DEV)
     view = buf[1:1 + T * TOPK].view(T, TOPK)
