@@ -159,9 +159,10 @@ def oracle_sample(seconds_budget: float, rng_seed: int = 2000):
 
     The sample keeps every row of the sweep (sum of M = 511 rows) and the first n_cols output
     columns, with n_cols chosen from a calibration run so the sample takes about
-    ``seconds_budget``.  The oracle's cost is proportional to multiply-adds, so its throughput
-    is reported as the full workload's algorithmic bytes scaled by the fraction of
-    multiply-adds done, per second.
+    ``seconds_budget``; when a whole step takes less than that, the whole step is repeated
+    instead.  The oracle's cost is proportional to multiply-adds, so its throughput is reported
+    as the full workload's algorithmic bytes scaled by the (fractional) number of steps done,
+    per second.
     """
     import numpy as np
 
@@ -173,19 +174,26 @@ def oracle_sample(seconds_budget: float, rng_seed: int = 2000):
     A = inputs.to_numpy_bits(inputs.bf16_gaussian((rows, K_DEC), seed=rng_seed))
     Bfull = inputs.to_numpy_bits(inputs.bf16_gaussian((N_DEC, K_DEC), seed=rng_seed + 1,
                                                       std=K_DEC ** -0.5))
+    oracle.gemm_bf16(A, Bfull[:8], threads=threads)    # warm-up (thread start, page-in)
     t0 = time.perf_counter()
-    oracle.gemm_bf16(A, Bfull[:8], threads=threads)
-    per_col = max((time.perf_counter() - t0) / 8, 1e-6)
-    n_cols = int(max(1, min(N_DEC, seconds_budget / per_col)))
+    oracle.gemm_bf16(A, Bfull[:128], threads=threads)
+    per_col = max((time.perf_counter() - t0) / 128, 1e-6)
+    if per_col * N_DEC >= seconds_budget:   # a column slice of one step fills the budget
+        n_cols, reps = int(max(1, seconds_budget / per_col)), 1
+    else:                                   # whole steps, repeated to fill the budget
+        n_cols, reps = N_DEC, max(1, int(round(seconds_budget / (per_col * N_DEC))))
     t0 = time.perf_counter()
-    oracle.gemm_bf16(A, Bfull[:n_cols], threads=threads)
+    for _ in range(reps):
+        oracle.gemm_bf16(A, Bfull[:n_cols], threads=threads)
     dt = time.perf_counter() - t0
     frac = n_cols / N_DEC
-    value = sweep_bytes() * frac / dt / 1e9
+    value = sweep_bytes() * frac * reps / dt / 1e9
+    what = (f"all {rows} rows of the M sweep x first {n_cols} of {N_DEC} output columns "
+            f"({frac:.4f} of the step's multiply-adds)" if reps == 1 else
+            f"the whole step (all {rows} rows of the M sweep x all {N_DEC} output columns), "
+            f"{reps} times")
     return {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"all {rows} rows of the M sweep x first {n_cols} of {N_DEC} output columns "
-                      f"({frac:.4f} of the step's multiply-adds) in {dt:.2f} s; value = step bytes x "
-                      f"fraction / time",
+            "sample": f"{what} in {dt:.2f} s; value = step bytes x steps done / time",
             "seconds": dt, "n_cols": n_cols}
 
 
