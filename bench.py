@@ -379,7 +379,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_sample(10.0)
+        cpu = oracle_sample(12.0)
         cpu = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
     if rank == 0:
@@ -670,12 +670,26 @@ def measure_per_m(bg, plan, As, Bs, Cs, dev, stream, n_copies, peaks):
 
 
 def measure_extras(bg, inputs, dev, stream, peaks):
-    """Prefill, FP8 and MoE workloads: throughput and roofline fraction (not part of `value`)."""
+    """The other workloads (small, prefill, FP8, W4A8, MoE and its layer steps, attention, the
+    split-K variant): throughput and roofline fraction (not part of `value`)."""
     import torch
     res = {}
     bf16_peak = peaks["bf16_tflops"]
     fp8_peak = 2.0 * bf16_peak          # nominal dense fp8 : bf16 ratio
     hbm = peaks["hbm_gbs"]
+    # the small correctness shape N = 256, K = 512 (its 256 KB of weights stay in L2, so this is
+    # launch latency, not HBM): per launch inside a graph
+    plan = weight_plan(256, 512)
+    B = inputs.bf16_gaussian((256, 512), seed=1001, device=dev)
+    for M in [1, 3, 8, 17, 64]:
+        A = inputs.bf16_gaussian((M, 512), seed=1002, device=dev)
+        C = torch.empty((M, 256), dtype=torch.bfloat16, device=dev)
+        t = graph_time_per_launch([lambda: bg.bi_gemm_run(plan, A, B, C, stream=stream)] * 16,
+                                  stream, reps=8)
+        b = 2 * (M * 512 + 256 * 512 + M * 256)
+        res[f"small_N256_K512_M{M}"] = {"us": t * 1e6, "GB/s": b / t / 1e9,
+                                        "TFLOP/s": 2 * M * 256 * 512 / t / 1e12}
+        del A, C
     # prefill, M = 16384 and 4096
     for (N, K) in [(7168, 2048), (2048, 7168)]:
         plan = weight_plan(N, K)
@@ -695,7 +709,7 @@ def measure_extras(bg, inputs, dev, stream, peaks):
     plan = weight_plan(N, K, bg.BI_DTYPE_E4M3_BLOCKSCALED)
     qbs = [inputs.e4m3_gaussian((N, K), seed=4001 + i, device=dev) for i in range(4)]
     sb = inputs.scales_log_uniform((N // 128, KB), seed=4002, device=dev)
-    for M in [1, 64, 4096]:
+    for M in [1, 4, 16, 64, 256, 1024, 4096]:
         qa = inputs.e4m3_gaussian((M, K), seed=4003, device=dev)
         sa = inputs.scales_log_uniform((KB, ((M + 3) // 4) * 4), seed=4004, device=dev)[:, :M]
         C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
