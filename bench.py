@@ -556,7 +556,7 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
     # holds one such step, and replays run one after another on the timed stream.  The timed
     # region also holds the first step's copy-in and the last step's copy-out, so it moves every
     # step's input and result (and one more of each at the two ends of the pipeline).
-    graph_ms, graph_err = None, None
+    graph_ms, graph_err, check_ok = None, None, None
     try:
         A_buf = [{m: torch.empty((m, K_DEC), dtype=torch.bfloat16, device=dev) for m in M_SWEEP}
                  for _ in range(2)]
@@ -604,6 +604,17 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
                 graphs[s % 2].replay()
         graph_ms = timed(replays)
         del graphs
+        # the last step's results, now in pinned host memory, against the same GEMMs run on the
+        # device directly
+        last = (steps - 1) % 2
+        check_ok = True
+        with torch.cuda.stream(stream):
+            for i, m in enumerate(M_SWEEP):
+                ref = torch.empty((m, N_DEC), dtype=torch.bfloat16, device=dev)
+                bg.bi_gemm_run(plan, A_host[:m].to(dev), Bs[(last * len(M_SWEEP) + i) % n_copies], ref,
+                               stream=stream)
+                torch.cuda.synchronize()
+                check_ok &= bool(torch.equal(ref.cpu().view(torch.int16), C_host[m].view(torch.int16)))
     except RuntimeError as e:   # capture refused: report the call-by-call number alone
         graph_err = str(e).splitlines()[0][:200]
         torch.cuda.synchronize()
@@ -628,6 +639,8 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
                              "alternating streams"}}
     if graph_err:
         out["graph_capture_error"] = graph_err
+    if check_ok is not None:
+        out["results_match_device_run"] = check_ok
     return out
 
 
