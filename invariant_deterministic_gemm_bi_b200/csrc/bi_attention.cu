@@ -3,7 +3,8 @@
 // One CTA serves one (sequence, key/value head) pair -- or, split-KV, a part of its chunks --
 // with one warp per query head of the group (grouped-query attention).  A sequence's keys are cut
 // into kChunks = 4 chunks by its own length, and every chunk is reduced by chunk_attention():
-// blocks of 32 keys in ascending order, lane j scoring key j (q . k_j summed over d ascending),
+// blocks of 32 keys in ascending order, lane j scoring key j (q . k_j as two partial sums over
+// the even and the odd d, each ascending, then added),
 // an online softmax whose block max and block sum are fixed butterflies, and the value sum
 // o = o * corr + sum_j p_j v_j with j ascending.  merge() combines two chunk results, always as
 // ((c0 + c1) + (c2 + c3)).  The no-split kernel and the split-KV kernels run exactly this
@@ -58,6 +59,19 @@ __device__ __forceinline__ Partial merge(const Partial &a, const Partial &b)
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         r.o[i] = fmaf(b.o[i], fb, a.o[i] * fa);
+    return r;
+}
+
+// Two fused multiply-adds in one instruction (sm_100's packed fp32 pipe): r.x = fma(a.x, b.x, c.x)
+// and r.y = fma(a.y, b.y, c.y), each rounded to nearest like fmaf.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
     return r;
 }
 
@@ -140,22 +154,21 @@ __device__ Partial chunk_attention(const AttnArgs &a, int64_t b, int kvh, int k0
         const uint8_t *ks = kv_s + (blk % S) * 2 * kBlockKeys * kRowStride;
         const uint8_t *vs = ks + kBlockKeys * kRowStride;
         if (warp < a.group) {
-            // lane j: the score of key j of the block, d ascending
+            // lane j: the score of key j of the block, as two partial sums -- even d and odd d,
+            // each in ascending d -- added at the end
             const int key = k0 + blk * kBlockKeys + lane;
-            const float *qh = q_s + warp * kD;
+            const float2 *qh = reinterpret_cast<const float2 *>(q_s + warp * kD);
             const uint4 *krow = reinterpret_cast<const uint4 *>(ks + lane * kRowStride);
-            float s = 0.0f;
+            float2 s2 = make_float2(0.0f, 0.0f);
 #pragma unroll 4
             for (int piece = 0; piece < 16; ++piece) {
                 const uint4 raw = krow[piece];
                 const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float2 f = __bfloat1622float2(h2[t]);
-                    s = fmaf(qh[piece * 8 + 2 * t], f.x, s);
-                    s = fmaf(qh[piece * 8 + 2 * t + 1], f.y, s);
-                }
+                for (int t = 0; t < 4; ++t)
+                    s2 = fma2(qh[piece * 4 + t], __bfloat1622float2(h2[t]), s2);
             }
+            float s = s2.x + s2.y;
             s = key < k1 ? s * a.scale : -INFINITY;
             float mb = s;
 #pragma unroll
@@ -169,24 +182,22 @@ __device__ Partial chunk_attention(const AttnArgs &a, int64_t b, int kvh, int k0
             for (int off = 16; off > 0; off >>= 1)
                 ps = ps + __shfl_xor_sync(kFull, ps, off);
             st.l = fmaf(st.l, corr, ps);
-            float acc[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                acc[i] = st.o[i] * corr;
+            // o = o * corr + sum_j p_j v_j, j ascending (two dimensions per packed FMA: the same
+            // roundings as four fmaf)
+            float2 acc01 = make_float2(st.o[0] * corr, st.o[1] * corr);
+            float2 acc23 = make_float2(st.o[2] * corr, st.o[3] * corr);
             for (int j = 0; j < kBlockKeys; ++j) {
                 const float pj = __shfl_sync(kFull, p, j);
+                const float2 pp = make_float2(pj, pj);
                 const __nv_bfloat162 *vrow =
                     reinterpret_cast<const __nv_bfloat162 *>(vs + j * kRowStride) + lane * 2;
-                const float2 v01 = __bfloat1622float2(vrow[0]);
-                const float2 v23 = __bfloat1622float2(vrow[1]);
-                acc[0] = fmaf(pj, v01.x, acc[0]);
-                acc[1] = fmaf(pj, v01.y, acc[1]);
-                acc[2] = fmaf(pj, v23.x, acc[2]);
-                acc[3] = fmaf(pj, v23.y, acc[3]);
+                acc01 = fma2(pp, __bfloat1622float2(vrow[0]), acc01);
+                acc23 = fma2(pp, __bfloat1622float2(vrow[1]), acc23);
             }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                st.o[i] = acc[i];
+            st.o[0] = acc01.x;
+            st.o[1] = acc01.y;
+            st.o[2] = acc23.x;
+            st.o[3] = acc23.y;
             st.m = m_new;
         }
         group_sync(grp);   // the stage is refilled in the next iteration
