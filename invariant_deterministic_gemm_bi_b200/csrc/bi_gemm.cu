@@ -81,12 +81,13 @@ struct KernelEntry {
 // in two forms: its preferred number of 128-byte K chunks per pipeline stage (3-D TMA boxes;
 // needs K to be a multiple of the chunk), and one chunk per stage for any other K.  The bf16
 // 128 x 32 and the FP8 128 x 64 tiles have a third, small-batch form with twice the preferred
-// chunks per stage, and a wide form that runs two adjacent tiles in lockstep on one A operand
-// (see dense_kernel_for).
+// chunks per stage (the bf16 tile a fourth, tiny-batch form with 16), and a wide form that runs
+// two adjacent tiles in lockstep on one A operand (see dense_kernel_for).
 const KernelEntry kKernels[] = {
     BI_ENTRY(64, 32, 1, false, false),  BI_ENTRY(64, 32, 4, false, false),
     BI_ENTRY(128, 32, 1, false, false), BI_ENTRY(128, 32, 4, false, false),
-    BI_ENTRY(128, 32, 8, false, false), BI_ENTRY_SPLIT2(128, 64, 2, false),
+    BI_ENTRY(128, 32, 8, false, false), BI_ENTRY(128, 32, 16, false, false),
+    BI_ENTRY_SPLIT2(128, 64, 2, false),
     BI_ENTRY(128, 64, 1, false, false), BI_ENTRY(128, 64, 2, false, false),
     BI_ENTRY(128, 32, 1, true, false),  BI_ENTRY(128, 32, 4, true, false),
     BI_ENTRY(128, 64, 1, true, false),  BI_ENTRY(128, 64, 2, true, false),
@@ -165,8 +166,9 @@ RingGeom ring_geometry(const KernelEntry *k, int a_rows)
     // The kernel relies on 2 <= sa <= sb (the A-slot reuse test reads the consumed ring) and, for
     // FP8, on sb groups outlasting the partial-product ring.  Every tile in kKernels satisfies
     // this for every a_rows in [8, BM], except the small-batch forms, which are valid up to 64
-    // (bf16, 8 chunks) and 96 (FP8, 4 chunks) rows and used up to kSmallBatchRows = 64; set_rows reports a violation and the launch is
-    // refused.  tests/test_abi.py checks the reported depths.
+    // (bf16, 8 chunks) and 96 (FP8, 4 chunks) rows and used up to kSmallBatchRows = 64, and the
+    // bf16 tiny-batch form (16 chunks), valid and used up to 8 rows; set_rows reports a violation
+    // and the launch is refused.  tests/test_abi.py checks the reported depths.
     return RingGeom{sa, sb, static_cast<uint32_t>(a_stride), static_cast<uint32_t>(a_region)};
 }
 
@@ -296,6 +298,10 @@ struct bi_plan_s {
     // (dense plans only; may be null).  It issues the same MMAs in the same K order, so a row's
     // result does not depend on which of the two a launch takes.
     const KernelEntry *kernel_small = nullptr;
+    // The bf16 small-batch tile with twice its chunks again (16 per group), for launches whose A
+    // boxes hold at most 8 rows (dense bf16 128 x 32 plans only; may be null).  Same MMAs, same
+    // K order.
+    const KernelEntry *kernel_tiny = nullptr;
     // Two adjacent tiles in lockstep on one A operand (the same MMA instructions in the same K
     // order), for dense launches with more tiles than SMs and grouped launches with at least a
     // tile's worth of rows per expert on average.  May be null.
@@ -586,12 +592,17 @@ int b_box_rows_for(const KernelEntry *k)
 // the per-group wait and commit overhead of the MMA thread, and the ring still holds two groups
 // of A and of B (and, for FP8, more groups than partial-product buffers).
 constexpr int kSmallBatchRows = 64;
+// ... and at most this many rows, the tiny-batch form (16 chunks per group): the 8-row A boxes
+// leave room for two 64 KB groups of B.
+constexpr int kTinyBatchRows = 8;
 
 // A dense launch with more tiles than the device has SMs takes the plan's wide form (when it has
 // one): a CTA runs two adjacent column tiles in lockstep, so each A chunk is loaded once for both
 // and the launch needs half the CTAs, i.e. fewer waves.
 const KernelEntry *dense_kernel_for(const bi_plan_s *plan, const DeviceInfo *d, int64_t M)
 {
+    if (plan->kernel_tiny && a_box_rows_for(plan->kernel_tiny, M) <= kTinyBatchRows)
+        return plan->kernel_tiny;
     if (plan->kernel_small && a_box_rows_for(plan->kernel_small, M) <= kSmallBatchRows)
         return plan->kernel_small;
     if (plan->kernel_wide) {
@@ -697,6 +708,8 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     if (num_experts == 1 && !k->pair && k->bm == 128 && k->kc == preferred_chunks(k->bn) &&
         k->bn == (fp8 ? 64 : 32))
         p->kernel_small = find_kernel(128, k->bn, 2 * k->kc, fp8, false, w4);
+    if (p->kernel_small && !fp8 && p->kernel_small->kc == 8)
+        p->kernel_tiny = find_kernel(128, k->bn, 16, false, false, false);
     if (num_experts > 1 && !k->pair && k->bm == 128 && k->bn == 128) {
         for (int i = 0; i < kNumKernels; ++i)
             if (kKernels[i].nsplit == 2 && kKernels[i].grouped && kKernels[i].bn == 256)

@@ -527,7 +527,7 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC>::kThreads,
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32,256]");
     static_assert(!FP8 || BN <= 128, "FP8 keeps BN fp32 accumulators per thread: BN <= 128");
     static_assert(!(FP8 && GROUPED), "grouped FP8 is not built");
-    static_assert(KC >= 1 && KC <= 8, "1..8 chunks per group");
+    static_assert(KC >= 1 && KC <= 16, "1..16 chunks per group");
     static_assert(NSPLIT == 1 ||
                       (NSPLIT == 2 && (GROUPED ? (!FP8 && BN == 256) : BN == (FP8 ? 128 : 64))),
                   "split MMAs: dense bf16 64-wide, FP8 128-wide and grouped bf16 256-wide tiles as "
