@@ -253,6 +253,84 @@ __global__ void __launch_bounds__(WARPS * 32) moe_fill_kernel(const int32_t *__r
     }
 }
 
+// Few pairs (up to kPassPairs): one block per expert walks all pairs in passes of 256 x 8
+// consecutive pairs (thread t owns pairs 8t .. 8t+7 of a pass), ranking its hits with one block
+// scan per pass.  Same grouping as the segment kernels above; fewer steps when there are few pairs.
+constexpr int kPerThread = 8;
+constexpr int64_t kPassPairs = 4096;
+
+__global__ void __launch_bounds__(256) moe_count_pass_kernel(const int32_t *experts, int64_t n,
+                                                        int32_t *offsets)
+{
+    const int e = blockIdx.x;
+    int c = 0;
+    for (int64_t base = static_cast<int64_t>(threadIdx.x) * kPerThread; base < n;
+         base += static_cast<int64_t>(blockDim.x) * kPerThread) {
+#pragma unroll
+        for (int q = 0; q < kPerThread; ++q)
+            c += (base + q < n && experts[base + q] == e) ? 1 : 0;
+    }
+    __shared__ int part[256];
+    part[threadIdx.x] = c;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+        if (threadIdx.x < w)
+            part[threadIdx.x] += part[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0)
+        offsets[e + 1] = part[0];
+}
+
+__global__ void __launch_bounds__(256) moe_fill_pass_kernel(const int32_t *experts, int64_t n, int k,
+                                                       const int32_t *offsets, int32_t *token_of_row,
+                                                       int32_t *row_of_slot)
+{
+    // One block per expert.  A pass covers 256 * 8 consecutive pairs: thread t owns the 8 pairs
+    // [base + 8t, base + 8t + 8), so an exclusive scan of the per-thread hit counts in thread
+    // order places the expert's rows in ascending pair order.
+    const int e = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ int32_t wsum[8];
+    int32_t running = offsets[e];
+    const int64_t span = static_cast<int64_t>(blockDim.x) * kPerThread;
+    for (int64_t base = 0; base < n; base += span) {
+        const int64_t i0 = base + static_cast<int64_t>(threadIdx.x) * kPerThread;
+        uint32_t hits = 0;
+#pragma unroll
+        for (int q = 0; q < kPerThread; ++q)
+            if (i0 + q < n && experts[i0 + q] == e)
+                hits |= 1u << q;
+        const int cnt = __popc(hits);
+        int incl = cnt;   // inclusive scan inside the warp
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off)
+                incl += y;
+        }
+        if (lane == 31)
+            wsum[warp] = incl;
+        __syncthreads();
+        int32_t before = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            before += w < warp ? wsum[w] : 0;
+            total += wsum[w];
+        }
+        int32_t r = running + before + incl - cnt;
+#pragma unroll
+        for (int q = 0; q < kPerThread; ++q)
+            if ((hits >> q) & 1u) {
+                token_of_row[r] = static_cast<int32_t>((i0 + q) / k);
+                row_of_slot[i0 + q] = r;
+                ++r;
+            }
+        running += total;
+        __syncthreads();
+    }
+}
+
 // ---------------------------------------------------------------------------------------------
 // Gather and combine: 16-byte vectors of 8 bf16
 // ---------------------------------------------------------------------------------------------
@@ -397,6 +475,18 @@ bi_status_t bi_moe_dispatch(const int32_t *experts, int64_t T, int E, int k, int
     if (st != BI_OK)
         return st;
     const int64_t n = T * k;
+    if (n <= kPassPairs) {
+        moe_count_pass_kernel<<<E, 256, 0, stream>>>(experts, n, offsets);
+        if ((st = last_launch()) != BI_OK)
+            return st;
+        moe_scan_kernel<<<1, kMaxE, 0, stream>>>(offsets, E);
+        if ((st = last_launch()) != BI_OK)
+            return st;
+        if (n == 0)
+            return BI_OK;
+        moe_fill_pass_kernel<<<E, 256, 0, stream>>>(experts, n, k, offsets, token_of_row, row_of_slot);
+        return last_launch();
+    }
     const bool vec = aligned(experts, 16);
     const bool few = n <= kFewPairs;
     auto count = [&](auto vec_tag, auto warps_tag) {

@@ -46,7 +46,8 @@ def test_route_matches_oracle(T, kind):
     assert np.all(np.abs(wg - ow) <= 8e-6 * ow + 1e-12), float(np.max(np.abs(wg - ow) / ow))
 
 
-@pytest.mark.parametrize("T", [1, 7, 4096, 8192])
+# T * 8 pairs: up to 4096 the pass kernels, up to 16384 8-warp segments, above 32-warp segments
+@pytest.mark.parametrize("T", [1, 7, 1024, 4096, 8192])
 def test_dispatch_matches_oracle(T):
     g = inputs.generator(9500 + T, "cpu")
     experts = torch.randint(0, E, (T, TOPK), generator=g, dtype=torch.int32)
