@@ -217,7 +217,8 @@ bi_status_t bi_gemm_run_w4a8(bi_plan_t plan, int64_t M,
  * on `stream` (cudaMemcpyAsync; pinned host memory makes the copies asynchronous).  B and
  * scale_b are device pointers (resident weights).  A_dev / C_dev / scale_a_dev must be large
  * enough for M*lda, M*ldc and ceil(K/128)*ld_sa elements.  The call returns once everything is
- * enqueued; synchronise `stream` before reading C_host.
+ * enqueued; synchronise `stream` before reading C_host.  Every argument is checked before the
+ * first copy is enqueued, so a refused call has enqueued nothing.
  * Errors: as bi_gemm_run, plus BI_ERR_INVALID_ARG for missing staging buffers.
  */
 bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M,
@@ -252,8 +253,12 @@ bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M,
  * calls that overlap on the GPU (from several host threads or streams) race on it and must be
  * serialised by the caller.  The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call before any stream
- * capture.  Dense plans only (a grouped plan returns BI_ERR_INVALID_ARG).
- * Errors: as bi_gemm_run_host, plus BI_ERR_UNSUPPORTED_SHAPE when the scratch is too small.
+ * capture begins, so that the look-up never happens inside a capture.  The status word is read
+ * back on `stream` ahead of the one synchronisation, so the call touches no other stream.
+ * Dense plans only (a grouped plan returns BI_ERR_INVALID_ARG).
+ * Errors: as bi_gemm_run_host (scale_b must be 4-byte aligned; scale_a_host may have any
+ * alignment, it is only copied), plus BI_ERR_UNSUPPORTED_SHAPE when the scratch is too small
+ * or when M, lda, ldc or ld_sa alone exceeds BI_NOALLOC_SCRATCH_BYTES.
  */
 #define BI_NOALLOC_SCRATCH_BYTES (8u << 20)
 bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M,

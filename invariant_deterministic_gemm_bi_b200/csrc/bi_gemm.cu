@@ -486,6 +486,23 @@ bi_status_t check_common(const bi_plan_s *plan, int64_t rows, const void *A, int
     return BI_OK;
 }
 
+// FP8 scale arguments of a dense run with M > 0, N > 0 and K > 0: both scales present, the
+// K-block-major pitch of scale_a at least M, and 4-byte alignment of every scale pointer the
+// kernel reads (scale_a only when it is a device pointer the kernel reads directly).
+bi_status_t check_fp8_scales(int64_t M, const float *scale_a, int64_t ld_sa, const float *scale_b,
+                             bool scale_a_read_by_kernel)
+{
+    if (!scale_a || !scale_b)
+        return BI_ERR_DTYPE_MISMATCH;
+    if (ld_sa < M)
+        return BI_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(scale_b) & 3u)
+        return BI_ERR_ALIGNMENT;
+    if (scale_a_read_by_kernel && (reinterpret_cast<uintptr_t>(scale_a) & 3u))
+        return BI_ERR_ALIGNMENT;
+    return BI_OK;
+}
+
 // Rows of A one TMA load brings for a dense problem of M rows: the tile's 128 rows, or, when the
 // problem is smaller than one tile, only the rows that exist (rounded up to the 8-row swizzle
 // atom).  This changes which shared-memory rows are written, not the MMA or its K order.
@@ -814,12 +831,9 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
     const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
     if (fp8) {
         if (M > 0 && plan->n > 0 && plan->k > 0) {
-            if (!scale_a || !scale_b)
-                return BI_ERR_DTYPE_MISMATCH;
-            if (ld_sa < M)
-                return BI_ERR_INVALID_ARG;
-            if ((reinterpret_cast<uintptr_t>(scale_a) & 3u) || (reinterpret_cast<uintptr_t>(scale_b) & 3u))
-                return BI_ERR_ALIGNMENT;
+            const bi_status_t sst = check_fp8_scales(M, scale_a, ld_sa, scale_b, true);
+            if (sst != BI_OK)
+                return sst;
         }
     } else if (scale_a || scale_b) {
         return BI_ERR_DTYPE_MISMATCH;
@@ -928,6 +942,10 @@ bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M, const void *A_host, int6
     bi_status_t st = check_common(plan, M, A_dev, lda, B, ldb, C_dev, ldc);
     if (st != BI_OK)
         return st;
+    if (fp8 && plan->k > 0 && (st = check_fp8_scales(M, scale_a_dev, ld_sa, scale_b, true)) != BI_OK)
+        return st;
+    if (!fp8 && (scale_a_host || scale_b))
+        return BI_ERR_DTYPE_MISMATCH;
     if (plan->k > 0) {
         if (cudaMemcpyAsync(A_dev, A_host, static_cast<size_t>(M * lda * elt),
                             cudaMemcpyHostToDevice, stream) != cudaSuccess)
@@ -965,15 +983,20 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
     if (!C_host || (plan->k > 0 && !A_host))
         return BI_ERR_INVALID_ARG;
     if (fp8 && plan->k > 0) {
-        if (!scale_a_host || !scale_b)
-            return BI_ERR_DTYPE_MISMATCH;
-        if (ld_sa < M)
-            return BI_ERR_INVALID_ARG;
+        // scale_a_host is only copied (any alignment); scale_b is read by the kernel
+        const bi_status_t sst = check_fp8_scales(M, scale_a_host, ld_sa, scale_b, false);
+        if (sst != BI_OK)
+            return sst;
     } else if (!fp8 && (scale_a_host || scale_b)) {
         return BI_ERR_DTYPE_MISMATCH;
     }
     if (lda < plan->k || ldc < plan->n || (fp8 && ld_sa < 0))
         return BI_ERR_INVALID_ARG;
+    // Bound every factor of the scratch offsets before multiplying: no row count, pitch or
+    // scale pitch can exceed the scratch size, so each product below stays far inside int64.
+    const int64_t cap = static_cast<int64_t>(BI_NOALLOC_SCRATCH_BYTES);
+    if (M > cap || lda > cap || ldc > cap || (fp8 && ld_sa > cap))
+        return BI_ERR_UNSUPPORTED_SHAPE;
     // Scratch layout: [status word | A | C | scale_a], each part 256-byte aligned.
     const int64_t kb = (plan->k + 127) / 128;
     const int64_t a_off = 256;
@@ -1030,10 +1053,11 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
     if (cudaMemcpyAsync(C_host, C_dev, static_cast<size_t>(M * ldc * 2), cudaMemcpyDeviceToHost,
                         stream) != cudaSuccess)
         return BI_ERR_CUDA;
-    if (cudaStreamSynchronize(stream) != cudaSuccess)
-        return BI_ERR_CUDA;
+    // the status word comes back on the same stream, so one synchronisation covers C and it
     int host = 0;
-    if (cudaMemcpy(&host, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    if (cudaMemcpyAsync(&host, status, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return BI_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess)
         return BI_ERR_CUDA;
     return host == 0 ? BI_OK : static_cast<bi_status_t>(host);
 }

@@ -116,6 +116,62 @@ def test_run_rejects_bad_arguments_without_touching_a_device():
     assert lib.bi_gemm_run(fplan.handle, 4, 16, 128, 16, 128, 16, 64, 16, 3, 16, None) == S["BI_ERR_INVALID_ARG"]
 
 
+def test_noalloc_rejects_bad_arguments_before_any_device_call():
+    """The host-buffer entry point without allocation checks every argument before it touches a
+    device, so each refusal below comes back on a machine with or without a GPU and launches
+    nothing.  The pointer values are never dereferenced."""
+    lib = binding.load_library()
+    S = binding.STATUS
+    run = lib.bi_gemm_run_host_noalloc
+    bf = bg.bi_gemm_plan(256, 512)
+    f8 = bg.bi_gemm_plan(256, 512, bg.BI_DTYPE_E4M3_BLOCKSCALED)
+    # (plan, M, A_host, lda, B, ldb, C_host, ldc, scale_a_host, ld_sa, scale_b, stream)
+    assert run(None, 1, 256, 512, 256, 512, 256, 256, None, 0, None, None) == S["BI_ERR_INVALID_ARG"]
+    assert run(bf.handle, -1, 256, 512, 256, 512, 256, 256, None, 0, None, None) == S["BI_ERR_INVALID_ARG"]
+    # scales on a bf16 plan; FP8 without scale_b; FP8 scale_b not 4-byte aligned
+    assert run(bf.handle, 1, 256, 512, 256, 512, 256, 256, 256, 1, 256, None) == S["BI_ERR_DTYPE_MISMATCH"]
+    assert run(f8.handle, 1, 256, 512, 256, 512, 256, 256, 256, 1, None, None) == S["BI_ERR_DTYPE_MISMATCH"]
+    assert run(f8.handle, 4, 256, 512, 256, 512, 256, 256, 256, 4, 258, None) == S["BI_ERR_ALIGNMENT"]
+    assert run(f8.handle, 4, 256, 512, 256, 512, 256, 256, 256, 3, 256, None) == S["BI_ERR_INVALID_ARG"]
+    # a grouped plan
+    gp = bg.bi_gemm_plan(256, 512, 0, 4)
+    assert run(gp.handle, 1, 256, 512, 256, 512, 256, 256, None, 0, None, None) == S["BI_ERR_INVALID_ARG"]
+    # pitches whose products would overflow int64 are refused before any offset is computed:
+    # a K = 0 plan (C only) with a huge ldc, and huge lda / ld_sa
+    k0 = bg.bi_gemm_plan(256, 0)
+    assert run(k0.handle, 2, None, 0, None, 0, 256, 2 ** 62, None, 0, None, None) == \
+        S["BI_ERR_UNSUPPORTED_SHAPE"]
+    assert run(bf.handle, 2, 256, 2 ** 62, 256, 512, 256, 256, None, 0, None, None) == \
+        S["BI_ERR_UNSUPPORTED_SHAPE"]
+    assert run(f8.handle, 2, 256, 512, 256, 512, 256, 256, 256, 2 ** 61, 256, None) == \
+        S["BI_ERR_UNSUPPORTED_SHAPE"]
+    assert run(bf.handle, 2 ** 40, 256, 512, 256, 512, 256, 256, None, 0, None, None) == \
+        S["BI_ERR_UNSUPPORTED_SHAPE"]
+    # 373 decode rows need more than the 8 MiB scratch
+    dec = bg.bi_gemm_plan(4096, 7168)
+    assert run(dec.handle, 373, 256, 7168, 256, 7168, 256, 4096, None, 0, None, None) == \
+        S["BI_ERR_UNSUPPORTED_SHAPE"]
+    if not __import__("torch").cuda.is_available():
+        # valid arguments (scale_a_host may have any alignment: it is only copied)
+        assert run(f8.handle, 4, 256, 512, 256, 512, 256, 256, 258, 4, 256, None) == S["BI_ERR_NO_DEVICE"]
+        assert run(dec.handle, 372, 256, 7168, 256, 7168, 256, 4096, None, 0, None, None) == \
+            S["BI_ERR_NO_DEVICE"]
+
+
+def test_run_host_refuses_before_enqueueing_a_copy():
+    lib = binding.load_library()
+    S = binding.STATUS
+    f8 = bg.bi_gemm_plan(256, 512, bg.BI_DTYPE_E4M3_BLOCKSCALED)
+    bf = bg.bi_gemm_plan(256, 512)
+    # (plan, M, A_host, lda, B, ldb, C_host, ldc, sa_host, ld_sa, scale_b, A_dev, C_dev, sa_dev, stream)
+    assert lib.bi_gemm_run_host(f8.handle, 4, 256, 512, 256, 512, 256, 256, 256, 4, 258, 256, 256, 256,
+                                None) == S["BI_ERR_ALIGNMENT"]
+    assert lib.bi_gemm_run_host(f8.handle, 4, 256, 512, 256, 512, 256, 256, 256, 4, 256, 256, 256, 258,
+                                None) == S["BI_ERR_ALIGNMENT"]
+    assert lib.bi_gemm_run_host(bf.handle, 4, 256, 512, 256, 512, 256, 256, None, 0, 256, 256, 256, None,
+                                None) == S["BI_ERR_DTYPE_MISMATCH"]
+
+
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="a GPU is present")
 def test_valid_run_without_a_device_reports_no_device():
     lib = binding.load_library()
