@@ -63,6 +63,30 @@ def sweep_macs(n=N_DEC, k=K_DEC, ms=M_SWEEP):
     return sum(m * n * k for m in ms)
 
 
+def moe_routed_rows(bg, inputs, T, E, K, seed, dev, stream=None, topk=8):
+    """The grouped GEMM's inputs for T tokens, built on the GPU by the library's own MoE steps:
+    router logits ~ N(0, 1) (seeded, drawn on the host), bi_moe_route_topk (top-8, ties to the
+    lower expert), bi_moe_dispatch (stable grouping by expert) and bi_moe_gather_rows.  Returns
+    (A_perm [T*8, K] bf16, expert offsets int32 [E+1], number of experts with rows)."""
+    import torch
+    g = inputs.generator(seed, "cpu")
+    logits = torch.randn(T, E, generator=g, dtype=torch.float32).to(dev)
+    tokens = inputs.bf16_gaussian((T, K), seed=seed + 1, device=dev)
+    R = T * topk
+    ex = torch.empty((T, topk), dtype=torch.int32, device=dev)
+    w = torch.empty((T, topk), dtype=torch.float32, device=dev)
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    tok = torch.empty(R, dtype=torch.int32, device=dev)
+    ros = torch.empty(R, dtype=torch.int32, device=dev)
+    A = torch.empty((R, K), dtype=torch.bfloat16, device=dev)
+    bg.bi_moe_route_topk(logits, topk, ex, w, stream=stream)
+    bg.bi_moe_dispatch(ex, E, off, tok, ros, stream=stream)
+    bg.bi_moe_gather_rows(tokens, tok, A, stream=stream)
+    torch.cuda.synchronize()
+    active = int((off[1:] > off[:-1]).sum().item())
+    return A, off, active
+
+
 def load_peaks():
     path = os.path.join(REPO, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -472,11 +496,8 @@ def profile_case(args):
         E, N, K = 64, 2048, 7168
         plan = weight_plan(N, K, bg.BI_DTYPE_BF16, E)
         B = inputs.bf16_gaussian((E, N, K), seed=31, std=K ** -0.5, device=dev)
-        r = inputs.softmax_top8_routing(M, E, seed=32)
-        tokens = inputs.bf16_gaussian((M, K), seed=33, device=dev)
-        A = tokens[r.token_of_row.to(dev)].contiguous()
+        A, off, _ = moe_routed_rows(bg, inputs, M, E, K, seed=32, dev=dev)
         C = torch.empty((A.shape[0], N), dtype=torch.bfloat16, device=dev)
-        off = r.offsets.to(dev)
         calls = [lambda: bg.bi_grouped_gemm_run(plan, A, B, C, off) for _ in range(L)]
     for f in calls:
         f()
@@ -773,14 +794,10 @@ def measure_extras(bg, inputs, dev, stream, peaks):
     plan = weight_plan(N, K, bg.BI_DTYPE_BF16, E)
     B = inputs.bf16_gaussian((E, N, K), seed=5001, std=K ** -0.5, device=dev)
     for T in [1, 64, 1024, 8192]:
-        r = inputs.softmax_top8_routing(T, E, seed=5000 + T)
-        tokens = inputs.bf16_gaussian((T, K), seed=5002, device=dev)
-        A = tokens[r.token_of_row.to(dev)].contiguous()
+        A, off, active = moe_routed_rows(bg, inputs, T, E, K, seed=5000 + T, dev=dev, stream=stream)
         C = torch.empty((A.shape[0], N), dtype=torch.bfloat16, device=dev)
-        off = r.offsets.to(dev)
         t = graph_time_per_launch([lambda: bg.bi_grouped_gemm_run(plan, A, B, C, off, stream=stream)] * 3,
                                   stream, reps=4)
-        active = int((r.offsets[1:] > r.offsets[:-1]).sum())
         rows = A.shape[0]
         b = active * N * K * 2 + rows * K * 2 + rows * N * 2
         tf = 2 * rows * N * K / t / 1e12
@@ -807,7 +824,8 @@ def measure_extras(bg, inputs, dev, stream, peaks):
         steps = {
             "route": (lambda: bg.bi_moe_route_topk(logits, k, ex, w, stream=stream), T * E * 4 + T * k * 8),
             "dispatch": (lambda: bg.bi_moe_dispatch(ex, E, off, tok, ros, stream=stream), R * 4 * 3 + (E + 1) * 4),
-            "gather": (lambda: bg.bi_moe_gather_rows(toks, tok, A, stream=stream), 2 * R * K * 2 + R * 4),
+            # each token row is read from HBM once (its k copies hit L2): T rows in, R rows out
+            "gather": (lambda: bg.bi_moe_gather_rows(toks, tok, A, stream=stream), T * K * 2 + R * K * 2 + R * 4),
             "combine": (lambda: bg.bi_moe_combine(Cp, ros, w, Y, stream=stream), R * N * 2 + T * N * 2 + R * 8),
         }
         bg.bi_moe_route_topk(logits, k, ex, w, stream=stream)

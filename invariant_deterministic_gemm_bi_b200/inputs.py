@@ -17,17 +17,14 @@ Recipes (all seeded; a generator is ``torch.Generator(device)`` seeded with the 
 * e2m1 channel scales: 2^-j with integer j uniform in [1, 12]; zero points z = fp16(x * s),
                    x ~ N(0, 1), rounded to fp16 (RNE) and held in fp32; or, for the exactly
                    representable variant, z = i * 2^-6 with integer i uniform in [-64, 64].
-* MoE routing:     logits [T, E] ~ N(0, 1); each token takes the 8 largest logits (softmax is
-                   monotone, so this is top-8 by softmax); ties go to the lower expert index.
-                   The (token, slot) pairs are stably sorted by expert, so inside an expert's
-                   segment rows are in token order.
+* MoE router logits: [T, E] ~ N(0, 1) in fp32 (``torch.randn`` on a seeded generator).  Routing
+                   them (top-8, grouping by expert) is arithmetic of the MoE steps: the library's
+                   kernels do it on the GPU (include/bi_moe.h), the oracle on the CPU.
 
 Bits are returned as torch tensors (``torch.int16`` views for bf16, ``torch.uint8`` for e4m3)
 on the requested device; ``to_numpy_bits`` gives the host copies the oracle takes.
 """
 from __future__ import annotations
-
-from dataclasses import dataclass
 
 import numpy as np
 import torch
@@ -135,63 +132,6 @@ def to_numpy_bits(t: torch.Tensor) -> np.ndarray:
     if t.dtype == torch.int32:
         return t.detach().cpu().numpy()
     raise TypeError(f"unsupported dtype {t.dtype}")
-
-
-# ---------------------------------------------------------------------------------------------
-# MoE routing (harness preparation for the grouped GEMM)
-# ---------------------------------------------------------------------------------------------
-
-@dataclass
-class Routing:
-    """Result of routing T tokens to experts, grouped by expert."""
-    num_experts: int
-    token_of_row: torch.Tensor     # int64 [R]: which token each grouped row comes from
-    expert_of_row: torch.Tensor    # int64 [R]
-    offsets: torch.Tensor          # int32 [E+1], offsets[0] = 0, offsets[E] = R
-
-    @property
-    def rows(self) -> int:
-        return int(self.token_of_row.numel())
-
-
-def route_topk(logits: torch.Tensor, top_k: int = 8) -> torch.Tensor:
-    """Top-k experts per token by logit, ties to the lower expert index.  Returns int64 [T,k]."""
-    order = torch.sort(-logits, dim=1, stable=True).indices
-    return order[:, :top_k].contiguous()
-
-
-def group_by_expert(experts: torch.Tensor, num_experts: int) -> Routing:
-    """Stable-sort the (token, slot) pairs of ``experts`` [T, k] by expert id."""
-    T, k = experts.shape
-    flat = experts.reshape(-1).to(torch.int64)
-    tokens = torch.arange(T, device=experts.device, dtype=torch.int64).repeat_interleave(k)
-    order = torch.sort(flat, stable=True).indices
-    expert_of_row = flat[order]
-    token_of_row = tokens[order]
-    counts = torch.bincount(expert_of_row, minlength=num_experts)
-    offsets = torch.zeros(num_experts + 1, dtype=torch.int64, device=experts.device)
-    offsets[1:] = torch.cumsum(counts, 0)
-    return Routing(num_experts, token_of_row, expert_of_row, offsets.to(torch.int32))
-
-
-def softmax_top8_routing(T: int, num_experts: int, seed: int, device="cpu") -> Routing:
-    """Router logits ~ N(0,1) [T, E]; top-8 per token; grouped by expert."""
-    g = generator(seed, device)
-    logits = torch.randn(T, num_experts, generator=g, device=device, dtype=torch.float32)
-    return group_by_expert(route_topk(logits, 8), num_experts)
-
-
-def routing_from_assignment(experts_per_row: np.ndarray, num_experts: int,
-                            token_of_row: np.ndarray | None = None) -> Routing:
-    """Build a routing from an explicit expert id per row (rows already grouped by expert)."""
-    e = np.asarray(experts_per_row, dtype=np.int64)
-    assert np.all(np.diff(e) >= 0), "rows must already be grouped by expert"
-    counts = np.bincount(e, minlength=num_experts)
-    offsets = np.zeros(num_experts + 1, dtype=np.int64)
-    offsets[1:] = np.cumsum(counts)
-    tok = np.arange(e.size) if token_of_row is None else np.asarray(token_of_row)
-    return Routing(num_experts, torch.from_numpy(tok.astype(np.int64)),
-                   torch.from_numpy(e), torch.from_numpy(offsets.astype(np.int32)))
 
 
 # ---------------------------------------------------------------------------------------------

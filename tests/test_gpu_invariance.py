@@ -9,6 +9,7 @@ import torch
 
 import invariant_deterministic_gemm_bi_b200 as bg
 from invariant_deterministic_gemm_bi_b200 import inputs
+from tests import routing as routing_mod
 from tests.gpu_util import kblock_major_scales
 
 pytestmark = pytest.mark.gpu
@@ -196,10 +197,10 @@ def test_moe_rows_invariant_to_t_and_routing():
     # each test token alone (T = 1): its 8 (token, expert) rows
     g = inputs.generator(test_logits_seed, DEV)
     test_logits = torch.randn(16, E, generator=g, device=DEV)
-    test_experts = inputs.route_topk(test_logits, 8)
+    test_experts = routing_mod.topk_experts(test_logits, 8)
     ref = {}
     for i in range(16):
-        r = inputs.group_by_expert(test_experts[i:i + 1].cpu(), E)
+        r = routing_mod.route(test_logits[i:i + 1], E, 8)
         out = pair_bits(moe_outputs(plan, B, test_tokens[i:i + 1], r), r)
         for (t, e), v in out.items():
             ref[(i, e)] = v
@@ -210,7 +211,7 @@ def test_moe_rows_invariant_to_t_and_routing():
         pos = np.random.default_rng(T).choice(T, size=16, replace=False)
         tokens[torch.from_numpy(pos).to(DEV)] = test_tokens
         logits[torch.from_numpy(pos).to(DEV)] = test_logits
-        r = inputs.group_by_expert(inputs.route_topk(logits, 8).cpu(), E)
+        r = routing_mod.route(logits, E, 8)
         out = pair_bits(moe_outputs(plan, B, tokens, r), r)
         for i, p in enumerate(pos):
             for e in test_experts[i].tolist():
@@ -230,12 +231,12 @@ def test_moe_adversarial_routings(pattern):
     else:
         experts = np.concatenate([np.arange(8), np.full(392, 7)])
     experts = np.sort(experts)
-    r = inputs.routing_from_assignment(experts, E)
+    r = routing_mod.routing_from_assignment(experts, E)
     C = moe_outputs(plan, B, tokens, r)
     # every row equals the same token computed alone with its expert (a one-row call)
     for i in np.random.default_rng(1).choice(400, 40, replace=False):
         e = int(experts[i])
-        one = inputs.routing_from_assignment(np.array([e]), E)
+        one = routing_mod.routing_from_assignment(np.array([e]), E)
         C1 = moe_outputs(plan, B, tokens[i:i + 1], one)
         assert torch.equal(C1[0], C[i]), f"{pattern}: row {i}"
     # and the same as a dense call with that expert's weights, where the two plans share a tile

@@ -13,6 +13,7 @@ import torch
 import invariant_deterministic_gemm_bi_b200 as bg
 import oracle
 from invariant_deterministic_gemm_bi_b200 import inputs
+from tests import routing as routing_mod
 from tests import parity
 from tests.gpu_util import GuardedC, kblock_major_scales, strided_rows
 
@@ -255,7 +256,7 @@ def test_grouped_integers_bit_exact_wide_tile():
 @pytest.mark.parametrize("T", [1, 64, 8192])
 def test_grouped_full_size_sampled_rows(T):
     E, N, K = 64, 2048, 7168
-    routing = inputs.softmax_top8_routing(T, E, seed=5200 + T)
+    routing = routing_mod.softmax_top8_routing(T, E, seed=5200 + T)
     tokens = inputs.bf16_gaussian((T, K), seed=5201 + T, device=DEV)
     B = inputs.bf16_gaussian((E, N, K), seed=5202, std=K ** -0.5, device=DEV)
     A = tokens[routing.token_of_row.to(DEV)].contiguous()

@@ -16,6 +16,7 @@ import torch
 import oracle
 from invariant_deterministic_gemm_bi_b200 import inputs
 from tests import exact, golden_io
+from tests import routing as routing_mod
 
 
 def bf16_bits(x):
@@ -270,7 +271,9 @@ def test_grouped_rejects_malformed_offsets(bad):
 
 
 def test_routing_is_stable_top8_grouped_by_expert():
-    r = inputs.softmax_top8_routing(T=50, num_experts=64, seed=5)
+    """The grouped-GEMM tests' routing helper (built on the oracle's MoE steps) groups every token's
+    top-8 experts by expert, token order inside a segment, no duplicates, ties to the lower id."""
+    r = routing_mod.softmax_top8_routing(T=50, num_experts=64, seed=5)
     off = r.offsets.numpy()
     assert off[0] == 0 and off[-1] == 400 and np.all(np.diff(off) >= 0)
     e = r.expert_of_row.numpy()
@@ -279,6 +282,11 @@ def test_routing_is_stable_top8_grouped_by_expert():
         seg = slice(off[x], off[x + 1])
         assert np.all(e[seg] == x)
         assert np.all(np.diff(t[seg]) > 0)   # token order inside a segment, no duplicates
+    # every token appears exactly 8 times, with its 8 largest logits
+    g = inputs.generator(5, "cpu")
+    logits = torch.randn(50, 64, generator=g, dtype=torch.float32).numpy()
+    for tok in range(50):
+        experts = sorted(e[t == tok].tolist())
+        assert experts == sorted(np.argsort(-logits[tok], kind="stable")[:8].tolist())
     # ties go to the lower expert index
-    logits = torch.zeros(1, 16)
-    assert inputs.route_topk(logits, 8).tolist() == [list(range(8))]
+    assert routing_mod.topk_experts(torch.zeros(1, 16), 8).tolist() == [list(range(8))]
