@@ -92,7 +92,12 @@ typedef struct {
     int mma_m, mma_n, mma_k;   /* tcgen05.mma instruction shape */
     int stages;                /* depth of the B (weight) shared-memory ring */
     int k_order_id;            /* 0 = ascending K blocks, whole K per CTA, no split-K;
-                                  1 = fixed split-K research plan (see bi_gemm_plan_splitk) */
+                                  1 = fixed split-K research plan (see bi_gemm_plan_splitk);
+                                  2 = whole K per CTA in two fixed interleaved chains: the
+                                      128-byte K chunks 0, 2, 4, ... and 1, 3, 5, ... are each
+                                      accumulated in ascending K, then C = chain0 + chain1 once
+                                      (dense bf16 plans of 32-column tiles).  Fixed by K alone:
+                                      the same for every M, row position and scheduling form. */
     int threads_per_cta;
     int smem_bytes;            /* dynamic shared memory per CTA */
     int tmem_columns;          /* tensor-memory columns allocated per CTA */

@@ -46,36 +46,46 @@ struct KernelEntry {
     int nsplit;    // MMAs per K step (MMA N = bn / nsplit)
     bool ksplit;   // fixed-split-K research variant (fp32 partials + merge)
     bool w4;       // e2m1 weights with per-column scale and zero point (with fp8)
+    int chains;    // K chains of a dense bf16 tile (2: chunks of each parity summed apart, then added)
 };
 
 #define BI_ENTRY(BM, BN, KC, F8, GR)                                                               \
     KernelEntry{bi::Issue<F8, BN, 1, GR, KC>::kThreads, BM, BN, KC, F8, GR, false,                              \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, GR>,                                           \
-                bi::smem_bytes_for<BM, BN, KC, F8, GR>(), 1, false, false}
+                bi::smem_bytes_for<BM, BN, KC, F8, GR>(), 1, false, false, 1}
 #define BI_ENTRY_W4(BM, BN, KC)                                                                    \
     KernelEntry{bi::Issue<true, BN, 1, false, KC>::kThreads, BM, BN, KC, true, false, false,                       \
                 &bi::bi_gemm_kernel<BM, BN, KC, true, false, 1, false, true>,                      \
-                bi::smem_bytes_for<BM, BN, KC, true, false, 1, false, true>(), 1, false, true}
+                bi::smem_bytes_for<BM, BN, KC, true, false, 1, false, true>(), 1, false, true, 1}
 #define BI_ENTRY_W4_SPLIT2(BM, BN, KC)                                                             \
     KernelEntry{bi::Issue<true, BN, 2, false, KC>::kThreads, BM, BN, KC, true, false, false,                       \
                 &bi::bi_gemm_kernel<BM, BN, KC, true, false, 2, false, true>,                      \
-                bi::smem_bytes_for<BM, BN, KC, true, false, 2, false, true>(), 2, false, true}
+                bi::smem_bytes_for<BM, BN, KC, true, false, 2, false, true>(), 2, false, true, 1}
 #define BI_ENTRY_KSPLIT(BM, BN, KC)                                                                \
     KernelEntry{bi::Issue<false, BN, 1, false, KC>::kThreads, BM, BN, KC, false, false, false,                     \
                 &bi::bi_gemm_kernel<BM, BN, KC, false, false, 1, true>,                            \
-                bi::smem_bytes_for<BM, BN, KC, false, false, 1, true>(), 1, true, false}
+                bi::smem_bytes_for<BM, BN, KC, false, false, 1, true>(), 1, true, false, 1}
 #define BI_ENTRY_SPLIT2(BM, BN, KC, F8)                                                            \
     KernelEntry{bi::Issue<F8, BN, 2, false, KC>::kThreads, BM, BN, KC, F8, false, false,                           \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, false, 2>,                                     \
-                bi::smem_bytes_for<BM, BN, KC, F8, false, 2>(), 2, false, false}
+                bi::smem_bytes_for<BM, BN, KC, F8, false, 2>(), 2, false, false, 1}
 #define BI_ENTRY_GROUPED_SPLIT2(BM, BN, KC)                                                        \
     KernelEntry{bi::Issue<false, BN, 2, true, KC>::kThreads, BM, BN, KC, false, true, false,                      \
                 &bi::bi_gemm_kernel<BM, BN, KC, false, true, 2>,                                   \
-                bi::smem_bytes_for<BM, BN, KC, false, true, 2>(), 2, false, false}
+                bi::smem_bytes_for<BM, BN, KC, false, true, 2>(), 2, false, false, 1}
 #define BI_PAIR(BN, KC, F8, GR)                                                                    \
     KernelEntry{bi::Epi<F8, BN>::kThreads, 256, BN, KC, F8, GR, true,                              \
                 &bi::bi_gemm_kernel_pair<BN, KC, F8, GR>,                                          \
-                bi::smem_bytes_for_pair<BN, KC, F8, GR>(), 1, false, false}
+                bi::smem_bytes_for_pair<BN, KC, F8, GR>(), 1, false, false, 1}
+
+#define BI_ENTRY_CH2(BM, BN, KC)                                                                   \
+    KernelEntry{bi::Issue<false, BN, 1, false, KC, 2>::kThreads, BM, BN, KC, false, false, false,   \
+                &bi::bi_gemm_kernel<BM, BN, KC, false, false, 1, false, false, 2>,                 \
+                bi::smem_bytes_for<BM, BN, KC, false, false, 1, false, false, 2>(), 1, false, false, 2}
+#define BI_ENTRY_CH2_SPLIT2(BM, BN, KC)                                                            \
+    KernelEntry{bi::Issue<false, BN, 2, false, KC, 2>::kThreads, BM, BN, KC, false, false, false,   \
+                &bi::bi_gemm_kernel<BM, BN, KC, false, false, 2, false, false, 2>,                 \
+                bi::smem_bytes_for<BM, BN, KC, false, false, 2, false, false, 2>(), 2, false, false, 2}
 
 // Narrow tiles (BN <= 64) run on one CTA; wide ones (BN >= 128) on a CTA pair.  Every tile comes
 // in two forms: its preferred number of 128-byte K chunks per pipeline stage (3-D TMA boxes;
@@ -84,10 +94,12 @@ struct KernelEntry {
 // chunks per stage (the bf16 tile a fourth, tiny-batch form with 16), and a wide form that runs
 // two adjacent tiles in lockstep on one A operand (see dense_kernel_for).
 const KernelEntry kKernels[] = {
-    BI_ENTRY(64, 32, 1, false, false),  BI_ENTRY(64, 32, 4, false, false),
-    BI_ENTRY(128, 32, 1, false, false), BI_ENTRY(128, 32, 4, false, false),
-    BI_ENTRY(128, 32, 8, false, false), BI_ENTRY(128, 32, 16, false, false),
-    BI_ENTRY_SPLIT2(128, 64, 2, false),
+    // bf16 32-column tiles: 64-row MMA, two K chains on two issuing threads (the plan form, the
+    // small- and tiny-batch forms, one chunk per stage for K not a multiple of 64, and the wide
+    // lockstep form)
+    BI_ENTRY_CH2(64, 32, 1),            BI_ENTRY_CH2(64, 32, 4),
+    BI_ENTRY_CH2(64, 32, 8),            BI_ENTRY_CH2(64, 32, 16),
+    BI_ENTRY_CH2_SPLIT2(64, 64, 4),
     BI_ENTRY(128, 64, 1, false, false), BI_ENTRY(128, 64, 2, false, false),
     BI_ENTRY(128, 32, 1, true, false),  BI_ENTRY(128, 32, 4, true, false),
     BI_ENTRY(128, 64, 1, true, false),  BI_ENTRY(128, 64, 2, true, false),
@@ -111,12 +123,13 @@ constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
 
 int preferred_chunks(int bn) { return bn <= 32 ? 4 : 2; }
 
-const KernelEntry *find_kernel(int bm, int bn, int kc, bool fp8, bool grouped, bool w4 = false)
+const KernelEntry *find_kernel(int bm, int bn, int kc, bool fp8, bool grouped, bool w4 = false,
+                               int chains = 1)
 {
     for (int i = 0; i < kNumKernels; ++i)
         if (kKernels[i].bm == bm && kKernels[i].bn == bn && kKernels[i].kc == kc &&
             kKernels[i].fp8 == fp8 && kKernels[i].grouped == grouped && kKernels[i].nsplit == 1 &&
-            !kKernels[i].ksplit && kKernels[i].w4 == w4)
+            !kKernels[i].ksplit && kKernels[i].w4 == w4 && kKernels[i].chains == chains)
             return &kKernels[i];
     return nullptr;
 }
@@ -166,9 +179,10 @@ RingGeom ring_geometry(const KernelEntry *k, int a_rows)
     // The kernel relies on 2 <= sa <= sb (the A-slot reuse test reads the consumed ring) and, for
     // FP8, on sb groups outlasting the partial-product ring.  Every tile in kKernels satisfies
     // this for every a_rows in [8, BM], except the small-batch forms, which are valid up to 64
-    // (bf16, 8 chunks) and 96 (FP8, 4 chunks) rows and used up to kSmallBatchRows = 64, and the
-    // bf16 tiny-batch form (16 chunks), valid and used up to 8 rows; set_rows reports a violation
-    // and the launch is refused.  tests/test_abi.py checks the reported depths.
+    // (bf16, 8 chunks) and 96 (FP8, 4 chunks) rows and used up to bi_plan_s::small_rows (64; 32
+    // for two-chain bf16 plans), and the bf16 tiny-batch form (16 chunks), valid and used up to 8
+    // rows; set_rows reports a violation and the launch is refused.  tests/test_abi.py checks the
+    // reported depths.
     return RingGeom{sa, sb, static_cast<uint32_t>(a_stride), static_cast<uint32_t>(a_region)};
 }
 
@@ -192,10 +206,10 @@ TileChoice choose_tile(int64_t N, int64_t K, bi_dtype_t dtype, int experts)
         int dtype, experts, bm, bn;
     };
     static const Row table[] = {
-        {4096, 7168, BI_DTYPE_BF16, 1, 128, 32},              // decode-shaped projection
+        {4096, 7168, BI_DTYPE_BF16, 1, 64, 32},               // decode-shaped projection
         {7168, 2048, BI_DTYPE_BF16, 1, 256, 256},             // prefill-shaped, wide N (CTA pair)
         {2048, 7168, BI_DTYPE_BF16, 1, 256, 256},             // prefill-shaped, long K (CTA pair)
-        {256, 512, BI_DTYPE_BF16, 1, 128, 32},                // small correctness shape
+        {256, 512, BI_DTYPE_BF16, 1, 64, 32},                 // small correctness shape
         {7168, 7168, BI_DTYPE_E4M3_BLOCKSCALED, 1, 128, 64},  // FP8 projection
         {7168, 7168, BI_DTYPE_E2M1_W4A8, 1, 128, 64},         // the same projection, e2m1 weights
         {2048, 7168, BI_DTYPE_BF16, 64, 128, 128},            // MoE experts
@@ -219,7 +233,7 @@ TileChoice choose_tile(int64_t N, int64_t K, bi_dtype_t dtype, int experts)
             return {256, bn};
     if ((N + 63) / 64 >= 100)
         return {128, 64};
-    return {128, 32};
+    return {dtype == BI_DTYPE_BF16 ? 64 : 128, 32};
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -306,6 +320,7 @@ struct bi_plan_s {
     // order), for dense launches with more tiles than SMs and grouped launches with at least a
     // tile's worth of rows per expert on average.  May be null.
     const KernelEntry *kernel_wide = nullptr;
+    int small_rows = 64;     // kernel_small serves launches whose A boxes hold at most this many rows
     uint64_t timeout_ns = 2000000000ull;
     uint32_t debug_flags = 0;
     uint32_t flags = 0;      // BI_PLAN_* flags
@@ -503,6 +518,14 @@ bi_status_t check_fp8_scales(int64_t M, const float *scale_a, int64_t ld_sa, con
     return BI_OK;
 }
 
+// Dense bf16 plans of 32-column tiles use the 64-row MMA with two K chains: with two issuing
+// threads the 64 x 32 x 16 instruction issues at ~29 cycles (one thread: ~57 cycles, whatever the
+// shape), and it reads half the shared-memory A rows of the 128-row one.
+int chains_for(const TileChoice &tile, bool fp8, int experts)
+{
+    return (!fp8 && experts == 1 && tile.bm == 64 && tile.bn == 32) ? 2 : 1;
+}
+
 // Rows of A one TMA load brings for a dense problem of M rows: the tile's 128 rows, or, when the
 // problem is smaller than one tile, only the rows that exist (rounded up to the 8-row swizzle
 // atom).  This changes which shared-memory rows are written, not the MMA or its K order.
@@ -604,13 +627,12 @@ int b_box_rows_for(const KernelEntry *k)
     return k->pair ? k->bn / 2 : k->bn;
 }
 
-// A dense launch of M rows whose A boxes hold at most this many rows takes the plan's
+// A dense launch of M rows whose A boxes hold at most bi_plan_s::small_rows rows takes the plan's
 // small-batch kernel form (when it has one): with few A rows, groups of twice the chunks halve
-// the per-group wait and commit overhead of the MMA thread, and the ring still holds two groups
-// of A and of B (and, for FP8, more groups than partial-product buffers).
-constexpr int kSmallBatchRows = 64;
-// ... and at most this many rows, the tiny-batch form (16 chunks per group): the 8-row A boxes
-// leave room for two 64 KB groups of B.
+// the per-group wait and commit overhead of the MMA threads, and the ring still holds two groups
+// of A and of B (and, for FP8, more groups than partial-product buffers).  At most this many
+// rows take the tiny-batch form (16 chunks per group): the 8-row A boxes leave room for two
+// 64 KB groups of B.
 constexpr int kTinyBatchRows = 8;
 
 // A dense launch with more tiles than the device has SMs takes the plan's wide form (when it has
@@ -620,7 +642,7 @@ const KernelEntry *dense_kernel_for(const bi_plan_s *plan, const DeviceInfo *d, 
 {
     if (plan->kernel_tiny && a_box_rows_for(plan->kernel_tiny, M) <= kTinyBatchRows)
         return plan->kernel_tiny;
-    if (plan->kernel_small && a_box_rows_for(plan->kernel_small, M) <= kSmallBatchRows)
+    if (plan->kernel_small && a_box_rows_for(plan->kernel_small, M) <= plan->small_rows)
         return plan->kernel_small;
     if (plan->kernel_wide) {
         const int64_t tiles = (M + plan->kernel->bm - 1) / plan->kernel->bm *
@@ -711,7 +733,8 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     const TileChoice tile = choose_tile(N, K, dtype, num_experts);
     const int chunk_elems = fp8 ? 128 : 64;
     const int kc = ((K > 0 && K % chunk_elems == 0) || w4) ? preferred_chunks(tile.bn) : 1;
-    const KernelEntry *k = find_kernel(tile.bm, tile.bn, kc, fp8, num_experts > 1, w4);
+    const int chains = chains_for(tile, fp8, num_experts);
+    const KernelEntry *k = find_kernel(tile.bm, tile.bn, kc, fp8, num_experts > 1, w4, chains);
     if (!k)
         return BI_ERR_UNSUPPORTED_SHAPE;
     bi_plan_s *p = new (std::nothrow) bi_plan_s();
@@ -722,21 +745,25 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     p->dtype = dtype;
     p->experts = num_experts;
     p->kernel = k;
-    if (num_experts == 1 && !k->pair && k->bm == 128 && k->kc == preferred_chunks(k->bn) &&
-        k->bn == (fp8 ? 64 : 32))
-        p->kernel_small = find_kernel(128, k->bn, 2 * k->kc, fp8, false, w4);
+    if (num_experts == 1 && !k->pair && (k->bm == 128 || k->chains == 2) &&
+        k->kc == preferred_chunks(k->bn) && k->bn == (fp8 ? 64 : 32))
+        p->kernel_small = find_kernel(k->bm, k->bn, 2 * k->kc, fp8, false, w4, chains);
     if (p->kernel_small && !fp8 && p->kernel_small->kc == 8)
-        p->kernel_tiny = find_kernel(128, k->bn, 16, false, false, false);
+        p->kernel_tiny = find_kernel(k->bm, k->bn, 16, false, false, false, chains);
+    // two-chain plans take the 8-chunk form up to 32 rows: their 64-row A boxes would leave a
+    // 64 KB B ring at 8 chunks, while 4 chunks keep six B groups in flight
+    p->small_rows = chains == 2 ? 32 : 64;
     if (num_experts > 1 && !k->pair && k->bm == 128 && k->bn == 128) {
         for (int i = 0; i < kNumKernels; ++i)
             if (kKernels[i].nsplit == 2 && kKernels[i].grouped && kKernels[i].bn == 256)
                 p->kernel_wide = &kKernels[i];
     }
-    if (num_experts == 1 && !k->pair && k->bm == 128 && k->bn == (fp8 ? 64 : 32) &&
-        K % chunk_elems == 0) {
+    if (num_experts == 1 && !k->pair && (k->bm == 128 || k->chains == 2) &&
+        k->bn == (fp8 ? 64 : 32) && K % chunk_elems == 0 && K > 0) {
         for (int i = 0; i < kNumKernels; ++i)
-            if (kKernels[i].nsplit == 2 && kKernels[i].bm == 128 && kKernels[i].bn == 2 * k->bn &&
-                kKernels[i].fp8 == fp8 && kKernels[i].w4 == w4 && !kKernels[i].grouped)
+            if (kKernels[i].nsplit == 2 && kKernels[i].bm == k->bm && kKernels[i].bn == 2 * k->bn &&
+                kKernels[i].fp8 == fp8 && kKernels[i].w4 == w4 && !kKernels[i].grouped &&
+                kKernels[i].chains == chains)
                 p->kernel_wide = &kKernels[i];
     }
     *out = p;
@@ -782,13 +809,13 @@ bi_status_t bi_gemm_plan_describe(bi_plan_t plan, bi_plan_info_t *info)
     const RingGeom g = ring_geometry(plan->kernel, plan->kernel->bm);
     info->stages = g.sb;
     info->stages_a = g.sa;
-    info->k_order_id = plan->k_splits > 1 ? 1 : 0;
+    info->k_order_id = plan->k_splits > 1 ? 1 : plan->kernel->chains == 2 ? 2 : 0;
     info->k_splits = plan->k_splits;
     info->threads_per_cta = plan->kernel->threads;
     info->smem_bytes = plan->kernel->smem;
     const int nacc = fp8 ? ((512 / plan->kernel->bn) < 8 ? (512 / plan->kernel->bn) : 8) : 2;
     int cols = 32;
-    while (cols < nacc * plan->kernel->bn)
+    while (cols < nacc * plan->kernel->bn * plan->kernel->chains)
         cols *= 2;
     info->tmem_columns = cols;
     return BI_OK;

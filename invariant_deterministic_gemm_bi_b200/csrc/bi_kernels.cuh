@@ -73,12 +73,15 @@ struct Epi {
 //   - by K-chunk parity, in the other dense FP8 forms with an even number of chunks per group: each
 //     128-wide K chunk has its own partial-product buffer, and the epilogue promotes the buffers in
 //     ascending kb whoever issued them.
+//   - by K-chunk parity in the dense bf16 kernels with two K chains (CH = 2, any NSPLIT): chain p
+//     accumulates the chunks of parity p into an accumulator of its own, and the epilogue adds
+//     the two chains once.
 // The grouped wide form (two 128 x 128 instructions per K step) is bound by shared-memory bandwidth
 // instead and keeps one issuer.  The second issuer is the warp after the epilogue warps.
-template <bool FP8, int BN, int NSPLIT, bool GROUPED = false, int KC = 1>
+template <bool FP8, int BN, int NSPLIT, bool GROUPED = false, int KC = 1, int CH = 1>
 struct Issue {
-    static constexpr bool kBySplit = !GROUPED && NSPLIT == 2;
-    static constexpr bool kByChunk = FP8 && !GROUPED && NSPLIT == 1 && KC % 2 == 0;
+    static constexpr bool kByChunk = !GROUPED && KC % 2 == 0 && (FP8 ? NSPLIT == 1 : CH == 2);
+    static constexpr bool kBySplit = !GROUPED && NSPLIT == 2 && !kByChunk;
     static constexpr int kIssuers = (kBySplit || kByChunk) ? 2 : 1;
     static constexpr int kSecondWarp = 2 + Epi<FP8, BN>::kWarps;
     static constexpr int kThreads = Epi<FP8, BN>::kThreads + (kIssuers - 1) * 32;
@@ -507,6 +510,12 @@ __global__ void __launch_bounds__(256) bi_w4_rowsum_kernel(const uint8_t *a, int
 // SPLIT   : the fixed-split-K research variant (bf16 dense only, not the batch-invariant product
 //           path): a work unit is one K split of a tile and its epilogue writes fp32 partial
 //           sums; bi_splitk_merge_kernel adds the splits in a fixed order.
+// CH      : K chains of a dense bf16 tile, 1 or 2.  With 2, the 128-byte K chunks of even index
+//           are accumulated, in ascending K, into one accumulator and those of odd index into a
+//           second one, each by its own issuing thread, and the epilogue forms
+//           C = bf16_rne(chain0 + chain1) once (chain0 alone when K has one chunk).  The order is
+//           fixed by K alone -- the same for every M, row and scheduling form -- and stays inside
+//           one CTA: no workspace, no atomics, no cross-CTA reduction.
 // W4      : (with FP8, dense) B holds e2m1 weights with one power-of-two scale and one zero point
 //           per output column ("DeepSeek V4的batch invariance：大模型确定性推理的工程基石"
 //           (lshu.cn), section 4.3: W = W_fp4 * scale + zero, scale in {2^-j : j = 1..12}).  The
@@ -517,8 +526,8 @@ __global__ void __launch_bounds__(256) bi_w4_rowsum_kernel(const uint8_t *a, int
 //           the K sum changes no rounding.
 // The ring depths follow from (BM, BN, KC) (see Rings).
 template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool SPLIT = false,
-          bool W4 = false>
-__global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC>::kThreads, 1)
+          bool W4 = false, int CH = 1>
+__global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThreads, 1)
     bi_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_a8, const GemmParams p)
@@ -534,8 +543,9 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC>::kThreads,
                   "two half-width instructions");
     static_assert(!SPLIT || (!FP8 && !GROUPED && NSPLIT == 1), "split-K variant: bf16 dense");
     static_assert(!W4 || (FP8 && !GROUPED && !SPLIT), "e2m1 weights: the dense FP8 kernel");
+    static_assert(CH == 1 || (CH == 2 && !FP8 && !GROUPED && !SPLIT), "two K chains: dense bf16");
     constexpr int kMmaN = BN / NSPLIT;                   // MMA instruction N
-    using Iss = Issue<FP8, BN, NSPLIT, GROUPED, KC>;
+    using Iss = Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>;
     constexpr int kIssuers = Iss::kIssuers;              // threads issuing MMAs
     using R = Rings<BM, BN, KC>;
     constexpr int kElemsPerRow = FP8 ? 128 : 64;         // K elements per 128-byte row
@@ -546,7 +556,8 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC>::kThreads,
     // TMEM buffers: bf16 double-buffers the accumulator; FP8 rings kNumAcc partial products
     // (one per K chunk, at least two groups' worth so the promotion overlaps the next group).
     constexpr int kNumAcc = FP8 ? ((512 / BN) < 8 ? (512 / BN) : 8) : 2;
-    constexpr int kTmemColsNeeded = kNumAcc * BN;
+    constexpr int kAccCols = FP8 ? BN : CH * BN;         // columns of one buffer (bf16: CH chains)
+    constexpr int kTmemColsNeeded = kNumAcc * kAccCols;
     constexpr uint32_t kTmemCols = kTmemColsNeeded <= 32    ? 32
                                    : kTmemColsNeeded <= 64  ? 64
                                    : kTmemColsNeeded <= 128 ? 128
@@ -855,7 +866,7 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC>::kThreads,
                         break;
                     }
                     ptx::tc_fence_after_sync();
-                    d_tmem = tmem_base + a * BN;
+                    d_tmem = tmem_base + a * kAccCols;
                 }
                 // chunks and groups of this work unit (the whole K of a tile, or one K split)
                 int unit_nkb = nkb, unit_nkg = nkg;
@@ -893,13 +904,16 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC>::kThreads,
                         uint32_t d = d_tmem;
                         if constexpr (FP8)   // chunk c of the group has partial buffer acc_iter + c
                             d = tmem_base + ((acc_iter + static_cast<uint32_t>(c)) % kNumAcc) * BN;
+                        else if constexpr (CH == 2)   // the chain of the chunk's parity
+                            d = d_tmem + static_cast<uint32_t>(chunk & 1) * BN;
                         const uint64_t a_desc = a_slot + ((c * a_cp) >> 4);
                         const uint64_t b_desc = b_slot + ((c * R::kBChunkBytes) >> 4);
 #pragma unroll
                         for (int q = 0; q < kMmaPerStage; ++q) {
                             const uint64_t step = static_cast<uint64_t>((q * kBytesPerMmaK) >> 4);
-                            // bf16: accumulate across the whole K of the tile; FP8: one K chunk
-                            const uint32_t accumulate = (q > 0) ? 1u : (FP8 ? 0u : (chunk > 0 ? 1u : 0u));
+                            // bf16: accumulate across the whole K of the tile (of the chunk's
+                            // chain); FP8: one K chunk
+                            const uint32_t accumulate = (q > 0) ? 1u : (FP8 ? 0u : (chunk >= CH ? 1u : 0u));
 #pragma unroll
                             for (int j = 0; j < kSplitsPerIssuer; ++j) {
                                 // split sp: B rows and accumulator columns [sp kMmaN, (sp+1) kMmaN)
@@ -983,17 +997,31 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC>::kThreads,
                 ptx::tc_fence_after_sync();
 #pragma unroll 1
                 for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t r[32];
-                    ptx::tmem_ld_32x32b_x32(tmem_base + lane_addr + a * BN + c * 32, r);
+                    uint32_t r[32], r1[32];
+                    const uint32_t col = tmem_base + lane_addr + a * kAccCols + c * 32;
+                    ptx::tmem_ld_32x32b_x32(col, r);
+                    if constexpr (CH == 2)
+                        ptx::tmem_ld_32x32b_x32(col + BN, r1);
                     ptx::tmem_wait_ld(r);
+                    if constexpr (CH == 2)
+                        ptx::tmem_wait_ld(r1);
                     if (c == BN / 32 - 1) {
                         ptx::tc_fence_before_sync();
                         ptx::mbar_arrive(&acce_bar[a]);   // accumulator free for the next tile
                     }
                     float v[32];
+                    if constexpr (CH == 2) {
+                        // C = chain 0 + chain 1, once, in this order (one chunk: chain 0 alone)
+                        const bool two = nkb > 1;
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj)
-                        v[jj] = __uint_as_float(r[jj]);
+                        for (int jj = 0; jj < 32; ++jj)
+                            v[jj] = two ? __uint_as_float(r[jj]) + __uint_as_float(r1[jj])
+                                        : __uint_as_float(r[jj]);
+                    } else {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            v[jj] = __uint_as_float(r[jj]);
+                    }
                     if (row_ok) {
                         if constexpr (SPLIT)
                             store_row_chunk32_f32(p.ws + tc.split * p.ws_split_stride +
@@ -1134,7 +1162,7 @@ __global__ void bi_splitk_merge_kernel(const float *ws, int64_t ld_ws, int64_t s
 }
 
 template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool SPLIT = false,
-          bool W4 = false>
+          bool W4 = false, int CH = 1>
 constexpr int smem_bytes_for()
 {
     return 1024 + kRingBytes + 1024 + (GROUPED ? 2 * (kMaxExperts + 1) * 4 : 0);

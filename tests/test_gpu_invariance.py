@@ -103,23 +103,24 @@ def test_decode_rows_invariant_across_m_sweep():
 
 
 def test_scheduling_forms_of_one_plan_agree_bitwise():
-    # One 128x32 plan, ragged in N (the last 64-column lockstep pair is half outside N) and in K
-    # (113 chunks: the last 2-chunk group is short).  M = 1 takes the small-batch form, M = 100
-    # the plan's own form, M = 300 (387 tiles > 148 SMs) the wide lockstep form: a row's bits must
-    # not depend on which of them ran it.
+    # One 64x32 two-chain plan, ragged in N (the last 64-column lockstep pair is half outside N)
+    # and in K (113 chunks: an odd count, so chain 0 has one chunk more than chain 1, and the last
+    # group of every form is short).  M = 1 takes the tiny-batch form (16 chunks per stage), M = 20
+    # the small-batch form (8), M = 64 the plan's own form (4), M = 100 and 300 (258 and 645 tiles
+    # > 148 SMs) the wide lockstep form: a row's bits must not depend on which of them ran it.
     N, K = 4128, 7232
     B = inputs.bf16_gaussian((N, K), seed=2101, std=K ** -0.5, device=DEV)
     f = Dense(B)
     info = bg.bi_gemm_plan_describe(f.plan)
-    assert (info["block_m"], info["block_n"]) == (128, 32)
+    assert (info["block_m"], info["block_n"], info["k_order_id"]) == (64, 32, 2)
     test_rows = inputs.bf16_gaussian((24, K), seed=2102, device=DEV)
     ref = alone(f, test_rows)
-    for M in [100, 300]:
+    for M in [20, 64, 100, 300]:
         s = inputs.derived_seed(2100, M, 0)
         fresh = lambda m, s=s: inputs.bf16_gaussian((m, K), seed=s, device=DEV)
         check_in_batch(f, test_rows, ref, M, s, fresh)
         check_in_batch(f, test_rows, ref, M, M, fresh,
-                       positions=[q for q in (0, 127, 128, M - 1) if q < M])
+                       positions=sorted({q for q in (0, 63, 64, 127, 128, M - 1) if q < M}))
 
 
 # ---------------------------------------------------------------------------------------------

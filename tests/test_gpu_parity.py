@@ -98,15 +98,16 @@ def test_ragged_integers_bit_exact(M, N, K):
 
 
 def test_wide_lockstep_form_ragged_integers_bit_exact():
-    # 128x32 plan at M = 300: 387 tiles > 148 SMs, so pairs of adjacent tiles run in lockstep on
-    # one A operand; N = 4128 leaves the last pair half outside N, K = 7232 a short last group.
+    # 64x32 two-chain plan at M = 300: 645 tiles > 148 SMs, so pairs of adjacent tiles run in
+    # lockstep on one A operand; N = 4128 leaves the last pair half outside N, K = 7232 (113
+    # chunks) gives the chains unequal lengths and a short last group.
     M, N, K = 300, 4128, 7232
     A = inputs.bf16_integers((M, K), seed=2201, device=DEV)
     B = inputs.bf16_integers((N, K), seed=2202, device=DEV)
     C, plan = run_dense(A, B)
     info = bg.bi_gemm_plan_describe(plan)
-    assert (info["block_m"], info["block_n"]) == (128, 32)
-    rows = [0, 1, 127, 128, 200, 255, 256, 299]
+    assert (info["block_m"], info["block_n"]) == (64, 32)
+    rows = [0, 1, 63, 64, 127, 128, 200, 255, 256, 299]
     _, cbits = oracle.gemm_bf16_rows(inputs.to_numpy_bits(A), inputs.to_numpy_bits(B), rows)
     parity.assert_bits_equal_values(parity.bits(C)[rows], cbits, f"wide form {M}x{N}x{K}")
 
