@@ -82,10 +82,11 @@ struct KernelEntry {
     KernelEntry{bi::Issue<false, BN, 1, false, KC, 2>::kThreads, BM, BN, KC, false, false, false,   \
                 &bi::bi_gemm_kernel<BM, BN, KC, false, false, 1, false, false, 2>,                 \
                 bi::smem_bytes_for<BM, BN, KC, false, false, 1, false, false, 2>(), 1, false, false, 2}
-#define BI_ENTRY_CH2_SPLIT2(BM, BN, KC)                                                            \
-    KernelEntry{bi::Issue<false, BN, 2, false, KC, 2>::kThreads, BM, BN, KC, false, false, false,   \
-                &bi::bi_gemm_kernel<BM, BN, KC, false, false, 2, false, false, 2>,                 \
-                bi::smem_bytes_for<BM, BN, KC, false, false, 2, false, false, 2>(), 2, false, false, 2}
+#define BI_ENTRY_CH2_SPLITN(BM, BN, KC, NS)                                                        \
+    KernelEntry{bi::Issue<false, BN, NS, false, KC, 2>::kThreads, BM, BN, KC, false, false, false,  \
+                &bi::bi_gemm_kernel<BM, BN, KC, false, false, NS, false, false, 2>,                \
+                bi::smem_bytes_for<BM, BN, KC, false, false, NS, false, false, 2>(), NS, false,    \
+                false, 2}
 
 // Narrow tiles (BN <= 64) run on one CTA; wide ones (BN >= 128) on a CTA pair.  Every tile comes
 // in two forms: its preferred number of 128-byte K chunks per pipeline stage (3-D TMA boxes;
@@ -96,10 +97,10 @@ struct KernelEntry {
 const KernelEntry kKernels[] = {
     // bf16 32-column tiles: 64-row MMA, two K chains on two issuing threads (the plan form, the
     // small- and tiny-batch forms, one chunk per stage for K not a multiple of 64, and the wide
-    // lockstep form)
+    // lockstep forms of two and four tiles)
     BI_ENTRY_CH2(64, 32, 1),            BI_ENTRY_CH2(64, 32, 4),
     BI_ENTRY_CH2(64, 32, 8),            BI_ENTRY_CH2(64, 32, 16),
-    BI_ENTRY_CH2_SPLIT2(64, 64, 4),
+    BI_ENTRY_CH2_SPLITN(64, 64, 4, 2),  BI_ENTRY_CH2_SPLITN(64, 128, 2, 4),
     BI_ENTRY(128, 64, 1, false, false), BI_ENTRY(128, 64, 2, false, false),
     BI_ENTRY(128, 32, 1, true, false),  BI_ENTRY(128, 32, 4, true, false),
     BI_ENTRY(128, 64, 1, true, false),  BI_ENTRY(128, 64, 2, true, false),
@@ -320,6 +321,9 @@ struct bi_plan_s {
     // order), for dense launches with more tiles than SMs and grouped launches with at least a
     // tile's worth of rows per expert on average.  May be null.
     const KernelEntry *kernel_wide = nullptr;
+    // Four adjacent tiles in lockstep (two-chain plans), for dense launches whose lockstep pairs
+    // still outnumber the SMs.  May be null.
+    const KernelEntry *kernel_wide4 = nullptr;
     int small_rows = 64;     // kernel_small serves launches whose A boxes hold at most this many rows
     uint64_t timeout_ns = 2000000000ull;
     uint32_t debug_flags = 0;
@@ -577,6 +581,20 @@ GemmParams base_params(const bi_plan_s *plan, const KernelEntry *k, int64_t rows
     return p;
 }
 
+// Dense problems of fewer than 8 rows on one-CTA tiles: a 2-D map of A with boxes of exactly M
+// rows, for the kernel's per-chunk A loads (bi::GemmParams::a_exact_rows), so that no A load
+// reaches past the last row (TMA fills such rows slowly).  Leaves *map alone otherwise.
+bi_status_t exact_rows_map(const KernelEntry *k, CUtensorMap *map, const void *A, bool fp8, int64_t K,
+                           int64_t M, int64_t lda, GemmParams *p)
+{
+    if (k->pair || k->grouped || M >= 8)
+        return BI_OK;
+    const bi_status_t st = encode_operand(map, A, fp8, K, M, lda, static_cast<int>(M), 1);
+    if (st == BI_OK)
+        p->a_exact_rows = static_cast<int32_t>(M);
+    return st;
+}
+
 // Launch kernel entry k.  `units` is the number of work tiles; a one-CTA kernel gets
 // min(units, #SMs) CTAs, a pair kernel min(units, co-resident pairs) clusters of two CTAs.  Every
 // launch is a programmatic dependent of the previous kernel in the stream: it may start (and set
@@ -645,10 +663,13 @@ const KernelEntry *dense_kernel_for(const bi_plan_s *plan, const DeviceInfo *d, 
     if (plan->kernel_small && a_box_rows_for(plan->kernel_small, M) <= plan->small_rows)
         return plan->kernel_small;
     if (plan->kernel_wide) {
-        const int64_t tiles = (M + plan->kernel->bm - 1) / plan->kernel->bm *
-                              ((plan->n + plan->kernel->bn - 1) / plan->kernel->bn);
-        if (tiles > d->num_sms)
+        const int64_t m_blocks = (M + plan->kernel->bm - 1) / plan->kernel->bm;
+        const int64_t n_blocks = (plan->n + plan->kernel->bn - 1) / plan->kernel->bn;
+        if (m_blocks * n_blocks > d->num_sms) {
+            if (plan->kernel_wide4 && m_blocks * ((n_blocks + 1) / 2) > d->num_sms)
+                return plan->kernel_wide4;
             return plan->kernel_wide;
+        }
     }
     return plan->kernel;
 }
@@ -761,10 +782,13 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     if (num_experts == 1 && !k->pair && (k->bm == 128 || k->chains == 2) &&
         k->bn == (fp8 ? 64 : 32) && K % chunk_elems == 0 && K > 0) {
         for (int i = 0; i < kNumKernels; ++i)
-            if (kKernels[i].nsplit == 2 && kKernels[i].bm == k->bm && kKernels[i].bn == 2 * k->bn &&
-                kKernels[i].fp8 == fp8 && kKernels[i].w4 == w4 && !kKernels[i].grouped &&
-                kKernels[i].chains == chains)
-                p->kernel_wide = &kKernels[i];
+            if (kKernels[i].bm == k->bm && kKernels[i].fp8 == fp8 && kKernels[i].w4 == w4 &&
+                !kKernels[i].grouped && kKernels[i].chains == chains && !kKernels[i].ksplit) {
+                if (kKernels[i].nsplit == 2 && kKernels[i].bn == 2 * k->bn)
+                    p->kernel_wide = &kKernels[i];
+                if (kKernels[i].nsplit == 4 && kKernels[i].bn == 4 * k->bn)
+                    p->kernel_wide4 = &kKernels[i];
+            }
     }
     *out = p;
     return BI_OK;
@@ -892,8 +916,11 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
     p.scale_a = scale_a;
     p.ld_sa = ld_sa;
     p.scale_b = scale_b;
+    CUtensorMap ta_exact = ta;
+    if ((st = exact_rows_map(k, &ta_exact, A, fp8, plan->k, M, lda, &p)) != BI_OK)
+        return st;
     const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-    return launch_main(k, d, ta, tb, ta, p, tiles, stream);
+    return launch_main(k, d, ta, tb, ta_exact, p, tiles, stream);
 }
 
 bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *A, int64_t lda,
@@ -1073,8 +1100,11 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
         p.scale_a = fp8 ? sa_dev : nullptr;
         p.ld_sa = fp8 ? ld_sa : 0;
         p.scale_b = fp8 ? scale_b : nullptr;
+        CUtensorMap ta_exact = ta;
+        if ((st = exact_rows_map(k, &ta_exact, A_dev, fp8, plan->k, M, lda, &p)) != BI_OK)
+            return st;
         const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-        if ((st = launch_main(k, d, ta, tb, ta, p, tiles, stream)) != BI_OK)
+        if ((st = launch_main(k, d, ta, tb, ta_exact, p, tiles, stream)) != BI_OK)
             return st;
     }
     if (cudaMemcpyAsync(C_host, C_dev, static_cast<size_t>(M * ldc * 2), cudaMemcpyDeviceToHost,
@@ -1174,8 +1204,11 @@ bi_status_t bi_gemm_run_w4a8(bi_plan_t plan, int64_t M, const void *A, int64_t l
                                workspace) != cudaSuccess)
             return BI_ERR_CUDA;
     }
+    CUtensorMap ta_exact = ta;
+    if ((st = exact_rows_map(k, &ta_exact, A, true, plan->k, M, lda, &p)) != BI_OK)
+        return st;
     const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-    return launch_main(k, d, ta, tb, ta, p, tiles, stream);
+    return launch_main(k, d, ta, tb, ta_exact, p, tiles, stream);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -1268,8 +1301,11 @@ bi_status_t bi_gemm_run_splitk(bi_plan_t plan, int64_t M, const void *A, int64_t
     p.ws = static_cast<float *>(workspace);
     p.ld_ws = (plan->n + 3) / 4 * 4;
     p.ws_split_stride = M * p.ld_ws;
+    CUtensorMap ta_exact = ta;
+    if ((st = exact_rows_map(k, &ta_exact, A, false, plan->k, M, lda, &p)) != BI_OK)
+        return st;
     const int64_t units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks * plan->k_splits;
-    if ((st = launch_main(k, d, ta, tb, ta, p, units, stream)) != BI_OK)
+    if ((st = launch_main(k, d, ta, tb, ta_exact, p, units, stream)) != BI_OK)
         return st;
     const int64_t total = M * plan->n;
     const int64_t blocks = (total + 255) / 256;

@@ -103,6 +103,10 @@ struct GemmParams {
     int32_t num_experts;     // grouped: E
     int32_t raster_m;        // dense raster band height in m-blocks
     int32_t a_box_rows;      // rows of A one TMA load brings (<= BM, a multiple of 8)
+    int32_t a_exact_rows;    // dense problems of fewer than 8 rows: each K chunk of an A group
+                             // is loaded as its own 2-D box of exactly this many rows (the third
+                             // tensor map) into its 1024-byte chunk slot, so no load reaches past
+                             // the end of A (TMA fills such rows slowly); 0 otherwise
     int32_t sa, sb;          // ring depths in groups (2..kMaxSA, sa..kMaxSB)
     uint32_t a_stride;       // bytes between A slots (KC * a_box_rows * 128)
     uint32_t b_offset;       // byte offset of the B ring in the ring region
@@ -503,7 +507,8 @@ __global__ void __launch_bounds__(256) bi_w4_rowsum_kernel(const uint8_t *a, int
 //           chunks of a tile one by one in ascending K: KC changes no bit of the result.
 // NSPLIT  : MMAs per K step.  The MMA instruction is BM x (BN / NSPLIT) x K; split s covers the
 //           tile's columns [s BN/NSPLIT, (s+1) BN/NSPLIT) and accumulates into the same columns
-//           of the TMEM accumulator (FP8: of each partial-product buffer).  NSPLIT = 2 runs two
+//           of the TMEM accumulator (FP8: of each partial-product buffer).  NSPLIT = 4 (two-chain
+//           bf16 only) runs four adjacent 32-column tiles the same way.  NSPLIT = 2 runs two
 //           adjacent (BN/2)-wide tiles of a plan in lockstep on one A operand: every output
 //           element is still computed by a BM x (BN/2) x K instruction sequence in ascending K
 //           (FP8: and promoted in ascending kb), as in a (BN/2)-wide launch.
@@ -538,9 +543,10 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
     static_assert(!(FP8 && GROUPED), "grouped FP8 is not built");
     static_assert(KC >= 1 && KC <= 16, "1..16 chunks per group");
     static_assert(NSPLIT == 1 ||
-                      (NSPLIT == 2 && (GROUPED ? (!FP8 && BN == 256) : BN == (FP8 ? 128 : 64))),
+                      (NSPLIT == 2 && (GROUPED ? (!FP8 && BN == 256) : BN == (FP8 ? 128 : 64))) ||
+                      (NSPLIT == 4 && CH == 2 && BN == 128),
                   "split MMAs: dense bf16 64-wide, FP8 128-wide and grouped bf16 256-wide tiles as "
-                  "two half-width instructions");
+                  "two half-width instructions; two-chain bf16 128-wide tiles as four quarters");
     static_assert(!SPLIT || (!FP8 && !GROUPED && NSPLIT == 1), "split-K variant: bf16 dense");
     static_assert(!W4 || (FP8 && !GROUPED && !SPLIT), "e2m1 weights: the dense FP8 kernel");
     static_assert(CH == 1 || (CH == 2 && !FP8 && !GROUPED && !SPLIT), "two K chains: dense bf16");
@@ -612,7 +618,7 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
         ptx::fence_mbarrier_init();
         ptx::prefetch_tmap(&tmap_a);
         ptx::prefetch_tmap(&tmap_b);
-        if constexpr (GROUPED)
+        if (GROUPED || p.a_exact_rows > 0)
             ptx::prefetch_tmap(&tmap_a8);
     }
     if (warp == 1) {
@@ -784,7 +790,18 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
                     int nsub = 0;
                     if constexpr (GROUPED)
                         nsub = short_segment_boxes(ca.tc, kShortSegmentRows);
-                    if (nsub == 0) {
+                    if (!GROUPED && p.a_exact_rows > 0) {
+                        // fewer than 8 rows: one exact-height box per chunk that exists in K;
+                        // the chunk slot's rows past them keep stale data, which feeds only
+                        // output rows that are never stored
+                        const int first = ca.tc.kb0 + ca.kg * KC;
+                        const int left = ca.tc.kb0 + ca.tc.nkb - first;
+                        const int nc = left < KC ? left : KC;
+                        ptx::mbar_arrive_expect_tx(&full[fs], static_cast<uint32_t>(nc * p.a_exact_rows) * kRowBytes);
+                        for (int c = 0; c < nc; ++c)
+                            ptx::tma_load_2d(smem_a + as * p.a_stride + c * a_chunk_pitch, &tmap_a8, &full[fs],
+                                             (first + c) * kElemsPerRow, ca.tc.m0, pol);
+                    } else if (nsub == 0) {
                         ptx::mbar_arrive_expect_tx(&full[fs], KC * a_chunk_pitch);
                         load(smem_a + as * p.a_stride, &tmap_a, &full[fs], ca.tc.kb0, ca.kg, ca.tc.m0);
                     } else {
