@@ -12,12 +12,14 @@ from .oracle import (  # noqa: F401
     f64_to_e2m1,
     fp16_to_f64,
     gemm_bf16,
+    gemm_bf16_exact_integers,
     gemm_bf16_rows,
     gemm_fp8_blockscaled,
     gemm_fp8_rows,
     gemm_w4a8,
     gemm_w4a8_rows,
     grouped_gemm_bf16,
+    grouped_gemm_bf16_exact_integers,
     quantize_e2m1,
 )
 from . import attention, moe  # noqa: F401,E402

@@ -184,6 +184,26 @@ uint16_t oracle_f64_to_bf16_rne(double x)
     return (uint16_t)(sign | field);
 }
 
+/* Array forms of the codecs: the scalar codecs above applied to each element in turn (no other
+ * arithmetic), so that whole tensors convert without one foreign call per element. */
+void oracle_bf16_to_f64_array(const uint16_t *bits, double *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_bf16_to_f64(bits[i]);
+}
+
+void oracle_e4m3_to_f64_array(const uint8_t *bits, double *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_e4m3_to_f64(bits[i]);
+}
+
+void oracle_f64_to_bf16_rne_array(const double *x, uint16_t *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_f64_to_bf16_rne(x[i]);
+}
+
 /* ----------------------------------------------------------------------------------------- */
 /* Row-parallel driver                                                                         */
 /* ----------------------------------------------------------------------------------------- */

@@ -45,6 +45,12 @@ class OracleLib:
         lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         lib.oracle_f64_to_bf16_rne.restype = ctypes.c_uint16
         lib.oracle_f64_to_bf16_rne.argtypes = [ctypes.c_double]
+        lib.oracle_bf16_to_f64_array.restype = None
+        lib.oracle_bf16_to_f64_array.argtypes = [vp, vp, i64]
+        lib.oracle_e4m3_to_f64_array.restype = None
+        lib.oracle_e4m3_to_f64_array.argtypes = [vp, vp, i64]
+        lib.oracle_f64_to_bf16_rne_array.restype = None
+        lib.oracle_f64_to_bf16_rne_array.argtypes = [vp, vp, i64]
         lib.oracle_gemm_bf16.restype = i32
         lib.oracle_gemm_bf16.argtypes = [i64, i64, i64, vp, vp, vp, vp, i32]
         lib.oracle_gemm_fp8_blockscaled.restype = i32
@@ -97,28 +103,26 @@ def _c(a, dtype):
 
 
 # ---------------------------------------------------------------------------------------------
-# codecs (scalar, and vectorised by looping in C one element at a time)
+# codecs (scalar, and over whole arrays by looping in C one element at a time)
 # ---------------------------------------------------------------------------------------------
 
 def bf16_to_f64(bits, lib=None) -> np.ndarray:
-    """bf16 bit patterns -> exact fp64 values (oracle codec)."""
+    """bf16 bit patterns -> exact fp64 values (oracle codec, applied element by element in C)."""
     lib = lib or _lib()
     b = np.asarray(bits, dtype=np.uint16)
+    flat = np.ascontiguousarray(b.reshape(-1))
     out = np.empty(b.shape, dtype=np.float64)
-    flat, oflat = b.reshape(-1), out.reshape(-1)
-    for i in range(flat.size):
-        oflat[i] = lib.oracle_bf16_to_f64(int(flat[i]))
+    lib.oracle_bf16_to_f64_array(_ptr(flat), _ptr(out), flat.size)
     return out
 
 
 def e4m3_to_f64(bits, lib=None) -> np.ndarray:
-    """e4m3 (fn) bit patterns -> exact fp64 values (oracle codec)."""
+    """e4m3 (fn) bit patterns -> exact fp64 values (oracle codec, element by element in C)."""
     lib = lib or _lib()
     b = np.asarray(bits, dtype=np.uint8)
+    flat = np.ascontiguousarray(b.reshape(-1))
     out = np.empty(b.shape, dtype=np.float64)
-    flat, oflat = b.reshape(-1), out.reshape(-1)
-    for i in range(flat.size):
-        oflat[i] = lib.oracle_e4m3_to_f64(int(flat[i]))
+    lib.oracle_e4m3_to_f64_array(_ptr(flat), _ptr(out), flat.size)
     return out
 
 
@@ -170,13 +174,13 @@ def quantize_e2m1(W_bits, w_scale, w_zero=None, fp16: bool = False, lib=None) ->
 
 
 def f64_to_bf16(x, lib=None) -> np.ndarray:
-    """fp64 values -> bf16 bit patterns, round to nearest even (oracle codec)."""
+    """fp64 values -> bf16 bit patterns, round to nearest even (oracle codec, element by element
+    in C)."""
     lib = lib or _lib()
     v = np.asarray(x, dtype=np.float64)
+    flat = np.ascontiguousarray(v.reshape(-1))
     out = np.empty(v.shape, dtype=np.uint16)
-    flat, oflat = v.reshape(-1), out.reshape(-1)
-    for i in range(flat.size):
-        oflat[i] = lib.oracle_f64_to_bf16_rne(float(flat[i]))
+    lib.oracle_f64_to_bf16_rne_array(_ptr(flat), _ptr(out), flat.size)
     return out
 
 
@@ -293,3 +297,51 @@ def gemm_fp8_rows(QA_bits, QB_bits, SA, SB, rows, threads: int | None = None):
     rows = np.asarray(rows, dtype=np.int64)
     return gemm_fp8_blockscaled(_c(QA_bits, np.uint8)[rows], QB_bits,
                                 _c(SA, np.float32)[rows], SB, threads)
+
+
+# ---------------------------------------------------------------------------------------------
+# Exact-integer GEMMs (the integer variants of the workloads, at full size)
+# ---------------------------------------------------------------------------------------------
+
+def _exact_integer_operand(bits: np.ndarray, name: str, limit: float) -> np.ndarray:
+    """The fp64 values of bf16 bits that must all be integers of magnitude <= limit."""
+    x = bf16_to_f64(bits)
+    if not np.all(np.isfinite(x)) or not np.all(x == np.round(x)) or np.max(np.abs(x), initial=0) > limit:
+        raise ValueError(f"{name} holds values that are not integers of magnitude <= {limit}")
+    return x
+
+
+def gemm_bf16_exact_integers(A_bits: np.ndarray, B_bits: np.ndarray):
+    """C = A . B^T for bf16 A [M,K], B [N,K] whose entries are all small integers.
+
+    This is the definition of ``gemm_bf16`` for inputs on which it is exact by construction: with
+    |a|, |b| <= 2^8 and K <= 2^30, every product and every partial sum is an integer below 2^53,
+    so the fp64 sum is the exact integer result in any order, and a library fp64 matmul computes
+    it.  The result is rounded once to bf16 (RNE) as ``gemm_bf16`` does.  Inputs outside that
+    range raise ValueError instead of returning a rounded result.  Returns (cref, c bf16 bits).
+    """
+    A = _exact_integer_operand(_c(A_bits, np.uint16), "A", 256.0)
+    B = _exact_integer_operand(_c(B_bits, np.uint16), "B", 256.0)
+    assert A.shape[1] == B.shape[1], "A and B disagree on K"
+    if A.shape[1] > (1 << 30):
+        raise ValueError("K too large for an exact fp64 sum")
+    cref = A @ B.T
+    return cref, f64_to_bf16(cref)
+
+
+def grouped_gemm_bf16_exact_integers(A_bits, B_bits, offsets):
+    """The grouped GEMM (``grouped_gemm_bf16``) on small-integer inputs, exact as in
+    ``gemm_bf16_exact_integers``: C[r] = A[r] . B_e^T for the rows r of expert e's segment."""
+    A = _c(A_bits, np.uint16)
+    B = _c(B_bits, np.uint16)
+    off = _c(offsets, np.int64)
+    R, K = A.shape
+    E, N, K2 = B.shape
+    assert K == K2 and off.shape == (E + 1,)
+    if off[0] != 0 or off[E] != R or np.any(np.diff(off) < 0):
+        raise ValueError("malformed expert offsets")
+    cref = np.zeros((R, N), dtype=np.float64)
+    for e in range(E):
+        if off[e + 1] > off[e]:
+            cref[off[e]:off[e + 1]], _ = gemm_bf16_exact_integers(A[off[e]:off[e + 1]], B[e])
+    return cref, f64_to_bf16(cref)

@@ -132,8 +132,10 @@ def test_k_zero_writes_zeros_and_m_zero_is_a_noop():
 # dense bf16, full-size workloads, sampled rows
 # ---------------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("N,K,M", [(4096, 7168, 1), (4096, 7168, 256), (7168, 2048, 16384),
-                                   (2048, 7168, 16384), (2048, 7168, 1024)])
+@pytest.mark.parametrize("N,K,M", [(4096, 7168, 1), (4096, 7168, 16), (4096, 7168, 64),
+                                   (4096, 7168, 256), (7168, 2048, 1024), (7168, 2048, 4096),
+                                   (7168, 2048, 16384), (2048, 7168, 1024), (2048, 7168, 4096),
+                                   (2048, 7168, 16384)])
 def test_full_size_sampled_rows(N, K, M):
     A = inputs.bf16_gaussian((M, K), seed=2000 + M, device=DEV)
     B = inputs.bf16_gaussian((N, K), seed=2001, std=K ** -0.5, device=DEV)
@@ -254,7 +256,7 @@ def test_grouped_integers_bit_exact_wide_tile():
     parity.assert_bits_equal_values(parity.bits(C), cbits, "grouped integer")
 
 
-@pytest.mark.parametrize("T", [1, 64, 8192])
+@pytest.mark.parametrize("T", [1, 64, 1024, 8192])
 def test_grouped_full_size_sampled_rows(T):
     E, N, K = 64, 2048, 7168
     routing = routing_mod.softmax_top8_routing(T, E, seed=5200 + T)

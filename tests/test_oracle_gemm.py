@@ -290,3 +290,42 @@ def test_routing_is_stable_top8_grouped_by_expert():
         assert experts == sorted(np.argsort(-logits[tok], kind="stable")[:8].tolist())
     # ties go to the lower expert index
     assert routing_mod.topk_experts(torch.zeros(1, 16), 8).tolist() == [list(range(8))]
+
+
+# ---------------------------------------------------------------------------------------------
+# exact-integer GEMMs (the integer variants at full size)
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K,lo,hi", [(7, 33, 64, -4, 4), (40, 17, 300, -4, 4), (3, 5, 7, -256, 256)])
+def test_exact_integer_gemm_equals_the_scalar_oracle_and_int64(M, N, K, lo, hi):
+    A = inputs.bf16_integers((M, K), seed=M + 1, lo=lo, hi=hi)
+    B = inputs.bf16_integers((N, K), seed=N + 2, lo=lo, hi=hi)
+    Ab, Bb = inputs.to_numpy_bits(A), inputs.to_numpy_bits(B)
+    cref, cb = oracle.gemm_bf16_exact_integers(Ab, Bb)
+    cref2, cb2 = oracle.gemm_bf16(Ab, Bb)
+    assert np.array_equal(cb, cb2) and np.array_equal(cref, cref2)
+    exact = A.to(torch.int64).numpy() @ B.to(torch.int64).numpy().T
+    assert np.array_equal(cref, exact.astype(np.float64))
+
+
+def test_exact_integer_gemm_refuses_inputs_it_cannot_sum_exactly():
+    ok = inputs.to_numpy_bits(inputs.bf16_integers((2, 8), seed=1))
+    half = inputs.to_numpy_bits(torch.full((2, 8), 0.5, dtype=torch.bfloat16))
+    big = inputs.to_numpy_bits(torch.full((2, 8), 512.0, dtype=torch.bfloat16))
+    for bad in (half, big):
+        with pytest.raises(ValueError):
+            oracle.gemm_bf16_exact_integers(bad, ok)
+        with pytest.raises(ValueError):
+            oracle.gemm_bf16_exact_integers(ok, bad)
+
+
+def test_exact_integer_grouped_gemm_equals_the_scalar_oracle():
+    E, N, K = 5, 24, 96
+    off = np.array([0, 3, 3, 10, 11, 20], dtype=np.int32)   # expert 1 empty, expert 3 one row
+    A = inputs.to_numpy_bits(inputs.bf16_integers((20, K), seed=7))
+    B = inputs.to_numpy_bits(inputs.bf16_integers((E, N, K), seed=8))
+    cref, cb = oracle.grouped_gemm_bf16_exact_integers(A, B, off)
+    cref2, cb2 = oracle.grouped_gemm_bf16(A, B, off)
+    assert np.array_equal(cb, cb2) and np.array_equal(cref, cref2)
+    with pytest.raises(ValueError):
+        oracle.grouped_gemm_bf16_exact_integers(A, B, np.array([0, 3, 2, 10, 11, 20], np.int32))
