@@ -523,146 +523,162 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
-    """The same sweep end to end: every step copies its A slices in from pinned host memory and
-    its C results back out.
+def gpu_numa_node(dev) -> int | None:
+    """NUMA node of the GPU's PCI device (sysfs), found through NVML by the device UUID."""
+    try:
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        for i in range(pynvml.nvmlDeviceGetCount()):
+            h = pynvml.nvmlDeviceGetHandleByIndex(i)
+            u = pynvml.nvmlDeviceGetUUID(h)
+            u = u.decode() if isinstance(u, bytes) else u
+            if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                bus = pynvml.nvmlDeviceGetPciInfo(h).busId
+                bus = bus.decode() if isinstance(bus, bytes) else bus
+                dom, rest = bus.split(":", 1)
+                path = f"/sys/bus/pci/devices/{int(dom, 16):04x}:{rest.lower()}/numa_node"
+                with open(path) as f:
+                    return int(f.read().strip())
+    except Exception:
+        return None
+    return None
 
-    The reported value pipelines a step's copies against the neighbouring steps' GEMMs, as a
-    serving loop would (see below), captured in CUDA graphs.  `eager` is the host-buffer entry
-    point bi_gemm_run_host called GEMM by GEMM from Python: consecutive GEMMs alternate between
-    two streams, each with its own device staging buffers (within a stream the copy-in, kernel and
-    copy-out of a call stay in order)."""
+
+def node_cpus(node: int) -> set:
+    try:
+        with open(f"/sys/devices/system/node/node{node}/cpulist") as f:
+            text = f.read().strip()
+    except OSError:
+        return set()
+    cpus = set()
+    for part in text.split(","):
+        if "-" in part:
+            a, b = part.split("-")
+            cpus.update(range(int(a), int(b) + 1))
+        elif part:
+            cpus.add(int(part))
+    return cpus
+
+
+def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
+    """The same sweep end to end through the library's host-buffer call.
+
+    Each step is one bi_gemm_run_host_batch call with the sweep's nine GEMMs: pinned host A
+    slices in, the kernels, pinned host C results out.  The library runs the copy-ins on a
+    copy-in stream, the kernels on the compute stream and the copy-outs on a copy-out stream,
+    ordered by its own events over 27 staging slots (three steps): a step's copy-ins run under the
+    previous step's kernels and its copy-outs under the kernels two steps later.  The host buffers are pinned on the GPU's NUMA node when it is known.  The record
+    also holds the pinned copy bandwidth measured in this run (one 256 MiB cudaMemcpyAsync each
+    way), the bound the copies cannot beat."""
     import torch
     from invariant_deterministic_gemm_bi_b200 import inputs
-    steps = max(2, min(args.steps, 200))
-    steps -= steps % 2
-    A_host = inputs.bf16_gaussian((max(M_SWEEP), K_DEC), seed=77).pin_memory()
-    C_host = {m: torch.empty((m, N_DEC), dtype=torch.bfloat16).pin_memory() for m in M_SWEEP}
-    streams = [torch.cuda.Stream(device=dev) for _ in range(2)]
-    A_dev = [torch.empty((max(M_SWEEP), K_DEC), dtype=torch.bfloat16, device=dev) for _ in streams]
-    C_dev = [torch.empty((max(M_SWEEP), N_DEC), dtype=torch.bfloat16, device=dev) for _ in streams]
+    steps = max(2, min(args.steps, 400))
+    node = gpu_numa_node(dev)
+    affinity = None
+    if node is not None and node >= 0 and hasattr(os, "sched_setaffinity"):
+        here = os.sched_getaffinity(0)
+        local = node_cpus(node) & here
+        if local:
+            affinity = here
+            os.sched_setaffinity(0, local)   # pinned pages are placed on the allocating CPU's node
+    try:
+        A_host = inputs.bf16_gaussian((max(M_SWEEP), K_DEC), seed=77).pin_memory()
+        C_host = {m: torch.empty((m, N_DEC), dtype=torch.bfloat16).pin_memory() for m in M_SWEEP}
+        probe_h = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    finally:
+        if affinity is not None:
+            os.sched_setaffinity(0, affinity)
+    probe_d = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def copy_gbs(dst, src):
+        best = None
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                dst.copy_(src, non_blocking=True)
+                e1.record(stream)
+                e1.synchronize()
+                t = e0.elapsed_time(e1) * 1e-3
+                best = t if best is None else min(best, t)
+        return probe_h.numel() / best / 1e9
+    h2d_gbs = copy_gbs(probe_d, probe_h)
+    d2h_gbs = copy_gbs(probe_h, probe_d)
+    del probe_d, probe_h
+
     n_copies = len(Bs)
+    arrays = [bg.host_gemm_array([(A_host[:m], Bs[(ph * len(M_SWEEP) + i) % n_copies], C_host[m])
+                                  for i, m in enumerate(M_SWEEP)]) for ph in range(n_copies)]
+    # three steps' worth of staging slots: a step's copy-ins run while the previous step computes,
+    # and its copy-outs two steps later
+    staging = torch.empty(bg.bi_gemm_host_batch_staging_bytes(plan, arrays[0], 3 * len(M_SWEEP)),
+                          dtype=torch.uint8, device=dev)
+    cin, cout = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    cap = torch.cuda.Stream(device=dev)
 
-    def step(s):
-        for i, m in enumerate(M_SWEEP):
-            j = i % 2
-            bg.bi_gemm_run_host(plan, A_host[:m], Bs[(s * len(M_SWEEP) + i) % n_copies],
-                                C_host[m], A_dev[j], C_dev[j], stream=streams[j])
+    def batch(s, compute):
+        bg.bi_gemm_run_host_batch(plan, arrays[s % n_copies], staging, copy_in=cin, compute=compute,
+                                  copy_out=cout)
 
-    def timed(run_steps):
+    # One CUDA graph holds 3 x n_copies consecutive steps (three turns of the weight rotation) and
+    # a flush: inside it the library's events let the steps' copies overlap the neighbouring
+    # steps' kernels; consecutive replays run in stream order.
+    for s in range(n_copies):
+        batch(s, stream)                      # outside capture: status words, kernel attributes
+    bg.bi_gemm_host_batch_flush(plan, copy_in=cin, compute=stream, copy_out=cout)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    per_graph = 3 * n_copies
+    with torch.cuda.graph(graph, stream=cap):
+        for s in range(per_graph):
+            batch(s, cap)
+        bg.bi_gemm_host_batch_flush(plan, copy_in=cin, compute=cap, copy_out=cout)
+    replays = max(1, steps // per_graph)
+    steps = replays * per_graph
+
+    def timed():
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for st in streams:
-            st.wait_event(e0)
-        run_steps()
-        for st in streams:
-            ev = torch.cuda.Event()
-            ev.record(st)
-            stream.wait_event(ev)
-        e1.record(stream)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(replays):
+                graph.replay()
+            e1.record(stream)
         torch.cuda.synchronize()
         return max_over_ranks(e0.elapsed_time(e1), device=dev)
 
-    for s in range(3):
-        step(s)
-    eager_ms = timed(lambda: [step(s) for s in range(steps)])
-
-    # Software-pipelined, as a serving loop would run it: while step s's nine GEMMs run back to
-    # back on the compute stream (bi_gemm_run, so consecutive launches overlap set-up and tail),
-    # a copy-in stream brings step s+1's A slices from pinned host memory and a copy-out stream
-    # returns step s-1's C results to pinned host memory.  Device staging alternates between two
-    # buffers by step parity; graph p (one per parity, which is also the weight-rotation phase)
-    # holds one such step, and replays run one after another on the timed stream.  The timed
-    # region also holds the first step's copy-in and the last step's copy-out, so it moves every
-    # step's input and result (and one more of each at the two ends of the pipeline).
-    graph_ms, graph_err, check_ok = None, None, None
-    try:
-        A_buf = [{m: torch.empty((m, K_DEC), dtype=torch.bfloat16, device=dev) for m in M_SWEEP}
-                 for _ in range(2)]
-        C_buf = [{m: torch.empty((m, N_DEC), dtype=torch.bfloat16, device=dev) for m in M_SWEEP}
-                 for _ in range(2)]
-        cap, cin, cout = (torch.cuda.Stream(device=dev) for _ in range(3))
-
-        def copy_in(par):
-            for m in M_SWEEP:
-                A_buf[par][m].copy_(A_host[:m], non_blocking=True)
-
-        def copy_out(par):
-            for m in M_SWEEP:
-                C_host[m].copy_(C_buf[par][m], non_blocking=True)
-
-        def pipelined_step(par):
-            cin.wait_stream(cap)    # fork
-            cout.wait_stream(cap)
-            with torch.cuda.stream(cin):
-                copy_in(1 - par)                      # the next step's input
-            with torch.cuda.stream(cout):
-                copy_out(1 - par)                     # the previous step's result
-            for i, m in enumerate(M_SWEEP):
-                bg.bi_gemm_run(plan, A_buf[par][m], Bs[(par * len(M_SWEEP) + i) % n_copies],
-                               C_buf[par][m], stream=cap)
-            cap.wait_stream(cin)    # join
-            cap.wait_stream(cout)
-
-        graphs = []
-        for par in range(2):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=cap):
-                pipelined_step(par)
-            graphs.append(g)
-
-        def replays():   # on the timed stream, after its start event
-            with torch.cuda.stream(stream):
-                copy_in(0)                            # the first step's input
-                for s in range(steps):
-                    graphs[s % 2].replay()
-                copy_out((steps - 1) % 2)             # the last step's result
-        with torch.cuda.stream(stream):
-            copy_in(0)
-            for s in range(4):
-                graphs[s % 2].replay()
-        graph_ms = timed(replays)
-        del graphs
-        # the last step's results, now in pinned host memory, against the same GEMMs run on the
-        # device directly
-        last = (steps - 1) % 2
-        check_ok = True
-        with torch.cuda.stream(stream):
-            for i, m in enumerate(M_SWEEP):
-                ref = torch.empty((m, N_DEC), dtype=torch.bfloat16, device=dev)
-                bg.bi_gemm_run(plan, A_host[:m].to(dev), Bs[(last * len(M_SWEEP) + i) % n_copies], ref,
-                               stream=stream)
-                torch.cuda.synchronize()
-                check_ok &= bool(torch.equal(ref.cpu().view(torch.int16), C_host[m].view(torch.int16)))
-    except RuntimeError as e:   # capture refused: report the call-by-call number alone
-        graph_err = str(e).splitlines()[0][:200]
-        torch.cuda.synchronize()
-        timed(lambda: None)      # every rank takes the same collective steps
-        graph_ms = None
+    with torch.cuda.stream(stream):
+        graph.replay()
+    ms = timed()
+    del graph
+    # the last step's results, now in pinned host memory, against the same GEMMs run directly
+    last = (steps - 1) % n_copies
+    check_ok = True
+    with torch.cuda.stream(stream):
+        for i, m in enumerate(M_SWEEP):
+            ref = torch.empty((m, N_DEC), dtype=torch.bfloat16, device=dev)
+            bg.bi_gemm_run(plan, A_host[:m].to(dev), Bs[(last * len(M_SWEEP) + i) % n_copies], ref,
+                           stream=stream)
+            torch.cuda.synchronize()
+            check_ok &= bool(torch.equal(ref.cpu().view(torch.int16), C_host[m].view(torch.int16)))
 
     h2d = sum(m * K_DEC * 2 for m in M_SWEEP)
     d2h = sum(m * N_DEC * 2 for m in M_SWEEP)
-    per = lambda ms: sweep_bytes() * steps * world / (ms * 1e-3) / 1e9
-    out = {"value": per(graph_ms if graph_ms is not None else eager_ms), "unit": "GB/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-           "ms_per_step": (graph_ms if graph_ms is not None else eager_ms) / steps,
-           "path": ("software-pipelined steps: step s's nine GEMMs (bi_gemm_run) back to back on "
-                    "the compute stream while step s+1's nine A slices come in from pinned host "
-                    "memory and step s-1's nine C results go out to pinned host memory on two "
-                    "copy streams; double-buffered device staging; one CUDA graph per buffer "
-                    "parity, replayed step by step") if graph_ms is not None else
-                   "bi_gemm_run_host per GEMM, issued call by call (graph capture refused)",
-           "eager": {"value": per(eager_ms), "ms_per_step": eager_ms / steps,
-                     "path": "bi_gemm_run_host per GEMM (pinned host A -> device, kernel, device C -> "
-                             "pinned host) issued call by call from Python, consecutive GEMMs on two "
-                             "alternating streams"}}
-    if graph_err:
-        out["graph_capture_error"] = graph_err
-    if check_ok is not None:
-        out["results_match_device_run"] = check_ok
-    return out
+    return {"value": sweep_bytes() * steps * world / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": ms / steps,
+            "path": ("bi_gemm_run_host_batch, one call per step with the sweep's nine GEMMs: copy-ins "
+                     "on a copy-in stream, kernels on the compute stream, copy-outs (two steps "
+                     "later) on a copy-out stream, ordered by the library's events over 27 staging "
+                     "slots; %d steps and a flush per captured CUDA graph, replayed back to back"
+                     % per_graph),
+            "copy_floor_ms_per_step": max(h2d / h2d_gbs, d2h / d2h_gbs) / 1e6,
+            "pinned_h2d_gbs": h2d_gbs, "pinned_d2h_gbs": d2h_gbs,
+            "gpu_numa_node": node, "host_buffers_on_gpu_node": affinity is not None,
+            "results_match_device_run": check_ok}
 
 
 def graph_time_per_launch(fn_list, stream, reps=20):

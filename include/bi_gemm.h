@@ -236,6 +236,72 @@ bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M,
                              cudaStream_t stream);
 
 /*
+ * A batch of dense GEMMs from host memory, pipelined behind the ABI.
+ *
+ * Each call is the GEMM of bi_gemm_run (C = A . B^T, "DeepSeek V4的batch invariance：大模型确定性
+ * 推理的工程基石" (lshu.cn), section 2.1; every row of C bit-identical to the same row computed in
+ * any other batch, "DeepSeek不惜代价保住它！V4关键特性被挖出来了" (QbitAI), section "什么是batch
+ * invariance") with A, scale_a and C in host memory and B, scale_b on the device:
+ *   M, A_host [M][lda], B [N][ldb] (device), C_host [M][ldc] bf16, scale_a_host
+ *   [ceil(K/128)][ld_sa] and scale_b (device) as bi_gemm_run (FP8 plans only; NULL for bf16).
+ * Call i's A (and scale_a) is copied into staging slot (running count) % S on copy_in; once all
+ * of the batch's copy-ins have landed, its GEMMs run on compute in call order.  The batch's C
+ * results are copied back to its C_host buffers on copy_out by the second batch call of this
+ * plan after it (or by bi_gemm_host_batch_flush): they are queued after that batch's copy-ins
+ * and wait for this batch's kernels, which by then have finished.  (A copy-out queued while its
+ * kernel is still running holds up the copies queued after it; deferring it lets later copy-ins
+ * run under the kernels.)  A slot is refilled only after its previous copy-out has completed.
+ * S is the number of slots the staging buffer holds (2 to 32): give it three batches' worth.
+ * At most 1024 calls.
+ * The call returns once everything is enqueued.  A batch's results are in host memory once
+ * copy_out reaches the copy-outs that a later batch call (or the flush) enqueued:
+ * synchronise copy_out after bi_gemm_host_batch_flush to wait for all of them.  Host buffers
+ * must stay valid until then; pinned host memory makes the copies asynchronous.  The three
+ * streams may be the same stream (no overlap).
+ * Staging: caller-owned device memory, 256-byte aligned; bi_gemm_host_batch_staging_bytes(plan,
+ * n, calls, S) gives the bytes for S slots of these calls (0 for invalid arguments or S outside
+ * 2..32); the library allocates nothing.  Passing a different staging buffer (or a batch with a
+ * different largest call) first flushes and makes the first copy-in wait for every copy-out
+ * issued so far.  One batch per plan at a time (a plan-wide lock).
+ * Stream capture: when compute is capturing, the first batch of the capture forks copy_in and
+ * copy_out from compute (copy-outs pending from before the capture must have been flushed, else
+ * BI_ERR_INVALID_ARG), the slots are ordered among the capture's own batches, and
+ * bi_gemm_host_batch_flush, called before the capture ends, enqueues the last copy-outs and
+ * joins both copy streams back into compute.  Replays of the graph are ordered by their stream.
+ * Errors: every call's arguments are checked before anything is enqueued (as bi_gemm_run; the
+ * scale_a of a call is only copied and may have any alignment); BI_ERR_INVALID_ARG for a
+ * missing or short staging buffer, BI_ERR_ALIGNMENT for a misaligned one.  A CUDA failure while
+ * enqueueing returns BI_ERR_CUDA with the work before it enqueued.  BI_ERR_INVALID_ARG also for
+ * a staging buffer of fewer than two slots.  Grouped, split-K and e2m1 plans are refused.
+ */
+typedef struct {
+    int64_t M;
+    const void *A_host;         /* host [M][lda] */
+    int64_t lda;
+    const void *B;              /* device [N][ldb] */
+    int64_t ldb;
+    void *C_host;               /* host [M][ldc] bf16 */
+    int64_t ldc;
+    const float *scale_a_host;  /* FP8: host [ceil(K/128)][ld_sa]; NULL for bf16 */
+    int64_t ld_sa;
+    const float *scale_b;       /* FP8: device [ceil(N/128)][ceil(K/128)]; NULL for bf16 */
+} bi_host_gemm_t;
+
+size_t bi_gemm_host_batch_staging_bytes(bi_plan_t plan, int n, const bi_host_gemm_t *calls,
+                                        int slots);
+
+bi_status_t bi_gemm_run_host_batch(bi_plan_t plan, int n, const bi_host_gemm_t *calls,
+                                   void *staging, size_t staging_bytes,
+                                   cudaStream_t copy_in, cudaStream_t compute,
+                                   cudaStream_t copy_out);
+
+/* Enqueue the copy-outs still pending from the plan's last host batches on copy_out (each after
+ * its batch's kernels); under stream capture also join copy_in and copy_out back into compute.
+ * Returns BI_OK when nothing is pending. */
+bi_status_t bi_gemm_host_batch_flush(bi_plan_t plan, cudaStream_t copy_in, cudaStream_t compute,
+                                     cudaStream_t copy_out);
+
+/*
  * Dense GEMM from host memory for callers that must not allocate device memory.
  *
  * Some callers cannot call cudaMalloc: their device memory is owned by another allocator (a

@@ -31,6 +31,10 @@ from .binding import (  # noqa: F401
     bi_gemm_run,
     bi_gemm_run_host,
     bi_gemm_run_host_noalloc,
+    bi_gemm_run_host_batch,
+    bi_gemm_host_batch_flush,
+    bi_gemm_host_batch_staging_bytes,
+    host_gemm_array,
     bi_gemm_run_splitk,
     bi_gemm_run_w4a8,
     bi_gemm_set_wait_timeout,

@@ -35,6 +35,7 @@ EXPORTED = [
     "bi_gemm_plan_describe", "bi_gemm_run", "bi_grouped_gemm_run", "bi_gemm_run_host",
     "bi_gemm_sync_status", "bi_gemm_set_wait_timeout", "bi_gemm_debug_set_flags",
     "bi_gemm_run_host_noalloc", "bi_gemm_plan_set_flags",
+    "bi_gemm_host_batch_staging_bytes", "bi_gemm_run_host_batch", "bi_gemm_host_batch_flush",
     "bi_gemm_plan_splitk", "bi_gemm_splitk_workspace_bytes", "bi_gemm_run_splitk",
     "bi_gemm_w4a8_workspace_bytes", "bi_gemm_run_w4a8",
     "bi_moe_route_topk", "bi_moe_dispatch", "bi_moe_gather_rows", "bi_moe_combine",
@@ -63,6 +64,16 @@ class PlanInfo(ctypes.Structure):
 
     def as_dict(self):
         return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+class HostGemm(ctypes.Structure):
+    """bi_host_gemm_t: one GEMM of a bi_gemm_run_host_batch call."""
+    _fields_ = [
+        ("M", ctypes.c_int64), ("A_host", ctypes.c_void_p), ("lda", ctypes.c_int64),
+        ("B", ctypes.c_void_p), ("ldb", ctypes.c_int64), ("C_host", ctypes.c_void_p),
+        ("ldc", ctypes.c_int64), ("scale_a_host", ctypes.c_void_p), ("ld_sa", ctypes.c_int64),
+        ("scale_b", ctypes.c_void_p),
+    ]
 
 
 _LIB = None
@@ -94,6 +105,13 @@ def load_library(path: str = LIB_PATH):
     lib.bi_grouped_gemm_run.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, vp]
     lib.bi_gemm_run_host.restype = i32
     lib.bi_gemm_run_host.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, i64, vp, vp, vp, vp, vp]
+    lib.bi_gemm_host_batch_staging_bytes.restype = ctypes.c_size_t
+    lib.bi_gemm_host_batch_staging_bytes.argtypes = [vp, i32, ctypes.POINTER(HostGemm), i32]
+    lib.bi_gemm_run_host_batch.restype = i32
+    lib.bi_gemm_run_host_batch.argtypes = [vp, i32, ctypes.POINTER(HostGemm), vp, ctypes.c_size_t, vp,
+                                           vp, vp]
+    lib.bi_gemm_host_batch_flush.restype = i32
+    lib.bi_gemm_host_batch_flush.argtypes = [vp, vp, vp, vp]
     lib.bi_gemm_run_host_noalloc.restype = i32
     lib.bi_gemm_run_host_noalloc.argtypes = [vp, i64, vp, i64, vp, i64, vp, i64, vp, i64, vp, vp]
     lib.bi_gemm_sync_status.restype = i32
@@ -255,6 +273,45 @@ def bi_gemm_run_host_noalloc(plan: Plan, A_host, B, C_host, scale_a_host=None, s
                                                  _ptr(scale_b), _stream_handle(stream))
     _check(st, "bi_gemm_run_host_noalloc")
     return C_host
+
+
+def host_gemm_array(calls) -> "ctypes.Array":
+    """A bi_host_gemm_t array from (A_host, B, C_host[, scale_a_host, scale_b]) tuples of tensors
+    (host A / C / scale_a, device B / scale_b; ld_sa is scale_a's row pitch)."""
+    arr = (HostGemm * len(calls))()
+    for i, c in enumerate(calls):
+        A, B, C = c[0], c[1], c[2]
+        sa = c[3] if len(c) > 3 else None
+        sb = c[4] if len(c) > 4 else None
+        arr[i] = HostGemm(A.shape[0], _ptr(A), A.stride(0), _ptr(B), B.stride(0), _ptr(C),
+                          C.stride(0), _ptr(sa), sa.stride(0) if sa is not None else 0, _ptr(sb))
+    return arr
+
+
+def bi_gemm_host_batch_staging_bytes(plan: Plan, calls, slots: int = 6) -> int:
+    arr = calls if isinstance(calls, ctypes.Array) else host_gemm_array(calls)
+    return int(load_library().bi_gemm_host_batch_staging_bytes(plan.handle, len(arr), arr, slots))
+
+
+def bi_gemm_run_host_batch(plan: Plan, calls, staging, copy_in=None, compute=None, copy_out=None):
+    """Pipelined host-buffer GEMMs: the calls' A come in on copy_in, their GEMMs run on compute,
+    and their C go out on copy_out with the next batch call or bi_gemm_host_batch_flush (see
+    include/bi_gemm.h).  `calls` is a list of tuples as for host_gemm_array, or such an array;
+    `staging` a device tensor of at least bi_gemm_host_batch_staging_bytes bytes.  Returns once
+    enqueued."""
+    arr = calls if isinstance(calls, ctypes.Array) else host_gemm_array(calls)
+    nbytes = staging.numel() * staging.element_size()
+    _check(load_library().bi_gemm_run_host_batch(plan.handle, len(arr), arr, _ptr(staging), nbytes,
+                                                 _stream_handle(copy_in), _stream_handle(compute),
+                                                 _stream_handle(copy_out)),
+           "bi_gemm_run_host_batch")
+
+
+def bi_gemm_host_batch_flush(plan: Plan, copy_in=None, compute=None, copy_out=None):
+    """Enqueue the last host batch's copy-outs (and, under capture, join the copy streams)."""
+    _check(load_library().bi_gemm_host_batch_flush(plan.handle, _stream_handle(copy_in),
+                                                   _stream_handle(compute), _stream_handle(copy_out)),
+           "bi_gemm_host_batch_flush")
 
 
 def bi_gemm_sync_status(plan: Plan, stream=None, raise_on_error: bool = True) -> int:

@@ -13,6 +13,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <deque>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -304,6 +305,40 @@ bi_status_t current_device(int *dev_out, DeviceInfo **info_out)
 // The plan object
 // ---------------------------------------------------------------------------------------------
 
+// Staging slots of bi_gemm_run_host_batch: as many as the caller's staging holds, 2 to
+// kMaxHostSlots.  A slot is refilled once its previous copy-out has completed, so the copy-in
+// stream runs up to (slots - 1) GEMMs ahead of the kernels.
+constexpr int kMaxHostSlots = 32;
+
+// A batch's copy-outs are enqueued this many batches later (or by a flush): by then the kernels
+// they wait for have long finished, so they never hold up the copy-ins queued behind them.
+constexpr int kHostDefer = 2;
+
+// A copy-out of bi_gemm_run_host_batch that waits for a later batch (or a flush) to be issued.
+struct PendingOut {
+    void *c_host;
+    const void *c_dev;
+    size_t bytes;
+    int slot;
+};
+
+struct HostPipe {
+    cudaEvent_t in_done[kMaxHostSlots] = {};
+    cudaEvent_t gemm_done[kMaxHostSlots] = {};
+    cudaEvent_t out_done[kMaxHostSlots] = {};
+    uint64_t next = 0;                  // calls issued so far (slot = next % slots)
+    const void *staging = nullptr;      // layout of the last batch
+    size_t slot_bytes = 0;
+    int slots = 0;
+    // copy-outs of the last kHostDefer batches, not yet enqueued, oldest first, each with the
+    // gemm_done slot recorded after that batch's kernels
+    std::deque<std::pair<std::vector<PendingOut>, int>> pending;
+    // stream capture: the capture the batches belong to, and its own slot order
+    unsigned long long cap_id = 0;
+    uint64_t cap_next = 0;
+    uint32_t cap_used = 0;              // slots filled inside the capture
+};
+
 struct bi_plan_s {
     int64_t n = 0, k = 0;
     bi_dtype_t dtype = BI_DTYPE_BF16;
@@ -331,6 +366,10 @@ struct bi_plan_s {
     int k_splits = 1;        // > 1: fixed-split-K research plan (bi_gemm_plan_splitk)
     std::mutex mu;
     int *status[kMaxDevices] = {};
+    // bi_gemm_run_host_batch, per device: the events that order the reuse of each staging slot
+    // (copy-in done, GEMM done, copy-out done), the next slot, and the staging layout last used
+    HostPipe *pipe[kMaxDevices] = {};
+    std::mutex pipe_mu;      // one host batch of this plan at a time (the slot order is shared)
 };
 
 namespace {
@@ -805,6 +844,15 @@ bi_status_t bi_gemm_plan_destroy(bi_plan_t plan)
             cudaSetDevice(d);
             cudaFree(plan->status[d]);
         }
+        if (plan->pipe[d]) {
+            cudaSetDevice(d);
+            for (int i = 0; i < kMaxHostSlots; ++i) {
+                cudaEventDestroy(plan->pipe[d]->in_done[i]);
+                cudaEventDestroy(plan->pipe[d]->gemm_done[i]);
+                cudaEventDestroy(plan->pipe[d]->out_done[i]);
+            }
+            delete plan->pipe[d];
+        }
     }
     if (have_dev)
         cudaSetDevice(cur);
@@ -1016,6 +1064,265 @@ bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M, const void *A_host, int6
     if (cudaMemcpyAsync(C_host, C_dev, static_cast<size_t>(M * ldc * 2), cudaMemcpyDeviceToHost,
                         stream) != cudaSuccess)
         return BI_ERR_CUDA;
+    return BI_OK;
+}
+
+// The plan's host-batch state on this device, created with its events on first use.
+static bi_status_t host_pipe_for(bi_plan_s *plan, int dev, HostPipe **out)
+{
+    HostPipe *hp = plan->pipe[dev];
+    if (!hp) {
+        hp = new (std::nothrow) HostPipe();
+        if (!hp)
+            return BI_ERR_INVALID_ARG;
+        for (int i = 0; i < kMaxHostSlots; ++i)
+            if (cudaEventCreateWithFlags(&hp->in_done[i], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&hp->gemm_done[i], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&hp->out_done[i], cudaEventDisableTiming) != cudaSuccess) {
+                cudaGetLastError();
+                for (int j = 0; j < kMaxHostSlots; ++j) {
+                    if (hp->in_done[j]) cudaEventDestroy(hp->in_done[j]);
+                    if (hp->gemm_done[j]) cudaEventDestroy(hp->gemm_done[j]);
+                    if (hp->out_done[j]) cudaEventDestroy(hp->out_done[j]);
+                }
+                delete hp;
+                return BI_ERR_CUDA;
+            }
+        plan->pipe[dev] = hp;
+    }
+    *out = hp;
+    return BI_OK;
+}
+
+// Enqueue on copy_out, after each batch's kernels, the copy-outs pending from all but the newest
+// `keep` batches (oldest first).
+static bi_status_t host_batch_flush(HostPipe *hp, cudaStream_t copy_out, size_t keep = 0)
+{
+    while (hp->pending.size() > keep) {
+        const auto &b = hp->pending.front();
+        if (cudaStreamWaitEvent(copy_out, hp->gemm_done[b.second], 0) != cudaSuccess)
+            return BI_ERR_CUDA;
+        for (const PendingOut &o : b.first)
+            if (cudaMemcpyAsync(o.c_host, o.c_dev, o.bytes, cudaMemcpyDeviceToHost, copy_out) != cudaSuccess ||
+                cudaEventRecord(hp->out_done[o.slot], copy_out) != cudaSuccess)
+                return BI_ERR_CUDA;
+        hp->pending.pop_front();
+    }
+    return BI_OK;
+}
+
+// Bytes of one staging slot of bi_gemm_run_host_batch for these calls: A, C and (FP8) scale_a
+// of the largest call, each rounded up to 256 bytes.  Returns -1 for arguments no call may have.
+static int64_t host_batch_slot_bytes(const bi_plan_s *plan, int n, const bi_host_gemm_t *calls)
+{
+    const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
+    const int elt = fp8 ? 1 : 2;
+    const int64_t kb = (plan->k + 127) / 128;
+    const int64_t cap = int64_t(1) << 40;   // bounds every factor, so no product below can wrap
+    int64_t a = 0, c = 0, sa = 0;
+    for (int i = 0; i < n; ++i) {
+        const bi_host_gemm_t &g = calls[i];
+        if (g.M < 0 || g.M > cap || g.lda < 0 || g.lda > cap || g.ldc < 0 || g.ldc > cap ||
+            g.ld_sa < 0 || g.ld_sa > cap)
+            return -1;
+        a = a > g.M * g.lda * elt ? a : g.M * g.lda * elt;
+        c = c > g.M * g.ldc * 2 ? c : g.M * g.ldc * 2;
+        if (fp8)
+            sa = sa > kb * g.ld_sa * 4 ? sa : kb * g.ld_sa * 4;
+    }
+    return round256(a) + round256(c) + round256(sa);
+}
+
+size_t bi_gemm_host_batch_staging_bytes(bi_plan_t plan, int n, const bi_host_gemm_t *calls, int slots)
+{
+    if (!plan || n < 0 || (n > 0 && !calls) || slots < 2 || slots > kMaxHostSlots)
+        return 0;
+    const int64_t slot = host_batch_slot_bytes(plan, n, calls);
+    return slot < 0 ? 0 : static_cast<size_t>(slot) * static_cast<size_t>(slots);
+}
+
+bi_status_t bi_gemm_run_host_batch(bi_plan_t plan, int n, const bi_host_gemm_t *calls, void *staging,
+                                   size_t staging_bytes, cudaStream_t copy_in, cudaStream_t compute,
+                                   cudaStream_t copy_out)
+{
+    if (!plan || n < 0 || (n > 0 && !calls))
+        return BI_ERR_INVALID_ARG;
+    if (plan->experts != 1 || plan->k_splits > 1)
+        return BI_ERR_INVALID_ARG;
+    if (plan->dtype == BI_DTYPE_E2M1_W4A8)
+        return BI_ERR_DTYPE_MISMATCH;
+    if (n == 0 || plan->n == 0)
+        return BI_OK;
+    const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
+    const int elt = fp8 ? 1 : 2;
+    const int64_t kb = (plan->k + 127) / 128;
+    const int64_t slot_bytes = host_batch_slot_bytes(plan, n, calls);
+    if (slot_bytes < 0)
+        return BI_ERR_INVALID_ARG;
+    if (!staging || slot_bytes == 0 || staging_bytes < static_cast<size_t>(slot_bytes) * 2)
+        return BI_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(staging) & 255u)
+        return BI_ERR_ALIGNMENT;
+    const size_t fit = staging_bytes / static_cast<size_t>(slot_bytes);
+    const int slots = fit > static_cast<size_t>(kMaxHostSlots) ? kMaxHostSlots : static_cast<int>(fit);
+    int64_t a_max = 0, c_max = 0;
+    for (int i = 0; i < n; ++i) {
+        a_max = a_max > calls[i].M * calls[i].lda * elt ? a_max : calls[i].M * calls[i].lda * elt;
+        c_max = c_max > calls[i].M * calls[i].ldc * 2 ? c_max : calls[i].M * calls[i].ldc * 2;
+    }
+    const int64_t c_off = round256(a_max), s_off = c_off + round256(c_max);
+    // Validate every call before enqueueing anything (against slot 0's addresses: every slot has
+    // the same alignment).
+    unsigned char *base = static_cast<unsigned char *>(staging);
+    for (int i = 0; i < n; ++i) {
+        const bi_host_gemm_t &g = calls[i];
+        if (g.M == 0)
+            continue;
+        if (!g.C_host || (plan->k > 0 && !g.A_host))
+            return BI_ERR_INVALID_ARG;
+        bi_status_t st = check_common(plan, g.M, base, g.lda, g.B, g.ldb, base + c_off, g.ldc);
+        if (st != BI_OK)
+            return st;
+        if (fp8 && plan->k > 0) {
+            if ((st = check_fp8_scales(g.M, g.scale_a_host, g.ld_sa, g.scale_b, false)) != BI_OK)
+                return st;
+        } else if (!fp8 && (g.scale_a_host || g.scale_b)) {
+            return BI_ERR_DTYPE_MISMATCH;
+        }
+    }
+    int dev = 0;
+    DeviceInfo *d = nullptr;
+    bi_status_t st = current_device(&dev, &d);
+    if (st != BI_OK)
+        return st;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    unsigned long long cap_id = 0;
+    if (cudaStreamGetCaptureInfo(compute, &cap, &cap_id) != cudaSuccess)
+        return BI_ERR_CUDA;
+    const bool captured = cap == cudaStreamCaptureStatusActive;
+    std::lock_guard<std::mutex> lock(plan->pipe_mu);
+    HostPipe *hp = nullptr;
+    if ((st = host_pipe_for(plan, dev, &hp)) != BI_OK)
+        return st;
+    if (captured) {
+        if (hp->cap_id != cap_id) {
+            // the first batch of this capture: copy-outs pending from outside it would run at
+            // replay instead of now, so they must have been flushed; the copy streams join the
+            // capture by waiting on the compute stream once
+            if (!hp->pending.empty())
+                return BI_ERR_INVALID_ARG;
+            if (cudaEventRecord(hp->gemm_done[0], compute) != cudaSuccess ||
+                cudaStreamWaitEvent(copy_in, hp->gemm_done[0], 0) != cudaSuccess ||
+                cudaStreamWaitEvent(copy_out, hp->gemm_done[0], 0) != cudaSuccess)
+                return BI_ERR_CUDA;
+            hp->cap_id = cap_id;
+            hp->cap_next = 0;
+            hp->cap_used = 0;
+        }
+    } else {
+        // A different staging buffer or layout than the last batch: the slots may overlap the
+        // old ones, so the first copy-in waits for every copy-out issued so far.
+        const bool relayout = hp->staging != staging || hp->slot_bytes != static_cast<size_t>(slot_bytes) ||
+                              hp->slots != slots;
+        if (relayout) {
+            if ((st = host_batch_flush(hp, copy_out)) != BI_OK)
+                return st;
+            if (hp->next > 0)
+                for (int i = 0; i < hp->slots; ++i)
+                    if (cudaStreamWaitEvent(copy_in, hp->out_done[i], 0) != cudaSuccess)
+                        return BI_ERR_CUDA;
+            hp->next = 0;
+        }
+        hp->staging = staging;
+        hp->slot_bytes = static_cast<size_t>(slot_bytes);
+        hp->slots = slots;
+    }
+    // This batch's copy-ins (a slot is refilled once its previous copy-out has completed); then
+    // the copy-outs of the batch kHostDefer batches back, queued after these copy-ins, behind
+    // kernels that have long finished; then this batch's kernels after one wait for its
+    // copy-ins.  A copy-out queued while its kernel is still running would hold up the copies
+    // queued after it.
+    std::vector<PendingOut> outs;
+    outs.reserve(static_cast<size_t>(n));
+    int last_slot = -1;
+    for (int i = 0; i < n; ++i) {
+        const bi_host_gemm_t &g = calls[i];
+        if (g.M == 0)
+            continue;
+        uint64_t &next = captured ? hp->cap_next : hp->next;
+        const int slot = static_cast<int>(next % static_cast<uint64_t>(slots));
+        ++next;
+        unsigned char *A_dev = base + slot * slot_bytes;
+        float *sa_dev = reinterpret_cast<float *>(A_dev + s_off);
+        const bool reused = captured ? ((hp->cap_used >> slot) & 1u) != 0 : true;
+        if (reused && cudaStreamWaitEvent(copy_in, hp->out_done[slot], 0) != cudaSuccess)
+            return BI_ERR_CUDA;
+        if (captured)
+            hp->cap_used |= 1u << slot;
+        last_slot = slot;
+        if (plan->k > 0) {
+            if (cudaMemcpyAsync(A_dev, g.A_host, static_cast<size_t>(g.M * g.lda * elt),
+                                cudaMemcpyHostToDevice, copy_in) != cudaSuccess)
+                return BI_ERR_CUDA;
+            if (fp8 && cudaMemcpyAsync(sa_dev, g.scale_a_host, static_cast<size_t>(kb * g.ld_sa * 4),
+                                       cudaMemcpyHostToDevice, copy_in) != cudaSuccess)
+                return BI_ERR_CUDA;
+        }
+        outs.push_back(PendingOut{g.C_host, A_dev + c_off, static_cast<size_t>(g.M * g.ldc * 2), slot});
+    }
+    if ((st = host_batch_flush(hp, copy_out, kHostDefer - 1)) != BI_OK)
+        return st;
+    if (last_slot < 0)
+        return BI_OK;
+    if (cudaEventRecord(hp->in_done[last_slot], copy_in) != cudaSuccess ||
+        cudaStreamWaitEvent(compute, hp->in_done[last_slot], 0) != cudaSuccess)
+        return BI_ERR_CUDA;
+    size_t j = 0;
+    for (int i = 0; i < n; ++i) {
+        const bi_host_gemm_t &g = calls[i];
+        if (g.M == 0)
+            continue;
+        unsigned char *A_dev = base + outs[j++].slot * slot_bytes;
+        if ((st = bi_gemm_run(plan, g.M, A_dev, g.lda, g.B, g.ldb, A_dev + c_off, g.ldc,
+                              fp8 ? reinterpret_cast<float *>(A_dev + s_off) : nullptr, g.ld_sa,
+                              fp8 ? g.scale_b : nullptr, compute)) != BI_OK)
+            return st;
+    }
+    if (cudaEventRecord(hp->gemm_done[last_slot], compute) != cudaSuccess)
+        return BI_ERR_CUDA;
+    hp->pending.emplace_back(std::move(outs), last_slot);
+    return BI_OK;
+}
+
+bi_status_t bi_gemm_host_batch_flush(bi_plan_t plan, cudaStream_t copy_in, cudaStream_t compute,
+                                     cudaStream_t copy_out)
+{
+    if (!plan)
+        return BI_ERR_INVALID_ARG;
+    int dev = 0;
+    DeviceInfo *d = nullptr;
+    bi_status_t st = current_device(&dev, &d);
+    if (st != BI_OK)
+        return st;
+    std::lock_guard<std::mutex> lock(plan->pipe_mu);
+    HostPipe *hp = plan->pipe[dev];
+    if (!hp)
+        return BI_OK;
+    if ((st = host_batch_flush(hp, copy_out)) != BI_OK)
+        return st;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    unsigned long long cap_id = 0;
+    if (cudaStreamGetCaptureInfo(compute, &cap, &cap_id) != cudaSuccess)
+        return BI_ERR_CUDA;
+    if (cap == cudaStreamCaptureStatusActive && cap_id == hp->cap_id) {
+        // join both copy streams back into the compute stream so the capture can end
+        if (cudaEventRecord(hp->in_done[0], copy_in) != cudaSuccess ||
+            cudaEventRecord(hp->out_done[0], copy_out) != cudaSuccess ||
+            cudaStreamWaitEvent(compute, hp->in_done[0], 0) != cudaSuccess ||
+            cudaStreamWaitEvent(compute, hp->out_done[0], 0) != cudaSuccess)
+            return BI_ERR_CUDA;
+        hp->cap_id = 0;
+    }
     return BI_OK;
 }
 

@@ -176,6 +176,45 @@ def test_run_host_refuses_before_enqueueing_a_copy():
                                 None) == S["BI_ERR_DTYPE_MISMATCH"]
 
 
+def test_host_batch_rejects_bad_arguments_before_any_device_call():
+    """The pipelined host-buffer batch checks every call and the staging buffer before it touches
+    a device; the pointer values are never dereferenced."""
+    lib = binding.load_library()
+    S = binding.STATUS
+    HG = binding.HostGemm
+    plan = bg.bi_gemm_plan(256, 512)
+    ok = HG(4, 4096, 512, 4096, 512, 4096, 256, None, 0, None)
+    arr = (HG * 2)(ok, HG(0, None, 512, None, 512, None, 256, None, 0, None))
+    slot = 4 * 512 * 2 + 4 * 256 * 2                  # the largest A and C
+    need = lib.bi_gemm_host_batch_staging_bytes(plan.handle, 2, arr, 6)
+    assert need == 6 * slot
+    assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 2, arr, 1) == 0
+    assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 2, arr, 33) == 0
+    run = lib.bi_gemm_run_host_batch
+    assert run(None, 2, arr, 4096, need, None, None, None) == S["BI_ERR_INVALID_ARG"]
+    assert run(plan.handle, 0, None, None, 0, None, None, None) == 0           # empty batch
+    assert run(plan.handle, 2, arr, None, need, None, None, None) == S["BI_ERR_INVALID_ARG"]
+    assert run(plan.handle, 2, arr, 4096, 2 * slot - 256, None, None, None) == S["BI_ERR_INVALID_ARG"]
+    assert run(plan.handle, 2, arr, 4096 + 16, need, None, None, None) == S["BI_ERR_ALIGNMENT"]
+    bad = [HG(4, 4096, 512, 4096, 512, 4096, 256, 4096, 4, 4096),     # scales on a bf16 plan
+           HG(4, 4096, 500, 4096, 512, 4096, 256, None, 0, None),     # lda below K
+           HG(4, 4096, 516, 4096, 512, 4096, 256, None, 0, None),     # lda not a 16-byte pitch
+           HG(-1, 4096, 512, 4096, 512, 4096, 256, None, 0, None),
+           HG(4, None, 512, 4096, 512, 4096, 256, None, 0, None)]
+    want = ["BI_ERR_DTYPE_MISMATCH", "BI_ERR_INVALID_ARG", "BI_ERR_ALIGNMENT", "BI_ERR_INVALID_ARG",
+            "BI_ERR_INVALID_ARG"]
+    for b, w in zip(bad, want):
+        one = (HG * 1)(b)
+        assert run(plan.handle, 1, one, 4096, 1 << 20, None, None, None) == S[w], w
+    gp = bg.bi_gemm_plan(256, 512, 0, 4)
+    assert run(gp.handle, 2, arr, 4096, need, None, None, None) == S["BI_ERR_INVALID_ARG"]
+    f8 = bg.bi_gemm_plan(256, 512, bg.BI_DTYPE_E4M3_BLOCKSCALED)
+    one = (HG * 1)(HG(4, 4096, 512, 4096, 512, 4096, 256, 4096, 4, 4098))  # scale_b misaligned
+    assert run(f8.handle, 1, one, 4096, 1 << 20, None, None, None) == S["BI_ERR_ALIGNMENT"]
+    if not __import__("torch").cuda.is_available():
+        assert run(plan.handle, 2, arr, 4096, need, None, None, None) == S["BI_ERR_NO_DEVICE"]
+
+
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="a GPU is present")
 def test_valid_run_without_a_device_reports_no_device():
     lib = binding.load_library()
