@@ -124,6 +124,21 @@ const char *bi_status_string(bi_status_t status);
 bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
                          int num_experts);
 
+/*
+ * A plan for the output columns [n_begin, n_end) of a dense plan (column-parallel sharding: one
+ * GPU per column shard, "DeepSeek V4的batch invariance：大模型确定性推理的工程基石" (lshu.cn),
+ * section 2.2, on every device computing the same thing).  It keeps `full`'s tile, MMA
+ * instruction and K order (and scheduling forms), so column n of C computed with it, from rows
+ * [n_begin, n_end) of B, is bit-identical to column n_begin + n of the full GEMM.  (A plan made
+ * for the shard's own (N, K) may choose a different tile and K order, and then differ in the
+ * last bits.)  Run it like any dense plan with N = n_end - n_begin: B is the shard's [N][ldb]
+ * rows, C its [M][ldc] columns; for FP8, scale_b starts at block row n_begin / 128.
+ * Errors: BI_ERR_INVALID_ARG for a grouped or split-K plan or a range outside [0, N];
+ * BI_ERR_UNSUPPORTED_SHAPE for an FP8 plan and n_begin not a multiple of 128.  The shard plan is
+ * independent of `full` once made; destroy it with bi_gemm_plan_destroy.
+ */
+bi_status_t bi_gemm_plan_column_shard(bi_plan_t *out, bi_plan_t full, int64_t n_begin, int64_t n_end);
+
 /* Destroy a plan and free its device status words.  NULL is accepted. */
 bi_status_t bi_gemm_plan_destroy(bi_plan_t plan);
 

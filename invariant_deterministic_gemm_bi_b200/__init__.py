@@ -32,6 +32,7 @@ from .binding import (  # noqa: F401
     bi_gemm_run_host,
     bi_gemm_run_host_noalloc,
     bi_gemm_run_host_batch,
+    bi_gemm_plan_column_shard,
     bi_gemm_host_batch_flush,
     bi_gemm_host_batch_staging_bytes,
     host_gemm_array,

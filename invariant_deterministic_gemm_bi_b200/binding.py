@@ -36,6 +36,7 @@ EXPORTED = [
     "bi_gemm_sync_status", "bi_gemm_set_wait_timeout", "bi_gemm_debug_set_flags",
     "bi_gemm_run_host_noalloc", "bi_gemm_plan_set_flags",
     "bi_gemm_host_batch_staging_bytes", "bi_gemm_run_host_batch", "bi_gemm_host_batch_flush",
+    "bi_gemm_plan_column_shard",
     "bi_gemm_plan_splitk", "bi_gemm_splitk_workspace_bytes", "bi_gemm_run_splitk",
     "bi_gemm_w4a8_workspace_bytes", "bi_gemm_run_w4a8",
     "bi_moe_route_topk", "bi_moe_dispatch", "bi_moe_gather_rows", "bi_moe_combine",
@@ -110,6 +111,8 @@ def load_library(path: str = LIB_PATH):
     lib.bi_gemm_run_host_batch.restype = i32
     lib.bi_gemm_run_host_batch.argtypes = [vp, i32, ctypes.POINTER(HostGemm), vp, ctypes.c_size_t, vp,
                                            vp, vp]
+    lib.bi_gemm_plan_column_shard.restype = i32
+    lib.bi_gemm_plan_column_shard.argtypes = [ctypes.POINTER(vp), vp, i64, i64]
     lib.bi_gemm_host_batch_flush.restype = i32
     lib.bi_gemm_host_batch_flush.argtypes = [vp, vp, vp, vp]
     lib.bi_gemm_run_host_noalloc.restype = i32
@@ -305,6 +308,14 @@ def bi_gemm_run_host_batch(plan: Plan, calls, staging, copy_in=None, compute=Non
                                                  _stream_handle(copy_in), _stream_handle(compute),
                                                  _stream_handle(copy_out)),
            "bi_gemm_run_host_batch")
+
+
+def bi_gemm_plan_column_shard(full: Plan, n_begin: int, n_end: int) -> Plan:
+    """A plan for output columns [n_begin, n_end) of `full` with `full`'s tile and K order."""
+    h = ctypes.c_void_p()
+    _check(load_library().bi_gemm_plan_column_shard(ctypes.byref(h), full.handle, n_begin, n_end),
+           "bi_gemm_plan_column_shard")
+    return Plan(h.value, n_end - n_begin, full.k, full.dtype, 1)
 
 
 def bi_gemm_host_batch_flush(plan: Plan, copy_in=None, compute=None, copy_out=None):

@@ -833,6 +833,38 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     return BI_OK;
 }
 
+bi_status_t bi_gemm_plan_column_shard(bi_plan_t *out, bi_plan_t full, int64_t n_begin, int64_t n_end)
+{
+    if (!out)
+        return BI_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!full || full->experts != 1 || full->k_splits > 1)
+        return BI_ERR_INVALID_ARG;
+    if (n_begin < 0 || n_end < n_begin || n_end > full->n)
+        return BI_ERR_INVALID_ARG;
+    // FP8 weights carry one scale per 128 x 128 block: a shard must start on a block boundary so
+    // that its columns keep their scale blocks (the caller passes scale_b from row n_begin / 128)
+    if (full->dtype == BI_DTYPE_E4M3_BLOCKSCALED && n_begin % 128 != 0)
+        return BI_ERR_UNSUPPORTED_SHAPE;
+    bi_plan_s *p = new (std::nothrow) bi_plan_s();
+    if (!p)
+        return BI_ERR_INVALID_ARG;
+    p->n = n_end - n_begin;
+    p->k = full->k;
+    p->dtype = full->dtype;
+    p->experts = 1;
+    p->kernel = full->kernel;
+    p->kernel_small = full->kernel_small;
+    p->kernel_tiny = full->kernel_tiny;
+    p->kernel_wide = full->kernel_wide;
+    p->kernel_wide4 = full->kernel_wide4;
+    p->small_rows = full->small_rows;
+    p->timeout_ns = full->timeout_ns;
+    p->flags = full->flags;
+    *out = p;
+    return BI_OK;
+}
+
 bi_status_t bi_gemm_plan_destroy(bi_plan_t plan)
 {
     if (!plan)

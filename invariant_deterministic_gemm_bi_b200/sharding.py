@@ -1,11 +1,14 @@
 """Host-side helpers for running the batch-invariant GEMM on several GPUs, one process each.
 
 The GEMM shards with no numerical exchange: split the rows of A (M-sharding: independent token
-batches) or the rows of B (N-sharding: column-parallel weights, whole K per output column).  Each
-rank runs the same plan -- a pure function of (N, K, dtype) -- so every row gets the same bits on
-every GPU as it would alone.  Splitting K is not offered: summing partial products across ranks is
-split-K, which the method excludes.  The only collectives are gathers of finished rows (a copy,
-exact) and the max of per-rank timings.
+batches) or the rows of B (N-sharding: column-parallel weights, whole K per output column).  With
+M-sharding each rank runs the same plan -- a pure function of (N, K, dtype) -- so every row gets
+the same bits on every GPU as it would alone.  With N-sharding each rank runs a column-shard plan
+of the full plan (bi_gemm_plan_column_shard): a plan made for the shard's own (N/G, K) may pick
+another tile and K order, and its columns would differ from the single-GPU ones in the last bits.
+Splitting K is not offered: summing partial products across ranks is split-K, which the method
+excludes.  The only collectives are gathers of finished rows or columns (a copy, exact) and the
+max of per-rank timings.
 """
 from __future__ import annotations
 
@@ -18,6 +21,28 @@ def shard_range(total: int, world: int, rank: int) -> tuple[int, int]:
     begin = rank * base + min(rank, extra)
     end = begin + base + (1 if rank < extra else 0)
     return begin, end
+
+
+def column_shard_range(n: int, world: int, rank: int, align: int = 32) -> tuple[int, int]:
+    """[begin, end) of the output columns rank `rank` of `world` owns in column-parallel sharding:
+    contiguous, balanced in units of `align` columns (the tile width, or 128 for FP8 weights,
+    whose scale blocks a shard must not split)."""
+    if align < 1:
+        raise ValueError("bad alignment")
+    units = (n + align - 1) // align
+    b, e = shard_range(units, world, rank)
+    return min(b * align, n), min(e * align, n)
+
+
+def column_shard_plan(full_plan, world: int, rank: int):
+    """(begin, end, plan) of this rank's column shard of a dense plan, made with
+    bi_gemm_plan_column_shard so that every column keeps the full plan's tile and K order, and
+    so its bits.  FP8 shards are aligned to the 128-column scale blocks."""
+    from . import binding
+    info = binding.bi_gemm_plan_describe(full_plan)
+    align = 128 if info["dtype"] == binding.BI_DTYPE_E4M3_BLOCKSCALED else info["block_n"]
+    b, e = column_shard_range(info["n"], world, rank, align)
+    return b, e, binding.bi_gemm_plan_column_shard(full_plan, b, e)
 
 
 def max_over_ranks(value: float, device=None) -> float:
@@ -50,3 +75,23 @@ def gather_rows(local, total: int, device=None):
         b, e = shard_range(total, world, r)
         out.append(parts[r][: e - b])
     return torch.cat(out).view(local.dtype).reshape((total,) + row_shape)
+
+
+def gather_columns(local, total_cols: int, align: int = 32, device=None):
+    """All-gather the column shards of `local` [rows, cols] (rank r holds the columns
+    column_shard_range(total_cols, world, r, align)) into one [rows, total_cols] tensor on every
+    rank.  A copy of finished values: exact."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size()
+    widths = [e - b for b, e in (column_shard_range(total_cols, world, r, align) for r in range(world))]
+    widest = max(widths)
+    rows = local.shape[0]
+    elt = local.element_size()
+    raw = local.contiguous().view(torch.uint8).reshape(rows, -1)
+    pad = torch.zeros((rows, widest * elt), dtype=torch.uint8, device=local.device)
+    pad[:, : raw.shape[1]] = raw
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad)
+    out = torch.cat([parts[r][:, : widths[r] * elt] for r in range(world)], dim=1)
+    return out.contiguous().view(local.dtype).reshape(rows, total_cols)

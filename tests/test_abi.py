@@ -215,6 +215,34 @@ def test_host_batch_rejects_bad_arguments_before_any_device_call():
         assert run(plan.handle, 2, arr, 4096, need, None, None, None) == S["BI_ERR_NO_DEVICE"]
 
 
+def test_column_shard_plans_keep_the_full_plan():
+    """A shard of the decode plan keeps its tile and two-chain K order, where a plan made for the
+    shard's own shape would not (2048 x 7168 is the prefill table entry: a CTA-pair tile with one
+    chain), so its columns would differ from the full GEMM's in the last bits."""
+    lib = binding.load_library()
+    S = binding.STATUS
+    full = bg.bi_gemm_plan(4096, 7168)
+    fi = bg.bi_gemm_plan_describe(full)
+    shard = bg.bi_gemm_plan_column_shard(full, 2048, 4096)
+    si = bg.bi_gemm_plan_describe(shard)
+    for key in ("block_m", "block_n", "block_k", "cta_group", "mma_m", "mma_n", "mma_k", "k_order_id",
+                "threads_per_cta", "tmem_columns"):
+        assert si[key] == fi[key], key
+    assert si["n"] == 2048 and si["k"] == 7168
+    own = bg.bi_gemm_plan_describe(bg.bi_gemm_plan(2048, 7168))
+    assert (own["block_m"], own["k_order_id"]) != (fi["block_m"], fi["k_order_id"])
+    import ctypes
+    h = ctypes.c_void_p()
+    assert lib.bi_gemm_plan_column_shard(ctypes.byref(h), full.handle, 10, 4097) == S["BI_ERR_INVALID_ARG"]
+    assert lib.bi_gemm_plan_column_shard(ctypes.byref(h), full.handle, 20, 10) == S["BI_ERR_INVALID_ARG"]
+    assert lib.bi_gemm_plan_column_shard(None, full.handle, 0, 10) == S["BI_ERR_INVALID_ARG"]
+    grouped = bg.bi_gemm_plan(2048, 7168, 0, 64)
+    assert lib.bi_gemm_plan_column_shard(ctypes.byref(h), grouped.handle, 0, 10) == S["BI_ERR_INVALID_ARG"]
+    f8 = bg.bi_gemm_plan(7168, 7168, bg.BI_DTYPE_E4M3_BLOCKSCALED)
+    assert lib.bi_gemm_plan_column_shard(ctypes.byref(h), f8.handle, 64, 7168) == S["BI_ERR_UNSUPPORTED_SHAPE"]
+    assert bg.bi_gemm_plan_describe(bg.bi_gemm_plan_column_shard(f8, 3584, 7168))["block_n"] == 64
+
+
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="a GPU is present")
 def test_valid_run_without_a_device_reports_no_device():
     lib = binding.load_library()
