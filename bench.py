@@ -278,6 +278,8 @@ def main():
                     help="M for --profile (MoE: tokens T; attention: batch, sequences of length 4096)")
     ap.add_argument("--profile-splits", type=int, default=4, help="attention: KV splits (1, 2, 4)")
     ap.add_argument("--profile-launches", type=int, default=4)
+    ap.add_argument("--profile-nk", choices=["7168x2048", "2048x7168"], default="7168x2048",
+                    help="prefill: the (N, K) of the weight")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
@@ -442,7 +444,7 @@ def profile_case(args):
     M, L = args.profile_m, args.profile_launches
     calls = []
     if args.profile in ("decode", "prefill"):
-        N, K = (N_DEC, K_DEC) if args.profile == "decode" else (7168, 2048)
+        N, K = (N_DEC, K_DEC) if args.profile == "decode" else tuple(map(int, args.profile_nk.split("x")))
         plan = weight_plan(N, K)
         copies = 3 if args.profile == "decode" else 1
         Bs = [inputs.bf16_gaussian((N, K), seed=11 + i, std=K ** -0.5, device=dev) for i in range(copies)]

@@ -154,37 +154,41 @@ RingGeom ring_geometry(const KernelEntry *k, int a_rows)
             st = bi::kMaxSB;
         return RingGeom{st, st, static_cast<uint32_t>(a_bytes), static_cast<uint32_t>(st * a_bytes)};
     }
+    const int ring = k->grouped ? bi::kRingBytesGrouped : bi::kRingBytes1;
     const int a_stride = k->kc * a_rows * chunk;
-    const int over = (k->bm - a_rows) * chunk;     // the MMA reads BM rows from each A chunk
+    // The MMA reads BM rows from every A chunk: past the last loaded row of the last A slot it
+    // reads on into the B ring, which lies right after the A region and must reach that far.
+    const int over = (k->bm - a_rows) * chunk;
     const int b_stride = k->kc * k->bn * chunk;
+    auto a_region_of = [&](int s) { return (s * a_stride + 1023) / 1024 * 1024; };
     int sa, sb, a_region;
     if (k->bn >= 128) {
-        sa = (bi::kRingBytes - over) / (a_stride + b_stride);
+        sa = ring / (a_stride + b_stride);
         if (sa > bi::kMaxSA)
             sa = bi::kMaxSA;
         sb = sa;
-        a_region = (sa * a_stride + over + 1023) / 1024 * 1024;
-        if (a_region + sb * b_stride > bi::kRingBytes)
-            --sa, --sb, a_region = (sa * a_stride + over + 1023) / 1024 * 1024;
+        a_region = a_region_of(sa);
+        if (a_region + sb * b_stride > ring)
+            --sa, --sb, a_region = a_region_of(sa);
     } else {
-        sa = (96 * 1024 - over) / a_stride;
+        sa = (96 * 1024) / a_stride;
         sa = sa < 2 ? 2 : sa > bi::kMaxSA ? bi::kMaxSA : sa;
         for (;; --sa) {   // deepest A ring that still leaves B at least as deep
-            a_region = (sa * a_stride + over + 1023) / 1024 * 1024;
-            sb = (bi::kRingBytes - a_region) / b_stride;
+            a_region = a_region_of(sa);
+            sb = (ring - a_region) / b_stride;
             if (sb > bi::kMaxSB)
                 sb = bi::kMaxSB;
             if (sb >= sa || sa == 2)
                 break;
         }
     }
+    if (a_region + sb * b_stride < sa * a_stride + over)
+        sb = 0;   // the MMA's reads would leave the ring: reported as an invalid geometry
     // The kernel relies on 2 <= sa <= sb (the A-slot reuse test reads the consumed ring) and, for
     // FP8, on sb groups outlasting the partial-product ring.  Every tile in kKernels satisfies
-    // this for every a_rows in [8, BM], except the small-batch forms, which are valid up to 64
-    // (bf16, 8 chunks) and 96 (FP8, 4 chunks) rows and used up to bi_plan_s::small_rows (64; 32
-    // for two-chain bf16 plans), and the bf16 tiny-batch form (16 chunks), valid and used up to 8
-    // rows; set_rows reports a violation and the launch is refused.  tests/test_abi.py checks the
-    // reported depths.
+    // this for every a_rows in [8, BM], except the bf16 tiny-batch form (16 chunks per group),
+    // valid up to 24 rows and used up to 8; set_rows reports a violation and the launch is
+    // refused.  tests/test_abi.py checks the reported depths.
     return RingGeom{sa, sb, static_cast<uint32_t>(a_stride), static_cast<uint32_t>(a_region)};
 }
 

@@ -51,7 +51,12 @@ namespace bi {
 
 constexpr int kBlockM = 128;        // largest output-tile height = largest MMA M (cta_group::1)
 constexpr int kRowBytes = 128;      // K bytes per stage per row: one 128-byte swizzle row
-constexpr int kRingBytes = 200 * 1024;   // shared memory for the two operand rings
+constexpr int kRingBytes = 200 * 1024;   // shared memory for the two operand rings of a CTA pair
+// One-CTA kernels: as much of the 227 KB (232 448 bytes) a CTA may hold as the rest leaves: the
+// static shared memory (1 KB: the 1024-byte alignment of the dynamic array pads it), the
+// alignment slack, the barriers and (grouped) the expert tables.
+constexpr int kRingBytes1 = 224 * 1024;
+constexpr int kRingBytesGrouped = 214 * 1024;
 constexpr int kEpilogueWarps = 4;                       // bf16 (and narrow FP8) epilogue warps
 constexpr int kThreads = (2 + kEpilogueWarps) * 32;
 
@@ -67,22 +72,20 @@ struct Epi {
 
 // MMA-issuing threads of a kernel.  A thread's next tcgen05.mma waits on the issue of its previous
 // one, which costs ~50 cycles beyond the instruction's math for these tile shapes; two issuing
-// threads overlap that cost.  Two issuers split the work so that every accumulator still receives
-// its instructions from one thread in ascending K:
-//   - by column half, in the dense wide lockstep form (NSPLIT = 2);
-//   - by K-chunk parity, in the other dense FP8 forms with an even number of chunks per group: each
-//     128-wide K chunk has its own partial-product buffer, and the epilogue promotes the buffers in
-//     ascending kb whoever issued them.
-//   - by K-chunk parity in the dense bf16 kernels with two K chains (CH = 2, any NSPLIT): chain p
-//     accumulates the chunks of parity p into an accumulator of its own, and the epilogue adds
-//     the two chains once.
-// The grouped wide form (two 128 x 128 instructions per K step) is bound by shared-memory bandwidth
-// instead and keeps one issuer.  The second issuer is the warp after the epilogue warps.
+// threads overlap that cost.  Two issuers split the work by K-chunk parity, so that every
+// accumulator still receives its instructions from one thread in ascending K:
+//   - in the dense FP8 kernels with an even number of chunks per group: each 128-wide K chunk has
+//     its own partial-product buffer, and the epilogue promotes the buffers in ascending kb
+//     whoever issued them;
+//   - in the dense bf16 kernels with two K chains (CH = 2): chain p accumulates the chunks of
+//     parity p into an accumulator of its own, and the epilogue adds the two chains once.
+// Grouped kernels keep one issuer: their instructions are wide enough (128 x 128 or 128 x 256)
+// for one thread to keep the tensor pipe fed.  The second issuer is the warp after the epilogue
+// warps.
 template <bool FP8, int BN, int NSPLIT, bool GROUPED = false, int KC = 1, int CH = 1>
 struct Issue {
-    static constexpr bool kByChunk = !GROUPED && KC % 2 == 0 && (FP8 ? NSPLIT == 1 : CH == 2);
-    static constexpr bool kBySplit = !GROUPED && NSPLIT == 2 && !kByChunk;
-    static constexpr int kIssuers = (kBySplit || kByChunk) ? 2 : 1;
+    static constexpr bool kByChunk = !GROUPED && KC % 2 == 0 && (FP8 || CH == 2);
+    static constexpr int kIssuers = kByChunk ? 2 : 1;
     static constexpr int kSecondWarp = 2 + Epi<FP8, BN>::kWarps;
     static constexpr int kThreads = Epi<FP8, BN>::kThreads + (kIssuers - 1) * 32;
 };
@@ -150,12 +153,23 @@ struct TileCoord {
 
 // Operand rings.  A pipeline stage ("group") carries KC 128-byte K chunks: KC chunks of A rows
 // and KC chunks of BN B rows.  The ring depths and the A slot size are chosen per launch by the
-// host (GemmParams::sa, sb, a_stride, b_offset) inside kRingBytes: when a dense problem has
-// fewer rows than the tile, an A slot only holds the roundup(M, 8) rows TMA brings, which leaves
-// more of shared memory to the B (weight) ring.  The ring geometry decides how far ahead loads
-// run, never what the MMA computes.
+// host (GemmParams::sa, sb, a_stride, b_offset) inside the kernel's ring bytes (ring_bytes_1cta):
+// when a dense problem has fewer rows than the tile, an A slot only holds the rows TMA brings,
+// which leaves more of shared memory to the B (weight) ring.  The MMA still reads BM rows from
+// every A chunk; the rows past the loaded ones lie in the next chunk, slot or the B ring (the host
+// keeps them inside the ring) and feed only output rows that are never stored.  The ring geometry
+// decides how far ahead loads run, never what the MMA computes.
 constexpr int kMaxSA = 8;
 constexpr int kMaxSB = 32;
+
+template <bool GROUPED>
+__host__ __device__ constexpr int ring_bytes_1cta()
+{
+    return GROUPED ? kRingBytesGrouped : kRingBytes1;
+}
+static_assert(1024 + 1024 + kRingBytes1 + 1024 <= 232448, "one-CTA dense ring too large");
+static_assert(1024 + 1024 + kRingBytesGrouped + 1024 + 2 * (kMaxExperts + 1) * 4 <= 232448,
+              "one-CTA grouped ring too large");
 
 template <int BM, int BN, int KC>
 struct Rings {
@@ -505,13 +519,15 @@ __global__ void __launch_bounds__(256) bi_w4_rowsum_kernel(const uint8_t *a, int
 //           box per operand (chunk index as the third coordinate), so the producer and MMA
 //           threads pay their per-stage handshakes once per KC chunks.  The MMA still walks the
 //           chunks of a tile one by one in ascending K: KC changes no bit of the result.
-// NSPLIT  : MMAs per K step.  The MMA instruction is BM x (BN / NSPLIT) x K; split s covers the
-//           tile's columns [s BN/NSPLIT, (s+1) BN/NSPLIT) and accumulates into the same columns
-//           of the TMEM accumulator (FP8: of each partial-product buffer).  NSPLIT = 4 (two-chain
-//           bf16 only) runs four adjacent 32-column tiles the same way.  NSPLIT = 2 runs two
-//           adjacent (BN/2)-wide tiles of a plan in lockstep on one A operand: every output
-//           element is still computed by a BM x (BN/2) x K instruction sequence in ascending K
-//           (FP8: and promoted in ascending kb), as in a (BN/2)-wide launch.
+// NSPLIT  : adjacent tiles of a plan, each BN/NSPLIT wide, that one CTA runs in lockstep on one
+//           A operand (the wide forms: 2, or 4 for two-chain bf16 plans).  One BM x BN x K
+//           instruction covers them at every K step, into adjacent TMEM columns.  tcgen05 forms
+//           every element of D from its own row of A and column of B, accumulator and K step,
+//           the same way whatever the instruction's N, so each output element gets the bits the
+//           plan's (BN/NSPLIT)-wide instruction gives it, with the same K order (FP8: promoted in
+//           the same ascending kb); the invariance tests compare the forms bit for bit, also on
+//           inputs built to expose a different internal summation (wide exponent spreads,
+//           cancellation).
 // SPLIT   : the fixed-split-K research variant (bf16 dense only, not the batch-invariant product
 //           path): a work unit is one K split of a tile and its epilogue writes fp32 partial
 //           sums; bi_splitk_merge_kernel adds the splits in a fixed order.
@@ -545,12 +561,12 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
     static_assert(NSPLIT == 1 ||
                       (NSPLIT == 2 && (GROUPED ? (!FP8 && BN == 256) : BN == (FP8 ? 128 : 64))) ||
                       (NSPLIT == 4 && CH == 2 && BN == 128),
-                  "split MMAs: dense bf16 64-wide, FP8 128-wide and grouped bf16 256-wide tiles as "
-                  "two half-width instructions; two-chain bf16 128-wide tiles as four quarters");
+                  "lockstep tiles: dense bf16 64-wide, FP8 128-wide and grouped bf16 256-wide "
+                  "tiles hold two plan tiles; two-chain bf16 128-wide tiles hold four");
     static_assert(!SPLIT || (!FP8 && !GROUPED && NSPLIT == 1), "split-K variant: bf16 dense");
     static_assert(!W4 || (FP8 && !GROUPED && !SPLIT), "e2m1 weights: the dense FP8 kernel");
     static_assert(CH == 1 || (CH == 2 && !FP8 && !GROUPED && !SPLIT), "two K chains: dense bf16");
-    constexpr int kMmaN = BN / NSPLIT;                   // MMA instruction N
+    constexpr int kMmaN = BN;                            // MMA instruction N (all NSPLIT tiles)
     using Iss = Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>;
     constexpr int kIssuers = Iss::kIssuers;              // threads issuing MMAs
     using R = Rings<BM, BN, KC>;
@@ -585,7 +601,7 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *smem_a = smem;
     uint8_t *smem_b = smem + p.b_offset;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kRingBytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + ring_bytes_1cta<GROUPED>());
     // full[j % sb]: both TMA loads of group j landed (two arrivals: the B load and, issued
     // later, the A load).  consumed[j % sb]: the MMAs of group j completed, which frees B slot
     // j % sb and A slot j % sa (one commit per group).  A group's two arrivals always land in
@@ -844,14 +860,12 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
         }
     } else if (warp == 1 || (kIssuers > 1 && warp == Iss::kSecondWarp)) {
         // ------------------------------------------------------------------ MMA issuers
-        // Issuer `iss` issues the MMAs of split iss (wide form) or of the K chunks of parity iss
-        // (FP8), each accumulator's instructions in ascending K.  Both issuers wait on the same
-        // barriers, and each commits every group (the consumed and accumulator-full barriers count
-        // one commit per issuer), so a slot or an accumulator is handed on when both are done.
+        // Issuer `iss` issues the MMAs of the K chunks of parity iss (FP8, two-chain bf16), each
+        // accumulator's instructions in ascending K.  Both issuers wait on the same barriers, and
+        // each commits every group (the consumed and accumulator-full barriers count one commit
+        // per issuer), so a slot or an accumulator is handed on when both are done.
         const int iss = warp == 1 ? 0 : 1;
-        const int split_iss = Iss::kBySplit ? iss : 0;
         const int chunk_iss = Iss::kByChunk ? iss : 0;
-        constexpr int kSplitsPerIssuer = Iss::kBySplit ? NSPLIT / 2 : NSPLIT;
         if (lane == 0) {
             const int SA = p.sa, SB = p.sb;
             int sa = 0, sb = 0;      // ring slots of the next group
@@ -931,18 +945,11 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
                             // bf16: accumulate across the whole K of the tile (of the chunk's
                             // chain); FP8: one K chunk
                             const uint32_t accumulate = (q > 0) ? 1u : (FP8 ? 0u : (chunk >= CH ? 1u : 0u));
-#pragma unroll
-                            for (int j = 0; j < kSplitsPerIssuer; ++j) {
-                                // split sp: B rows and accumulator columns [sp kMmaN, (sp+1) kMmaN)
-                                const int sp = j + split_iss;
-                                const uint64_t b_sp = static_cast<uint64_t>((sp * kMmaN * kRowBytes) >> 4);
-                                if constexpr (FP8)
-                                    ptx::mma_e4m3_ss(d + sp * kMmaN, a_desc + step, b_desc + b_sp + step,
-                                                     kIdesc, accumulate);
-                                else
-                                    ptx::mma_bf16_ss(d + sp * kMmaN, a_desc + step, b_desc + b_sp + step,
-                                                     kIdesc, accumulate);
-                            }
+                            // all BN columns (every lockstep tile) in one instruction
+                            if constexpr (FP8)
+                                ptx::mma_e4m3_ss(d, a_desc + step, b_desc + step, kIdesc, accumulate);
+                            else
+                                ptx::mma_bf16_ss(d, a_desc + step, b_desc + step, kIdesc, accumulate);
                         }
                         return true;
                     };
@@ -1182,7 +1189,7 @@ template <int BM, int BN, int KC, bool FP8, bool GROUPED, int NSPLIT = 1, bool S
           bool W4 = false, int CH = 1>
 constexpr int smem_bytes_for()
 {
-    return 1024 + kRingBytes + 1024 + (GROUPED ? 2 * (kMaxExperts + 1) * 4 : 0);
+    return 1024 + ring_bytes_1cta<GROUPED>() + 1024 + (GROUPED ? 2 * (kMaxExperts + 1) * 4 : 0);
 }
 
 } // namespace bi

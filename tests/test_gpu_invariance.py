@@ -123,6 +123,43 @@ def test_scheduling_forms_of_one_plan_agree_bitwise():
                        positions=sorted({q for q in (0, 63, 64, 127, 128, M - 1) if q < M}))
 
 
+def adversarial_bf16(shape, kind, seed):
+    """bf16 operands built to expose any difference in how an instruction sums its K products:
+    exponents spread over 2^-24..2^24 ("wide"), pairs that cancel to a few ulps ("cancel"), or a
+    small background under 1 % large spikes ("spikes")."""
+    g = torch.Generator().manual_seed(seed)
+    if kind == "spikes":
+        x = torch.randn(shape, generator=g) * 2.0 ** -10
+        mask = torch.rand(shape, generator=g) < 0.01
+        x[mask] = torch.randn(int(mask.sum()), generator=g) * 2.0 ** 10
+        return x.to(torch.bfloat16).to(DEV)
+    e = torch.randint(-24, 25, shape, generator=g).float()
+    sign = torch.randint(0, 2, shape, generator=g).float() * 2 - 1
+    x = sign * (1 + torch.rand(shape, generator=g)) * torch.exp2(e)
+    if kind == "cancel":
+        odd = x[..., 1::2]
+        x[..., 1::2] = -x[..., 0::2][..., : odd.shape[-1]] * (
+            1 + 2.0 ** -7 * torch.randint(-2, 3, odd.shape, generator=g).float())
+    return x.to(torch.bfloat16).to(DEV)
+
+
+@pytest.mark.parametrize("kind", ["wide", "cancel", "spikes"])
+def test_scheduling_forms_agree_bitwise_on_adversarial_inputs(kind):
+    # The wide lockstep forms issue one 64 x 64 or 64 x 128 instruction where the plan's own form
+    # issues 64 x 32 ones; the rows of every form must still carry the M = 1 bits, on inputs whose
+    # sums depend on the order and width of each instruction's internal reduction.
+    N, K = 4128, 7232
+    B = adversarial_bf16((N, K), kind, 2201)
+    f = Dense(B)
+    test_rows = adversarial_bf16((16, K), kind, 2202)
+    ref = alone(f, test_rows)
+    for M in [8, 20, 64, 100, 300]:
+        s = inputs.derived_seed(2200, M, 0)
+        fresh = lambda m, s=s: adversarial_bf16((m, K), kind, s)
+        check_in_batch(f, test_rows, ref, M, s, fresh,
+                       positions=sorted({q for q in (0, 31, 63, 64, 127, 128, 255, M - 1) if q < M}))
+
+
 # ---------------------------------------------------------------------------------------------
 # prefill-shaped: both shapes, M in {1024, 4096, 16384}, plus the 1024-row subset test
 # ---------------------------------------------------------------------------------------------
@@ -168,6 +205,35 @@ def test_fp8_rows_invariant_across_m_sweep():
                            scales=test_scales,
                            fresh_scales=lambda m, s=s: inputs.scales_log_uniform((m, KB), seed=s + 1,
                                                                                  device=DEV))
+
+
+def e4m3_any_codes(shape, seed):
+    """Uniformly random e4m3 codes over the whole format (subnormals to +-448, no NaN)."""
+    g = torch.Generator().manual_seed(seed)
+    c = torch.randint(0, 256, shape, generator=g, dtype=torch.int32)
+    c = torch.where((c & 0x7F) == 0x7F, c - 1, c)   # 0x7F / 0xFF are NaN in e4m3fn
+    return c.to(torch.uint8).view(torch.float8_e4m3fn).to(DEV)
+
+
+def test_fp8_forms_agree_bitwise_on_full_range_codes():
+    # The FP8 wide lockstep form issues one 128 x 128 x 32 instruction where the plan's form
+    # issues 128 x 64 x 32 ones; with codes spread over the whole e4m3 range the products of one
+    # instruction span ~2^34, so any difference in its internal alignment would show.
+    N = K = 7168
+    KB = K // 128
+    qb = e4m3_any_codes((N, K), 4101)
+    sb = inputs.scales_log_uniform((N // 128, KB), seed=4102, device=DEV)
+    f = Dense(qb, bg.BI_DTYPE_E4M3_BLOCKSCALED, scale_b=sb)
+    test_rows = e4m3_any_codes((8, K), 4103)
+    test_scales = inputs.scales_log_uniform((8, KB), seed=4104, device=DEV)
+    ref = alone(f, test_rows, test_scales)
+    for M in [16, 256, 1024]:
+        s = inputs.derived_seed(4100, M)
+        check_in_batch(f, test_rows, ref, M, s, lambda m, s=s: e4m3_any_codes((m, K), s),
+                       scales=test_scales,
+                       fresh_scales=lambda m, s=s: inputs.scales_log_uniform((m, KB), seed=s + 1,
+                                                                             device=DEV),
+                       positions=[0, 127, 128, M - 1] if M > 128 else [0, M - 1])
 
 
 # ---------------------------------------------------------------------------------------------
@@ -250,3 +316,21 @@ def test_moe_adversarial_routings(pattern):
             {"smem_bytes": dense_info["smem_bytes"]}
         if same:
             assert torch.equal(f(tokens).view(torch.int16), C)
+
+
+@pytest.mark.parametrize("kind", ["cancel", "spikes"])
+def test_moe_wide_form_agrees_bitwise_on_adversarial_inputs(kind):
+    # 1200 rows over 8 experts (>= 128 per expert on average) take the grouped wide form, one
+    # 128 x 256 instruction per K step; a row alone takes the plan's 128 x 128 form.
+    E, N, K = 8, 2048, 7168
+    plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_BF16, E)
+    B = adversarial_bf16((E, N, K), kind, 5201)
+    tokens = adversarial_bf16((1200, K), kind, 5202)
+    experts = np.sort(np.random.default_rng(5203).integers(0, E, 1200))
+    r = routing_mod.routing_from_assignment(experts, E)
+    C = moe_outputs(plan, B, tokens, r)
+    for i in np.random.default_rng(5204).choice(1200, 24, replace=False):
+        e = int(experts[i])
+        one = routing_mod.routing_from_assignment(np.array([e]), E)
+        C1 = moe_outputs(plan, B, tokens[i:i + 1], one)
+        assert torch.equal(C1[0], C[i]), f"{kind}: row {i}"
