@@ -75,11 +75,14 @@ typedef enum {
 /* Opaque, library-owned plan. */
 typedef struct bi_plan_s *bi_plan_t;
 
-/* What a plan fixed.  None of it depends on M, except the pipeline grouping, which is reported
- * for a full-height tile: a launch whose whole problem has fewer rows than one tile sizes its A
- * slots to those rows and deepens both rings, and a bf16 128 x 32 (FP8 128 x 64) plan groups 8
- * (4) K chunks per pipeline stage when A has at most 64 rows (scheduling only; the tile, the MMA
- * instruction and the K order are fixed, so no row's result changes). */
+/* What a plan fixed.  None of it depends on M, except the scheduling, which is reported for a
+ * full-height tile: a launch whose whole problem has fewer rows than one tile sizes its A slots
+ * to those rows and deepens both rings; a bf16 64 x 32 (FP8 128 x 64) plan groups 8 (4) K chunks
+ * per pipeline stage when A has at most 32 (64) rows, and the bf16 plan 16 below 8 rows; and a
+ * launch with more tiles than SMs runs two or four adjacent tiles in lockstep, with one
+ * instruction as wide as those tiles together.  The tile, the instruction's M and K and the K
+ * order are fixed, and tcgen05 computes each output element the same way whatever the
+ * instruction's N, so no row's result changes. */
 typedef struct {
     int64_t n, k;              /* the plan's N and K */
     int dtype;                 /* bi_dtype_t */
@@ -95,9 +98,14 @@ typedef struct {
                                   1 = fixed split-K research plan (see bi_gemm_plan_splitk);
                                   2 = whole K per CTA in two fixed interleaved chains: the
                                       128-byte K chunks 0, 2, 4, ... and 1, 3, 5, ... are each
-                                      accumulated in ascending K, then C = chain0 + chain1 once
-                                      (dense bf16 plans of 32-column tiles).  Fixed by K alone:
-                                      the same for every M, row position and scheduling form. */
+                                      accumulated in ascending K, then C = chain0 + chain1 once;
+                                  3 = whole K per CTA in four fixed interleaved chains: chain c
+                                      accumulates the chunks c, c + 4, c + 8, ... in ascending K,
+                                      then C = (chain0 + chain1) + (chain2 + chain3) once, chains
+                                      that K leaves empty left out (dense bf16 plans of
+                                      32-column tiles).
+                                  Every order is fixed by K alone: the same for every M, row
+                                  position and scheduling form. */
     int threads_per_cta;
     int smem_bytes;            /* dynamic shared memory per CTA */
     int tmem_columns;          /* tensor-memory columns allocated per CTA */

@@ -79,29 +79,30 @@ struct KernelEntry {
                 &bi::bi_gemm_kernel_pair<BN, KC, F8, GR>,                                          \
                 bi::smem_bytes_for_pair<BN, KC, F8, GR>(), 1, false, false, 1}
 
-#define BI_ENTRY_CH2(BM, BN, KC)                                                                   \
-    KernelEntry{bi::Issue<false, BN, 1, false, KC, 2>::kThreads, BM, BN, KC, false, false, false,   \
-                &bi::bi_gemm_kernel<BM, BN, KC, false, false, 1, false, false, 2>,                 \
-                bi::smem_bytes_for<BM, BN, KC, false, false, 1, false, false, 2>(), 1, false, false, 2}
-#define BI_ENTRY_CH2_SPLITN(BM, BN, KC, NS)                                                        \
-    KernelEntry{bi::Issue<false, BN, NS, false, KC, 2>::kThreads, BM, BN, KC, false, false, false,  \
-                &bi::bi_gemm_kernel<BM, BN, KC, false, false, NS, false, false, 2>,                \
-                bi::smem_bytes_for<BM, BN, KC, false, false, NS, false, false, 2>(), NS, false,    \
-                false, 2}
+#define BI_ENTRY_CHAINS(BM, BN, KC, CHN)                                                           \
+    KernelEntry{bi::Issue<false, BN, 1, false, KC, CHN>::kThreads, BM, BN, KC, false, false, false, \
+                &bi::bi_gemm_kernel<BM, BN, KC, false, false, 1, false, false, CHN>,               \
+                bi::smem_bytes_for<BM, BN, KC, false, false, 1, false, false, CHN>(), 1, false,    \
+                false, CHN}
+#define BI_ENTRY_CHAINS_SPLITN(BM, BN, KC, NS, CHN)                                                \
+    KernelEntry{bi::Issue<false, BN, NS, false, KC, CHN>::kThreads, BM, BN, KC, false, false,      \
+                false, &bi::bi_gemm_kernel<BM, BN, KC, false, false, NS, false, false, CHN>,       \
+                bi::smem_bytes_for<BM, BN, KC, false, false, NS, false, false, CHN>(), NS, false,  \
+                false, CHN}
 
 // Narrow tiles (BN <= 64) run on one CTA; wide ones (BN >= 128) on a CTA pair.  Every tile comes
 // in two forms: its preferred number of 128-byte K chunks per pipeline stage (3-D TMA boxes;
 // needs K to be a multiple of the chunk), and one chunk per stage for any other K.  The bf16
-// 128 x 32 and the FP8 128 x 64 tiles have a third, small-batch form with twice the preferred
-// chunks per stage (the bf16 tile a fourth, tiny-batch form with 16), and a wide form that runs
-// two adjacent tiles in lockstep on one A operand (see dense_kernel_for).
+// 64 x 32 and the FP8 128 x 64 tiles have a third, small-batch form with twice the preferred
+// chunks per stage (the bf16 tile a fourth, tiny-batch form with 16), and wide forms that run
+// two (bf16: or four) adjacent tiles in lockstep on one A operand (see dense_kernel_for).
 const KernelEntry kKernels[] = {
-    // bf16 32-column tiles: 64-row MMA, two K chains on two issuing threads (the plan form, the
-    // small- and tiny-batch forms, one chunk per stage for K not a multiple of 64, and the wide
-    // lockstep forms of two and four tiles)
-    BI_ENTRY_CH2(64, 32, 1),            BI_ENTRY_CH2(64, 32, 4),
-    BI_ENTRY_CH2(64, 32, 8),            BI_ENTRY_CH2(64, 32, 16),
-    BI_ENTRY_CH2_SPLITN(64, 64, 4, 2),  BI_ENTRY_CH2_SPLITN(64, 128, 2, 4),
+    // bf16 32-column tiles: 64-row MMA, four K chains on up to four issuing threads (the plan
+    // form, the small- and tiny-batch forms, one chunk per stage for K not a multiple of 64, and
+    // the wide lockstep forms of two and four tiles)
+    BI_ENTRY_CHAINS(64, 32, 1, 4),            BI_ENTRY_CHAINS(64, 32, 4, 4),
+    BI_ENTRY_CHAINS(64, 32, 8, 4),            BI_ENTRY_CHAINS(64, 32, 16, 4),
+    BI_ENTRY_CHAINS_SPLITN(64, 64, 4, 2, 4),  BI_ENTRY_CHAINS_SPLITN(64, 128, 2, 4, 4),
     BI_ENTRY(128, 64, 1, false, false), BI_ENTRY(128, 64, 2, false, false),
     BI_ENTRY(128, 32, 1, true, false),  BI_ENTRY(128, 32, 4, true, false),
     BI_ENTRY(128, 64, 1, true, false),  BI_ENTRY(128, 64, 2, true, false),
@@ -360,7 +361,7 @@ struct bi_plan_s {
     // order), for dense launches with more tiles than SMs and grouped launches with at least a
     // tile's worth of rows per expert on average.  May be null.
     const KernelEntry *kernel_wide = nullptr;
-    // Four adjacent tiles in lockstep (two-chain plans), for dense launches whose lockstep pairs
+    // Four adjacent tiles in lockstep (bf16 plans with K chains), for dense launches whose lockstep pairs
     // still outnumber the SMs.  May be null.
     const KernelEntry *kernel_wide4 = nullptr;
     int small_rows = 64;     // kernel_small serves launches whose A boxes hold at most this many rows
@@ -565,12 +566,13 @@ bi_status_t check_fp8_scales(int64_t M, const float *scale_a, int64_t ld_sa, con
     return BI_OK;
 }
 
-// Dense bf16 plans of 32-column tiles use the 64-row MMA with two K chains: with two issuing
-// threads the 64 x 32 x 16 instruction issues at ~29 cycles (one thread: ~57 cycles, whatever the
-// shape), and it reads half the shared-memory A rows of the 128-row one.
+// Dense bf16 plans of 32-column tiles use the 64-row MMA with four K chains on four issuing
+// threads: one thread issues a tcgen05.mma every ~57 cycles whatever the shape, two on
+// independent accumulators every ~29 and four every ~25 cycles, close to the 24 shared-memory
+// wavefronts one 64 x 32 x 16 instruction reads (half the A rows of the 128-row instruction).
 int chains_for(const TileChoice &tile, bool fp8, int experts)
 {
-    return (!fp8 && experts == 1 && tile.bm == 64 && tile.bn == 32) ? 2 : 1;
+    return (!fp8 && experts == 1 && tile.bm == 64 && tile.bn == 32) ? 4 : 1;
 }
 
 // Rows of A one TMA load brings for a dense problem of M rows: the tile's 128 rows, or, when the
@@ -692,16 +694,16 @@ int b_box_rows_for(const KernelEntry *k)
 // small-batch kernel form (when it has one): with few A rows, groups of twice the chunks halve
 // the per-group wait and commit overhead of the MMA threads, and the ring still holds two groups
 // of A and of B (and, for FP8, more groups than partial-product buffers).  At most this many
-// rows take the tiny-batch form (16 chunks per group): the 8-row A boxes leave room for two
-// 64 KB groups of B.
-constexpr int kTinyBatchRows = 8;
+// rows take the tiny-batch form (16 chunks per group), whose per-chunk A loads of exactly M rows
+// (bi::GemmParams::a_exact_rows) cost 16 TMA issues per group: it pays below 8 rows only.
+constexpr int kTinyBatchRows = 7;
 
 // A dense launch with more tiles than the device has SMs takes the plan's wide form (when it has
 // one): a CTA runs two adjacent column tiles in lockstep, so each A chunk is loaded once for both
 // and the launch needs half the CTAs, i.e. fewer waves.
 const KernelEntry *dense_kernel_for(const bi_plan_s *plan, const DeviceInfo *d, int64_t M)
 {
-    if (plan->kernel_tiny && a_box_rows_for(plan->kernel_tiny, M) <= kTinyBatchRows)
+    if (plan->kernel_tiny && M <= kTinyBatchRows)
         return plan->kernel_tiny;
     if (plan->kernel_small && a_box_rows_for(plan->kernel_small, M) <= plan->small_rows)
         return plan->kernel_small;
@@ -809,20 +811,20 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     p->dtype = dtype;
     p->experts = num_experts;
     p->kernel = k;
-    if (num_experts == 1 && !k->pair && (k->bm == 128 || k->chains == 2) &&
+    if (num_experts == 1 && !k->pair && (k->bm == 128 || k->chains > 1) &&
         k->kc == preferred_chunks(k->bn) && k->bn == (fp8 ? 64 : 32))
         p->kernel_small = find_kernel(k->bm, k->bn, 2 * k->kc, fp8, false, w4, chains);
     if (p->kernel_small && !fp8 && p->kernel_small->kc == 8)
         p->kernel_tiny = find_kernel(k->bm, k->bn, 16, false, false, false, chains);
-    // two-chain plans take the 8-chunk form up to 32 rows: their 64-row A boxes would leave a
-    // 64 KB B ring at 8 chunks, while 4 chunks keep six B groups in flight
-    p->small_rows = chains == 2 ? 32 : 64;
+    // plans with K chains take the 8-chunk form up to 32 rows: their 64-row A boxes would leave
+    // a 96 KB B ring at 8 chunks, while 4 chunks keep eight B groups in flight
+    p->small_rows = chains > 1 ? 32 : 64;
     if (num_experts > 1 && !k->pair && k->bm == 128 && k->bn == 128) {
         for (int i = 0; i < kNumKernels; ++i)
             if (kKernels[i].nsplit == 2 && kKernels[i].grouped && kKernels[i].bn == 256)
                 p->kernel_wide = &kKernels[i];
     }
-    if (num_experts == 1 && !k->pair && (k->bm == 128 || k->chains == 2) &&
+    if (num_experts == 1 && !k->pair && (k->bm == 128 || k->chains > 1) &&
         k->bn == (fp8 ? 64 : 32) && K % chunk_elems == 0 && K > 0) {
         for (int i = 0; i < kNumKernels; ++i)
             if (kKernels[i].bm == k->bm && kKernels[i].fp8 == fp8 && kKernels[i].w4 == w4 &&
@@ -917,7 +919,7 @@ bi_status_t bi_gemm_plan_describe(bi_plan_t plan, bi_plan_info_t *info)
     const RingGeom g = ring_geometry(plan->kernel, plan->kernel->bm);
     info->stages = g.sb;
     info->stages_a = g.sa;
-    info->k_order_id = plan->k_splits > 1 ? 1 : plan->kernel->chains == 2 ? 2 : 0;
+    info->k_order_id = plan->k_splits > 1 ? 1 : plan->kernel->chains == 4 ? 3 : plan->kernel->chains == 2 ? 2 : 0;
     info->k_splits = plan->k_splits;
     info->threads_per_cta = plan->kernel->threads;
     info->smem_bytes = plan->kernel->smem;

@@ -71,21 +71,27 @@ struct Epi {
 };
 
 // MMA-issuing threads of a kernel.  A thread's next tcgen05.mma waits on the issue of its previous
-// one, which costs ~50 cycles beyond the instruction's math for these tile shapes; two issuing
-// threads overlap that cost.  Two issuers split the work by K-chunk parity, so that every
-// accumulator still receives its instructions from one thread in ascending K:
-//   - in the dense FP8 kernels with an even number of chunks per group: each 128-wide K chunk has
-//     its own partial-product buffer, and the epilogue promotes the buffers in ascending kb
-//     whoever issued them;
-//   - in the dense bf16 kernels with two K chains (CH = 2): chain p accumulates the chunks of
-//     parity p into an accumulator of its own, and the epilogue adds the two chains once.
+// one, which costs ~57 cycles whatever the instruction's shape; several issuing threads overlap
+// that cost.  The K chunks of a group are dealt to the issuers round robin (chunk c to issuer
+// c % kIssuers), so that every accumulator still receives its instructions from one thread in
+// ascending K:
+//   - in the dense FP8 kernels with an even number of chunks per group (two issuers): each
+//     128-wide K chunk has its own partial-product buffer, and the epilogue promotes the buffers
+//     in ascending kb whoever issued them;
+//   - in the dense bf16 kernels with CH = 2 or 4 K chains: chain c accumulates the chunks with
+//     chunk % CH == c into an accumulator of its own, and the epilogue adds the chains once.  As
+//     many issuers as chains when a group's chunk count allows it (kIssuers divides both CH and
+//     KC), so each chain belongs to one issuer.
 // Grouped kernels keep one issuer: their instructions are wide enough (128 x 128 or 128 x 256)
-// for one thread to keep the tensor pipe fed.  The second issuer is the warp after the epilogue
+// for one thread to keep the tensor pipe fed.  The extra issuers are the warps after the epilogue
 // warps.
 template <bool FP8, int BN, int NSPLIT, bool GROUPED = false, int KC = 1, int CH = 1>
 struct Issue {
-    static constexpr bool kByChunk = !GROUPED && KC % 2 == 0 && (FP8 || CH == 2);
-    static constexpr int kIssuers = kByChunk ? 2 : 1;
+    static constexpr int kIssuers = GROUPED ? 1
+                                    : FP8   ? (KC % 2 == 0 ? 2 : 1)
+                                    : (CH == 4 && KC % 4 == 0) ? 4
+                                    : (CH >= 2 && KC % 2 == 0) ? 2 : 1;
+    static constexpr bool kByChunk = kIssuers > 1;
     static constexpr int kSecondWarp = 2 + Epi<FP8, BN>::kWarps;
     static constexpr int kThreads = Epi<FP8, BN>::kThreads + (kIssuers - 1) * 32;
 };
@@ -520,7 +526,7 @@ __global__ void __launch_bounds__(256) bi_w4_rowsum_kernel(const uint8_t *a, int
 //           threads pay their per-stage handshakes once per KC chunks.  The MMA still walks the
 //           chunks of a tile one by one in ascending K: KC changes no bit of the result.
 // NSPLIT  : adjacent tiles of a plan, each BN/NSPLIT wide, that one CTA runs in lockstep on one
-//           A operand (the wide forms: 2, or 4 for two-chain bf16 plans).  One BM x BN x K
+//           A operand (the wide forms: 2, or 4 for bf16 plans with K chains).  One BM x BN x K
 //           instruction covers them at every K step, into adjacent TMEM columns.  tcgen05 forms
 //           every element of D from its own row of A and column of B, accumulator and K step,
 //           the same way whatever the instruction's N, so each output element gets the bits the
@@ -531,12 +537,13 @@ __global__ void __launch_bounds__(256) bi_w4_rowsum_kernel(const uint8_t *a, int
 // SPLIT   : the fixed-split-K research variant (bf16 dense only, not the batch-invariant product
 //           path): a work unit is one K split of a tile and its epilogue writes fp32 partial
 //           sums; bi_splitk_merge_kernel adds the splits in a fixed order.
-// CH      : K chains of a dense bf16 tile, 1 or 2.  With 2, the 128-byte K chunks of even index
-//           are accumulated, in ascending K, into one accumulator and those of odd index into a
-//           second one, each by its own issuing thread, and the epilogue forms
-//           C = bf16_rne(chain0 + chain1) once (chain0 alone when K has one chunk).  The order is
-//           fixed by K alone -- the same for every M, row and scheduling form -- and stays inside
-//           one CTA: no workspace, no atomics, no cross-CTA reduction.
+// CH      : K chains of a dense bf16 tile, 1, 2 or 4.  Chain c accumulates, in ascending K, the
+//           128-byte K chunks with chunk % CH == c into an accumulator of its own (each chain
+//           issued by one thread), and the epilogue adds the chains once, in a fixed tree:
+//           C = bf16_rne(chain0 + chain1) for 2, C = bf16_rne((chain0 + chain1) + (chain2 +
+//           chain3)) for 4, leaving out the chains K leaves empty.  The order is fixed by K
+//           alone -- the same for every M, row and scheduling form -- and stays inside one CTA:
+//           no workspace, no atomics, no cross-CTA reduction.
 // W4      : (with FP8, dense) B holds e2m1 weights with one power-of-two scale and one zero point
 //           per output column ("DeepSeek V4的batch invariance：大模型确定性推理的工程基石"
 //           (lshu.cn), section 4.3: W = W_fp4 * scale + zero, scale in {2^-j : j = 1..12}).  The
@@ -560,12 +567,13 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
     static_assert(KC >= 1 && KC <= 16, "1..16 chunks per group");
     static_assert(NSPLIT == 1 ||
                       (NSPLIT == 2 && (GROUPED ? (!FP8 && BN == 256) : BN == (FP8 ? 128 : 64))) ||
-                      (NSPLIT == 4 && CH == 2 && BN == 128),
+                      (NSPLIT == 4 && CH >= 2 && BN == 128),
                   "lockstep tiles: dense bf16 64-wide, FP8 128-wide and grouped bf16 256-wide "
-                  "tiles hold two plan tiles; two-chain bf16 128-wide tiles hold four");
+                  "tiles hold two plan tiles; bf16 128-wide tiles with K chains hold four");
     static_assert(!SPLIT || (!FP8 && !GROUPED && NSPLIT == 1), "split-K variant: bf16 dense");
     static_assert(!W4 || (FP8 && !GROUPED && !SPLIT), "e2m1 weights: the dense FP8 kernel");
-    static_assert(CH == 1 || (CH == 2 && !FP8 && !GROUPED && !SPLIT), "two K chains: dense bf16");
+    static_assert(CH == 1 || ((CH == 2 || CH == 4) && !FP8 && !GROUPED && !SPLIT),
+                  "two or four K chains: dense bf16");
     constexpr int kMmaN = BN;                            // MMA instruction N (all NSPLIT tiles)
     using Iss = Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>;
     constexpr int kIssuers = Iss::kIssuers;              // threads issuing MMAs
@@ -577,7 +585,7 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
     constexpr int kRowsPerWarp = BM / 4;                 // output rows owned by one epilogue warp
     // TMEM buffers: bf16 double-buffers the accumulator; FP8 rings kNumAcc partial products
     // (one per K chunk, at least two groups' worth so the promotion overlaps the next group).
-    constexpr int kNumAcc = FP8 ? ((512 / BN) < 8 ? (512 / BN) : 8) : 2;
+    constexpr int kNumAcc = FP8 ? ((512 / BN) < 8 ? (512 / BN) : 8) : (2 * CH * BN <= 512 ? 2 : 1);
     constexpr int kAccCols = FP8 ? BN : CH * BN;         // columns of one buffer (bf16: CH chains)
     constexpr int kTmemColsNeeded = kNumAcc * kAccCols;
     constexpr uint32_t kTmemCols = kTmemColsNeeded <= 32    ? 32
@@ -611,7 +619,7 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
     uint64_t *accf_bar = consumed + kMaxSB;    // accumulator (or partial) full
     uint64_t *acce_bar = accf_bar + kNumAcc;   // accumulator (or partial) empty
     uint64_t *drain_bar = acce_bar + kNumAcc;  // one per MMA issuer
-    uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(drain_bar + 2);
+    uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(drain_bar + 4);   // up to 4 issuers
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
     int32_t *grp_prefix = reinterpret_cast<int32_t *>(tmem_base_smem + 4);   // [E+1]
     int32_t *grp_offs = grp_prefix + (GROUPED ? (kMaxExperts + 1) : 0);       // [E+1]
@@ -858,13 +866,14 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
                                nullptr);
             }
         }
-    } else if (warp == 1 || (kIssuers > 1 && warp == Iss::kSecondWarp)) {
+    } else if (warp == 1 || (kIssuers > 1 && warp >= Iss::kSecondWarp &&
+                             warp < Iss::kSecondWarp + kIssuers - 1)) {
         // ------------------------------------------------------------------ MMA issuers
-        // Issuer `iss` issues the MMAs of the K chunks of parity iss (FP8, two-chain bf16), each
-        // accumulator's instructions in ascending K.  Both issuers wait on the same barriers, and
+        // Issuer `iss` issues the MMAs of the K chunks c with c % kIssuers == iss, each
+        // accumulator's instructions in ascending K.  All issuers wait on the same barriers, and
         // each commits every group (the consumed and accumulator-full barriers count one commit
-        // per issuer), so a slot or an accumulator is handed on when both are done.
-        const int iss = warp == 1 ? 0 : 1;
+        // per issuer), so a slot or an accumulator is handed on when all are done.
+        const int iss = warp == 1 ? 0 : 1 + static_cast<int>(warp) - Iss::kSecondWarp;
         const int chunk_iss = Iss::kByChunk ? iss : 0;
         if (lane == 0) {
             const int SA = p.sa, SB = p.sb;
@@ -935,8 +944,8 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
                         uint32_t d = d_tmem;
                         if constexpr (FP8)   // chunk c of the group has partial buffer acc_iter + c
                             d = tmem_base + ((acc_iter + static_cast<uint32_t>(c)) % kNumAcc) * BN;
-                        else if constexpr (CH == 2)   // the chain of the chunk's parity
-                            d = d_tmem + static_cast<uint32_t>(chunk & 1) * BN;
+                        else if constexpr (CH > 1)   // the chain of the chunk: chunk % CH
+                            d = d_tmem + static_cast<uint32_t>(chunk % CH) * BN;
                         const uint64_t a_desc = a_slot + ((c * a_cp) >> 4);
                         const uint64_t b_desc = b_slot + ((c * R::kBChunkBytes) >> 4);
 #pragma unroll
@@ -959,8 +968,8 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
                     if (nc >= KC) {
                         if constexpr (Iss::kByChunk) {
 #pragma unroll
-                            for (int j = 0; j < KC / 2; ++j)
-                                issue_chunk(2 * j + chunk_iss, kg * KC + 2 * j + chunk_iss);
+                            for (int j = 0; j < KC / kIssuers; ++j)
+                                issue_chunk(kIssuers * j + chunk_iss, kg * KC + kIssuers * j + chunk_iss);
                         } else {
 #pragma unroll
                             for (int c = 0; c < KC; ++c)
@@ -968,7 +977,7 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
                         }
                     } else {
 #pragma unroll 1
-                        for (int c = chunk_iss; c < nc; c += (Iss::kByChunk ? 2 : 1))
+                        for (int c = chunk_iss; c < nc; c += kIssuers)
                             issue_chunk(c, kg * KC + c);
                     }
                     if constexpr (FP8)
@@ -1023,19 +1032,15 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
                 for (int c = 0; c < BN / 32; ++c) {
                     uint32_t r[32], r1[32];
                     const uint32_t col = tmem_base + lane_addr + a * kAccCols + c * 32;
+                    float v[32];
                     ptx::tmem_ld_32x32b_x32(col, r);
-                    if constexpr (CH == 2)
+                    if constexpr (CH >= 2)
                         ptx::tmem_ld_32x32b_x32(col + BN, r1);
                     ptx::tmem_wait_ld(r);
-                    if constexpr (CH == 2)
+                    if constexpr (CH >= 2)
                         ptx::tmem_wait_ld(r1);
-                    if (c == BN / 32 - 1) {
-                        ptx::tc_fence_before_sync();
-                        ptx::mbar_arrive(&acce_bar[a]);   // accumulator free for the next tile
-                    }
-                    float v[32];
-                    if constexpr (CH == 2) {
-                        // C = chain 0 + chain 1, once, in this order (one chunk: chain 0 alone)
+                    if constexpr (CH >= 2) {
+                        // chain 0 + chain 1 (one chunk in K: chain 0 alone)
                         const bool two = nkb > 1;
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj)
@@ -1045,6 +1050,25 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj)
                             v[jj] = __uint_as_float(r[jj]);
+                    }
+                    if constexpr (CH == 4) {
+                        // C = (chain 0 + chain 1) + (chain 2 + chain 3), in this order; the
+                        // chains that K leaves empty (fewer than four chunks) are left out
+                        if (nkb > 2) {
+                            ptx::tmem_ld_32x32b_x32(col + 2 * BN, r);
+                            ptx::tmem_ld_32x32b_x32(col + 3 * BN, r1);
+                            ptx::tmem_wait_ld(r);
+                            ptx::tmem_wait_ld(r1);
+                            const bool four = nkb > 3;
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj)
+                                v[jj] += four ? __uint_as_float(r[jj]) + __uint_as_float(r1[jj])
+                                              : __uint_as_float(r[jj]);
+                        }
+                    }
+                    if (c == BN / 32 - 1) {
+                        ptx::tc_fence_before_sync();
+                        ptx::mbar_arrive(&acce_bar[a]);   // accumulator free for the next tile
                     }
                     if (row_ok) {
                         if constexpr (SPLIT)

@@ -48,10 +48,10 @@ def test_plan_describe_is_m_free_and_sane():
                           (7168, 7168, 2, 1), (256, 512, 2, 1)]:
         info = bg.bi_gemm_plan_describe(bg.bi_gemm_plan(N, K, dt, E))
         assert info["n"] == N and info["k"] == K and info["num_experts"] == E
-        # dense bf16 plans of 32-column tiles reduce K in two interleaved chains (k_order_id 2) on
-        # the 64-row MMA; every other plan in one ascending chain
+        # dense bf16 plans of 32-column tiles reduce K in four interleaved chains (k_order_id 3)
+        # on the 64-row MMA; every other plan in one ascending chain
         narrow_bf16 = dt == 0 and E == 1 and info["block_n"] == 32
-        assert info["k_order_id"] == (2 if narrow_bf16 else 0) and info["block_m"] in (64, 128, 256)
+        assert info["k_order_id"] == (3 if narrow_bf16 else 0) and info["block_m"] in (64, 128, 256)
         assert info["block_m"] == 64 or not narrow_bf16
         assert info["mma_m"] == info["block_m"] and 2 <= info["stages_a"] <= info["stages"]
         assert info["cta_group"] == (2 if info["block_m"] == 256 else 1)
@@ -216,7 +216,7 @@ def test_host_batch_rejects_bad_arguments_before_any_device_call():
 
 
 def test_column_shard_plans_keep_the_full_plan():
-    """A shard of the decode plan keeps its tile and two-chain K order, where a plan made for the
+    """A shard of the decode plan keeps its tile and four-chain K order, where a plan made for the
     shard's own shape would not (2048 x 7168 is the prefill table entry: a CTA-pair tile with one
     chain), so its columns would differ from the full GEMM's in the last bits."""
     lib = binding.load_library()

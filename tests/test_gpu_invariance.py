@@ -103,16 +103,17 @@ def test_decode_rows_invariant_across_m_sweep():
 
 
 def test_scheduling_forms_of_one_plan_agree_bitwise():
-    # One 64x32 two-chain plan, ragged in N (the last 64-column lockstep pair is half outside N)
-    # and in K (113 chunks: an odd count, so chain 0 has one chunk more than chain 1, and the last
-    # group of every form is short).  M = 1 takes the tiny-batch form (16 chunks per stage), M = 20
-    # the small-batch form (8), M = 64 the plan's own form (4), M = 100 and 300 (258 and 645 tiles
-    # > 148 SMs) the wide lockstep form: a row's bits must not depend on which of them ran it.
+    # One 64x32 four-chain plan, ragged in N (the last 64-column lockstep pair is half outside N)
+    # and in K (113 chunks: chain 0 has 29 chunks and chains 1-3 have 28, and the last group of
+    # every form is short).  M = 1 takes the tiny-batch form (16 chunks per stage), M = 20 the
+    # small-batch form (8), M = 64 the plan's own form (4), M = 100 (258 tiles > 148 SMs) the
+    # two-tile and M = 300 (645 tiles) the four-tile lockstep form: a row's bits must not depend
+    # on which of them ran it.
     N, K = 4128, 7232
     B = inputs.bf16_gaussian((N, K), seed=2101, std=K ** -0.5, device=DEV)
     f = Dense(B)
     info = bg.bi_gemm_plan_describe(f.plan)
-    assert (info["block_m"], info["block_n"], info["k_order_id"]) == (64, 32, 2)
+    assert (info["block_m"], info["block_n"], info["k_order_id"]) == (64, 32, 3)
     test_rows = inputs.bf16_gaussian((24, K), seed=2102, device=DEV)
     ref = alone(f, test_rows)
     for M in [20, 64, 100, 300]:

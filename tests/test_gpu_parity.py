@@ -97,10 +97,32 @@ def test_ragged_integers_bit_exact(M, N, K):
     parity.assert_bits_equal_values(parity.bits(C), cbits, f"ragged integer {M}x{N}x{K}")
 
 
+@pytest.mark.parametrize("K", [64, 128, 192, 256, 320, 448, 136, 200])
+@pytest.mark.parametrize("M", [1, 8, 40])
+def test_four_chain_plans_with_few_chunks(M, K):
+    # The 32-column bf16 plans reduce K in four chains (chunk c to chain c % 4) and add them as
+    # (c0 + c1) + (c2 + c3); K of 1..7 chunks leaves chains empty or short, including ragged K
+    # (136, 200: the one-chunk-per-stage form).
+    N = 256
+    plan = bg.bi_gemm_plan(N, K)
+    assert bg.bi_gemm_plan_describe(plan)["k_order_id"] == 3
+    A = inputs.bf16_integers((M, K), seed=2300 + M + K)
+    B = inputs.bf16_integers((N, K), seed=2301 + K)
+    C, _ = run_dense(A.to(DEV), B.to(DEV))
+    _, cbits = oracle_bf16(A, B)
+    parity.assert_bits_equal_values(parity.bits(C), cbits, f"integers M={M} K={K}")
+    A = inputs.bf16_gaussian((M, K), seed=2310 + M + K)
+    B = inputs.bf16_gaussian((N, K), seed=2311 + K)
+    C, _ = run_dense(A.to(DEV), B.to(DEV))
+    cref, _ = oracle_bf16(A, B)
+    parity.assert_within_tolerance(parity.bits(C), cref, K, parity.rms(A.float().numpy()),
+                                   parity.rms(B.float().numpy()), f"gaussian M={M} K={K}")
+
+
 def test_wide_lockstep_form_ragged_integers_bit_exact():
-    # 64x32 two-chain plan at M = 300: 645 tiles > 148 SMs, so pairs of adjacent tiles run in
-    # lockstep on one A operand; N = 4128 leaves the last pair half outside N, K = 7232 (113
-    # chunks) gives the chains unequal lengths and a short last group.
+    # 64x32 four-chain plan at M = 300: 645 tiles > 148 SMs, so four adjacent tiles run in
+    # lockstep on one A operand; N = 4128 leaves the last group of tiles partly outside N,
+    # K = 7232 (113 chunks) gives the chains unequal lengths and a short last group.
     M, N, K = 300, 4128, 7232
     A = inputs.bf16_integers((M, K), seed=2201, device=DEV)
     B = inputs.bf16_integers((N, K), seed=2202, device=DEV)

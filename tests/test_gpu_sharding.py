@@ -1,7 +1,7 @@
 """Column-parallel sharding on one GPU: each column shard computed with a column-shard plan of the
 full plan, then placed side by side, must equal the full GEMM bit for bit (the shards run one
 after another here; on several GPUs each rank runs its own, and tests/test_dist_gloo.py checks the
-gather).  Covers the decode plan (two chains), a CTA-pair prefill plan and an FP8 plan."""
+gather).  Covers the decode plan (four chains), a CTA-pair prefill plan and an FP8 plan."""
 import pytest
 import torch
 
