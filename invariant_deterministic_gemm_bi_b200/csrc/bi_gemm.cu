@@ -70,10 +70,6 @@ struct KernelEntry {
     KernelEntry{bi::Issue<F8, BN, 2, false, KC>::kThreads, BM, BN, KC, F8, false, false,                           \
                 &bi::bi_gemm_kernel<BM, BN, KC, F8, false, 2>,                                     \
                 bi::smem_bytes_for<BM, BN, KC, F8, false, 2>(), 2, false, false, 1}
-#define BI_ENTRY_GROUPED_SPLIT2(BM, BN, KC)                                                        \
-    KernelEntry{bi::Issue<false, BN, 2, true, KC>::kThreads, BM, BN, KC, false, true, false,                      \
-                &bi::bi_gemm_kernel<BM, BN, KC, false, true, 2>,                                   \
-                bi::smem_bytes_for<BM, BN, KC, false, true, 2>(), 2, false, false, 1}
 #define BI_PAIR(BN, KC, F8, GR)                                                                    \
     KernelEntry{bi::Epi<F8, BN>::kThreads, 256, BN, KC, F8, GR, true,                              \
                 &bi::bi_gemm_kernel_pair<BN, KC, F8, GR>,                                          \
@@ -110,7 +106,8 @@ const KernelEntry kKernels[] = {
     BI_ENTRY(128, 32, 1, false, true),  BI_ENTRY(128, 32, 4, false, true),
     BI_ENTRY(128, 64, 1, false, true),  BI_ENTRY(128, 64, 2, false, true),
     BI_ENTRY(128, 128, 1, false, true), BI_ENTRY(128, 128, 2, false, true),
-    BI_ENTRY_GROUPED_SPLIT2(128, 256, 1),
+    // grouped wide form: 2 x 2 tiles of the 128 x 128 MoE plan on a CTA pair
+    BI_PAIR(256, 1, false, true),
     BI_PAIR(128, 1, false, false),      BI_PAIR(128, 2, false, false),
     BI_PAIR(256, 1, false, false),      BI_PAIR(256, 2, false, false),
     BI_PAIR(128, 1, true, false),       BI_PAIR(128, 2, true, false),
@@ -353,13 +350,14 @@ struct bi_plan_s {
     // (dense plans only; may be null).  It issues the same MMAs in the same K order, so a row's
     // result does not depend on which of the two a launch takes.
     const KernelEntry *kernel_small = nullptr;
-    // The bf16 small-batch tile with twice its chunks again (16 per group), for launches whose A
-    // boxes hold at most 8 rows (dense bf16 128 x 32 plans only; may be null).  Same MMAs, same
-    // K order.
+    // The bf16 small-batch tile with twice its chunks again (16 per group), for launches of
+    // fewer than 8 rows (dense bf16 64 x 32 plans only; may be null).  Same MMAs, same K order.
     const KernelEntry *kernel_tiny = nullptr;
-    // Two adjacent tiles in lockstep on one A operand (the same MMA instructions in the same K
-    // order), for dense launches with more tiles than SMs and grouped launches with at least a
-    // tile's worth of rows per expert on average.  May be null.
+    // Dense: two adjacent tiles in lockstep on one A operand, for launches with more tiles than
+    // SMs.  Grouped: 2 x 2 tiles of the plan on a CTA pair (one 256 x 256 cta_group::2
+    // instruction per K step), for launches with at least a tile's worth of rows per expert on
+    // average.  Either way one instruction covers the tiles, in the plan's K order, and gives
+    // every element the plan's bits.  May be null.
     const KernelEntry *kernel_wide = nullptr;
     // Four adjacent tiles in lockstep (bf16 plans with K chains), for dense launches whose lockstep pairs
     // still outnumber the SMs.  May be null.
@@ -821,7 +819,7 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     p->small_rows = chains > 1 ? 32 : 64;
     if (num_experts > 1 && !k->pair && k->bm == 128 && k->bn == 128) {
         for (int i = 0; i < kNumKernels; ++i)
-            if (kKernels[i].nsplit == 2 && kKernels[i].grouped && kKernels[i].bn == 256)
+            if (kKernels[i].pair && kKernels[i].grouped && kKernels[i].bn == 256)
                 p->kernel_wide = &kKernels[i];
     }
     if (num_experts == 1 && !k->pair && (k->bm == 128 || k->chains > 1) &&
@@ -1033,8 +1031,8 @@ bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *
     int *status = nullptr;
     if ((st = plan_status_word(plan, dev, &status)) != BI_OK)
         return st;
-    // With at least a tile's worth of rows per expert on average, adjacent column tiles run in
-    // lockstep on one A operand (the wide form: same MMA instructions, same K order).
+    // With at least a tile's worth of rows per expert on average, 2 x 2 plan tiles run on a CTA
+    // pair (the wide form: one wider instruction, same K order, same bits).
     const KernelEntry *k = plan->kernel;
     if (plan->kernel_wide && total_rows >= static_cast<int64_t>(plan->kernel->bm) * plan->experts)
         k = plan->kernel_wide;

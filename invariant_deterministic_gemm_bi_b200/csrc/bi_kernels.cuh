@@ -82,8 +82,8 @@ struct Epi {
 //     chunk % CH == c into an accumulator of its own, and the epilogue adds the chains once.  As
 //     many issuers as chains when a group's chunk count allows it (kIssuers divides both CH and
 //     KC), so each chain belongs to one issuer.
-// Grouped kernels keep one issuer: their instructions are wide enough (128 x 128 or 128 x 256)
-// for one thread to keep the tensor pipe fed.  The extra issuers are the warps after the epilogue
+// Grouped kernels keep one issuer: their 128 x 128 instructions are wide enough for one thread
+// to keep the tensor pipe fed.  The extra issuers are the warps after the epilogue
 // warps.
 template <bool FP8, int BN, int NSPLIT, bool GROUPED = false, int KC = 1, int CH = 1>
 struct Issue {
@@ -565,11 +565,10 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
     static_assert(!FP8 || BN <= 128, "FP8 keeps BN fp32 accumulators per thread: BN <= 128");
     static_assert(!(FP8 && GROUPED), "grouped FP8 is not built");
     static_assert(KC >= 1 && KC <= 16, "1..16 chunks per group");
-    static_assert(NSPLIT == 1 ||
-                      (NSPLIT == 2 && (GROUPED ? (!FP8 && BN == 256) : BN == (FP8 ? 128 : 64))) ||
+    static_assert(NSPLIT == 1 || (NSPLIT == 2 && !GROUPED && BN == (FP8 ? 128 : 64)) ||
                       (NSPLIT == 4 && CH >= 2 && BN == 128),
-                  "lockstep tiles: dense bf16 64-wide, FP8 128-wide and grouped bf16 256-wide "
-                  "tiles hold two plan tiles; bf16 128-wide tiles with K chains hold four");
+                  "lockstep tiles: dense bf16 64-wide and FP8 128-wide tiles hold two plan "
+                  "tiles; bf16 128-wide tiles with K chains hold four");
     static_assert(!SPLIT || (!FP8 && !GROUPED && NSPLIT == 1), "split-K variant: bf16 dense");
     static_assert(!W4 || (FP8 && !GROUPED && !SPLIT), "e2m1 weights: the dense FP8 kernel");
     static_assert(CH == 1 || ((CH == 2 || CH == 4) && !FP8 && !GROUPED && !SPLIT),

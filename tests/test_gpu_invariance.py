@@ -124,23 +124,25 @@ def test_scheduling_forms_of_one_plan_agree_bitwise():
                        positions=sorted({q for q in (0, 63, 64, 127, 128, M - 1) if q < M}))
 
 
-def adversarial_bf16(shape, kind, seed):
+def adversarial_bf16(shape, kind, seed, device="cpu"):
     """bf16 operands built to expose any difference in how an instruction sums its K products:
     exponents spread over 2^-24..2^24 ("wide"), pairs that cancel to a few ulps ("cancel"), or a
-    small background under 1 % large spikes ("spikes")."""
-    g = torch.Generator().manual_seed(seed)
+    small background under 1 % large spikes ("spikes").  Drawn on `device`, returned on the GPU."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    kw = dict(generator=g, device=device)
     if kind == "spikes":
-        x = torch.randn(shape, generator=g) * 2.0 ** -10
-        mask = torch.rand(shape, generator=g) < 0.01
-        x[mask] = torch.randn(int(mask.sum()), generator=g) * 2.0 ** 10
+        x = torch.randn(shape, **kw) * 2.0 ** -10
+        mask = torch.rand(shape, **kw) < 0.01
+        x = torch.where(mask, torch.randn(shape, **kw) * 2.0 ** 10, x)
         return x.to(torch.bfloat16).to(DEV)
-    e = torch.randint(-24, 25, shape, generator=g).float()
-    sign = torch.randint(0, 2, shape, generator=g).float() * 2 - 1
-    x = sign * (1 + torch.rand(shape, generator=g)) * torch.exp2(e)
+    e = torch.randint(-24, 25, shape, **kw).float()
+    sign = torch.randint(0, 2, shape, **kw).float() * 2 - 1
+    x = sign * (1 + torch.rand(shape, **kw)) * torch.exp2(e)
+    del e, sign
     if kind == "cancel":
         odd = x[..., 1::2]
         x[..., 1::2] = -x[..., 0::2][..., : odd.shape[-1]] * (
-            1 + 2.0 ** -7 * torch.randint(-2, 3, odd.shape, generator=g).float())
+            1 + 2.0 ** -7 * torch.randint(-2, 3, odd.shape, **kw).float())
     return x.to(torch.bfloat16).to(DEV)
 
 
@@ -321,16 +323,19 @@ def test_moe_adversarial_routings(pattern):
 
 @pytest.mark.parametrize("kind", ["cancel", "spikes"])
 def test_moe_wide_form_agrees_bitwise_on_adversarial_inputs(kind):
-    # 1200 rows over 8 experts (>= 128 per expert on average) take the grouped wide form, one
-    # 128 x 256 instruction per K step; a row alone takes the plan's 128 x 128 form.
-    E, N, K = 8, 2048, 7168
+    # 8448 rows over the 64 experts (>= 128 per expert on average) take the grouped wide form:
+    # 2 x 2 tiles of the 128 x 128 plan on a CTA pair, one 256 x 256 cta_group::2 instruction
+    # per K step.  A row alone takes the plan's own 128 x 128 form.
+    E, N, K, R = 64, 2048, 7168, 8448
     plan = bg.bi_gemm_plan(N, K, bg.BI_DTYPE_BF16, E)
-    B = adversarial_bf16((E, N, K), kind, 5201)
-    tokens = adversarial_bf16((1200, K), kind, 5202)
-    experts = np.sort(np.random.default_rng(5203).integers(0, E, 1200))
+    info = bg.bi_gemm_plan_describe(plan)
+    assert (info["block_m"], info["block_n"]) == (128, 128)
+    B = adversarial_bf16((E, N, K), kind, 5201, device=DEV)
+    tokens = adversarial_bf16((R, K), kind, 5202, device=DEV)
+    experts = np.sort(np.random.default_rng(5203).integers(0, E, R))
     r = routing_mod.routing_from_assignment(experts, E)
     C = moe_outputs(plan, B, tokens, r)
-    for i in np.random.default_rng(5204).choice(1200, 24, replace=False):
+    for i in np.random.default_rng(5204).choice(R, 24, replace=False):
         e = int(experts[i])
         one = routing_mod.routing_from_assignment(np.array([e]), E)
         C1 = moe_outputs(plan, B, tokens[i:i + 1], one)
