@@ -573,7 +573,7 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
     ordered by its own events over 27 staging slots (three steps): a step's copy-ins run under the
     previous step's kernels and its copy-outs under the kernels two steps later.  The host buffers are pinned on the GPU's NUMA node when it is known.  The record
     also holds the pinned copy bandwidth measured in this run (one 256 MiB cudaMemcpyAsync each
-    way), the bound the copies cannot beat."""
+    way, then both at once on two streams), the bound the copies cannot beat."""
     import torch
     from invariant_deterministic_gemm_bi_b200 import inputs
     steps = max(2, min(args.steps, 400))
@@ -608,7 +608,29 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
         return probe_h.numel() / best / 1e9
     h2d_gbs = copy_gbs(probe_d, probe_h)
     d2h_gbs = copy_gbs(probe_h, probe_d)
-    del probe_d, probe_h
+    # both directions at once, on two streams: whether the link carries them in parallel
+    probe_d2 = torch.empty_like(probe_d)
+    probe_h2 = torch.empty_like(probe_h).pin_memory()
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    both = None
+    for _ in range(3):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        with torch.cuda.stream(s_in):
+            probe_d.copy_(probe_h, non_blocking=True)
+        with torch.cuda.stream(s_out):
+            probe_h2.copy_(probe_d2, non_blocking=True)
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
+        e1.record(stream)
+        e1.synchronize()
+        t = e0.elapsed_time(e1) * 1e-3
+        both = t if both is None else min(both, t)
+    duplex_gbs = 2 * probe_h.numel() / both / 1e9
+    del probe_d, probe_h, probe_d2, probe_h2
 
     n_copies = len(Bs)
     arrays = [bg.host_gemm_array([(A_host[:m], Bs[(ph * len(M_SWEEP) + i) % n_copies], C_host[m])
@@ -677,8 +699,9 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
                      "later) on a copy-out stream, ordered by the library's events over 27 staging "
                      "slots; %d steps and a flush per captured CUDA graph, replayed back to back"
                      % per_graph),
-            "copy_floor_ms_per_step": max(h2d / h2d_gbs, d2h / d2h_gbs) / 1e6,
+            "copy_floor_ms_per_step": max(h2d / h2d_gbs, d2h / d2h_gbs, (h2d + d2h) / duplex_gbs) / 1e6,
             "pinned_h2d_gbs": h2d_gbs, "pinned_d2h_gbs": d2h_gbs,
+            "pinned_both_directions_gbs": duplex_gbs,
             "gpu_numa_node": node, "host_buffers_on_gpu_node": affinity is not None,
             "results_match_device_run": check_ok}
 
@@ -724,11 +747,18 @@ def measure_per_m(bg, plan, As, Bs, Cs, dev, stream, n_copies, peaks):
 def measure_extras(bg, inputs, dev, stream, peaks):
     """The other workloads (small, prefill, FP8, W4A8, MoE and its layer steps, attention, the
     split-K variant): throughput and roofline fraction (not part of `value`)."""
+    import time
     import torch
     res = {}
     bf16_peak = peaks["bf16_tflops"]
     fp8_peak = 2.0 * bf16_peak          # nominal dense fp8 : bf16 ratio
     hbm = peaks["hbm_gbs"]
+
+    def settle():
+        # a pause between workloads, so that one does not start under the power and clock state a
+        # kilowatt-class predecessor (the prefill GEMMs) left behind
+        torch.cuda.synchronize()
+        time.sleep(1.0)
     # the small correctness shape N = 256, K = 512 (its 256 KB of weights stay in L2, so this is
     # launch latency, not HBM): per launch inside a graph
     plan = weight_plan(256, 512)
@@ -742,6 +772,7 @@ def measure_extras(bg, inputs, dev, stream, peaks):
         res[f"small_N256_K512_M{M}"] = {"us": t * 1e6, "GB/s": b / t / 1e9,
                                         "TFLOP/s": 2 * M * 256 * 512 / t / 1e12}
         del A, C
+    settle()
     # prefill, M = 16384 and 4096
     for (N, K) in [(7168, 2048), (2048, 7168)]:
         plan = weight_plan(N, K)
@@ -755,6 +786,7 @@ def measure_extras(bg, inputs, dev, stream, peaks):
             res[f"prefill_N{N}_K{K}_M{M}"] = {"us": t * 1e6, "TFLOP/s": tf,
                                               "tensor_frac": tf / bf16_peak}
             del A, C
+    settle()
     # FP8 N = K = 7168
     N = K = 7168
     KB = K // 128
@@ -773,6 +805,7 @@ def measure_extras(bg, inputs, dev, stream, peaks):
         res[f"fp8_M{M}"] = {"us": t * 1e6, "TFLOP/s": tf, "tensor_frac": tf / fp8_peak,
                             "GB/s": b / t / 1e9, "hbm_frac": b / t / 1e9 / hbm}
     del qbs
+    settle()
     # e2m1 weights (per-channel 2^-j scale and fp16 zero point) x e4m3 activations, N = K = 7168;
     # 8 weight copies (205 MB) rotate so that every launch reads W from HBM
     plan = weight_plan(N, K, bg.BI_DTYPE_E2M1_W4A8)
@@ -807,6 +840,7 @@ def measure_extras(bg, inputs, dev, stream, peaks):
     b = N * K * 2 + N * K // 2 + 8 * N
     res["quantize_e2m1_7168x7168"] = {"us": t * 1e6, "GB/s": b / t / 1e9, "hbm_frac": b / t / 1e9 / hbm}
     del Wb, Qw
+    settle()
     # MoE: 64 experts, N = 2048, K = 7168, top-8
     E, N, K = 64, 2048, 7168
     plan = weight_plan(N, K, bg.BI_DTYPE_BF16, E)
@@ -853,6 +887,7 @@ def measure_extras(bg, inputs, dev, stream, peaks):
             res[f"moe_layer_T{T}_{name}"] = {"us": t * 1e6, "GB/s": b / t / 1e9,
                                              "hbm_frac": b / t / 1e9 / hbm}
         del A, Cp, Y, toks
+    settle()
     # Dual-kernel decode attention: Hq = 32, Hkv = 8, D = 128, bf16 KV cache, every sequence at
     # length L; no split vs split-KV (bitwise equal outputs).  Bytes: K and V once, Q and O.
     import math
@@ -878,6 +913,7 @@ def measure_extras(bg, inputs, dev, stream, peaks):
         res[f"attention_B{Bsz}_L{L}_splits{splits}"]["bitwise_equal_to_no_split"] = all(
             torch.equal(outs[1].view(torch.int16), o.view(torch.int16)) for o in outs.values())
         del Q, Kc, Vc, O, ws
+    settle()
     # Fixed-split-K research variant on the decode shape (not the product path): what dropping
     # split-K costs at small M.  Bytes are the algorithmic ones (workspace traffic not counted).
     N, K = N_DEC, K_DEC

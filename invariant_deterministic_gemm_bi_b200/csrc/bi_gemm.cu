@@ -153,7 +153,7 @@ RingGeom ring_geometry(const KernelEntry *k, int a_rows)
         return RingGeom{st, st, static_cast<uint32_t>(a_bytes), static_cast<uint32_t>(st * a_bytes)};
     }
     const int ring = k->grouped ? bi::kRingBytesGrouped : bi::kRingBytes1;
-    const int a_stride = k->kc * a_rows * chunk;
+    const int a_stride = (k->kc * a_rows * chunk + 1023) / 1024 * 1024;   // slots start on swizzle atoms
     // The MMA reads BM rows from every A chunk: past the last loaded row of the last A slot it
     // reads on into the B ring, which lies right after the A region and must reach that far.
     const int over = (k->bm - a_rows) * chunk;
@@ -624,20 +624,6 @@ GemmParams base_params(const bi_plan_s *plan, const KernelEntry *k, int64_t rows
     return p;
 }
 
-// Dense problems of fewer than 8 rows on one-CTA tiles: a 2-D map of A with boxes of exactly M
-// rows, for the kernel's per-chunk A loads (bi::GemmParams::a_exact_rows), so that no A load
-// reaches past the last row (TMA fills such rows slowly).  Leaves *map alone otherwise.
-bi_status_t exact_rows_map(const KernelEntry *k, CUtensorMap *map, const void *A, bool fp8, int64_t K,
-                           int64_t M, int64_t lda, GemmParams *p)
-{
-    if (k->pair || k->grouped || M >= 8)
-        return BI_OK;
-    const bi_status_t st = encode_operand(map, A, fp8, K, M, lda, static_cast<int>(M), 1);
-    if (st == BI_OK)
-        p->a_exact_rows = static_cast<int32_t>(M);
-    return st;
-}
-
 // Launch kernel entry k.  `units` is the number of work tiles; a one-CTA kernel gets
 // min(units, #SMs) CTAs, a pair kernel min(units, co-resident pairs) clusters of two CTAs.  Every
 // launch is a programmatic dependent of the previous kernel in the stream: it may start (and set
@@ -676,11 +662,15 @@ bi_status_t launch_main(const KernelEntry *k, const DeviceInfo *d, const CUtenso
     return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
-// Rows of A one TMA box covers and rows of B one box covers, for this plan and M.  A pair CTA
-// owns 128 rows of a tile; a dense problem smaller than that boxes only its roundup(M, 8) rows.
+// Rows of A one TMA box covers and rows of B one box covers, for this plan and M.  One-CTA
+// kernels load exactly the problem's rows when it has fewer than a tile's (see
+// bi::GemmParams::a_box_rows).  A pair CTA owns 128 rows of a tile; a dense problem smaller than
+// that boxes its roundup(M, 8) rows.
 int a_box_rows_for(const KernelEntry *k, int64_t M)
 {
-    return dense_a_box_rows(M, k->pair ? 128 : k->bm);
+    if (k->pair)
+        return dense_a_box_rows(M, 128);
+    return M >= k->bm ? k->bm : static_cast<int>(M);
 }
 
 int b_box_rows_for(const KernelEntry *k)
@@ -692,8 +682,8 @@ int b_box_rows_for(const KernelEntry *k)
 // small-batch kernel form (when it has one): with few A rows, groups of twice the chunks halve
 // the per-group wait and commit overhead of the MMA threads, and the ring still holds two groups
 // of A and of B (and, for FP8, more groups than partial-product buffers).  At most this many
-// rows take the tiny-batch form (16 chunks per group), whose per-chunk A loads of exactly M rows
-// (bi::GemmParams::a_exact_rows) cost 16 TMA issues per group: it pays below 8 rows only.
+// rows take the tiny-batch form (16 chunks per group): its 16 KB groups of A rows cost little
+// shared memory only while the batch stays below 8 rows.
 constexpr int kTinyBatchRows = 7;
 
 // A dense launch with more tiles than the device has SMs takes the plan's wide form (when it has
@@ -1000,11 +990,8 @@ bi_status_t bi_gemm_run(bi_plan_t plan, int64_t M, const void *A, int64_t lda, c
     p.scale_a = scale_a;
     p.ld_sa = ld_sa;
     p.scale_b = scale_b;
-    CUtensorMap ta_exact = ta;
-    if ((st = exact_rows_map(k, &ta_exact, A, fp8, plan->k, M, lda, &p)) != BI_OK)
-        return st;
     const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-    return launch_main(k, d, ta, tb, ta_exact, p, tiles, stream);
+    return launch_main(k, d, ta, tb, ta, p, tiles, stream);
 }
 
 bi_status_t bi_grouped_gemm_run(bi_plan_t plan, int64_t total_rows, const void *A, int64_t lda,
@@ -1443,11 +1430,8 @@ bi_status_t bi_gemm_run_host_noalloc(bi_plan_t plan, int64_t M, const void *A_ho
         p.scale_a = fp8 ? sa_dev : nullptr;
         p.ld_sa = fp8 ? ld_sa : 0;
         p.scale_b = fp8 ? scale_b : nullptr;
-        CUtensorMap ta_exact = ta;
-        if ((st = exact_rows_map(k, &ta_exact, A_dev, fp8, plan->k, M, lda, &p)) != BI_OK)
-            return st;
         const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-        if ((st = launch_main(k, d, ta, tb, ta_exact, p, tiles, stream)) != BI_OK)
+        if ((st = launch_main(k, d, ta, tb, ta, p, tiles, stream)) != BI_OK)
             return st;
     }
     if (cudaMemcpyAsync(C_host, C_dev, static_cast<size_t>(M * ldc * 2), cudaMemcpyDeviceToHost,
@@ -1547,11 +1531,8 @@ bi_status_t bi_gemm_run_w4a8(bi_plan_t plan, int64_t M, const void *A, int64_t l
                                workspace) != cudaSuccess)
             return BI_ERR_CUDA;
     }
-    CUtensorMap ta_exact = ta;
-    if ((st = exact_rows_map(k, &ta_exact, A, true, plan->k, M, lda, &p)) != BI_OK)
-        return st;
     const int64_t tiles = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks;
-    return launch_main(k, d, ta, tb, ta_exact, p, tiles, stream);
+    return launch_main(k, d, ta, tb, ta, p, tiles, stream);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -1644,11 +1625,8 @@ bi_status_t bi_gemm_run_splitk(bi_plan_t plan, int64_t M, const void *A, int64_t
     p.ws = static_cast<float *>(workspace);
     p.ld_ws = (plan->n + 3) / 4 * 4;
     p.ws_split_stride = M * p.ld_ws;
-    CUtensorMap ta_exact = ta;
-    if ((st = exact_rows_map(k, &ta_exact, A, false, plan->k, M, lda, &p)) != BI_OK)
-        return st;
     const int64_t units = static_cast<int64_t>(p.num_m_blocks) * p.num_n_blocks * plan->k_splits;
-    if ((st = launch_main(k, d, ta, tb, ta_exact, p, units, stream)) != BI_OK)
+    if ((st = launch_main(k, d, ta, tb, ta, p, units, stream)) != BI_OK)
         return st;
     const int64_t total = M * plan->n;
     const int64_t blocks = (total + 255) / 256;

@@ -9,10 +9,10 @@
 // K-slices of the tile in ascending order into one TMEM accumulator (no split-K, no atomics,
 // no cross-CTA reduction).  The tile shape, the MMA instruction shape and the K order are
 // template constants chosen by the host plan from (N, K, dtype) only.  Rows past the end of A
-// are zero-filled by TMA and never stored.  When the whole problem has fewer than 128 rows,
-// TMA brings only the first roundup(M, 8) rows of the A tile; the MMA still runs on all 128
-// rows, and the rows never loaded feed only output rows that are never stored (every output
-// element depends on its own A row alone).  The CTA <-> tile mapping does depend on M, which is
+// are zero-filled by TMA and never stored.  When the whole problem has fewer rows than a tile,
+// TMA brings only those rows of the A tile; the MMA still runs on all BM rows, and the rows never
+// loaded feed only output rows that are never stored (every output element depends on its own A
+// row alone).  The CTA <-> tile mapping does depend on M, which is
 // harmless: it decides where a tile is computed, not how.
 //
 // Roles inside a CTA (6 warps = 192 threads):
@@ -111,13 +111,15 @@ struct GemmParams {
     int32_t num_m_blocks;    // dense: ceil(M / BM)
     int32_t num_experts;     // grouped: E
     int32_t raster_m;        // dense raster band height in m-blocks
-    int32_t a_box_rows;      // rows of A one TMA load brings (<= BM, a multiple of 8)
-    int32_t a_exact_rows;    // dense problems of fewer than 8 rows: each K chunk of an A group
-                             // is loaded as its own 2-D box of exactly this many rows (the third
-                             // tensor map) into its 1024-byte chunk slot, so no load reaches past
-                             // the end of A (TMA fills such rows slowly); 0 otherwise
+    int32_t a_box_rows;      // rows of A one TMA load brings: BM, or, when the whole dense problem
+                             // has fewer rows, exactly its rows (no load reaches past the end of
+                             // A; TMA fills such rows slowly).  Chunk c of an A slot then starts
+                             // c * a_box_rows * 128 bytes in, inside a 1024-byte swizzle atom when
+                             // a_box_rows is not a multiple of 8: tcgen05 applies the 128-byte
+                             // swizzle to the absolute shared-memory address, as TMA does when it
+                             // writes the box, so the descriptors need no base offset.
     int32_t sa, sb;          // ring depths in groups (2..kMaxSA, sa..kMaxSB)
-    uint32_t a_stride;       // bytes between A slots (KC * a_box_rows * 128)
+    uint32_t a_stride;       // bytes between A slots (KC * a_box_rows * 128, rounded up to 1024)
     uint32_t b_offset;       // byte offset of the B ring in the ring region
     int32_t pair_a1;         // CTA pair: 1 if the peer CTA loads A rows (the problem has > 128)
     int32_t prefetch_b;      // dense, resident weights: request the first B groups before the
@@ -641,7 +643,7 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
         ptx::fence_mbarrier_init();
         ptx::prefetch_tmap(&tmap_a);
         ptx::prefetch_tmap(&tmap_b);
-        if (GROUPED || p.a_exact_rows > 0)
+        if (GROUPED)
             ptx::prefetch_tmap(&tmap_a8);
     }
     if (warp == 1) {
@@ -813,18 +815,7 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
                     int nsub = 0;
                     if constexpr (GROUPED)
                         nsub = short_segment_boxes(ca.tc, kShortSegmentRows);
-                    if (!GROUPED && p.a_exact_rows > 0) {
-                        // fewer than 8 rows: one exact-height box per chunk that exists in K;
-                        // the chunk slot's rows past them keep stale data, which feeds only
-                        // output rows that are never stored
-                        const int first = ca.tc.kb0 + ca.kg * KC;
-                        const int left = ca.tc.kb0 + ca.tc.nkb - first;
-                        const int nc = left < KC ? left : KC;
-                        ptx::mbar_arrive_expect_tx(&full[fs], static_cast<uint32_t>(nc * p.a_exact_rows) * kRowBytes);
-                        for (int c = 0; c < nc; ++c)
-                            ptx::tma_load_2d(smem_a + as * p.a_stride + c * a_chunk_pitch, &tmap_a8, &full[fs],
-                                             (first + c) * kElemsPerRow, ca.tc.m0, pol);
-                    } else if (nsub == 0) {
+                    if (nsub == 0) {
                         ptx::mbar_arrive_expect_tx(&full[fs], KC * a_chunk_pitch);
                         load(smem_a + as * p.a_stride, &tmap_a, &full[fs], ca.tc.kb0, ca.kg, ca.tc.m0);
                     } else {
@@ -879,7 +870,8 @@ __global__ void __launch_bounds__(Issue<FP8, BN, NSPLIT, GROUPED, KC, CH>::kThre
             int sa = 0, sb = 0;      // ring slots of the next group
             uint32_t pb = 0;         // phase of full[sb] / consumed[sb]
             // Shared-memory descriptors are linear in the address (start address >> 4 in the low
-            // bits), so every slot / chunk / K-step descriptor is a base plus an offset.
+            // bits), so every slot / chunk / K-step descriptor is a base plus an offset (a chunk
+            // of fewer than 8 rows' pitch starts inside a swizzle atom: see a_box_rows).
             const uint64_t a_desc0 = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_a));
             const uint64_t b_desc0 = ptx::sw128_kmajor_desc(ptx::smem_u32(smem_b));
             // A of a short grouped segment: 8-row groups KC * 1024 bytes apart, chunks 1024 apart

@@ -224,6 +224,30 @@ def test_fp8_pow2_scales_integers_bit_exact(M, N, K):
     parity.assert_bits_equal_values(parity.bits(C), cbits, f"fp8 integer {M}x{N}x{K}")
 
 
+# A problem with fewer rows than a tile loads exactly its rows: chunk c of an A slot then starts
+# c * M * 128 bytes in, inside a 1024-byte swizzle atom whenever M is not a multiple of 8.
+EXACT_HEIGHT_M = [1, 2, 3, 5, 6, 7, 9, 15, 17, 23, 33, 63]
+
+
+@pytest.mark.parametrize("M", EXACT_HEIGHT_M)
+def test_exact_height_a_rows_bf16_bit_exact(M):
+    N, K = 512, 2048      # the 64 x 32 plan: every form below 64 rows
+    A = inputs.bf16_integers((M, K), seed=2400 + M)
+    B = inputs.bf16_integers((N, K), seed=2401)
+    C, _ = run_dense(A.to(DEV), B.to(DEV))
+    _, cbits = oracle_bf16(A, B)
+    parity.assert_bits_equal_values(parity.bits(C), cbits, f"bf16 integers M={M}")
+
+
+@pytest.mark.parametrize("M", EXACT_HEIGHT_M + [100, 127])
+def test_exact_height_a_rows_fp8_bit_exact(M):
+    qa, qb, sa, sb = fp8_case(M, 256, 1024, seed=4300 + M, integer=True)
+    C = run_fp8(qa, qb, sa, sb)
+    _, cbits = oracle.gemm_fp8_blockscaled(inputs.to_numpy_bits(qa), inputs.to_numpy_bits(qb),
+                                           sa.numpy(), sb.numpy())
+    parity.assert_bits_equal_values(parity.bits(C), cbits, f"fp8 integer M={M}")
+
+
 @pytest.mark.parametrize("M", [1, 64, 4096])
 def test_fp8_full_size_sampled_rows(M):
     N = K = 7168

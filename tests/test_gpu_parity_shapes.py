@@ -8,7 +8,7 @@ invariance with a bitwise equality).  These cases run every scheduling form of t
 real shapes:
 
 * decode 4096 x 7168 at every M of the sweep: the tiny-batch (M <= 8), small-batch (<= 32),
-  plan (64) and wide lockstep forms (128, 256), with the exact-height A loads below 8 rows;
+  plan (64) and wide lockstep forms (128, 256), with A boxes of exactly M rows below a tile;
 * prefill 7168 x 2048 and 2048 x 7168 at M = 1024 and 4096 (CTA-pair tiles, several waves);
 * grouped 64 x 2048 x 7168 at T = 64 and 1024 tokens routed top-8 by a seeded softmax (the
   routing comes from the oracle's MoE steps), every row.
