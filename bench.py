@@ -568,12 +568,16 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
     """The same sweep end to end through the library's host-buffer call.
 
     Each step is one bi_gemm_run_host_batch call with the sweep's nine GEMMs: pinned host A
-    slices in, the kernels, pinned host C results out.  The library runs the copy-ins on a
-    copy-in stream, the kernels on the compute stream and the copy-outs on a copy-out stream,
-    ordered by its own events over 27 staging slots (three steps): a step's copy-ins run under the
-    previous step's kernels and its copy-outs under the kernels two steps later.  The host buffers are pinned on the GPU's NUMA node when it is known.  The record
+    slices in, the kernels, pinned host C results out.  The slices of a step lie back to back in
+    one pinned block for A and one for C, so the library moves each with one copy.  It runs the
+    copy-ins on a copy-in stream, the kernels on the compute stream and the copy-outs on a
+    copy-out stream, ordered by its own events over 3 staging regions (one per step in flight):
+    a step's copy-in runs under the previous step's kernels and its copy-out under the kernels
+    two steps later.  The host buffers are pinned on the GPU's NUMA node when it is known.  The
+    record
     also holds the pinned copy bandwidth measured in this run (one 256 MiB cudaMemcpyAsync each
-    way, then both at once on two streams), the bound the copies cannot beat."""
+    way, then both at once on two streams) and the time of the step's own copy-in and copy-out
+    run alone at once (copy_floor_ms_per_step), the bound the end-to-end step cannot beat."""
     import torch
     from invariant_deterministic_gemm_bi_b200 import inputs
     steps = max(2, min(args.steps, 400))
@@ -585,9 +589,17 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
         if local:
             affinity = here
             os.sched_setaffinity(0, local)   # pinned pages are placed on the allocating CPU's node
+    rows = sum(M_SWEEP)
+    offs = {}
+    o = 0
+    for m in M_SWEEP:
+        offs[m] = o
+        o += m
     try:
-        A_host = inputs.bf16_gaussian((max(M_SWEEP), K_DEC), seed=77).pin_memory()
-        C_host = {m: torch.empty((m, N_DEC), dtype=torch.bfloat16).pin_memory() for m in M_SWEEP}
+        # one step's activations and results, each laid out back to back in one pinned block (as
+        # a serving loop's activation arena would be): the library moves each with one copy
+        A_block = inputs.bf16_gaussian((rows, K_DEC), seed=77).pin_memory()
+        C_block = torch.empty((rows, N_DEC), dtype=torch.bfloat16).pin_memory()
         probe_h = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
     finally:
         if affinity is not None:
@@ -632,12 +644,38 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
     duplex_gbs = 2 * probe_h.numel() / both / 1e9
     del probe_d, probe_h, probe_d2, probe_h2
 
+    # the step's own copies alone (its activations in, its results out, on two streams at once):
+    # the bound the end-to-end step cannot beat
+    a_dev = torch.empty_like(A_block, device=dev)
+    c_dev = torch.empty_like(C_block, device=dev)
+    copies = None
+    for _ in range(5):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        with torch.cuda.stream(s_in):
+            a_dev.copy_(A_block, non_blocking=True)
+        with torch.cuda.stream(s_out):
+            C_block.copy_(c_dev, non_blocking=True)
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
+        e1.record(stream)
+        e1.synchronize()
+        t = e0.elapsed_time(e1)
+        copies = t if copies is None else min(copies, t)
+    del a_dev, c_dev
+
+    # each block is one allocation: the library may move a step's slices with one copy each way
+    bg.bi_gemm_plan_set_flags(plan, bg.BI_PLAN_RESIDENT_WEIGHTS | bg.BI_PLAN_HOST_ROW_BLOCKS)
     n_copies = len(Bs)
-    arrays = [bg.host_gemm_array([(A_host[:m], Bs[(ph * len(M_SWEEP) + i) % n_copies], C_host[m])
+    arrays = [bg.host_gemm_array([(A_block[offs[m]:offs[m] + m], Bs[(ph * len(M_SWEEP) + i) % n_copies],
+                                   C_block[offs[m]:offs[m] + m])
                                   for i, m in enumerate(M_SWEEP)]) for ph in range(n_copies)]
-    # three steps' worth of staging slots: a step's copy-ins run while the previous step computes,
-    # and its copy-outs two steps later
-    staging = torch.empty(bg.bi_gemm_host_batch_staging_bytes(plan, arrays[0], 3 * len(M_SWEEP)),
+    # three steps' worth of staging regions: a step's copy-ins run while the previous step
+    # computes, and its copy-outs two steps later
+    staging = torch.empty(bg.bi_gemm_host_batch_staging_bytes(plan, arrays[0], 3),
                           dtype=torch.uint8, device=dev)
     cin, cout = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     cap = torch.cuda.Stream(device=dev)
@@ -684,22 +722,24 @@ def measure_e2e(bg, plan, Bs, dev, stream, args, world, barrier):
     with torch.cuda.stream(stream):
         for i, m in enumerate(M_SWEEP):
             ref = torch.empty((m, N_DEC), dtype=torch.bfloat16, device=dev)
-            bg.bi_gemm_run(plan, A_host[:m].to(dev), Bs[(last * len(M_SWEEP) + i) % n_copies], ref,
-                           stream=stream)
+            bg.bi_gemm_run(plan, A_block[offs[m]:offs[m] + m].to(dev), Bs[(last * len(M_SWEEP) + i) % n_copies],
+                           ref, stream=stream)
             torch.cuda.synchronize()
-            check_ok &= bool(torch.equal(ref.cpu().view(torch.int16), C_host[m].view(torch.int16)))
+            check_ok &= bool(torch.equal(ref.cpu().view(torch.int16),
+                                         C_block[offs[m]:offs[m] + m].view(torch.int16)))
 
     h2d = sum(m * K_DEC * 2 for m in M_SWEEP)
     d2h = sum(m * N_DEC * 2 for m in M_SWEEP)
     return {"value": sweep_bytes() * steps * world / (ms * 1e-3) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": ms / steps,
-            "path": ("bi_gemm_run_host_batch, one call per step with the sweep's nine GEMMs: copy-ins "
-                     "on a copy-in stream, kernels on the compute stream, copy-outs (two steps "
-                     "later) on a copy-out stream, ordered by the library's events over 27 staging "
-                     "slots; %d steps and a flush per captured CUDA graph, replayed back to back"
-                     % per_graph),
-            "copy_floor_ms_per_step": max(h2d / h2d_gbs, d2h / d2h_gbs, (h2d + d2h) / duplex_gbs) / 1e6,
+            "path": ("bi_gemm_run_host_batch, one call per step with the sweep's nine GEMMs, whose "
+                     "activations and results lie back to back in one pinned block each: one "
+                     "copy-in on a copy-in stream, the kernels on the compute stream, one copy-out "
+                     "(two steps later) on a copy-out stream, ordered by the library's events over "
+                     "3 staging regions; %d steps and a flush per captured CUDA graph, replayed "
+                     "back to back" % per_graph),
+            "copy_floor_ms_per_step": copies,
             "pinned_h2d_gbs": h2d_gbs, "pinned_d2h_gbs": d2h_gbs,
             "pinned_both_directions_gbs": duplex_gbs,
             "gpu_numa_node": node, "host_buffers_on_gpu_node": affinity is not None,

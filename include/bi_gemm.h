@@ -267,35 +267,39 @@ bi_status_t bi_gemm_run_host(bi_plan_t plan, int64_t M,
  * invariance") with A, scale_a and C in host memory and B, scale_b on the device:
  *   M, A_host [M][lda], B [N][ldb] (device), C_host [M][ldc] bf16, scale_a_host
  *   [ceil(K/128)][ld_sa] and scale_b (device) as bi_gemm_run (FP8 plans only; NULL for bf16).
- * Call i's A (and scale_a) is copied into staging slot (running count) % S on copy_in; once all
- * of the batch's copy-ins have landed, its GEMMs run on compute in call order.  The batch's C
- * results are copied back to its C_host buffers on copy_out by the second batch call of this
- * plan after it (or by bi_gemm_host_batch_flush): they are queued after that batch's copy-ins
- * and wait for this batch's kernels, which by then have finished.  (A copy-out queued while its
- * kernel is still running holds up the copies queued after it; deferring it lets later copy-ins
- * run under the kernels.)  A slot is refilled only after its previous copy-out has completed.
- * S is the number of slots the staging buffer holds (2 to 32): give it three batches' worth.
- * At most 1024 calls.
+ * Each batch owns one region of the staging buffer (batch count % S).  On copy_in its calls' A
+ * (and scale_a) are copied into it; with BI_PLAN_HOST_ROW_BLOCKS, calls whose host A rows begin
+ * where the previous call's end (a batch laid out back to back in host memory) share one copy.  Once all of the batch's
+ * copy-ins have landed, its GEMMs run on compute in call order, writing C into the region.  The
+ * C results are copied back to the C_host buffers on copy_out (with that flag, again one copy
+ * for calls whose host C rows follow each other) by the second batch call of this plan after it (or by
+ * bi_gemm_host_batch_flush): they are queued after that batch's copy-ins and wait for this
+ * batch's kernels, which by then have finished.  (A copy-out queued while its kernel is still
+ * running holds up the copies queued after it; deferring it lets later copy-ins run under the
+ * kernels.)  A region is refilled only after its previous batch's copy-outs have completed.
+ * S is the number of regions the staging buffer holds (2 to 32): give it three.  At most 1024
+ * calls per batch.
  * The call returns once everything is enqueued.  A batch's results are in host memory once
  * copy_out reaches the copy-outs that a later batch call (or the flush) enqueued:
  * synchronise copy_out after bi_gemm_host_batch_flush to wait for all of them.  Host buffers
  * must stay valid until then; pinned host memory makes the copies asynchronous.  The three
  * streams may be the same stream (no overlap).
  * Staging: caller-owned device memory, 256-byte aligned; bi_gemm_host_batch_staging_bytes(plan,
- * n, calls, S) gives the bytes for S slots of these calls (0 for invalid arguments or S outside
- * 2..32); the library allocates nothing.  Passing a different staging buffer (or a batch with a
- * different largest call) first flushes and makes the first copy-in wait for every copy-out
- * issued so far.  One batch per plan at a time (a plan-wide lock).
+ * n, calls, S) gives the bytes for S regions of these calls (0 for invalid arguments, more than
+ * 1024 calls or S outside 2..32); the library allocates nothing.  Passing a different staging
+ * buffer (or a batch whose region has another size) first flushes and makes the copy-ins wait
+ * for every copy-out issued so far.  One batch per plan at a time (a plan-wide lock).
  * Stream capture: when compute is capturing, the first batch of the capture forks copy_in and
  * copy_out from compute (copy-outs pending from before the capture must have been flushed, else
- * BI_ERR_INVALID_ARG), the slots are ordered among the capture's own batches, and
+ * BI_ERR_INVALID_ARG), the regions are ordered among the capture's own batches, and
  * bi_gemm_host_batch_flush, called before the capture ends, enqueues the last copy-outs and
  * joins both copy streams back into compute.  Replays of the graph are ordered by their stream.
  * Errors: every call's arguments are checked before anything is enqueued (as bi_gemm_run; the
  * scale_a of a call is only copied and may have any alignment); BI_ERR_INVALID_ARG for a
  * missing or short staging buffer, BI_ERR_ALIGNMENT for a misaligned one.  A CUDA failure while
  * enqueueing returns BI_ERR_CUDA with the work before it enqueued.  BI_ERR_INVALID_ARG also for
- * a staging buffer of fewer than two slots.  Grouped, split-K and e2m1 plans are refused.
+ * a staging buffer of fewer than two regions or more than 1024 calls.  Grouped, split-K and
+ * e2m1 plans are refused.
  */
 typedef struct {
     int64_t M;
@@ -419,9 +423,14 @@ bi_status_t bi_gemm_run_splitk(bi_plan_t plan, int64_t M,
  * previous kernel in the stream is still running; it still waits for that kernel to complete
  * before it reads A or scale_a or writes C or the status word.  The flag changes when B is
  * read, never a result.  Off by default; grouped plans ignore it.
+ * BI_PLAN_HOST_ROW_BLOCKS: the caller promises that, within one bi_gemm_run_host_batch, host
+ * buffers of consecutive calls that touch end to start (A_host after A_host, C_host after
+ * C_host) belong to one host allocation.  The batch then moves each such run of calls with one
+ * copy (a copy may not span two allocations).  Off by default: one copy per call.
  * Errors: BI_ERR_INVALID_ARG (plan == NULL or an unknown flag bit).
  */
 #define BI_PLAN_RESIDENT_WEIGHTS 1u
+#define BI_PLAN_HOST_ROW_BLOCKS 2u
 bi_status_t bi_gemm_plan_set_flags(bi_plan_t plan, uint32_t flags);
 
 /*

@@ -17,6 +17,7 @@ from .binding import (  # noqa: F401
     BI_DTYPE_E2M1_W4A8,
     BI_DTYPE_E4M3_BLOCKSCALED,
     BI_PLAN_RESIDENT_WEIGHTS,
+    BI_PLAN_HOST_ROW_BLOCKS,
     BiGemmError,
     Plan,
     bi_decode_attention,

@@ -21,6 +21,7 @@ BI_DTYPE_E4M3_BLOCKSCALED = 1
 BI_DTYPE_E2M1_W4A8 = 2
 BI_DEBUG_SKIP_FIRST_LOAD = 1
 BI_PLAN_RESIDENT_WEIGHTS = 1
+BI_PLAN_HOST_ROW_BLOCKS = 2
 
 STATUS_NAMES = {
     0: "BI_OK", 1: "BI_ERR_INVALID_ARG", 2: "BI_ERR_ALIGNMENT", 3: "BI_ERR_UNSUPPORTED_SHAPE",
@@ -291,7 +292,7 @@ def host_gemm_array(calls) -> "ctypes.Array":
     return arr
 
 
-def bi_gemm_host_batch_staging_bytes(plan: Plan, calls, slots: int = 6) -> int:
+def bi_gemm_host_batch_staging_bytes(plan: Plan, calls, slots: int = 3) -> int:
     arr = calls if isinstance(calls, ctypes.Array) else host_gemm_array(calls)
     return int(load_library().bi_gemm_host_batch_staging_bytes(plan.handle, len(arr), arr, slots))
 
@@ -383,7 +384,8 @@ def bi_gemm_run_w4a8(plan: Plan, A, scale_a, W, w_scale, C, w_zero=None, workspa
 
 
 def bi_gemm_plan_set_flags(plan: Plan, flags: int):
-    """BI_PLAN_RESIDENT_WEIGHTS: B is never written by an earlier kernel on the launch's stream."""
+    """BI_PLAN_RESIDENT_WEIGHTS: B is never written by an earlier kernel on the launch's stream.
+    BI_PLAN_HOST_ROW_BLOCKS: touching host buffers of one host batch are one allocation."""
     _check(load_library().bi_gemm_plan_set_flags(plan.handle, flags), "bi_gemm_plan_set_flags")
 
 

@@ -307,10 +307,11 @@ bi_status_t current_device(int *dev_out, DeviceInfo **info_out)
 // The plan object
 // ---------------------------------------------------------------------------------------------
 
-// Staging slots of bi_gemm_run_host_batch: as many as the caller's staging holds, 2 to
-// kMaxHostSlots.  A slot is refilled once its previous copy-out has completed, so the copy-in
-// stream runs up to (slots - 1) GEMMs ahead of the kernels.
+// Staging regions of bi_gemm_run_host_batch: one per batch in flight, as many as the caller's
+// staging holds, 2 to kMaxHostSlots.  A region is refilled once its previous batch's copy-outs
+// have completed, so the copy-in stream runs up to (regions - 1) batches ahead of the kernels.
 constexpr int kMaxHostSlots = 32;
+constexpr int kMaxHostCalls = 1024;   // GEMMs in one batch
 
 // A batch's copy-outs are enqueued this many batches later (or by a flush): by then the kernels
 // they wait for have long finished, so they never hold up the copy-ins queued behind them.
@@ -321,24 +322,23 @@ struct PendingOut {
     void *c_host;
     const void *c_dev;
     size_t bytes;
-    int slot;
 };
 
 struct HostPipe {
     cudaEvent_t in_done[kMaxHostSlots] = {};
     cudaEvent_t gemm_done[kMaxHostSlots] = {};
     cudaEvent_t out_done[kMaxHostSlots] = {};
-    uint64_t next = 0;                  // calls issued so far (slot = next % slots)
+    uint64_t next = 0;                  // batches issued so far (region = next % slots)
     const void *staging = nullptr;      // layout of the last batch
-    size_t slot_bytes = 0;
-    int slots = 0;
-    // copy-outs of the last kHostDefer batches, not yet enqueued, oldest first, each with the
-    // gemm_done slot recorded after that batch's kernels
+    size_t slot_bytes = 0;              // bytes of one region
+    int slots = 0;                      // regions
+    // copy-outs of the last kHostDefer batches, not yet enqueued, oldest first, each with its
+    // region (whose gemm_done was recorded after that batch's kernels)
     std::deque<std::pair<std::vector<PendingOut>, int>> pending;
-    // stream capture: the capture the batches belong to, and its own slot order
+    // stream capture: the capture the batches belong to, and its own region order
     unsigned long long cap_id = 0;
     uint64_t cap_next = 0;
-    uint32_t cap_used = 0;              // slots filled inside the capture
+    uint32_t cap_used = 0;              // regions filled inside the capture
 };
 
 struct bi_plan_s {
@@ -929,7 +929,7 @@ bi_status_t bi_gemm_set_wait_timeout(bi_plan_t plan, uint64_t timeout_ns)
 
 bi_status_t bi_gemm_plan_set_flags(bi_plan_t plan, uint32_t flags)
 {
-    if (!plan || (flags & ~BI_PLAN_RESIDENT_WEIGHTS))
+    if (!plan || (flags & ~(BI_PLAN_RESIDENT_WEIGHTS | BI_PLAN_HOST_ROW_BLOCKS)))
         return BI_ERR_INVALID_ARG;
     plan->flags = flags;
     return BI_OK;
@@ -1126,49 +1126,99 @@ static bi_status_t host_batch_flush(HostPipe *hp, cudaStream_t copy_out, size_t 
         if (cudaStreamWaitEvent(copy_out, hp->gemm_done[b.second], 0) != cudaSuccess)
             return BI_ERR_CUDA;
         for (const PendingOut &o : b.first)
-            if (cudaMemcpyAsync(o.c_host, o.c_dev, o.bytes, cudaMemcpyDeviceToHost, copy_out) != cudaSuccess ||
-                cudaEventRecord(hp->out_done[o.slot], copy_out) != cudaSuccess)
+            if (cudaMemcpyAsync(o.c_host, o.c_dev, o.bytes, cudaMemcpyDeviceToHost, copy_out) != cudaSuccess)
                 return BI_ERR_CUDA;
+        if (cudaEventRecord(hp->out_done[b.second], copy_out) != cudaSuccess)
+            return BI_ERR_CUDA;
         hp->pending.pop_front();
     }
     return BI_OK;
 }
 
-// Bytes of one staging slot of bi_gemm_run_host_batch for these calls: A, C and (FP8) scale_a
-// of the largest call, each rounded up to 256 bytes.  Returns -1 for arguments no call may have.
-static int64_t host_batch_slot_bytes(const bi_plan_s *plan, int n, const bi_host_gemm_t *calls)
+// Where the calls of one host batch live in its staging region: the A rows of every call, then
+// the C rows, then (FP8) the scale_a blocks.  With BI_PLAN_HOST_ROW_BLOCKS a call whose host A
+// rows begin where the previous call's end shares that call's copy (one run), and likewise for
+// C, so a batch laid out back to back in one host allocation moves with one copy each way
+// instead of one per call (without the flag nothing says two touching buffers are one
+// allocation, and a copy may not span two).  Every run starts on a 256-byte boundary; a call
+// inside a run sits at its host offset from the run's start.
+struct HostRun {
+    const void *host;   // first byte in host memory
+    int64_t off;        // offset in the region's A (or C) part
+    int64_t bytes;
+};
+
+struct BatchLayout {
+    std::vector<int64_t> a_off, c_off, s_off;   // per call, within their parts (-1: M == 0)
+    std::vector<HostRun> a_runs, c_runs;
+    int64_t a_part = 0, c_part = 0, s_part = 0;
+    int64_t bytes() const { return a_part + c_part + s_part; }
+};
+
+// Returns false for arguments no call may have (negative or huge sizes).
+static bool host_batch_layout(const bi_plan_s *plan, int n, const bi_host_gemm_t *calls, BatchLayout *L)
 {
     const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
     const int elt = fp8 ? 1 : 2;
     const int64_t kb = (plan->k + 127) / 128;
     const int64_t cap = int64_t(1) << 40;   // bounds every factor, so no product below can wrap
+    L->a_off.assign(static_cast<size_t>(n), -1);
+    L->c_off.assign(static_cast<size_t>(n), -1);
+    L->s_off.assign(static_cast<size_t>(n), -1);
     int64_t a = 0, c = 0, sa = 0;
+    const bool merge = (plan->flags & BI_PLAN_HOST_ROW_BLOCKS) != 0;
+    auto place = [merge](std::vector<HostRun> &runs, int64_t &end, const void *host, int64_t bytes) {
+        const unsigned char *h = static_cast<const unsigned char *>(host);
+        if (merge && !runs.empty()) {
+            HostRun &r = runs.back();
+            if (static_cast<const unsigned char *>(r.host) + r.bytes == h) {
+                const int64_t off = r.off + r.bytes;
+                r.bytes += bytes;
+                end = r.off + r.bytes;
+                return off;
+            }
+        }
+        const int64_t off = round256(end);
+        runs.push_back(HostRun{host, off, bytes});
+        end = off + bytes;
+        return off;
+    };
     for (int i = 0; i < n; ++i) {
         const bi_host_gemm_t &g = calls[i];
         if (g.M < 0 || g.M > cap || g.lda < 0 || g.lda > cap || g.ldc < 0 || g.ldc > cap ||
             g.ld_sa < 0 || g.ld_sa > cap)
-            return -1;
-        a = a > g.M * g.lda * elt ? a : g.M * g.lda * elt;
-        c = c > g.M * g.ldc * 2 ? c : g.M * g.ldc * 2;
-        if (fp8)
-            sa = sa > kb * g.ld_sa * 4 ? sa : kb * g.ld_sa * 4;
+            return false;
+        if (g.M == 0)
+            continue;
+        if (plan->k > 0)
+            L->a_off[i] = place(L->a_runs, a, g.A_host, g.M * g.lda * elt);
+        L->c_off[i] = place(L->c_runs, c, g.C_host, g.M * g.ldc * 2);
+        if (fp8 && plan->k > 0) {
+            L->s_off[i] = sa;
+            sa += round256(kb * g.ld_sa * 4);
+        }
     }
-    return round256(a) + round256(c) + round256(sa);
+    L->a_part = round256(a);
+    L->c_part = round256(c);
+    L->s_part = sa;
+    return true;
 }
 
 size_t bi_gemm_host_batch_staging_bytes(bi_plan_t plan, int n, const bi_host_gemm_t *calls, int slots)
 {
-    if (!plan || n < 0 || (n > 0 && !calls) || slots < 2 || slots > kMaxHostSlots)
+    if (!plan || n < 0 || n > kMaxHostCalls || (n > 0 && !calls) || slots < 2 || slots > kMaxHostSlots)
         return 0;
-    const int64_t slot = host_batch_slot_bytes(plan, n, calls);
-    return slot < 0 ? 0 : static_cast<size_t>(slot) * static_cast<size_t>(slots);
+    BatchLayout L;
+    if (!host_batch_layout(plan, n, calls, &L))
+        return 0;
+    return static_cast<size_t>(L.bytes()) * static_cast<size_t>(slots);
 }
 
 bi_status_t bi_gemm_run_host_batch(bi_plan_t plan, int n, const bi_host_gemm_t *calls, void *staging,
                                    size_t staging_bytes, cudaStream_t copy_in, cudaStream_t compute,
                                    cudaStream_t copy_out)
 {
-    if (!plan || n < 0 || (n > 0 && !calls))
+    if (!plan || n < 0 || n > kMaxHostCalls || (n > 0 && !calls))
         return BI_ERR_INVALID_ARG;
     if (plan->experts != 1 || plan->k_splits > 1)
         return BI_ERR_INVALID_ARG;
@@ -1177,33 +1227,30 @@ bi_status_t bi_gemm_run_host_batch(bi_plan_t plan, int n, const bi_host_gemm_t *
     if (n == 0 || plan->n == 0)
         return BI_OK;
     const bool fp8 = plan->dtype == BI_DTYPE_E4M3_BLOCKSCALED;
-    const int elt = fp8 ? 1 : 2;
     const int64_t kb = (plan->k + 127) / 128;
-    const int64_t slot_bytes = host_batch_slot_bytes(plan, n, calls);
-    if (slot_bytes < 0)
+    BatchLayout L;
+    if (!host_batch_layout(plan, n, calls, &L))
         return BI_ERR_INVALID_ARG;
-    if (!staging || slot_bytes == 0 || staging_bytes < static_cast<size_t>(slot_bytes) * 2)
+    const int64_t region_bytes = L.bytes();
+    if (region_bytes == 0)
+        return BI_OK;   // every call has M == 0
+    if (!staging || staging_bytes < static_cast<size_t>(region_bytes) * 2)
         return BI_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(staging) & 255u)
         return BI_ERR_ALIGNMENT;
-    const size_t fit = staging_bytes / static_cast<size_t>(slot_bytes);
+    const size_t fit = staging_bytes / static_cast<size_t>(region_bytes);
     const int slots = fit > static_cast<size_t>(kMaxHostSlots) ? kMaxHostSlots : static_cast<int>(fit);
-    int64_t a_max = 0, c_max = 0;
-    for (int i = 0; i < n; ++i) {
-        a_max = a_max > calls[i].M * calls[i].lda * elt ? a_max : calls[i].M * calls[i].lda * elt;
-        c_max = c_max > calls[i].M * calls[i].ldc * 2 ? c_max : calls[i].M * calls[i].ldc * 2;
-    }
-    const int64_t c_off = round256(a_max), s_off = c_off + round256(c_max);
-    // Validate every call before enqueueing anything (against slot 0's addresses: every slot has
-    // the same alignment).
     unsigned char *base = static_cast<unsigned char *>(staging);
+    // Validate every call before enqueueing anything, at its addresses in region 0 (every region
+    // has the same alignment).
     for (int i = 0; i < n; ++i) {
         const bi_host_gemm_t &g = calls[i];
         if (g.M == 0)
             continue;
         if (!g.C_host || (plan->k > 0 && !g.A_host))
             return BI_ERR_INVALID_ARG;
-        bi_status_t st = check_common(plan, g.M, base, g.lda, g.B, g.ldb, base + c_off, g.ldc);
+        unsigned char *A_dev = plan->k > 0 ? base + L.a_off[i] : base;
+        bi_status_t st = check_common(plan, g.M, A_dev, g.lda, g.B, g.ldb, base + L.a_part + L.c_off[i], g.ldc);
         if (st != BI_OK)
             return st;
         if (fp8 && plan->k > 0) {
@@ -1243,9 +1290,9 @@ bi_status_t bi_gemm_run_host_batch(bi_plan_t plan, int n, const bi_host_gemm_t *
             hp->cap_used = 0;
         }
     } else {
-        // A different staging buffer or layout than the last batch: the slots may overlap the
-        // old ones, so the first copy-in waits for every copy-out issued so far.
-        const bool relayout = hp->staging != staging || hp->slot_bytes != static_cast<size_t>(slot_bytes) ||
+        // A different staging buffer or layout than the last batch: the regions may overlap the
+        // old ones, so the copy-ins wait for every copy-out issued so far.
+        const bool relayout = hp->staging != staging || hp->slot_bytes != static_cast<size_t>(region_bytes) ||
                               hp->slots != slots;
         if (relayout) {
             if ((st = host_batch_flush(hp, copy_out)) != BI_OK)
@@ -1257,63 +1304,57 @@ bi_status_t bi_gemm_run_host_batch(bi_plan_t plan, int n, const bi_host_gemm_t *
             hp->next = 0;
         }
         hp->staging = staging;
-        hp->slot_bytes = static_cast<size_t>(slot_bytes);
+        hp->slot_bytes = static_cast<size_t>(region_bytes);
         hp->slots = slots;
     }
-    // This batch's copy-ins (a slot is refilled once its previous copy-out has completed); then
-    // the copy-outs of the batch kHostDefer batches back, queued after these copy-ins, behind
-    // kernels that have long finished; then this batch's kernels after one wait for its
-    // copy-ins.  A copy-out queued while its kernel is still running would hold up the copies
-    // queued after it.
-    std::vector<PendingOut> outs;
-    outs.reserve(static_cast<size_t>(n));
-    int last_slot = -1;
-    for (int i = 0; i < n; ++i) {
-        const bi_host_gemm_t &g = calls[i];
-        if (g.M == 0)
-            continue;
-        uint64_t &next = captured ? hp->cap_next : hp->next;
-        const int slot = static_cast<int>(next % static_cast<uint64_t>(slots));
-        ++next;
-        unsigned char *A_dev = base + slot * slot_bytes;
-        float *sa_dev = reinterpret_cast<float *>(A_dev + s_off);
-        const bool reused = captured ? ((hp->cap_used >> slot) & 1u) != 0 : true;
-        if (reused && cudaStreamWaitEvent(copy_in, hp->out_done[slot], 0) != cudaSuccess)
+    // This batch's copy-ins into its region (refilled once the region's previous copy-outs have
+    // completed); then the copy-outs of the batch kHostDefer batches back, queued after these
+    // copy-ins, behind kernels that have long finished; then this batch's kernels after one wait
+    // for its copy-ins.  A copy-out queued while its kernel is still running would hold up the
+    // copies queued after it.
+    uint64_t &next = captured ? hp->cap_next : hp->next;
+    const int r = static_cast<int>(next % static_cast<uint64_t>(slots));
+    ++next;
+    unsigned char *R = base + r * region_bytes;
+    const bool reused = captured ? ((hp->cap_used >> r) & 1u) != 0 : true;
+    if (reused && cudaStreamWaitEvent(copy_in, hp->out_done[r], 0) != cudaSuccess)
+        return BI_ERR_CUDA;
+    if (captured)
+        hp->cap_used |= 1u << r;
+    for (const HostRun &run : L.a_runs)
+        if (cudaMemcpyAsync(R + run.off, run.host, static_cast<size_t>(run.bytes), cudaMemcpyHostToDevice,
+                            copy_in) != cudaSuccess)
             return BI_ERR_CUDA;
-        if (captured)
-            hp->cap_used |= 1u << slot;
-        last_slot = slot;
-        if (plan->k > 0) {
-            if (cudaMemcpyAsync(A_dev, g.A_host, static_cast<size_t>(g.M * g.lda * elt),
-                                cudaMemcpyHostToDevice, copy_in) != cudaSuccess)
+    if (fp8)
+        for (int i = 0; i < n; ++i)
+            if (L.s_off[i] >= 0 &&
+                cudaMemcpyAsync(R + L.a_part + L.c_part + L.s_off[i], calls[i].scale_a_host,
+                                static_cast<size_t>(kb * calls[i].ld_sa * 4), cudaMemcpyHostToDevice,
+                                copy_in) != cudaSuccess)
                 return BI_ERR_CUDA;
-            if (fp8 && cudaMemcpyAsync(sa_dev, g.scale_a_host, static_cast<size_t>(kb * g.ld_sa * 4),
-                                       cudaMemcpyHostToDevice, copy_in) != cudaSuccess)
-                return BI_ERR_CUDA;
-        }
-        outs.push_back(PendingOut{g.C_host, A_dev + c_off, static_cast<size_t>(g.M * g.ldc * 2), slot});
-    }
+    std::vector<PendingOut> outs;
+    outs.reserve(L.c_runs.size());
+    for (const HostRun &run : L.c_runs)
+        outs.push_back(PendingOut{const_cast<void *>(run.host), R + L.a_part + run.off,
+                                  static_cast<size_t>(run.bytes)});
     if ((st = host_batch_flush(hp, copy_out, kHostDefer - 1)) != BI_OK)
         return st;
-    if (last_slot < 0)
-        return BI_OK;
-    if (cudaEventRecord(hp->in_done[last_slot], copy_in) != cudaSuccess ||
-        cudaStreamWaitEvent(compute, hp->in_done[last_slot], 0) != cudaSuccess)
+    if (cudaEventRecord(hp->in_done[r], copy_in) != cudaSuccess ||
+        cudaStreamWaitEvent(compute, hp->in_done[r], 0) != cudaSuccess)
         return BI_ERR_CUDA;
-    size_t j = 0;
     for (int i = 0; i < n; ++i) {
         const bi_host_gemm_t &g = calls[i];
         if (g.M == 0)
             continue;
-        unsigned char *A_dev = base + outs[j++].slot * slot_bytes;
-        if ((st = bi_gemm_run(plan, g.M, A_dev, g.lda, g.B, g.ldb, A_dev + c_off, g.ldc,
-                              fp8 ? reinterpret_cast<float *>(A_dev + s_off) : nullptr, g.ld_sa,
-                              fp8 ? g.scale_b : nullptr, compute)) != BI_OK)
+        unsigned char *A_dev = plan->k > 0 ? R + L.a_off[i] : R;
+        float *sa_dev = fp8 && plan->k > 0 ? reinterpret_cast<float *>(R + L.a_part + L.c_part + L.s_off[i]) : nullptr;
+        if ((st = bi_gemm_run(plan, g.M, A_dev, g.lda, g.B, g.ldb, R + L.a_part + L.c_off[i], g.ldc,
+                              sa_dev, g.ld_sa, fp8 ? g.scale_b : nullptr, compute)) != BI_OK)
             return st;
     }
-    if (cudaEventRecord(hp->gemm_done[last_slot], compute) != cudaSuccess)
+    if (cudaEventRecord(hp->gemm_done[r], compute) != cudaSuccess)
         return BI_ERR_CUDA;
-    hp->pending.emplace_back(std::move(outs), last_slot);
+    hp->pending.emplace_back(std::move(outs), r);
     return BI_OK;
 }
 

@@ -190,6 +190,25 @@ def test_host_batch_rejects_bad_arguments_before_any_device_call():
     assert need == 6 * slot
     assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 2, arr, 1) == 0
     assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 2, arr, 33) == 0
+    many = (HG * 1025)(*([ok] * 1025))
+    assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 1025, many, 3) == 0
+    assert lib.bi_gemm_run_host_batch(plan.handle, 1025, many, 4096, 1 << 30, None, None, None) == \
+        S["BI_ERR_INVALID_ARG"]
+    # with BI_PLAN_HOST_ROW_BLOCKS, calls whose host rows follow one another share one copy and
+    # one run of the region: one-row calls with a 1040-byte pitch take 2080 bytes of A together
+    # (2304 rounded), 2 x 1280 apart
+    apart = (HG * 2)(HG(1, 4096, 520, 4096, 512, 1 << 20, 256, None, 0, None),
+                     HG(1, 8192, 520, 4096, 512, 2 << 20, 256, None, 0, None))
+    adjacent = (HG * 2)(HG(1, 4096, 520, 4096, 512, 1 << 20, 256, None, 0, None),
+                        HG(1, 4096 + 1040, 520, 4096, 512, (1 << 20) + 512, 256, None, 0, None))
+    # without BI_PLAN_HOST_ROW_BLOCKS touching buffers are copied apart (they may be two allocations)
+    assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 2, apart, 2) == 2 * (2560 + 1024)
+    assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 2, adjacent, 2) == 2 * (2560 + 1024)
+    assert lib.bi_gemm_plan_set_flags(plan.handle, 4) == S["BI_ERR_INVALID_ARG"]
+    assert lib.bi_gemm_plan_set_flags(plan.handle, binding.BI_PLAN_HOST_ROW_BLOCKS) == 0
+    assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 2, apart, 2) == 2 * (2560 + 1024)
+    assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 2, adjacent, 2) == 2 * (2304 + 1024)
+    assert lib.bi_gemm_plan_set_flags(plan.handle, 0) == 0
     run = lib.bi_gemm_run_host_batch
     assert run(None, 2, arr, 4096, need, None, None, None) == S["BI_ERR_INVALID_ARG"]
     assert run(plan.handle, 0, None, None, 0, None, None, None) == 0           # empty batch
@@ -258,7 +277,7 @@ def test_plan_flags_accept_known_bits_only():
     assert lib.bi_gemm_plan_set_flags(None, 0) == S["BI_ERR_INVALID_ARG"]
     assert lib.bi_gemm_plan_set_flags(plan.handle, bg.BI_PLAN_RESIDENT_WEIGHTS) == 0
     assert lib.bi_gemm_plan_set_flags(plan.handle, 0) == 0
-    assert lib.bi_gemm_plan_set_flags(plan.handle, 2) == S["BI_ERR_INVALID_ARG"]
+    assert lib.bi_gemm_plan_set_flags(plan.handle, 4) == S["BI_ERR_INVALID_ARG"]
     assert lib.bi_gemm_plan_set_flags(plan.handle, 0x80000000) == S["BI_ERR_INVALID_ARG"]
     # the flags change when B is read, never the plan
     before = bg.bi_gemm_plan_describe(plan)

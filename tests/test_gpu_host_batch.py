@@ -1,6 +1,7 @@
 """bi_gemm_run_host_batch: host-buffer GEMMs pipelined behind the ABI (copy-in, kernel and
-copy-out on three streams, staging slots reused in turn, a batch's copy-outs enqueued two
-batches later or by a flush).
+copy-out on three streams, one staging region per batch reused in turn, a batch's copy-outs
+enqueued two batches later or by a flush, calls whose host rows follow one another moved with
+one copy).
 
 Each batch's results must equal the same GEMMs run by bi_gemm_run on device buffers, bit for bit
 (batch invariance: a row's bits do not depend on which call, slot or stream carried it), and the
@@ -43,7 +44,7 @@ def test_batches_match_device_runs_and_the_oracle():
             C = torch.full((M, N), float("nan"), dtype=torch.bfloat16).pin_memory()
             calls.append((A, Bs[(b + i) % 2], C))
         batches.append(calls)
-    need = bg.bi_gemm_host_batch_staging_bytes(plan, batches[0], 3 * len(Ms))
+    need = bg.bi_gemm_host_batch_staging_bytes(plan, batches[0], 3)
     staging = [torch.empty(need, dtype=torch.uint8, device=DEV) for _ in range(2)]
     torch.cuda.synchronize()
     for b, calls in enumerate(batches):   # no synchronisation between batches; staging changes at b = 2
@@ -98,7 +99,7 @@ def test_batches_captured_in_a_graph_match_device_runs():
             C = torch.full((M, N), float("nan"), dtype=torch.bfloat16).pin_memory()
             calls.append((A, B, C))
         batches.append(calls)
-    staging = torch.empty(bg.bi_gemm_host_batch_staging_bytes(plan, batches[0], 8), dtype=torch.uint8,
+    staging = torch.empty(bg.bi_gemm_host_batch_staging_bytes(plan, batches[0], 3), dtype=torch.uint8,
                           device=DEV)
     cin, cout, cap = (torch.cuda.Stream() for _ in range(3))
     for calls in batches:   # once outside capture (first-use set-up)
@@ -121,3 +122,42 @@ def test_batches_captured_in_a_graph_match_device_runs():
             ref = device_run(plan, A, B_)
             assert torch.equal(C.view(torch.int16), ref.view(torch.int16)), f"batch {b} call {i}"
     del g
+
+
+def test_back_to_back_host_rows_share_copies_and_match_device_runs():
+    """With BI_PLAN_HOST_ROW_BLOCKS a batch whose A (and C) slices lie back to back in one pinned
+    block moves them with one copy each way; interleaved with batches whose slices do not (and
+    whose staging region therefore has another size), every result still equals the device run
+    bit for bit."""
+    N, K = 4096, 7168
+    plan = bg.bi_gemm_plan(N, K)
+    bg.bi_gemm_plan_set_flags(plan, bg.BI_PLAN_HOST_ROW_BLOCKS)   # each block is one allocation
+    B = inputs.bf16_gaussian((N, K), seed=5701, std=K ** -0.5, device=DEV)
+    Ms = [1, 2, 4, 8, 16, 32, 64, 128, 256]
+    offs = np.concatenate([[0], np.cumsum(Ms)])
+    blocks = []
+    for b in range(3):
+        A = inputs.bf16_gaussian((int(offs[-1]), K), seed=5710 + b).pin_memory()
+        C = torch.full((int(offs[-1]), N), float("nan"), dtype=torch.bfloat16).pin_memory()
+        blocks.append((A, C))
+    def calls_of(b, adjacent):
+        A, C = blocks[b]
+        if adjacent:
+            return [(A[offs[i]:offs[i + 1]], B, C[offs[i]:offs[i + 1]]) for i in range(len(Ms))]
+        # the same slices in reverse call order: no call's rows follow the previous call's
+        return [(A[offs[i]:offs[i + 1]], B, C[offs[i]:offs[i + 1]]) for i in reversed(range(len(Ms)))]
+    batches = [calls_of(0, True), calls_of(1, False), calls_of(2, True)]
+    need = max(bg.bi_gemm_host_batch_staging_bytes(plan, c, 3) for c in batches)
+    staging = torch.empty(need, dtype=torch.uint8, device=DEV)
+    cin, cmp, cout = (torch.cuda.Stream() for _ in range(3))
+    torch.cuda.synchronize()
+    for calls in batches:
+        bg.bi_gemm_run_host_batch(plan, calls, staging, copy_in=cin, compute=cmp, copy_out=cout)
+    bg.bi_gemm_host_batch_flush(plan, copy_in=cin, compute=cmp, copy_out=cout)
+    cout.synchronize()
+    bg.bi_gemm_sync_status(plan, stream=cmp)
+    for b, calls in enumerate(batches):
+        for i, (A, B_, C) in enumerate(calls):
+            ref = device_run(plan, A, B_)
+            assert torch.equal(C.view(torch.int16), ref.view(torch.int16)), f"batch {b} call {i}"
+
