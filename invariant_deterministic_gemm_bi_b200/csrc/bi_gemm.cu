@@ -362,6 +362,10 @@ struct bi_plan_s {
     // Four adjacent tiles in lockstep (bf16 plans with K chains), for dense launches whose lockstep pairs
     // still outnumber the SMs.  May be null.
     const KernelEntry *kernel_wide4 = nullptr;
+    // CTA-pair plans 256 columns wide: the same tile cut in two 128-column halves, each run by
+    // its own pair with a 256 x 128 instruction in the same K order, for launches with fewer
+    // tiles than co-resident pairs.  May be null.
+    const KernelEntry *kernel_half = nullptr;
     int small_rows = 64;     // kernel_small serves launches whose A boxes hold at most this many rows
     uint64_t timeout_ns = 2000000000ull;
     uint32_t debug_flags = 0;
@@ -691,6 +695,12 @@ constexpr int kTinyBatchRows = 7;
 // and the launch needs half the CTAs, i.e. fewer waves.
 const KernelEntry *dense_kernel_for(const bi_plan_s *plan, const DeviceInfo *d, int64_t M)
 {
+    if (plan->kernel_half) {
+        const int64_t m_blocks = (M + plan->kernel->bm - 1) / plan->kernel->bm;
+        const int64_t n_blocks = (plan->n + plan->kernel->bn - 1) / plan->kernel->bn;
+        if (m_blocks * n_blocks < pair_grid_limit(plan->kernel, d))
+            return plan->kernel_half;
+    }
     if (plan->kernel_tiny && M <= kTinyBatchRows)
         return plan->kernel_tiny;
     if (plan->kernel_small && a_box_rows_for(plan->kernel_small, M) <= plan->small_rows)
@@ -807,6 +817,8 @@ bi_status_t bi_gemm_plan(bi_plan_t *out, int64_t N, int64_t K, bi_dtype_t dtype,
     // plans with K chains take the 8-chunk form up to 32 rows: their 64-row A boxes would leave
     // a 96 KB B ring at 8 chunks, while 4 chunks keep eight B groups in flight
     p->small_rows = chains > 1 ? 32 : 64;
+    if (num_experts == 1 && k->pair && k->bn == 256)
+        p->kernel_half = find_kernel(256, 128, k->kc, fp8, false, w4, chains);
     if (num_experts > 1 && !k->pair && k->bm == 128 && k->bn == 128) {
         for (int i = 0; i < kNumKernels; ++i)
             if (kKernels[i].pair && kKernels[i].grouped && kKernels[i].bn == 256)
@@ -852,6 +864,7 @@ bi_status_t bi_gemm_plan_column_shard(bi_plan_t *out, bi_plan_t full, int64_t n_
     p->kernel_tiny = full->kernel_tiny;
     p->kernel_wide = full->kernel_wide;
     p->kernel_wide4 = full->kernel_wide4;
+    p->kernel_half = full->kernel_half;
     p->small_rows = full->small_rows;
     p->timeout_ns = full->timeout_ns;
     p->flags = full->flags;

@@ -75,9 +75,9 @@ struct Epi {
 // that cost.  The K chunks of a group are dealt to the issuers round robin (chunk c to issuer
 // c % kIssuers), so that every accumulator still receives its instructions from one thread in
 // ascending K:
-//   - in the dense FP8 kernels with an even number of chunks per group (two issuers): each
-//     128-wide K chunk has its own partial-product buffer, and the epilogue promotes the buffers
-//     in ascending kb whoever issued them;
+//   - in the dense FP8 kernels with an even number of chunks per group (four issuers when the
+//     count is a multiple of 4, else two): each 128-wide K chunk has its own partial-product
+//     buffer, and the epilogue promotes the buffers in ascending kb whoever issued them;
 //   - in the dense bf16 kernels with CH = 2 or 4 K chains: chain c accumulates the chunks with
 //     chunk % CH == c into an accumulator of its own, and the epilogue adds the chains once.  As
 //     many issuers as chains when a group's chunk count allows it (kIssuers divides both CH and
@@ -88,7 +88,7 @@ struct Epi {
 template <bool FP8, int BN, int NSPLIT, bool GROUPED = false, int KC = 1, int CH = 1>
 struct Issue {
     static constexpr int kIssuers = GROUPED ? 1
-                                    : FP8   ? (KC % 2 == 0 ? 2 : 1)
+                                    : FP8   ? (KC % 4 == 0 ? 4 : KC % 2 == 0 ? 2 : 1)
                                     : (CH == 4 && KC % 4 == 0) ? 4
                                     : (CH >= 2 && KC % 2 == 0) ? 2 : 1;
     static constexpr bool kByChunk = kIssuers > 1;
