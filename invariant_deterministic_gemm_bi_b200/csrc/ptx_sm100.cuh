@@ -1,7 +1,7 @@
 // ptx_sm100.cuh -- hand-written inline-PTX wrappers for sm_100a: mbarrier, TMA tensor loads,
 // tcgen05 (tensor-memory allocation, MMA, commit, loads, fences) and small helpers.
 //
-// No TMA load here uses .multicast::cluster: every CTA loads its own tiles.
+// No TMA load here multicasts to other CTAs of a cluster: every CTA loads its own tiles.
 #pragma once
 
 #include <cstdint>
