@@ -292,9 +292,10 @@ def host_gemm_array(calls) -> "ctypes.Array":
     return arr
 
 
-def bi_gemm_host_batch_staging_bytes(plan: Plan, calls, slots: int = 3) -> int:
+def bi_gemm_host_batch_staging_bytes(plan: Plan, calls, regions: int = 3) -> int:
+    """Bytes of staging for `regions` batches like `calls` in flight (2..32; 0 if invalid)."""
     arr = calls if isinstance(calls, ctypes.Array) else host_gemm_array(calls)
-    return int(load_library().bi_gemm_host_batch_staging_bytes(plan.handle, len(arr), arr, slots))
+    return int(load_library().bi_gemm_host_batch_staging_bytes(plan.handle, len(arr), arr, regions))
 
 
 def bi_gemm_run_host_batch(plan: Plan, calls, staging, copy_in=None, compute=None, copy_out=None):

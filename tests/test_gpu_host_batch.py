@@ -4,8 +4,8 @@ enqueued two batches later or by a flush, calls whose host rows follow one anoth
 one copy).
 
 Each batch's results must equal the same GEMMs run by bi_gemm_run on device buffers, bit for bit
-(batch invariance: a row's bits do not depend on which call, slot or stream carried it), and the
-integer variant must match the oracle exactly.  Consecutive batches reuse the slots without any
+(batch invariance: a row's bits do not depend on which call, region or stream carried it), and the
+integer variant must match the oracle exactly.  Consecutive batches reuse the regions without any
 synchronisation in between, and a change of staging buffer mid-stream must still order every
 copy correctly.
 """
