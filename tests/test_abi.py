@@ -209,6 +209,23 @@ def test_host_batch_rejects_bad_arguments_before_any_device_call():
     assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 2, apart, 2) == 2 * (2560 + 1024)
     assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 2, adjacent, 2) == 2 * (2304 + 1024)
     assert lib.bi_gemm_plan_set_flags(plan.handle, 0) == 0
+    # three calls, the first two touching in A and the last two in C: two A runs, two C runs
+    mixed = (HG * 3)(HG(1, 4096, 520, 4096, 512, 1 << 20, 256, None, 0, None),
+                     HG(1, 4096 + 1040, 520, 4096, 512, 3 << 20, 256, None, 0, None),
+                     HG(1, 1 << 16, 520, 4096, 512, (3 << 20) + 512, 256, None, 0, None))
+    assert lib.bi_gemm_plan_set_flags(plan.handle, binding.BI_PLAN_HOST_ROW_BLOCKS) == 0
+    # A: run of 2080 bytes, then a run of 1040 at 2304 -> 3344 -> 3584; C: 512 at 0, then a run of
+    # 1024 at 512 -> 1536
+    assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 3, mixed, 3) == 3 * (3584 + 1536)
+    assert lib.bi_gemm_plan_set_flags(plan.handle, 0) == 0
+    assert lib.bi_gemm_host_batch_staging_bytes(plan.handle, 3, mixed, 3) == 3 * (3840 + 1536)
+    # FP8: each call's scale_a block has its own 256-byte run after A and C
+    f8p = bg.bi_gemm_plan(256, 512, bg.BI_DTYPE_E4M3_BLOCKSCALED)
+    f8calls = (HG * 2)(HG(2, 4096, 512, 4096, 512, 1 << 20, 256, 8192, 2, 4096),
+                       HG(3, 1 << 16, 512, 4096, 512, 2 << 20, 256, 16384, 3, 4096))
+    # A: 1024 (-> 1024) + 1536 -> 2560; C: 1024 + 1536 -> 2560; scales: 4 x 2 x 4 = 32 -> 256,
+    # 4 x 3 x 4 = 48 -> 256
+    assert lib.bi_gemm_host_batch_staging_bytes(f8p.handle, 2, f8calls, 2) == 2 * (2560 + 2560 + 512)
     run = lib.bi_gemm_run_host_batch
     assert run(None, 2, arr, 4096, need, None, None, None) == S["BI_ERR_INVALID_ARG"]
     assert run(plan.handle, 0, None, None, 0, None, None, None) == 0           # empty batch
