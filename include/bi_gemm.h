@@ -315,7 +315,7 @@ typedef struct {
 } bi_host_gemm_t;
 
 size_t bi_gemm_host_batch_staging_bytes(bi_plan_t plan, int n, const bi_host_gemm_t *calls,
-                                        int slots);
+                                        int regions);
 
 bi_status_t bi_gemm_run_host_batch(bi_plan_t plan, int n, const bi_host_gemm_t *calls,
                                    void *staging, size_t staging_bytes,

@@ -1217,14 +1217,14 @@ static bool host_batch_layout(const bi_plan_s *plan, int n, const bi_host_gemm_t
     return true;
 }
 
-size_t bi_gemm_host_batch_staging_bytes(bi_plan_t plan, int n, const bi_host_gemm_t *calls, int slots)
+size_t bi_gemm_host_batch_staging_bytes(bi_plan_t plan, int n, const bi_host_gemm_t *calls, int regions)
 {
-    if (!plan || n < 0 || n > kMaxHostCalls || (n > 0 && !calls) || slots < 2 || slots > kMaxHostSlots)
+    if (!plan || n < 0 || n > kMaxHostCalls || (n > 0 && !calls) || regions < 2 || regions > kMaxHostSlots)
         return 0;
     BatchLayout L;
     if (!host_batch_layout(plan, n, calls, &L))
         return 0;
-    return static_cast<size_t>(L.bytes()) * static_cast<size_t>(slots);
+    return static_cast<size_t>(L.bytes()) * static_cast<size_t>(regions);
 }
 
 bi_status_t bi_gemm_run_host_batch(bi_plan_t plan, int n, const bi_host_gemm_t *calls, void *staging,
