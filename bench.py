@@ -386,6 +386,7 @@ def main():
             tr = json.load(f)
         if tr.get("kernel_source_hash") == kernel_source_hash():
             roofline["traffic"] = tr["bytes_per_launch"]
+            roofline["traffic_from"] = tr["kernel"]
 
     # row invariance on this workload: the M=256 rows against the same rows run at M=1
     row_diffs = 0
@@ -510,10 +511,13 @@ def profile_case(args):
 
 
 def kernel_label(bg, plan) -> str:
+    """The plan's kernel: its tile, instruction K order, and the full-height ring depths (each
+    launch picks one of the plan's scheduling forms by M; the sweep runs five of them)."""
     i = bg.bi_gemm_plan_describe(plan)
     dt = {0: "bf16", 1: "e4m3", 2: "e2m1 x e4m3"}[i["dtype"]]
-    return (f"bi_gemm_kernel<BM={i['block_m']},BN={i['block_n']},{dt}>"
-            f" rings A{i['stages_a']}/B{i['stages']}")
+    order = {0: "ascending K", 1: "split-K", 2: "two K chains", 3: "four K chains"}[i["k_order_id"]]
+    return (f"bi_gemm_kernel<BM={i['block_m']},BN={i['block_n']},{dt}>, {order},"
+            f" every scheduling form of the plan (full-height rings A{i['stages_a']}/B{i['stages']})")
 
 
 def kernel_source_hash() -> str:
